@@ -1,0 +1,212 @@
+"""Python face of the fp64 CPU oracle (ssd_oracle.c) -- TEST INFRASTRUCTURE.
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this module.  It shares nothing with the CUDA library:
+it loads ``liboracle.so`` (built from ``ssd_oracle.c`` by ``build_oracle``)
+and passes plain float64 numpy arrays.
+
+Routes (see the C file for the equations and their sources):
+  recurrence(...)  O1, the step recurrence h_t = e^{a_t} h_{t-1} + B_t x_t^T
+  brute(...)       O2, the materialised 1-semiseparable matrix (tiny T)
+  chunked(...)     O3, the chunked algorithm with every intermediate
+
+Parity is pinned for every route (tests/test_oracle_pins.py); nothing here is
+"parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ssd_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+
+def build_oracle(force: bool = False) -> str:
+    """Compile ssd_oracle.c with gcc into liboracle.so (next to the source)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread", _SRC, "-o", tmp, "-lm"]
+        )
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+class _Shape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("B", "T", "H", "P", "G", "N", "chunk", "a_per_state")]
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build_oracle()
+        lib = ctypes.CDLL(_LIB)
+        dp = ctypes.POINTER(ctypes.c_double)
+        ip = ctypes.POINTER(ctypes.c_int)
+        sp = ctypes.POINTER(_Shape)
+        lib.oracle_recurrence.argtypes = [sp, dp, dp, dp, dp, dp, ip, ctypes.c_int, ctypes.c_int,
+                                          dp, dp, dp, ctypes.c_int]
+        lib.oracle_brute.argtypes = [sp, dp, dp, dp, dp, dp, ip, ctypes.c_int, dp, dp, ctypes.c_int]
+        lib.oracle_chunked.argtypes = [sp, dp, dp, dp, dp, dp, ip, ctypes.c_int, dp, dp, dp, dp, dp,
+                                       ctypes.c_int]
+        for f in (lib.oracle_recurrence, lib.oracle_brute, lib.oracle_chunked):
+            f.restype = ctypes.c_int
+        lib.oracle_set_mutation.argtypes = [ctypes.c_int]
+        lib.oracle_set_mutation.restype = None
+        lib.oracle_get_mutation.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def set_mutation(m: int) -> None:
+    """Plant mistake number ``m`` in every oracle route (0 = none).  Tests only."""
+    _load().oracle_set_mutation(int(m))
+
+
+def default_threads() -> int:
+    return max(1, os.cpu_count() or 1)
+
+
+@dataclass
+class Problem:
+    """One SSD problem as float64 arrays, exactly the values a device receives."""
+
+    x: np.ndarray  # [B,T,H,P]
+    a: np.ndarray  # [B,T,H] or [B,T,H,N]
+    Bm: np.ndarray  # [B,T,G,N]
+    Cm: np.ndarray  # [B,T,G,N]
+    D: np.ndarray | None  # [H]
+
+    @property
+    def dims(self):
+        B, T, H, P = self.x.shape
+        G, N = self.Bm.shape[2], self.Bm.shape[3]
+        return B, T, H, P, G, N
+
+    @property
+    def a_per_state(self) -> bool:
+        return self.a.ndim == 4
+
+
+def _f64(arr):
+    if arr is None:
+        return None
+    out = np.ascontiguousarray(np.asarray(arr, dtype=np.float64))
+    return out
+
+
+def _ptr(arr):
+    if arr is None:
+        return ctypes.POINTER(ctypes.c_double)()
+    return arr.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _shape(prob: Problem, chunk: int) -> _Shape:
+    B, T, H, P, G, N = prob.dims
+    return _Shape(B, T, H, P, G, N, int(chunk), int(prob.a_per_state))
+
+
+def _chains(prob: Problem, chains):
+    B, T, H, P, G, N = prob.dims
+    if chains is None:
+        chains = [(b, h) for b in range(B) for h in range(H)]
+    arr = np.ascontiguousarray(np.asarray(chains, dtype=np.int32).reshape(-1, 2))
+    if arr.size and (arr[:, 0].max() >= B or arr[:, 1].max() >= H or arr.min() < 0):
+        raise ValueError("chain index out of range")
+    return arr
+
+
+def _prep(prob: Problem):
+    p = Problem(_f64(prob.x), _f64(prob.a), _f64(prob.Bm), _f64(prob.Cm), _f64(prob.D))
+    B, T, H, P, G, N = p.dims
+    if H % G:
+        raise ValueError("H must be a multiple of G")
+    if p.a.shape[:3] != (B, T, H) or (p.a.ndim == 4 and p.a.shape[3] != N):
+        raise ValueError("a has the wrong shape")
+    if p.Cm.shape != p.Bm.shape:
+        raise ValueError("Bm and Cm differ in shape")
+    return p
+
+
+def recurrence(prob: Problem, chains=None, t_end=None, chunk=0, want_y=True, nthreads=None):
+    """O1.  Returns dict(y=[C,T,P] (rows >= t_end are zero), final=[C,N,P],
+    bounds=[C,nc,N,P] state after each chunk when chunk>0)."""
+    lib = _load()
+    p = _prep(prob)
+    B, T, H, P, G, N = p.dims
+    ch = _chains(p, chains)
+    C = ch.shape[0]
+    t_end = T if t_end is None else int(t_end)
+    y = np.zeros((C, T, P)) if want_y else None
+    fin = np.zeros((C, N, P))
+    bounds = np.zeros((C, T // chunk, N, P)) if chunk else None
+    rc = lib.oracle_recurrence(ctypes.byref(_shape(p, chunk)), _ptr(p.x), _ptr(p.a), _ptr(p.Bm),
+                               _ptr(p.Cm), _ptr(p.D), ch.ctypes.data_as(ctypes.POINTER(ctypes.c_int)),
+                               C, t_end, _ptr(y), _ptr(fin), _ptr(bounds),
+                               nthreads or default_threads())
+    if rc:
+        raise ValueError("oracle_recurrence rejected its arguments")
+    return {"y": y, "final": fin, "bounds": bounds, "chains": ch}
+
+
+def brute(prob: Problem, chains=None, nthreads=None):
+    """O2 (O(T^3 N) per chain).  Returns dict(y=[C,T,P], final=[C,N,P])."""
+    lib = _load()
+    p = _prep(prob)
+    B, T, H, P, G, N = p.dims
+    if T > 512:
+        raise ValueError("brute force is for tiny T")
+    ch = _chains(p, chains)
+    C = ch.shape[0]
+    y = np.zeros((C, T, P))
+    fin = np.zeros((C, N, P))
+    rc = lib.oracle_brute(ctypes.byref(_shape(p, 0)), _ptr(p.x), _ptr(p.a), _ptr(p.Bm), _ptr(p.Cm),
+                          _ptr(p.D), ch.ctypes.data_as(ctypes.POINTER(ctypes.c_int)), C, _ptr(y),
+                          _ptr(fin), nthreads or default_threads())
+    if rc:
+        raise ValueError("oracle_brute rejected its arguments")
+    return {"y": y, "final": fin, "chains": ch}
+
+
+def chunked(prob: Problem, chunk: int, chains=None, nthreads=None):
+    """O3.  Returns dict(cum=[C,nc,Q,Na], S=[C,nc,N,P], Hin=[C,nc,N,P], y=[C,T,P],
+    final=[C,N,P]); Na = N for per-state decay, else 1."""
+    lib = _load()
+    p = _prep(prob)
+    B, T, H, P, G, N = p.dims
+    if chunk <= 0 or T % chunk:
+        raise ValueError("chunk must divide T")
+    ch = _chains(p, chains)
+    C = ch.shape[0]
+    nc = T // chunk
+    Na = N if p.a_per_state else 1
+    cum = np.zeros((C, nc, chunk, Na))
+    S = np.zeros((C, nc, N, P))
+    Hin = np.zeros((C, nc, N, P))
+    y = np.zeros((C, T, P))
+    fin = np.zeros((C, N, P))
+    rc = lib.oracle_chunked(ctypes.byref(_shape(p, chunk)), _ptr(p.x), _ptr(p.a), _ptr(p.Bm),
+                            _ptr(p.Cm), _ptr(p.D), ch.ctypes.data_as(ctypes.POINTER(ctypes.c_int)), C,
+                            _ptr(cum), _ptr(S), _ptr(Hin), _ptr(y), _ptr(fin),
+                            nthreads or default_threads())
+    if rc:
+        raise ValueError("oracle_chunked rejected its arguments")
+    return {"cum": cum, "S": S, "Hin": Hin, "y": y, "final": fin, "chains": ch}
+
+
+def to_bthp(res_y: np.ndarray, chains: np.ndarray, B: int, H: int) -> np.ndarray:
+    """Scatter per-chain y [C,T,P] into [B,T,H,P] (all chains must be present)."""
+    C, T, P = res_y.shape
+    out = np.zeros((B, T, H, P))
+    for c, (b, h) in enumerate(chains):
+        out[b, :, h, :] = res_y[c]
+    return out
