@@ -1,0 +1,467 @@
+"""Throughput of the chunked SSD forward on B200 (tokens/s and roofline fraction).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--path auto|modular|simt|fused] [--impl ours|reference]
+
+One step = one ssd_forward over one batch of the workload's synthetic inputs
+(already resident in HBM); the L2 is flushed (a 256 MB write) before every
+timed step.  Each step is timed with CUDA events on the launching stream; the
+K steps are bracketed by a barrier and a device synchronise; the slowest rank
+sets the time.  Under torchrun every rank runs its own independent batch of
+the same workload (weak scaling, no collective on the data path).
+
+Rank 0 prints ONE JSON line.  ``--impl reference`` times the fp64 CPU oracle
+(the reference arm: a bounded sample of the same workload per step).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from ssd_chunked_forward_b200 import ssd  # noqa: E402
+from ssd_chunked_forward_b200.workloads import WORKLOADS, generate  # noqa: E402
+
+DEFAULT_WORKLOAD = "mamba2_2p7b"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PATHS = {"auto": ssd.PATH_AUTO, "modular": ssd.PATH_MODULAR, "simt": ssd.PATH_SIMT,
+         "fused": ssd.PATH_FUSED}
+
+
+# ----------------------------------------------------------------- model ----
+
+def algorithmic(w):
+    """Algorithmic FLOPs and HBM bytes of one forward.
+
+    Per token-head: FLOPs = 2NP (chunk state) + 2NP (incoming-state term)
+    + Q*P (causal half of the masked product with X) + Q*N*G/H (causal half
+    of C B^T, shared by the heads of a group).  Bytes: x and y once, B and C
+    once per group, a, D and the final state."""
+    B, T, H, P, N, G, Q = w.B, w.T, w.H, w.P, w.N, w.G, w.chunk
+    el = 2 if w.dtype == "bf16" else 4
+    th = B * T * H
+    flops = th * (4 * N * P + Q * P + Q * N * G / H)
+    a_bytes = B * T * H * (N if w.a_per_state else 1) * 4
+    byts = (2 * B * T * H * P * el + 2 * B * T * G * N * el + a_bytes + H * 4 + B * H * N * P * 4)
+    return flops, byts
+
+
+def kernel_bytes(w, name):
+    """Algorithmic bytes of one launch of a step kernel: each tensor it must
+    read or write, once."""
+    B, T, H, P, N, G, Q = w.B, w.T, w.H, w.P, w.N, w.G, w.chunk
+    nc = T // Q
+    el = 2 if w.dtype == "bf16" else 4
+    na = N if w.a_per_state else 1
+    x = B * T * H * P * el
+    bc = B * T * G * N * el
+    a = B * T * H * na * 4
+    cum = B * H * nc * Q * na * 4
+    st = B * H * nc * N * P * 4
+    fin = B * H * N * P * 4
+    if name == "chunk_cumsum":
+        return a + cum
+    if name == "chunk_state":
+        return x + bc + cum + st
+    if name == "state_pass":
+        return st + st + B * H * nc * na * 4 + fin
+    if name in ("chunk_scan", "diag_scan"):
+        return x + 2 * bc + cum + st + x + H * 4
+    if name == "fused":
+        return algorithmic(w)[1]
+    raise KeyError(name)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def traffic_record(kernel, workload):
+    """dram bytes per launch from a committed ncu capture, valid only while the
+    kernel's source is unchanged (hash recorded with the capture)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    r = rec.get(kernel, {}).get(workload)
+    if not r:
+        return None
+    src = os.path.join(ROOT, r["source"])
+    if not os.path.exists(src):
+        return None
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return r["bytes_per_launch"] if h == r["source_sha256_16"] else None
+
+
+# ---------------------------------------------------------------- clocks ----
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML every ~10 ms."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index):
+        self.samples, self.reasons = [], 0
+        self.ok = False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report that, never guess
+            self.err = repr(e)
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------ oracle leg ----
+
+def chain_problem(inp, b, h, t_end):
+    """float64 copy of chain (b, h)'s first t_end tokens: the exact values the
+    device receives (bf16/fp32 widen exactly to float64)."""
+    from oracle import ssd_oracle as O
+    H, G = inp["x"].shape[2], inp["Bm"].shape[2]
+    g = h // (H // G)
+    f = lambda t: t.to(torch.float64).numpy()
+    return O.Problem(f(inp["x"][b:b + 1, :t_end, h:h + 1].contiguous()),
+                     f(inp["a"][b:b + 1, :t_end, h:h + 1].contiguous()),
+                     f(inp["Bm"][b:b + 1, :t_end, g:g + 1].contiguous()),
+                     f(inp["Cm"][b:b + 1, :t_end, g:g + 1].contiguous()),
+                     f(inp["D"][h:h + 1].contiguous()))
+
+
+def oracle_sample(w, inp, budget_s, nthreads):
+    """Time the fp64 oracle recurrence on a bounded sample of the workload:
+    whole-width chains (b, h) in b-major order over their first t_end tokens,
+    sized from a short calibration run to take about budget_s seconds."""
+    from oracle import ssd_oracle as O
+
+    chains = [(b, h) for b in range(w.B) for h in range(w.H)]
+    t_cal = min(w.T, 256)
+    p = chain_problem(inp, 0, 0, t_cal)
+    t0 = time.perf_counter()
+    O.recurrence(p, nthreads=1)
+    per_token_chain = (time.perf_counter() - t0) / t_cal
+    par = max(1, nthreads)
+    n_chains = min(len(chains), max(par, 1))
+    t_end = int(min(w.T, max(16, budget_s * par / (per_token_chain * n_chains))))
+    if t_end == w.T:  # room for more chains
+        n_chains = int(min(len(chains), max(n_chains, budget_s * par / (per_token_chain * w.T))))
+    sel = chains[:n_chains]
+    # one multi-chain problem: stack the chains as heads of one batch row
+    import numpy as np
+    probs = [chain_problem(inp, b, h, t_end) for (b, h) in sel]
+    x = np.concatenate([q.x for q in probs], axis=2)
+    a = np.concatenate([q.a for q in probs], axis=2)
+    Bm = np.concatenate([q.Bm for q in probs], axis=2)
+    Cm = np.concatenate([q.Cm for q in probs], axis=2)
+    D = np.concatenate([q.D for q in probs])
+    prob = O.Problem(x, a, Bm, Cm, D)
+    t0 = time.perf_counter()
+    O.recurrence(prob, nthreads=par)
+    dt = time.perf_counter() - t0
+    tokens = n_chains * t_end / w.H  # a token carries all H heads
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": min(par, n_chains), "kind": "oracle",
+            "sample": f"{n_chains} of {w.B * w.H} (batch, head) chains x first {t_end} of {w.T} "
+                      f"tokens, fp64 recurrence, {dt:.2f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    w = WORKLOADS[args.workload]
+    inp = generate(w)
+    nthreads = os.cpu_count() or 1
+    per_step = max(0.2, min(2.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(w, inp, per_step, nthreads)
+    vals = [oracle_sample(w, inp, per_step, nthreads) for _ in range(args.steps)]
+    v = statistics.median(r["value"] for r in vals)
+    line = {
+        "impl": "reference", "metric": "SSD forward tokens/s (B*T per second)", "value": v,
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * w.tokens / v, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "P": w.P, "N": w.N, "G": w.G,
+                   "chunk": w.chunk, "parallelism": "none (CPU oracle)"},
+        "cpu_baseline": {"kind": "oracle", "cores": vals[0]["cores"], "sample": vals[0]["sample"],
+                         "value": v, "unit": "tokens/s"},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# ---------------------------------------------------------------- GPU leg ----
+
+def step_kernels(w, path_used):
+    if path_used == "fused":
+        return ["fused"]
+    return ["chunk_cumsum", "chunk_state", "state_pass", "diag_scan" if w.a_per_state else "chunk_scan"]
+
+
+def time_steps_split(w, dev, shape, ws, flush, reps, impl):
+    """Per-kernel device times (ms) of the modular path, by calling the step
+    entry points one by one with events between them on one stream."""
+    st = torch.cuda.current_stream()
+    nc = w.T // w.chunk
+    cum_t = torch.empty(w.B * w.H * nc * w.chunk * (w.N if w.a_per_state else 1),
+                        dtype=torch.float32, device=dev["x"].device)
+    states = torch.empty((w.B, w.H, nc, w.N, w.P), dtype=torch.float32, device=dev["x"].device)
+    fin = torch.empty((w.B, w.H, w.N, w.P), dtype=torch.float32, device=dev["x"].device)
+    y = torch.empty_like(dev["x"])
+    names = step_kernels(w, "modular")
+    times = {n: [] for n in names}
+    for r in range(reps):
+        flush()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        ev[0].record(st)
+        ssd.chunk_cumsum(shape, dev["a"], cum_t)
+        ev[1].record(st)
+        ssd.chunk_state(shape, dev["x"], dev["Bm"], cum_t, states, impl=impl)
+        ev[2].record(st)
+        ssd.state_pass(shape, cum_t, states, fin)
+        ev[3].record(st)
+        ssd.chunk_scan(shape, dev["x"], dev["Bm"], dev["Cm"], cum_t, states, dev["D"], y, impl=impl)
+        ev[4].record(st)
+        torch.cuda.synchronize()
+        if r == 0:
+            continue  # warm-up
+        for i, n in enumerate(names):
+            times[n].append(ev[i].elapsed_time(ev[i + 1]))
+    del cum_t, states, fin, y
+    return {n: statistics.mean(v) for n, v in times.items()}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(WORKLOADS))
+    ap.add_argument("--path", default="auto", choices=list(PATHS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
+
+    w = WORKLOADS[args.workload]
+    inp = generate(w, seed=w.seed + 1000 * rank)  # each rank: its own batch
+    dev = {k: v.to(device) for k, v in inp.items()}
+    shape = ssd.shape_of(dev["x"], dev["a"], dev["Bm"], w.chunk)
+    path = PATHS[args.path]
+    if not ssd.path_supported(shape, path):
+        raise SystemExit(f"path {args.path} does not serve workload {w.name}")
+    path_used = args.path
+    if path == ssd.PATH_AUTO:
+        path_used = "fused" if ssd.path_supported(shape, ssd.PATH_FUSED) else "modular"
+    ws = ssd.alloc_workspace(shape, device)
+    y = torch.empty_like(dev["x"])
+    fin = torch.empty((w.B, w.H, w.N, w.P), dtype=torch.float32, device=device)
+    scratch = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+
+    def flush():
+        scratch.fill_(1)
+
+    def fwd():
+        ssd.forward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], dev["D"], w.chunk, y=y,
+                    final_state=fin, workspace=ws, path=path)
+
+    st = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        flush()
+        fwd()
+    torch.cuda.synchronize()
+    code = ssd.device_status(ws)
+    if code != ssd.SSD_OK:
+        raise SystemExit(f"device status after warm-up: {ssd.status_string(code)}")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        for i in range(args.steps):
+            flush()
+            starts[i].record(st)
+            fwd()
+            ends[i].record(st)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    code = ssd.device_status(ws)
+    if code != ssd.SSD_OK:
+        raise SystemExit(f"device status after timing: {ssd.status_string(code)}")
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms = sum(step_ms) / len(step_ms)
+    if dist:
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    tokens_all = w.tokens * world
+    value = tokens_all / (ms / 1e3)
+
+    # ---- dominant kernel: per-kernel split with events --------------------
+    peaks, peak_src = load_peaks()
+    flops, byts = algorithmic(w)
+    t_roof = max(flops / (peaks["bf16_tflops"] * 1e12), byts / (peaks["hbm_gbs"] * 1e9))
+    if path_used == "fused":
+        split = {"fused": ms}
+    else:
+        impl = ssd.IMPL_SIMT if path_used == "simt" else ssd.IMPL_AUTO
+        split = time_steps_split(w, dev, shape, ws, flush, 11, impl)
+    dom = max(split, key=split.get)
+    dom_ms = split[dom]
+    dom_bytes = kernel_bytes(w, dom)
+    achieved = dom_bytes / (dom_ms / 1e3) / 1e9
+    kernel_name = {"fused": "ssd_fused_kernel"}.get(dom, "ssd_" + dom)
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": traffic_record(kernel_name, w.name),
+                "kernel": kernel_name, "algorithmic_bytes_per_launch": dom_bytes,
+                "peak_source": f"{peak_src} (hbm_gbs)"}
+
+    # ---- end to end through the host-buffer entry point -------------------
+    e2e = None
+    if not args.no_e2e:
+        pin = {k: v.pin_memory() for k, v in inp.items()}
+        y_h = torch.empty_like(inp["x"]).pin_memory()
+        f_h = torch.empty((w.B, w.H, w.N, w.P), dtype=torch.float32).pin_memory()
+        buf = torch.empty(ssd.forward_host_bytes(shape), dtype=torch.uint8, device=device)
+        e2e_steps = max(3, min(args.steps, 20))
+
+        def fwd_host():
+            ssd.forward_host(shape, pin["x"], pin["a"], pin["Bm"], pin["Cm"], pin["D"], y_h, f_h, buf)
+
+        for _ in range(3):
+            fwd_host()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0.record(st)
+        for _ in range(e2e_steps):
+            fwd_host()
+        e1.record(st)
+        torch.cuda.synchronize()
+        e_ms = e0.elapsed_time(e1) / e2e_steps
+        if dist:
+            t = torch.tensor([e_ms], device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        h2d = sum(v.numel() * v.element_size() for v in inp.values())
+        d2h = y_h.numel() * y_h.element_size() + f_h.numel() * 4
+        e2e = {"value": tokens_all / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms, "steps": e2e_steps,
+               "api": "ssd_forward_host (pinned host buffers)"}
+        del buf
+
+    # ---- CPU oracle baseline (rank 0, N = 1 only) -------------------------
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_sample(w, inp, 15.0, os.cpu_count() or 1)
+
+    if rank == 0:
+        launches = len(step_kernels(w, path_used)) * args.steps
+        line = {
+            "metric": "SSD forward tokens/s (B*T per second)", "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+            "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "P": w.P, "N": w.N,
+                       "G": w.G, "chunk": w.chunk, "a_per_state": w.a_per_state,
+                       "global_batch": w.B * world, "seq_len": w.T,
+                       "parallelism": f"independent batch per GPU x{world}", "path": path_used,
+                       "l2": "flushed (256 MB write) before every timed step"},
+            "roofline": roofline,
+            "roofline_forward": {"t_roof_us": t_roof * 1e6, "t_us": ms * 1e3,
+                                 "frac": t_roof / (ms / 1e3), "flops_alg": flops,
+                                 "bytes_alg": byts, "bound": "hbm" if byts / peaks["hbm_gbs"] / 1e9 >=
+                                 flops / peaks["bf16_tflops"] / 1e12 else "tensor",
+                                 "peaks": {"hbm_gbs": peaks["hbm_gbs"],
+                                           "bf16_tflops": peaks["bf16_tflops"], "source": peak_src}},
+            "kernel_split_ms": split,
+            "clocks": sampler.summary(),
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line))
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

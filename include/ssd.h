@@ -1,0 +1,188 @@
+/*
+ * ssd.h -- C ABI of libssd: the chunked Structured State-Space Duality (SSD)
+ * forward on NVIDIA B200 (sm_100a).
+ *
+ * The operation (for each batch b and head h, with g = h / (H/G)):
+ *
+ *   y_t = sum_{s<=t} C_t^T B_s * exp(sum_{k=s+1..t} a_k) * x_s + D[h] * x_t
+ *   h_t = exp(a_t) h_{t-1} + B_t x_t^T  (h_{-1} = 0),  final state = h_{T-1}
+ *
+ * Sources: llms.blog "State Space Models and Mamba (Mamba-1 and Mamba-2) ...",
+ * section "The SSD Theoretical Equivalence" (the 1-semiseparable matrix
+ * M_{i,j} = C_i^T (prod_{k=j+1..i} a_k) B_j and the state-space view), with
+ * the decays given here as logarithms; section "Continuous-to-Discrete
+ * Discretization" for the skip term D x_t; aiwiki "State Space Duality",
+ * section "Two algorithms for one operator", for the chunked evaluation
+ * (quadratic masked form inside a chunk, one summarised state between
+ * chunks); "On Structured State-Space Duality" (ICML 2026), item (i), for the
+ * diagonal generalisation (one log-decay per state index n).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every tensor argument is a DEVICE pointer to a contiguous row-major
+ *    buffer that the caller owns; the library allocates nothing and keeps no
+ *    state between calls.  Tensors are 16-byte aligned.
+ *  - Shapes (nc = T / chunk, Q = chunk):
+ *        x, y           [B, T, H, P]   dtype (f32 or bf16)
+ *        a              [B, T, H]      f32 log-decays (a <= 0 assumed, not checked)
+ *                       [B, T, H, N]   when a_per_state != 0
+ *        Bm, Cm         [B, T, G, N]   dtype
+ *        D              [H]            f32, may be NULL (no skip term)
+ *        final_state    [B, H, N, P]   f32, may be NULL
+ *        cum            [B, H, nc, Q]  f32  ([B, H, nc, Q, N] when a_per_state)
+ *        states         [B, H, nc, N, P] f32
+ *  - Requirements: all sizes >= 1, T % chunk == 0, H % G == 0, chunk <= 1024,
+ *    N <= 256, P <= 256.  Violations return SSD_ERR_INVALID_ARG before any
+ *    work is queued.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *    compute entry point is asynchronous on it; a return of SSD_OK means the
+ *    work was queued.  Launch failures return SSD_ERR_CUDA.  Problems found
+ *    on the device (a bounded wait that ran out) are recorded in the
+ *    workspace status word and reported by ssd_device_status().  No kernel
+ *    traps or asserts.
+ */
+#ifndef SSD_H_
+#define SSD_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SSD_OK = 0,
+    SSD_ERR_INVALID_ARG = 1, /* null pointer, bad size, misalignment       */
+    SSD_ERR_UNSUPPORTED = 2, /* valid, but not served by the requested path */
+    SSD_ERR_WORKSPACE = 3,   /* workspace missing or too small              */
+    SSD_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed        */
+    SSD_ERR_TIMEOUT = 5      /* a bounded device-side wait ran out          */
+} ssd_status;
+
+typedef enum { SSD_DTYPE_F32 = 0, SSD_DTYPE_BF16 = 1 } ssd_dtype;
+
+typedef struct {
+    int B, T, H, P, G, N, chunk;
+    int a_per_state; /* 0: a[B,T,H]; 1: a[B,T,H,N] (diagonal SSM)      */
+    int dtype;       /* ssd_dtype of x, Bm, Cm and y                    */
+} ssd_shape;
+
+typedef void* ssd_stream; /* a cudaStream_t */
+
+/* Execution paths for ssd_forward_path(). */
+enum {
+    SSD_PATH_AUTO = 0,    /* fastest path that serves the shape                 */
+    SSD_PATH_MODULAR = 1, /* chunk_cumsum -> chunk_state -> state_pass -> chunk_scan
+                             (or diag_scan), each a separate kernel, states in HBM */
+    SSD_PATH_SIMT = 2,    /* the same four steps on CUDA cores only (fp32 math)  */
+    SSD_PATH_FUSED = 3    /* one persistent kernel: chunk states, inter-chunk pass
+                             and outputs fused; states never leave L2             */
+};
+
+/* Implementations for the per-step entry points. */
+enum { SSD_IMPL_AUTO = 0, SSD_IMPL_SIMT = 1, SSD_IMPL_TC = 2 };
+
+/* Test-only flag for ssd_forward_path(): the fused path's first state hand-off
+ * is never published, so the bounded wait behind it must run out and report
+ * SSD_ERR_TIMEOUT through ssd_device_status().  Never set it otherwise. */
+#define SSD_FLAG_TEST_STALL 0x100u
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* ssd_status_string(ssd_status s);
+
+/* Bytes of device workspace ssd_forward()/ssd_forward_path() need for this
+ * shape (the maximum over paths).  Returns 0 when the shape is invalid; any
+ * valid shape needs at least 256 bytes, so 0 is unambiguous. */
+size_t ssd_workspace_size(const ssd_shape* shape);
+
+/* 1 if `path` (SSD_PATH_*) serves this shape on this build, else 0. */
+int ssd_path_supported(const ssd_shape* shape, unsigned path);
+
+/* The whole forward: y (and final_state when non-NULL) from x, a, Bm, Cm, D.
+ * `workspace` (device, >= ssd_workspace_size bytes, 256-byte aligned) is
+ * scratch owned by the caller and must not be shared by calls that overlap
+ * in time.  Equivalent to ssd_forward_path(..., SSD_PATH_AUTO, 0). */
+ssd_status ssd_forward(const ssd_shape* shape, const void* x, const float* a, const void* Bm,
+                       const void* Cm, const float* D, void* y, float* final_state,
+                       void* workspace, size_t ws_bytes, ssd_stream stream);
+
+/* As ssd_forward, with an explicit path (SSD_PATH_*) and flags
+ * (SSD_FLAG_TEST_STALL or 0).  SSD_ERR_UNSUPPORTED when the path does not
+ * serve the shape. */
+ssd_status ssd_forward_path(const ssd_shape* shape, const void* x, const float* a,
+                            const void* Bm, const void* Cm, const float* D, void* y,
+                            float* final_state, void* workspace, size_t ws_bytes,
+                            ssd_stream stream, unsigned path, unsigned flags);
+
+/* Synchronises `stream`, then returns the status word a previous
+ * ssd_forward* call on this workspace left (SSD_OK, or SSD_ERR_TIMEOUT when
+ * a bounded device wait ran out), or SSD_ERR_CUDA when the stream reports an
+ * error. */
+ssd_status ssd_device_status(const void* workspace, ssd_stream stream);
+
+/* ---- the forward from host memory --------------------------------------- */
+
+/* Device bytes ssd_forward_host() needs in `dev_buf` for this shape: staging
+ * for x, a, Bm, Cm, D, y and the final state plus the forward's workspace.
+ * 0 when the shape is invalid. */
+size_t ssd_forward_host_bytes(const ssd_shape* shape);
+
+/* The forward with HOST inputs and outputs: queues on `stream` the copies of
+ * x, a, Bm, Cm (and D when non-NULL) into `dev_buf` (a caller-owned DEVICE
+ * buffer of >= ssd_forward_host_bytes bytes, 256-byte aligned), the forward
+ * (SSD_PATH_AUTO), and the copies of y (and the final state when final_h is
+ * non-NULL) back to host memory.  Host buffers should be page-locked for the
+ * copies to be asynchronous; the caller synchronises the stream before
+ * reading y_h.  Same validation and errors as ssd_forward. */
+ssd_status ssd_forward_host(const ssd_shape* shape, const void* x_h, const float* a_h,
+                            const void* Bm_h, const void* Cm_h, const float* D_h, void* y_h,
+                            float* final_h, void* dev_buf, size_t dev_bytes, ssd_stream stream);
+
+/* ---- the steps of the path, callable one by one ------------------------- */
+
+/* Step 1, ssd_chunk_cumsum: cum[b,h,k,j(,n)] = sum_{i<=j} a[b, kQ+i, h(, n)],
+ * an inclusive prefix sum that restarts at every chunk (aiwiki "State Space
+ * Duality", "Two algorithms for one operator": the decay is accumulated in
+ * log space within a chunk).  Warp-shuffle scan. */
+ssd_status ssd_chunk_cumsum(const ssd_shape* shape, const float* a, float* cum, ssd_stream stream);
+
+/* Step 2, ssd_chunk_state: the state each chunk builds from a zero start,
+ * states[b,h,k,n,p] = sum_j Bm[b,kQ+j,g,n] * exp(cum_{k,Q-1} - cum_{k,j}) * x[b,kQ+j,h,p]
+ * (per n for a_per_state), i.e. (B_k o w)^T X_k -- llms.blog "The Chunk-Wise
+ * SSD Algorithm", item 3 (end-of-chunk state H_k in R^{N x P}).
+ * impl: SSD_IMPL_TC runs tcgen05 MMAs fed by TMA (bf16, N = 128, P = 64,
+ * chunk in {64,128,256}, scalar decay); SSD_IMPL_SIMT runs on CUDA cores. */
+ssd_status ssd_chunk_state(const ssd_shape* shape, const void* x, const void* Bm,
+                           const float* cum, float* states, ssd_stream stream, unsigned impl);
+
+/* Step 3, ssd_state_pass: sequential over chunks, independent per
+ * (b, h, n, p): in place, states[k] := h_{k-1} (the state entering chunk k,
+ * h_{-1} = 0) where h_k = exp(cum_{k,Q-1}) h_{k-1} + S_k; final_state (may be
+ * NULL) := h_{nc-1}.  llms.blog "The Chunk-Wise SSD Algorithm", item 4. */
+ssd_status ssd_state_pass(const ssd_shape* shape, const float* cum, float* states,
+                          float* final_state, ssd_stream stream);
+
+/* Step 4, ssd_chunk_scan (scalar decay): for t = kQ+i,
+ * y_t = sum_{j<=i} (C_t . B_{kQ+j}) exp(cum_i - cum_j) x_{kQ+j}
+ *       + exp(cum_i) C_t^T Hin_k + D[h] x_t,
+ * the masked quadratic form with the decay mask built on chip plus the
+ * incoming-state term (llms.blog "The Chunk-Wise SSD Algorithm", items 2 and
+ * 5; the factor exp(cum_i) on the state term is the decay from the chunk start
+ * to t).  Hin = states after ssd_state_pass.  D may be NULL. */
+ssd_status ssd_chunk_scan(const ssd_shape* shape, const void* x, const void* Bm, const void* Cm,
+                          const float* cum, const float* Hin, const float* D, void* y,
+                          ssd_stream stream, unsigned impl);
+
+/* Step 5, ssd_diag_scan (a_per_state != 0): the same output with one decay
+ * per state index, y_t = sum_{j<=i} sum_n C_t[n] B_j[n] exp(cum_i[n]-cum_j[n]) x_j
+ * + sum_n C_t[n] exp(cum_i[n]) Hin_k[n,:] + D[h] x_t ("On Structured
+ * State-Space Duality", item (i)). */
+ssd_status ssd_diag_scan(const ssd_shape* shape, const void* x, const void* Bm, const void* Cm,
+                         const float* cum, const float* Hin, const float* D, void* y,
+                         ssd_stream stream, unsigned impl);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSD_H_ */

@@ -1,0 +1,35 @@
+// kernels.h -- launchers of the libssd kernels (internal; the public ABI is include/ssd.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace ssd {
+
+struct Dims {
+    int B, T, H, P, G, N, Q, nc;
+    bool diag;  // per-state log-decay a[B,T,H,N]
+    bool bf16;  // x, Bm, Cm, y are bf16 (else fp32)
+};
+
+// ---- CUDA-core kernels (any supported size, fp32 arithmetic) --------------
+cudaError_t launch_chunk_cumsum(const Dims& d, const float* a, float* cum, cudaStream_t st);
+cudaError_t launch_chunk_state_simt(const Dims& d, const void* x, const void* Bm, const float* cum,
+                                    float* states, cudaStream_t st);
+cudaError_t launch_state_pass(const Dims& d, const float* cum, float* states, float* fin,
+                              cudaStream_t st);
+// output step; serves the scalar (chunk_scan) and the per-state (diag_scan) decay
+cudaError_t launch_chunk_scan_simt(const Dims& d, const void* x, const void* Bm, const void* Cm,
+                                   const float* cum, const float* Hin, const float* D, void* y,
+                                   cudaStream_t st);
+
+// ---- tensor-core kernels (tcgen05 + TMEM + TMA) ----------------------------
+bool chunk_state_tc_supported(const Dims& d);
+cudaError_t launch_chunk_state_tc(const Dims& d, const void* x, const void* Bm, const float* cum,
+                                  float* states, cudaStream_t st);
+bool chunk_scan_tc_supported(const Dims& d);
+cudaError_t launch_chunk_scan_tc(const Dims& d, const void* x, const void* Bm, const void* Cm,
+                                 const float* cum, const float* Hin, const float* D, void* y,
+                                 cudaStream_t st);
+
+}  // namespace ssd

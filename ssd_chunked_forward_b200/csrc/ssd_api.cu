@@ -1,0 +1,308 @@
+// ssd_api.cu -- the C ABI of libssd (declared in include/ssd.h): argument
+// validation, workspace layout, path selection and launches on the caller's
+// stream.  No allocation happens here; every buffer belongs to the caller.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/ssd.h"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+using ssd::Dims;
+
+constexpr size_t kAlign = 256;
+constexpr size_t kCtrlBytes = 256;  // status word and counters
+
+inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+ssd_status check_shape(const ssd_shape* s) {
+    if (!s) return SSD_ERR_INVALID_ARG;
+    if (s->B < 1 || s->T < 1 || s->H < 1 || s->P < 1 || s->G < 1 || s->N < 1 || s->chunk < 1)
+        return SSD_ERR_INVALID_ARG;
+    if (s->T % s->chunk != 0 || s->H % s->G != 0) return SSD_ERR_INVALID_ARG;
+    if (s->chunk > 1024 || s->N > 256 || s->P > 256) return SSD_ERR_INVALID_ARG;
+    if (s->dtype != SSD_DTYPE_F32 && s->dtype != SSD_DTYPE_BF16) return SSD_ERR_INVALID_ARG;
+    if (s->a_per_state != 0 && s->a_per_state != 1) return SSD_ERR_INVALID_ARG;
+    // every flattened index fits comfortably in 63 bits; guard the int grid dims
+    const long long nc = s->T / s->chunk;
+    if ((long long)s->B * s->H > 0x7fffffffLL || nc * ((s->chunk + 31) / 32) > 0x7fffffffLL)
+        return SSD_ERR_INVALID_ARG;
+    return SSD_OK;
+}
+
+Dims dims_of(const ssd_shape* s) {
+    Dims d;
+    d.B = s->B; d.T = s->T; d.H = s->H; d.P = s->P; d.G = s->G; d.N = s->N; d.Q = s->chunk;
+    d.nc = s->T / s->chunk;
+    d.diag = s->a_per_state != 0;
+    d.bf16 = s->dtype == SSD_DTYPE_BF16;
+    return d;
+}
+
+size_t cum_bytes(const Dims& d) {
+    return (size_t)d.B * d.H * d.nc * d.Q * (d.diag ? d.N : 1) * sizeof(float);
+}
+size_t states_bytes(const Dims& d) {
+    return (size_t)d.B * d.H * d.nc * d.N * d.P * sizeof(float);
+}
+
+struct Workspace {
+    int* ctrl;
+    float* cum;
+    float* states;
+};
+
+size_t modular_ws(const Dims& d) {
+    return kCtrlBytes + round_up(cum_bytes(d), kAlign) + round_up(states_bytes(d), kAlign);
+}
+
+Workspace carve(void* ws, const Dims& d) {
+    char* p = (char*)ws;
+    Workspace w;
+    w.ctrl = (int*)p;
+    p += kCtrlBytes;
+    w.cum = (float*)p;
+    p += round_up(cum_bytes(d), kAlign);
+    w.states = (float*)p;
+    return w;
+}
+
+ssd_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA; }
+
+ssd_status run_modular(const Dims& d, const void* x, const float* a, const void* Bm,
+                       const void* Cm, const float* D, void* y, float* fin, const Workspace& w,
+                       cudaStream_t st, bool allow_tc) {
+    cudaError_t e = ssd::launch_chunk_cumsum(d, a, w.cum, st);
+    if (e != cudaSuccess) return SSD_ERR_CUDA;
+    const bool tc_state = allow_tc && ssd::chunk_state_tc_supported(d);
+    e = tc_state ? ssd::launch_chunk_state_tc(d, x, Bm, w.cum, w.states, st)
+                 : ssd::launch_chunk_state_simt(d, x, Bm, w.cum, w.states, st);
+    if (e != cudaSuccess) return SSD_ERR_CUDA;
+    e = ssd::launch_state_pass(d, w.cum, w.states, fin, st);
+    if (e != cudaSuccess) return SSD_ERR_CUDA;
+    const bool tc_scan = allow_tc && ssd::chunk_scan_tc_supported(d);
+    e = tc_scan ? ssd::launch_chunk_scan_tc(d, x, Bm, Cm, w.cum, w.states, D, y, st)
+                : ssd::launch_chunk_scan_simt(d, x, Bm, Cm, w.cum, w.states, D, y, st);
+    return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ssd_status_string(ssd_status s) {
+    switch (s) {
+        case SSD_OK: return "SSD_OK";
+        case SSD_ERR_INVALID_ARG: return "SSD_ERR_INVALID_ARG: invalid argument";
+        case SSD_ERR_UNSUPPORTED: return "SSD_ERR_UNSUPPORTED: shape not served by this path";
+        case SSD_ERR_WORKSPACE: return "SSD_ERR_WORKSPACE: workspace missing or too small";
+        case SSD_ERR_CUDA: return "SSD_ERR_CUDA: CUDA call or launch failed";
+        case SSD_ERR_TIMEOUT: return "SSD_ERR_TIMEOUT: a bounded device wait ran out";
+    }
+    return "SSD_ERR_UNKNOWN";
+}
+
+size_t ssd_workspace_size(const ssd_shape* shape) {
+    if (check_shape(shape) != SSD_OK) return 0;
+    return modular_ws(dims_of(shape));
+}
+
+int ssd_path_supported(const ssd_shape* shape, unsigned path) {
+    if (check_shape(shape) != SSD_OK) return 0;
+    const Dims d = dims_of(shape);
+    switch (path) {
+        case SSD_PATH_AUTO: return 1;
+        case SSD_PATH_SIMT: return 1;
+        case SSD_PATH_MODULAR: return 1;
+        case SSD_PATH_FUSED: return 0;
+        default: return 0;
+    }
+    (void)d;
+}
+
+ssd_status ssd_forward_path(const ssd_shape* shape, const void* x, const float* a, const void* Bm,
+                            const void* Cm, const float* D, void* y, float* final_state,
+                            void* workspace, size_t ws_bytes, ssd_stream stream, unsigned path,
+                            unsigned flags) {
+    ssd_status st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    if (!x || !a || !Bm || !Cm || !y) return SSD_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(a) || !aligned16(Bm) || !aligned16(Cm) || !aligned16(y) ||
+        (D && !aligned16(D)) || (final_state && !aligned16(final_state)))
+        return SSD_ERR_INVALID_ARG;
+    if ((flags & ~SSD_FLAG_TEST_STALL) != 0) return SSD_ERR_INVALID_ARG;
+    if (path > SSD_PATH_FUSED) return SSD_ERR_INVALID_ARG;
+    const Dims d = dims_of(shape);
+    if (!workspace || ((uintptr_t)workspace % kAlign) != 0) return SSD_ERR_WORKSPACE;
+    if (ws_bytes < ssd_workspace_size(shape)) return SSD_ERR_WORKSPACE;
+    if (!ssd_path_supported(shape, path)) return SSD_ERR_UNSUPPORTED;
+    cudaStream_t cs = (cudaStream_t)stream;
+    const Workspace w = carve(workspace, d);
+    if (cudaMemsetAsync(w.ctrl, 0, kCtrlBytes, cs) != cudaSuccess) return SSD_ERR_CUDA;
+    switch (path) {
+        case SSD_PATH_SIMT:
+            return run_modular(d, x, a, Bm, Cm, D, y, final_state, w, cs, false);
+        case SSD_PATH_MODULAR:
+        case SSD_PATH_AUTO:
+        default:
+            return run_modular(d, x, a, Bm, Cm, D, y, final_state, w, cs, true);
+    }
+}
+
+ssd_status ssd_forward(const ssd_shape* shape, const void* x, const float* a, const void* Bm,
+                       const void* Cm, const float* D, void* y, float* final_state, void* workspace,
+                       size_t ws_bytes, ssd_stream stream) {
+    return ssd_forward_path(shape, x, a, Bm, Cm, D, y, final_state, workspace, ws_bytes, stream,
+                            SSD_PATH_AUTO, 0u);
+}
+
+static size_t host_layout(const ssd_shape* s, size_t off[8]) {
+    // x, a, Bm, Cm, D, y, final, workspace -- each 256-byte aligned
+    const Dims d = dims_of(s);
+    const size_t el = d.bf16 ? 2 : 4;
+    const size_t sizes[8] = {
+        (size_t)d.B * d.T * d.H * d.P * el,
+        (size_t)d.B * d.T * d.H * (d.diag ? d.N : 1) * sizeof(float),
+        (size_t)d.B * d.T * d.G * d.N * el,
+        (size_t)d.B * d.T * d.G * d.N * el,
+        (size_t)d.H * sizeof(float),
+        (size_t)d.B * d.T * d.H * d.P * el,
+        (size_t)d.B * d.H * d.N * d.P * sizeof(float),
+        ssd_workspace_size(s)};
+    size_t total = 0;
+    for (int i = 0; i < 8; ++i) {
+        off[i] = total;
+        total += round_up(sizes[i], kAlign);
+    }
+    return total;
+}
+
+size_t ssd_forward_host_bytes(const ssd_shape* shape) {
+    if (check_shape(shape) != SSD_OK) return 0;
+    size_t off[8];
+    return host_layout(shape, off);
+}
+
+ssd_status ssd_forward_host(const ssd_shape* shape, const void* x_h, const float* a_h,
+                            const void* Bm_h, const void* Cm_h, const float* D_h, void* y_h,
+                            float* final_h, void* dev_buf, size_t dev_bytes, ssd_stream stream) {
+    ssd_status st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    if (!x_h || !a_h || !Bm_h || !Cm_h || !y_h) return SSD_ERR_INVALID_ARG;
+    if (!dev_buf || ((uintptr_t)dev_buf % kAlign) != 0) return SSD_ERR_WORKSPACE;
+    size_t off[8];
+    const size_t need = host_layout(shape, off);
+    if (dev_bytes < need) return SSD_ERR_WORKSPACE;
+    const Dims d = dims_of(shape);
+    const size_t el = d.bf16 ? 2 : 4;
+    char* base = (char*)dev_buf;
+    cudaStream_t cs = (cudaStream_t)stream;
+    const size_t nx = (size_t)d.B * d.T * d.H * d.P * el;
+    const size_t na = (size_t)d.B * d.T * d.H * (d.diag ? d.N : 1) * sizeof(float);
+    const size_t nbc = (size_t)d.B * d.T * d.G * d.N * el;
+    if (cudaMemcpyAsync(base + off[0], x_h, nx, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+        cudaMemcpyAsync(base + off[1], a_h, na, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+        cudaMemcpyAsync(base + off[2], Bm_h, nbc, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+        cudaMemcpyAsync(base + off[3], Cm_h, nbc, cudaMemcpyHostToDevice, cs) != cudaSuccess)
+        return SSD_ERR_CUDA;
+    if (D_h && cudaMemcpyAsync(base + off[4], D_h, (size_t)d.H * sizeof(float),
+                               cudaMemcpyHostToDevice, cs) != cudaSuccess)
+        return SSD_ERR_CUDA;
+    float* fin_d = final_h ? (float*)(base + off[6]) : nullptr;
+    st = ssd_forward(shape, base + off[0], (const float*)(base + off[1]), base + off[2],
+                     base + off[3], D_h ? (const float*)(base + off[4]) : nullptr, base + off[5],
+                     fin_d, base + off[7], need - off[7], stream);
+    if (st != SSD_OK) return st;
+    if (cudaMemcpyAsync(y_h, base + off[5], nx, cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+        return SSD_ERR_CUDA;
+    if (final_h && cudaMemcpyAsync(final_h, fin_d, (size_t)d.B * d.H * d.N * d.P * sizeof(float),
+                                   cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+        return SSD_ERR_CUDA;
+    return SSD_OK;
+}
+
+ssd_status ssd_device_status(const void* workspace, ssd_stream stream) {
+    if (!workspace) return SSD_ERR_WORKSPACE;
+    cudaStream_t cs = (cudaStream_t)stream;
+    if (cudaStreamSynchronize(cs) != cudaSuccess) return SSD_ERR_CUDA;
+    int word = 0;
+    if (cudaMemcpy(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return SSD_ERR_CUDA;
+    if (word == ssd::kDevOk) return SSD_OK;
+    if (word == ssd::kDevTimeout) return SSD_ERR_TIMEOUT;
+    return SSD_ERR_CUDA;
+}
+
+ssd_status ssd_chunk_cumsum(const ssd_shape* shape, const float* a, float* cum, ssd_stream stream) {
+    ssd_status st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    if (!a || !cum || !aligned16(a) || !aligned16(cum)) return SSD_ERR_INVALID_ARG;
+    return cuda_status(ssd::launch_chunk_cumsum(dims_of(shape), a, cum, (cudaStream_t)stream));
+}
+
+ssd_status ssd_chunk_state(const ssd_shape* shape, const void* x, const void* Bm, const float* cum,
+                           float* states, ssd_stream stream, unsigned impl) {
+    ssd_status st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    if (!x || !Bm || !cum || !states) return SSD_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(Bm) || !aligned16(cum) || !aligned16(states))
+        return SSD_ERR_INVALID_ARG;
+    if (impl > SSD_IMPL_TC) return SSD_ERR_INVALID_ARG;
+    const Dims d = dims_of(shape);
+    const bool tc_ok = ssd::chunk_state_tc_supported(d);
+    if (impl == SSD_IMPL_TC && !tc_ok) return SSD_ERR_UNSUPPORTED;
+    const bool use_tc = impl == SSD_IMPL_TC || (impl == SSD_IMPL_AUTO && tc_ok);
+    cudaStream_t cs = (cudaStream_t)stream;
+    return cuda_status(use_tc ? ssd::launch_chunk_state_tc(d, x, Bm, cum, states, cs)
+                              : ssd::launch_chunk_state_simt(d, x, Bm, cum, states, cs));
+}
+
+ssd_status ssd_state_pass(const ssd_shape* shape, const float* cum, float* states,
+                          float* final_state, ssd_stream stream) {
+    ssd_status st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    if (!cum || !states || !aligned16(cum) || !aligned16(states) ||
+        (final_state && !aligned16(final_state)))
+        return SSD_ERR_INVALID_ARG;
+    return cuda_status(
+        ssd::launch_state_pass(dims_of(shape), cum, states, final_state, (cudaStream_t)stream));
+}
+
+static ssd_status scan_common(const ssd_shape* shape, const void* x, const void* Bm,
+                              const void* Cm, const float* cum, const float* Hin, const float* D,
+                              void* y, ssd_stream stream, unsigned impl, bool want_diag) {
+    ssd_status st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    if ((shape->a_per_state != 0) != want_diag) return SSD_ERR_INVALID_ARG;
+    if (!x || !Bm || !Cm || !cum || !Hin || !y) return SSD_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(Bm) || !aligned16(Cm) || !aligned16(cum) || !aligned16(Hin) ||
+        !aligned16(y) || (D && !aligned16(D)))
+        return SSD_ERR_INVALID_ARG;
+    if (impl > SSD_IMPL_TC) return SSD_ERR_INVALID_ARG;
+    const Dims d = dims_of(shape);
+    const bool tc_ok = ssd::chunk_scan_tc_supported(d);
+    if (impl == SSD_IMPL_TC && !tc_ok) return SSD_ERR_UNSUPPORTED;
+    const bool use_tc = impl == SSD_IMPL_TC || (impl == SSD_IMPL_AUTO && tc_ok);
+    cudaStream_t cs = (cudaStream_t)stream;
+    return cuda_status(use_tc ? ssd::launch_chunk_scan_tc(d, x, Bm, Cm, cum, Hin, D, y, cs)
+                              : ssd::launch_chunk_scan_simt(d, x, Bm, Cm, cum, Hin, D, y, cs));
+}
+
+ssd_status ssd_chunk_scan(const ssd_shape* shape, const void* x, const void* Bm, const void* Cm,
+                          const float* cum, const float* Hin, const float* D, void* y,
+                          ssd_stream stream, unsigned impl) {
+    return scan_common(shape, x, Bm, Cm, cum, Hin, D, y, stream, impl, false);
+}
+
+ssd_status ssd_diag_scan(const ssd_shape* shape, const void* x, const void* Bm, const void* Cm,
+                         const float* cum, const float* Hin, const float* D, void* y,
+                         ssd_stream stream, unsigned impl) {
+    return scan_common(shape, x, Bm, Cm, cum, Hin, D, y, stream, impl, true);
+}
+
+}  // extern "C"

@@ -1,0 +1,222 @@
+"""ctypes binding of libssd (include/ssd.h): argument marshalling only.
+
+Every step of the computation runs in the library's CUDA kernels; this module
+turns torch tensors into device pointers, the current torch stream into a
+``cudaStream_t`` and status codes into exceptions.  There is no fallback: if
+``libssd.so`` is missing or fails to load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libssd.so")
+
+SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_WORKSPACE, SSD_ERR_CUDA, SSD_ERR_TIMEOUT = range(6)
+SSD_DTYPE_F32, SSD_DTYPE_BF16 = 0, 1
+PATH_AUTO, PATH_MODULAR, PATH_SIMT, PATH_FUSED = 0, 1, 2, 3
+IMPL_AUTO, IMPL_SIMT, IMPL_TC = 0, 1, 2
+FLAG_TEST_STALL = 0x100
+
+EXPORTS = [
+    "ssd_status_string", "ssd_workspace_size", "ssd_path_supported", "ssd_forward",
+    "ssd_forward_path", "ssd_device_status", "ssd_chunk_cumsum", "ssd_chunk_state",
+    "ssd_state_pass", "ssd_chunk_scan", "ssd_diag_scan", "ssd_forward_host_bytes",
+    "ssd_forward_host",
+]
+
+
+class SSDError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)}")
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("B", "T", "H", "P", "G", "N", "chunk", "a_per_state", "dtype")]
+
+    def __repr__(self):
+        return "Shape(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Open libssd.so (built by ``ssd_chunked_forward_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"libssd.so not built ({path}); run python -m ssd_chunked_forward_b200.build")
+    lib = ctypes.CDLL(path)
+    vp, fp, sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t
+    sp = ctypes.POINTER(Shape)
+    lib.ssd_status_string.argtypes = [ctypes.c_int]
+    lib.ssd_status_string.restype = ctypes.c_char_p
+    lib.ssd_workspace_size.argtypes = [sp]
+    lib.ssd_workspace_size.restype = sz
+    lib.ssd_path_supported.argtypes = [sp, ctypes.c_uint]
+    lib.ssd_path_supported.restype = ctypes.c_int
+    lib.ssd_forward.argtypes = [sp, vp, fp, vp, vp, fp, vp, fp, vp, sz, vp]
+    lib.ssd_forward_path.argtypes = [sp, vp, fp, vp, vp, fp, vp, fp, vp, sz, vp, ctypes.c_uint, ctypes.c_uint]
+    lib.ssd_device_status.argtypes = [vp, vp]
+    lib.ssd_chunk_cumsum.argtypes = [sp, fp, fp, vp]
+    lib.ssd_chunk_state.argtypes = [sp, vp, vp, fp, fp, vp, ctypes.c_uint]
+    lib.ssd_state_pass.argtypes = [sp, fp, fp, fp, vp]
+    lib.ssd_chunk_scan.argtypes = [sp, vp, vp, vp, fp, fp, fp, vp, vp, ctypes.c_uint]
+    lib.ssd_diag_scan.argtypes = [sp, vp, vp, vp, fp, fp, fp, vp, vp, ctypes.c_uint]
+    lib.ssd_forward_host_bytes.argtypes = [sp]
+    lib.ssd_forward_host_bytes.restype = sz
+    lib.ssd_forward_host.argtypes = [sp, vp, fp, vp, vp, fp, vp, fp, vp, sz, vp]
+    for name in ("ssd_forward", "ssd_forward_path", "ssd_device_status", "ssd_chunk_cumsum",
+                 "ssd_chunk_state", "ssd_state_pass", "ssd_chunk_scan", "ssd_diag_scan",
+                 "ssd_forward_host"):
+        getattr(lib, name).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def status_string(code: int) -> str:
+    return load().ssd_status_string(int(code)).decode()
+
+
+def _check(code: int, where: str):
+    if code != SSD_OK:
+        raise SSDError(code, where)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def make_shape(B, T, H, P, G, N, chunk, a_per_state=False, dtype="bf16") -> Shape:
+    dt = SSD_DTYPE_BF16 if dtype in ("bf16", torch.bfloat16) else SSD_DTYPE_F32
+    return Shape(int(B), int(T), int(H), int(P), int(G), int(N), int(chunk), int(bool(a_per_state)), dt)
+
+
+def shape_of(x: torch.Tensor, a: torch.Tensor, Bm: torch.Tensor, chunk: int) -> Shape:
+    B, T, H, P = x.shape
+    G, N = Bm.shape[2], Bm.shape[3]
+    return make_shape(B, T, H, P, G, N, chunk, a.dim() == 4, x.dtype)
+
+
+def workspace_size(shape: Shape) -> int:
+    return int(load().ssd_workspace_size(ctypes.byref(shape)))
+
+
+def path_supported(shape: Shape, path: int) -> bool:
+    return bool(load().ssd_path_supported(ctypes.byref(shape), int(path)))
+
+
+def alloc_workspace(shape: Shape, device=None) -> torch.Tensor:
+    n = workspace_size(shape)
+    if n == 0:
+        raise SSDError(SSD_ERR_INVALID_ARG, "ssd_workspace_size")
+    # torch's caching allocator returns >= 512-byte aligned blocks
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def _check_inputs(x, a, Bm, Cm, D):
+    for name, t in (("x", x), ("a", a), ("Bm", Bm), ("Cm", Cm)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if a.dtype != torch.float32:
+        raise ValueError("a must be float32")
+    if x.dtype not in (torch.float32, torch.bfloat16) or Bm.dtype != x.dtype or Cm.dtype != x.dtype:
+        raise ValueError("x, Bm, Cm must share dtype float32 or bfloat16")
+    if D is not None and (D.dtype != torch.float32 or not D.is_cuda or not D.is_contiguous()):
+        raise ValueError("D must be a contiguous float32 CUDA tensor")
+
+
+def forward(x, a, Bm, Cm, D=None, chunk=256, *, y=None, final_state=None, want_final=True,
+            workspace=None, path=PATH_AUTO, flags=0, stream=None):
+    """y[B,T,H,P] (and final state [B,H,N,P] fp32) of the chunked SSD forward.
+
+    x [B,T,H,P], Bm/Cm [B,T,G,N] (float32 or bfloat16, same dtype), a [B,T,H]
+    or [B,T,H,N] float32 log-decays, D [H] float32 or None.  Asynchronous on
+    the current torch stream (or ``stream``)."""
+    _check_inputs(x, a, Bm, Cm, D)
+    shape = shape_of(x, a, Bm, chunk)
+    B, T, H, P = x.shape
+    N = Bm.shape[3]
+    if y is None:
+        y = torch.empty_like(x)
+    if final_state is None and want_final:
+        final_state = torch.empty((B, H, N, P), dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = alloc_workspace(shape, x.device)
+    code = load().ssd_forward_path(ctypes.byref(shape), _ptr(x), _ptr(a), _ptr(Bm), _ptr(Cm),
+                                   _ptr(D), _ptr(y), _ptr(final_state), _ptr(workspace),
+                                   workspace.numel(), _stream(stream), int(path), int(flags))
+    _check(code, "ssd_forward_path")
+    return y, final_state
+
+
+def device_status(workspace, stream=None) -> int:
+    """Synchronise and return the workspace status word (SSD_OK or an error)."""
+    return int(load().ssd_device_status(_ptr(workspace), _stream(stream)))
+
+
+def chunk_cumsum(shape: Shape, a, cum=None, stream=None):
+    nc = shape.T // shape.chunk
+    if cum is None:
+        dims = (shape.B, shape.H, nc, shape.chunk) + ((shape.N,) if shape.a_per_state else ())
+        cum = torch.empty(dims, dtype=torch.float32, device=a.device)
+    _check(load().ssd_chunk_cumsum(ctypes.byref(shape), _ptr(a), _ptr(cum), _stream(stream)),
+           "ssd_chunk_cumsum")
+    return cum
+
+
+def chunk_state(shape: Shape, x, Bm, cum, states=None, impl=IMPL_AUTO, stream=None):
+    nc = shape.T // shape.chunk
+    if states is None:
+        states = torch.empty((shape.B, shape.H, nc, shape.N, shape.P), dtype=torch.float32,
+                             device=x.device)
+    _check(load().ssd_chunk_state(ctypes.byref(shape), _ptr(x), _ptr(Bm), _ptr(cum), _ptr(states),
+                                  _stream(stream), int(impl)), "ssd_chunk_state")
+    return states
+
+
+def state_pass(shape: Shape, cum, states, final_state=None, stream=None):
+    _check(load().ssd_state_pass(ctypes.byref(shape), _ptr(cum), _ptr(states), _ptr(final_state),
+                                 _stream(stream)), "ssd_state_pass")
+    return states, final_state
+
+
+def chunk_scan(shape: Shape, x, Bm, Cm, cum, Hin, D=None, y=None, impl=IMPL_AUTO, stream=None):
+    if y is None:
+        y = torch.empty_like(x)
+    fn = load().ssd_diag_scan if shape.a_per_state else load().ssd_chunk_scan
+    _check(fn(ctypes.byref(shape), _ptr(x), _ptr(Bm), _ptr(Cm), _ptr(cum), _ptr(Hin), _ptr(D),
+              _ptr(y), _stream(stream), int(impl)),
+           "ssd_diag_scan" if shape.a_per_state else "ssd_chunk_scan")
+    return y
+
+
+def forward_host_bytes(shape: Shape) -> int:
+    return int(load().ssd_forward_host_bytes(ctypes.byref(shape)))
+
+
+def forward_host(shape: Shape, x_h, a_h, Bm_h, Cm_h, D_h, y_h, final_h, dev_buf, stream=None):
+    """The forward from HOST buffers (pinned for asynchrony): the library copies
+    the inputs to ``dev_buf``, runs, and copies y (and the final state) back,
+    all queued on the stream.  The caller synchronises."""
+    _check(load().ssd_forward_host(ctypes.byref(shape), _ptr(x_h), _ptr(a_h), _ptr(Bm_h), _ptr(Cm_h),
+                                   _ptr(D_h), _ptr(y_h), _ptr(final_h), _ptr(dev_buf),
+                                   dev_buf.numel(), _stream(stream)), "ssd_forward_host")

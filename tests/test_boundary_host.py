@@ -1,0 +1,127 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function include/ssd.h declares, sizes workspaces as documented and
+rejects bad arguments with the documented status before touching the GPU."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from ssd_chunked_forward_b200 import ssd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ssd.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ssd_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from ssd_chunked_forward_b200.build import build
+    build()
+    return ssd.load()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert "ssd_forward" in names and len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(ssd.EXPORTS) == names
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        s = ssd.status_string(code)
+        assert s.startswith("SSD_")
+    assert ssd.status_string(99) == "SSD_ERR_UNKNOWN"
+
+
+def _shape(**kw):
+    base = dict(B=2, T=512, H=4, P=64, G=1, N=128, chunk=256, a_per_state=False, dtype="bf16")
+    base.update(kw)
+    return ssd.make_shape(**base)
+
+
+def test_workspace_size_arithmetic(lib):
+    s = _shape()
+    nc = 512 // 256
+    cum = 2 * 4 * nc * 256 * 4
+    states = 2 * 4 * nc * 128 * 64 * 4
+    rup = lambda v: (v + 255) // 256 * 256
+    assert ssd.workspace_size(s) >= 256 + rup(cum) + rup(states)
+    s4 = _shape(a_per_state=True, N=64, chunk=128)
+    assert ssd.workspace_size(s4) >= 256 + rup(2 * 4 * 4 * 128 * 64 * 4)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(T=500),            # T % chunk
+    dict(H=3, G=2),         # H % G
+    dict(B=0), dict(N=0), dict(P=0), dict(chunk=0),
+    dict(chunk=2048, T=2048),
+    dict(N=512), dict(P=300),
+    dict(dtype=7),
+])
+def test_invalid_shapes_rejected(lib, bad):
+    if bad.get("dtype") == 7:
+        s = _shape()
+        s.dtype = 7
+    else:
+        s = _shape(**bad)
+    assert ssd.workspace_size(s) == 0
+    assert not ssd.path_supported(s, ssd.PATH_AUTO)
+    code = lib.ssd_forward(ctypes.byref(s), 256, 256, 256, 256, None, 256, None, 256, 1 << 40, None)
+    assert code == ssd.SSD_ERR_INVALID_ARG
+
+
+def test_null_and_misaligned_pointers_rejected(lib):
+    s = _shape()
+    ok = 1 << 20  # a 16-byte aligned fake address; never dereferenced
+    ws = ssd.workspace_size(s)
+    f = lambda *a: lib.ssd_forward(ctypes.byref(s), *a)
+    assert f(None, ok, ok, ok, None, ok, None, ok, ws, None) == ssd.SSD_ERR_INVALID_ARG
+    assert f(ok, None, ok, ok, None, ok, None, ok, ws, None) == ssd.SSD_ERR_INVALID_ARG
+    assert f(ok, ok, ok, ok, None, None, None, ok, ws, None) == ssd.SSD_ERR_INVALID_ARG
+    assert f(ok + 2, ok, ok, ok, None, ok, None, ok, ws, None) == ssd.SSD_ERR_INVALID_ARG
+    assert f(ok, ok, ok, ok, ok + 4, ok, None, ok, ws, None) == ssd.SSD_ERR_INVALID_ARG
+    # workspace: missing, misaligned, too small
+    assert f(ok, ok, ok, ok, None, ok, None, None, ws, None) == ssd.SSD_ERR_WORKSPACE
+    assert f(ok, ok, ok, ok, None, ok, None, ok + 16, ws, None) == ssd.SSD_ERR_WORKSPACE
+    assert f(ok, ok, ok, ok, None, ok, None, ok, ws - 1, None) == ssd.SSD_ERR_WORKSPACE
+    # unknown path or flag
+    g = lambda path, flags: lib.ssd_forward_path(ctypes.byref(s), ok, ok, ok, ok, None, ok, None,
+                                                 ok, ws, None, path, flags)
+    assert g(9, 0) == ssd.SSD_ERR_INVALID_ARG
+    assert g(0, 0x1) == ssd.SSD_ERR_INVALID_ARG
+
+
+def test_step_entry_points_validate(lib):
+    s = _shape()
+    ok = 1 << 20
+    assert lib.ssd_chunk_cumsum(ctypes.byref(s), None, ok, None) == ssd.SSD_ERR_INVALID_ARG
+    assert lib.ssd_chunk_state(ctypes.byref(s), ok, ok, ok, None, None, 0) == ssd.SSD_ERR_INVALID_ARG
+    assert lib.ssd_chunk_state(ctypes.byref(s), ok, ok, ok, ok, None, 7) == ssd.SSD_ERR_INVALID_ARG
+    assert lib.ssd_state_pass(ctypes.byref(s), ok, None, None, None) == ssd.SSD_ERR_INVALID_ARG
+    # scan entry points check the decay variant they serve
+    assert lib.ssd_diag_scan(ctypes.byref(s), ok, ok, ok, ok, ok, None, ok, None, 0) == \
+        ssd.SSD_ERR_INVALID_ARG
+    s4 = _shape(a_per_state=True)
+    assert lib.ssd_chunk_scan(ctypes.byref(s4), ok, ok, ok, ok, ok, None, ok, None, 0) == \
+        ssd.SSD_ERR_INVALID_ARG
+
+
+def test_host_entry_point_validates(lib):
+    s = _shape()
+    ok = 1 << 20
+    need = ssd.forward_host_bytes(s)
+    assert need > ssd.workspace_size(s)
+    f = lambda *a: lib.ssd_forward_host(ctypes.byref(s), *a)
+    assert f(None, ok, ok, ok, None, ok, None, ok, need, None) == ssd.SSD_ERR_INVALID_ARG
+    assert f(ok, ok, ok, ok, None, ok, None, ok, need - 1, None) == ssd.SSD_ERR_WORKSPACE
+    assert f(ok, ok, ok, ok, None, ok, None, ok + 16, need, None) == ssd.SSD_ERR_WORKSPACE

@@ -1,0 +1,248 @@
+"""GPU parity of libssd against the fp64 oracle, through the C ABI.
+
+Per-step parity (each kernel fed the oracle's own fp64 intermediates, cast to
+fp32), end-to-end parity on small cases that span several tiles with ragged
+edges, the library's invariants, and edge shapes.  Full-size workloads are in
+test_gpu_workloads.py.  Tolerances: 1e-4 for fp32 inputs, 2e-2 for bf16
+inputs with fp32 accumulation, as ||y - y_ref||_inf / ||y_ref||_inf.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import ssd_oracle as O
+from ssd_chunked_forward_b200 import ssd
+from ssd_chunked_forward_b200.workloads import generate, small_case
+from tests.gpu_helpers import (TOL_BF16, TOL_F32, chain_problem, parity_on_chains, rel_err,
+                               run_forward, to_dev, tol_for)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    ssd.load()  # a missing library is an error, not a skip
+
+
+CASES = [
+    small_case(B=2, T=96, H=3, P=24, N=20, G=1, chunk=32, dtype="f32", seed=1),
+    small_case(B=1, T=150, H=2, P=70, N=33, G=2, chunk=30, dtype="f32", seed=2),
+    small_case(B=1, T=192, H=4, P=64, N=128, G=2, chunk=64, dtype="bf16", seed=3),
+    small_case(B=2, T=768, H=3, P=64, N=128, G=1, chunk=256, dtype="bf16", seed=4),
+    small_case(B=1, T=384, H=5, P=64, N=128, G=1, chunk=128, dtype="bf16", seed=5),
+    small_case(B=2, T=256, H=2, P=64, N=64, G=1, chunk=128, dtype="bf16", a_per_state=True, seed=6),
+    small_case(B=1, T=60, H=2, P=10, N=12, G=1, chunk=20, dtype="f32", a_per_state=True, seed=7),
+]
+EDGE = [
+    small_case(B=1, T=1, H=1, P=1, N=1, G=1, chunk=1, dtype="f32", seed=8),
+    small_case(B=1, T=5, H=1, P=3, N=2, G=1, chunk=1, dtype="f32", seed=9),
+    small_case(B=1, T=7, H=2, P=5, N=3, G=2, chunk=7, dtype="f32", seed=10),
+    small_case(B=3, T=64, H=1, P=1, N=1, G=1, chunk=64, dtype="bf16", seed=11),
+    small_case(B=1, T=1024, H=1, P=8, N=8, G=1, chunk=1024, dtype="f32", seed=12),
+]
+
+
+def _ids(cases):
+    return [c.name + ("_diag" if c.a_per_state else "") + "_" + c.dtype for c in cases]
+
+
+def _all_chains(w):
+    return [(b, h) for b in range(w.B) for h in range(w.H)]
+
+
+def _paths():
+    return [ssd.PATH_SIMT, ssd.PATH_MODULAR, ssd.PATH_AUTO, ssd.PATH_FUSED]
+
+
+@pytest.mark.parametrize("w", CASES + EDGE, ids=_ids(CASES + EDGE))
+@pytest.mark.parametrize("path", _paths(), ids=["simt", "modular", "auto", "fused"])
+def test_forward_matches_oracle(w, path):
+    inp = generate(w)
+    dev = to_dev(inp)
+    shape = ssd.shape_of(dev["x"], dev["a"], dev["Bm"], w.chunk)
+    if not ssd.path_supported(shape, path):
+        pytest.skip("path does not serve this shape")
+    y, fin = run_forward(w, dev, path=path)
+    ey, ef = parity_on_chains(inp, y, fin, _all_chains(w))
+    tol = tol_for(w)
+    assert ey <= tol, f"y rel err {ey:.3e}"
+    assert ef <= tol, f"final-state rel err {ef:.3e}"
+
+
+def _oracle_chunked(inp, w):
+    """O3 per chain, as [B,H,...] float64 arrays."""
+    prob = O.Problem(*(inp[k].to(torch.float64).numpy() for k in ("x", "a", "Bm", "Cm", "D")))
+    r = O.chunked(prob, w.chunk)
+    nc = w.T // w.chunk
+    cum = r["cum"].reshape(w.B, w.H, nc, w.chunk, -1)
+    if not w.a_per_state:
+        cum = cum[..., 0]
+    S = r["S"].reshape(w.B, w.H, nc, w.N, w.P)
+    Hin = r["Hin"].reshape(w.B, w.H, nc, w.N, w.P)
+    y = r["y"].reshape(w.B, w.H, w.T, w.P).transpose(0, 2, 1, 3)
+    fin = r["final"].reshape(w.B, w.H, w.N, w.P)
+    return cum, S, Hin, y, fin
+
+
+def _impls(shape, which):
+    out = [ssd.IMPL_SIMT]
+    return out + ([ssd.IMPL_TC] if which(shape) else [])
+
+
+def _tc_state_ok(shape):
+    return shape.dtype == ssd.SSD_DTYPE_BF16 and not shape.a_per_state and shape.N == 128 \
+        and shape.P == 64 and shape.chunk in (64, 128, 256)
+
+
+@pytest.mark.parametrize("w", CASES, ids=_ids(CASES))
+def test_step_chunk_cumsum(w):
+    inp = generate(w)
+    dev = to_dev(inp)
+    shape = ssd.shape_of(dev["x"], dev["a"], dev["Bm"], w.chunk)
+    cum = ssd.chunk_cumsum(shape, dev["a"])
+    torch.cuda.synchronize()
+    ref = _oracle_chunked(inp, w)[0]
+    assert rel_err(cum.cpu().numpy().astype(np.float64), ref) < 1e-5
+
+
+@pytest.mark.parametrize("w", CASES, ids=_ids(CASES))
+@pytest.mark.parametrize("impl", [ssd.IMPL_SIMT, ssd.IMPL_TC], ids=["simt", "tc"])
+def test_step_chunk_state(w, impl):
+    inp = generate(w)
+    dev = to_dev(inp)
+    shape = ssd.shape_of(dev["x"], dev["a"], dev["Bm"], w.chunk)
+    cum, S, _, _, _ = _oracle_chunked(inp, w)
+    cum_d = torch.from_numpy(cum.astype(np.float32)).cuda().contiguous()
+    try:
+        got = ssd.chunk_state(shape, dev["x"], dev["Bm"], cum_d, impl=impl)
+    except ssd.SSDError as e:
+        if e.code == ssd.SSD_ERR_UNSUPPORTED:
+            pytest.skip("tensor-core chunk_state does not serve this shape")
+        raise
+    torch.cuda.synchronize()
+    assert rel_err(got.cpu().numpy().astype(np.float64), S) <= tol_for(w)
+
+
+@pytest.mark.parametrize("w", CASES, ids=_ids(CASES))
+def test_step_state_pass(w):
+    inp = generate(w)
+    shape = ssd.make_shape(w.B, w.T, w.H, w.P, w.G, w.N, w.chunk, w.a_per_state, w.dtype)
+    cum, S, Hin, _, fin = _oracle_chunked(inp, w)
+    cum_d = torch.from_numpy(cum.astype(np.float32)).cuda().contiguous()
+    st = torch.from_numpy(S.astype(np.float32)).cuda().contiguous()
+    fin_d = torch.empty((w.B, w.H, w.N, w.P), dtype=torch.float32, device="cuda")
+    ssd.state_pass(shape, cum_d, st, fin_d)
+    torch.cuda.synchronize()
+    assert rel_err(st.cpu().numpy().astype(np.float64), Hin) < 1e-5
+    assert rel_err(fin_d.cpu().numpy().astype(np.float64), fin) < 1e-5
+
+
+@pytest.mark.parametrize("w", CASES, ids=_ids(CASES))
+@pytest.mark.parametrize("impl", [ssd.IMPL_SIMT, ssd.IMPL_TC], ids=["simt", "tc"])
+def test_step_chunk_scan(w, impl):
+    inp = generate(w)
+    dev = to_dev(inp)
+    shape = ssd.shape_of(dev["x"], dev["a"], dev["Bm"], w.chunk)
+    cum, _, Hin, y_ref, _ = _oracle_chunked(inp, w)
+    cum_d = torch.from_numpy(cum.astype(np.float32)).cuda().contiguous()
+    Hin_d = torch.from_numpy(Hin.astype(np.float32)).cuda().contiguous()
+    try:
+        y = ssd.chunk_scan(shape, dev["x"], dev["Bm"], dev["Cm"], cum_d, Hin_d, dev["D"], impl=impl)
+    except ssd.SSDError as e:
+        if e.code == ssd.SSD_ERR_UNSUPPORTED:
+            pytest.skip("tensor-core scan does not serve this shape")
+        raise
+    torch.cuda.synchronize()
+    assert rel_err(y.float().cpu().numpy().astype(np.float64), y_ref) <= tol_for(w)
+
+
+# ------------------------------------------------------------ invariants ----
+
+def _bf16_case(T=1024, H=4, G=1, seed=21, u_mean=-2.0):
+    return small_case(B=2, T=T, H=H, P=64, N=128, G=G, chunk=256, dtype="bf16", seed=seed,
+                      u_mean=u_mean)
+
+
+def test_chunk_size_invariance():
+    """The result does not depend on the chunk size ("State Space Duality":
+    the chunk boundary separates the two forms and nothing else)."""
+    w = _bf16_case()
+    dev = to_dev(generate(w))
+    outs = [ssd.forward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], dev["D"], q)
+            for q in (32, 64, 128, 256)]
+    torch.cuda.synchronize()
+    ref = outs[0][0].float().cpu().numpy()
+    for y, fin in outs[1:]:
+        assert rel_err(y.float().cpu().numpy(), ref) <= TOL_BF16
+        assert rel_err(fin.cpu().numpy(), outs[0][1].cpu().numpy()) <= 1e-3
+
+
+def test_diag_broadcast_equals_scalar():
+    """Per-state decays equal across n give the scalar result."""
+    w = small_case(B=1, T=512, H=2, P=64, N=64, G=1, chunk=128, dtype="bf16", seed=22)
+    dev = to_dev(generate(w))
+    y1, f1 = ssd.forward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], dev["D"], w.chunk)
+    a4 = dev["a"].unsqueeze(-1).expand(*dev["a"].shape, w.N).contiguous()
+    y2, f2 = ssd.forward(dev["x"], a4, dev["Bm"], dev["Cm"], dev["D"], w.chunk)
+    torch.cuda.synchronize()
+    assert rel_err(y2.float().cpu().numpy(), y1.float().cpu().numpy()) <= TOL_BF16
+    assert rel_err(f2.cpu().numpy(), f1.cpu().numpy()) <= 1e-3
+
+
+def test_grouping_equals_replication():
+    w = _bf16_case(H=8, G=2, seed=23)
+    dev = to_dev(generate(w))
+    y1, f1 = ssd.forward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], dev["D"], w.chunk)
+    rep = lambda m: m.repeat_interleave(w.H // w.G, dim=2).contiguous()
+    y2, f2 = ssd.forward(dev["x"], dev["a"], rep(dev["Bm"]), rep(dev["Cm"]), dev["D"], w.chunk)
+    torch.cuda.synchronize()
+    assert rel_err(y2.float().cpu().numpy(), y1.float().cpu().numpy()) <= 1e-6
+    assert rel_err(f2.cpu().numpy(), f1.cpu().numpy()) <= 1e-6
+
+
+def test_first_decay_and_causality():
+    w = _bf16_case(seed=24)
+    dev = to_dev(generate(w))
+    y0, _ = ssd.forward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], dev["D"], w.chunk)
+    a2 = dev["a"].clone()
+    a2[:, 0] = -9.0
+    y1, _ = ssd.forward(dev["x"], a2, dev["Bm"], dev["Cm"], dev["D"], w.chunk)
+    x2 = dev["x"].clone()
+    s = 700
+    x2[:, s] += 3.0
+    y2, _ = ssd.forward(x2, dev["a"], dev["Bm"], dev["Cm"], dev["D"], w.chunk)
+    torch.cuda.synchronize()
+    assert rel_err(y1.float().cpu().numpy(), y0.float().cpu().numpy()) <= 1e-6
+    assert torch.equal(y2[:, :s], y0[:, :s])
+    assert not torch.equal(y2[:, s:], y0[:, s:])
+
+
+@pytest.mark.parametrize("path", [ssd.PATH_SIMT, ssd.PATH_AUTO], ids=["simt", "auto"])
+def test_deterministic(path):
+    w = _bf16_case(seed=25)
+    dev = to_dev(generate(w))
+    r1 = ssd.forward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], dev["D"], w.chunk, path=path)
+    r2 = ssd.forward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], dev["D"], w.chunk, path=path)
+    torch.cuda.synchronize()
+    assert torch.equal(r1[0], r2[0]) and torch.equal(r1[1], r2[1])
+
+
+def test_host_buffer_entry_point():
+    """ssd_forward_host (host inputs and outputs, copies queued by the library)
+    gives the device forward's result bit for bit."""
+    w = _bf16_case(seed=26)
+    inp = generate(w)
+    dev = to_dev(inp)
+    y_ref, f_ref = ssd.forward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], dev["D"], w.chunk)
+    shape = ssd.shape_of(dev["x"], dev["a"], dev["Bm"], w.chunk)
+    pin = {k: v.pin_memory() for k, v in inp.items()}
+    y_h = torch.empty_like(inp["x"]).pin_memory()
+    f_h = torch.empty((w.B, w.H, w.N, w.P), dtype=torch.float32).pin_memory()
+    buf = torch.empty(ssd.forward_host_bytes(shape), dtype=torch.uint8, device="cuda")
+    ssd.forward_host(shape, pin["x"], pin["a"], pin["Bm"], pin["Cm"], pin["D"], y_h, f_h, buf)
+    torch.cuda.synchronize()
+    assert torch.equal(y_h, y_ref.cpu()) and torch.equal(f_h, f_ref.cpu())
