@@ -88,16 +88,6 @@ def _oracle_chunked(inp, w):
     return cum, S, Hin, y, fin
 
 
-def _impls(shape, which):
-    out = [ssd.IMPL_SIMT]
-    return out + ([ssd.IMPL_TC] if which(shape) else [])
-
-
-def _tc_state_ok(shape):
-    return shape.dtype == ssd.SSD_DTYPE_BF16 and not shape.a_per_state and shape.N == 128 \
-        and shape.P == 64 and shape.chunk in (64, 128, 256)
-
-
 @pytest.mark.parametrize("w", CASES, ids=_ids(CASES))
 def test_step_chunk_cumsum(w):
     inp = generate(w)
@@ -204,8 +194,13 @@ def test_grouping_equals_replication():
     assert rel_err(f2.cpu().numpy(), f1.cpu().numpy()) <= 1e-6
 
 
-def test_first_decay_and_causality():
-    w = _bf16_case(seed=24)
+@pytest.mark.parametrize("dtype,tol", [("f32", 1e-5), ("bf16", 4e-3)])
+def test_first_decay_and_causality(dtype, tol):
+    """a_0 multiplies nothing (the product in M_{i,j} runs over k = j+1..i):
+    changing it moves y only by rounding (cum values shift, so the fp32
+    differences round differently; bf16 outputs may flip one ulp).  Outputs
+    before a perturbed input are bitwise unchanged (causal masking)."""
+    w = small_case(B=2, T=1024, H=4, P=64, N=128, G=1, chunk=256, dtype=dtype, seed=24)
     dev = to_dev(generate(w))
     y0, _ = ssd.forward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], dev["D"], w.chunk)
     a2 = dev["a"].clone()
@@ -216,7 +211,7 @@ def test_first_decay_and_causality():
     x2[:, s] += 3.0
     y2, _ = ssd.forward(x2, dev["a"], dev["Bm"], dev["Cm"], dev["D"], w.chunk)
     torch.cuda.synchronize()
-    assert rel_err(y1.float().cpu().numpy(), y0.float().cpu().numpy()) <= 1e-6
+    assert rel_err(y1.float().cpu().numpy(), y0.float().cpu().numpy()) <= tol
     assert torch.equal(y2[:, :s], y0[:, :s])
     assert not torch.equal(y2[:, s:], y0[:, s:])
 
