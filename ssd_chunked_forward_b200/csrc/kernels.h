@@ -32,4 +32,12 @@ cudaError_t launch_chunk_scan_tc(const Dims& d, const void* x, const void* Bm, c
                                  const float* cum, const float* Hin, const float* D, void* y,
                                  cudaStream_t st);
 
+// one persistent kernel: block states, the inter-block recurrence (through an
+// L2-resident ring with bounded waits) and the outputs; 128-token blocks
+bool fused_supported(const Dims& d);
+size_t fused_ring_bytes(const Dims& d);
+cudaError_t launch_fused_tc(const Dims& d, const void* x, const float* a, const void* Bm,
+                            const void* Cm, const float* D, void* y, float* fin, float* ring,
+                            unsigned* flags, int* status, bool test_stall, cudaStream_t st);
+
 }  // namespace ssd

@@ -210,6 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::tc_fence_before();
     __syncthreads();
     if (warp == 1) {
+        __syncwarp();
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem, 128);
     }

@@ -1,0 +1,668 @@
+// scan_tc.cu -- the chunk output step on the fifth-generation tensor cores,
+// standalone (scan mode) and fused with the chunk-state and inter-chunk steps
+// (fused mode).
+//
+// Unit of work: a block of 128 tokens (the MMA's M) of one batch row b, for a
+// slice of `hpb` heads that share one B/C group.  For the block's tokens
+// t, s in [0, 128), head h, and cum the in-block inclusive prefix sum of the
+// log-decays a:
+//   S   = C B^T                         (scores, shared by the slice's heads)
+//   P   = S o L,  L[t,s] = exp(cum_t - cum_s) for s <= t, else 0
+//   Y   = P X                           (quadratic masked form, llms.blog
+//                                        "The Chunk-Wise SSD Algorithm", item 2)
+//   V   = C Hin                         (incoming state, item 5)
+//   y_t = Y_t + exp(cum_t) V_t + D x_t
+// The mask L is applied in registers between the TMEM scores and the bf16
+// operand in shared memory; it never reaches HBM.
+//
+// Fused mode also forms the block's own state Z = B^T (w o X),
+// w_s = exp(cum_127 - cum_s) (item 3), and the recurrence
+//   h_j = exp(cum_127) h_{j-1} + Z_j                         (item 4)
+// across blocks: each (b, h) chain hands its fp32 state from block j-1 to
+// block j through a two-slot ring in global memory (it stays in L2) and a
+// per-chain counter, with a bounded wait on the consumer side.  Work items are
+// ordered block-major and scheduled round-robin over persistent CTAs, so the
+// block a CTA waits for belongs to a smaller item index and can always finish.
+//
+// A chunk of 256 tokens is two such blocks: the strictly-lower 128x128 block
+// of its quadratic form goes through the exact factorisation
+// L[t,s] = exp(cum_t - cum_127) exp(cum_127 - cum_s), i.e. through the state
+// at the block boundary ("State Space Duality", "Two algorithms for one
+// operator": off-diagonal blocks are low-rank).
+//
+// Warp roles (320 threads): 0 TMA producer; 1 MMA issuer and TMEM owner;
+// 2-9 compute: two groups of four warps, each group covering all 128 TMEM
+// lanes, group g owning columns [32g, 32g+32) of P-wide tiles and
+// [64g, 64g+64) of the scores.  TMEM (512 columns): scores 0-127, then two
+// buffers of {Z, Y, V} x 64 columns, alternating per head.
+#include "../common.cuh"
+#include "../kernels.h"
+#include "../tc_common.cuh"
+#include "../tmap.h"
+
+namespace ssd {
+namespace {
+
+constexpr int kBlk = 128;
+constexpr int kN = 128;
+constexpr int kP = 64;
+constexpr int kStages = 3;
+constexpr int kHpbMax = 8;
+constexpr int kThreads = 320;
+constexpr uint32_t kTile = kBlk * 128;  // 128 rows x 128 bytes
+
+enum { kScan = 0, kFused = 1 };
+
+struct __align__(8) Bars {
+    uint64_t bc_full, bc_empty, s_full, s_empty;
+    uint64_t x_full[kStages], x_empty[kStages];
+    uint64_t xw_full, xw_empty, p_full, p_empty, h_full, h_empty;
+    uint64_t y_full[2], v_full[2], z_full[2], t_empty[2];
+    uint64_t done;
+};
+
+struct ScanParams {
+    const float* a;    // fused: log-decays [B,T,H]
+    const float* cum;  // scan: in-block cumsum [B,H,nblk,128]
+    const float* hin;  // scan: incoming states [B,H,nblk,N,P]
+    const float* D;    // [H] or null
+    float* ring;       // fused: [B*H][2][N*P]
+    unsigned* flags;   // fused: [B*H] blocks published per chain
+    float* fin;        // fused: final state [B,H,N,P] or null
+    int* status;       // device status word or null
+    int T, H, G, nblk, hpb, nslices, n_items;
+    int test_stall;
+};
+
+// smem layout (offsets from the 1024-aligned base)
+constexpr uint32_t OFF_B = 0;
+constexpr uint32_t OFF_C = OFF_B + 2 * kTile;
+constexpr uint32_t OFF_X = OFF_C + 2 * kTile;
+constexpr uint32_t OFF_XW = OFF_X + kStages * kTile;
+constexpr uint32_t OFF_P = OFF_XW + kTile;
+constexpr uint32_t OFF_H = OFF_P + 2 * kTile;
+constexpr uint32_t OFF_Y = OFF_H + kTile;
+constexpr uint32_t OFF_CUM = OFF_Y + 2 * kTile;
+constexpr uint32_t OFF_VEC = OFF_CUM + kHpbMax * kBlk * 4;
+constexpr uint32_t OFF_BAR = OFF_VEC + 4 * kBlk * 4;
+constexpr uint32_t OFF_MISC = OFF_BAR + ((sizeof(Bars) + 15) / 16) * 16;
+constexpr size_t kSmemBytes = 1024 + OFF_MISC + 16;
+
+// TMEM columns
+constexpr uint32_t COL_S = 0;
+__device__ __forceinline__ uint32_t col_z(int buf) { return 128 + 192 * buf; }
+__device__ __forceinline__ uint32_t col_y(int buf) { return 192 + 192 * buf; }
+__device__ __forceinline__ uint32_t col_v(int buf) { return 256 + 192 * buf; }
+
+__device__ __forceinline__ void compute_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_u32(unsigned* p, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+struct Item {
+    int b, j, h0, g;
+};
+__device__ __forceinline__ Item decode_item(int it, const ScanParams& p, int B) {
+    Item r;
+    const int per_blk = B * p.nslices;
+    r.j = it / per_blk;
+    const int rem = it - r.j * per_blk;
+    r.b = rem / p.nslices;
+    const int sl = rem - r.b * p.nslices;
+    const int HG = p.H / p.G;
+    const int spg = HG / p.hpb;
+    r.g = sl / spg;
+    r.h0 = r.g * HG + (sl - r.g * spg) * p.hpb;
+    return r;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
+                   const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y,
+                   const ScanParams p, int B) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+    uint8_t* sB = sm + OFF_B;
+    uint8_t* sC = sm + OFF_C;
+    uint8_t* sX = sm + OFF_X;
+    uint8_t* sXw = sm + OFF_XW;
+    uint8_t* sP = sm + OFF_P;
+    uint8_t* sH = sm + OFF_H;
+    uint8_t* sY = sm + OFF_Y;
+    float* sCum = reinterpret_cast<float*>(sm + OFF_CUM);  // [hpb][128]
+    float* sW = reinterpret_cast<float*>(sm + OFF_VEC);    // [128]
+    float* sColf = sW + kBlk;                              // [3][128]
+    Bars* bars = reinterpret_cast<Bars*>(sm + OFF_BAR);
+    uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
+    int* sAbort = reinterpret_cast<int*>(sm + OFF_MISC + 4);
+    volatile int* abort_v = sAbort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        tc::mbar_init(&bars->bc_full, 1);
+        tc::mbar_init(&bars->bc_empty, 1);
+        tc::mbar_init(&bars->s_full, 1);
+        tc::mbar_init(&bars->s_empty, 8);
+        for (int s = 0; s < kStages; ++s) {
+            tc::mbar_init(&bars->x_full[s], 1);
+            tc::mbar_init(&bars->x_empty[s], 9);  // Y MMA commit + 8 compute warps
+        }
+        tc::mbar_init(&bars->xw_full, 8);
+        tc::mbar_init(&bars->xw_empty, 1);
+        tc::mbar_init(&bars->p_full, 8);
+        tc::mbar_init(&bars->p_empty, 1);
+        tc::mbar_init(&bars->h_full, 8);
+        tc::mbar_init(&bars->h_empty, 1);
+        for (int s = 0; s < 2; ++s) {
+            tc::mbar_init(&bars->y_full[s], 1);
+            tc::mbar_init(&bars->v_full[s], 1);
+            tc::mbar_init(&bars->z_full[s], 1);
+            tc::mbar_init(&bars->t_empty[s], 8);
+        }
+        tc::mbar_init(&bars->done, 1);
+        *sAbort = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(sTmem, 512);
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = *sTmem;
+
+    auto fail = [&]() {
+        *reinterpret_cast<volatile int*>(sAbort) = 1;
+        if (p.status) atomicExch(p.status, kDevTimeout);
+    };
+
+    if (warp == 0) {
+        // =============================================== TMA producer ====
+        if (lane == 0) {
+            tc::prefetch_tmap(&tm_x);
+            tc::prefetch_tmap(&tm_b);
+            tc::prefetch_tmap(&tm_c);
+            tc::prefetch_tmap(&tm_y);
+            uint32_t xc = 0, itc = 0;
+            bool ok = true;
+            for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x, ++itc) {
+                const Item w = decode_item(it, p, B);
+                const int row0 = w.b * p.T + w.j * kBlk;
+                if (itc > 0 && !tc::mbar_wait(&bars->bc_empty, (itc - 1) & 1, abort_v)) {
+                    ok = false;
+                    break;
+                }
+                tc::mbar_arrive_expect_tx(&bars->bc_full, 4 * kTile);
+                tc::tma_load_3d(sB, &tm_b, &bars->bc_full, 0, w.g, row0);
+                tc::tma_load_3d(sB + kTile, &tm_b, &bars->bc_full, 64, w.g, row0);
+                tc::tma_load_3d(sC, &tm_c, &bars->bc_full, 0, w.g, row0);
+                tc::tma_load_3d(sC + kTile, &tm_c, &bars->bc_full, 64, w.g, row0);
+                for (int i = 0; i < p.hpb; ++i, ++xc) {
+                    const uint32_t st = xc % kStages;
+                    if (xc >= kStages &&
+                        !tc::mbar_wait(&bars->x_empty[st], ((xc / kStages) - 1) & 1, abort_v)) {
+                        ok = false;
+                        break;
+                    }
+                    tc::mbar_arrive_expect_tx(&bars->x_full[st], kTile);
+                    tc::tma_load_3d(sX + st * kTile, &tm_x, &bars->x_full[st], 0, w.h0 + i, row0);
+                }
+            }
+            if (!ok) fail();
+            // no copy may still be landing in shared memory when the CTA exits
+            const uint32_t first = xc > (uint32_t)kStages ? xc - kStages : 0u;
+            for (uint32_t c = first; c < xc; ++c)
+                tc::mbar_wait(&bars->x_full[c % kStages], (c / kStages) & 1, nullptr, 200000000ull);
+            if (itc > 0) tc::mbar_wait(&bars->bc_full, (itc - 1) & 1, nullptr, 200000000ull);
+        }
+    } else if (warp == 1) {
+        // ================================================ MMA issuer ====
+        if (lane == 0) {
+            constexpr uint32_t id_s = tc::idesc_bf16_f32(128, 128, 0, 0);
+            constexpr uint32_t id_z = tc::idesc_bf16_f32(128, kP, 1, 1);
+            constexpr uint32_t id_y = tc::idesc_bf16_f32(128, kP, 0, 1);
+            constexpr uint32_t id_v = tc::idesc_bf16_f32(128, kP, 0, 1);
+            const uint32_t aB = tc::smem_u32(sB), aC = tc::smem_u32(sC), aX = tc::smem_u32(sX);
+            const uint32_t aXw = tc::smem_u32(sXw), aP = tc::smem_u32(sP), aH = tc::smem_u32(sH);
+            uint32_t hc = 0, xc = 0, itc = 0;
+            bool ok = true;
+            auto issue_v = [&](uint32_t head) -> bool {
+                const int buf = head & 1;
+                if (!tc::mbar_wait(&bars->h_full, head & 1, abort_v)) return false;
+                tc::tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t ad = tc::smem_desc_sw128(aC + (kk >> 2) * kTile + (kk & 3) * 32, 16, 1024);
+                    const uint64_t bd = tc::smem_desc_sw128(aH + kk * 2048, kTile, 1024);
+                    tc::mma_ss(tmem + col_v(buf), ad, bd, id_v, kk > 0);
+                }
+                tc::mma_commit(&bars->v_full[buf]);
+                tc::mma_commit(&bars->h_empty);
+                return true;
+            };
+            for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x, ++itc) {
+                ok = tc::mbar_wait(&bars->bc_full, itc & 1, abort_v) &&
+                     (itc == 0 || tc::mbar_wait(&bars->s_empty, (itc - 1) & 1, abort_v));
+                if (!ok) break;
+                tc::tc_fence_after();
+                // scores S = C B^T: M = t, N = s, K = n (both K-major)
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * kTile + (kk & 3) * 32;
+                    tc::mma_ss(tmem + COL_S, tc::smem_desc_sw128(aC + off, 16, 1024),
+                               tc::smem_desc_sw128(aB + off, 16, 1024), id_s, kk > 0);
+                }
+                tc::mma_commit(&bars->s_full);
+                for (int i = 0; i < p.hpb; ++i, ++hc, ++xc) {
+                    const int buf = hc & 1;
+                    const uint32_t st = xc % kStages;
+                    if (hc >= 2 && !tc::mbar_wait(&bars->t_empty[buf], ((hc >> 1) - 1) & 1, abort_v)) {
+                        ok = false;
+                        break;
+                    }
+                    if (MODE == kFused) {
+                        // block state Z = B^T (w o X): M = n (MN-major B tile), N = p, K = s
+                        if (!tc::mbar_wait(&bars->xw_full, hc & 1, abort_v)) { ok = false; break; }
+                        tc::tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            tc::mma_ss(tmem + col_z(buf), tc::smem_desc_sw128(aB + kk * 2048, kTile, 1024),
+                                       tc::smem_desc_sw128(aXw + kk * 2048, kTile, 1024), id_z, kk > 0);
+                        tc::mma_commit(&bars->z_full[buf]);
+                        tc::mma_commit(&bars->xw_empty);
+                    }
+                    // Y = P X: M = t, N = p, K = s (P K-major, X MN-major)
+                    ok = tc::mbar_wait(&bars->p_full, hc & 1, abort_v) &&
+                         tc::mbar_wait(&bars->x_full[st], (xc / kStages) & 1, abort_v);
+                    if (!ok) break;
+                    tc::tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint64_t ad = tc::smem_desc_sw128(aP + (kk >> 2) * kTile + (kk & 3) * 32, 16, 1024);
+                        const uint64_t bd = tc::smem_desc_sw128(aX + st * kTile + kk * 2048, kTile, 1024);
+                        tc::mma_ss(tmem + col_y(buf), ad, bd, id_y, kk > 0);
+                    }
+                    tc::mma_commit(&bars->y_full[buf]);
+                    tc::mma_commit(&bars->p_empty);
+                    tc::mma_commit(&bars->x_empty[st]);
+                    // V = C Hin of the previous head (its state is ready by now)
+                    if (i > 0 && !issue_v(hc - 1)) { ok = false; break; }
+                }
+                if (!ok) break;
+                if (!issue_v(hc - 1)) { ok = false; break; }
+                tc::mma_commit(&bars->bc_empty);
+            }
+            if (!ok) fail();
+            // every MMA issued must be complete before TMEM is released
+            tc::mma_commit(&bars->done);
+            tc::mbar_wait(&bars->done, 0, nullptr, 200000000ull);
+        }
+    } else {
+        // ================================================ compute (8 warps) ====
+        const int ct = threadIdx.x - 64;  // 0..255
+        const int cg = ct >> 7;           // column group 0/1
+        const int quad = warp & 3;        // TMEM lane quadrant
+        const int row = quad * 32 + lane; // TMEM lane = tile row
+        const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+        uint32_t hc = 0, xc = 0, itc = 0;
+
+        auto sync_ok = [&](bool ok) -> bool {
+            if (!ok) fail();
+            compute_sync();
+            __syncwarp();
+            return *abort_v == 0;
+        };
+
+        for (int it = blockIdx.x; it < p.n_items; it += gridDim.x, ++itc) {
+            const Item w = decode_item(it, p, B);
+            const int tok0 = w.b * p.T + w.j * kBlk;
+            const bool last_blk = (w.j == p.nblk - 1);
+            // ---- per-block cumulative log-decay of every head of the slice
+            if (cg == 0) {
+                if (MODE == kFused) {
+                    const float* arow = p.a + (size_t)(tok0 + ct) * p.H + w.h0;
+                    for (int i = 0; i < p.hpb; ++i) sCum[i * kBlk + ct] = arow[i];
+                } else {
+                    for (int i = 0; i < p.hpb; ++i)
+                        sCum[i * kBlk + ct] =
+                            p.cum[(((size_t)w.b * p.H + w.h0 + i) * p.nblk + w.j) * kBlk + ct];
+                }
+            }
+            compute_sync();
+            if (MODE == kFused) {
+                const int cw = ct >> 5;  // compute warp 0..7 scans head cw
+                if (cw < p.hpb) {
+                    float* c = sCum + cw * kBlk + lane * 4;
+                    float v0 = c[0], v1 = v0 + c[1], v2 = v1 + c[2], v3 = v2 + c[3];
+                    const float excl = warp_inclusive_scan(v3) - v3;
+                    c[0] = v0 + excl; c[1] = v1 + excl; c[2] = v2 + excl; c[3] = v3 + excl;
+                }
+                compute_sync();
+            }
+            // ---- T5: y = Y + exp(cum) V + D x -> bf16 -> TMA store
+            auto epilogue = [&](int hi, uint32_t hcount, uint32_t xcount) -> bool {
+                const int eb = hcount & 1;
+                const uint32_t est = xcount % kStages;
+                bool eok = tc::mbar_wait(&bars->x_full[est], (xcount / kStages) & 1, abort_v) &&
+                           tc::mbar_wait(&bars->y_full[eb], (hcount >> 1) & 1, abort_v) &&
+                           tc::mbar_wait(&bars->v_full[eb], (hcount >> 1) & 1, abort_v);
+                if (ct == 0) tc::bulk_wait_read<1>();  // sY[eb] free again
+                if (!sync_ok(eok)) return false;
+                tc::tc_fence_after();
+                float yv[32], vv[32];
+                tc::tmem_ld32(lane_base + col_y(eb) + 32 * cg, yv);
+                tc::tmem_ld32(lane_base + col_v(eb) + 32 * cg, vv);
+                tc::tmem_ld_wait();
+                const float* ecum_src = sCum + hi * kBlk;
+                const float ecum = __expf(ecum_src[row]);
+                const float dv = p.D ? p.D[w.h0 + hi] : 0.f;
+                const uint8_t* xs = sX + est * kTile;
+                uint8_t* ys = sY + eb * kTile;
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const uint32_t off = tc::sw128_offset(row, 4 * cg + c4);
+                    uint4 xv = *reinterpret_cast<const uint4*>(xs + off);
+                    const uint32_t* xu = reinterpret_cast<const uint32_t*>(&xv);
+                    uint32_t o[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 xf = tc::unpack_bf16x2(xu[e]);
+                        const int k0 = 8 * c4 + 2 * e;
+                        const float y0 = fmaf(ecum, vv[k0], yv[k0]) + dv * xf.x;
+                        const float y1 = fmaf(ecum, vv[k0 + 1], yv[k0 + 1]) + dv * xf.y;
+                        o[e] = tc::pack_bf16x2(y0, y1);
+                    }
+                    *reinterpret_cast<uint4*>(ys + off) = make_uint4(o[0], o[1], o[2], o[3]);
+                }
+                tc::fence_proxy_async_smem();
+                tc::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    tc::mbar_arrive(&bars->t_empty[eb]);
+                    tc::mbar_arrive(&bars->x_empty[est]);
+                }
+                compute_sync();
+                if (ct == 0) {
+                    tc::tma_store_3d(&tm_y, ys, 0, w.h0 + hi, tok0);
+                    tc::bulk_commit();
+                }
+                return true;
+            };
+            bool ok = true;
+            for (int i = 0; i < p.hpb; ++i, ++hc, ++xc) {
+                const int h = w.h0 + i;
+                const int buf = hc & 1;
+                const uint32_t st = xc % kStages;
+                const float* cum = sCum + i * kBlk;
+                // ---- T1: decay vectors of this head
+                if (cg == 0) {
+                    const float c = cum[ct];
+                    sW[ct] = __expf(cum[kBlk - 1] - c);
+                    sColf[ct] = ct < 32 ? __expf(cum[31] - c) : 0.f;
+                    sColf[kBlk + ct] = ct < 64 ? __expf(cum[63] - c) : 0.f;
+                    sColf[2 * kBlk + ct] = ct < 96 ? __expf(cum[95] - c) : 0.f;
+                }
+                // ---- T2: weighted copy of x for the block state (fused)
+                if (MODE == kFused) {
+                    ok = tc::mbar_wait(&bars->x_full[st], (xc / kStages) & 1, abort_v) &&
+                         (hc == 0 || tc::mbar_wait(&bars->xw_empty, (hc - 1) & 1, abort_v));
+                    if (!sync_ok(ok)) break;
+                    const uint8_t* xs = sX + st * kTile;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int c = ct + 256 * q;
+                        const float wgt = sW[c >> 3];
+                        uint4 v = *reinterpret_cast<const uint4*>(xs + c * 16);
+                        uint32_t* u = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = tc::unpack_bf16x2(u[e]);
+                            u[e] = tc::pack_bf16x2(f.x * wgt, f.y * wgt);
+                        }
+                        *reinterpret_cast<uint4*>(sXw + c * 16) = v;
+                    }
+                    tc::fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(&bars->xw_full);
+                }
+                // ---- T3: P = S o L  -> bf16, K-major in sP
+                ok = (i > 0 || tc::mbar_wait(&bars->s_full, itc & 1, abort_v)) &&
+                     (hc == 0 || tc::mbar_wait(&bars->p_empty, (hc - 1) & 1, abort_v));
+                if (!sync_ok(ok)) break;
+                tc::tc_fence_after();
+                {
+                    const float ct_cum = cum[row];
+                    const float rowf = quad > 0 ? __expf(ct_cum - cum[32 * quad - 1]) : 0.f;
+                    const float* colf = sColf + (quad > 0 ? (quad - 1) * kBlk : 0);
+                    uint8_t* ptile = sP + cg * kTile;
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const int sb = 2 * cg + q;  // 32-column sub-block of s
+                        uint32_t pk[16];
+                        if (sb > quad) {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                        } else {
+                            float v[32];
+                            tc::tmem_ld32(lane_base + COL_S + 32 * sb, v);
+                            tc::tmem_ld_wait();
+                            if (sb < quad) {
+#pragma unroll
+                                for (int e = 0; e < 32; ++e) v[e] *= rowf * colf[32 * sb + e];
+                            } else {
+#pragma unroll
+                                for (int e = 0; e < 32; ++e) {
+                                    const int s = 32 * sb + e;
+                                    v[e] = (s <= row) ? v[e] * __expf(ct_cum - cum[s]) : 0.f;
+                                }
+                            }
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) pk[e] = tc::pack_bf16x2(v[2 * e], v[2 * e + 1]);
+                        }
+#pragma unroll
+                        for (int c4 = 0; c4 < 4; ++c4) {
+                            const uint32_t chunk = 4 * q + c4;
+                            *reinterpret_cast<uint4*>(ptile + tc::sw128_offset(row, chunk)) =
+                                make_uint4(pk[4 * c4], pk[4 * c4 + 1], pk[4 * c4 + 2], pk[4 * c4 + 3]);
+                        }
+                    }
+                }
+                tc::fence_proxy_async_smem();
+                tc::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    tc::mbar_arrive(&bars->p_full);
+                    if (i == p.hpb - 1) tc::mbar_arrive(&bars->s_empty);
+                }
+                // ---- T5 of the previous head
+                if (i > 0 && !epilogue(i - 1, hc - 1, xc - 1)) { ok = false; break; }
+                // ---- T4: incoming state (and, fused, the chain hand-off)
+                {
+                    const int chain = w.b * p.H + h;
+                    float hin[32];
+                    if (MODE == kFused) {
+                        ok = tc::mbar_wait(&bars->z_full[buf], (hc >> 1) & 1, abort_v) &&
+                             (hc == 0 || tc::mbar_wait(&bars->h_empty, (hc - 1) & 1, abort_v));
+                        if (ok && w.j > 0 && ct == 0) {
+                            // bounded wait for the previous block of this chain
+                            const unsigned* f = p.flags + chain;
+                            const uint64_t t0 = tc::globaltimer_ns();
+                            for (uint32_t spin = 0; ld_acquire_u32(f) < (unsigned)w.j; ++spin) {
+                                if ((spin & 15) == 15) {
+                                    if (*abort_v || (p.status && *(volatile int*)p.status) ||
+                                        tc::globaltimer_ns() - t0 > 2000000000ull) {
+                                        ok = false;
+                                        break;
+                                    }
+                                }
+                                __nanosleep(64);
+                            }
+                        }
+                        if (!sync_ok(ok)) break;
+                        tc::tc_fence_after();
+                        float zv[32];
+                        tc::tmem_ld32(lane_base + col_z(buf) + 32 * cg, zv);
+                        tc::tmem_ld_wait();
+                        const size_t slot = (size_t)kN * kP;
+                        float* ring = p.ring + (size_t)chain * 2 * slot;
+                        const size_t roff = (size_t)row * kP + 32 * cg;
+                        if (w.j > 0) {
+                            const float4* src = reinterpret_cast<const float4*>(ring + ((w.j - 1) & 1) * slot + roff);
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) {
+                                const float4 v = __ldcg(src + q);
+                                hin[4 * q] = v.x; hin[4 * q + 1] = v.y; hin[4 * q + 2] = v.z; hin[4 * q + 3] = v.w;
+                            }
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) hin[e] = 0.f;
+                        }
+                        const float eL = __expf(cum[kBlk - 1]);
+                        float hn[32];
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) hn[e] = fmaf(eL, hin[e], zv[e]);
+                        const bool publish = !(p.test_stall && chain == 0 && w.j == 0);
+                        if (publish) {
+                            float4* dst = reinterpret_cast<float4*>(ring + (w.j & 1) * slot + roff);
+#pragma unroll
+                            for (int q = 0; q < 8; ++q)
+                                __stcg(dst + q, make_float4(hn[4 * q], hn[4 * q + 1], hn[4 * q + 2], hn[4 * q + 3]));
+                            __threadfence();
+                        }
+                        if (last_blk && p.fin) {
+                            float4* fd = reinterpret_cast<float4*>(p.fin + (size_t)chain * kN * kP + roff);
+#pragma unroll
+                            for (int q = 0; q < 8; ++q)
+                                fd[q] = make_float4(hn[4 * q], hn[4 * q + 1], hn[4 * q + 2], hn[4 * q + 3]);
+                        }
+                        compute_sync();
+                        if (publish && ct == 0) st_release_u32(p.flags + chain, (unsigned)(w.j + 1));
+                    } else {
+                        ok = (hc == 0 || tc::mbar_wait(&bars->h_empty, (hc - 1) & 1, abort_v));
+                        if (!sync_ok(ok)) break;
+                        const float4* src = reinterpret_cast<const float4*>(
+                            p.hin + ((((size_t)w.b * p.H + h) * p.nblk + w.j) * kN + row) * kP + 32 * cg);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const float4 v = __ldg(src + q);
+                            hin[4 * q] = v.x; hin[4 * q + 1] = v.y; hin[4 * q + 2] = v.z; hin[4 * q + 3] = v.w;
+                        }
+                    }
+                    // Hin as the bf16 B operand of V = C Hin: rows n, 64 p per row (MN-major)
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        uint4 v;
+                        v.x = tc::pack_bf16x2(hin[8 * c4 + 0], hin[8 * c4 + 1]);
+                        v.y = tc::pack_bf16x2(hin[8 * c4 + 2], hin[8 * c4 + 3]);
+                        v.z = tc::pack_bf16x2(hin[8 * c4 + 4], hin[8 * c4 + 5]);
+                        v.w = tc::pack_bf16x2(hin[8 * c4 + 6], hin[8 * c4 + 7]);
+                        *reinterpret_cast<uint4*>(sH + tc::sw128_offset(row, 4 * cg + c4)) = v;
+                    }
+                    tc::fence_proxy_async_smem();
+                    tc::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(&bars->h_full);
+                }
+            }
+            if (!ok) break;
+            // ---- T5 of the slice's last head
+            if (!epilogue(p.hpb - 1, hc - 1, xc - 1)) break;
+        }
+        if (ct == 0) tc::bulk_wait<0>();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, 512);
+    }
+}
+
+int heads_per_item(const Dims& d) {
+    const int HG = d.H / d.G;
+    for (int c = kHpbMax; c >= 1; --c)
+        if (HG % c == 0) return c;
+    return 1;
+}
+
+int num_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+    return n > 0 ? n : 148;
+}
+
+template <int MODE>
+cudaError_t launch(const Dims& d, const void* x, const void* Bm, const void* Cm, void* y,
+                   ScanParams p, cudaStream_t st) {
+    CUtensorMap tx, tb, tcm, ty;
+    cudaError_t e = make_tmap_bf16_3d(&tx, x, d.P, d.H, (uint64_t)d.B * d.T, kBlk);
+    if (e == cudaSuccess) e = make_tmap_bf16_3d(&tb, Bm, d.N, d.G, (uint64_t)d.B * d.T, kBlk);
+    if (e == cudaSuccess) e = make_tmap_bf16_3d(&tcm, Cm, d.N, d.G, (uint64_t)d.B * d.T, kBlk);
+    if (e == cudaSuccess) e = make_tmap_bf16_3d(&ty, y, d.P, d.H, (uint64_t)d.B * d.T, kBlk);
+    if (e != cudaSuccess) return e;
+    p.T = d.T; p.H = d.H; p.G = d.G;
+    p.nblk = d.T / kBlk;
+    p.hpb = heads_per_item(d);
+    p.nslices = d.G * ((d.H / d.G) / p.hpb);
+    const long long items = (long long)p.nblk * d.B * p.nslices;
+    if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
+    p.n_items = (int)items;
+    const int grid = (int)(items < num_sms() ? items : num_sms());
+    e = cudaFuncSetAttribute(scan_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    scan_tc_kernel<MODE><<<grid, kThreads, kSmemBytes, st>>>(tx, tb, tcm, ty, p, d.B);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool chunk_scan_tc_supported(const Dims& d) {
+    return d.bf16 && !d.diag && d.N == kN && d.P == kP && d.Q == kBlk;
+}
+
+cudaError_t launch_chunk_scan_tc(const Dims& d, const void* x, const void* Bm, const void* Cm,
+                                 const float* cum, const float* Hin, const float* D, void* y,
+                                 cudaStream_t st) {
+    if (!chunk_scan_tc_supported(d)) return cudaErrorNotSupported;
+    ScanParams p = {};
+    p.cum = cum;
+    p.hin = Hin;
+    p.D = D;
+    return launch<kScan>(d, x, Bm, Cm, y, p, st);
+}
+
+bool fused_supported(const Dims& d) {
+    return d.bf16 && !d.diag && d.N == kN && d.P == kP && d.Q % kBlk == 0;
+}
+
+size_t fused_ring_bytes(const Dims& d) { return (size_t)d.B * d.H * 2 * kN * kP * sizeof(float); }
+
+cudaError_t launch_fused_tc(const Dims& d, const void* x, const float* a, const void* Bm,
+                            const void* Cm, const float* D, void* y, float* fin, float* ring,
+                            unsigned* flags, int* status, bool test_stall, cudaStream_t st) {
+    if (!fused_supported(d)) return cudaErrorNotSupported;
+    ScanParams p = {};
+    p.a = a;
+    p.D = D;
+    p.ring = ring;
+    p.flags = flags;
+    p.fin = fin;
+    p.status = status;
+    p.test_stall = test_stall ? 1 : 0;
+    return launch<kFused>(d, x, Bm, Cm, y, p, st);
+}
+
+}  // namespace ssd

@@ -44,39 +44,65 @@ Dims dims_of(const ssd_shape* s) {
     return d;
 }
 
+// The modular path runs its steps on 128-token blocks when the tensor-core
+// kernels serve the shape and the chunk is a multiple of 128 (a chunk of Q
+// tokens is Q/128 such blocks; the result is the same up to rounding).
+Dims modular_dims(const Dims& d) {
+    Dims e = d;
+    if (d.Q % 128 == 0 && d.Q > 128) {
+        e.Q = 128;
+        e.nc = d.T / 128;
+        if (!ssd::chunk_scan_tc_supported(e)) return d;
+    }
+    return e;
+}
+
 size_t cum_bytes(const Dims& d) {
     return (size_t)d.B * d.H * d.nc * d.Q * (d.diag ? d.N : 1) * sizeof(float);
 }
 size_t states_bytes(const Dims& d) {
     return (size_t)d.B * d.H * d.nc * d.N * d.P * sizeof(float);
 }
+size_t flags_bytes(const Dims& d) { return round_up((size_t)d.B * d.H * sizeof(unsigned), kAlign); }
 
 struct Workspace {
-    int* ctrl;
-    float* cum;
-    float* states;
+    int* ctrl;        // [0] = device status word
+    unsigned* flags;  // fused path: blocks published per (b, h) chain
+    float* ring;      // fused path: two fp32 state slots per chain
+    float* cum;       // modular path
+    float* states;    // modular path
 };
 
-size_t modular_ws(const Dims& d) {
-    return kCtrlBytes + round_up(cum_bytes(d), kAlign) + round_up(states_bytes(d), kAlign);
+size_t workspace_bytes(const Dims& d) {
+    const Dims m = modular_dims(d);
+    const size_t cum = round_up(cum_bytes(m) > cum_bytes(d) ? cum_bytes(m) : cum_bytes(d), kAlign);
+    const size_t st = round_up(states_bytes(m) > states_bytes(d) ? states_bytes(m) : states_bytes(d), kAlign);
+    const size_t ring = ssd::fused_supported(d) ? round_up(ssd::fused_ring_bytes(d), kAlign) : 0;
+    return kCtrlBytes + flags_bytes(d) + ring + cum + st;
 }
 
 Workspace carve(void* ws, const Dims& d) {
+    const Dims m = modular_dims(d);
     char* p = (char*)ws;
     Workspace w;
     w.ctrl = (int*)p;
     p += kCtrlBytes;
+    w.flags = (unsigned*)p;
+    p += flags_bytes(d);
+    w.ring = (float*)p;
+    p += ssd::fused_supported(d) ? round_up(ssd::fused_ring_bytes(d), kAlign) : 0;
     w.cum = (float*)p;
-    p += round_up(cum_bytes(d), kAlign);
+    p += round_up(cum_bytes(m) > cum_bytes(d) ? cum_bytes(m) : cum_bytes(d), kAlign);
     w.states = (float*)p;
     return w;
 }
 
 ssd_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA; }
 
-ssd_status run_modular(const Dims& d, const void* x, const float* a, const void* Bm,
+ssd_status run_modular(const Dims& d0, const void* x, const float* a, const void* Bm,
                        const void* Cm, const float* D, void* y, float* fin, const Workspace& w,
                        cudaStream_t st, bool allow_tc) {
+    const Dims d = allow_tc ? modular_dims(d0) : d0;
     cudaError_t e = ssd::launch_chunk_cumsum(d, a, w.cum, st);
     if (e != cudaSuccess) return SSD_ERR_CUDA;
     const bool tc_state = allow_tc && ssd::chunk_state_tc_supported(d);
@@ -109,7 +135,7 @@ const char* ssd_status_string(ssd_status s) {
 
 size_t ssd_workspace_size(const ssd_shape* shape) {
     if (check_shape(shape) != SSD_OK) return 0;
-    return modular_ws(dims_of(shape));
+    return workspace_bytes(dims_of(shape));
 }
 
 int ssd_path_supported(const ssd_shape* shape, unsigned path) {
@@ -119,10 +145,9 @@ int ssd_path_supported(const ssd_shape* shape, unsigned path) {
         case SSD_PATH_AUTO: return 1;
         case SSD_PATH_SIMT: return 1;
         case SSD_PATH_MODULAR: return 1;
-        case SSD_PATH_FUSED: return 0;
+        case SSD_PATH_FUSED: return ssd::fused_supported(d) ? 1 : 0;
         default: return 0;
     }
-    (void)d;
 }
 
 ssd_status ssd_forward_path(const ssd_shape* shape, const void* x, const float* a, const void* Bm,
@@ -143,12 +168,18 @@ ssd_status ssd_forward_path(const ssd_shape* shape, const void* x, const float* 
     if (!ssd_path_supported(shape, path)) return SSD_ERR_UNSUPPORTED;
     cudaStream_t cs = (cudaStream_t)stream;
     const Workspace w = carve(workspace, d);
-    if (cudaMemsetAsync(w.ctrl, 0, kCtrlBytes, cs) != cudaSuccess) return SSD_ERR_CUDA;
+    // status word and per-chain counters start at zero on every call
+    if (cudaMemsetAsync(w.ctrl, 0, kCtrlBytes + flags_bytes(d), cs) != cudaSuccess)
+        return SSD_ERR_CUDA;
+    if (path == SSD_PATH_AUTO) path = ssd::fused_supported(d) ? SSD_PATH_FUSED : SSD_PATH_MODULAR;
     switch (path) {
         case SSD_PATH_SIMT:
             return run_modular(d, x, a, Bm, Cm, D, y, final_state, w, cs, false);
+        case SSD_PATH_FUSED:
+            return cuda_status(ssd::launch_fused_tc(d, x, a, Bm, Cm, D, y, final_state, w.ring,
+                                                    w.flags, w.ctrl,
+                                                    (flags & SSD_FLAG_TEST_STALL) != 0, cs));
         case SSD_PATH_MODULAR:
-        case SSD_PATH_AUTO:
         default:
             return run_modular(d, x, a, Bm, Cm, D, y, final_state, w, cs, true);
     }

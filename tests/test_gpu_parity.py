@@ -34,6 +34,8 @@ CASES = [
     small_case(B=1, T=192, H=4, P=64, N=128, G=2, chunk=64, dtype="bf16", seed=3),
     small_case(B=2, T=768, H=3, P=64, N=128, G=1, chunk=256, dtype="bf16", seed=4),
     small_case(B=1, T=384, H=5, P=64, N=128, G=1, chunk=128, dtype="bf16", seed=5),
+    small_case(B=2, T=1024, H=8, P=64, N=128, G=2, chunk=256, dtype="bf16", seed=13, u_mean=-4.0),
+    small_case(B=1, T=2048, H=16, P=64, N=128, G=1, chunk=128, dtype="bf16", seed=14),
     small_case(B=2, T=256, H=2, P=64, N=64, G=1, chunk=128, dtype="bf16", a_per_state=True, seed=6),
     small_case(B=1, T=60, H=2, P=10, N=12, G=1, chunk=20, dtype="f32", a_per_state=True, seed=7),
 ]
@@ -241,3 +243,25 @@ def test_host_buffer_entry_point():
     ssd.forward_host(shape, pin["x"], pin["a"], pin["Bm"], pin["Cm"], pin["D"], y_h, f_h, buf)
     torch.cuda.synchronize()
     assert torch.equal(y_h, y_ref.cpu()) and torch.equal(f_h, f_ref.cpu())
+
+
+def test_fused_bounded_wait_reports_timeout():
+    """The fused path's hand-off wait is bounded: with the test flag that keeps
+    the first block of chain 0 from publishing its state, the waiting block
+    gives up, the device status reads SSD_ERR_TIMEOUT, and the context stays
+    usable (a normal call right after is correct)."""
+    w = small_case(B=1, T=512, H=8, P=64, N=128, G=1, chunk=128, dtype="bf16", seed=27)
+    inp = generate(w)
+    dev = to_dev(inp)
+    shape = ssd.shape_of(dev["x"], dev["a"], dev["Bm"], w.chunk)
+    if not ssd.path_supported(shape, ssd.PATH_FUSED):
+        pytest.skip("fused path not built for this shape")
+    ws = ssd.alloc_workspace(shape)
+    ssd.forward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], dev["D"], w.chunk, workspace=ws,
+                path=ssd.PATH_FUSED, flags=ssd.FLAG_TEST_STALL)
+    assert ssd.device_status(ws) == ssd.SSD_ERR_TIMEOUT
+    y, fin = ssd.forward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], dev["D"], w.chunk, workspace=ws,
+                         path=ssd.PATH_FUSED)
+    assert ssd.device_status(ws) == ssd.SSD_OK
+    ey, ef = parity_on_chains(inp, y, fin, _all_chains(w))
+    assert ey <= TOL_BF16 and ef <= TOL_BF16
