@@ -296,6 +296,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--B", type=int, default=None, help="override the batch (profiling small cases)")
+    ap.add_argument("--T", type=int, default=None, help="override the sequence length")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -314,6 +316,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
 
     w = WORKLOADS[args.workload]
+    if args.B or args.T:
+        w = w.scaled(B=args.B or w.B, T=args.T or w.T, name=w.name + f"_B{args.B or w.B}_T{args.T or w.T}")
     inp = generate(w, seed=w.seed + 1000 * rank)  # each rank: its own batch
     dev = {k: v.to(device) for k, v in inp.items()}
     shape = ssd.shape_of(dev["x"], dev["a"], dev["Bm"], w.chunk)

@@ -42,6 +42,18 @@ __device__ __forceinline__ void set_abort(int* abort_flag, int* status) {
     if (status) atomicExch(status, kDevTimeout);
 }
 
+// barrier over the 128 weighting/drain threads that ORs a predicate across them
+__device__ __forceinline__ bool group_sync_or(bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.or.pred po, 1, 128, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred)
+        : "memory");
+    return r != 0;
+}
+
 template <int Q>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
@@ -171,17 +183,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     make_float4(v1[4 * j], v1[4 * j + 1], v1[4 * j + 2], v1[4 * j + 3]);
             return true;
         };
-        for (int i = 0; ok && i < hpb; ++i) {
+        for (int i = 0; i < hpb; ++i) {
             const int h = h0 + i;
             const int st = i & 1;
             // decay weights of this head's chunk
             const float* cumk = cum + (((size_t)b * H + h) * nc + k) * Q;
             for (int s = ct; s < Q; s += 128) sCum[s] = cumk[s];
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            const float cend = sCum[Q - 1];
             ok = tc::mbar_wait(&bars->x_full[st], (i >> 1) & 1, abort_v) &&
                  (i == 0 || tc::mbar_wait(&bars->xw_empty, (i - 1) & 1, abort_v));
-            if (!ok) break;
+            if (!ok) set_abort(sAbort, status);
+            if (group_sync_or(!ok || *abort_v != 0)) { ok = false; break; }
+            const float cend = sCum[Q - 1];
             const uint8_t* xs = sX + st * kTileBytes;
             for (int c = ct; c < Q * 8; c += 128) {
                 const int s = c >> 3;  // token row; the 8 chunks of a row share w
@@ -201,8 +213,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc::mbar_arrive(&bars->xw_full);
                 tc::mbar_arrive(&bars->x_empty[st]);
             }
-            asm volatile("bar.sync 1, 128;" ::: "memory");  // sCum reuse
-            if (i > 0) ok = drain(i - 1);
+            if (i > 0) {
+                ok = drain(i - 1);
+                if (!ok) set_abort(sAbort, status);
+            }
+            // sCum is rewritten next head; the drain result decides for everyone
+            if (group_sync_or(!ok || *abort_v != 0)) { ok = false; break; }
         }
         if (ok && hpb > 0) ok = drain(hpb - 1);
         if (!ok) set_abort(sAbort, status);

@@ -95,6 +95,18 @@ __device__ __forceinline__ uint32_t col_y(int buf) { return 192 + 192 * buf; }
 __device__ __forceinline__ uint32_t col_v(int buf) { return 256 + 192 * buf; }
 
 __device__ __forceinline__ void compute_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+// barrier over the 256 compute threads that also ORs a predicate across them,
+// so every thread takes the same branch afterwards
+__device__ __forceinline__ bool compute_sync_or(bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.or.pred po, 1, 256, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred)
+        : "memory");
+    return r != 0;
+}
 
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
     unsigned v;
@@ -316,11 +328,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
         uint32_t hc = 0, xc = 0, itc = 0;
 
+        // Every abort decision of the compute warps goes through this reduction:
+        // a thread whose wait failed, or that sees another role's abort flag,
+        // makes all 256 compute threads leave together.
         auto sync_ok = [&](bool ok) -> bool {
             if (!ok) fail();
-            compute_sync();
+            const bool any = compute_sync_or(!ok || *abort_v != 0);
             __syncwarp();
-            return *abort_v == 0;
+            return !any;
         };
 
         for (int it = blockIdx.x; it < p.n_items; it += gridDim.x, ++itc) {
@@ -398,7 +413,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 return true;
             };
-            bool ok = true;
+            bool ok = true;      // this thread's wait results
+            bool alive = true;   // uniform across the compute threads
             for (int i = 0; i < p.hpb; ++i, ++hc, ++xc) {
                 const int h = w.h0 + i;
                 const int buf = hc & 1;
@@ -416,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (MODE == kFused) {
                     ok = tc::mbar_wait(&bars->x_full[st], (xc / kStages) & 1, abort_v) &&
                          (hc == 0 || tc::mbar_wait(&bars->xw_empty, (hc - 1) & 1, abort_v));
-                    if (!sync_ok(ok)) break;
+                    if (!sync_ok(ok)) { alive = false; break; }
                     const uint8_t* xs = sX + st * kTile;
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
@@ -438,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // ---- T3: P = S o L  -> bf16, K-major in sP
                 ok = (i > 0 || tc::mbar_wait(&bars->s_full, itc & 1, abort_v)) &&
                      (hc == 0 || tc::mbar_wait(&bars->p_empty, (hc - 1) & 1, abort_v));
-                if (!sync_ok(ok)) break;
+                if (!sync_ok(ok)) { alive = false; break; }
                 tc::tc_fence_after();
                 {
                     const float ct_cum = cum[row];
@@ -485,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (i == p.hpb - 1) tc::mbar_arrive(&bars->s_empty);
                 }
                 // ---- T5 of the previous head
-                if (i > 0 && !epilogue(i - 1, hc - 1, xc - 1)) { ok = false; break; }
+                if (i > 0 && !epilogue(i - 1, hc - 1, xc - 1)) { alive = false; break; }
                 // ---- T4: incoming state (and, fused, the chain hand-off)
                 {
                     const int chain = w.b * p.H + h;
@@ -508,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 __nanosleep(64);
                             }
                         }
-                        if (!sync_ok(ok)) break;
+                        if (!sync_ok(ok)) { alive = false; break; }
                         tc::tc_fence_after();
                         float zv[32];
                         tc::tmem_ld32(lane_base + col_z(buf) + 32 * cg, zv);
@@ -549,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (publish && ct == 0) st_release_u32(p.flags + chain, (unsigned)(w.j + 1));
                     } else {
                         ok = (hc == 0 || tc::mbar_wait(&bars->h_empty, (hc - 1) & 1, abort_v));
-                        if (!sync_ok(ok)) break;
+                        if (!sync_ok(ok)) { alive = false; break; }
                         const float4* src = reinterpret_cast<const float4*>(
                             p.hin + ((((size_t)w.b * p.H + h) * p.nblk + w.j) * kN + row) * kP + 32 * cg);
 #pragma unroll
@@ -574,7 +590,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (lane == 0) tc::mbar_arrive(&bars->h_full);
                 }
             }
-            if (!ok) break;
+            if (!alive) break;
             // ---- T5 of the slice's last head
             if (!epilogue(p.hpb - 1, hc - 1, xc - 1)) break;
         }

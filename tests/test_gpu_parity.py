@@ -170,7 +170,8 @@ def test_chunk_size_invariance():
     ref = outs[0][0].float().cpu().numpy()
     for y, fin in outs[1:]:
         assert rel_err(y.float().cpu().numpy(), ref) <= TOL_BF16
-        assert rel_err(fin.cpu().numpy(), outs[0][1].cpu().numpy()) <= 1e-3
+        # the tensor-core paths round the decay-weighted x to bf16 for the state
+        assert rel_err(fin.cpu().numpy(), outs[0][1].cpu().numpy()) <= TOL_BF16
 
 
 def test_diag_broadcast_equals_scalar():
