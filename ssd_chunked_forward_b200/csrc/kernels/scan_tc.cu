@@ -70,6 +70,7 @@ struct ScanParams {
     unsigned* flags;   // fused: [B*H] blocks published per chain
     float* fin;        // fused: final state [B,H,N,P] or null
     int* status;       // device status word or null
+    __nv_bfloat16* y;  // output [B,T,H,P]
     int T, H, G, nblk, hpb, nslices, n_items;
     int test_stall;
 };
@@ -81,8 +82,8 @@ constexpr uint32_t OFF_X = OFF_C + 2 * kTile;
 constexpr uint32_t OFF_XW = OFF_X + kStages * kTile;
 constexpr uint32_t OFF_P = OFF_XW + kTile;
 constexpr uint32_t OFF_H = OFF_P + 2 * kTile;
-constexpr uint32_t OFF_Y = OFF_H + kTile;
-constexpr uint32_t OFF_CUM = OFF_Y + 2 * kTile;
+constexpr uint32_t OFF_HIN = OFF_H + kTile;                 // fp32 [128][64], 32 KB
+constexpr uint32_t OFF_CUM = OFF_HIN + 2 * kTile;
 constexpr uint32_t OFF_VEC = OFF_CUM + kHpbMax * kBlk * 4;
 constexpr uint32_t OFF_BAR = OFF_VEC + 4 * kBlk * 4;
 constexpr uint32_t OFF_MISC = OFF_BAR + ((sizeof(Bars) + 15) / 16) * 16;
@@ -113,9 +114,22 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
+__device__ __forceinline__ unsigned ld_relaxed_u32(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 __device__ __forceinline__ void st_release_u32(unsigned* p, unsigned v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+
+__device__ __forceinline__ void cp_async16(void* sdst, const void* gsrc) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tc::smem_u32(sdst)), "l"(gsrc)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 struct Item {
     int b, j, h0, g;
@@ -137,8 +151,7 @@ __device__ __forceinline__ Item decode_item(int it, const ScanParams& p, int B) 
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
-                   const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y,
-                   const ScanParams p, int B) {
+                   const __grid_constant__ CUtensorMap tm_c, const ScanParams p, int B) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -148,13 +161,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* sXw = sm + OFF_XW;
     uint8_t* sP = sm + OFF_P;
     uint8_t* sH = sm + OFF_H;
-    uint8_t* sY = sm + OFF_Y;
+    uint8_t* sHin = sm + OFF_HIN;
     float* sCum = reinterpret_cast<float*>(sm + OFF_CUM);  // [hpb][128]
     float* sW = reinterpret_cast<float*>(sm + OFF_VEC);    // [128]
     float* sColf = sW + kBlk;                              // [3][128]
     Bars* bars = reinterpret_cast<Bars*>(sm + OFF_BAR);
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
     int* sAbort = reinterpret_cast<int*>(sm + OFF_MISC + 4);
+    volatile int* sReady = reinterpret_cast<volatile int*>(sm + OFF_MISC + 8);
     volatile int* abort_v = sAbort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -204,7 +218,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::prefetch_tmap(&tm_x);
             tc::prefetch_tmap(&tm_b);
             tc::prefetch_tmap(&tm_c);
-            tc::prefetch_tmap(&tm_y);
             uint32_t xc = 0, itc = 0;
             bool ok = true;
             for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x, ++itc) {
@@ -293,6 +306,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc::mma_commit(&bars->z_full[buf]);
                         tc::mma_commit(&bars->xw_empty);
                     }
+                    // V = C Hin of the previous head (its state was handed in before
+                    // this head's weighted x, so the wait is already satisfied)
+                    if (i > 0 && !issue_v(hc - 1)) { ok = false; break; }
                     // Y = P X: M = t, N = p, K = s (P K-major, X MN-major)
                     ok = tc::mbar_wait(&bars->p_full, hc & 1, abort_v) &&
                          tc::mbar_wait(&bars->x_full[st], (xc / kStages) & 1, abort_v);
@@ -307,8 +323,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc::mma_commit(&bars->y_full[buf]);
                     tc::mma_commit(&bars->p_empty);
                     tc::mma_commit(&bars->x_empty[st]);
-                    // V = C Hin of the previous head (its state is ready by now)
-                    if (i > 0 && !issue_v(hc - 1)) { ok = false; break; }
                 }
                 if (!ok) break;
                 if (!issue_v(hc - 1)) { ok = false; break; }
@@ -327,6 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row = quad * 32 + lane; // TMEM lane = tile row
         const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
         uint32_t hc = 0, xc = 0, itc = 0;
+        bool alive = true;  // uniform across the compute threads
 
         // Every abort decision of the compute warps goes through this reduction:
         // a thread whose wait failed, or that sees another role's abort flag,
@@ -337,22 +352,35 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             return !any;
         };
+        // per-item decay inputs (a or cum, hpb values per token row), loaded
+        // one item ahead into registers by the threads of column group 0
+        float anext[kHpbMax];
+        auto load_decays = [&](int it) {
+            if (cg != 0 || it >= p.n_items) return;
+            const Item w = decode_item(it, p, B);
+            if (MODE == kFused) {
+                const float* arow = p.a + (size_t)(w.b * p.T + w.j * kBlk + ct) * p.H + w.h0;
+#pragma unroll
+                for (int i = 0; i < kHpbMax; ++i) anext[i] = i < p.hpb ? __ldg(arow + i) : 0.f;
+            } else {
+#pragma unroll
+                for (int i = 0; i < kHpbMax; ++i)
+                    anext[i] = i < p.hpb ? __ldg(p.cum + (((size_t)w.b * p.H + w.h0 + i) * p.nblk + w.j) * kBlk + ct) : 0.f;
+            }
+        };
+        load_decays(blockIdx.x);
 
-        for (int it = blockIdx.x; it < p.n_items; it += gridDim.x, ++itc) {
+        for (int it = blockIdx.x; alive && it < p.n_items; it += gridDim.x, ++itc) {
             const Item w = decode_item(it, p, B);
             const int tok0 = w.b * p.T + w.j * kBlk;
             const bool last_blk = (w.j == p.nblk - 1);
             // ---- per-block cumulative log-decay of every head of the slice
             if (cg == 0) {
-                if (MODE == kFused) {
-                    const float* arow = p.a + (size_t)(tok0 + ct) * p.H + w.h0;
-                    for (int i = 0; i < p.hpb; ++i) sCum[i * kBlk + ct] = arow[i];
-                } else {
-                    for (int i = 0; i < p.hpb; ++i)
-                        sCum[i * kBlk + ct] =
-                            p.cum[(((size_t)w.b * p.H + w.h0 + i) * p.nblk + w.j) * kBlk + ct];
-                }
+#pragma unroll
+                for (int i = 0; i < kHpbMax; ++i)
+                    if (i < p.hpb) sCum[i * kBlk + ct] = anext[i];
             }
+            load_decays(it + gridDim.x);
             compute_sync();
             if (MODE == kFused) {
                 const int cw = ct >> 5;  // compute warp 0..7 scans head cw
@@ -364,29 +392,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 compute_sync();
             }
-            // ---- T5: y = Y + exp(cum) V + D x -> bf16 -> TMA store
+
+            // ---- T5: y = Y + exp(cum) V + D x -> bf16, straight to global
             auto epilogue = [&](int hi, uint32_t hcount, uint32_t xcount) -> bool {
                 const int eb = hcount & 1;
                 const uint32_t est = xcount % kStages;
-                bool eok = tc::mbar_wait(&bars->x_full[est], (xcount / kStages) & 1, abort_v) &&
-                           tc::mbar_wait(&bars->y_full[eb], (hcount >> 1) & 1, abort_v) &&
-                           tc::mbar_wait(&bars->v_full[eb], (hcount >> 1) & 1, abort_v);
-                if (ct == 0) tc::bulk_wait_read<1>();  // sY[eb] free again
+                const bool eok = tc::mbar_wait(&bars->x_full[est], (xcount / kStages) & 1, abort_v) &&
+                                 tc::mbar_wait(&bars->y_full[eb], (hcount >> 1) & 1, abort_v) &&
+                                 tc::mbar_wait(&bars->v_full[eb], (hcount >> 1) & 1, abort_v);
                 if (!sync_ok(eok)) return false;
                 tc::tc_fence_after();
                 float yv[32], vv[32];
                 tc::tmem_ld32(lane_base + col_y(eb) + 32 * cg, yv);
                 tc::tmem_ld32(lane_base + col_v(eb) + 32 * cg, vv);
                 tc::tmem_ld_wait();
-                const float* ecum_src = sCum + hi * kBlk;
-                const float ecum = __expf(ecum_src[row]);
-                const float dv = p.D ? p.D[w.h0 + hi] : 0.f;
+                const float ecum = __expf(sCum[hi * kBlk + row]);
+                const float dv = p.D ? __ldg(p.D + w.h0 + hi) : 0.f;
                 const uint8_t* xs = sX + est * kTile;
-                uint8_t* ys = sY + eb * kTile;
+                uint4 out[4];
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4) {
-                    const uint32_t off = tc::sw128_offset(row, 4 * cg + c4);
-                    uint4 xv = *reinterpret_cast<const uint4*>(xs + off);
+                    const uint4 xv = *reinterpret_cast<const uint4*>(xs + tc::sw128_offset(row, 4 * cg + c4));
                     const uint32_t* xu = reinterpret_cast<const uint32_t*>(&xv);
                     uint32_t o[4];
 #pragma unroll
@@ -397,30 +423,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float y1 = fmaf(ecum, vv[k0 + 1], yv[k0 + 1]) + dv * xf.y;
                         o[e] = tc::pack_bf16x2(y0, y1);
                     }
-                    *reinterpret_cast<uint4*>(ys + off) = make_uint4(o[0], o[1], o[2], o[3]);
+                    out[c4] = make_uint4(o[0], o[1], o[2], o[3]);
                 }
-                tc::fence_proxy_async_smem();
                 tc::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
                     tc::mbar_arrive(&bars->t_empty[eb]);
                     tc::mbar_arrive(&bars->x_empty[est]);
                 }
-                compute_sync();
-                if (ct == 0) {
-                    tc::tma_store_3d(&tm_y, ys, 0, w.h0 + hi, tok0);
-                    tc::bulk_commit();
-                }
+                // this thread's 32 outputs are 64 contiguous bytes of row t
+                uint4* yd = reinterpret_cast<uint4*>(
+                    p.y + ((size_t)(tok0 + row) * p.H + w.h0 + hi) * kP + 32 * cg);
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) yd[c4] = out[c4];
                 return true;
             };
-            bool ok = true;      // this thread's wait results
-            bool alive = true;   // uniform across the compute threads
+
+            bool ok = true;  // this thread's wait results
             for (int i = 0; i < p.hpb; ++i, ++hc, ++xc) {
                 const int h = w.h0 + i;
+                const int chain = w.b * p.H + h;
                 const int buf = hc & 1;
                 const uint32_t st = xc % kStages;
                 const float* cum = sCum + i * kBlk;
-                // ---- T1: decay vectors of this head
+                // ---- T1: decay vectors of this head; the hand-off flag is read
+                // now and used after T3, so its latency overlaps T2/T3
+                unsigned flagv = 0;
+                if (MODE == kFused && ct == 0 && w.j > 0) flagv = ld_relaxed_u32(p.flags + chain);
                 if (cg == 0) {
                     const float c = cum[ct];
                     sW[ct] = __expf(cum[kBlk - 1] - c);
@@ -454,7 +483,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // ---- T3: P = S o L  -> bf16, K-major in sP
                 ok = (i > 0 || tc::mbar_wait(&bars->s_full, itc & 1, abort_v)) &&
                      (hc == 0 || tc::mbar_wait(&bars->p_empty, (hc - 1) & 1, abort_v));
+                if (MODE == kFused && ct == 0) {
+                    const bool rdy = w.j == 0 || flagv >= (unsigned)w.j;
+                    if (rdy) fence_acq_rel_gpu();  // the relaxed read above becomes an acquire
+                    *sReady = rdy ? 1 : 0;
+                }
                 if (!sync_ok(ok)) { alive = false; break; }
+                // incoming state into shared memory now (async copies), used in T4
+                const bool ready = MODE == kScan || *sReady != 0;
+                const size_t slot = (size_t)kN * kP;
+                const float* hsrc = MODE == kFused
+                    ? p.ring + ((size_t)chain * 2 + ((w.j - 1) & 1)) * slot
+                    : p.hin + (((size_t)w.b * p.H + h) * p.nblk + w.j) * slot;
+                uint8_t* hdst = sHin + (size_t)row * 256 + cg * 128;
+                const bool need_h = MODE == kScan || w.j > 0;
+                if (need_h && ready) {
+                    const uint8_t* g = reinterpret_cast<const uint8_t*>(hsrc + (size_t)row * kP + 32 * cg);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) cp_async16(hdst + ((q ^ (row & 7)) << 4), g + q * 16);
+                    cp_async_commit();
+                }
                 tc::tc_fence_after();
                 {
                     const float ct_cum = cum[row];
@@ -504,75 +552,68 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (i > 0 && !epilogue(i - 1, hc - 1, xc - 1)) { alive = false; break; }
                 // ---- T4: incoming state (and, fused, the chain hand-off)
                 {
-                    const int chain = w.b * p.H + h;
-                    float hin[32];
-                    if (MODE == kFused) {
-                        ok = tc::mbar_wait(&bars->z_full[buf], (hc >> 1) & 1, abort_v) &&
-                             (hc == 0 || tc::mbar_wait(&bars->h_empty, (hc - 1) & 1, abort_v));
-                        if (ok && w.j > 0 && ct == 0) {
-                            // bounded wait for the previous block of this chain
-                            const unsigned* f = p.flags + chain;
-                            const uint64_t t0 = tc::globaltimer_ns();
-                            for (uint32_t spin = 0; ld_acquire_u32(f) < (unsigned)w.j; ++spin) {
-                                if ((spin & 15) == 15) {
-                                    if (*abort_v || (p.status && *(volatile int*)p.status) ||
-                                        tc::globaltimer_ns() - t0 > 2000000000ull) {
-                                        ok = false;
-                                        break;
-                                    }
+                    ok = (MODE == kScan || tc::mbar_wait(&bars->z_full[buf], (hc >> 1) & 1, abort_v)) &&
+                         (hc == 0 || tc::mbar_wait(&bars->h_empty, (hc - 1) & 1, abort_v));
+                    if (MODE == kFused && !ready && ct == 0 && ok) {
+                        // slow path: bounded wait for the previous block of this chain
+                        const unsigned* f = p.flags + chain;
+                        const uint64_t t0 = tc::globaltimer_ns();
+                        for (uint32_t spin = 0; ld_acquire_u32(f) < (unsigned)w.j; ++spin) {
+                            if ((spin & 15) == 15) {
+                                if (*abort_v || (p.status && *(volatile int*)p.status) ||
+                                    tc::globaltimer_ns() - t0 > 2000000000ull) {
+                                    ok = false;
+                                    break;
                                 }
-                                __nanosleep(64);
                             }
+                            __nanosleep(64);
                         }
-                        if (!sync_ok(ok)) { alive = false; break; }
+                    }
+                    if (!sync_ok(ok)) { alive = false; break; }
+                    float hin[32];
+                    if (need_h) {
+                        if (!ready) {
+                            const uint8_t* g = reinterpret_cast<const uint8_t*>(hsrc + (size_t)row * kP + 32 * cg);
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) cp_async16(hdst + ((q ^ (row & 7)) << 4), g + q * 16);
+                            cp_async_commit();
+                        }
+                        cp_async_wait_all();
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const float4 v = *reinterpret_cast<const float4*>(hdst + ((q ^ (row & 7)) << 4));
+                            hin[4 * q] = v.x; hin[4 * q + 1] = v.y; hin[4 * q + 2] = v.z; hin[4 * q + 3] = v.w;
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) hin[e] = 0.f;
+                    }
+                    if (MODE == kFused) {
                         tc::tc_fence_after();
                         float zv[32];
                         tc::tmem_ld32(lane_base + col_z(buf) + 32 * cg, zv);
                         tc::tmem_ld_wait();
-                        const size_t slot = (size_t)kN * kP;
-                        float* ring = p.ring + (size_t)chain * 2 * slot;
-                        const size_t roff = (size_t)row * kP + 32 * cg;
-                        if (w.j > 0) {
-                            const float4* src = reinterpret_cast<const float4*>(ring + ((w.j - 1) & 1) * slot + roff);
-#pragma unroll
-                            for (int q = 0; q < 8; ++q) {
-                                const float4 v = __ldcg(src + q);
-                                hin[4 * q] = v.x; hin[4 * q + 1] = v.y; hin[4 * q + 2] = v.z; hin[4 * q + 3] = v.w;
-                            }
-                        } else {
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) hin[e] = 0.f;
-                        }
                         const float eL = __expf(cum[kBlk - 1]);
-                        float hn[32];
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) hn[e] = fmaf(eL, hin[e], zv[e]);
+                        for (int e = 0; e < 32; ++e) zv[e] = fmaf(eL, hin[e], zv[e]);  // h_j
                         const bool publish = !(p.test_stall && chain == 0 && w.j == 0);
+                        const size_t roff = (size_t)row * kP + 32 * cg;
                         if (publish) {
-                            float4* dst = reinterpret_cast<float4*>(ring + (w.j & 1) * slot + roff);
+                            float4* dst = reinterpret_cast<float4*>(p.ring + ((size_t)chain * 2 + (w.j & 1)) * slot + roff);
 #pragma unroll
                             for (int q = 0; q < 8; ++q)
-                                __stcg(dst + q, make_float4(hn[4 * q], hn[4 * q + 1], hn[4 * q + 2], hn[4 * q + 3]));
-                            __threadfence();
+                                __stcg(dst + q, make_float4(zv[4 * q], zv[4 * q + 1], zv[4 * q + 2], zv[4 * q + 3]));
                         }
                         if (last_blk && p.fin) {
-                            float4* fd = reinterpret_cast<float4*>(p.fin + (size_t)chain * kN * kP + roff);
+                            float4* fd = reinterpret_cast<float4*>(p.fin + (size_t)chain * slot + roff);
 #pragma unroll
                             for (int q = 0; q < 8; ++q)
-                                fd[q] = make_float4(hn[4 * q], hn[4 * q + 1], hn[4 * q + 2], hn[4 * q + 3]);
+                                fd[q] = make_float4(zv[4 * q], zv[4 * q + 1], zv[4 * q + 2], zv[4 * q + 3]);
                         }
+                        // every thread's stores precede the barrier; one release at
+                        // gpu scope then publishes them all
                         compute_sync();
                         if (publish && ct == 0) st_release_u32(p.flags + chain, (unsigned)(w.j + 1));
-                    } else {
-                        ok = (hc == 0 || tc::mbar_wait(&bars->h_empty, (hc - 1) & 1, abort_v));
-                        if (!sync_ok(ok)) { alive = false; break; }
-                        const float4* src = reinterpret_cast<const float4*>(
-                            p.hin + ((((size_t)w.b * p.H + h) * p.nblk + w.j) * kN + row) * kP + 32 * cg);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            const float4 v = __ldg(src + q);
-                            hin[4 * q] = v.x; hin[4 * q + 1] = v.y; hin[4 * q + 2] = v.z; hin[4 * q + 3] = v.w;
-                        }
                     }
                     // Hin as the bf16 B operand of V = C Hin: rows n, 64 p per row (MN-major)
 #pragma unroll
@@ -592,9 +633,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!alive) break;
             // ---- T5 of the slice's last head
-            if (!epilogue(p.hpb - 1, hc - 1, xc - 1)) break;
+            if (!epilogue(p.hpb - 1, hc - 1, xc - 1)) { alive = false; break; }
         }
-        if (ct == 0) tc::bulk_wait<0>();
     }
     tc::tc_fence_before();
     __syncthreads();
@@ -605,11 +645,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+int num_sms();
+
+// Heads per work item: the largest divisor of H/G (at most kHpbMax) that still
+// leaves at least one item per SM for every block index, so that a block's
+// predecessor in the same chain was scheduled a full round earlier; when no
+// divisor does (few chains), the largest one, to share the scores most.
 int heads_per_item(const Dims& d) {
     const int HG = d.H / d.G;
-    for (int c = kHpbMax; c >= 1; --c)
-        if (HG % c == 0) return c;
-    return 1;
+    const int sms = num_sms();
+    int best = 0, largest = 1;
+    for (int c = 1; c <= kHpbMax; ++c) {
+        if (HG % c) continue;
+        largest = c;
+        if ((long long)d.B * d.G * (HG / c) >= sms) best = c;
+    }
+    return best > 0 ? best : largest;
 }
 
 int num_sms() {
@@ -622,12 +673,12 @@ int num_sms() {
 template <int MODE>
 cudaError_t launch(const Dims& d, const void* x, const void* Bm, const void* Cm, void* y,
                    ScanParams p, cudaStream_t st) {
-    CUtensorMap tx, tb, tcm, ty;
+    CUtensorMap tx, tb, tcm;
     cudaError_t e = make_tmap_bf16_3d(&tx, x, d.P, d.H, (uint64_t)d.B * d.T, kBlk);
     if (e == cudaSuccess) e = make_tmap_bf16_3d(&tb, Bm, d.N, d.G, (uint64_t)d.B * d.T, kBlk);
     if (e == cudaSuccess) e = make_tmap_bf16_3d(&tcm, Cm, d.N, d.G, (uint64_t)d.B * d.T, kBlk);
-    if (e == cudaSuccess) e = make_tmap_bf16_3d(&ty, y, d.P, d.H, (uint64_t)d.B * d.T, kBlk);
     if (e != cudaSuccess) return e;
+    p.y = reinterpret_cast<__nv_bfloat16*>(y);
     p.T = d.T; p.H = d.H; p.G = d.G;
     p.nblk = d.T / kBlk;
     p.hpb = heads_per_item(d);
@@ -639,7 +690,7 @@ cudaError_t launch(const Dims& d, const void* x, const void* Bm, const void* Cm,
     e = cudaFuncSetAttribute(scan_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemBytes);
     if (e != cudaSuccess) return e;
-    scan_tc_kernel<MODE><<<grid, kThreads, kSmemBytes, st>>>(tx, tb, tcm, ty, p, d.B);
+    scan_tc_kernel<MODE><<<grid, kThreads, kSmemBytes, st>>>(tx, tb, tcm, p, d.B);
     return cudaGetLastError();
 }
 
