@@ -7,11 +7,12 @@
 // t, s in [0, 128), head h, and cum the in-block inclusive prefix sum of the
 // log-decays a:
 //   S   = C B^T                         (scores, shared by the slice's heads)
-//   P   = S o L,  L[t,s] = exp(cum_t - cum_s) for s <= t, else 0
+//   P   = S o L + D I,  L[t,s] = exp(cum_t - cum_s) for s <= t, else 0
 //   Y   = P X                           (quadratic masked form, llms.blog
-//                                        "The Chunk-Wise SSD Algorithm", item 2)
+//                                        "The Chunk-Wise SSD Algorithm", item 2;
+//                                        the skip term D x_t rides on the diagonal)
 //   V   = C Hin                         (incoming state, item 5)
-//   y_t = Y_t + exp(cum_t) V_t + D x_t
+//   y_t = Y_t + exp(cum_t) V_t
 // The mask L is applied in registers between the TMEM scores and the bf16
 // operand in shared memory; it never reaches HBM.
 //
@@ -20,9 +21,11 @@
 //   h_j = exp(cum_127) h_{j-1} + Z_j                         (item 4)
 // across blocks: each (b, h) chain hands its fp32 state from block j-1 to
 // block j through a two-slot ring in global memory (it stays in L2) and a
-// per-chain counter, with a bounded wait on the consumer side.  Work items are
-// ordered block-major and scheduled round-robin over persistent CTAs, so the
-// block a CTA waits for belongs to a smaller item index and can always finish.
+// per-chain counter.  Two dedicated threads move the states with TMA and do
+// the acquire (bounded wait on the counter) and the release, so the compute
+// warps never wait on a fence.  Work items are ordered block-major and
+// scheduled round-robin over persistent CTAs, so the block a CTA waits for
+// belongs to a smaller item index and can always finish.
 //
 // A chunk of 256 tokens is two such blocks: the strictly-lower 128x128 block
 // of its quadratic form goes through the exact factorisation
@@ -30,11 +33,12 @@
 // at the block boundary ("State Space Duality", "Two algorithms for one
 // operator": off-diagonal blocks are low-rank).
 //
-// Warp roles (320 threads): 0 TMA producer; 1 MMA issuer and TMEM owner;
+// Warp roles (384 threads): 0 TMA producer; 1 MMA issuer and TMEM owner;
 // 2-9 compute: two groups of four warps, each group covering all 128 TMEM
 // lanes, group g owning columns [32g, 32g+32) of P-wide tiles and
-// [64g, 64g+64) of the scores.  TMEM (512 columns): scores 0-127, then two
-// buffers of {Z, Y, V} x 64 columns, alternating per head.
+// [64g, 64g+64) of the scores; 10 state loader; 11 state publisher (fused).
+// TMEM (512 columns): scores 0-127, then two buffers of {Z, Y, V} x 64
+// columns, alternating per head.
 #include "../common.cuh"
 #include "../kernels.h"
 #include "../tc_common.cuh"
@@ -46,10 +50,11 @@ namespace {
 constexpr int kBlk = 128;
 constexpr int kN = 128;
 constexpr int kP = 64;
-constexpr int kStages = 3;
+constexpr int kStages = 2;
 constexpr int kHpbMax = 8;
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
 constexpr uint32_t kTile = kBlk * 128;  // 128 rows x 128 bytes
+constexpr uint32_t kStateBytes = kN * kP * 4;
 
 enum { kScan = 0, kFused = 1 };
 
@@ -57,6 +62,7 @@ struct __align__(8) Bars {
     uint64_t bc_full, bc_empty, s_full, s_empty;
     uint64_t x_full[kStages], x_empty[kStages];
     uint64_t xw_full, xw_empty, p_full, p_empty, h_full, h_empty;
+    uint64_t hin_full, hin_free, hout_full;
     uint64_t y_full[2], v_full[2], z_full[2], t_empty[2];
     uint64_t done;
 };
@@ -64,13 +70,10 @@ struct __align__(8) Bars {
 struct ScanParams {
     const float* a;    // fused: log-decays [B,T,H]
     const float* cum;  // scan: in-block cumsum [B,H,nblk,128]
-    const float* hin;  // scan: incoming states [B,H,nblk,N,P]
     const float* D;    // [H] or null
-    float* ring;       // fused: [B*H][2][N*P]
     unsigned* flags;   // fused: [B*H] blocks published per chain
     float* fin;        // fused: final state [B,H,N,P] or null
     int* status;       // device status word or null
-    __nv_bfloat16* y;  // output [B,T,H,P]
     int T, H, G, nblk, hpb, nslices, n_items;
     int test_stall;
 };
@@ -81,9 +84,10 @@ constexpr uint32_t OFF_C = OFF_B + 2 * kTile;
 constexpr uint32_t OFF_X = OFF_C + 2 * kTile;
 constexpr uint32_t OFF_XW = OFF_X + kStages * kTile;
 constexpr uint32_t OFF_P = OFF_XW + kTile;
-constexpr uint32_t OFF_H = OFF_P + 2 * kTile;
-constexpr uint32_t OFF_HIN = OFF_H + kTile;                 // fp32 [128][64], 32 KB
-constexpr uint32_t OFF_CUM = OFF_HIN + 2 * kTile;
+constexpr uint32_t OFF_H = OFF_P + 2 * kTile;      // bf16 Hin, MN-major operand
+constexpr uint32_t OFF_HIN = OFF_H + kTile;        // fp32 state, two swizzled 128x32 boxes
+constexpr uint32_t OFF_Y = OFF_HIN + 2 * kTile;    // bf16 y staging for the TMA store
+constexpr uint32_t OFF_CUM = OFF_Y + kTile;
 constexpr uint32_t OFF_VEC = OFF_CUM + kHpbMax * kBlk * 4;
 constexpr uint32_t OFF_BAR = OFF_VEC + 4 * kBlk * 4;
 constexpr uint32_t OFF_MISC = OFF_BAR + ((sizeof(Bars) + 15) / 16) * 16;
@@ -108,28 +112,14 @@ __device__ __forceinline__ bool compute_sync_or(bool pred) {
         : "memory");
     return r != 0;
 }
-
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
     unsigned v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
-__device__ __forceinline__ unsigned ld_relaxed_u32(const unsigned* p) {
-    unsigned v;
-    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 __device__ __forceinline__ void st_release_u32(unsigned* p, unsigned v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
-
-__device__ __forceinline__ void cp_async16(void* sdst, const void* gsrc) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tc::smem_u32(sdst)), "l"(gsrc)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 struct Item {
     int b, j, h0, g;
@@ -148,10 +138,17 @@ __device__ __forceinline__ Item decode_item(int it, const ScanParams& p, int B) 
     return r;
 }
 
+// fp32 state tile in shared memory: two boxes of 128 rows x 32 floats, each
+// row 128 bytes with 16-byte chunk q stored at q ^ (row & 7)
+__device__ __forceinline__ uint32_t state_off(int row, int half, int q) {
+    return half * kTile + row * 128 + ((q ^ (row & 7)) << 4);
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
-                   const __grid_constant__ CUtensorMap tm_c, const ScanParams p, int B) {
+                   const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y,
+                   const __grid_constant__ CUtensorMap tm_st, const ScanParams p, int B) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -162,13 +159,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* sP = sm + OFF_P;
     uint8_t* sH = sm + OFF_H;
     uint8_t* sHin = sm + OFF_HIN;
+    uint8_t* sY = sm + OFF_Y;
     float* sCum = reinterpret_cast<float*>(sm + OFF_CUM);  // [hpb][128]
     float* sW = reinterpret_cast<float*>(sm + OFF_VEC);    // [128]
     float* sColf = sW + kBlk;                              // [3][128]
     Bars* bars = reinterpret_cast<Bars*>(sm + OFF_BAR);
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
     int* sAbort = reinterpret_cast<int*>(sm + OFF_MISC + 4);
-    volatile int* sReady = reinterpret_cast<volatile int*>(sm + OFF_MISC + 8);
     volatile int* abort_v = sAbort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -180,7 +177,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mbar_init(&bars->s_empty, 8);
         for (int s = 0; s < kStages; ++s) {
             tc::mbar_init(&bars->x_full[s], 1);
-            tc::mbar_init(&bars->x_empty[s], 9);  // Y MMA commit + 8 compute warps
+            // Y MMA commit (+ the 8 compute warps that weight x, fused)
+            tc::mbar_init(&bars->x_empty[s], MODE == kFused ? 9 : 1);
         }
         tc::mbar_init(&bars->xw_full, 8);
         tc::mbar_init(&bars->xw_empty, 1);
@@ -188,6 +186,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mbar_init(&bars->p_empty, 1);
         tc::mbar_init(&bars->h_full, 8);
         tc::mbar_init(&bars->h_empty, 1);
+        tc::mbar_init(&bars->hin_full, 1);
+        tc::mbar_init(&bars->hin_free, MODE == kFused ? 1 : 8);
+        tc::mbar_init(&bars->hout_full, 8);
         for (int s = 0; s < 2; ++s) {
             tc::mbar_init(&bars->y_full[s], 1);
             tc::mbar_init(&bars->v_full[s], 1);
@@ -307,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc::mma_commit(&bars->xw_empty);
                     }
                     // V = C Hin of the previous head (its state was handed in before
-                    // this head's weighted x, so the wait is already satisfied)
+                    // this head's weighted x, so the wait is normally satisfied)
                     if (i > 0 && !issue_v(hc - 1)) { ok = false; break; }
                     // Y = P X: M = t, N = p, K = s (P K-major, X MN-major)
                     ok = tc::mbar_wait(&bars->p_full, hc & 1, abort_v) &&
@@ -332,6 +333,81 @@ __global__ void __launch_bounds__(kThreads, 1)
             // every MMA issued must be complete before TMEM is released
             tc::mma_commit(&bars->done);
             tc::mbar_wait(&bars->done, 0, nullptr, 200000000ull);
+        }
+    } else if (warp == 10) {
+        // ========================================== incoming-state loader ====
+        if (lane == 0) {
+            tc::prefetch_tmap(&tm_st);
+            uint32_t hc = 0;
+            bool ok = true;
+            for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x) {
+                const Item w = decode_item(it, p, B);
+                for (int i = 0; i < p.hpb; ++i, ++hc) {
+                    const int chain = w.b * p.H + w.h0 + i;
+                    if (hc > 0 && !tc::mbar_wait(&bars->hin_free, (hc - 1) & 1, abort_v)) { ok = false; break; }
+                    if (MODE == kFused) {
+                        if (w.j == 0) {
+                            tc::mbar_arrive(&bars->hin_full);  // zero state: nothing to load
+                            continue;
+                        }
+                        // bounded wait for the previous block of this chain
+                        const unsigned* f = p.flags + chain;
+                        const uint64_t t0 = tc::globaltimer_ns();
+                        for (uint32_t spin = 0; ld_acquire_u32(f) < (unsigned)w.j; ++spin) {
+                            if ((spin & 15) == 15) {
+                                if (*abort_v || (p.status && *(volatile int*)p.status) ||
+                                    tc::globaltimer_ns() - t0 > 2000000000ull) {
+                                    ok = false;
+                                    break;
+                                }
+                            }
+                            __nanosleep(32);
+                        }
+                        if (!ok) break;
+                        tc::fence_proxy_async_global();  // the acquire orders the TMA read
+                        const int r0 = (chain * 2 + ((w.j - 1) & 1)) * kN;
+                        tc::mbar_arrive_expect_tx(&bars->hin_full, kStateBytes);
+                        tc::tma_load_2d(sHin, &tm_st, &bars->hin_full, 0, r0);
+                        tc::tma_load_2d(sHin + kTile, &tm_st, &bars->hin_full, 32, r0);
+                    } else {
+                        const int r0 = (chain * p.nblk + w.j) * kN;
+                        tc::mbar_arrive_expect_tx(&bars->hin_full, kStateBytes);
+                        tc::tma_load_2d(sHin, &tm_st, &bars->hin_full, 0, r0);
+                        tc::tma_load_2d(sHin + kTile, &tm_st, &bars->hin_full, 32, r0);
+                    }
+                }
+            }
+            if (!ok) fail();
+            if (hc > 0) tc::mbar_wait(&bars->hin_full, (hc - 1) & 1, nullptr, 200000000ull);
+        }
+    } else if (warp == 11) {
+        // ============================================== state publisher ====
+        if (MODE == kFused && lane == 0) {
+            uint32_t hc = 0;
+            bool ok = true;
+            for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x) {
+                const Item w = decode_item(it, p, B);
+                for (int i = 0; i < p.hpb; ++i, ++hc) {
+                    const int chain = w.b * p.H + w.h0 + i;
+                    if (!tc::mbar_wait(&bars->hout_full, hc & 1, abort_v)) { ok = false; break; }
+                    const bool publish = !(p.test_stall && chain == 0 && w.j == 0);
+                    if (publish) {
+                        const int r0 = (chain * 2 + (w.j & 1)) * kN;
+                        tc::tma_store_2d(&tm_st, sHin, 0, r0);
+                        tc::tma_store_2d(&tm_st, sHin + kTile, 32, r0);
+                        tc::bulk_commit();
+                        tc::bulk_wait_read<0>();
+                    }
+                    tc::mbar_arrive(&bars->hin_free);
+                    if (publish) {
+                        tc::bulk_wait<0>();
+                        tc::fence_proxy_async_global();
+                        st_release_u32(p.flags + chain, (unsigned)(w.j + 1));
+                    }
+                }
+            }
+            if (!ok) fail();
+            tc::bulk_wait<0>();
         }
     } else {
         // ================================================ compute (8 warps) ====
@@ -393,13 +469,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 compute_sync();
             }
 
-            // ---- T5: y = Y + exp(cum) V + D x -> bf16, straight to global
-            auto epilogue = [&](int hi, uint32_t hcount, uint32_t xcount) -> bool {
+            // ---- T5: y = Y + exp(cum) V -> bf16 -> shared staging -> TMA store
+            auto epilogue = [&](int hi, uint32_t hcount) -> bool {
                 const int eb = hcount & 1;
-                const uint32_t est = xcount % kStages;
-                const bool eok = tc::mbar_wait(&bars->x_full[est], (xcount / kStages) & 1, abort_v) &&
-                                 tc::mbar_wait(&bars->y_full[eb], (hcount >> 1) & 1, abort_v) &&
+                const bool eok = tc::mbar_wait(&bars->y_full[eb], (hcount >> 1) & 1, abort_v) &&
                                  tc::mbar_wait(&bars->v_full[eb], (hcount >> 1) & 1, abort_v);
+                if (ct == 0) tc::bulk_wait_read<0>();  // previous y tile left sY
                 if (!sync_ok(eok)) return false;
                 tc::tc_fence_after();
                 float yv[32], vv[32];
@@ -407,35 +482,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc::tmem_ld32(lane_base + col_v(eb) + 32 * cg, vv);
                 tc::tmem_ld_wait();
                 const float ecum = __expf(sCum[hi * kBlk + row]);
-                const float dv = p.D ? __ldg(p.D + w.h0 + hi) : 0.f;
-                const uint8_t* xs = sX + est * kTile;
-                uint4 out[4];
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4) {
-                    const uint4 xv = *reinterpret_cast<const uint4*>(xs + tc::sw128_offset(row, 4 * cg + c4));
-                    const uint32_t* xu = reinterpret_cast<const uint32_t*>(&xv);
                     uint32_t o[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float2 xf = tc::unpack_bf16x2(xu[e]);
                         const int k0 = 8 * c4 + 2 * e;
-                        const float y0 = fmaf(ecum, vv[k0], yv[k0]) + dv * xf.x;
-                        const float y1 = fmaf(ecum, vv[k0 + 1], yv[k0 + 1]) + dv * xf.y;
-                        o[e] = tc::pack_bf16x2(y0, y1);
+                        o[e] = tc::pack_bf16x2(fmaf(ecum, vv[k0], yv[k0]), fmaf(ecum, vv[k0 + 1], yv[k0 + 1]));
                     }
-                    out[c4] = make_uint4(o[0], o[1], o[2], o[3]);
+                    *reinterpret_cast<uint4*>(sY + tc::sw128_offset(row, 4 * cg + c4)) =
+                        make_uint4(o[0], o[1], o[2], o[3]);
                 }
+                tc::fence_proxy_async_smem();
                 tc::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) {
-                    tc::mbar_arrive(&bars->t_empty[eb]);
-                    tc::mbar_arrive(&bars->x_empty[est]);
+                if (lane == 0) tc::mbar_arrive(&bars->t_empty[eb]);
+                compute_sync();
+                if (ct == 0) {
+                    tc::tma_store_3d(&tm_y, sY, 0, w.h0 + hi, tok0);
+                    tc::bulk_commit();
                 }
-                // this thread's 32 outputs are 64 contiguous bytes of row t
-                uint4* yd = reinterpret_cast<uint4*>(
-                    p.y + ((size_t)(tok0 + row) * p.H + w.h0 + hi) * kP + 32 * cg);
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) yd[c4] = out[c4];
                 return true;
             };
 
@@ -446,10 +512,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int buf = hc & 1;
                 const uint32_t st = xc % kStages;
                 const float* cum = sCum + i * kBlk;
-                // ---- T1: decay vectors of this head; the hand-off flag is read
-                // now and used after T3, so its latency overlaps T2/T3
-                unsigned flagv = 0;
-                if (MODE == kFused && ct == 0 && w.j > 0) flagv = ld_relaxed_u32(p.flags + chain);
+                // ---- T1: decay vectors of this head
                 if (cg == 0) {
                     const float c = cum[ct];
                     sW[ct] = __expf(cum[kBlk - 1] - c);
@@ -478,33 +541,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tc::fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0) tc::mbar_arrive(&bars->xw_full);
+                    if (lane == 0) {
+                        tc::mbar_arrive(&bars->xw_full);
+                        tc::mbar_arrive(&bars->x_empty[st]);
+                    }
                 }
-                // ---- T3: P = S o L  -> bf16, K-major in sP
+                // ---- T3: P = S o L + D I  -> bf16, K-major in sP
                 ok = (i > 0 || tc::mbar_wait(&bars->s_full, itc & 1, abort_v)) &&
                      (hc == 0 || tc::mbar_wait(&bars->p_empty, (hc - 1) & 1, abort_v));
-                if (MODE == kFused && ct == 0) {
-                    const bool rdy = w.j == 0 || flagv >= (unsigned)w.j;
-                    if (rdy) fence_acq_rel_gpu();  // the relaxed read above becomes an acquire
-                    *sReady = rdy ? 1 : 0;
-                }
                 if (!sync_ok(ok)) { alive = false; break; }
-                // incoming state into shared memory now (async copies), used in T4
-                const bool ready = MODE == kScan || *sReady != 0;
-                const size_t slot = (size_t)kN * kP;
-                const float* hsrc = MODE == kFused
-                    ? p.ring + ((size_t)chain * 2 + ((w.j - 1) & 1)) * slot
-                    : p.hin + (((size_t)w.b * p.H + h) * p.nblk + w.j) * slot;
-                uint8_t* hdst = sHin + (size_t)row * 256 + cg * 128;
-                const bool need_h = MODE == kScan || w.j > 0;
-                if (need_h && ready) {
-                    const uint8_t* g = reinterpret_cast<const uint8_t*>(hsrc + (size_t)row * kP + 32 * cg);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) cp_async16(hdst + ((q ^ (row & 7)) << 4), g + q * 16);
-                    cp_async_commit();
-                }
                 tc::tc_fence_after();
                 {
+                    const float dv = p.D ? __ldg(p.D + h) : 0.f;
                     const float ct_cum = cum[row];
                     const float rowf = quad > 0 ? __expf(ct_cum - cum[32 * quad - 1]) : 0.f;
                     const float* colf = sColf + (quad > 0 ? (quad - 1) * kBlk : 0);
@@ -527,7 +575,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                                 for (int e = 0; e < 32; ++e) {
                                     const int s = 32 * sb + e;
-                                    v[e] = (s <= row) ? v[e] * __expf(ct_cum - cum[s]) : 0.f;
+                                    v[e] = (s < row) ? v[e] * __expf(ct_cum - cum[s])
+                                                     : (s == row ? v[e] + dv : 0.f);
                                 }
                             }
 #pragma unroll
@@ -549,44 +598,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (i == p.hpb - 1) tc::mbar_arrive(&bars->s_empty);
                 }
                 // ---- T5 of the previous head
-                if (i > 0 && !epilogue(i - 1, hc - 1, xc - 1)) { alive = false; break; }
-                // ---- T4: incoming state (and, fused, the chain hand-off)
+                if (i > 0 && !epilogue(i - 1, hc - 1)) { alive = false; break; }
+                // ---- T4: incoming state (and, fused, the block's own state out)
                 {
                     ok = (MODE == kScan || tc::mbar_wait(&bars->z_full[buf], (hc >> 1) & 1, abort_v)) &&
-                         (hc == 0 || tc::mbar_wait(&bars->h_empty, (hc - 1) & 1, abort_v));
-                    if (MODE == kFused && !ready && ct == 0 && ok) {
-                        // slow path: bounded wait for the previous block of this chain
-                        const unsigned* f = p.flags + chain;
-                        const uint64_t t0 = tc::globaltimer_ns();
-                        for (uint32_t spin = 0; ld_acquire_u32(f) < (unsigned)w.j; ++spin) {
-                            if ((spin & 15) == 15) {
-                                if (*abort_v || (p.status && *(volatile int*)p.status) ||
-                                    tc::globaltimer_ns() - t0 > 2000000000ull) {
-                                    ok = false;
-                                    break;
-                                }
-                            }
-                            __nanosleep(64);
-                        }
-                    }
+                         (hc == 0 || tc::mbar_wait(&bars->h_empty, (hc - 1) & 1, abort_v)) &&
+                         tc::mbar_wait(&bars->hin_full, hc & 1, abort_v);
                     if (!sync_ok(ok)) { alive = false; break; }
                     float hin[32];
-                    if (need_h) {
-                        if (!ready) {
-                            const uint8_t* g = reinterpret_cast<const uint8_t*>(hsrc + (size_t)row * kP + 32 * cg);
-#pragma unroll
-                            for (int q = 0; q < 8; ++q) cp_async16(hdst + ((q ^ (row & 7)) << 4), g + q * 16);
-                            cp_async_commit();
-                        }
-                        cp_async_wait_all();
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            const float4 v = *reinterpret_cast<const float4*>(hdst + ((q ^ (row & 7)) << 4));
-                            hin[4 * q] = v.x; hin[4 * q + 1] = v.y; hin[4 * q + 2] = v.z; hin[4 * q + 3] = v.w;
-                        }
-                    } else {
+                    const bool zero_in = MODE == kFused && w.j == 0;
+                    if (zero_in) {
 #pragma unroll
                         for (int e = 0; e < 32; ++e) hin[e] = 0.f;
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const float4 v = *reinterpret_cast<const float4*>(sHin + state_off(row, cg, q));
+                            hin[4 * q] = v.x; hin[4 * q + 1] = v.y; hin[4 * q + 2] = v.z; hin[4 * q + 3] = v.w;
+                        }
                     }
                     if (MODE == kFused) {
                         tc::tc_fence_after();
@@ -596,25 +625,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float eL = __expf(cum[kBlk - 1]);
 #pragma unroll
                         for (int e = 0; e < 32; ++e) zv[e] = fmaf(eL, hin[e], zv[e]);  // h_j
-                        const bool publish = !(p.test_stall && chain == 0 && w.j == 0);
-                        const size_t roff = (size_t)row * kP + 32 * cg;
-                        if (publish) {
-                            float4* dst = reinterpret_cast<float4*>(p.ring + ((size_t)chain * 2 + (w.j & 1)) * slot + roff);
 #pragma unroll
-                            for (int q = 0; q < 8; ++q)
-                                __stcg(dst + q, make_float4(zv[4 * q], zv[4 * q + 1], zv[4 * q + 2], zv[4 * q + 3]));
-                        }
+                        for (int q = 0; q < 8; ++q)
+                            *reinterpret_cast<float4*>(sHin + state_off(row, cg, q)) =
+                                make_float4(zv[4 * q], zv[4 * q + 1], zv[4 * q + 2], zv[4 * q + 3]);
                         if (last_blk && p.fin) {
-                            float4* fd = reinterpret_cast<float4*>(p.fin + (size_t)chain * slot + roff);
+                            float4* fd = reinterpret_cast<float4*>(p.fin + ((size_t)chain * kN + row) * kP + 32 * cg);
 #pragma unroll
                             for (int q = 0; q < 8; ++q)
                                 fd[q] = make_float4(zv[4 * q], zv[4 * q + 1], zv[4 * q + 2], zv[4 * q + 3]);
                         }
-                        // every thread's stores precede the barrier; one release at
-                        // gpu scope then publishes them all
-                        compute_sync();
-                        if (publish && ct == 0) st_release_u32(p.flags + chain, (unsigned)(w.j + 1));
+                        tc::fence_proxy_async_smem();  // the publisher's TMA store reads sHin
                     }
+                    tc::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(MODE == kFused ? &bars->hout_full : &bars->hin_free);
                     // Hin as the bf16 B operand of V = C Hin: rows n, 64 p per row (MN-major)
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4) {
@@ -626,15 +651,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         *reinterpret_cast<uint4*>(sH + tc::sw128_offset(row, 4 * cg + c4)) = v;
                     }
                     tc::fence_proxy_async_smem();
-                    tc::tc_fence_before();
                     __syncwarp();
                     if (lane == 0) tc::mbar_arrive(&bars->h_full);
                 }
             }
             if (!alive) break;
             // ---- T5 of the slice's last head
-            if (!epilogue(p.hpb - 1, hc - 1, xc - 1)) { alive = false; break; }
+            if (!epilogue(p.hpb - 1, hc - 1)) { alive = false; break; }
         }
+        if (ct == 0) tc::bulk_wait<0>();
     }
     tc::tc_fence_before();
     __syncthreads();
@@ -645,7 +670,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-int num_sms();
+int num_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+    return n > 0 ? n : 148;
+}
 
 // Heads per work item: the largest divisor of H/G (at most kHpbMax) that still
 // leaves at least one item per SM for every block index, so that a block's
@@ -663,22 +693,16 @@ int heads_per_item(const Dims& d) {
     return best > 0 ? best : largest;
 }
 
-int num_sms() {
-    int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
-    return n > 0 ? n : 148;
-}
-
 template <int MODE>
 cudaError_t launch(const Dims& d, const void* x, const void* Bm, const void* Cm, void* y,
-                   ScanParams p, cudaStream_t st) {
-    CUtensorMap tx, tb, tcm;
+                   const float* states, uint64_t state_rows, ScanParams p, cudaStream_t st) {
+    CUtensorMap tx, tb, tcm, ty, ts;
     cudaError_t e = make_tmap_bf16_3d(&tx, x, d.P, d.H, (uint64_t)d.B * d.T, kBlk);
     if (e == cudaSuccess) e = make_tmap_bf16_3d(&tb, Bm, d.N, d.G, (uint64_t)d.B * d.T, kBlk);
     if (e == cudaSuccess) e = make_tmap_bf16_3d(&tcm, Cm, d.N, d.G, (uint64_t)d.B * d.T, kBlk);
+    if (e == cudaSuccess) e = make_tmap_bf16_3d(&ty, y, d.P, d.H, (uint64_t)d.B * d.T, kBlk);
+    if (e == cudaSuccess) e = make_tmap_f32_rows64(&ts, states, state_rows);
     if (e != cudaSuccess) return e;
-    p.y = reinterpret_cast<__nv_bfloat16*>(y);
     p.T = d.T; p.H = d.H; p.G = d.G;
     p.nblk = d.T / kBlk;
     p.hpb = heads_per_item(d);
@@ -690,7 +714,7 @@ cudaError_t launch(const Dims& d, const void* x, const void* Bm, const void* Cm,
     e = cudaFuncSetAttribute(scan_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemBytes);
     if (e != cudaSuccess) return e;
-    scan_tc_kernel<MODE><<<grid, kThreads, kSmemBytes, st>>>(tx, tb, tcm, p, d.B);
+    scan_tc_kernel<MODE><<<grid, kThreads, kSmemBytes, st>>>(tx, tb, tcm, ty, ts, p, d.B);
     return cudaGetLastError();
 }
 
@@ -706,9 +730,8 @@ cudaError_t launch_chunk_scan_tc(const Dims& d, const void* x, const void* Bm, c
     if (!chunk_scan_tc_supported(d)) return cudaErrorNotSupported;
     ScanParams p = {};
     p.cum = cum;
-    p.hin = Hin;
     p.D = D;
-    return launch<kScan>(d, x, Bm, Cm, y, p, st);
+    return launch<kScan>(d, x, Bm, Cm, y, Hin, (uint64_t)d.B * d.H * (d.T / kBlk) * kN, p, st);
 }
 
 bool fused_supported(const Dims& d) {
@@ -724,12 +747,11 @@ cudaError_t launch_fused_tc(const Dims& d, const void* x, const float* a, const 
     ScanParams p = {};
     p.a = a;
     p.D = D;
-    p.ring = ring;
     p.flags = flags;
     p.fin = fin;
     p.status = status;
     p.test_stall = test_stall ? 1 : 0;
-    return launch<kFused>(d, x, Bm, Cm, y, p, st);
+    return launch<kFused>(d, x, Bm, Cm, y, ring, (uint64_t)d.B * d.H * 2 * kN, p, st);
 }
 
 }  // namespace ssd
