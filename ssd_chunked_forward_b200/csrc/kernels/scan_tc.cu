@@ -351,17 +351,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                             continue;
                         }
                         // bounded wait for the previous block of this chain
+                        // (exponential back-off keeps this thread off the issue slots
+                        // of the compute warps that share its scheduler)
                         const unsigned* f = p.flags + chain;
                         const uint64_t t0 = tc::globaltimer_ns();
+                        uint32_t nap = 32;
                         for (uint32_t spin = 0; ld_acquire_u32(f) < (unsigned)w.j; ++spin) {
-                            if ((spin & 15) == 15) {
+                            if ((spin & 7) == 7) {
                                 if (*abort_v || (p.status && *(volatile int*)p.status) ||
                                     tc::globaltimer_ns() - t0 > 2000000000ull) {
                                     ok = false;
                                     break;
                                 }
                             }
-                            __nanosleep(32);
+                            __nanosleep(nap);
+                            if (nap < 1024) nap <<= 1;
                         }
                         if (!ok) break;
                         tc::fence_proxy_async_global();  // the acquire orders the TMA read

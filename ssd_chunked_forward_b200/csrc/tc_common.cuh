@@ -56,19 +56,32 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
+// try_wait with a suspend-time hint: the thread sleeps until the phase
+// completes or about `hint_ns` passes, instead of spinning on issue slots
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity to complete.  Gives up
 // (returns false) once `budget_ns` of wall time has passed or *abort became
-// non-zero; callers then record a status and unwind.
+// non-zero; callers then record a status and unwind.  Between checks the
+// thread sleeps inside try_wait (at most ~0.5 ms per round).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort,
                                           uint64_t budget_ns = 2000000000ull) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    for (uint32_t i = 0;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 31) == 31) {
-            if (abort && *abort) return false;
-            if (globaltimer_ns() - t0 > budget_ns) return false;
-        }
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, 500000u)) return true;
+        if (abort && *abort) return false;
+        if (globaltimer_ns() - t0 > budget_ns) return false;
     }
 }
 
