@@ -89,7 +89,7 @@ constexpr uint32_t OFF_HIN = OFF_H + kTile;        // fp32 state, two swizzled 1
 constexpr uint32_t OFF_Y = OFF_HIN + 2 * kTile;    // bf16 y staging for the TMA store
 constexpr uint32_t OFF_CUM = OFF_Y + kTile;
 constexpr uint32_t OFF_VEC = OFF_CUM + kHpbMax * kBlk * 4;
-constexpr uint32_t OFF_BAR = OFF_VEC + 4 * kBlk * 4;
+constexpr uint32_t OFF_BAR = OFF_VEC + 5 * kBlk * 4;
 constexpr uint32_t OFF_MISC = OFF_BAR + ((sizeof(Bars) + 15) / 16) * 16;
 constexpr size_t kSmemBytes = 1024 + OFF_MISC + 16;
 
@@ -120,6 +120,15 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
 __device__ __forceinline__ void st_release_u32(unsigned* p, unsigned v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+
+// 2^x on the special-function unit (the hardware instruction, ~2^-22
+// relative error, ample for bf16 operands)
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+constexpr float kLog2e = 1.4426950408889634f;
 
 struct Item {
     int b, j, h0, g;
@@ -163,6 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* sCum = reinterpret_cast<float*>(sm + OFF_CUM);  // [hpb][128]
     float* sW = reinterpret_cast<float*>(sm + OFF_VEC);    // [128]
     float* sColf = sW + kBlk;                              // [3][128]
+    float* sC2 = sColf + 3 * kBlk;                         // [128] cum * log2(e)
     Bars* bars = reinterpret_cast<Bars*>(sm + OFF_BAR);
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
     int* sAbort = reinterpret_cast<int*>(sm + OFF_MISC + 4);
@@ -485,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc::tmem_ld32(lane_base + col_y(eb) + 32 * cg, yv);
                 tc::tmem_ld32(lane_base + col_v(eb) + 32 * cg, vv);
                 tc::tmem_ld_wait();
-                const float ecum = __expf(sCum[hi * kBlk + row]);
+                const float ecum = ex2_approx(sCum[hi * kBlk + row] * kLog2e);
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4) {
                     uint32_t o[4];
@@ -518,11 +528,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float* cum = sCum + i * kBlk;
                 // ---- T1: decay vectors of this head
                 if (cg == 0) {
-                    const float c = cum[ct];
-                    sW[ct] = __expf(cum[kBlk - 1] - c);
-                    sColf[ct] = ct < 32 ? __expf(cum[31] - c) : 0.f;
-                    sColf[kBlk + ct] = ct < 64 ? __expf(cum[63] - c) : 0.f;
-                    sColf[2 * kBlk + ct] = ct < 96 ? __expf(cum[95] - c) : 0.f;
+                    const float c = cum[ct] * kLog2e;
+                    sC2[ct] = c;
+                    sW[ct] = ex2_approx(cum[kBlk - 1] * kLog2e - c);
+                    sColf[ct] = ct < 32 ? ex2_approx(cum[31] * kLog2e - c) : 0.f;
+                    sColf[kBlk + ct] = ct < 64 ? ex2_approx(cum[63] * kLog2e - c) : 0.f;
+                    sColf[2 * kBlk + ct] = ct < 96 ? ex2_approx(cum[95] * kLog2e - c) : 0.f;
                 }
                 // ---- T2: weighted copy of x for the block state (fused)
                 if (MODE == kFused) {
@@ -556,32 +567,52 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!sync_ok(ok)) { alive = false; break; }
                 tc::tc_fence_after();
                 {
+                    // Row `row` (quad `quad` of 32 rows), columns [64 cg, 64 cg + 64) as two
+                    // 32-column sub-blocks sb.  sb < quad: below the diagonal, the mask
+                    // factorises as rowf * colf[s]; sb == quad: explicit exp2 per element;
+                    // sb > quad: masked out.  Both TMEM loads are issued before one wait.
                     const float dv = p.D ? __ldg(p.D + h) : 0.f;
-                    const float ct_cum = cum[row];
-                    const float rowf = quad > 0 ? __expf(ct_cum - cum[32 * quad - 1]) : 0.f;
+                    const float r2 = sC2[row];
+                    const float rowf = quad > 0 ? ex2_approx(r2 - sC2[32 * quad - 1]) : 0.f;
                     const float* colf = sColf + (quad > 0 ? (quad - 1) * kBlk : 0);
                     uint8_t* ptile = sP + cg * kTile;
-#pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        const int sb = 2 * cg + q;  // 32-column sub-block of s
+                    const int sb0 = 2 * cg, sb1 = 2 * cg + 1;
+                    float v0[32], v1[32];
+                    if (sb0 <= quad) tc::tmem_ld32(lane_base + COL_S + 32 * sb0, v0);
+                    if (sb1 <= quad) tc::tmem_ld32(lane_base + COL_S + 32 * sb1, v1);
+                    if (sb0 <= quad) tc::tmem_ld_wait();
+                    auto finish = [&](float (&v)[32], int sb, int q) {
                         uint32_t pk[16];
                         if (sb > quad) {
 #pragma unroll
                             for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                        } else if (sb < quad) {
+                            const float4* cf = reinterpret_cast<const float4*>(colf + 32 * sb);
+#pragma unroll
+                            for (int e4 = 0; e4 < 8; ++e4) {
+                                const float4 f = cf[e4];
+                                v[4 * e4 + 0] *= rowf * f.x;
+                                v[4 * e4 + 1] *= rowf * f.y;
+                                v[4 * e4 + 2] *= rowf * f.z;
+                                v[4 * e4 + 3] *= rowf * f.w;
+                            }
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) pk[e] = tc::pack_bf16x2(v[2 * e], v[2 * e + 1]);
                         } else {
-                            float v[32];
-                            tc::tmem_ld32(lane_base + COL_S + 32 * sb, v);
-                            tc::tmem_ld_wait();
-                            if (sb < quad) {
+                            const float4* c2 = reinterpret_cast<const float4*>(sC2 + 32 * sb);
+                            float m[32];
 #pragma unroll
-                                for (int e = 0; e < 32; ++e) v[e] *= rowf * colf[32 * sb + e];
-                            } else {
+                            for (int e4 = 0; e4 < 8; ++e4) {
+                                const float4 f = c2[e4];
+                                m[4 * e4 + 0] = f.x; m[4 * e4 + 1] = f.y;
+                                m[4 * e4 + 2] = f.z; m[4 * e4 + 3] = f.w;
+                            }
+                            const int rloc = row - 32 * sb;  // this row's column inside the block
 #pragma unroll
-                                for (int e = 0; e < 32; ++e) {
-                                    const int s = 32 * sb + e;
-                                    v[e] = (s < row) ? v[e] * __expf(ct_cum - cum[s])
-                                                     : (s == row ? v[e] + dv : 0.f);
-                                }
+                            for (int e = 0; e < 32; ++e) {
+                                // exponent <= 0 where it is used; masked lanes get a finite dummy
+                                const float ex = ex2_approx(e < rloc ? r2 - m[e] : 0.f);
+                                v[e] = e < rloc ? v[e] * ex : (e == rloc ? v[e] + dv : 0.f);
                             }
 #pragma unroll
                             for (int e = 0; e < 16; ++e) pk[e] = tc::pack_bf16x2(v[2 * e], v[2 * e + 1]);
@@ -592,7 +623,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             *reinterpret_cast<uint4*>(ptile + tc::sw128_offset(row, chunk)) =
                                 make_uint4(pk[4 * c4], pk[4 * c4 + 1], pk[4 * c4 + 2], pk[4 * c4 + 3]);
                         }
-                    }
+                    };
+                    finish(v0, sb0, 0);
+                    finish(v1, sb1, 1);
                 }
                 tc::fence_proxy_async_smem();
                 tc::tc_fence_before();
@@ -626,7 +659,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         float zv[32];
                         tc::tmem_ld32(lane_base + col_z(buf) + 32 * cg, zv);
                         tc::tmem_ld_wait();
-                        const float eL = __expf(cum[kBlk - 1]);
+                        const float eL = ex2_approx(cum[kBlk - 1] * kLog2e);
 #pragma unroll
                         for (int e = 0; e < 32; ++e) zv[e] = fmaf(eL, hin[e], zv[e]);  // h_j
 #pragma unroll
@@ -639,11 +672,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             for (int q = 0; q < 8; ++q)
                                 fd[q] = make_float4(zv[4 * q], zv[4 * q + 1], zv[4 * q + 2], zv[4 * q + 3]);
                         }
-                        tc::fence_proxy_async_smem();  // the publisher's TMA store reads sHin
                     }
-                    tc::tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) tc::mbar_arrive(MODE == kFused ? &bars->hout_full : &bars->hin_free);
                     // Hin as the bf16 B operand of V = C Hin: rows n, 64 p per row (MN-major)
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4) {
@@ -654,9 +683,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         v.w = tc::pack_bf16x2(hin[8 * c4 + 6], hin[8 * c4 + 7]);
                         *reinterpret_cast<uint4*>(sH + tc::sw128_offset(row, 4 * cg + c4)) = v;
                     }
+                    // one proxy fence covers the state written back into sHin (read by
+                    // the publisher's TMA store) and the bf16 operand in sH (read by the MMA)
                     tc::fence_proxy_async_smem();
+                    tc::tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) tc::mbar_arrive(&bars->h_full);
+                    if (lane == 0) {
+                        tc::mbar_arrive(MODE == kFused ? &bars->hout_full : &bars->hin_free);
+                        tc::mbar_arrive(&bars->h_full);
+                    }
                 }
             }
             if (!alive) break;
