@@ -34,9 +34,10 @@
 // operator": off-diagonal blocks are low-rank).
 //
 // Warp roles (384 threads): 0 TMA producer; 1 MMA issuer and TMEM owner;
-// 2-9 compute: two groups of four warps, each group covering all 128 TMEM
-// lanes, group g owning columns [32g, 32g+32) of P-wide tiles and
-// [64g, 64g+64) of the scores; 10 state loader; 11 state publisher (fused).
+// 2-5 group A (decay vectors, weighted x, masked scores P); 6-9 group B
+// (state step, output); 10 state loader; 11 state publisher (fused).  Each
+// group has one warp per TMEM lane quadrant (thread = tile row), and the two
+// groups work on different heads at the same time.
 // TMEM (512 columns): scores 0-127, then two buffers of {Z, Y, V} x 64
 // columns, alternating per head.
 #include "../common.cuh"
@@ -63,6 +64,7 @@ struct __align__(8) Bars {
     uint64_t x_full[kStages], x_empty[kStages];
     uint64_t xw_full, xw_empty, p_full, p_empty, h_full, h_empty;
     uint64_t hin_full, hin_free, hout_full;
+    uint64_t cum_full[2], cum_free[2];
     uint64_t y_full[2], v_full[2], z_full[2], t_empty[2];
     uint64_t done;
 };
@@ -88,7 +90,7 @@ constexpr uint32_t OFF_H = OFF_P + 2 * kTile;      // bf16 Hin, MN-major operand
 constexpr uint32_t OFF_HIN = OFF_H + kTile;        // fp32 state, two swizzled 128x32 boxes
 constexpr uint32_t OFF_Y = OFF_HIN + 2 * kTile;    // bf16 y staging for the TMA store
 constexpr uint32_t OFF_CUM = OFF_Y + kTile;
-constexpr uint32_t OFF_VEC = OFF_CUM + kHpbMax * kBlk * 4;
+constexpr uint32_t OFF_VEC = OFF_CUM + 2 * kHpbMax * kBlk * 4;
 constexpr uint32_t OFF_BAR = OFF_VEC + 5 * kBlk * 4;
 constexpr uint32_t OFF_MISC = OFF_BAR + ((sizeof(Bars) + 15) / 16) * 16;
 constexpr size_t kSmemBytes = 1024 + OFF_MISC + 16;
@@ -99,19 +101,6 @@ __device__ __forceinline__ uint32_t col_z(int buf) { return 128 + 192 * buf; }
 __device__ __forceinline__ uint32_t col_y(int buf) { return 192 + 192 * buf; }
 __device__ __forceinline__ uint32_t col_v(int buf) { return 256 + 192 * buf; }
 
-__device__ __forceinline__ void compute_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
-// barrier over the 256 compute threads that also ORs a predicate across them,
-// so every thread takes the same branch afterwards
-__device__ __forceinline__ bool compute_sync_or(bool pred) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\t"
-        "bar.red.or.pred po, 1, 256, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)pred)
-        : "memory");
-    return r != 0;
-}
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
     unsigned v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -169,7 +158,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* sH = sm + OFF_H;
     uint8_t* sHin = sm + OFF_HIN;
     uint8_t* sY = sm + OFF_Y;
-    float* sCum = reinterpret_cast<float*>(sm + OFF_CUM);  // [hpb][128]
+    float* sCum = reinterpret_cast<float*>(sm + OFF_CUM);  // [2][kHpbMax][128]
     float* sW = reinterpret_cast<float*>(sm + OFF_VEC);    // [128]
     float* sColf = sW + kBlk;                              // [3][128]
     float* sC2 = sColf + 3 * kBlk;                         // [128] cum * log2(e)
@@ -184,26 +173,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mbar_init(&bars->bc_full, 1);
         tc::mbar_init(&bars->bc_empty, 1);
         tc::mbar_init(&bars->s_full, 1);
-        tc::mbar_init(&bars->s_empty, 8);
+        tc::mbar_init(&bars->s_empty, 4);
         for (int s = 0; s < kStages; ++s) {
             tc::mbar_init(&bars->x_full[s], 1);
-            // Y MMA commit (+ the 8 compute warps that weight x, fused)
-            tc::mbar_init(&bars->x_empty[s], MODE == kFused ? 9 : 1);
+            // Y MMA commit (+ the 4 group-A warps that weight x, fused)
+            tc::mbar_init(&bars->x_empty[s], MODE == kFused ? 5 : 1);
         }
-        tc::mbar_init(&bars->xw_full, 8);
+        tc::mbar_init(&bars->xw_full, 4);
         tc::mbar_init(&bars->xw_empty, 1);
-        tc::mbar_init(&bars->p_full, 8);
+        tc::mbar_init(&bars->p_full, 4);
         tc::mbar_init(&bars->p_empty, 1);
-        tc::mbar_init(&bars->h_full, 8);
+        tc::mbar_init(&bars->h_full, 4);
         tc::mbar_init(&bars->h_empty, 1);
         tc::mbar_init(&bars->hin_full, 1);
-        tc::mbar_init(&bars->hin_free, MODE == kFused ? 1 : 8);
-        tc::mbar_init(&bars->hout_full, 8);
+        tc::mbar_init(&bars->hin_free, MODE == kFused ? 1 : 4);
+        tc::mbar_init(&bars->hout_full, 4);
+        for (int s = 0; s < 2; ++s) {
+            tc::mbar_init(&bars->cum_full[s], 4);
+            tc::mbar_init(&bars->cum_free[s], 4);
+        }
         for (int s = 0; s < 2; ++s) {
             tc::mbar_init(&bars->y_full[s], 1);
             tc::mbar_init(&bars->v_full[s], 1);
             tc::mbar_init(&bars->z_full[s], 1);
-            tc::mbar_init(&bars->t_empty[s], 8);
+            tc::mbar_init(&bars->t_empty[s], 4);
         }
         tc::mbar_init(&bars->done, 1);
         *sAbort = 0;
@@ -317,9 +310,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc::mma_commit(&bars->z_full[buf]);
                         tc::mma_commit(&bars->xw_empty);
                     }
-                    // V = C Hin of the previous head (its state was handed in before
-                    // this head's weighted x, so the wait is normally satisfied)
-                    if (i > 0 && !issue_v(hc - 1)) { ok = false; break; }
                     // Y = P X: M = t, N = p, K = s (P K-major, X MN-major)
                     ok = tc::mbar_wait(&bars->p_full, hc & 1, abort_v) &&
                          tc::mbar_wait(&bars->x_full[st], (xc / kStages) & 1, abort_v);
@@ -334,6 +324,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc::mma_commit(&bars->y_full[buf]);
                     tc::mma_commit(&bars->p_empty);
                     tc::mma_commit(&bars->x_empty[st]);
+                    // V = C Hin of the previous head (group B handed its state in while
+                    // group A built this head's operands)
+                    if (i > 0 && !issue_v(hc - 1)) { ok = false; break; }
                 }
                 if (!ok) break;
                 if (!issue_v(hc - 1)) { ok = false; break; }
@@ -424,264 +417,297 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::bulk_wait<0>();
         }
     } else {
-        // ================================================ compute (8 warps) ====
-        const int ct = threadIdx.x - 64;  // 0..255
-        const int cg = ct >> 7;           // column group 0/1
+        // ======================================= compute: two warpgroups ====
+        // Group A (warps 2-5) builds, per head, the decay vectors, the weighted
+        // copy of x and the masked score operand P; group B (warps 6-9) runs the
+        // state step and the output of the heads A has finished.  Each group has
+        // one warp per TMEM lane quadrant, so thread = tile row; the groups share
+        // no barrier and work on different heads at the same time.
+        const bool groupA = warp < 6;
+        const int gt = threadIdx.x - (groupA ? 64 : 192);  // 0..127 within the group
         const int quad = warp & 3;        // TMEM lane quadrant
         const int row = quad * 32 + lane; // TMEM lane = tile row
         const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-        uint32_t hc = 0, xc = 0, itc = 0;
-        bool alive = true;  // uniform across the compute threads
-
-        // Every abort decision of the compute warps goes through this reduction:
-        // a thread whose wait failed, or that sees another role's abort flag,
-        // makes all 256 compute threads leave together.
+        const int bar_id = groupA ? 1 : 2;
+        // Every abort decision of a group goes through this reduction, so the
+        // group's 128 threads always take the same branch.
         auto sync_ok = [&](bool ok) -> bool {
             if (!ok) fail();
-            const bool any = compute_sync_or(!ok || *abort_v != 0);
+            uint32_t r;
+            asm volatile(
+                "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\t"
+                "bar.red.or.pred po, %2, 128, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}"
+                : "=r"(r)
+                : "r"((uint32_t)(!ok || *abort_v != 0)), "r"(bar_id)
+                : "memory");
             __syncwarp();
-            return !any;
+            return r == 0;
         };
-        // per-item decay inputs (a or cum, hpb values per token row), loaded
-        // one item ahead into registers by the threads of column group 0
-        float anext[kHpbMax];
-        auto load_decays = [&](int it) {
-            if (cg != 0 || it >= p.n_items) return;
-            const Item w = decode_item(it, p, B);
-            if (MODE == kFused) {
-                const float* arow = p.a + (size_t)(w.b * p.T + w.j * kBlk + ct) * p.H + w.h0;
-#pragma unroll
-                for (int i = 0; i < kHpbMax; ++i) anext[i] = i < p.hpb ? __ldg(arow + i) : 0.f;
-            } else {
-#pragma unroll
-                for (int i = 0; i < kHpbMax; ++i)
-                    anext[i] = i < p.hpb ? __ldg(p.cum + (((size_t)w.b * p.H + w.h0 + i) * p.nblk + w.j) * kBlk + ct) : 0.f;
-            }
-        };
-        load_decays(blockIdx.x);
+        auto group_sync = [&]() { asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory"); };
 
-        for (int it = blockIdx.x; alive && it < p.n_items; it += gridDim.x, ++itc) {
-            const Item w = decode_item(it, p, B);
-            const int tok0 = w.b * p.T + w.j * kBlk;
-            const bool last_blk = (w.j == p.nblk - 1);
-            // ---- per-block cumulative log-decay of every head of the slice
-            if (cg == 0) {
-#pragma unroll
-                for (int i = 0; i < kHpbMax; ++i)
-                    if (i < p.hpb) sCum[i * kBlk + ct] = anext[i];
-            }
-            load_decays(it + gridDim.x);
-            compute_sync();
-            if (MODE == kFused) {
-                const int cw = ct >> 5;  // compute warp 0..7 scans head cw
-                if (cw < p.hpb) {
-                    float* c = sCum + cw * kBlk + lane * 4;
-                    float v0 = c[0], v1 = v0 + c[1], v2 = v1 + c[2], v3 = v2 + c[3];
-                    const float excl = warp_inclusive_scan(v3) - v3;
-                    c[0] = v0 + excl; c[1] = v1 + excl; c[2] = v2 + excl; c[3] = v3 + excl;
-                }
-                compute_sync();
-            }
-
-            // ---- T5: y = Y + exp(cum) V -> bf16 -> shared staging -> TMA store
-            auto epilogue = [&](int hi, uint32_t hcount) -> bool {
-                const int eb = hcount & 1;
-                const bool eok = tc::mbar_wait(&bars->y_full[eb], (hcount >> 1) & 1, abort_v) &&
-                                 tc::mbar_wait(&bars->v_full[eb], (hcount >> 1) & 1, abort_v);
-                if (ct == 0) tc::bulk_wait_read<0>();  // previous y tile left sY
-                if (!sync_ok(eok)) return false;
-                tc::tc_fence_after();
-                float yv[32], vv[32];
-                tc::tmem_ld32(lane_base + col_y(eb) + 32 * cg, yv);
-                tc::tmem_ld32(lane_base + col_v(eb) + 32 * cg, vv);
-                tc::tmem_ld_wait();
-                const float ecum = ex2_approx(sCum[hi * kBlk + row] * kLog2e);
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    uint32_t o[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int k0 = 8 * c4 + 2 * e;
-                        o[e] = tc::pack_bf16x2(fmaf(ecum, vv[k0], yv[k0]), fmaf(ecum, vv[k0 + 1], yv[k0 + 1]));
-                    }
-                    *reinterpret_cast<uint4*>(sY + tc::sw128_offset(row, 4 * cg + c4)) =
-                        make_uint4(o[0], o[1], o[2], o[3]);
-                }
-                tc::fence_proxy_async_smem();
-                tc::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&bars->t_empty[eb]);
-                compute_sync();
-                if (ct == 0) {
-                    tc::tma_store_3d(&tm_y, sY, 0, w.h0 + hi, tok0);
-                    tc::bulk_commit();
-                }
-                return true;
-            };
-
-            bool ok = true;  // this thread's wait results
-            for (int i = 0; i < p.hpb; ++i, ++hc, ++xc) {
-                const int h = w.h0 + i;
-                const int chain = w.b * p.H + h;
-                const int buf = hc & 1;
-                const uint32_t st = xc % kStages;
-                const float* cum = sCum + i * kBlk;
-                // ---- T1: decay vectors of this head
-                if (cg == 0) {
-                    const float c = cum[ct] * kLog2e;
-                    sC2[ct] = c;
-                    sW[ct] = ex2_approx(cum[kBlk - 1] * kLog2e - c);
-                    sColf[ct] = ct < 32 ? ex2_approx(cum[31] * kLog2e - c) : 0.f;
-                    sColf[kBlk + ct] = ct < 64 ? ex2_approx(cum[63] * kLog2e - c) : 0.f;
-                    sColf[2 * kBlk + ct] = ct < 96 ? ex2_approx(cum[95] * kLog2e - c) : 0.f;
-                }
-                // ---- T2: weighted copy of x for the block state (fused)
+        if (groupA) {
+            // ---------------------------------------------------- group A ----
+            uint32_t hc = 0, xc = 0, itc = 0;
+            float anext[kHpbMax];
+            auto load_decays = [&](int it) {
+                if (it >= p.n_items) return;
+                const Item w = decode_item(it, p, B);
                 if (MODE == kFused) {
-                    ok = tc::mbar_wait(&bars->x_full[st], (xc / kStages) & 1, abort_v) &&
-                         (hc == 0 || tc::mbar_wait(&bars->xw_empty, (hc - 1) & 1, abort_v));
-                    if (!sync_ok(ok)) { alive = false; break; }
-                    const uint8_t* xs = sX + st * kTile;
+                    const float* arow = p.a + (size_t)(w.b * p.T + w.j * kBlk + gt) * p.H + w.h0;
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int c = ct + 256 * q;
-                        const float wgt = sW[c >> 3];
-                        uint4 v = *reinterpret_cast<const uint4*>(xs + c * 16);
-                        uint32_t* u = reinterpret_cast<uint32_t*>(&v);
+                    for (int i = 0; i < kHpbMax; ++i) anext[i] = i < p.hpb ? __ldg(arow + i) : 0.f;
+                } else {
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 f = tc::unpack_bf16x2(u[e]);
-                            u[e] = tc::pack_bf16x2(f.x * wgt, f.y * wgt);
+                    for (int i = 0; i < kHpbMax; ++i)
+                        anext[i] = i < p.hpb ? __ldg(p.cum + (((size_t)w.b * p.H + w.h0 + i) * p.nblk + w.j) * kBlk + gt) : 0.f;
+                }
+            };
+            load_decays(blockIdx.x);
+            bool alive = true;
+            for (int it = blockIdx.x; alive && it < p.n_items; it += gridDim.x, ++itc) {
+                const Item w = decode_item(it, p, B);
+                float* cumbuf = sCum + (itc & 1) * (kHpbMax * kBlk);
+                // ---- cumulative log-decays of the slice's heads (buffer itc & 1)
+                if (!sync_ok(itc < 2 || tc::mbar_wait(&bars->cum_free[itc & 1], ((itc >> 1) - 1) & 1, abort_v)))
+                    break;
+#pragma unroll
+                for (int i = 0; i < kHpbMax; ++i)
+                    if (i < p.hpb) cumbuf[i * kBlk + gt] = anext[i];
+                load_decays(it + gridDim.x);
+                group_sync();
+                if (MODE == kFused) {
+                    // warp q scans heads q and q + 4 (128 values, 4 per lane)
+                    for (int hh = quad; hh < p.hpb; hh += 4) {
+                        float* c = cumbuf + hh * kBlk + lane * 4;
+                        float v0 = c[0], v1 = v0 + c[1], v2 = v1 + c[2], v3 = v2 + c[3];
+                        const float excl = warp_inclusive_scan(v3) - v3;
+                        c[0] = v0 + excl; c[1] = v1 + excl; c[2] = v2 + excl; c[3] = v3 + excl;
+                    }
+                    group_sync();
+                }
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&bars->cum_full[itc & 1]);
+
+                bool ok = true;
+                for (int i = 0; i < p.hpb; ++i, ++hc, ++xc) {
+                    const int h = w.h0 + i;
+                    const uint32_t st = xc % kStages;
+                    const float* cum = cumbuf + i * kBlk;
+                    // ---- T1: decay vectors of this head (thread = token row)
+                    {
+                        const float c = cum[gt] * kLog2e;
+                        sC2[gt] = c;
+                        sW[gt] = ex2_approx(cum[kBlk - 1] * kLog2e - c);
+                        sColf[gt] = gt < 32 ? ex2_approx(cum[31] * kLog2e - c) : 0.f;
+                        sColf[kBlk + gt] = gt < 64 ? ex2_approx(cum[63] * kLog2e - c) : 0.f;
+                        sColf[2 * kBlk + gt] = gt < 96 ? ex2_approx(cum[95] * kLog2e - c) : 0.f;
+                    }
+                    // ---- T2: weighted copy of x for the block state (fused)
+                    if (MODE == kFused) {
+                        ok = tc::mbar_wait(&bars->x_full[st], (xc / kStages) & 1, abort_v) &&
+                             (hc == 0 || tc::mbar_wait(&bars->xw_empty, (hc - 1) & 1, abort_v));
+                        if (!sync_ok(ok)) { alive = false; break; }
+                        const uint8_t* xs = sX + st * kTile;
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const int c = gt + 128 * q;
+                            const float wgt = sW[c >> 3];
+                            uint4 v = *reinterpret_cast<const uint4*>(xs + c * 16);
+                            uint32_t* u = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 f = tc::unpack_bf16x2(u[e]);
+                                u[e] = tc::pack_bf16x2(f.x * wgt, f.y * wgt);
+                            }
+                            *reinterpret_cast<uint4*>(sXw + c * 16) = v;
                         }
-                        *reinterpret_cast<uint4*>(sXw + c * 16) = v;
+                        tc::fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tc::mbar_arrive(&bars->xw_full);
+                            tc::mbar_arrive(&bars->x_empty[st]);
+                        }
+                    }
+                    // ---- T3: P = S o L + D I -> bf16, K-major in sP
+                    ok = (i > 0 || tc::mbar_wait(&bars->s_full, itc & 1, abort_v)) &&
+                         (hc == 0 || tc::mbar_wait(&bars->p_empty, (hc - 1) & 1, abort_v));
+                    if (!sync_ok(ok)) { alive = false; break; }
+                    tc::tc_fence_after();
+                    {
+                        // Row `row` (quad `quad`), 32-column sub-blocks sb of s: sb < quad
+                        // below the diagonal, the mask factorises as rowf * colf[s];
+                        // sb == quad: explicit exp2 per element; sb > quad: masked out.
+                        const float dv = p.D ? __ldg(p.D + h) : 0.f;
+                        const float r2 = sC2[row];
+                        const float rowf = quad > 0 ? ex2_approx(r2 - sC2[32 * quad - 1]) : 0.f;
+                        const float* colf = sColf + (quad > 0 ? (quad - 1) * kBlk : 0);
+                        auto finish = [&](float (&v)[32], int sb) {
+                            uint32_t pk[16];
+                            if (sb > quad) {
+#pragma unroll
+                                for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                            } else if (sb < quad) {
+                                const float4* cf = reinterpret_cast<const float4*>(colf + 32 * sb);
+#pragma unroll
+                                for (int e4 = 0; e4 < 8; ++e4) {
+                                    const float4 f = cf[e4];
+                                    v[4 * e4 + 0] *= rowf * f.x;
+                                    v[4 * e4 + 1] *= rowf * f.y;
+                                    v[4 * e4 + 2] *= rowf * f.z;
+                                    v[4 * e4 + 3] *= rowf * f.w;
+                                }
+#pragma unroll
+                                for (int e = 0; e < 16; ++e) pk[e] = tc::pack_bf16x2(v[2 * e], v[2 * e + 1]);
+                            } else {
+                                const float4* c2 = reinterpret_cast<const float4*>(sC2 + 32 * sb);
+                                float m[32];
+#pragma unroll
+                                for (int e4 = 0; e4 < 8; ++e4) {
+                                    const float4 f = c2[e4];
+                                    m[4 * e4 + 0] = f.x; m[4 * e4 + 1] = f.y;
+                                    m[4 * e4 + 2] = f.z; m[4 * e4 + 3] = f.w;
+                                }
+#pragma unroll
+                                for (int e = 0; e < 32; ++e) {
+                                    // exponent <= 0 where used; masked lanes get a finite dummy
+                                    const float ex = ex2_approx(e < lane ? r2 - m[e] : 0.f);
+                                    v[e] = e < lane ? v[e] * ex : (e == lane ? v[e] + dv : 0.f);
+                                }
+#pragma unroll
+                                for (int e = 0; e < 16; ++e) pk[e] = tc::pack_bf16x2(v[2 * e], v[2 * e + 1]);
+                            }
+                            uint8_t* ptile = sP + (sb >> 1) * kTile;
+#pragma unroll
+                            for (int c4 = 0; c4 < 4; ++c4) {
+                                const uint32_t chunk = 4 * (sb & 1) + c4;
+                                *reinterpret_cast<uint4*>(ptile + tc::sw128_offset(row, chunk)) =
+                                    make_uint4(pk[4 * c4], pk[4 * c4 + 1], pk[4 * c4 + 2], pk[4 * c4 + 3]);
+                            }
+                        };
+#pragma unroll
+                        for (int pair = 0; pair < 2; ++pair) {
+                            const int sb0 = 2 * pair, sb1 = 2 * pair + 1;
+                            float v0[32], v1[32];
+                            if (sb0 <= quad) tc::tmem_ld32(lane_base + COL_S + 32 * sb0, v0);
+                            if (sb1 <= quad) tc::tmem_ld32(lane_base + COL_S + 32 * sb1, v1);
+                            if (sb0 <= quad) tc::tmem_ld_wait();
+                            finish(v0, sb0);
+                            finish(v1, sb1);
+                        }
                     }
                     tc::fence_proxy_async_smem();
+                    tc::tc_fence_before();
                     __syncwarp();
                     if (lane == 0) {
-                        tc::mbar_arrive(&bars->xw_full);
-                        tc::mbar_arrive(&bars->x_empty[st]);
+                        tc::mbar_arrive(&bars->p_full);
+                        if (i == p.hpb - 1) tc::mbar_arrive(&bars->s_empty);
                     }
                 }
-                // ---- T3: P = S o L + D I  -> bf16, K-major in sP
-                ok = (i > 0 || tc::mbar_wait(&bars->s_full, itc & 1, abort_v)) &&
-                     (hc == 0 || tc::mbar_wait(&bars->p_empty, (hc - 1) & 1, abort_v));
-                if (!sync_ok(ok)) { alive = false; break; }
-                tc::tc_fence_after();
-                {
-                    // Row `row` (quad `quad` of 32 rows), columns [64 cg, 64 cg + 64) as two
-                    // 32-column sub-blocks sb.  sb < quad: below the diagonal, the mask
-                    // factorises as rowf * colf[s]; sb == quad: explicit exp2 per element;
-                    // sb > quad: masked out.  Both TMEM loads are issued before one wait.
-                    const float dv = p.D ? __ldg(p.D + h) : 0.f;
-                    const float r2 = sC2[row];
-                    const float rowf = quad > 0 ? ex2_approx(r2 - sC2[32 * quad - 1]) : 0.f;
-                    const float* colf = sColf + (quad > 0 ? (quad - 1) * kBlk : 0);
-                    uint8_t* ptile = sP + cg * kTile;
-                    const int sb0 = 2 * cg, sb1 = 2 * cg + 1;
-                    float v0[32], v1[32];
-                    if (sb0 <= quad) tc::tmem_ld32(lane_base + COL_S + 32 * sb0, v0);
-                    if (sb1 <= quad) tc::tmem_ld32(lane_base + COL_S + 32 * sb1, v1);
-                    if (sb0 <= quad) tc::tmem_ld_wait();
-                    auto finish = [&](float (&v)[32], int sb, int q) {
-                        uint32_t pk[16];
-                        if (sb > quad) {
+            }
+        } else {
+            // ---------------------------------------------------- group B ----
+            uint32_t hc = 0, itc = 0;
+            bool alive = true;
+            for (int it = blockIdx.x; alive && it < p.n_items; it += gridDim.x, ++itc) {
+                const Item w = decode_item(it, p, B);
+                const int tok0 = w.b * p.T + w.j * kBlk;
+                const bool last_blk = (w.j == p.nblk - 1);
+                const float* cumbuf = sCum + (itc & 1) * (kHpbMax * kBlk);
+                if (!sync_ok(tc::mbar_wait(&bars->cum_full[itc & 1], (itc >> 1) & 1, abort_v))) break;
+
+                // ---- T5: y = Y + exp(cum) V -> bf16 -> shared staging -> TMA store
+                auto epilogue = [&](int hi, uint32_t hcount) -> bool {
+                    const int eb = hcount & 1;
+                    const bool eok = tc::mbar_wait(&bars->y_full[eb], (hcount >> 1) & 1, abort_v) &&
+                                     tc::mbar_wait(&bars->v_full[eb], (hcount >> 1) & 1, abort_v);
+                    if (gt == 0) tc::bulk_wait_read<0>();  // previous y tile left sY
+                    if (!sync_ok(eok)) return false;
+                    tc::tc_fence_after();
+                    const float ecum = ex2_approx(cumbuf[hi * kBlk + row] * kLog2e);
 #pragma unroll
-                            for (int e = 0; e < 16; ++e) pk[e] = 0u;
-                        } else if (sb < quad) {
-                            const float4* cf = reinterpret_cast<const float4*>(colf + 32 * sb);
-#pragma unroll
-                            for (int e4 = 0; e4 < 8; ++e4) {
-                                const float4 f = cf[e4];
-                                v[4 * e4 + 0] *= rowf * f.x;
-                                v[4 * e4 + 1] *= rowf * f.y;
-                                v[4 * e4 + 2] *= rowf * f.z;
-                                v[4 * e4 + 3] *= rowf * f.w;
-                            }
-#pragma unroll
-                            for (int e = 0; e < 16; ++e) pk[e] = tc::pack_bf16x2(v[2 * e], v[2 * e + 1]);
-                        } else {
-                            const float4* c2 = reinterpret_cast<const float4*>(sC2 + 32 * sb);
-                            float m[32];
-#pragma unroll
-                            for (int e4 = 0; e4 < 8; ++e4) {
-                                const float4 f = c2[e4];
-                                m[4 * e4 + 0] = f.x; m[4 * e4 + 1] = f.y;
-                                m[4 * e4 + 2] = f.z; m[4 * e4 + 3] = f.w;
-                            }
-                            const int rloc = row - 32 * sb;  // this row's column inside the block
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) {
-                                // exponent <= 0 where it is used; masked lanes get a finite dummy
-                                const float ex = ex2_approx(e < rloc ? r2 - m[e] : 0.f);
-                                v[e] = e < rloc ? v[e] * ex : (e == rloc ? v[e] + dv : 0.f);
-                            }
-#pragma unroll
-                            for (int e = 0; e < 16; ++e) pk[e] = tc::pack_bf16x2(v[2 * e], v[2 * e + 1]);
-                        }
+                    for (int half = 0; half < 2; ++half) {
+                        float yv[32], vv[32];
+                        tc::tmem_ld32(lane_base + col_y(eb) + 32 * half, yv);
+                        tc::tmem_ld32(lane_base + col_v(eb) + 32 * half, vv);
+                        tc::tmem_ld_wait();
 #pragma unroll
                         for (int c4 = 0; c4 < 4; ++c4) {
-                            const uint32_t chunk = 4 * q + c4;
-                            *reinterpret_cast<uint4*>(ptile + tc::sw128_offset(row, chunk)) =
-                                make_uint4(pk[4 * c4], pk[4 * c4 + 1], pk[4 * c4 + 2], pk[4 * c4 + 3]);
+                            uint32_t o[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int k0 = 8 * c4 + 2 * e;
+                                o[e] = tc::pack_bf16x2(fmaf(ecum, vv[k0], yv[k0]), fmaf(ecum, vv[k0 + 1], yv[k0 + 1]));
+                            }
+                            *reinterpret_cast<uint4*>(sY + tc::sw128_offset(row, 4 * half + c4)) =
+                                make_uint4(o[0], o[1], o[2], o[3]);
                         }
-                    };
-                    finish(v0, sb0, 0);
-                    finish(v1, sb1, 1);
-                }
-                tc::fence_proxy_async_smem();
-                tc::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    tc::mbar_arrive(&bars->p_full);
-                    if (i == p.hpb - 1) tc::mbar_arrive(&bars->s_empty);
-                }
-                // ---- T5 of the previous head
-                if (i > 0 && !epilogue(i - 1, hc - 1)) { alive = false; break; }
-                // ---- T4: incoming state (and, fused, the block's own state out)
-                {
+                    }
+                    tc::fence_proxy_async_smem();
+                    tc::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(&bars->t_empty[eb]);
+                    group_sync();
+                    if (gt == 0) {
+                        tc::tma_store_3d(&tm_y, sY, 0, w.h0 + hi, tok0);
+                        tc::bulk_commit();
+                    }
+                    return true;
+                };
+
+                bool ok = true;
+                for (int i = 0; i < p.hpb; ++i, ++hc) {
+                    const int h = w.h0 + i;
+                    const int chain = w.b * p.H + h;
+                    const int buf = hc & 1;
+                    const float* cum = cumbuf + i * kBlk;
+                    // ---- T4: incoming state (and, fused, the block's own state out)
                     ok = (MODE == kScan || tc::mbar_wait(&bars->z_full[buf], (hc >> 1) & 1, abort_v)) &&
                          (hc == 0 || tc::mbar_wait(&bars->h_empty, (hc - 1) & 1, abort_v)) &&
                          tc::mbar_wait(&bars->hin_full, hc & 1, abort_v);
                     if (!sync_ok(ok)) { alive = false; break; }
-                    float hin[32];
+                    tc::tc_fence_after();
                     const bool zero_in = MODE == kFused && w.j == 0;
-                    if (zero_in) {
+                    const float eL = ex2_approx(cum[kBlk - 1] * kLog2e);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) hin[e] = 0.f;
-                    } else {
+                    for (int half = 0; half < 2; ++half) {
+                        float hin[32];
+                        if (zero_in) {
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            const float4 v = *reinterpret_cast<const float4*>(sHin + state_off(row, cg, q));
-                            hin[4 * q] = v.x; hin[4 * q + 1] = v.y; hin[4 * q + 2] = v.z; hin[4 * q + 3] = v.w;
+                            for (int e = 0; e < 32; ++e) hin[e] = 0.f;
+                        } else {
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) {
+                                const float4 v = *reinterpret_cast<const float4*>(sHin + state_off(row, half, q));
+                                hin[4 * q] = v.x; hin[4 * q + 1] = v.y; hin[4 * q + 2] = v.z; hin[4 * q + 3] = v.w;
+                            }
                         }
-                    }
-                    if (MODE == kFused) {
-                        tc::tc_fence_after();
-                        float zv[32];
-                        tc::tmem_ld32(lane_base + col_z(buf) + 32 * cg, zv);
-                        tc::tmem_ld_wait();
-                        const float eL = ex2_approx(cum[kBlk - 1] * kLog2e);
+                        if (MODE == kFused) {
+                            float zv[32];
+                            tc::tmem_ld32(lane_base + col_z(buf) + 32 * half, zv);
+                            tc::tmem_ld_wait();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) zv[e] = fmaf(eL, hin[e], zv[e]);  // h_j
-#pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            *reinterpret_cast<float4*>(sHin + state_off(row, cg, q)) =
-                                make_float4(zv[4 * q], zv[4 * q + 1], zv[4 * q + 2], zv[4 * q + 3]);
-                        if (last_blk && p.fin) {
-                            float4* fd = reinterpret_cast<float4*>(p.fin + ((size_t)chain * kN + row) * kP + 32 * cg);
+                            for (int e = 0; e < 32; ++e) zv[e] = fmaf(eL, hin[e], zv[e]);  // h_j
 #pragma unroll
                             for (int q = 0; q < 8; ++q)
-                                fd[q] = make_float4(zv[4 * q], zv[4 * q + 1], zv[4 * q + 2], zv[4 * q + 3]);
-                        }
-                    }
-                    // Hin as the bf16 B operand of V = C Hin: rows n, 64 p per row (MN-major)
+                                *reinterpret_cast<float4*>(sHin + state_off(row, half, q)) =
+                                    make_float4(zv[4 * q], zv[4 * q + 1], zv[4 * q + 2], zv[4 * q + 3]);
+                            if (last_blk && p.fin) {
+                                float4* fd = reinterpret_cast<float4*>(p.fin + ((size_t)chain * kN + row) * kP + 32 * half);
 #pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4) {
-                        uint4 v;
-                        v.x = tc::pack_bf16x2(hin[8 * c4 + 0], hin[8 * c4 + 1]);
-                        v.y = tc::pack_bf16x2(hin[8 * c4 + 2], hin[8 * c4 + 3]);
-                        v.z = tc::pack_bf16x2(hin[8 * c4 + 4], hin[8 * c4 + 5]);
-                        v.w = tc::pack_bf16x2(hin[8 * c4 + 6], hin[8 * c4 + 7]);
-                        *reinterpret_cast<uint4*>(sH + tc::sw128_offset(row, 4 * cg + c4)) = v;
+                                for (int q = 0; q < 8; ++q)
+                                    fd[q] = make_float4(zv[4 * q], zv[4 * q + 1], zv[4 * q + 2], zv[4 * q + 3]);
+                            }
+                        }
+                        // Hin as the bf16 B operand of V = C Hin: rows n, 64 p (MN-major)
+#pragma unroll
+                        for (int c4 = 0; c4 < 4; ++c4) {
+                            uint4 v;
+                            v.x = tc::pack_bf16x2(hin[8 * c4 + 0], hin[8 * c4 + 1]);
+                            v.y = tc::pack_bf16x2(hin[8 * c4 + 2], hin[8 * c4 + 3]);
+                            v.z = tc::pack_bf16x2(hin[8 * c4 + 4], hin[8 * c4 + 5]);
+                            v.w = tc::pack_bf16x2(hin[8 * c4 + 6], hin[8 * c4 + 7]);
+                            *reinterpret_cast<uint4*>(sH + tc::sw128_offset(row, 4 * half + c4)) = v;
+                        }
                     }
                     // one proxy fence covers the state written back into sHin (read by
                     // the publisher's TMA store) and the bf16 operand in sH (read by the MMA)
@@ -692,13 +718,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc::mbar_arrive(MODE == kFused ? &bars->hout_full : &bars->hin_free);
                         tc::mbar_arrive(&bars->h_full);
                     }
+                    // ---- T5 of the previous head (its V product ran meanwhile)
+                    if (i > 0 && !epilogue(i - 1, hc - 1)) { alive = false; break; }
                 }
+                if (!alive) break;
+                if (!epilogue(p.hpb - 1, hc - 1)) break;
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&bars->cum_free[itc & 1]);
             }
-            if (!alive) break;
-            // ---- T5 of the slice's last head
-            if (!epilogue(p.hpb - 1, hc - 1)) { alive = false; break; }
+            if (gt == 0) tc::bulk_wait<0>();
         }
-        if (ct == 0) tc::bulk_wait<0>();
     }
     tc::tc_fence_before();
     __syncthreads();
