@@ -33,11 +33,12 @@
 // at the block boundary ("State Space Duality", "Two algorithms for one
 // operator": off-diagonal blocks are low-rank).
 //
-// Warp roles (384 threads): 0 TMA producer; 1 MMA issuer and TMEM owner;
-// 2-5 group A (decay vectors, weighted x, masked scores P); 6-9 group B
-// (state step, output); 10 state loader; 11 state publisher (fused).  Each
-// group has one warp per TMEM lane quadrant (thread = tile row), and the two
-// groups work on different heads at the same time.
+// Warp roles (640 threads): 0 TMA producer; 1 MMA issuer and TMEM owner;
+// 2-9 group A (decay vectors, weighted x, masked scores P); 10-17 group B
+// (state step, output); 18 state loader; 19 state publisher (fused).  Each
+// group has two warps per TMEM lane quadrant (thread = tile row, the two
+// warps splitting the columns), and the two groups work on different heads
+// at the same time.
 // TMEM (512 columns): scores 0-127, then two buffers of {Z, Y, V} x 64
 // columns, alternating per head.
 #include "../common.cuh"
@@ -53,7 +54,7 @@ constexpr int kN = 128;
 constexpr int kP = 64;
 constexpr int kStages = 2;
 constexpr int kHpbMax = 8;
-constexpr int kThreads = 384;
+constexpr int kThreads = 640;
 constexpr uint32_t kTile = kBlk * 128;  // 128 rows x 128 bytes
 constexpr uint32_t kStateBytes = kN * kP * 4;
 
@@ -173,30 +174,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mbar_init(&bars->bc_full, 1);
         tc::mbar_init(&bars->bc_empty, 1);
         tc::mbar_init(&bars->s_full, 1);
-        tc::mbar_init(&bars->s_empty, 4);
+        tc::mbar_init(&bars->s_empty, 8);
         for (int s = 0; s < kStages; ++s) {
             tc::mbar_init(&bars->x_full[s], 1);
-            // Y MMA commit (+ the 4 group-A warps that weight x, fused)
-            tc::mbar_init(&bars->x_empty[s], MODE == kFused ? 5 : 1);
+            // Y MMA commit (+ the 8 group-A warps that weight x, fused)
+            tc::mbar_init(&bars->x_empty[s], MODE == kFused ? 9 : 1);
         }
-        tc::mbar_init(&bars->xw_full, 4);
+        tc::mbar_init(&bars->xw_full, 8);
         tc::mbar_init(&bars->xw_empty, 1);
-        tc::mbar_init(&bars->p_full, 4);
+        tc::mbar_init(&bars->p_full, 8);
         tc::mbar_init(&bars->p_empty, 1);
-        tc::mbar_init(&bars->h_full, 4);
+        tc::mbar_init(&bars->h_full, 8);
         tc::mbar_init(&bars->h_empty, 1);
         tc::mbar_init(&bars->hin_full, 1);
-        tc::mbar_init(&bars->hin_free, MODE == kFused ? 1 : 4);
-        tc::mbar_init(&bars->hout_full, 4);
+        tc::mbar_init(&bars->hin_free, MODE == kFused ? 1 : 8);
+        tc::mbar_init(&bars->hout_full, 8);
         for (int s = 0; s < 2; ++s) {
-            tc::mbar_init(&bars->cum_full[s], 4);
-            tc::mbar_init(&bars->cum_free[s], 4);
+            tc::mbar_init(&bars->cum_full[s], 8);
+            tc::mbar_init(&bars->cum_free[s], 8);
         }
         for (int s = 0; s < 2; ++s) {
             tc::mbar_init(&bars->y_full[s], 1);
             tc::mbar_init(&bars->v_full[s], 1);
             tc::mbar_init(&bars->z_full[s], 1);
-            tc::mbar_init(&bars->t_empty[s], 4);
+            tc::mbar_init(&bars->t_empty[s], 8);
         }
         tc::mbar_init(&bars->done, 1);
         *sAbort = 0;
@@ -337,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::mma_commit(&bars->done);
             tc::mbar_wait(&bars->done, 0, nullptr, 200000000ull);
         }
-    } else if (warp == 10) {
+    } else if (warp == 18) {
         // ========================================== incoming-state loader ====
         if (lane == 0) {
             tc::prefetch_tmap(&tm_st);
@@ -387,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) fail();
             if (hc > 0) tc::mbar_wait(&bars->hin_full, (hc - 1) & 1, nullptr, 200000000ull);
         }
-    } else if (warp == 11) {
+    } else if (warp == 19) {
         // ============================================== state publisher ====
         if (MODE == kFused && lane == 0) {
             uint32_t hc = 0;
@@ -423,8 +424,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // state step and the output of the heads A has finished.  Each group has
         // one warp per TMEM lane quadrant, so thread = tile row; the groups share
         // no barrier and work on different heads at the same time.
-        const bool groupA = warp < 6;
-        const int gt = threadIdx.x - (groupA ? 64 : 192);  // 0..127 within the group
+        const bool groupA = warp < 10;
+        const int gt = threadIdx.x - (groupA ? 64 : 320);  // 0..255 within the group
+        const int cg = gt >> 7;           // column half of this warp (0/1)
         const int quad = warp & 3;        // TMEM lane quadrant
         const int row = quad * 32 + lane; // TMEM lane = tile row
         const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
@@ -436,21 +438,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t r;
             asm volatile(
                 "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\t"
-                "bar.red.or.pred po, %2, 128, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}"
+                "bar.red.or.pred po, %2, 256, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}"
                 : "=r"(r)
                 : "r"((uint32_t)(!ok || *abort_v != 0)), "r"(bar_id)
                 : "memory");
             __syncwarp();
             return r == 0;
         };
-        auto group_sync = [&]() { asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory"); };
+        auto group_sync = [&]() { asm volatile("bar.sync %0, 256;" ::"r"(bar_id) : "memory"); };
 
         if (groupA) {
             // ---------------------------------------------------- group A ----
             uint32_t hc = 0, xc = 0, itc = 0;
             float anext[kHpbMax];
             auto load_decays = [&](int it) {
-                if (it >= p.n_items) return;
+                if (cg != 0 || it >= p.n_items) return;
                 const Item w = decode_item(it, p, B);
                 if (MODE == kFused) {
                     const float* arow = p.a + (size_t)(w.b * p.T + w.j * kBlk + gt) * p.H + w.h0;
@@ -470,14 +472,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // ---- cumulative log-decays of the slice's heads (buffer itc & 1)
                 if (!sync_ok(itc < 2 || tc::mbar_wait(&bars->cum_free[itc & 1], ((itc >> 1) - 1) & 1, abort_v)))
                     break;
+                if (cg == 0) {
 #pragma unroll
-                for (int i = 0; i < kHpbMax; ++i)
-                    if (i < p.hpb) cumbuf[i * kBlk + gt] = anext[i];
+                    for (int i = 0; i < kHpbMax; ++i)
+                        if (i < p.hpb) cumbuf[i * kBlk + gt] = anext[i];
+                }
                 load_decays(it + gridDim.x);
                 group_sync();
                 if (MODE == kFused) {
-                    // warp q scans heads q and q + 4 (128 values, 4 per lane)
-                    for (int hh = quad; hh < p.hpb; hh += 4) {
+                    // group warp gw scans head gw (128 values, 4 per lane)
+                    for (int hh = gt >> 5; hh < p.hpb; hh += 8) {
                         float* c = cumbuf + hh * kBlk + lane * 4;
                         float v0 = c[0], v1 = v0 + c[1], v2 = v1 + c[2], v3 = v2 + c[3];
                         const float excl = warp_inclusive_scan(v3) - v3;
@@ -493,8 +497,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int h = w.h0 + i;
                     const uint32_t st = xc % kStages;
                     const float* cum = cumbuf + i * kBlk;
-                    // ---- T1: decay vectors of this head (thread = token row)
-                    {
+                    // ---- T1: decay vectors of this head (thread = token row).  The
+                    // previous head's mask build reads them, so wait for the group.
+                    if (i > 0) group_sync();
+                    if (cg == 0) {
                         const float c = cum[gt] * kLog2e;
                         sC2[gt] = c;
                         sW[gt] = ex2_approx(cum[kBlk - 1] * kLog2e - c);
@@ -509,8 +515,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (!sync_ok(ok)) { alive = false; break; }
                         const uint8_t* xs = sX + st * kTile;
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            const int c = gt + 128 * q;
+                        for (int q = 0; q < 4; ++q) {
+                            const int c = gt + 256 * q;
                             const float wgt = sW[c >> 3];
                             uint4 v = *reinterpret_cast<const uint4*>(xs + c * 16);
                             uint32_t* u = reinterpret_cast<uint32_t*>(&v);
@@ -585,14 +591,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                         };
 #pragma unroll
-                        for (int pair = 0; pair < 2; ++pair) {
-                            const int sb0 = 2 * pair, sb1 = 2 * pair + 1;
-                            float v0[32], v1[32];
-                            if (sb0 <= quad) tc::tmem_ld32(lane_base + COL_S + 32 * sb0, v0);
-                            if (sb1 <= quad) tc::tmem_ld32(lane_base + COL_S + 32 * sb1, v1);
-                            if (sb0 <= quad) tc::tmem_ld_wait();
-                            finish(v0, sb0);
-                            finish(v1, sb1);
+                        for (int k = 0; k < 2; ++k) {
+                            const int sb = 2 * cg + k;  // this warp's two 32-column sub-blocks
+                            float v[32];
+                            if (sb <= quad) {
+                                tc::tmem_ld32(lane_base + COL_S + 32 * sb, v);
+                                tc::tmem_ld_wait();
+                            }
+                            finish(v, sb);
                         }
                     }
                     tc::fence_proxy_async_smem();
@@ -624,8 +630,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!sync_ok(eok)) return false;
                     tc::tc_fence_after();
                     const float ecum = ex2_approx(cumbuf[hi * kBlk + row] * kLog2e);
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
+                    {
+                        const int half = cg;
                         float yv[32], vv[32];
                         tc::tmem_ld32(lane_base + col_y(eb) + 32 * half, yv);
                         tc::tmem_ld32(lane_base + col_v(eb) + 32 * half, vv);
@@ -668,8 +674,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc::tc_fence_after();
                     const bool zero_in = MODE == kFused && w.j == 0;
                     const float eL = ex2_approx(cum[kBlk - 1] * kLog2e);
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
+                    {
+                        const int half = cg;
                         float hin[32];
                         if (zero_in) {
 #pragma unroll
