@@ -138,6 +138,31 @@ ssd_status ssd_forward_host(const ssd_shape* shape, const void* x_h, const float
                             const void* Bm_h, const void* Cm_h, const float* D_h, void* y_h,
                             float* final_h, void* dev_buf, size_t dev_bytes, ssd_stream stream);
 
+/* ---- the forward without any allocation by the caller ------------------- */
+
+/* For callers that cannot allocate device memory when they call (a captured
+ * or allocator-frozen serving loop, a plugin given only its input and output
+ * buffers): the fused forward with its scratch in a fixed 24 MiB device array
+ * inside this library, present on every GPU that loads it until the process
+ * exits.  The pages have no counterpart; it is a deployment convenience.
+ *  - Inputs and outputs are as for ssd_forward (device pointers, caller owned);
+ *    nothing is allocated and no workspace is passed.
+ *  - Serves what SSD_PATH_FUSED serves (else SSD_ERR_UNSUPPORTED), with at most
+ *    360 (batch x head) chains: more returns SSD_ERR_WORKSPACE before any work
+ *    is queued.
+ *  - The first call on a device looks up the array's device address (with that
+ *    device current) and caches it; make that first call before any stream
+ *    capture.
+ *  - Every call shares the one array: calls that overlap on the GPU (other
+ *    streams, other host threads) race and must be serialised by the caller.
+ *    The array keeps the last call's contents; the status word and hand-off
+ *    counters are cleared at the start of each call.
+ *  - The device status word is not exposed; use ssd_forward with a workspace
+ *    when ssd_device_status is needed. */
+ssd_status ssd_forward_noalloc(const ssd_shape* shape, const void* x, const float* a,
+                               const void* Bm, const void* Cm, const float* D, void* y,
+                               float* final_state, ssd_stream stream);
+
 /* ---- the steps of the path, callable one by one ------------------------- */
 
 /* Step 1, ssd_chunk_cumsum: cum[b,h,k,j(,n)] = sum_{i<=j} a[b, kQ+i, h(, n)],

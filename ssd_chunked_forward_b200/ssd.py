@@ -25,7 +25,7 @@ EXPORTS = [
     "ssd_status_string", "ssd_workspace_size", "ssd_path_supported", "ssd_forward",
     "ssd_forward_path", "ssd_device_status", "ssd_chunk_cumsum", "ssd_chunk_state",
     "ssd_state_pass", "ssd_chunk_scan", "ssd_diag_scan", "ssd_forward_host_bytes",
-    "ssd_forward_host",
+    "ssd_forward_host", "ssd_forward_noalloc",
 ]
 
 
@@ -72,7 +72,8 @@ def load(path: str = LIB_PATH):
     lib.ssd_forward_host_bytes.argtypes = [sp]
     lib.ssd_forward_host_bytes.restype = sz
     lib.ssd_forward_host.argtypes = [sp, vp, fp, vp, vp, fp, vp, fp, vp, sz, vp]
-    for name in ("ssd_forward", "ssd_forward_path", "ssd_device_status", "ssd_chunk_cumsum",
+    lib.ssd_forward_noalloc.argtypes = [sp, vp, fp, vp, vp, fp, vp, fp, vp]
+    for name in ("ssd_forward_noalloc", "ssd_forward", "ssd_forward_path", "ssd_device_status", "ssd_chunk_cumsum",
                  "ssd_chunk_state", "ssd_state_pass", "ssd_chunk_scan", "ssd_diag_scan",
                  "ssd_forward_host"):
         getattr(lib, name).restype = ctypes.c_int
@@ -220,3 +221,20 @@ def forward_host(shape: Shape, x_h, a_h, Bm_h, Cm_h, D_h, y_h, final_h, dev_buf,
     _check(load().ssd_forward_host(ctypes.byref(shape), _ptr(x_h), _ptr(a_h), _ptr(Bm_h), _ptr(Cm_h),
                                    _ptr(D_h), _ptr(y_h), _ptr(final_h), _ptr(dev_buf),
                                    dev_buf.numel(), _stream(stream)), "ssd_forward_host")
+
+
+def forward_noalloc(x, a, Bm, Cm, D=None, chunk=256, *, y=None, final_state=None, stream=None):
+    """The fused forward with the library's own fixed scratch (no workspace,
+    nothing allocated by the library); see ssd_forward_noalloc in ssd.h."""
+    _check_inputs(x, a, Bm, Cm, D)
+    shape = shape_of(x, a, Bm, chunk)
+    B, T, H, P = x.shape
+    N = Bm.shape[3]
+    if y is None:
+        y = torch.empty_like(x)
+    if final_state is None:
+        final_state = torch.empty((B, H, N, P), dtype=torch.float32, device=x.device)
+    _check(load().ssd_forward_noalloc(ctypes.byref(shape), _ptr(x), _ptr(a), _ptr(Bm), _ptr(Cm),
+                                      _ptr(D), _ptr(y), _ptr(final_state), _stream(stream)),
+           "ssd_forward_noalloc")
+    return y, final_state
