@@ -514,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                              (hc == 0 || tc::mbar_wait(&bars->xw_empty, (hc - 1) & 1, abort_v));
                         if (!sync_ok(ok)) { alive = false; break; }
                         const uint8_t* xs = sX + st * kTile;
-#pragma unroll
+#pragma unroll 1
                         for (int q = 0; q < 4; ++q) {
                             const int c = gt + 256 * q;
                             const float wgt = sW[c >> 3];
@@ -547,58 +547,55 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float r2 = sC2[row];
                         const float rowf = quad > 0 ? ex2_approx(r2 - sC2[32 * quad - 1]) : 0.f;
                         const float* colf = sColf + (quad > 0 ? (quad - 1) * kBlk : 0);
-                        auto finish = [&](float (&v)[32], int sb) {
-                            uint32_t pk[16];
+                        // this warp's 64 columns, 16 at a time (a rolled loop keeps the
+                        // code small: 20 warps share the instruction cache)
+                        uint8_t* ptile = sP + cg * kTile;
+#pragma unroll 1
+                        for (int c16 = 0; c16 < 4; ++c16) {
+                            const int s0 = 64 * cg + 16 * c16;  // first column of the chunk
+                            const int sb = s0 >> 5;             // its 32-column sub-block
+                            uint32_t pk[8];
                             if (sb > quad) {
 #pragma unroll
-                                for (int e = 0; e < 16; ++e) pk[e] = 0u;
-                            } else if (sb < quad) {
-                                const float4* cf = reinterpret_cast<const float4*>(colf + 32 * sb);
-#pragma unroll
-                                for (int e4 = 0; e4 < 8; ++e4) {
-                                    const float4 f = cf[e4];
-                                    v[4 * e4 + 0] *= rowf * f.x;
-                                    v[4 * e4 + 1] *= rowf * f.y;
-                                    v[4 * e4 + 2] *= rowf * f.z;
-                                    v[4 * e4 + 3] *= rowf * f.w;
-                                }
-#pragma unroll
-                                for (int e = 0; e < 16; ++e) pk[e] = tc::pack_bf16x2(v[2 * e], v[2 * e + 1]);
+                                for (int e = 0; e < 8; ++e) pk[e] = 0u;
                             } else {
-                                const float4* c2 = reinterpret_cast<const float4*>(sC2 + 32 * sb);
-                                float m[32];
-#pragma unroll
-                                for (int e4 = 0; e4 < 8; ++e4) {
-                                    const float4 f = c2[e4];
-                                    m[4 * e4 + 0] = f.x; m[4 * e4 + 1] = f.y;
-                                    m[4 * e4 + 2] = f.z; m[4 * e4 + 3] = f.w;
-                                }
-#pragma unroll
-                                for (int e = 0; e < 32; ++e) {
-                                    // exponent <= 0 where used; masked lanes get a finite dummy
-                                    const float ex = ex2_approx(e < lane ? r2 - m[e] : 0.f);
-                                    v[e] = e < lane ? v[e] * ex : (e == lane ? v[e] + dv : 0.f);
-                                }
-#pragma unroll
-                                for (int e = 0; e < 16; ++e) pk[e] = tc::pack_bf16x2(v[2 * e], v[2 * e + 1]);
-                            }
-                            uint8_t* ptile = sP + (sb >> 1) * kTile;
-#pragma unroll
-                            for (int c4 = 0; c4 < 4; ++c4) {
-                                const uint32_t chunk = 4 * (sb & 1) + c4;
-                                *reinterpret_cast<uint4*>(ptile + tc::sw128_offset(row, chunk)) =
-                                    make_uint4(pk[4 * c4], pk[4 * c4 + 1], pk[4 * c4 + 2], pk[4 * c4 + 3]);
-                            }
-                        };
-#pragma unroll
-                        for (int k = 0; k < 2; ++k) {
-                            const int sb = 2 * cg + k;  // this warp's two 32-column sub-blocks
-                            float v[32];
-                            if (sb <= quad) {
-                                tc::tmem_ld32(lane_base + COL_S + 32 * sb, v);
+                                float v[16];
+                                tc::tmem_ld16(lane_base + COL_S + s0, v);
                                 tc::tmem_ld_wait();
+                                if (sb < quad) {
+                                    const float4* cf = reinterpret_cast<const float4*>(colf + s0);
+#pragma unroll
+                                    for (int e4 = 0; e4 < 4; ++e4) {
+                                        const float4 f = cf[e4];
+                                        v[4 * e4 + 0] *= rowf * f.x;
+                                        v[4 * e4 + 1] *= rowf * f.y;
+                                        v[4 * e4 + 2] *= rowf * f.z;
+                                        v[4 * e4 + 3] *= rowf * f.w;
+                                    }
+                                } else {
+                                    const float4* c2 = reinterpret_cast<const float4*>(sC2 + s0);
+                                    float m[16];
+#pragma unroll
+                                    for (int e4 = 0; e4 < 4; ++e4) {
+                                        const float4 f = c2[e4];
+                                        m[4 * e4 + 0] = f.x; m[4 * e4 + 1] = f.y;
+                                        m[4 * e4 + 2] = f.z; m[4 * e4 + 3] = f.w;
+                                    }
+                                    const int rl = row - s0;  // the diagonal's column in the chunk
+#pragma unroll
+                                    for (int e = 0; e < 16; ++e) {
+                                        // exponent <= 0 where used; masked lanes get a finite dummy
+                                        const float ex = ex2_approx(e < rl ? r2 - m[e] : 0.f);
+                                        v[e] = e < rl ? v[e] * ex : (e == rl ? v[e] + dv : 0.f);
+                                    }
+                                }
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) pk[e] = tc::pack_bf16x2(v[2 * e], v[2 * e + 1]);
                             }
-                            finish(v, sb);
+                            *reinterpret_cast<uint4*>(ptile + tc::sw128_offset(row, 2 * c16)) =
+                                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                            *reinterpret_cast<uint4*>(ptile + tc::sw128_offset(row, 2 * c16 + 1)) =
+                                make_uint4(pk[4], pk[5], pk[6], pk[7]);
                         }
                     }
                     tc::fence_proxy_async_smem();
@@ -621,114 +618,120 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float* cumbuf = sCum + (itc & 1) * (kHpbMax * kBlk);
                 if (!sync_ok(tc::mbar_wait(&bars->cum_full[itc & 1], (itc >> 1) & 1, abort_v))) break;
 
-                // ---- T5: y = Y + exp(cum) V -> bf16 -> shared staging -> TMA store
-                auto epilogue = [&](int hi, uint32_t hcount) -> bool {
-                    const int eb = hcount & 1;
-                    const bool eok = tc::mbar_wait(&bars->y_full[eb], (hcount >> 1) & 1, abort_v) &&
-                                     tc::mbar_wait(&bars->v_full[eb], (hcount >> 1) & 1, abort_v);
-                    if (gt == 0) tc::bulk_wait_read<0>();  // previous y tile left sY
-                    if (!sync_ok(eok)) return false;
-                    tc::tc_fence_after();
-                    const float ecum = ex2_approx(cumbuf[hi * kBlk + row] * kLog2e);
-                    {
-                        const int half = cg;
-                        float yv[32], vv[32];
-                        tc::tmem_ld32(lane_base + col_y(eb) + 32 * half, yv);
-                        tc::tmem_ld32(lane_base + col_v(eb) + 32 * half, vv);
-                        tc::tmem_ld_wait();
-#pragma unroll
-                        for (int c4 = 0; c4 < 4; ++c4) {
-                            uint32_t o[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int k0 = 8 * c4 + 2 * e;
-                                o[e] = tc::pack_bf16x2(fmaf(ecum, vv[k0], yv[k0]), fmaf(ecum, vv[k0 + 1], yv[k0 + 1]));
-                            }
-                            *reinterpret_cast<uint4*>(sY + tc::sw128_offset(row, 4 * half + c4)) =
-                                make_uint4(o[0], o[1], o[2], o[3]);
-                        }
-                    }
-                    tc::fence_proxy_async_smem();
-                    tc::tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) tc::mbar_arrive(&bars->t_empty[eb]);
-                    group_sync();
-                    if (gt == 0) {
-                        tc::tma_store_3d(&tm_y, sY, 0, w.h0 + hi, tok0);
-                        tc::bulk_commit();
-                    }
-                    return true;
-                };
-
+                // Iteration i runs the state step of head i (i < hpb) and then the
+                // output of head i - 1 (i > 0), whose V product ran meanwhile; one
+                // copy of each body keeps the code small.
                 bool ok = true;
-                for (int i = 0; i < p.hpb; ++i, ++hc) {
-                    const int h = w.h0 + i;
-                    const int chain = w.b * p.H + h;
-                    const int buf = hc & 1;
-                    const float* cum = cumbuf + i * kBlk;
-                    // ---- T4: incoming state (and, fused, the block's own state out)
-                    ok = (MODE == kScan || tc::mbar_wait(&bars->z_full[buf], (hc >> 1) & 1, abort_v)) &&
-                         (hc == 0 || tc::mbar_wait(&bars->h_empty, (hc - 1) & 1, abort_v)) &&
-                         tc::mbar_wait(&bars->hin_full, hc & 1, abort_v);
-                    if (!sync_ok(ok)) { alive = false; break; }
-                    tc::tc_fence_after();
-                    const bool zero_in = MODE == kFused && w.j == 0;
-                    const float eL = ex2_approx(cum[kBlk - 1] * kLog2e);
-                    {
-                        const int half = cg;
-                        float hin[32];
-                        if (zero_in) {
+                for (int i = 0; i <= p.hpb; ++i) {
+                    if (i < p.hpb) {
+                        // ---- T4: incoming state (and, fused, the block's own state out)
+                        const int h = w.h0 + i;
+                        const int chain = w.b * p.H + h;
+                        const int buf = hc & 1;
+                        const float* cum = cumbuf + i * kBlk;
+                        ok = (MODE == kScan || tc::mbar_wait(&bars->z_full[buf], (hc >> 1) & 1, abort_v)) &&
+                             (hc == 0 || tc::mbar_wait(&bars->h_empty, (hc - 1) & 1, abort_v)) &&
+                             tc::mbar_wait(&bars->hin_full, hc & 1, abort_v);
+                        if (!sync_ok(ok)) { alive = false; break; }
+                        tc::tc_fence_after();
+                        const bool zero_in = MODE == kFused && w.j == 0;
+                        const float eL = ex2_approx(cum[kBlk - 1] * kLog2e);
+                        // this warp's 32 columns of the state, 16 at a time
+#pragma unroll 1
+                        for (int c = 0; c < 2; ++c) {
+                            float hin[16];
+                            if (zero_in) {
 #pragma unroll
-                            for (int e = 0; e < 32; ++e) hin[e] = 0.f;
-                        } else {
+                                for (int e = 0; e < 16; ++e) hin[e] = 0.f;
+                            } else {
 #pragma unroll
-                            for (int q = 0; q < 8; ++q) {
-                                const float4 v = *reinterpret_cast<const float4*>(sHin + state_off(row, half, q));
-                                hin[4 * q] = v.x; hin[4 * q + 1] = v.y; hin[4 * q + 2] = v.z; hin[4 * q + 3] = v.w;
+                                for (int q = 0; q < 4; ++q) {
+                                    const float4 v = *reinterpret_cast<const float4*>(sHin + state_off(row, cg, 4 * c + q));
+                                    hin[4 * q] = v.x; hin[4 * q + 1] = v.y; hin[4 * q + 2] = v.z; hin[4 * q + 3] = v.w;
+                                }
+                            }
+                            if (MODE == kFused) {
+                                float zv[16];
+                                tc::tmem_ld16(lane_base + col_z(buf) + 32 * cg + 16 * c, zv);
+                                tc::tmem_ld_wait();
+#pragma unroll
+                                for (int e = 0; e < 16; ++e) zv[e] = fmaf(eL, hin[e], zv[e]);  // h_j
+#pragma unroll
+                                for (int q = 0; q < 4; ++q)
+                                    *reinterpret_cast<float4*>(sHin + state_off(row, cg, 4 * c + q)) =
+                                        make_float4(zv[4 * q], zv[4 * q + 1], zv[4 * q + 2], zv[4 * q + 3]);
+                                if (last_blk && p.fin) {
+                                    float4* fd = reinterpret_cast<float4*>(
+                                        p.fin + ((size_t)chain * kN + row) * kP + 32 * cg + 16 * c);
+#pragma unroll
+                                    for (int q = 0; q < 4; ++q)
+                                        fd[q] = make_float4(zv[4 * q], zv[4 * q + 1], zv[4 * q + 2], zv[4 * q + 3]);
+                                }
+                            }
+                            // Hin as the bf16 B operand of V = C Hin: rows n, 64 p (MN-major)
+#pragma unroll
+                            for (int c8 = 0; c8 < 2; ++c8) {
+                                uint4 v;
+                                v.x = tc::pack_bf16x2(hin[8 * c8 + 0], hin[8 * c8 + 1]);
+                                v.y = tc::pack_bf16x2(hin[8 * c8 + 2], hin[8 * c8 + 3]);
+                                v.z = tc::pack_bf16x2(hin[8 * c8 + 4], hin[8 * c8 + 5]);
+                                v.w = tc::pack_bf16x2(hin[8 * c8 + 6], hin[8 * c8 + 7]);
+                                *reinterpret_cast<uint4*>(sH + tc::sw128_offset(row, 4 * cg + 2 * c + c8)) = v;
                             }
                         }
-                        if (MODE == kFused) {
-                            float zv[32];
-                            tc::tmem_ld32(lane_base + col_z(buf) + 32 * half, zv);
+                        // one proxy fence covers the state written back into sHin (read by
+                        // the publisher's TMA store) and the bf16 operand in sH (read by the MMA)
+                        tc::fence_proxy_async_smem();
+                        tc::tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tc::mbar_arrive(MODE == kFused ? &bars->hout_full : &bars->hin_free);
+                            tc::mbar_arrive(&bars->h_full);
+                        }
+                        ++hc;
+                    }
+                    if (i > 0) {
+                        // ---- T5: y = Y + exp(cum) V -> bf16 -> staging -> TMA store
+                        const int hi = i - 1;
+                        const uint32_t hcount = hc - (i < p.hpb ? 2 : 1);
+                        const int eb = hcount & 1;
+                        const bool eok = tc::mbar_wait(&bars->y_full[eb], (hcount >> 1) & 1, abort_v) &&
+                                         tc::mbar_wait(&bars->v_full[eb], (hcount >> 1) & 1, abort_v);
+                        if (gt == 0) tc::bulk_wait_read<0>();  // previous y tile left sY
+                        if (!sync_ok(eok)) { alive = false; break; }
+                        tc::tc_fence_after();
+                        const float ecum = ex2_approx(cumbuf[hi * kBlk + row] * kLog2e);
+#pragma unroll 1
+                        for (int c = 0; c < 2; ++c) {
+                            float yv[16], vv[16];
+                            tc::tmem_ld16(lane_base + col_y(eb) + 32 * cg + 16 * c, yv);
+                            tc::tmem_ld16(lane_base + col_v(eb) + 32 * cg + 16 * c, vv);
                             tc::tmem_ld_wait();
 #pragma unroll
-                            for (int e = 0; e < 32; ++e) zv[e] = fmaf(eL, hin[e], zv[e]);  // h_j
+                            for (int c8 = 0; c8 < 2; ++c8) {
+                                uint32_t o[4];
 #pragma unroll
-                            for (int q = 0; q < 8; ++q)
-                                *reinterpret_cast<float4*>(sHin + state_off(row, half, q)) =
-                                    make_float4(zv[4 * q], zv[4 * q + 1], zv[4 * q + 2], zv[4 * q + 3]);
-                            if (last_blk && p.fin) {
-                                float4* fd = reinterpret_cast<float4*>(p.fin + ((size_t)chain * kN + row) * kP + 32 * half);
-#pragma unroll
-                                for (int q = 0; q < 8; ++q)
-                                    fd[q] = make_float4(zv[4 * q], zv[4 * q + 1], zv[4 * q + 2], zv[4 * q + 3]);
+                                for (int e = 0; e < 4; ++e) {
+                                    const int k0 = 8 * c8 + 2 * e;
+                                    o[e] = tc::pack_bf16x2(fmaf(ecum, vv[k0], yv[k0]),
+                                                           fmaf(ecum, vv[k0 + 1], yv[k0 + 1]));
+                                }
+                                *reinterpret_cast<uint4*>(sY + tc::sw128_offset(row, 4 * cg + 2 * c + c8)) =
+                                    make_uint4(o[0], o[1], o[2], o[3]);
                             }
                         }
-                        // Hin as the bf16 B operand of V = C Hin: rows n, 64 p (MN-major)
-#pragma unroll
-                        for (int c4 = 0; c4 < 4; ++c4) {
-                            uint4 v;
-                            v.x = tc::pack_bf16x2(hin[8 * c4 + 0], hin[8 * c4 + 1]);
-                            v.y = tc::pack_bf16x2(hin[8 * c4 + 2], hin[8 * c4 + 3]);
-                            v.z = tc::pack_bf16x2(hin[8 * c4 + 4], hin[8 * c4 + 5]);
-                            v.w = tc::pack_bf16x2(hin[8 * c4 + 6], hin[8 * c4 + 7]);
-                            *reinterpret_cast<uint4*>(sH + tc::sw128_offset(row, 4 * half + c4)) = v;
+                        tc::fence_proxy_async_smem();
+                        tc::tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) tc::mbar_arrive(&bars->t_empty[eb]);
+                        group_sync();
+                        if (gt == 0) {
+                            tc::tma_store_3d(&tm_y, sY, 0, w.h0 + hi, tok0);
+                            tc::bulk_commit();
                         }
                     }
-                    // one proxy fence covers the state written back into sHin (read by
-                    // the publisher's TMA store) and the bf16 operand in sH (read by the MMA)
-                    tc::fence_proxy_async_smem();
-                    tc::tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tc::mbar_arrive(MODE == kFused ? &bars->hout_full : &bars->hin_free);
-                        tc::mbar_arrive(&bars->h_full);
-                    }
-                    // ---- T5 of the previous head (its V product ran meanwhile)
-                    if (i > 0 && !epilogue(i - 1, hc - 1)) { alive = false; break; }
                 }
                 if (!alive) break;
-                if (!epilogue(p.hpb - 1, hc - 1)) break;
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&bars->cum_free[itc & 1]);
             }
