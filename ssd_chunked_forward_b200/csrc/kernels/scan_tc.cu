@@ -41,6 +41,8 @@
 // at the same time.
 // TMEM (512 columns): scores 0-127, then two buffers of {Z, Y, V} x 64
 // columns, alternating per head.
+#include <stdlib.h>
+
 #include "../common.cuh"
 #include "../kernels.h"
 #include "../tc_common.cuh"
@@ -218,25 +220,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
 
     if (warp == 0) {
-        // =============================================== TMA producer ====
+        // =============================================== TMA producers ====
+        // lane 0 streams x (one tile per head); lane 1 loads each item's B and C
+        // tiles once the previous item's products no longer read them.  Two
+        // threads, so that x never waits behind the B/C release.
         if (lane == 0) {
             tc::prefetch_tmap(&tm_x);
-            tc::prefetch_tmap(&tm_b);
-            tc::prefetch_tmap(&tm_c);
-            uint32_t xc = 0, itc = 0;
+            uint32_t xc = 0;
             bool ok = true;
-            for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x, ++itc) {
+            for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x) {
                 const Item w = decode_item(it, p, B);
                 const int row0 = w.b * p.T + w.j * kBlk;
-                if (itc > 0 && !tc::mbar_wait(&bars->bc_empty, (itc - 1) & 1, abort_v)) {
-                    ok = false;
-                    break;
-                }
-                tc::mbar_arrive_expect_tx(&bars->bc_full, 4 * kTile);
-                tc::tma_load_3d(sB, &tm_b, &bars->bc_full, 0, w.g, row0);
-                tc::tma_load_3d(sB + kTile, &tm_b, &bars->bc_full, 64, w.g, row0);
-                tc::tma_load_3d(sC, &tm_c, &bars->bc_full, 0, w.g, row0);
-                tc::tma_load_3d(sC + kTile, &tm_c, &bars->bc_full, 64, w.g, row0);
                 for (int i = 0; i < p.hpb; ++i, ++xc) {
                     const uint32_t st = xc % kStages;
                     if (xc >= kStages &&
@@ -253,6 +247,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t first = xc > (uint32_t)kStages ? xc - kStages : 0u;
             for (uint32_t c = first; c < xc; ++c)
                 tc::mbar_wait(&bars->x_full[c % kStages], (c / kStages) & 1, nullptr, 200000000ull);
+        } else if (lane == 1) {
+            tc::prefetch_tmap(&tm_b);
+            tc::prefetch_tmap(&tm_c);
+            uint32_t itc = 0;
+            bool ok = true;
+            for (int it = blockIdx.x; it < p.n_items; it += gridDim.x, ++itc) {
+                const Item w = decode_item(it, p, B);
+                const int row0 = w.b * p.T + w.j * kBlk;
+                if (itc > 0 && !tc::mbar_wait(&bars->bc_empty, (itc - 1) & 1, abort_v)) {
+                    ok = false;
+                    break;
+                }
+                tc::mbar_arrive_expect_tx(&bars->bc_full, 4 * kTile);
+                tc::tma_load_3d(sB, &tm_b, &bars->bc_full, 0, w.g, row0);
+                tc::tma_load_3d(sB + kTile, &tm_b, &bars->bc_full, 64, w.g, row0);
+                tc::tma_load_3d(sC, &tm_c, &bars->bc_full, 0, w.g, row0);
+                tc::tma_load_3d(sC + kTile, &tm_c, &bars->bc_full, 64, w.g, row0);
+            }
+            if (!ok) fail();
             if (itc > 0) tc::mbar_wait(&bars->bc_full, (itc - 1) & 1, nullptr, 200000000ull);
         }
     } else if (warp == 1) {
@@ -760,6 +773,11 @@ int num_sms() {
 // divisor does (few chains), the largest one, to share the scores most.
 int heads_per_item(const Dims& d) {
     const int HG = d.H / d.G;
+    // tuning override: SSD_HEADS_PER_ITEM=<divisor of H/G, at most 8>
+    if (const char* env = getenv("SSD_HEADS_PER_ITEM")) {
+        const int c = atoi(env);
+        if (c >= 1 && c <= kHpbMax && HG % c == 0) return c;
+    }
     const int sms = num_sms();
     int best = 0, largest = 1;
     for (int c = 1; c <= kHpbMax; ++c) {

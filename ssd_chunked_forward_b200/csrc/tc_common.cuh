@@ -70,6 +70,18 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
     return ok != 0;
 }
 
+// Slow path of mbar_wait, kept out of line so that the many wait sites stay
+// small in the instruction cache.
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, const volatile int* abort,
+                                            uint64_t budget_ns) {
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, 500000u)) return true;
+        if (abort && *abort) return false;
+        if (globaltimer_ns() - t0 > budget_ns) return false;
+    }
+}
+
 // Bounded wait for the phase with the given parity to complete.  Gives up
 // (returns false) once `budget_ns` of wall time has passed or *abort became
 // non-zero; callers then record a status and unwind.  Between checks the
@@ -77,12 +89,7 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort,
                                           uint64_t budget_ns = 2000000000ull) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    for (;;) {
-        if (mbar_try_wait_sleep(bar, parity, 500000u)) return true;
-        if (abort && *abort) return false;
-        if (globaltimer_ns() - t0 > budget_ns) return false;
-    }
+    return mbar_wait_slow(bar, parity, abort, budget_ns);
 }
 
 // ------------------------------------------------------ async-proxy fences ----
