@@ -40,7 +40,8 @@
 // warps splitting the columns), and the two groups work on different heads
 // at the same time.
 // TMEM (512 columns): scores 0-127, then two buffers of {Z, Y, V} x 64
-// columns, alternating per head.
+// columns, alternating per head; Z is released after the state step, Y and V
+// after the output, so the next block state can start before the output.
 #include <stdlib.h>
 
 #include "../common.cuh"
@@ -68,7 +69,7 @@ struct __align__(8) Bars {
     uint64_t xw_full, xw_empty, p_full, p_empty, h_full, h_empty;
     uint64_t hin_full, hin_free, hout_full;
     uint64_t cum_full[2], cum_free[2];
-    uint64_t y_full[2], v_full[2], z_full[2], t_empty[2];
+    uint64_t y_full[2], v_full[2], z_full[2], z_empty[2], yv_empty[2];
     uint64_t done;
 };
 
@@ -199,7 +200,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::mbar_init(&bars->y_full[s], 1);
             tc::mbar_init(&bars->v_full[s], 1);
             tc::mbar_init(&bars->z_full[s], 1);
-            tc::mbar_init(&bars->t_empty[s], 8);
+            tc::mbar_init(&bars->z_empty[s], 8);   // group B read Z (state step)
+            tc::mbar_init(&bars->yv_empty[s], 8);  // group B read Y and V (output)
         }
         tc::mbar_init(&bars->done, 1);
         *sAbort = 0;
@@ -309,13 +311,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int i = 0; i < p.hpb; ++i, ++hc, ++xc) {
                     const int buf = hc & 1;
                     const uint32_t st = xc % kStages;
-                    if (hc >= 2 && !tc::mbar_wait(&bars->t_empty[buf], ((hc >> 1) - 1) & 1, abort_v)) {
-                        ok = false;
-                        break;
-                    }
                     if (MODE == kFused) {
-                        // block state Z = B^T (w o X): M = n (MN-major B tile), N = p, K = s
-                        if (!tc::mbar_wait(&bars->xw_full, hc & 1, abort_v)) { ok = false; break; }
+                        // block state Z = B^T (w o X): M = n (MN-major B tile), N = p, K = s.
+                        // Its buffer is free once group B's state step of head hc-2 read it.
+                        ok = (hc < 2 || tc::mbar_wait(&bars->z_empty[buf], ((hc >> 1) - 1) & 1, abort_v)) &&
+                             tc::mbar_wait(&bars->xw_full, hc & 1, abort_v);
+                        if (!ok) break;
                         tc::tc_fence_after();
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk)
@@ -324,8 +325,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc::mma_commit(&bars->z_full[buf]);
                         tc::mma_commit(&bars->xw_empty);
                     }
-                    // Y = P X: M = t, N = p, K = s (P K-major, X MN-major)
-                    ok = tc::mbar_wait(&bars->p_full, hc & 1, abort_v) &&
+                    // V = C Hin of the previous head as soon as group B handed the state
+                    // in (issued before Y, which waits for group A's operands)
+                    if (i > 0 && !issue_v(hc - 1)) { ok = false; break; }
+                    // Y = P X: M = t, N = p, K = s (P K-major, X MN-major).  Y and V of this
+                    // buffer are free once group B's output of head hc-2 read them.
+                    ok = (hc < 2 || tc::mbar_wait(&bars->yv_empty[buf], ((hc >> 1) - 1) & 1, abort_v)) &&
+                         tc::mbar_wait(&bars->p_full, hc & 1, abort_v) &&
                          tc::mbar_wait(&bars->x_full[st], (xc / kStages) & 1, abort_v);
                     if (!ok) break;
                     tc::tc_fence_after();
@@ -338,9 +344,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc::mma_commit(&bars->y_full[buf]);
                     tc::mma_commit(&bars->p_empty);
                     tc::mma_commit(&bars->x_empty[st]);
-                    // V = C Hin of the previous head (group B handed its state in while
-                    // group A built this head's operands)
-                    if (i > 0 && !issue_v(hc - 1)) { ok = false; break; }
                 }
                 if (!ok) break;
                 if (!issue_v(hc - 1)) { ok = false; break; }
@@ -700,6 +703,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (lane == 0) {
                             tc::mbar_arrive(MODE == kFused ? &bars->hout_full : &bars->hin_free);
                             tc::mbar_arrive(&bars->h_full);
+                            if (MODE == kFused) tc::mbar_arrive(&bars->z_empty[buf]);
                         }
                         ++hc;
                     }
@@ -736,7 +740,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc::fence_proxy_async_smem();
                         tc::tc_fence_before();
                         __syncwarp();
-                        if (lane == 0) tc::mbar_arrive(&bars->t_empty[eb]);
+                        if (lane == 0) tc::mbar_arrive(&bars->yv_empty[eb]);
                         group_sync();
                         if (gt == 0) {
                             tc::tma_store_3d(&tm_y, sY, 0, w.h0 + hi, tok0);
