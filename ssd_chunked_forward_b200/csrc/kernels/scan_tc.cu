@@ -67,9 +67,9 @@ struct __align__(8) Bars {
     uint64_t bc_full, bc_empty, s_full, s_empty;
     uint64_t x_full[kStages], x_empty[kStages];
     uint64_t xw_full, xw_empty, p_full, p_empty, h_full, h_empty;
-    uint64_t hin_full, hin_free, hout_full;
+    uint64_t hin_full, hin_free, hout_full, hout_free;
     uint64_t cum_full[2], cum_free[2];
-    uint64_t y_full[2], v_full[2], z_full[2], z_empty[2], yv_empty[2];
+    uint64_t y_full[2], v_full[2], yv_empty[2], z_full, z_empty;
     uint64_t done;
 };
 
@@ -89,21 +89,23 @@ constexpr uint32_t OFF_B = 0;
 constexpr uint32_t OFF_C = OFF_B + 2 * kTile;
 constexpr uint32_t OFF_X = OFF_C + 2 * kTile;
 constexpr uint32_t OFF_XW = OFF_X + kStages * kTile;
-constexpr uint32_t OFF_P = OFF_XW + kTile;
-constexpr uint32_t OFF_H = OFF_P + 2 * kTile;      // bf16 Hin, MN-major operand
-constexpr uint32_t OFF_HIN = OFF_H + kTile;        // fp32 state, two swizzled 128x32 boxes
-constexpr uint32_t OFF_Y = OFF_HIN + 2 * kTile;    // bf16 y staging for the TMA store
+constexpr uint32_t OFF_H = OFF_XW + kTile;         // bf16 Hin, MN-major operand
+constexpr uint32_t OFF_HIN = OFF_H + kTile;        // fp32 incoming state, two swizzled 128x32 boxes
+constexpr uint32_t OFF_HOUT = OFF_HIN + 2 * kTile; // fp32 outgoing state, same layout
+constexpr uint32_t OFF_Y = OFF_HOUT + 2 * kTile;   // bf16 y staging for the TMA store
 constexpr uint32_t OFF_CUM = OFF_Y + kTile;
 constexpr uint32_t OFF_VEC = OFF_CUM + 2 * kHpbMax * kBlk * 4;
 constexpr uint32_t OFF_BAR = OFF_VEC + 5 * kBlk * 4;
 constexpr uint32_t OFF_MISC = OFF_BAR + ((sizeof(Bars) + 15) / 16) * 16;
 constexpr size_t kSmemBytes = 1024 + OFF_MISC + 16;
+static_assert(kSmemBytes <= 232448, "shared memory above the 227 KB per-block limit");
 
 // TMEM columns
-constexpr uint32_t COL_S = 0;
-__device__ __forceinline__ uint32_t col_z(int buf) { return 128 + 192 * buf; }
-__device__ __forceinline__ uint32_t col_y(int buf) { return 192 + 192 * buf; }
-__device__ __forceinline__ uint32_t col_v(int buf) { return 256 + 192 * buf; }
+constexpr uint32_t COL_S = 0;    // scores, 128 fp32 columns
+constexpr uint32_t COL_P = 128;  // masked scores as the bf16 A operand, 64 columns
+constexpr uint32_t COL_Z = 192;  // block state, 64 columns
+__device__ __forceinline__ uint32_t col_y(int buf) { return 256 + 128 * buf; }
+__device__ __forceinline__ uint32_t col_v(int buf) { return 320 + 128 * buf; }
 
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
     unsigned v;
@@ -158,9 +160,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* sC = sm + OFF_C;
     uint8_t* sX = sm + OFF_X;
     uint8_t* sXw = sm + OFF_XW;
-    uint8_t* sP = sm + OFF_P;
     uint8_t* sH = sm + OFF_H;
     uint8_t* sHin = sm + OFF_HIN;
+    uint8_t* sHout = sm + OFF_HOUT;
     uint8_t* sY = sm + OFF_Y;
     float* sCum = reinterpret_cast<float*>(sm + OFF_CUM);  // [2][kHpbMax][128]
     float* sW = reinterpret_cast<float*>(sm + OFF_VEC);    // [128]
@@ -190,8 +192,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mbar_init(&bars->h_full, 8);
         tc::mbar_init(&bars->h_empty, 1);
         tc::mbar_init(&bars->hin_full, 1);
-        tc::mbar_init(&bars->hin_free, MODE == kFused ? 1 : 8);
-        tc::mbar_init(&bars->hout_full, 8);
+        tc::mbar_init(&bars->hin_free, 8);   // group B read the incoming state
+        tc::mbar_init(&bars->hout_full, 8);  // group B wrote the outgoing state
+        tc::mbar_init(&bars->hout_free, 1);  // the publisher's store read it
+        tc::mbar_init(&bars->z_full, 1);
+        tc::mbar_init(&bars->z_empty, 8);
         for (int s = 0; s < 2; ++s) {
             tc::mbar_init(&bars->cum_full[s], 8);
             tc::mbar_init(&bars->cum_free[s], 8);
@@ -199,8 +204,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < 2; ++s) {
             tc::mbar_init(&bars->y_full[s], 1);
             tc::mbar_init(&bars->v_full[s], 1);
-            tc::mbar_init(&bars->z_full[s], 1);
-            tc::mbar_init(&bars->z_empty[s], 8);   // group B read Z (state step)
             tc::mbar_init(&bars->yv_empty[s], 8);  // group B read Y and V (output)
         }
         tc::mbar_init(&bars->done, 1);
@@ -278,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t id_y = tc::idesc_bf16_f32(128, kP, 0, 1);
             constexpr uint32_t id_v = tc::idesc_bf16_f32(128, kP, 0, 1);
             const uint32_t aB = tc::smem_u32(sB), aC = tc::smem_u32(sC), aX = tc::smem_u32(sX);
-            const uint32_t aXw = tc::smem_u32(sXw), aP = tc::smem_u32(sP), aH = tc::smem_u32(sH);
+            const uint32_t aXw = tc::smem_u32(sXw), aH = tc::smem_u32(sH);
             uint32_t hc = 0, xc = 0, itc = 0;
             bool ok = true;
             auto issue_v = [&](uint32_t head) -> bool {
@@ -313,22 +316,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t st = xc % kStages;
                     if (MODE == kFused) {
                         // block state Z = B^T (w o X): M = n (MN-major B tile), N = p, K = s.
-                        // Its buffer is free once group B's state step of head hc-2 read it.
-                        ok = (hc < 2 || tc::mbar_wait(&bars->z_empty[buf], ((hc >> 1) - 1) & 1, abort_v)) &&
+                        // Its columns are free once group B's state step of the previous
+                        // head read them.
+                        ok = (hc < 1 || tc::mbar_wait(&bars->z_empty, (hc - 1) & 1, abort_v)) &&
                              tc::mbar_wait(&bars->xw_full, hc & 1, abort_v);
                         if (!ok) break;
                         tc::tc_fence_after();
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk)
-                            tc::mma_ss(tmem + col_z(buf), tc::smem_desc_sw128(aB + kk * 2048, kTile, 1024),
+                            tc::mma_ss(tmem + COL_Z, tc::smem_desc_sw128(aB + kk * 2048, kTile, 1024),
                                        tc::smem_desc_sw128(aXw + kk * 2048, kTile, 1024), id_z, kk > 0);
-                        tc::mma_commit(&bars->z_full[buf]);
+                        tc::mma_commit(&bars->z_full);
                         tc::mma_commit(&bars->xw_empty);
                     }
                     // V = C Hin of the previous head as soon as group B handed the state
                     // in (issued before Y, which waits for group A's operands)
                     if (i > 0 && !issue_v(hc - 1)) { ok = false; break; }
-                    // Y = P X: M = t, N = p, K = s (P K-major, X MN-major).  Y and V of this
+                    // Y = P X: M = t, N = p, K = s (P from TMEM, X MN-major).  Y and V of this
                     // buffer are free once group B's output of head hc-2 read them.
                     ok = (hc < 2 || tc::mbar_wait(&bars->yv_empty[buf], ((hc >> 1) - 1) & 1, abort_v)) &&
                          tc::mbar_wait(&bars->p_full, hc & 1, abort_v) &&
@@ -337,9 +341,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc::tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
-                        const uint64_t ad = tc::smem_desc_sw128(aP + (kk >> 2) * kTile + (kk & 3) * 32, 16, 1024);
+                        // 16 K values of P = 8 TMEM columns
                         const uint64_t bd = tc::smem_desc_sw128(aX + st * kTile + kk * 2048, kTile, 1024);
-                        tc::mma_ss(tmem + col_y(buf), ad, bd, id_y, kk > 0);
+                        tc::mma_ts(tmem + col_y(buf), tmem + COL_P + kk * 8, bd, id_y, kk > 0);
                     }
                     tc::mma_commit(&bars->y_full[buf]);
                     tc::mma_commit(&bars->p_empty);
@@ -417,12 +421,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const bool publish = !(p.test_stall && chain == 0 && w.j == 0);
                     if (publish) {
                         const int r0 = (chain * 2 + (w.j & 1)) * kN;
-                        tc::tma_store_2d(&tm_st, sHin, 0, r0);
-                        tc::tma_store_2d(&tm_st, sHin + kTile, 32, r0);
+                        tc::tma_store_2d(&tm_st, sHout, 0, r0);
+                        tc::tma_store_2d(&tm_st, sHout + kTile, 32, r0);
                         tc::bulk_commit();
                         tc::bulk_wait_read<0>();
                     }
-                    tc::mbar_arrive(&bars->hin_free);
+                    tc::mbar_arrive(&bars->hout_free);
                     if (publish) {
                         tc::bulk_wait<0>();
                         tc::fence_proxy_async_global();
@@ -550,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tc::mbar_arrive(&bars->x_empty[st]);
                         }
                     }
-                    // ---- T3: P = S o L + D I -> bf16, K-major in sP
+                    // ---- T3: P = S o L + D I -> bf16, into TMEM as the A operand of Y = P X
                     ok = (i > 0 || tc::mbar_wait(&bars->s_full, itc & 1, abort_v)) &&
                          (hc == 0 || tc::mbar_wait(&bars->p_empty, (hc - 1) & 1, abort_v));
                     if (!sync_ok(ok)) { alive = false; break; }
@@ -565,7 +569,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float* colf = sColf + (quad > 0 ? (quad - 1) * kBlk : 0);
                         // this warp's 64 columns, 16 at a time (a rolled loop keeps the
                         // code small: 20 warps share the instruction cache)
-                        uint8_t* ptile = sP + cg * kTile;
 #pragma unroll 1
                         for (int c16 = 0; c16 < 4; ++c16) {
                             const int s0 = 64 * cg + 16 * c16;  // first column of the chunk
@@ -608,13 +611,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                                 for (int e = 0; e < 8; ++e) pk[e] = tc::pack_bf16x2(v[2 * e], v[2 * e + 1]);
                             }
-                            *reinterpret_cast<uint4*>(ptile + tc::sw128_offset(row, 2 * c16)) =
-                                make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                            *reinterpret_cast<uint4*>(ptile + tc::sw128_offset(row, 2 * c16 + 1)) =
-                                make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                            // row `row`, columns s0..s0+15 -> 8 TMEM columns (2 bf16 each)
+                            tc::tmem_st8(lane_base + COL_P + (s0 >> 1), pk);
                         }
                     }
-                    tc::fence_proxy_async_smem();
+                    tc::tmem_st_wait();
                     tc::tc_fence_before();
                     __syncwarp();
                     if (lane == 0) {
@@ -643,9 +644,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         // ---- T4: incoming state (and, fused, the block's own state out)
                         const int h = w.h0 + i;
                         const int chain = w.b * p.H + h;
-                        const int buf = hc & 1;
                         const float* cum = cumbuf + i * kBlk;
-                        ok = (MODE == kScan || tc::mbar_wait(&bars->z_full[buf], (hc >> 1) & 1, abort_v)) &&
+                        ok = (MODE == kScan || tc::mbar_wait(&bars->z_full, hc & 1, abort_v)) &&
+                             (MODE == kScan || hc == 0 || tc::mbar_wait(&bars->hout_free, (hc - 1) & 1, abort_v)) &&
                              (hc == 0 || tc::mbar_wait(&bars->h_empty, (hc - 1) & 1, abort_v)) &&
                              tc::mbar_wait(&bars->hin_full, hc & 1, abort_v);
                         if (!sync_ok(ok)) { alive = false; break; }
@@ -668,13 +669,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                             if (MODE == kFused) {
                                 float zv[16];
-                                tc::tmem_ld16(lane_base + col_z(buf) + 32 * cg + 16 * c, zv);
+                                tc::tmem_ld16(lane_base + COL_Z + 32 * cg + 16 * c, zv);
                                 tc::tmem_ld_wait();
 #pragma unroll
                                 for (int e = 0; e < 16; ++e) zv[e] = fmaf(eL, hin[e], zv[e]);  // h_j
 #pragma unroll
                                 for (int q = 0; q < 4; ++q)
-                                    *reinterpret_cast<float4*>(sHin + state_off(row, cg, 4 * c + q)) =
+                                    *reinterpret_cast<float4*>(sHout + state_off(row, cg, 4 * c + q)) =
                                         make_float4(zv[4 * q], zv[4 * q + 1], zv[4 * q + 2], zv[4 * q + 3]);
                                 if (last_blk && p.fin) {
                                     float4* fd = reinterpret_cast<float4*>(
@@ -695,15 +696,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 *reinterpret_cast<uint4*>(sH + tc::sw128_offset(row, 4 * cg + 2 * c + c8)) = v;
                             }
                         }
-                        // one proxy fence covers the state written back into sHin (read by
-                        // the publisher's TMA store) and the bf16 operand in sH (read by the MMA)
+                        // one proxy fence covers the outgoing state in sHout (read by the
+                        // publisher's TMA store) and the bf16 operand in sH (read by the MMA)
                         tc::fence_proxy_async_smem();
                         tc::tc_fence_before();
                         __syncwarp();
                         if (lane == 0) {
-                            tc::mbar_arrive(MODE == kFused ? &bars->hout_full : &bars->hin_free);
+                            tc::mbar_arrive(&bars->hin_free);
                             tc::mbar_arrive(&bars->h_full);
-                            if (MODE == kFused) tc::mbar_arrive(&bars->z_empty[buf]);
+                            if (MODE == kFused) {
+                                tc::mbar_arrive(&bars->hout_full);
+                                tc::mbar_arrive(&bars->z_empty);
+                            }
                         }
                         ++hc;
                     }
