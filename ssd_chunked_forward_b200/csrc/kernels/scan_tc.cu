@@ -70,6 +70,7 @@ struct __align__(8) Bars {
     uint64_t hin_full, hin_free, hout_full, hout_free;
     uint64_t cum_full[2], cum_free[2];
     uint64_t y_full[2], v_full[2], yv_empty[2], z_full, z_empty;
+    uint64_t done_y;
     uint64_t done;
 };
 
@@ -95,7 +96,8 @@ constexpr uint32_t OFF_HOUT = OFF_HIN + 2 * kTile; // fp32 outgoing state, same 
 constexpr uint32_t OFF_Y = OFF_HOUT + 2 * kTile;   // bf16 y staging for the TMA store
 constexpr uint32_t OFF_CUM = OFF_Y + kTile;
 constexpr uint32_t OFF_VEC = OFF_CUM + 2 * kHpbMax * kBlk * 4;
-constexpr uint32_t OFF_BAR = OFF_VEC + 5 * kBlk * 4;
+constexpr uint32_t OFF_DV = OFF_VEC + 5 * kBlk * 4;  // [2][kHpbMax] D of the item's heads
+constexpr uint32_t OFF_BAR = OFF_DV + 2 * kHpbMax * 4;
 constexpr uint32_t OFF_MISC = OFF_BAR + ((sizeof(Bars) + 15) / 16) * 16;
 constexpr size_t kSmemBytes = 1024 + OFF_MISC + 16;
 static_assert(kSmemBytes <= 232448, "shared memory above the 227 KB per-block limit");
@@ -168,6 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* sW = reinterpret_cast<float*>(sm + OFF_VEC);    // [128]
     float* sColf = sW + kBlk;                              // [3][128]
     float* sC2 = sColf + 3 * kBlk;                         // [128] cum * log2(e)
+    float* sDv = reinterpret_cast<float*>(sm + OFF_DV);    // [2][kHpbMax]
     Bars* bars = reinterpret_cast<Bars*>(sm + OFF_BAR);
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
     int* sAbort = reinterpret_cast<int*>(sm + OFF_MISC + 4);
@@ -207,6 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::mbar_init(&bars->yv_empty[s], 8);  // group B read Y and V (output)
         }
         tc::mbar_init(&bars->done, 1);
+        tc::mbar_init(&bars->done_y, 1);
         *sAbort = 0;
         tc::fence_mbar_init();
     }
@@ -228,7 +232,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // =============================================== TMA producers ====
         // lane 0 streams x (one tile per head); lane 1 loads each item's B and C
         // tiles once the previous item's products no longer read them.  Two
-        // threads, so that x never waits behind the B/C release.
+        // threads, so that x never waits behind the B/C release.  Lane 2 issues
+        // the Y products.
         if (lane == 0) {
             tc::prefetch_tmap(&tm_x);
             uint32_t xc = 0;
@@ -272,28 +277,67 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok) fail();
             if (itc > 0) tc::mbar_wait(&bars->bc_full, (itc - 1) & 1, nullptr, 200000000ull);
+        } else if (lane == 2) {
+            // ===================================== MMA issuer: Y = P X ====
+            // A thread of its own next to the one that issues S, Z and V: with
+            // all four products on one thread, issuing took most of each head's
+            // time and group B's state step waited on it.
+            constexpr uint32_t id_y = tc::idesc_bf16_f32(128, kP, 0, 1);
+            const uint64_t dX = tc::smem_desc_sw128(tc::smem_u32(sX), kTile, 1024);
+            uint32_t hc = 0;  // heads so far = x tiles so far
+            bool ok = true;
+            for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x) {
+                for (int i = 0; i < p.hpb; ++i, ++hc) {
+                    const int buf = hc & 1;
+                    const uint32_t st = hc % kStages;
+                    // M = t, N = p, K = s (P from TMEM, X MN-major).  Y's buffer is
+                    // free once group B's output of head hc-2 read it.
+                    ok = (hc < 2 || tc::mbar_wait(&bars->yv_empty[buf], ((hc >> 1) - 1) & 1, abort_v)) &&
+                         tc::mbar_wait(&bars->p_full, hc & 1, abort_v) &&
+                         tc::mbar_wait(&bars->x_full[st], (hc / kStages) & 1, abort_v);
+                    if (!ok) break;
+                    tc::tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)  // 16 K values of P = 8 TMEM columns
+                        tc::mma_ts(tmem + col_y(buf), tmem + COL_P + kk * 8,
+                                   tc::desc_adv(dX, st * kTile + kk * 2048), id_y, kk > 0);
+                    tc::mma_commit(&bars->y_full[buf]);
+                    tc::mma_commit(&bars->p_empty);
+                    tc::mma_commit(&bars->x_empty[st]);
+                }
+            }
+            if (!ok) fail();
+            tc::mma_commit(&bars->done_y);
+            tc::mbar_wait(&bars->done_y, 0, nullptr, 200000000ull);
         }
     } else if (warp == 1) {
-        // ================================================ MMA issuer ====
+        // ===================================== MMA issuer: S, Z and V ====
+        // (the products Y = P X are issued by warp 0, lane 2)
         if (lane == 0) {
             constexpr uint32_t id_s = tc::idesc_bf16_f32(128, 128, 0, 0);
             constexpr uint32_t id_z = tc::idesc_bf16_f32(128, kP, 1, 1);
-            constexpr uint32_t id_y = tc::idesc_bf16_f32(128, kP, 0, 1);
             constexpr uint32_t id_v = tc::idesc_bf16_f32(128, kP, 0, 1);
-            const uint32_t aB = tc::smem_u32(sB), aC = tc::smem_u32(sC), aX = tc::smem_u32(sX);
-            const uint32_t aXw = tc::smem_u32(sXw), aH = tc::smem_u32(sH);
-            uint32_t hc = 0, xc = 0, itc = 0;
+            // operand descriptors at their tile bases (K-major: 16-element K
+            // steps inside a 64-element block, blocks kTile apart; MN-major:
+            // 16-row K steps of 2048 bytes)
+            const uint64_t dC = tc::smem_desc_sw128(tc::smem_u32(sC), 16, 1024);
+            const uint64_t dBk = tc::smem_desc_sw128(tc::smem_u32(sB), 16, 1024);
+            const uint64_t dBm = tc::smem_desc_sw128(tc::smem_u32(sB), kTile, 1024);
+            const uint64_t dXw = tc::smem_desc_sw128(tc::smem_u32(sXw), kTile, 1024);
+            const uint64_t dH = tc::smem_desc_sw128(tc::smem_u32(sH), kTile, 1024);
+            uint32_t hc = 0, itc = 0;
             bool ok = true;
             auto issue_v = [&](uint32_t head) -> bool {
+                // V = C Hin: M = t, N = p, K = n.  Its buffer was read by group B's
+                // output of head-2, which B finished before the state step of
+                // `head` that h_full reports.
                 const int buf = head & 1;
                 if (!tc::mbar_wait(&bars->h_full, head & 1, abort_v)) return false;
                 tc::tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t ad = tc::smem_desc_sw128(aC + (kk >> 2) * kTile + (kk & 3) * 32, 16, 1024);
-                    const uint64_t bd = tc::smem_desc_sw128(aH + kk * 2048, kTile, 1024);
-                    tc::mma_ss(tmem + col_v(buf), ad, bd, id_v, kk > 0);
-                }
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_ss(tmem + col_v(buf), tc::desc_adv(dC, (kk >> 2) * kTile + (kk & 3) * 32),
+                               tc::desc_adv(dH, kk * 2048), id_v, kk > 0);
                 tc::mma_commit(&bars->v_full[buf]);
                 tc::mma_commit(&bars->h_empty);
                 return true;
@@ -307,13 +351,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * kTile + (kk & 3) * 32;
-                    tc::mma_ss(tmem + COL_S, tc::smem_desc_sw128(aC + off, 16, 1024),
-                               tc::smem_desc_sw128(aB + off, 16, 1024), id_s, kk > 0);
+                    tc::mma_ss(tmem + COL_S, tc::desc_adv(dC, off), tc::desc_adv(dBk, off), id_s, kk > 0);
                 }
                 tc::mma_commit(&bars->s_full);
-                for (int i = 0; i < p.hpb; ++i, ++hc, ++xc) {
-                    const int buf = hc & 1;
-                    const uint32_t st = xc % kStages;
+                for (int i = 0; i < p.hpb; ++i, ++hc) {
                     if (MODE == kFused) {
                         // block state Z = B^T (w o X): M = n (MN-major B tile), N = p, K = s.
                         // Its columns are free once group B's state step of the previous
@@ -324,30 +365,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc::tc_fence_after();
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk)
-                            tc::mma_ss(tmem + COL_Z, tc::smem_desc_sw128(aB + kk * 2048, kTile, 1024),
-                                       tc::smem_desc_sw128(aXw + kk * 2048, kTile, 1024), id_z, kk > 0);
+                            tc::mma_ss(tmem + COL_Z, tc::desc_adv(dBm, kk * 2048), tc::desc_adv(dXw, kk * 2048),
+                                       id_z, kk > 0);
                         tc::mma_commit(&bars->z_full);
                         tc::mma_commit(&bars->xw_empty);
                     }
-                    // V = C Hin of the previous head as soon as group B handed the state
-                    // in (issued before Y, which waits for group A's operands)
+                    // V of the previous head as soon as group B handed its state in
                     if (i > 0 && !issue_v(hc - 1)) { ok = false; break; }
-                    // Y = P X: M = t, N = p, K = s (P from TMEM, X MN-major).  Y and V of this
-                    // buffer are free once group B's output of head hc-2 read them.
-                    ok = (hc < 2 || tc::mbar_wait(&bars->yv_empty[buf], ((hc >> 1) - 1) & 1, abort_v)) &&
-                         tc::mbar_wait(&bars->p_full, hc & 1, abort_v) &&
-                         tc::mbar_wait(&bars->x_full[st], (xc / kStages) & 1, abort_v);
-                    if (!ok) break;
-                    tc::tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        // 16 K values of P = 8 TMEM columns
-                        const uint64_t bd = tc::smem_desc_sw128(aX + st * kTile + kk * 2048, kTile, 1024);
-                        tc::mma_ts(tmem + col_y(buf), tmem + COL_P + kk * 8, bd, id_y, kk > 0);
-                    }
-                    tc::mma_commit(&bars->y_full[buf]);
-                    tc::mma_commit(&bars->p_empty);
-                    tc::mma_commit(&bars->x_empty[st]);
                 }
                 if (!ok) break;
                 if (!issue_v(hc - 1)) { ok = false; break; }
@@ -389,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 }
                             }
                             __nanosleep(nap);
-                            if (nap < 1024) nap <<= 1;
+                            if (nap < 256) nap <<= 1;
                         }
                         if (!ok) break;
                         tc::fence_proxy_async_global();  // the acquire orders the TMA read
@@ -438,12 +462,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::bulk_wait<0>();
         }
     } else {
-        // ======================================= compute: two warpgroups ====
-        // Group A (warps 2-5) builds, per head, the decay vectors, the weighted
-        // copy of x and the masked score operand P; group B (warps 6-9) runs the
-        // state step and the output of the heads A has finished.  Each group has
-        // one warp per TMEM lane quadrant, so thread = tile row; the groups share
-        // no barrier and work on different heads at the same time.
+        // ===================================== compute: two groups of 8 warps ====
+        // Group A (warps 2-9) builds, per head, the decay vectors, the weighted
+        // copy of x and the masked score operand P; group B (warps 10-17) runs
+        // the state step and the output of the heads A has finished.  Each group
+        // has two warps per TMEM lane quadrant (thread = tile row, the two split
+        // the columns); the groups share no barrier and work on different heads
+        // at the same time.
         const bool groupA = warp < 10;
         const int gt = threadIdx.x - (groupA ? 64 : 320);  // 0..255 within the group
         const int cg = gt >> 7;           // column half of this warp (0/1)
@@ -471,9 +496,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             // ---------------------------------------------------- group A ----
             uint32_t hc = 0, xc = 0, itc = 0;
             float anext[kHpbMax];
+            float dnext = 0.f;
             auto load_decays = [&](int it) {
                 if (cg != 0 || it >= p.n_items) return;
                 const Item w = decode_item(it, p, B);
+                dnext = (p.D && gt < p.hpb) ? __ldg(p.D + w.h0 + gt) : 0.f;
                 if (MODE == kFused) {
                     const float* arow = p.a + (size_t)(w.b * p.T + w.j * kBlk + gt) * p.H + w.h0;
 #pragma unroll
@@ -496,6 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int i = 0; i < kHpbMax; ++i)
                         if (i < p.hpb) cumbuf[i * kBlk + gt] = anext[i];
+                    if (gt < kHpbMax) sDv[(itc & 1) * kHpbMax + gt] = dnext;
                 }
                 load_decays(it + gridDim.x);
                 group_sync();
@@ -514,7 +542,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
                 bool ok = true;
                 for (int i = 0; i < p.hpb; ++i, ++hc, ++xc) {
-                    const int h = w.h0 + i;
                     const uint32_t st = xc % kStages;
                     const float* cum = cumbuf + i * kBlk;
                     // ---- T1: decay vectors of this head (thread = token row).  The
@@ -534,17 +561,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                              (hc == 0 || tc::mbar_wait(&bars->xw_empty, (hc - 1) & 1, abort_v));
                         if (!sync_ok(ok)) { alive = false; break; }
                         const uint8_t* xs = sX + st * kTile;
-#pragma unroll 1
+#pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             const int c = gt + 256 * q;
                             const float wgt = sW[c >> 3];
+                            const uint32_t w2 = tc::pack_bf16x2(wgt, wgt);
                             uint4 v = *reinterpret_cast<const uint4*>(xs + c * 16);
-                            uint32_t* u = reinterpret_cast<uint32_t*>(&v);
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const float2 f = tc::unpack_bf16x2(u[e]);
-                                u[e] = tc::pack_bf16x2(f.x * wgt, f.y * wgt);
-                            }
+                            v.x = tc::mul_bf16x2(v.x, w2);
+                            v.y = tc::mul_bf16x2(v.y, w2);
+                            v.z = tc::mul_bf16x2(v.z, w2);
+                            v.w = tc::mul_bf16x2(v.w, w2);
                             *reinterpret_cast<uint4*>(sXw + c * 16) = v;
                         }
                         tc::fence_proxy_async_smem();
@@ -563,56 +589,59 @@ __global__ void __launch_bounds__(kThreads, 1)
                         // Row `row` (quad `quad`), 32-column sub-blocks sb of s: sb < quad
                         // below the diagonal, the mask factorises as rowf * colf[s];
                         // sb == quad: explicit exp2 per element; sb > quad: masked out.
-                        const float dv = p.D ? __ldg(p.D + h) : 0.f;
+                        const float dv = sDv[(itc & 1) * kHpbMax + i];
                         const float r2 = sC2[row];
                         const float rowf = quad > 0 ? ex2_approx(r2 - sC2[32 * quad - 1]) : 0.f;
                         const float* colf = sColf + (quad > 0 ? (quad - 1) * kBlk : 0);
-                        // this warp's 64 columns, 16 at a time (a rolled loop keeps the
-                        // code small: 20 warps share the instruction cache)
+                        // this warp's 64 columns as two 32-column sub-blocks sb (one TMEM
+                        // load each; a rolled loop keeps the code small: 20 warps share
+                        // the instruction cache)
 #pragma unroll 1
-                        for (int c16 = 0; c16 < 4; ++c16) {
-                            const int s0 = 64 * cg + 16 * c16;  // first column of the chunk
-                            const int sb = s0 >> 5;             // its 32-column sub-block
-                            uint32_t pk[8];
+                        for (int k = 0; k < 2; ++k) {
+                            const int sb = 2 * cg + k;
+                            const int s0 = 32 * sb;  // first column of the sub-block
+                            uint32_t pk[16];
                             if (sb > quad) {
+                                // above the diagonal P is zero for every head: written
+                                // once, never overwritten
+                                if (hc != 0) continue;
 #pragma unroll
-                                for (int e = 0; e < 8; ++e) pk[e] = 0u;
+                                for (int e = 0; e < 16; ++e) pk[e] = 0u;
                             } else {
-                                float v[16];
-                                tc::tmem_ld16(lane_base + COL_S + s0, v);
+                                float v[32];
+                                tc::tmem_ld32(lane_base + COL_S + s0, v);
                                 tc::tmem_ld_wait();
                                 if (sb < quad) {
                                     const float4* cf = reinterpret_cast<const float4*>(colf + s0);
+                                    const float2 rr = make_float2(rowf, rowf);
+                                    float2* v2 = reinterpret_cast<float2*>(v);
 #pragma unroll
-                                    for (int e4 = 0; e4 < 4; ++e4) {
+                                    for (int e4 = 0; e4 < 8; ++e4) {
                                         const float4 f = cf[e4];
-                                        v[4 * e4 + 0] *= rowf * f.x;
-                                        v[4 * e4 + 1] *= rowf * f.y;
-                                        v[4 * e4 + 2] *= rowf * f.z;
-                                        v[4 * e4 + 3] *= rowf * f.w;
+                                        v2[2 * e4] = tc::mul2(v2[2 * e4], tc::mul2(rr, make_float2(f.x, f.y)));
+                                        v2[2 * e4 + 1] = tc::mul2(v2[2 * e4 + 1], tc::mul2(rr, make_float2(f.z, f.w)));
                                     }
                                 } else {
                                     const float4* c2 = reinterpret_cast<const float4*>(sC2 + s0);
-                                    float m[16];
+                                    const int rl = row - s0;  // the diagonal's column in the sub-block
 #pragma unroll
-                                    for (int e4 = 0; e4 < 4; ++e4) {
+                                    for (int e4 = 0; e4 < 8; ++e4) {
                                         const float4 f = c2[e4];
-                                        m[4 * e4 + 0] = f.x; m[4 * e4 + 1] = f.y;
-                                        m[4 * e4 + 2] = f.z; m[4 * e4 + 3] = f.w;
-                                    }
-                                    const int rl = row - s0;  // the diagonal's column in the chunk
+                                        const float m[4] = {f.x, f.y, f.z, f.w};
 #pragma unroll
-                                    for (int e = 0; e < 16; ++e) {
-                                        // exponent <= 0 where used; masked lanes get a finite dummy
-                                        const float ex = ex2_approx(e < rl ? r2 - m[e] : 0.f);
-                                        v[e] = e < rl ? v[e] * ex : (e == rl ? v[e] + dv : 0.f);
+                                        for (int q = 0; q < 4; ++q) {
+                                            const int e = 4 * e4 + q;
+                                            // exponent <= 0 where used; masked lanes get a finite dummy
+                                            const float ex = ex2_approx(e < rl ? r2 - m[q] : 0.f);
+                                            v[e] = e < rl ? v[e] * ex : (e == rl ? v[e] + dv : 0.f);
+                                        }
                                     }
                                 }
 #pragma unroll
-                                for (int e = 0; e < 8; ++e) pk[e] = tc::pack_bf16x2(v[2 * e], v[2 * e + 1]);
+                                for (int e = 0; e < 16; ++e) pk[e] = tc::pack_bf16x2(v[2 * e], v[2 * e + 1]);
                             }
-                            // row `row`, columns s0..s0+15 -> 8 TMEM columns (2 bf16 each)
-                            tc::tmem_st8(lane_base + COL_P + (s0 >> 1), pk);
+                            // row `row`, columns s0..s0+31 -> 16 TMEM columns (2 bf16 each)
+                            tc::tmem_st16(lane_base + COL_P + (s0 >> 1), pk);
                         }
                     }
                     tc::tmem_st_wait();
@@ -671,8 +700,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 float zv[16];
                                 tc::tmem_ld16(lane_base + COL_Z + 32 * cg + 16 * c, zv);
                                 tc::tmem_ld_wait();
+                                {
+                                    const float2 e2 = make_float2(eL, eL);
+                                    float2* z2 = reinterpret_cast<float2*>(zv);
+                                    const float2* h2 = reinterpret_cast<const float2*>(hin);
 #pragma unroll
-                                for (int e = 0; e < 16; ++e) zv[e] = fmaf(eL, hin[e], zv[e]);  // h_j
+                                    for (int e = 0; e < 8; ++e) z2[e] = tc::fma2(e2, h2[e], z2[e]);  // h_j
+                                }
 #pragma unroll
                                 for (int q = 0; q < 4; ++q)
                                     *reinterpret_cast<float4*>(sHout + state_off(row, cg, 4 * c + q)) =
@@ -734,8 +768,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                                 for (int e = 0; e < 4; ++e) {
                                     const int k0 = 8 * c8 + 2 * e;
-                                    o[e] = tc::pack_bf16x2(fmaf(ecum, vv[k0], yv[k0]),
-                                                           fmaf(ecum, vv[k0 + 1], yv[k0 + 1]));
+                                    const float2 r = tc::fma2(make_float2(ecum, ecum), make_float2(vv[k0], vv[k0 + 1]),
+                                                              make_float2(yv[k0], yv[k0 + 1]));
+                                    o[e] = tc::pack_bf16x2(r.x, r.y);
                                 }
                                 *reinterpret_cast<uint4*>(sY + tc::sw128_offset(row, 4 * cg + 2 * c + c8)) =
                                     make_uint4(o[0], o[1], o[2], o[3]);
