@@ -180,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         tc::mbar_init(&bars->bc_full, 1);
-        tc::mbar_init(&bars->bc_empty, 1);
+        tc::mbar_init(&bars->bc_empty, 2);  // both MMA issuers are done with B and C
         tc::mbar_init(&bars->s_full, 1);
         tc::mbar_init(&bars->s_empty, 8);
         for (int s = 0; s < kStages; ++s) {
@@ -278,54 +278,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) fail();
             if (itc > 0) tc::mbar_wait(&bars->bc_full, (itc - 1) & 1, nullptr, 200000000ull);
         } else if (lane == 2) {
-            // ===================================== MMA issuer: Y = P X ====
-            // A thread of its own next to the one that issues S, Z and V: with
-            // all four products on one thread, issuing took most of each head's
-            // time and group B's state step waited on it.
+            // ============================== MMA issuer: V = C Hin and Y = P X ====
+            // A thread of its own next to the one that issues S and Z: issuing
+            // eight N = 64 products takes several hundred cycles, and group B's
+            // state step needs V of the previous head and Z of its own, which
+            // are now issued side by side.
             constexpr uint32_t id_y = tc::idesc_bf16_f32(128, kP, 0, 1);
-            const uint64_t dX = tc::smem_desc_sw128(tc::smem_u32(sX), kTile, 1024);
-            uint32_t hc = 0;  // heads so far = x tiles so far
-            bool ok = true;
-            for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x) {
-                for (int i = 0; i < p.hpb; ++i, ++hc) {
-                    const int buf = hc & 1;
-                    const uint32_t st = hc % kStages;
-                    // M = t, N = p, K = s (P from TMEM, X MN-major).  Y's buffer is
-                    // free once group B's output of head hc-2 read it.
-                    ok = (hc < 2 || tc::mbar_wait(&bars->yv_empty[buf], ((hc >> 1) - 1) & 1, abort_v)) &&
-                         tc::mbar_wait(&bars->p_full, hc & 1, abort_v) &&
-                         tc::mbar_wait(&bars->x_full[st], (hc / kStages) & 1, abort_v);
-                    if (!ok) break;
-                    tc::tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)  // 16 K values of P = 8 TMEM columns
-                        tc::mma_ts(tmem + col_y(buf), tmem + COL_P + kk * 8,
-                                   tc::desc_adv(dX, st * kTile + kk * 2048), id_y, kk > 0);
-                    tc::mma_commit(&bars->y_full[buf]);
-                    tc::mma_commit(&bars->p_empty);
-                    tc::mma_commit(&bars->x_empty[st]);
-                }
-            }
-            if (!ok) fail();
-            tc::mma_commit(&bars->done_y);
-            tc::mbar_wait(&bars->done_y, 0, nullptr, 200000000ull);
-        }
-    } else if (warp == 1) {
-        // ===================================== MMA issuer: S, Z and V ====
-        // (the products Y = P X are issued by warp 0, lane 2)
-        if (lane == 0) {
-            constexpr uint32_t id_s = tc::idesc_bf16_f32(128, 128, 0, 0);
-            constexpr uint32_t id_z = tc::idesc_bf16_f32(128, kP, 1, 1);
             constexpr uint32_t id_v = tc::idesc_bf16_f32(128, kP, 0, 1);
-            // operand descriptors at their tile bases (K-major: 16-element K
-            // steps inside a 64-element block, blocks kTile apart; MN-major:
-            // 16-row K steps of 2048 bytes)
+            const uint64_t dX = tc::smem_desc_sw128(tc::smem_u32(sX), kTile, 1024);
             const uint64_t dC = tc::smem_desc_sw128(tc::smem_u32(sC), 16, 1024);
-            const uint64_t dBk = tc::smem_desc_sw128(tc::smem_u32(sB), 16, 1024);
-            const uint64_t dBm = tc::smem_desc_sw128(tc::smem_u32(sB), kTile, 1024);
-            const uint64_t dXw = tc::smem_desc_sw128(tc::smem_u32(sXw), kTile, 1024);
             const uint64_t dH = tc::smem_desc_sw128(tc::smem_u32(sH), kTile, 1024);
-            uint32_t hc = 0, itc = 0;
+            uint32_t hc = 0;  // heads so far = x tiles so far
             bool ok = true;
             auto issue_v = [&](uint32_t head) -> bool {
                 // V = C Hin: M = t, N = p, K = n.  Its buffer was read by group B's
@@ -342,6 +305,50 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc::mma_commit(&bars->h_empty);
                 return true;
             };
+            for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x) {
+                for (int i = 0; i < p.hpb; ++i, ++hc) {
+                    const int buf = hc & 1;
+                    // V of the previous head as soon as group B handed its state in
+                    if (i > 0 && !issue_v(hc - 1)) { ok = false; break; }
+                    const uint32_t st = hc % kStages;
+                    // M = t, N = p, K = s (P from TMEM, X MN-major).  Y's buffer is
+                    // free once group B's output of head hc-2 read it.
+                    ok = (hc < 2 || tc::mbar_wait(&bars->yv_empty[buf], ((hc >> 1) - 1) & 1, abort_v)) &&
+                         tc::mbar_wait(&bars->p_full, hc & 1, abort_v) &&
+                         tc::mbar_wait(&bars->x_full[st], (hc / kStages) & 1, abort_v);
+                    if (!ok) break;
+                    tc::tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)  // 16 K values of P = 8 TMEM columns
+                        tc::mma_ts(tmem + col_y(buf), tmem + COL_P + kk * 8,
+                                   tc::desc_adv(dX, st * kTile + kk * 2048), id_y, kk > 0);
+                    tc::mma_commit(&bars->y_full[buf]);
+                    tc::mma_commit(&bars->p_empty);
+                    tc::mma_commit(&bars->x_empty[st]);
+                }
+                if (!ok) break;
+                if (!issue_v(hc - 1)) { ok = false; break; }
+                tc::mma_commit(&bars->bc_empty);  // this item's V products read C
+            }
+            if (!ok) fail();
+            tc::mma_commit(&bars->done_y);
+            tc::mbar_wait(&bars->done_y, 0, nullptr, 200000000ull);
+        }
+    } else if (warp == 1) {
+        // ========================================= MMA issuer: S and Z ====
+        // (V and Y are issued by warp 0, lane 2)
+        if (lane == 0) {
+            constexpr uint32_t id_s = tc::idesc_bf16_f32(128, 128, 0, 0);
+            constexpr uint32_t id_z = tc::idesc_bf16_f32(128, kP, 1, 1);
+            // operand descriptors at their tile bases (K-major: 16-element K
+            // steps inside a 64-element block, blocks kTile apart; MN-major:
+            // 16-row K steps of 2048 bytes)
+            const uint64_t dC = tc::smem_desc_sw128(tc::smem_u32(sC), 16, 1024);
+            const uint64_t dBk = tc::smem_desc_sw128(tc::smem_u32(sB), 16, 1024);
+            const uint64_t dBm = tc::smem_desc_sw128(tc::smem_u32(sB), kTile, 1024);
+            const uint64_t dXw = tc::smem_desc_sw128(tc::smem_u32(sXw), kTile, 1024);
+            uint32_t hc = 0, itc = 0;
+            bool ok = true;
             for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x, ++itc) {
                 ok = tc::mbar_wait(&bars->bc_full, itc & 1, abort_v) &&
                      (itc == 0 || tc::mbar_wait(&bars->s_empty, (itc - 1) & 1, abort_v));
@@ -370,12 +377,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc::mma_commit(&bars->z_full);
                         tc::mma_commit(&bars->xw_empty);
                     }
-                    // V of the previous head as soon as group B handed its state in
-                    if (i > 0 && !issue_v(hc - 1)) { ok = false; break; }
                 }
                 if (!ok) break;
-                if (!issue_v(hc - 1)) { ok = false; break; }
-                tc::mma_commit(&bars->bc_empty);
+                tc::mma_commit(&bars->bc_empty);  // this item's S and Z products read B and C
             }
             if (!ok) fail();
             // every MMA issued must be complete before TMEM is released
