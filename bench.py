@@ -245,6 +245,30 @@ def run_reference(args, rank, world):
     return 0
 
 
+# ------------------------------------------------------------ multi-rank ----
+
+def rank_seed(w, rank: int) -> int:
+    """Seed of rank `rank`'s batch: every rank runs its own independent batch
+    of the same workload (weak scaling)."""
+    return w.seed + 1000 * rank
+
+
+def max_over_ranks(value: float, dist=None, device="cpu") -> float:
+    """The slowest rank's figure; every rank takes part (identity without a
+    process group)."""
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(tokens_per_rank: int, world: int, ms: float) -> float:
+    """Tokens per second of the whole job: every rank's tokens over the
+    slowest rank's time per step."""
+    return tokens_per_rank * world / (ms / 1e3)
+
+
 # ---------------------------------------------------------------- GPU leg ----
 
 def step_kernels(w, path_used):
@@ -318,7 +342,7 @@ def main():
     w = WORKLOADS[args.workload]
     if args.B or args.T:
         w = w.scaled(B=args.B or w.B, T=args.T or w.T, name=w.name + f"_B{args.B or w.B}_T{args.T or w.T}")
-    inp = generate(w, seed=w.seed + 1000 * rank)  # each rank: its own batch
+    inp = generate(w, seed=rank_seed(w, rank))  # each rank: its own batch
     dev = {k: v.to(device) for k, v in inp.items()}
     shape = ssd.shape_of(dev["x"], dev["a"], dev["Bm"], w.chunk)
     path = PATHS[args.path]
@@ -367,13 +391,8 @@ def main():
     if code != ssd.SSD_OK:
         raise SystemExit(f"device status after timing: {ssd.status_string(code)}")
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    ms = sum(step_ms) / len(step_ms)
-    if dist:
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    tokens_all = w.tokens * world
-    value = tokens_all / (ms / 1e3)
+    ms = max_over_ranks(sum(step_ms) / len(step_ms), dist, device)
+    value = whole_job_rate(w.tokens, world, ms)
 
     # ---- dominant kernel: per-kernel split with events --------------------
     peaks, peak_src = load_peaks()
@@ -418,14 +437,10 @@ def main():
             fwd_host()
         e1.record(st)
         torch.cuda.synchronize()
-        e_ms = e0.elapsed_time(e1) / e2e_steps
-        if dist:
-            t = torch.tensor([e_ms], device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dist, device)
         h2d = sum(v.numel() * v.element_size() for v in inp.values())
         d2h = y_h.numel() * y_h.element_size() + f_h.numel() * 4
-        e2e = {"value": tokens_all / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        e2e = {"value": whole_job_rate(w.tokens, world, e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e_ms, "steps": e2e_steps,
                "api": "ssd_forward_host (pinned host buffers)"}
         del buf
