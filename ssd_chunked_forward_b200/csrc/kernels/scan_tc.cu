@@ -13,8 +13,12 @@
 //                                        the skip term D x_t rides on the diagonal)
 //   V   = C Hin                         (incoming state, item 5)
 //   y_t = Y_t + exp(cum_t) V_t
-// The mask L is applied in registers between the TMEM scores and the bf16
-// operand in shared memory; it never reaches HBM.
+// The mask L is applied in registers between the fp32 scores in TMEM and the
+// bf16 operand P, which goes back to TMEM as the A operand of Y = P X; it never
+// reaches shared memory or HBM.  The in-block mask uses 32-token sub-blocks:
+// below the diagonal sub-block L factorises as exp(cum_t - cum_e) exp(cum_e -
+// cum_s) with e the last token before row t's sub-block (both factors <= 1);
+// on it, exp2 runs per element.
 //
 // Fused mode also forms the block's own state Z = B^T (w o X),
 // w_s = exp(cum_127 - cum_s) (item 3), and the recurrence
@@ -33,15 +37,16 @@
 // at the block boundary ("State Space Duality", "Two algorithms for one
 // operator": off-diagonal blocks are low-rank).
 //
-// Warp roles (640 threads): 0 TMA producer; 1 MMA issuer and TMEM owner;
-// 2-9 group A (decay vectors, weighted x, masked scores P); 10-17 group B
-// (state step, output); 18 state loader; 19 state publisher (fused).  Each
-// group has two warps per TMEM lane quadrant (thread = tile row, the two
-// warps splitting the columns), and the two groups work on different heads
-// at the same time.
-// TMEM (512 columns): scores 0-127, then two buffers of {Z, Y, V} x 64
-// columns, alternating per head; Z is released after the state step, Y and V
-// after the output, so the next block state can start before the output.
+// Warp roles (640 threads): warp 0 lane 0 streams x, lane 1 loads B and C,
+// lane 2 issues V and Y; warp 1 issues S and Z and owns TMEM; 2-9 group A
+// (decay vectors, weighted x, masked scores P); 10-17 group B (state step,
+// output); 18 state loader; 19 state publisher (fused).  Each group has two
+// warps per TMEM lane quadrant (thread = tile row, the two warps splitting
+// the columns), and the two groups work on different heads at the same time.
+// TMEM (512 columns): scores S 0-127, P 128-191 (bf16 pairs), Z 192-255, then
+// Y and V for two heads (256 + 128 * (head & 1), + 64 for V).  Shared memory
+// holds the incoming and the outgoing fp32 state separately, so the loader
+// fetches the next head's state while the publisher still stores this one.
 #include <stdlib.h>
 
 #include "../common.cuh"
