@@ -350,7 +350,7 @@ def main():
         raise SystemExit(f"path {args.path} does not serve workload {w.name}")
     path_used = args.path
     if path == ssd.PATH_AUTO:
-        path_used = "fused" if ssd.path_supported(shape, ssd.PATH_FUSED) else "modular"
+        path_used = "fused" if ssd.auto_path(shape) == ssd.PATH_FUSED else "modular"
     ws = ssd.alloc_workspace(shape, device)
     y = torch.empty_like(dev["x"])
     fin = torch.empty((w.B, w.H, w.N, w.P), dtype=torch.float32, device=device)

@@ -98,6 +98,18 @@ size_t ssd_workspace_size(const ssd_shape* shape);
 /* 1 if `path` (SSD_PATH_*) serves this shape on this build, else 0. */
 int ssd_path_supported(const ssd_shape* shape, unsigned path);
 
+/* The path SSD_PATH_AUTO runs for this shape (SSD_PATH_FUSED or
+ * SSD_PATH_MODULAR), or -1 for an invalid shape.  The fused kernel hands each
+ * (batch, head) chain's state from one 128-token block to the next, so its
+ * time is bounded below by the chain length times that hand-off (about 4 us
+ * per block measured on B200); the modular path pays about 2.6x the fused
+ * path's memory traffic but runs all blocks of a chain at once.  With fewer
+ * than 76 chains (batch x heads) the chain bound exceeds the modular path's
+ * cost at any sequence length, so AUTO takes the modular path there.  This
+ * choice has no counterpart on the pages; it only picks between two exact
+ * evaluations of the same forward. */
+int ssd_auto_path(const ssd_shape* shape);
+
 /* The whole forward: y (and final_state when non-NULL) from x, a, Bm, Cm, D.
  * `workspace` (device, >= ssd_workspace_size bytes, 256-byte aligned) is
  * scratch owned by the caller and must not be shared by calls that overlap

@@ -150,6 +150,17 @@ int ssd_path_supported(const ssd_shape* shape, unsigned path) {
     }
 }
 
+int ssd_auto_path(const ssd_shape* shape) {
+    if (check_shape(shape) != SSD_OK) return -1;
+    const Dims d = dims_of(shape);
+    // fewer chains than this: the fused kernel's per-block hand-off (~4 us on
+    // B200) times the chain length exceeds the modular path's cost (~53 ns per
+    // head-block, i.e. chains x 53 ns per block)
+    constexpr long long kFusedMinChains = 76;
+    if (ssd::fused_supported(d) && (long long)d.B * d.H >= kFusedMinChains) return SSD_PATH_FUSED;
+    return SSD_PATH_MODULAR;
+}
+
 ssd_status ssd_forward_path(const ssd_shape* shape, const void* x, const float* a, const void* Bm,
                             const void* Cm, const float* D, void* y, float* final_state,
                             void* workspace, size_t ws_bytes, ssd_stream stream, unsigned path,
@@ -171,7 +182,7 @@ ssd_status ssd_forward_path(const ssd_shape* shape, const void* x, const float* 
     // status word and per-chain counters start at zero on every call
     if (cudaMemsetAsync(w.ctrl, 0, kCtrlBytes + flags_bytes(d), cs) != cudaSuccess)
         return SSD_ERR_CUDA;
-    if (path == SSD_PATH_AUTO) path = ssd::fused_supported(d) ? SSD_PATH_FUSED : SSD_PATH_MODULAR;
+    if (path == SSD_PATH_AUTO) path = (unsigned)ssd_auto_path(shape);
     switch (path) {
         case SSD_PATH_SIMT:
             return run_modular(d, x, a, Bm, Cm, D, y, final_state, w, cs, false);

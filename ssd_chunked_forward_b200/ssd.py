@@ -25,7 +25,7 @@ EXPORTS = [
     "ssd_status_string", "ssd_workspace_size", "ssd_path_supported", "ssd_forward",
     "ssd_forward_path", "ssd_device_status", "ssd_chunk_cumsum", "ssd_chunk_state",
     "ssd_state_pass", "ssd_chunk_scan", "ssd_diag_scan", "ssd_forward_host_bytes",
-    "ssd_forward_host", "ssd_forward_noalloc",
+    "ssd_forward_host", "ssd_forward_noalloc", "ssd_auto_path",
 ]
 
 
@@ -61,6 +61,8 @@ def load(path: str = LIB_PATH):
     lib.ssd_workspace_size.restype = sz
     lib.ssd_path_supported.argtypes = [sp, ctypes.c_uint]
     lib.ssd_path_supported.restype = ctypes.c_int
+    lib.ssd_auto_path.argtypes = [sp]
+    lib.ssd_auto_path.restype = ctypes.c_int
     lib.ssd_forward.argtypes = [sp, vp, fp, vp, vp, fp, vp, fp, vp, sz, vp]
     lib.ssd_forward_path.argtypes = [sp, vp, fp, vp, vp, fp, vp, fp, vp, sz, vp, ctypes.c_uint, ctypes.c_uint]
     lib.ssd_device_status.argtypes = [vp, vp]
@@ -123,6 +125,11 @@ def workspace_size(shape: Shape) -> int:
 
 def path_supported(shape: Shape, path: int) -> bool:
     return bool(load().ssd_path_supported(ctypes.byref(shape), int(path)))
+
+
+def auto_path(shape: Shape) -> int:
+    """The path SSD_PATH_AUTO takes for this shape (PATH_FUSED or PATH_MODULAR)."""
+    return int(load().ssd_auto_path(ctypes.byref(shape)))
 
 
 def alloc_workspace(shape: Shape, device=None) -> torch.Tensor:

@@ -125,3 +125,17 @@ def test_host_entry_point_validates(lib):
     assert f(None, ok, ok, ok, None, ok, None, ok, need, None) == ssd.SSD_ERR_INVALID_ARG
     assert f(ok, ok, ok, ok, None, ok, None, ok, need - 1, None) == ssd.SSD_ERR_WORKSPACE
     assert f(ok, ok, ok, ok, None, ok, None, ok + 16, need, None) == ssd.SSD_ERR_WORKSPACE
+
+
+def test_auto_path_choice(lib):
+    """AUTO takes the fused kernel for the Mamba-2 shapes with enough (batch,
+    head) chains and the modular path for few long chains, fp32 and the
+    per-state variant; an invalid shape gives -1."""
+    fused = ssd.make_shape(4, 8192, 80, 64, 1, 128, 256)            # 320 chains
+    assert ssd.auto_path(fused) == ssd.PATH_FUSED
+    assert ssd.auto_path(ssd.make_shape(8, 2048, 24, 64, 1, 128, 256)) == ssd.PATH_FUSED   # 192
+    assert ssd.auto_path(ssd.make_shape(1, 8192, 80, 64, 1, 128, 256)) == ssd.PATH_FUSED   # 80
+    assert ssd.auto_path(ssd.make_shape(1, 262144, 32, 64, 8, 128, 256)) == ssd.PATH_MODULAR  # 32
+    assert ssd.auto_path(ssd.make_shape(4, 8192, 80, 64, 1, 128, 256, dtype="f32")) == ssd.PATH_MODULAR
+    assert ssd.auto_path(ssd.make_shape(4, 4096, 16, 64, 1, 64, 128, a_per_state=True)) == ssd.PATH_MODULAR
+    assert ssd.auto_path(ssd.make_shape(1, 100, 2, 64, 1, 128, 64)) == -1  # T % chunk != 0
