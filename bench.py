@@ -277,9 +277,22 @@ def step_kernels(w, path_used):
     return ["chunk_cumsum", "chunk_state", "state_pass", "diag_scan" if w.a_per_state else "chunk_scan"]
 
 
-def time_steps_split(w, dev, shape, ws, flush, reps, impl):
+def step_workload(w, impl):
+    """The shape the modular path's steps run on: where the tensor-core kernels
+    serve the workload and the chunk is a multiple of 128, the library runs
+    the steps on 128-token blocks (the same result up to rounding)."""
+    if (impl != ssd.IMPL_SIMT and w.dtype == "bf16" and not w.a_per_state and w.N == 128
+            and w.P == 64 and w.chunk % 128 == 0 and w.chunk > 128):
+        return w.scaled(chunk=128)
+    return w
+
+
+def time_steps_split(w, dev, flush, reps, impl):
     """Per-kernel device times (ms) of the modular path, by calling the step
-    entry points one by one with events between them on one stream."""
+    entry points one by one with events between them on one stream, on the
+    shape the library's modular path uses (step_workload)."""
+    w = step_workload(w, impl)
+    shape = ssd.shape_of(dev["x"], dev["a"], dev["Bm"], w.chunk)
     st = torch.cuda.current_stream()
     nc = w.T // w.chunk
     cum_t = torch.empty(w.B * w.H * nc * w.chunk * (w.N if w.a_per_state else 1),
@@ -402,10 +415,11 @@ def main():
         split = {"fused": ms}
     else:
         impl = ssd.IMPL_SIMT if path_used == "simt" else ssd.IMPL_AUTO
-        split = time_steps_split(w, dev, shape, ws, flush, 11, impl)
+        split = time_steps_split(w, dev, flush, 11, impl)
     dom = max(split, key=split.get)
     dom_ms = split[dom]
-    dom_bytes = kernel_bytes(w, dom)
+    dom_bytes = kernel_bytes(w if path_used == "fused" else
+                             step_workload(w, ssd.IMPL_SIMT if path_used == "simt" else ssd.IMPL_AUTO), dom)
     achieved = dom_bytes / (dom_ms / 1e3) / 1e9
     kernel_name = {"fused": "ssd_fused_kernel"}.get(dom, "ssd_" + dom)
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",

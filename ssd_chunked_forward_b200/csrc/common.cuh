@@ -19,6 +19,14 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(v);
 }
 
+// 2^x on the special-function unit (the hardware instruction, ~2^-22
+// relative error; denormal results flush to zero)
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ float warp_inclusive_scan(float v) {
     const int lane = threadIdx.x & 31;
 #pragma unroll

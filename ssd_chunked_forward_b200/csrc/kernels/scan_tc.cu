@@ -123,13 +123,6 @@ __device__ __forceinline__ void st_release_u32(unsigned* p, unsigned v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// 2^x on the special-function unit (the hardware instruction, ~2^-22
-// relative error, ample for bf16 operands)
-__device__ __forceinline__ float ex2_approx(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct Item {

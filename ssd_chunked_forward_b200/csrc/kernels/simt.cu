@@ -344,14 +344,164 @@ __global__ void __launch_bounds__(256) chunk_scan_simt_kernel(
     }
 }
 
+// ============================================================== step 5 ====
+// Output of one chunk for the per-state decay, a 32-row by 64-column tile per
+// block, with the mask factorised per 32-token sub-block.  For rows i of the
+// tile (first row i0) and a column sub-block j < i0, with e = i0 - 1 the last
+// token before the tile,
+//   exp(cum_i[n] - cum_j[n]) = exp(cum_i[n] - cum_e[n]) * exp(cum_e[n] - cum_j[n]),
+// both factors <= 1 (a <= 0, j <= e < i), so
+//   S[i,j] = sum_n C~_i[n] B~_j[n],  C~_i = C_i exp(cum_i - cum_e),  B~_j = B_j exp(cum_e - cum_j)
+// is a plain contraction and only the diagonal sub-block takes one exp per
+// (i, j, n) term ("State Space Duality", "Two algorithms for one operator":
+// off-diagonal blocks go through the state at the block boundary, here one
+// per state index n as in the diagonal SSM of "On Structured State-Space
+// Duality", item (i)).  exp is 2^x on the special-function unit, with the
+// decays pre-scaled by log2(e).
+template <typename T>
+__global__ void __launch_bounds__(256) diag_scan_simt_kernel(
+    const T* __restrict__ x, const T* __restrict__ Bm, const T* __restrict__ Cm,
+    const float* __restrict__ cum, const float* __restrict__ Hin, const float* __restrict__ D,
+    T* __restrict__ y, int Tlen, int H, int P, int G, int N, int Q, int nc) {
+    extern __shared__ float sm[];
+    const int NS = N + 1;
+    float* Cs = sm;               // [32][NS] C of the tile's rows
+    float* Ct = Cs + 32 * NS;     // [32][NS] C~ (off-diagonal sub-blocks)
+    float* cr = Ct + 32 * NS;     // [32][NS] rows' cum * log2(e)
+    float* Bs = cr + 32 * NS;     // [32][NS] B of a column sub-block (scaled to B~ off the diagonal)
+    float* cc = Bs + 32 * NS;     // [32][NS] its cum * log2(e)
+    float* rf = cc + 32 * NS;     // [NS] cum_e * log2(e)
+    float* Xs = rf + NS;          // [32][65]
+    float* Ps = Xs + 32 * 65;     // [32][33]
+    float* Hs = Ps + 32 * 33;     // [32][65]
+    constexpr float kL2e = 1.4426950408889634f;
+    const int nrt = (Q + 31) / 32;
+    const int k = blockIdx.x / nrt, i0 = (blockIdx.x % nrt) * 32;
+    const int bh = blockIdx.y, b = bh / H, h = bh % H, g = h / (H / G);
+    const int p0 = blockIdx.z * 64;
+    const int tid = threadIdx.x, ti = tid >> 3, tp = tid & 7;
+    const float* cumk = cum + ((size_t)bh * nc + k) * (size_t)Q * N;
+    const size_t tk = (size_t)k * Q;
+
+    for (int idx = tid; idx < 32 * N; idx += 256) {
+        const int ii = idx / N, n = idx % N, i = i0 + ii;
+        Cs[ii * NS + n] = (i < Q) ? to_f32(Cm[(((size_t)b * Tlen + tk + i) * G + g) * N + n]) : 0.f;
+        cr[ii * NS + n] = (i < Q) ? cumk[(size_t)i * N + n] * kL2e : 0.f;
+    }
+    for (int n = tid; n < N; n += 256) rf[n] = i0 > 0 ? cumk[(size_t)(i0 - 1) * N + n] * kL2e : 0.f;
+    __syncthreads();
+    if (i0 > 0) {
+        for (int idx = tid; idx < 32 * N; idx += 256) {
+            const int ii = idx / N, n = idx % N;
+            Ct[ii * NS + n] = Cs[ii * NS + n] * ex2_approx(cr[ii * NS + n] - rf[n]);
+        }
+    }
+
+    float acc[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) acc[m] = 0.f;
+    const int i_last = min(i0 + 31, Q - 1);
+    for (int j0 = 0; j0 <= i_last; j0 += 32) {
+        const bool on_diag = (j0 == i0);
+        __syncthreads();
+        for (int idx = tid; idx < 32 * N; idx += 256) {
+            const int jj = idx / N, n = idx % N, j = j0 + jj;
+            const float bv = (j < Q) ? to_f32(Bm[(((size_t)b * Tlen + tk + j) * G + g) * N + n]) : 0.f;
+            const float cj = (j < Q) ? cumk[(size_t)j * N + n] * kL2e : 0.f;
+            cc[jj * NS + n] = cj;
+            // off the diagonal: B~_j = B_j exp(cum_e - cum_j), exponent <= 0
+            Bs[jj * NS + n] = on_diag ? bv : bv * ex2_approx(rf[n] - cj);
+        }
+        for (int idx = tid; idx < 32 * 64; idx += 256) {
+            const int jj = idx / 64, p = idx % 64, j = j0 + jj;
+            Xs[jj * 65 + p] = (j < Q && p0 + p < P)
+                                  ? to_f32(x[(((size_t)b * Tlen + tk + j) * H + h) * P + p0 + p])
+                                  : 0.f;
+        }
+        __syncthreads();
+        const int i = i0 + ti;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int jj = tp * 4 + c, j = j0 + jj;
+            float s = 0.f;
+            if (j <= i && i < Q) {
+                const float* bj = Bs + jj * NS;
+                if (on_diag) {
+                    const float* ci = Cs + ti * NS;
+                    const float* cri = cr + ti * NS;
+                    const float* ccj = cc + jj * NS;
+                    for (int n = 0; n < N; ++n) s = fmaf(ci[n] * bj[n], ex2_approx(cri[n] - ccj[n]), s);
+                } else {
+                    const float* ci = Ct + ti * NS;
+                    for (int n = 0; n < N; ++n) s = fmaf(ci[n], bj[n], s);
+                }
+            }
+            Ps[ti * 33 + jj] = s;
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int jj = 0; jj < 32; ++jj) {
+            const float pv = Ps[ti * 33 + jj];
+#pragma unroll
+            for (int m = 0; m < 8; ++m) acc[m] = fmaf(pv, Xs[jj * 65 + tp + 8 * m], acc[m]);
+        }
+    }
+    // incoming-state term: sum_n C_i[n] exp(cum_i[n]) Hin[n, :]
+    float acc2[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) acc2[m] = 0.f;
+    const float* Hk = Hin + ((size_t)bh * nc + k) * (size_t)N * P;
+    for (int n0 = 0; n0 < N; n0 += 32) {
+        __syncthreads();
+        for (int idx = tid; idx < 32 * 64; idx += 256) {
+            const int nn = idx / 64, p = idx % 64;
+            Hs[nn * 65 + p] = (n0 + nn < N && p0 + p < P) ? Hk[(size_t)(n0 + nn) * P + p0 + p] : 0.f;
+        }
+        __syncthreads();
+        const int nmax = min(32, N - n0);
+        for (int nn = 0; nn < nmax; ++nn) {
+            const float cv = Cs[ti * NS + n0 + nn] * ex2_approx(cr[ti * NS + n0 + nn]);
+#pragma unroll
+            for (int m = 0; m < 8; ++m) acc2[m] = fmaf(cv, Hs[nn * 65 + tp + 8 * m], acc2[m]);
+        }
+    }
+    const int i = i0 + ti;
+    if (i >= Q) return;
+    const float dv = D ? D[h] : 0.f;
+    const size_t row = (((size_t)b * Tlen + tk + i) * H + h) * P;
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+        const int p = p0 + tp + 8 * m;
+        if (p < P) {
+            const float xv = to_f32(x[row + p]);
+            y[row + p] = from_f32<T>(acc[m] + acc2[m] + dv * xv);
+        }
+    }
+}
+
 cudaError_t launch_chunk_scan_simt(const Dims& d, const void* x, const void* Bm, const void* Cm,
                                    const float* cum, const float* Hin, const float* D, void* y,
                                    cudaStream_t st) {
     const int NS = d.N + 1;
-    size_t smem = (size_t)(2 * 32 * NS + 32 * 65 + 32 * 33 + 32 * 65) * sizeof(float);
-    smem += (d.diag ? (size_t)2 * 32 * NS : 64) * sizeof(float);
     dim3 grid(d.nc * ((d.Q + 31) / 32), d.B * d.H, (d.P + 63) / 64);
     cudaError_t e = cudaSuccess;
+    if (d.diag) {
+        const size_t dsmem = (size_t)(5 * 32 * NS + NS + 32 * 65 + 32 * 33 + 32 * 65) * sizeof(float);
+#define SSD_DIAG_LAUNCH(TT)                                                                       \
+    do {                                                                                          \
+        e = cudaFuncSetAttribute(diag_scan_simt_kernel<TT>,                                       \
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsmem);        \
+        if (e != cudaSuccess) return e;                                                           \
+        diag_scan_simt_kernel<TT><<<grid, 256, dsmem, st>>>(                                      \
+            (const TT*)x, (const TT*)Bm, (const TT*)Cm, cum, Hin, D, (TT*)y, d.T, d.H, d.P, d.G,  \
+            d.N, d.Q, d.nc);                                                                      \
+    } while (0)
+        if (d.bf16) SSD_DIAG_LAUNCH(__nv_bfloat16); else SSD_DIAG_LAUNCH(float);
+#undef SSD_DIAG_LAUNCH
+        return cudaGetLastError();
+    }
+    size_t smem = (size_t)(2 * 32 * NS + 32 * 65 + 32 * 33 + 32 * 65) * sizeof(float);
+    smem += (size_t)64 * sizeof(float);
 #define SSD_SCAN_LAUNCH(TT, DG)                                                                   \
     do {                                                                                          \
         e = cudaFuncSetAttribute(chunk_scan_simt_kernel<TT, DG>,                                  \
@@ -361,11 +511,7 @@ cudaError_t launch_chunk_scan_simt(const Dims& d, const void* x, const void* Bm,
             (const TT*)x, (const TT*)Bm, (const TT*)Cm, cum, Hin, D, (TT*)y, d.T, d.H, d.P, d.G, \
             d.N, d.Q, d.nc);                                                                      \
     } while (0)
-    if (d.bf16) {
-        if (d.diag) SSD_SCAN_LAUNCH(__nv_bfloat16, true); else SSD_SCAN_LAUNCH(__nv_bfloat16, false);
-    } else {
-        if (d.diag) SSD_SCAN_LAUNCH(float, true); else SSD_SCAN_LAUNCH(float, false);
-    }
+    if (d.bf16) SSD_SCAN_LAUNCH(__nv_bfloat16, false); else SSD_SCAN_LAUNCH(float, false);
 #undef SSD_SCAN_LAUNCH
     return cudaGetLastError();
 }
