@@ -224,16 +224,13 @@ cudaError_t launch_state_pass(const Dims& d, const float* cum, float* states, fl
     return cudaGetLastError();
 }
 
-// ============================================================ step 4/5 ====
-// Output of one chunk, a 32-row by 64-column tile per block:
-//   y_i = sum_{j<=i} S[i,j] x_j + (state term) + D x_i,
-//   scalar decay:    S[i,j] = (C_i . B_j) exp(cum_i - cum_j),
-//                    state term = exp(cum_i) C_i^T Hin;
-//   per-state decay: S[i,j] = sum_n C_i[n] B_j[n] exp(cum_i[n] - cum_j[n]),
-//                    state term = sum_n C_i[n] exp(cum_i[n]) Hin[n,:].
+// ============================================================== step 4 ====
+// Output of one chunk (scalar decay), a 32-row by 64-column tile per block:
+//   y_i = sum_{j<=i} S[i,j] x_j + exp(cum_i) C_i^T Hin + D x_i,
+//   S[i,j] = (C_i . B_j) exp(cum_i - cum_j).
 // The mask S is built in shared memory per 32x32 block and never stored.
 // Thread (ti = tid/8, tp = tid%8) owns row ti and columns tp + 8m, m < 8.
-template <typename T, bool DIAG>
+template <typename T>
 __global__ void __launch_bounds__(256) chunk_scan_simt_kernel(
     const T* __restrict__ x, const T* __restrict__ Bm, const T* __restrict__ Cm,
     const float* __restrict__ cum, const float* __restrict__ Hin, const float* __restrict__ D,
@@ -246,21 +243,20 @@ __global__ void __launch_bounds__(256) chunk_scan_simt_kernel(
     float* Ps = Xs + 32 * 65;          // [32][33]
     float* Hs = Ps + 32 * 33;          // [32][65]
     float* cr = Hs + 32 * 65;          // rows' cum: [32] or [32][NS]
-    float* cc = cr + (DIAG ? 32 * NS : 32);  // cols' cum
+    float* cc = cr + 32;               // cols' cum
     const int nrt = (Q + 31) / 32;
     const int k = blockIdx.x / nrt, i0 = (blockIdx.x % nrt) * 32;
     const int bh = blockIdx.y, b = bh / H, h = bh % H, g = h / (H / G);
     const int p0 = blockIdx.z * 64;
     const int tid = threadIdx.x, ti = tid >> 3, tp = tid & 7;
-    const float* cumk = cum + ((size_t)bh * nc + k) * (size_t)Q * (DIAG ? N : 1);
+    const float* cumk = cum + ((size_t)bh * nc + k) * (size_t)Q;
     const size_t tk = (size_t)k * Q;
 
     for (int idx = tid; idx < 32 * N; idx += 256) {
         const int ii = idx / N, n = idx % N, i = i0 + ii;
         Cs[ii * NS + n] = (i < Q) ? to_f32(Cm[(((size_t)b * Tlen + tk + i) * G + g) * N + n]) : 0.f;
-        if (DIAG) cr[ii * NS + n] = (i < Q) ? cumk[(size_t)i * N + n] : 0.f;
     }
-    if (!DIAG && tid < 32) cr[tid] = (i0 + tid < Q) ? cumk[i0 + tid] : 0.f;
+    if (tid < 32) cr[tid] = (i0 + tid < Q) ? cumk[i0 + tid] : 0.f;
 
     float acc[8];
 #pragma unroll
@@ -272,9 +268,8 @@ __global__ void __launch_bounds__(256) chunk_scan_simt_kernel(
             const int jj = idx / N, n = idx % N, j = j0 + jj;
             Bs[jj * NS + n] =
                 (j < Q) ? to_f32(Bm[(((size_t)b * Tlen + tk + j) * G + g) * N + n]) : 0.f;
-            if (DIAG) cc[jj * NS + n] = (j < Q) ? cumk[(size_t)j * N + n] : 0.f;
         }
-        if (!DIAG && tid < 32) cc[tid] = (j0 + tid < Q) ? cumk[j0 + tid] : 0.f;
+        if (tid < 32) cc[tid] = (j0 + tid < Q) ? cumk[j0 + tid] : 0.f;
         for (int idx = tid; idx < 32 * 64; idx += 256) {
             const int jj = idx / 64, p = idx % 64, j = j0 + jj;
             Xs[jj * 65 + p] = (j < Q && p0 + p < P)
@@ -290,14 +285,8 @@ __global__ void __launch_bounds__(256) chunk_scan_simt_kernel(
             if (j <= i && i < Q) {
                 const float* ci = Cs + ti * NS;
                 const float* bj = Bs + jj * NS;
-                if (DIAG) {
-                    const float* cri = cr + ti * NS;
-                    const float* ccj = cc + jj * NS;
-                    for (int n = 0; n < N; ++n) s = fmaf(ci[n] * bj[n], expf(cri[n] - ccj[n]), s);
-                } else {
-                    for (int n = 0; n < N; ++n) s = fmaf(ci[n], bj[n], s);
-                    s *= expf(cr[ti] - cc[jj]);
-                }
+                for (int n = 0; n < N; ++n) s = fmaf(ci[n], bj[n], s);
+                s *= expf(cr[ti] - cc[jj]);
             }
             Ps[ti * 33 + jj] = s;
         }
@@ -323,15 +312,14 @@ __global__ void __launch_bounds__(256) chunk_scan_simt_kernel(
         __syncthreads();
         const int nmax = min(32, N - n0);
         for (int nn = 0; nn < nmax; ++nn) {
-            float cv = Cs[ti * NS + n0 + nn];
-            if (DIAG) cv *= expf(cr[ti * NS + n0 + nn]);
+            const float cv = Cs[ti * NS + n0 + nn];
 #pragma unroll
             for (int m = 0; m < 8; ++m) acc2[m] = fmaf(cv, Hs[nn * 65 + tp + 8 * m], acc2[m]);
         }
     }
     const int i = i0 + ti;
     if (i >= Q) return;
-    const float sc = DIAG ? 1.f : expf(cr[ti]);
+    const float sc = expf(cr[ti]);
     const float dv = D ? D[h] : 0.f;
     const size_t row = (((size_t)b * Tlen + tk + i) * H + h) * P;
 #pragma unroll
@@ -522,16 +510,16 @@ cudaError_t launch_chunk_scan_simt(const Dims& d, const void* x, const void* Bm,
     }
     size_t smem = (size_t)(2 * 32 * NS + 32 * 65 + 32 * 33 + 32 * 65) * sizeof(float);
     smem += (size_t)64 * sizeof(float);
-#define SSD_SCAN_LAUNCH(TT, DG)                                                                   \
+#define SSD_SCAN_LAUNCH(TT)                                                                       \
     do {                                                                                          \
-        e = cudaFuncSetAttribute(chunk_scan_simt_kernel<TT, DG>,                                  \
+        e = cudaFuncSetAttribute(chunk_scan_simt_kernel<TT>,                                      \
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);         \
         if (e != cudaSuccess) return e;                                                           \
-        chunk_scan_simt_kernel<TT, DG><<<grid, 256, smem, st>>>(                                  \
+        chunk_scan_simt_kernel<TT><<<grid, 256, smem, st>>>(                                      \
             (const TT*)x, (const TT*)Bm, (const TT*)Cm, cum, Hin, D, (TT*)y, d.T, d.H, d.P, d.G, \
             d.N, d.Q, d.nc);                                                                      \
     } while (0)
-    if (d.bf16) SSD_SCAN_LAUNCH(__nv_bfloat16, false); else SSD_SCAN_LAUNCH(float, false);
+    if (d.bf16) SSD_SCAN_LAUNCH(__nv_bfloat16); else SSD_SCAN_LAUNCH(float);
 #undef SSD_SCAN_LAUNCH
     return cudaGetLastError();
 }
