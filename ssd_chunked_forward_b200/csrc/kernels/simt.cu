@@ -181,8 +181,12 @@ cudaError_t launch_chunk_state_simt(const Dims& d, const void* x, const void* Bm
 }
 
 // ============================================================ step 3 ======
-// One thread per (b,h,n,p) chain, sequential over chunks.  The next chunk's
-// state and decay are loaded before the current update so the loads overlap.
+// One thread per (b,h,n,p) chain, sequential over chunks.  States and chunk
+// decays are read in groups of kPassGroup chunks, the next group's loads
+// issued before the current group's updates, so each thread keeps 2 x 8
+// loads in flight (a long chain is otherwise bound by one load's latency per
+// chunk).  In place: the slot of chunk k receives the state entering it.
+constexpr int kPassGroup = 8;
 template <bool DIAG>
 __global__ void __launch_bounds__(256) state_pass_kernel(const float* __restrict__ cum,
                                                          float* __restrict__ states,
@@ -198,17 +202,33 @@ __global__ void __launch_bounds__(256) state_pass_kernel(const float* __restrict
     const float* ce = cum + bh * (long long)nc * Q * (DIAG ? N : 1) +
                       (DIAG ? (size_t)(Q - 1) * N + n : (size_t)(Q - 1));
     const size_t cstep = (size_t)Q * (DIAG ? N : 1);
+    float sb[kPassGroup], cb[kPassGroup];
+#pragma unroll
+    for (int u = 0; u < kPassGroup; ++u) {
+        sb[u] = u < nc ? sp[(size_t)u * NP] : 0.f;
+        cb[u] = u < nc ? ce[(size_t)u * cstep] : 0.f;
+    }
     float hval = 0.f;
-    float s_next = sp[0];
-    float c_next = ce[0];
-    for (int k = 0; k < nc; ++k) {
-        const float s = s_next, c = c_next;
-        if (k + 1 < nc) {
-            s_next = sp[(size_t)(k + 1) * NP];
-            c_next = ce[(size_t)(k + 1) * cstep];
+    for (int k0 = 0; k0 < nc; k0 += kPassGroup) {
+        float s[kPassGroup], c[kPassGroup];
+#pragma unroll
+        for (int u = 0; u < kPassGroup; ++u) {
+            s[u] = sb[u];
+            c[u] = cb[u];
+            const int kn = k0 + kPassGroup + u;
+            if (kn < nc) {
+                sb[u] = sp[(size_t)kn * NP];
+                cb[u] = ce[(size_t)kn * cstep];
+            }
         }
-        sp[(size_t)k * NP] = hval;
-        hval = fmaf(expf(c), hval, s);
+#pragma unroll
+        for (int u = 0; u < kPassGroup; ++u) {
+            const int k = k0 + u;
+            if (k < nc) {
+                sp[(size_t)k * NP] = hval;
+                hval = fmaf(expf(c[u]), hval, s[u]);
+            }
+        }
     }
     if (fin) fin[bh * NP + r] = hval;
 }
