@@ -76,7 +76,11 @@ enum {
                              (or diag_scan), each a separate kernel, states in HBM */
     SSD_PATH_SIMT = 2,    /* the same four steps on CUDA cores only (fp32 math)  */
     SSD_PATH_FUSED = 3    /* one persistent kernel: chunk states, inter-chunk pass
-                             and outputs fused; states never leave L2             */
+                             and outputs fused; states never leave L2.  Its blocks
+                             wait on one another, so the library orders every fused
+                             launch on a device after the previous one, whatever
+                             the stream (copies and other kernels still overlap);
+                             not while the stream is being captured into a graph */
 };
 
 /* Implementations for the per-step entry points. */

@@ -40,4 +40,12 @@ cudaError_t launch_fused_tc(const Dims& d, const void* x, const float* a, const 
                             const void* Cm, const float* D, void* y, float* fin, float* ring,
                             unsigned* flags, int* status, bool test_stall, cudaStream_t st);
 
+// launch_fused_tc ordered after the previous fused launch on this device, on
+// whatever stream that was: the persistent kernel's blocks wait on one
+// another, which needs all of them resident, so two such kernels must not
+// share the GPU.  Skipped while `st` is being captured into a graph.
+cudaError_t launch_fused_ordered(const Dims& d, const void* x, const float* a, const void* Bm,
+                                 const void* Cm, const float* D, void* y, float* fin, float* ring,
+                                 unsigned* flags, int* status, bool test_stall, cudaStream_t st);
+
 }  // namespace ssd

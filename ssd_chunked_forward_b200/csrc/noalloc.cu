@@ -79,6 +79,6 @@ extern "C" ssd_status ssd_forward_noalloc(const ssd_shape* shape, const void* x,
     // the status word and the per-chain counters start at zero on every call
     if (cudaMemsetAsync(p, 0, kCtrl + kFlags, cs) != cudaSuccess) return SSD_ERR_CUDA;
     const cudaError_t e =
-        ssd::launch_fused_tc(d, x, a, Bm, Cm, D, y, final_state, ring, flags, ctrl, false, cs);
+        ssd::launch_fused_ordered(d, x, a, Bm, Cm, D, y, final_state, ring, flags, ctrl, false, cs);
     return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }

@@ -2,6 +2,8 @@
 // validation, workspace layout, path selection and launches on the caller's
 // stream.  No allocation happens here; every buffer belongs to the caller.
 #include <cuda_runtime.h>
+
+#include <mutex>
 #include <stdint.h>
 #include <string.h>
 
@@ -99,6 +101,12 @@ Workspace carve(void* ws, const Dims& d) {
 
 ssd_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA; }
 
+// one event per device: the end of the last fused launch
+constexpr int kMaxDevices = 64;
+std::mutex g_fused_mu;
+cudaEvent_t g_fused_done[kMaxDevices] = {};
+bool g_fused_seen[kMaxDevices] = {};
+
 ssd_status run_modular(const Dims& d0, const void* x, const float* a, const void* Bm,
                        const void* Cm, const float* D, void* y, float* fin, const Workspace& w,
                        cudaStream_t st, bool allow_tc) {
@@ -118,6 +126,33 @@ ssd_status run_modular(const Dims& d0, const void* x, const float* a, const void
 }
 
 }  // namespace
+
+namespace ssd {
+cudaError_t launch_fused_ordered(const Dims& d, const void* x, const float* a, const void* Bm,
+                                 const void* Cm, const float* D, void* y, float* fin, float* ring,
+                                 unsigned* flags, int* status, bool test_stall, cudaStream_t st) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) return cudaErrorInvalidValue;
+    int dev = 0;
+    if (cap != cudaStreamCaptureStatusNone || cudaGetDevice(&dev) != cudaSuccess || dev < 0 ||
+        dev >= kMaxDevices)
+        return launch_fused_tc(d, x, a, Bm, Cm, D, y, fin, ring, flags, status, test_stall, st);
+    std::lock_guard<std::mutex> lock(g_fused_mu);
+    if (!g_fused_done[dev]) {
+        cudaError_t e = cudaEventCreateWithFlags(&g_fused_done[dev], cudaEventDisableTiming);
+        if (e != cudaSuccess) return e;
+    }
+    if (g_fused_seen[dev]) {
+        cudaError_t e = cudaStreamWaitEvent(st, g_fused_done[dev], 0);
+        if (e != cudaSuccess) return e;
+    }
+    cudaError_t e = launch_fused_tc(d, x, a, Bm, Cm, D, y, fin, ring, flags, status, test_stall, st);
+    if (e != cudaSuccess) return e;
+    e = cudaEventRecord(g_fused_done[dev], st);
+    if (e == cudaSuccess) g_fused_seen[dev] = true;
+    return e;
+}
+}  // namespace ssd
 
 extern "C" {
 
@@ -187,7 +222,7 @@ ssd_status ssd_forward_path(const ssd_shape* shape, const void* x, const float* 
         case SSD_PATH_SIMT:
             return run_modular(d, x, a, Bm, Cm, D, y, final_state, w, cs, false);
         case SSD_PATH_FUSED:
-            return cuda_status(ssd::launch_fused_tc(d, x, a, Bm, Cm, D, y, final_state, w.ring,
+            return cuda_status(ssd::launch_fused_ordered(d, x, a, Bm, Cm, D, y, final_state, w.ring,
                                                     w.flags, w.ctrl,
                                                     (flags & SSD_FLAG_TEST_STALL) != 0, cs));
         case SSD_PATH_MODULAR:

@@ -266,3 +266,31 @@ def test_fused_bounded_wait_reports_timeout():
     assert ssd.device_status(ws) == ssd.SSD_OK
     ey, ef = parity_on_chains(inp, y, fin, _all_chains(w))
     assert ey <= TOL_BF16 and ef <= TOL_BF16
+
+
+def test_fused_on_two_streams():
+    """Forwards issued on two streams at once (each with its own workspace):
+    the library orders the fused launches, so both finish with SSD_OK and give
+    the single-stream result bit for bit."""
+    w = small_case(B=2, T=2048, H=16, P=64, N=128, G=1, chunk=256, dtype="bf16", seed=21)
+    inp = generate(w)
+    dev = to_dev(inp)
+    shape = ssd.shape_of(dev["x"], dev["a"], dev["Bm"], w.chunk)
+    if not ssd.path_supported(shape, ssd.PATH_FUSED):
+        pytest.skip("fused path does not serve this shape")
+    y_ref, f_ref = ssd.forward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], dev["D"], w.chunk,
+                               path=ssd.PATH_FUSED)
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    wss = [ssd.alloc_workspace(shape) for _ in streams]
+    outs = []
+    for r in range(6):
+        s = r % 2
+        with torch.cuda.stream(streams[s]):
+            outs.append(ssd.forward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], dev["D"], w.chunk,
+                                    workspace=wss[s], path=ssd.PATH_FUSED, stream=streams[s]))
+    torch.cuda.synchronize()
+    for s in range(2):
+        assert ssd.device_status(wss[s], streams[s]) == ssd.SSD_OK
+    for y, f in outs:
+        assert torch.equal(y, y_ref) and torch.equal(f, f_ref)
