@@ -117,11 +117,14 @@ static double Dval(const double* D, int h) {
  * state space view; "Continuous-to-Discrete Discretization", D x_t.) */
 static void recurrence_chain(const oracle_shape* s, const double* x, const double* a,
                              const double* Bm, const double* Cm, const double* D,
-                             int b, int h, int t_end, double* y, double* fin,
-                             double* bounds) {
+                             const double* init, int b, int h, int t_end, double* y,
+                             double* fin, double* bounds) {
     const int N = s->N, P = s->P, Q = s->chunk;
     const int g = group_of(s, h);
     double* st = (double*)calloc((size_t)N * P, sizeof(double));
+    /* h_{-1}: zero, or the given state of this (b, h) chain (resuming a
+     * sequence from the state a previous call ended with) */
+    if (init) memcpy(st, init + ((size_t)b * s->H + h) * N * P, (size_t)N * P * sizeof(double));
     double* e = (double*)malloc((size_t)N * sizeof(double));
     double* prev = (double*)malloc((size_t)N * P * sizeof(double));
     const double dh = Dval(D, h);
@@ -317,6 +320,7 @@ typedef struct {
     int route; /* 1 = O1, 2 = O2, 3 = O3 */
     const oracle_shape* s;
     const double *x, *a, *Bm, *Cm, *D;
+    const double* init; /* [B][H][N][P] initial states (O1 only), or NULL */
     const int* chains; /* pairs (b, h) */
     int n_chains;
     int t_end;
@@ -341,7 +345,7 @@ static void* worker(void* arg) {
         double* fin = j->fin ? j->fin + (size_t)c * NP : NULL;
         if (j->route == 1) {
             double* bd = j->bounds ? j->bounds + (size_t)c * nc * NP : NULL;
-            recurrence_chain(s, j->x, j->a, j->Bm, j->Cm, j->D, b, h, j->t_end, y, fin, bd);
+            recurrence_chain(s, j->x, j->a, j->Bm, j->Cm, j->D, j->init, b, h, j->t_end, y, fin, bd);
         } else if (j->route == 2) {
             brute_chain(s, j->x, j->a, j->Bm, j->Cm, j->D, b, h, y, fin);
         } else {
@@ -378,6 +382,19 @@ int oracle_recurrence(const oracle_shape* s, const double* x, const double* a,
     job_t j;
     memset(&j, 0, sizeof j);
     j.route = 1; j.s = s; j.x = x; j.a = a; j.Bm = Bm; j.Cm = Cm; j.D = D;
+    j.chains = chains; j.n_chains = n_chains; j.t_end = t_end;
+    j.y = y; j.fin = fin; j.bounds = bounds;
+    return run(&j, nthreads);
+}
+
+/* O1 from given initial states init[B][H][N][P] (NULL: zero). */
+int oracle_recurrence_init(const oracle_shape* s, const double* x, const double* a,
+                           const double* Bm, const double* Cm, const double* D,
+                           const double* init, const int* chains, int n_chains, int t_end,
+                           double* y, double* fin, double* bounds, int nthreads) {
+    job_t j;
+    memset(&j, 0, sizeof j);
+    j.route = 1; j.s = s; j.x = x; j.a = a; j.Bm = Bm; j.Cm = Cm; j.D = D; j.init = init;
     j.chains = chains; j.n_chains = n_chains; j.t_end = t_end;
     j.y = y; j.fin = fin; j.bounds = bounds;
     return run(&j, nthreads);

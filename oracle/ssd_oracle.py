@@ -55,10 +55,12 @@ def _load():
         sp = ctypes.POINTER(_Shape)
         lib.oracle_recurrence.argtypes = [sp, dp, dp, dp, dp, dp, ip, ctypes.c_int, ctypes.c_int,
                                           dp, dp, dp, ctypes.c_int]
+        lib.oracle_recurrence_init.argtypes = [sp, dp, dp, dp, dp, dp, dp, ip, ctypes.c_int, ctypes.c_int,
+                                               dp, dp, dp, ctypes.c_int]
         lib.oracle_brute.argtypes = [sp, dp, dp, dp, dp, dp, ip, ctypes.c_int, dp, dp, ctypes.c_int]
         lib.oracle_chunked.argtypes = [sp, dp, dp, dp, dp, dp, ip, ctypes.c_int, dp, dp, dp, dp, dp,
                                        ctypes.c_int]
-        for f in (lib.oracle_recurrence, lib.oracle_brute, lib.oracle_chunked):
+        for f in (lib.oracle_recurrence, lib.oracle_recurrence_init, lib.oracle_brute, lib.oracle_chunked):
             f.restype = ctypes.c_int
         lib.oracle_set_mutation.argtypes = [ctypes.c_int]
         lib.oracle_set_mutation.restype = None
@@ -137,22 +139,28 @@ def _prep(prob: Problem):
     return p
 
 
-def recurrence(prob: Problem, chains=None, t_end=None, chunk=0, want_y=True, nthreads=None):
+def recurrence(prob: Problem, chains=None, t_end=None, chunk=0, want_y=True, nthreads=None,
+               initial=None):
     """O1.  Returns dict(y=[C,T,P] (rows >= t_end are zero), final=[C,N,P],
-    bounds=[C,nc,N,P] state after each chunk when chunk>0)."""
+    bounds=[C,nc,N,P] state after each chunk when chunk>0).  ``initial``
+    [B,H,N,P]: the state h_{-1} each chain starts from (default zero)."""
     lib = _load()
     p = _prep(prob)
     B, T, H, P, G, N = p.dims
+    init = _f64(initial)
+    if init is not None and init.shape != (B, H, N, P):
+        raise ValueError("initial state must be [B,H,N,P]")
     ch = _chains(p, chains)
     C = ch.shape[0]
     t_end = T if t_end is None else int(t_end)
     y = np.zeros((C, T, P)) if want_y else None
     fin = np.zeros((C, N, P))
     bounds = np.zeros((C, T // chunk, N, P)) if chunk else None
-    rc = lib.oracle_recurrence(ctypes.byref(_shape(p, chunk)), _ptr(p.x), _ptr(p.a), _ptr(p.Bm),
-                               _ptr(p.Cm), _ptr(p.D), ch.ctypes.data_as(ctypes.POINTER(ctypes.c_int)),
-                               C, t_end, _ptr(y), _ptr(fin), _ptr(bounds),
-                               nthreads or default_threads())
+    rc = lib.oracle_recurrence_init(ctypes.byref(_shape(p, chunk)), _ptr(p.x), _ptr(p.a), _ptr(p.Bm),
+                                    _ptr(p.Cm), _ptr(p.D), _ptr(init),
+                                    ch.ctypes.data_as(ctypes.POINTER(ctypes.c_int)),
+                                    C, t_end, _ptr(y), _ptr(fin), _ptr(bounds),
+                                    nthreads or default_threads())
     if rc:
         raise ValueError("oracle_recurrence rejected its arguments")
     return {"y": y, "final": fin, "bounds": bounds, "chains": ch}

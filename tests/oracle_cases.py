@@ -96,3 +96,24 @@ def exact_rational_brute(xq, lam, Bq, Cq, Dq):
                 row[p] += cb * prod * xq[s][p]
         y.append(row)
     return y
+
+
+def free_response(prob: Problem, h0):
+    """Zero input (x == 0): the state only decays, h_t = exp(sum_{k<=t} a_k) o h0,
+    so y_t[p] = sum_n C_t[n] exp(sum_{k<=t} a_k[n]) h0[n, p] -- the closed form of
+    the unforced recurrence (llms.blog "The SSD Theoretical Equivalence", the
+    state-space view with B x = 0).  Returns [B,H,T,P] and the final [B,H,N,P]."""
+    B, T, H, P = prob.x.shape
+    G, N = prob.Bm.shape[2], prob.Bm.shape[3]
+    y = np.zeros((B, H, T, P))
+    fin = np.zeros((B, H, N, P))
+    for b in range(B):
+        for h in range(H):
+            g = h // (H // G)
+            a = prob.a[b, :, h] if prob.a.ndim == 3 else prob.a[b, :, h, :]
+            cum = np.cumsum(a, axis=0)  # inclusive: the decay of h0 up to and including t
+            dec = np.exp(cum) if prob.a.ndim == 4 else np.exp(cum)[:, None] * np.ones((1, N))
+            for t in range(T):
+                y[b, h, t] = (prob.Cm[b, t, g, :] * dec[t]) @ h0[b, h]
+            fin[b, h] = dec[T - 1][:, None] * h0[b, h]
+    return y, fin

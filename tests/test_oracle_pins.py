@@ -18,7 +18,7 @@ import pytest
 from oracle import ssd_oracle as O
 from oracle.ssd_oracle import Problem
 from tests.oracle_cases import (all_y, causal_conv_direct, causal_conv_fft, causal_linear_attention,
-                                exact_rational_brute, lti_kernel, random_problem, rel_inf)
+                                exact_rational_brute, free_response, lti_kernel, random_problem, rel_inf)
 
 SHAPES = [
     # B, T, H, P, G, N
@@ -242,3 +242,45 @@ def test_golden_impulse_response_decay_085():
     prob = Problem(x, a, one, one, None)
     for route in (O.recurrence(prob), O.brute(prob), O.chunked(prob, 4)):
         assert np.max(np.abs(route["y"][0, :, 0] - rows[:, 1])) < 1e-14
+
+
+@pytest.mark.parametrize("per_state", [False, True])
+def test_initial_state_resumes_a_split_sequence(per_state):
+    """Running the first t1 tokens, then the rest from the state they ended with,
+    gives the single run's y and final state: the initial state is exactly the
+    h_{-1} the recurrence would have carried (a sequence split across calls)."""
+    rng = np.random.default_rng(31 + per_state)
+    prob = random_problem(rng, B=2, T=40, H=3, P=4, G=1, N=5, per_state=per_state)
+    B, T, H, P = prob.x.shape
+    N = prob.Bm.shape[3]
+    full = O.recurrence(prob)
+    for t1 in (1, 17, 39):
+        cut = lambda arr, sl: None if arr is None else arr[:, sl]
+        first = O.Problem(prob.x[:, :t1], cut(prob.a, slice(0, t1)), prob.Bm[:, :t1], prob.Cm[:, :t1], prob.D)
+        rest = O.Problem(prob.x[:, t1:], cut(prob.a, slice(t1, None)), prob.Bm[:, t1:], prob.Cm[:, t1:], prob.D)
+        r1 = O.recurrence(first)
+        r2 = O.recurrence(rest, initial=r1["final"].reshape(B, H, N, P))
+        y = np.concatenate([all_y(r1, B, H), all_y(r2, B, H)], axis=2)
+        assert rel_inf(y, all_y(full, B, H)) < 1e-12
+        assert rel_inf(r2["final"], full["final"]) < 1e-12
+
+
+@pytest.mark.parametrize("per_state", [False, True])
+def test_initial_state_free_response(per_state):
+    """x == 0: y is the decayed initial state read out by C (closed form)."""
+    rng = np.random.default_rng(41 + per_state)
+    prob = random_problem(rng, B=1, T=25, H=2, P=3, G=1, N=4, per_state=per_state)
+    prob = O.Problem(np.zeros_like(prob.x), prob.a, prob.Bm, prob.Cm, prob.D)
+    h0 = rng.standard_normal((1, 2, 4, 3))
+    res = O.recurrence(prob, initial=h0)
+    y_ref, fin_ref = free_response(prob, h0)
+    assert rel_inf(all_y(res, 1, 2), y_ref) < 1e-12
+    assert rel_inf(res["final"].reshape(fin_ref.shape), fin_ref) < 1e-12
+
+
+def test_zero_initial_state_is_the_default():
+    rng = np.random.default_rng(51)
+    prob = random_problem(rng, B=2, T=9, H=2, P=3, G=2, N=4)
+    a = O.recurrence(prob)
+    b = O.recurrence(prob, initial=np.zeros((2, 2, 4, 3)))
+    assert np.array_equal(a["y"], b["y"]) and np.array_equal(a["final"], b["final"])
