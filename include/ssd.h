@@ -130,6 +130,21 @@ ssd_status ssd_forward_path(const ssd_shape* shape, const void* x, const float* 
                             float* final_state, void* workspace, size_t ws_bytes,
                             ssd_stream stream, unsigned path, unsigned flags);
 
+/* ssd_forward_path() with the chains starting from a given state instead of
+ * zero: initial_state[B][H][N][P] fp32 (device, 16-byte aligned; NULL means
+ * zero) is h_{-1} of every (batch, head) chain, so a sequence split across
+ * calls resumes exactly -- pass the final_state of the call that ended where
+ * this one starts.  The recurrence h_t = exp(a_t) h_{t-1} + B_t x_t^T of the
+ * SSD state-space view ("State Space Models and Mamba ...", llms.blog, "The
+ * SSD Theoretical Equivalence") with h_{-1} given; the pages' forward starts
+ * from zero.  initial_state may alias final_state (it is read before any
+ * final state is written).  Errors as for ssd_forward_path(). */
+ssd_status ssd_forward_init(const ssd_shape* shape, const void* x, const float* a,
+                            const void* Bm, const void* Cm, const float* D,
+                            const float* initial_state, void* y, float* final_state,
+                            void* workspace, size_t ws_bytes, ssd_stream stream, unsigned path,
+                            unsigned flags);
+
 /* Synchronises `stream`, then returns the status word a previous
  * ssd_forward* call on this workspace left (SSD_OK, or SSD_ERR_TIMEOUT when
  * a bounded device wait ran out), or SSD_ERR_CUDA when the stream reports an

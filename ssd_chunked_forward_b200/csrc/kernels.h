@@ -16,8 +16,9 @@ struct Dims {
 cudaError_t launch_chunk_cumsum(const Dims& d, const float* a, float* cum, cudaStream_t st);
 cudaError_t launch_chunk_state_simt(const Dims& d, const void* x, const void* Bm, const float* cum,
                                     float* states, cudaStream_t st);
+// init: [B,H,N,P] state entering the first chunk, or null for zero
 cudaError_t launch_state_pass(const Dims& d, const float* cum, float* states, float* fin,
-                              cudaStream_t st);
+                              const float* init, cudaStream_t st);
 // output step; serves the scalar (chunk_scan) and the per-state (diag_scan) decay
 cudaError_t launch_chunk_scan_simt(const Dims& d, const void* x, const void* Bm, const void* Cm,
                                    const float* cum, const float* Hin, const float* D, void* y,
@@ -38,7 +39,8 @@ bool fused_supported(const Dims& d);
 size_t fused_ring_bytes(const Dims& d);
 cudaError_t launch_fused_tc(const Dims& d, const void* x, const float* a, const void* Bm,
                             const void* Cm, const float* D, void* y, float* fin, float* ring,
-                            unsigned* flags, int* status, bool test_stall, cudaStream_t st);
+                            unsigned* flags, int* status, bool test_stall, cudaStream_t st,
+                            const float* init = nullptr);
 
 // launch_fused_tc ordered after the previous fused launch on this device, on
 // whatever stream that was: the persistent kernel's blocks wait on one
@@ -46,6 +48,7 @@ cudaError_t launch_fused_tc(const Dims& d, const void* x, const float* a, const 
 // share the GPU.  Skipped while `st` is being captured into a graph.
 cudaError_t launch_fused_ordered(const Dims& d, const void* x, const float* a, const void* Bm,
                                  const void* Cm, const float* D, void* y, float* fin, float* ring,
-                                 unsigned* flags, int* status, bool test_stall, cudaStream_t st);
+                                 unsigned* flags, int* status, bool test_stall, cudaStream_t st,
+                                 const float* init = nullptr);
 
 }  // namespace ssd

@@ -88,6 +88,7 @@ struct ScanParams {
     int* status;       // device status word or null
     int T, H, G, nblk, hpb, nslices, n_items;
     int test_stall;
+    int has_init;      // fused: chains start from tm_init's states, not zero
 };
 
 // smem layout (offsets from the 1024-aligned base)
@@ -152,7 +153,8 @@ template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
                    const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y,
-                   const __grid_constant__ CUtensorMap tm_st, const ScanParams p, int B) {
+                   const __grid_constant__ CUtensorMap tm_st, const __grid_constant__ CUtensorMap tm_init,
+                   const ScanParams p, int B) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -397,7 +399,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (hc > 0 && !tc::mbar_wait(&bars->hin_free, (hc - 1) & 1, abort_v)) { ok = false; break; }
                     if (MODE == kFused) {
                         if (w.j == 0) {
-                            tc::mbar_arrive(&bars->hin_full);  // zero state: nothing to load
+                            if (p.has_init) {  // the given initial state of the chain
+                                tc::mbar_arrive_expect_tx(&bars->hin_full, kStateBytes);
+                                tc::tma_load_2d(sHin, &tm_init, &bars->hin_full, 0, chain * kN);
+                                tc::tma_load_2d(sHin + kTile, &tm_init, &bars->hin_full, 32, chain * kN);
+                            } else {
+                                tc::mbar_arrive(&bars->hin_full);  // zero state: nothing to load
+                            }
                             continue;
                         }
                         // bounded wait for the previous block of this chain
@@ -682,7 +690,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                              tc::mbar_wait(&bars->hin_full, hc & 1, abort_v);
                         if (!sync_ok(ok)) { alive = false; break; }
                         tc::tc_fence_after();
-                        const bool zero_in = MODE == kFused && w.j == 0;
+                        const bool zero_in = MODE == kFused && w.j == 0 && !p.has_init;
                         const float eL = ex2_approx(cum[kBlk - 1] * kLog2e);
                         // this warp's 32 columns of the state, 16 at a time
 #pragma unroll 1
@@ -831,13 +839,19 @@ int heads_per_item(const Dims& d) {
 
 template <int MODE>
 cudaError_t launch(const Dims& d, const void* x, const void* Bm, const void* Cm, void* y,
-                   const float* states, uint64_t state_rows, ScanParams p, cudaStream_t st) {
-    CUtensorMap tx, tb, tcm, ty, ts;
+                   const float* states, uint64_t state_rows, ScanParams p, cudaStream_t st,
+                   const float* init = nullptr) {
+    CUtensorMap tx, tb, tcm, ty, ts, ti;
     cudaError_t e = make_tmap_bf16_3d(&tx, x, d.P, d.H, (uint64_t)d.B * d.T, kBlk);
     if (e == cudaSuccess) e = make_tmap_bf16_3d(&tb, Bm, d.N, d.G, (uint64_t)d.B * d.T, kBlk);
     if (e == cudaSuccess) e = make_tmap_bf16_3d(&tcm, Cm, d.N, d.G, (uint64_t)d.B * d.T, kBlk);
     if (e == cudaSuccess) e = make_tmap_bf16_3d(&ty, y, d.P, d.H, (uint64_t)d.B * d.T, kBlk);
     if (e == cudaSuccess) e = make_tmap_f32_rows64(&ts, states, state_rows);
+    // the initial states [B*H*N][P] (a stand-in map over `states` when there are none)
+    if (e == cudaSuccess)
+        e = init ? make_tmap_f32_rows64(&ti, init, (uint64_t)d.B * d.H * kN)
+                 : make_tmap_f32_rows64(&ti, states, state_rows);
+    p.has_init = init ? 1 : 0;
     if (e != cudaSuccess) return e;
     p.T = d.T; p.H = d.H; p.G = d.G;
     p.nblk = d.T / kBlk;
@@ -850,7 +864,7 @@ cudaError_t launch(const Dims& d, const void* x, const void* Bm, const void* Cm,
     e = cudaFuncSetAttribute(scan_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemBytes);
     if (e != cudaSuccess) return e;
-    scan_tc_kernel<MODE><<<grid, kThreads, kSmemBytes, st>>>(tx, tb, tcm, ty, ts, p, d.B);
+    scan_tc_kernel<MODE><<<grid, kThreads, kSmemBytes, st>>>(tx, tb, tcm, ty, ts, ti, p, d.B);
     return cudaGetLastError();
 }
 
@@ -878,7 +892,8 @@ size_t fused_ring_bytes(const Dims& d) { return (size_t)d.B * d.H * 2 * kN * kP 
 
 cudaError_t launch_fused_tc(const Dims& d, const void* x, const float* a, const void* Bm,
                             const void* Cm, const float* D, void* y, float* fin, float* ring,
-                            unsigned* flags, int* status, bool test_stall, cudaStream_t st) {
+                            unsigned* flags, int* status, bool test_stall, cudaStream_t st,
+                            const float* init) {
     if (!fused_supported(d)) return cudaErrorNotSupported;
     ScanParams p = {};
     p.a = a;
@@ -887,7 +902,7 @@ cudaError_t launch_fused_tc(const Dims& d, const void* x, const float* a, const 
     p.fin = fin;
     p.status = status;
     p.test_stall = test_stall ? 1 : 0;
-    return launch<kFused>(d, x, Bm, Cm, y, ring, (uint64_t)d.B * d.H * 2 * kN, p, st);
+    return launch<kFused>(d, x, Bm, Cm, y, ring, (uint64_t)d.B * d.H * 2 * kN, p, st, init);
 }
 
 }  // namespace ssd

@@ -190,8 +190,9 @@ constexpr int kPassGroup = 8;
 template <bool DIAG>
 __global__ void __launch_bounds__(256) state_pass_kernel(const float* __restrict__ cum,
                                                          float* __restrict__ states,
-                                                         float* __restrict__ fin, int N, int P,
-                                                         int Q, int nc, long long total) {
+                                                         float* __restrict__ fin,
+                                                         const float* __restrict__ init, int N,
+                                                         int P, int Q, int nc, long long total) {
     const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (e >= total) return;
     const int NP = N * P;
@@ -208,7 +209,7 @@ __global__ void __launch_bounds__(256) state_pass_kernel(const float* __restrict
         sb[u] = u < nc ? sp[(size_t)u * NP] : 0.f;
         cb[u] = u < nc ? ce[(size_t)u * cstep] : 0.f;
     }
-    float hval = 0.f;
+    float hval = init ? init[bh * NP + r] : 0.f;  // the state entering chunk 0
     for (int k0 = 0; k0 < nc; k0 += kPassGroup) {
         float s[kPassGroup], c[kPassGroup];
 #pragma unroll
@@ -234,13 +235,13 @@ __global__ void __launch_bounds__(256) state_pass_kernel(const float* __restrict
 }
 
 cudaError_t launch_state_pass(const Dims& d, const float* cum, float* states, float* fin,
-                              cudaStream_t st) {
+                              const float* init, cudaStream_t st) {
     const long long total = (long long)d.B * d.H * d.N * d.P;
     const unsigned blocks = (unsigned)((total + 255) / 256);
     if (d.diag)
-        state_pass_kernel<true><<<blocks, 256, 0, st>>>(cum, states, fin, d.N, d.P, d.Q, d.nc, total);
+        state_pass_kernel<true><<<blocks, 256, 0, st>>>(cum, states, fin, init, d.N, d.P, d.Q, d.nc, total);
     else
-        state_pass_kernel<false><<<blocks, 256, 0, st>>>(cum, states, fin, d.N, d.P, d.Q, d.nc, total);
+        state_pass_kernel<false><<<blocks, 256, 0, st>>>(cum, states, fin, init, d.N, d.P, d.Q, d.nc, total);
     return cudaGetLastError();
 }
 

@@ -109,7 +109,7 @@ bool g_fused_seen[kMaxDevices] = {};
 
 ssd_status run_modular(const Dims& d0, const void* x, const float* a, const void* Bm,
                        const void* Cm, const float* D, void* y, float* fin, const Workspace& w,
-                       cudaStream_t st, bool allow_tc) {
+                       cudaStream_t st, bool allow_tc, const float* init) {
     const Dims d = allow_tc ? modular_dims(d0) : d0;
     cudaError_t e = ssd::launch_chunk_cumsum(d, a, w.cum, st);
     if (e != cudaSuccess) return SSD_ERR_CUDA;
@@ -117,7 +117,7 @@ ssd_status run_modular(const Dims& d0, const void* x, const float* a, const void
     e = tc_state ? ssd::launch_chunk_state_tc(d, x, Bm, w.cum, w.states, st)
                  : ssd::launch_chunk_state_simt(d, x, Bm, w.cum, w.states, st);
     if (e != cudaSuccess) return SSD_ERR_CUDA;
-    e = ssd::launch_state_pass(d, w.cum, w.states, fin, st);
+    e = ssd::launch_state_pass(d, w.cum, w.states, fin, init, st);
     if (e != cudaSuccess) return SSD_ERR_CUDA;
     const bool tc_scan = allow_tc && ssd::chunk_scan_tc_supported(d);
     e = tc_scan ? ssd::launch_chunk_scan_tc(d, x, Bm, Cm, w.cum, w.states, D, y, st)
@@ -130,13 +130,14 @@ ssd_status run_modular(const Dims& d0, const void* x, const float* a, const void
 namespace ssd {
 cudaError_t launch_fused_ordered(const Dims& d, const void* x, const float* a, const void* Bm,
                                  const void* Cm, const float* D, void* y, float* fin, float* ring,
-                                 unsigned* flags, int* status, bool test_stall, cudaStream_t st) {
+                                 unsigned* flags, int* status, bool test_stall, cudaStream_t st,
+                                 const float* init) {
     cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
     if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) return cudaErrorInvalidValue;
     int dev = 0;
     if (cap != cudaStreamCaptureStatusNone || cudaGetDevice(&dev) != cudaSuccess || dev < 0 ||
         dev >= kMaxDevices)
-        return launch_fused_tc(d, x, a, Bm, Cm, D, y, fin, ring, flags, status, test_stall, st);
+        return launch_fused_tc(d, x, a, Bm, Cm, D, y, fin, ring, flags, status, test_stall, st, init);
     std::lock_guard<std::mutex> lock(g_fused_mu);
     if (!g_fused_done[dev]) {
         cudaError_t e = cudaEventCreateWithFlags(&g_fused_done[dev], cudaEventDisableTiming);
@@ -146,7 +147,7 @@ cudaError_t launch_fused_ordered(const Dims& d, const void* x, const float* a, c
         cudaError_t e = cudaStreamWaitEvent(st, g_fused_done[dev], 0);
         if (e != cudaSuccess) return e;
     }
-    cudaError_t e = launch_fused_tc(d, x, a, Bm, Cm, D, y, fin, ring, flags, status, test_stall, st);
+    cudaError_t e = launch_fused_tc(d, x, a, Bm, Cm, D, y, fin, ring, flags, status, test_stall, st, init);
     if (e != cudaSuccess) return e;
     e = cudaEventRecord(g_fused_done[dev], st);
     if (e == cudaSuccess) g_fused_seen[dev] = true;
@@ -196,15 +197,16 @@ int ssd_auto_path(const ssd_shape* shape) {
     return SSD_PATH_MODULAR;
 }
 
-ssd_status ssd_forward_path(const ssd_shape* shape, const void* x, const float* a, const void* Bm,
-                            const void* Cm, const float* D, void* y, float* final_state,
-                            void* workspace, size_t ws_bytes, ssd_stream stream, unsigned path,
-                            unsigned flags) {
+ssd_status ssd_forward_init(const ssd_shape* shape, const void* x, const float* a, const void* Bm,
+                            const void* Cm, const float* D, const float* initial_state, void* y,
+                            float* final_state, void* workspace, size_t ws_bytes,
+                            ssd_stream stream, unsigned path, unsigned flags) {
     ssd_status st = check_shape(shape);
     if (st != SSD_OK) return st;
     if (!x || !a || !Bm || !Cm || !y) return SSD_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(a) || !aligned16(Bm) || !aligned16(Cm) || !aligned16(y) ||
-        (D && !aligned16(D)) || (final_state && !aligned16(final_state)))
+        (D && !aligned16(D)) || (final_state && !aligned16(final_state)) ||
+        (initial_state && !aligned16(initial_state)))
         return SSD_ERR_INVALID_ARG;
     if ((flags & ~SSD_FLAG_TEST_STALL) != 0) return SSD_ERR_INVALID_ARG;
     if (path > SSD_PATH_FUSED) return SSD_ERR_INVALID_ARG;
@@ -220,15 +222,24 @@ ssd_status ssd_forward_path(const ssd_shape* shape, const void* x, const float* 
     if (path == SSD_PATH_AUTO) path = (unsigned)ssd_auto_path(shape);
     switch (path) {
         case SSD_PATH_SIMT:
-            return run_modular(d, x, a, Bm, Cm, D, y, final_state, w, cs, false);
+            return run_modular(d, x, a, Bm, Cm, D, y, final_state, w, cs, false, initial_state);
         case SSD_PATH_FUSED:
             return cuda_status(ssd::launch_fused_ordered(d, x, a, Bm, Cm, D, y, final_state, w.ring,
-                                                    w.flags, w.ctrl,
-                                                    (flags & SSD_FLAG_TEST_STALL) != 0, cs));
+                                                         w.flags, w.ctrl,
+                                                         (flags & SSD_FLAG_TEST_STALL) != 0, cs,
+                                                         initial_state));
         case SSD_PATH_MODULAR:
         default:
-            return run_modular(d, x, a, Bm, Cm, D, y, final_state, w, cs, true);
+            return run_modular(d, x, a, Bm, Cm, D, y, final_state, w, cs, true, initial_state);
     }
+}
+
+ssd_status ssd_forward_path(const ssd_shape* shape, const void* x, const float* a, const void* Bm,
+                            const void* Cm, const float* D, void* y, float* final_state,
+                            void* workspace, size_t ws_bytes, ssd_stream stream, unsigned path,
+                            unsigned flags) {
+    return ssd_forward_init(shape, x, a, Bm, Cm, D, nullptr, y, final_state, workspace, ws_bytes,
+                            stream, path, flags);
 }
 
 ssd_status ssd_forward(const ssd_shape* shape, const void* x, const float* a, const void* Bm,
@@ -347,7 +358,7 @@ ssd_status ssd_state_pass(const ssd_shape* shape, const float* cum, float* state
         (final_state && !aligned16(final_state)))
         return SSD_ERR_INVALID_ARG;
     return cuda_status(
-        ssd::launch_state_pass(dims_of(shape), cum, states, final_state, (cudaStream_t)stream));
+        ssd::launch_state_pass(dims_of(shape), cum, states, final_state, nullptr, (cudaStream_t)stream));
 }
 
 static ssd_status scan_common(const ssd_shape* shape, const void* x, const void* Bm,

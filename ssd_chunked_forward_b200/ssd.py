@@ -25,7 +25,7 @@ EXPORTS = [
     "ssd_status_string", "ssd_workspace_size", "ssd_path_supported", "ssd_forward",
     "ssd_forward_path", "ssd_device_status", "ssd_chunk_cumsum", "ssd_chunk_state",
     "ssd_state_pass", "ssd_chunk_scan", "ssd_diag_scan", "ssd_forward_host_bytes",
-    "ssd_forward_host", "ssd_forward_noalloc", "ssd_auto_path",
+    "ssd_forward_host", "ssd_forward_noalloc", "ssd_auto_path", "ssd_forward_init",
 ]
 
 
@@ -65,6 +65,8 @@ def load(path: str = LIB_PATH):
     lib.ssd_auto_path.restype = ctypes.c_int
     lib.ssd_forward.argtypes = [sp, vp, fp, vp, vp, fp, vp, fp, vp, sz, vp]
     lib.ssd_forward_path.argtypes = [sp, vp, fp, vp, vp, fp, vp, fp, vp, sz, vp, ctypes.c_uint, ctypes.c_uint]
+    lib.ssd_forward_init.argtypes = [sp, vp, fp, vp, vp, fp, fp, vp, fp, vp, sz, vp, ctypes.c_uint,
+                                     ctypes.c_uint]
     lib.ssd_device_status.argtypes = [vp, vp]
     lib.ssd_chunk_cumsum.argtypes = [sp, fp, fp, vp]
     lib.ssd_chunk_state.argtypes = [sp, vp, vp, fp, fp, vp, ctypes.c_uint]
@@ -75,7 +77,8 @@ def load(path: str = LIB_PATH):
     lib.ssd_forward_host_bytes.restype = sz
     lib.ssd_forward_host.argtypes = [sp, vp, fp, vp, vp, fp, vp, fp, vp, sz, vp]
     lib.ssd_forward_noalloc.argtypes = [sp, vp, fp, vp, vp, fp, vp, fp, vp]
-    for name in ("ssd_forward_noalloc", "ssd_forward", "ssd_forward_path", "ssd_device_status", "ssd_chunk_cumsum",
+    for name in ("ssd_forward_noalloc", "ssd_forward", "ssd_forward_path", "ssd_forward_init",
+                 "ssd_device_status", "ssd_chunk_cumsum",
                  "ssd_chunk_state", "ssd_state_pass", "ssd_chunk_scan", "ssd_diag_scan",
                  "ssd_forward_host"):
         getattr(lib, name).restype = ctypes.c_int
@@ -153,13 +156,17 @@ def _check_inputs(x, a, Bm, Cm, D):
 
 
 def forward(x, a, Bm, Cm, D=None, chunk=256, *, y=None, final_state=None, want_final=True,
-            workspace=None, path=PATH_AUTO, flags=0, stream=None):
+            workspace=None, path=PATH_AUTO, flags=0, stream=None, initial_state=None):
     """y[B,T,H,P] (and final state [B,H,N,P] fp32) of the chunked SSD forward.
 
     x [B,T,H,P], Bm/Cm [B,T,G,N] (float32 or bfloat16, same dtype), a [B,T,H]
-    or [B,T,H,N] float32 log-decays, D [H] float32 or None.  Asynchronous on
-    the current torch stream (or ``stream``)."""
+    or [B,T,H,N] float32 log-decays, D [H] float32 or None, initial_state
+    [B,H,N,P] float32 or None (zero).  Asynchronous on the current torch
+    stream (or ``stream``)."""
     _check_inputs(x, a, Bm, Cm, D)
+    if initial_state is not None and (initial_state.dtype != torch.float32 or not initial_state.is_cuda
+                                      or not initial_state.is_contiguous()):
+        raise ValueError("initial_state must be a contiguous float32 CUDA tensor")
     shape = shape_of(x, a, Bm, chunk)
     B, T, H, P = x.shape
     N = Bm.shape[3]
@@ -169,6 +176,15 @@ def forward(x, a, Bm, Cm, D=None, chunk=256, *, y=None, final_state=None, want_f
         final_state = torch.empty((B, H, N, P), dtype=torch.float32, device=x.device)
     if workspace is None:
         workspace = alloc_workspace(shape, x.device)
+    if initial_state is not None:
+        if tuple(initial_state.shape) != (B, H, N, P):
+            raise ValueError("initial_state must be [B,H,N,P]")
+        code = load().ssd_forward_init(ctypes.byref(shape), _ptr(x), _ptr(a), _ptr(Bm), _ptr(Cm),
+                                       _ptr(D), _ptr(initial_state), _ptr(y), _ptr(final_state),
+                                       _ptr(workspace), workspace.numel(), _stream(stream), int(path),
+                                       int(flags))
+        _check(code, "ssd_forward_init")
+        return y, final_state
     code = load().ssd_forward_path(ctypes.byref(shape), _ptr(x), _ptr(a), _ptr(Bm), _ptr(Cm),
                                    _ptr(D), _ptr(y), _ptr(final_state), _ptr(workspace),
                                    workspace.numel(), _stream(stream), int(path), int(flags))

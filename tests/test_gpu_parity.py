@@ -294,3 +294,59 @@ def test_fused_on_two_streams():
         assert ssd.device_status(wss[s], streams[s]) == ssd.SSD_OK
     for y, f in outs:
         assert torch.equal(y, y_ref) and torch.equal(f, f_ref)
+
+
+INIT_CASES = [
+    small_case(B=2, T=1024, H=8, P=64, N=128, G=2, chunk=256, dtype="bf16", seed=61),
+    small_case(B=1, T=384, H=5, P=64, N=128, G=1, chunk=128, dtype="bf16", seed=62),
+    small_case(B=1, T=150, H=2, P=70, N=33, G=2, chunk=30, dtype="f32", seed=63),
+    small_case(B=2, T=256, H=2, P=64, N=64, G=1, chunk=128, dtype="bf16", a_per_state=True, seed=64),
+]
+
+
+@pytest.mark.parametrize("w", INIT_CASES, ids=_ids(INIT_CASES))
+@pytest.mark.parametrize("path", _paths(), ids=["simt", "modular", "auto", "fused"])
+def test_initial_state_matches_oracle(w, path):
+    """ssd_forward_init: every chain starts from a given state h_{-1}; y and the
+    final state match the oracle's recurrence started from the same state."""
+    inp = generate(w)
+    dev = to_dev(inp)
+    shape = ssd.shape_of(dev["x"], dev["a"], dev["Bm"], w.chunk)
+    if not ssd.path_supported(shape, path):
+        pytest.skip("path does not serve this shape")
+    g = torch.Generator().manual_seed(w.seed + 7)
+    h0 = torch.randn((w.B, w.H, w.N, w.P), generator=g, dtype=torch.float64)
+    y, fin = ssd.forward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], dev["D"], w.chunk, path=path,
+                         initial_state=h0.to(torch.float32).cuda())
+    torch.cuda.synchronize()
+    prob = O.Problem(*(inp[k].to(torch.float64).numpy() for k in ("x", "a", "Bm", "Cm", "D")))
+    ref = O.recurrence(prob, initial=h0.to(torch.float32).to(torch.float64).numpy())
+    yr = ref["y"].reshape(w.B, w.H, w.T, w.P).transpose(0, 2, 1, 3)
+    ey = rel_err(y.float().cpu().numpy().astype(np.float64), yr)
+    ef = rel_err(fin.cpu().numpy().astype(np.float64), ref["final"].reshape(w.B, w.H, w.N, w.P))
+    tol = tol_for(w)
+    assert ey <= tol, f"y rel err {ey:.3e}"
+    assert ef <= tol, f"final rel err {ef:.3e}"
+
+
+@pytest.mark.parametrize("path", [ssd.PATH_AUTO, ssd.PATH_FUSED, ssd.PATH_MODULAR], ids=["auto", "fused", "modular"])
+def test_split_sequence_resumes(path):
+    """A sequence run in two calls -- the second from the first's final state,
+    passed in place (initial_state aliases final_state) -- gives the one-call
+    result up to rounding."""
+    w = small_case(B=2, T=2048, H=8, P=64, N=128, G=1, chunk=256, dtype="bf16", seed=65)
+    inp = generate(w)
+    dev = to_dev(inp)
+    y_full, f_full = ssd.forward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], dev["D"], w.chunk, path=path)
+    t1 = 768
+    part = lambda t, sl: t[:, sl].contiguous()
+    y1, f1 = ssd.forward(part(dev["x"], slice(0, t1)), part(dev["a"], slice(0, t1)),
+                         part(dev["Bm"], slice(0, t1)), part(dev["Cm"], slice(0, t1)), dev["D"], w.chunk,
+                         path=path)
+    y2, f2 = ssd.forward(part(dev["x"], slice(t1, None)), part(dev["a"], slice(t1, None)),
+                         part(dev["Bm"], slice(t1, None)), part(dev["Cm"], slice(t1, None)), dev["D"],
+                         w.chunk, path=path, initial_state=f1, final_state=f1)
+    torch.cuda.synchronize()
+    y = torch.cat([y1, y2], dim=1).float()
+    assert rel_err(y.cpu().numpy(), y_full.float().cpu().numpy()) <= TOL_BF16
+    assert rel_err(f1.cpu().numpy(), f_full.cpu().numpy()) <= TOL_BF16
