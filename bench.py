@@ -323,6 +323,52 @@ def time_steps_split(w, dev, flush, reps, impl):
     return {n: statistics.mean(v) for n, v in times.items()}
 
 
+def run_decode(args, device):
+    """The decode step (ssd_decode_step) on the workload's batch and heads: one
+    token per (batch, head) chain, the fp32 state read and written in place.
+    Algorithmic bytes: the state twice plus x, y, a, B and C of one token."""
+    w = WORKLOADS[args.workload]
+    g = torch.Generator().manual_seed(w.seed + 500)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    x = torch.randn((w.B, w.H, w.P), generator=g).to(dt).to(device)
+    a = (-torch.rand((w.B, w.H) + ((w.N,) if w.a_per_state else ()), generator=g)).to(device)
+    Bm = (torch.randn((w.B, w.G, w.N), generator=g) / w.N ** 0.5).to(dt).to(device)
+    Cm = (torch.randn((w.B, w.G, w.N), generator=g) / w.N ** 0.5).to(dt).to(device)
+    D = torch.randn((w.H,), generator=g).to(device)
+    state = torch.randn((w.B, w.H, w.N, w.P), generator=g).to(device)
+    y = torch.empty_like(x)
+    scratch = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    st = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        scratch.fill_(1)
+        ssd.decode_step(x, a, Bm, Cm, D, state, y=y)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for e0, e1 in ev:
+        scratch.fill_(1)
+        e0.record(st)
+        ssd.decode_step(x, a, Bm, Cm, D, state, y=y)
+        e1.record(st)
+    torch.cuda.synchronize()
+    ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev)
+    el = 2 if w.dtype == "bf16" else 4
+    byts = (2 * w.B * w.H * w.N * w.P * 4 + 2 * w.B * w.H * w.P * el
+            + w.B * w.H * (w.N if w.a_per_state else 1) * 4 + 2 * w.B * w.G * w.N * el + w.H * 4)
+    peaks, src = load_peaks()
+    achieved = byts / (ms / 1e3) / 1e9
+    print(json.dumps({
+        "metric": "SSD decode step tokens/s (one token per batch row)", "value": w.B / (ms / 1e3),
+        "unit": "tokens/s", "ms_per_step": ms, "steps": args.steps, "warmup": args.warmup,
+        "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name + "_decode", "B": w.B, "H": w.H, "P": w.P, "N": w.N, "G": w.G,
+                   "a_per_state": w.a_per_state, "l2": "flushed (256 MB write) before every step"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "algorithmic_bytes_per_launch": byts,
+                     "kernel": "ssd_decode_step", "peak_source": f"{src} (hbm_gbs)"},
+        "gpu_launches": args.steps}))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -335,6 +381,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--B", type=int, default=None, help="override the batch (profiling small cases)")
     ap.add_argument("--T", type=int, default=None, help="override the sequence length")
+    ap.add_argument("--decode", action="store_true",
+                    help="time the recurrent decode step (one token per chain) on the workload's "
+                         "batch and heads instead of the forward; prints its own JSON line")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -347,6 +396,8 @@ def main():
 
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
+    if args.decode:
+        return run_decode(args, device)
     dist = None
     if world > 1:
         import torch.distributed as dist

@@ -237,6 +237,24 @@ ssd_status ssd_diag_scan(const ssd_shape* shape, const void* x, const void* Bm, 
                          const float* cum, const float* Hin, const float* D, void* y,
                          ssd_stream stream, unsigned impl);
 
+/* One recurrent step for a batch of single tokens -- the inference (decode)
+ * form of the same operator: per (batch b, head h),
+ *     h <- exp(a) o h + B x^T,     y = C^T h + D[h] x
+ * ("State Space Models and Mamba ...", llms.blog, "The Duality of Inference
+ * and Training": the recurrent view used to generate token by token; the
+ * state is the one ssd_forward* returned as final_state, so a prefill by
+ * ssd_forward then steps here continue the same sequence).
+ * shape: T == 1 and chunk == 1; other fields as for ssd_forward.
+ * x[B][H][P] and Bm, Cm[B][G][N] (dtype of the shape); a[B][H] (or
+ * [B][H][N] when a_per_state) fp32 log-decays; D[H] fp32 or NULL;
+ * state[B][H][N][P] fp32, updated in place; y[B][H][P] (dtype).  Device
+ * pointers, 16-byte aligned; asynchronous on `stream`.  Returns
+ * SSD_ERR_INVALID_ARG for a bad shape or pointer, SSD_ERR_CUDA if the launch
+ * fails. */
+ssd_status ssd_decode_step(const ssd_shape* shape, const void* x, const float* a, const void* Bm,
+                           const void* Cm, const float* D, float* state, void* y,
+                           ssd_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -24,6 +24,11 @@ cudaError_t launch_chunk_scan_simt(const Dims& d, const void* x, const void* Bm,
                                    const float* cum, const float* Hin, const float* D, void* y,
                                    cudaStream_t st);
 
+// one recurrent step for single tokens (decode): state[B,H,N,P] updated in place
+cudaError_t launch_decode_step(const Dims& d, const void* x, const float* a, const void* Bm,
+                               const void* Cm, const float* D, float* state, void* y,
+                               cudaStream_t st);
+
 // ---- tensor-core kernels (tcgen05 + TMEM + TMA) ----------------------------
 bool chunk_state_tc_supported(const Dims& d);
 cudaError_t launch_chunk_state_tc(const Dims& d, const void* x, const void* Bm, const float* cum,

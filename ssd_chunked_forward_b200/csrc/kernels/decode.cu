@@ -1,0 +1,102 @@
+// decode.cu -- one recurrent step for a batch of single tokens.
+//
+// Per (batch b, head h): h <- exp(a) o h + B x^T, y = C^T h + D x (the
+// recurrent view of the operator, "State Space Models and Mamba ...",
+// llms.blog, "The Duality of Inference and Training").  The step is bound by
+// reading and writing the fp32 state: one block per (b, h) streams its N x P
+// state once, thread (p, n-slice) owning column p of a slice of the rows, so
+// every warp access is a contiguous row segment; y is reduced over the
+// n-slices in shared memory.
+#include "../common.cuh"
+#include "../kernels.h"
+
+namespace ssd {
+namespace {
+
+constexpr int kDecThreads = 512;
+
+template <typename T, bool DIAG>
+__global__ void __launch_bounds__(kDecThreads) decode_step_kernel(
+    const T* __restrict__ x, const float* __restrict__ a, const T* __restrict__ Bm,
+    const T* __restrict__ Cm, const float* __restrict__ D, float* __restrict__ state,
+    T* __restrict__ y, int H, int P, int G, int N) {
+    extern __shared__ float sm[];
+    float* sB = sm;          // [N]
+    float* sC = sB + N;      // [N]
+    float* sE = sC + N;      // [N] exp(a) per state index (scalar decay: all equal)
+    float* sX = sE + N;      // [P]
+    float* sY = sX + P;      // [row slices][lanes] partial sums of y
+    const int bh = blockIdx.x, b = bh / H, h = bh % H, g = h / (H / G);
+    const int tid = threadIdx.x;
+    const float* ab = a + (size_t)bh * (DIAG ? N : 1);
+    for (int n = tid; n < N; n += kDecThreads) {
+        sB[n] = to_f32(Bm[((size_t)b * G + g) * N + n]);
+        sC[n] = to_f32(Cm[((size_t)b * G + g) * N + n]);
+        sE[n] = expf(DIAG ? ab[n] : ab[0]);
+    }
+    for (int p = tid; p < P; p += kDecThreads) sX[p] = to_f32(x[(size_t)bh * P + p]);
+    __syncthreads();
+    // column p = tid % pw (pw = min(P, threads) lanes per row), rows n = slice,
+    // slice + ns, ...; each thread loads a batch of its rows before updating any,
+    // so a block has its whole state in flight at once (one memory latency, not
+    // one per row)
+    constexpr int kRows = 16;
+    const int pw = P < kDecThreads ? P : kDecThreads;
+    const int ns = kDecThreads / pw;  // row slices
+    float* hs = state + (size_t)bh * N * P;
+    for (int p0 = 0; p0 < P; p0 += pw) {
+        const int p = p0 + tid % pw, sl = tid / pw;
+        float acc = 0.f;
+        if (sl < ns && p < P) {
+            const float xp = sX[p];
+            for (int n0 = sl; n0 < N; n0 += kRows * ns) {
+                float hv[kRows];
+#pragma unroll
+                for (int r = 0; r < kRows; ++r) {
+                    const int n = n0 + r * ns;
+                    hv[r] = n < N ? hs[(size_t)n * P + p] : 0.f;
+                }
+#pragma unroll
+                for (int r = 0; r < kRows; ++r) {
+                    const int n = n0 + r * ns;
+                    if (n < N) {
+                        const float hn = fmaf(sE[n], hv[r], sB[n] * xp);
+                        hs[(size_t)n * P + p] = hn;
+                        acc = fmaf(sC[n], hn, acc);
+                    }
+                }
+            }
+        }
+        if (sl < ns) sY[sl * pw + tid % pw] = acc;
+        __syncthreads();
+        if (tid < pw && p0 + tid < P) {
+            float s = 0.f;
+            for (int k = 0; k < ns; ++k) s += sY[k * pw + tid];
+            const int pp = p0 + tid;
+            y[(size_t)bh * P + pp] = from_f32<T>(s + (D ? D[h] : 0.f) * sX[pp]);
+        }
+        __syncthreads();
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_decode_step(const Dims& d, const void* x, const float* a, const void* Bm,
+                               const void* Cm, const float* D, float* state, void* y,
+                               cudaStream_t st) {
+    const int pw = d.P < kDecThreads ? d.P : kDecThreads;
+    const size_t smem = (size_t)(3 * d.N + d.P + (kDecThreads / pw) * pw) * sizeof(float);
+    const unsigned grid = (unsigned)(d.B * d.H);
+#define SSD_DEC_LAUNCH(TT, DG)                                                                    \
+    decode_step_kernel<TT, DG><<<grid, kDecThreads, smem, st>>>(                                  \
+        (const TT*)x, a, (const TT*)Bm, (const TT*)Cm, D, state, (TT*)y, d.H, d.P, d.G, d.N)
+    if (d.bf16) {
+        if (d.diag) SSD_DEC_LAUNCH(__nv_bfloat16, true); else SSD_DEC_LAUNCH(__nv_bfloat16, false);
+    } else {
+        if (d.diag) SSD_DEC_LAUNCH(float, true); else SSD_DEC_LAUNCH(float, false);
+    }
+#undef SSD_DEC_LAUNCH
+    return cudaGetLastError();
+}
+
+}  // namespace ssd

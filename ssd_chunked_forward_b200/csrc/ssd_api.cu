@@ -393,4 +393,16 @@ ssd_status ssd_diag_scan(const ssd_shape* shape, const void* x, const void* Bm, 
     return scan_common(shape, x, Bm, Cm, cum, Hin, D, y, stream, impl, true);
 }
 
+ssd_status ssd_decode_step(const ssd_shape* shape, const void* x, const float* a, const void* Bm,
+                           const void* Cm, const float* D, float* state, void* y,
+                           ssd_stream stream) {
+    if (check_shape(shape) != SSD_OK || shape->T != 1 || shape->chunk != 1) return SSD_ERR_INVALID_ARG;
+    if (!x || !a || !Bm || !Cm || !state || !y) return SSD_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(a) || !aligned16(Bm) || !aligned16(Cm) || !aligned16(state) ||
+        !aligned16(y) || (D && !aligned16(D)))
+        return SSD_ERR_INVALID_ARG;
+    return cuda_status(ssd::launch_decode_step(dims_of(shape), x, a, Bm, Cm, D, state, y,
+                                               (cudaStream_t)stream));
+}
+
 }  // extern "C"

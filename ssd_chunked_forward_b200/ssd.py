@@ -26,6 +26,7 @@ EXPORTS = [
     "ssd_forward_path", "ssd_device_status", "ssd_chunk_cumsum", "ssd_chunk_state",
     "ssd_state_pass", "ssd_chunk_scan", "ssd_diag_scan", "ssd_forward_host_bytes",
     "ssd_forward_host", "ssd_forward_noalloc", "ssd_auto_path", "ssd_forward_init",
+    "ssd_decode_step",
 ]
 
 
@@ -77,8 +78,9 @@ def load(path: str = LIB_PATH):
     lib.ssd_forward_host_bytes.restype = sz
     lib.ssd_forward_host.argtypes = [sp, vp, fp, vp, vp, fp, vp, fp, vp, sz, vp]
     lib.ssd_forward_noalloc.argtypes = [sp, vp, fp, vp, vp, fp, vp, fp, vp]
+    lib.ssd_decode_step.argtypes = [sp, vp, fp, vp, vp, fp, fp, vp, vp]
     for name in ("ssd_forward_noalloc", "ssd_forward", "ssd_forward_path", "ssd_forward_init",
-                 "ssd_device_status", "ssd_chunk_cumsum",
+                 "ssd_device_status", "ssd_chunk_cumsum", "ssd_decode_step",
                  "ssd_chunk_state", "ssd_state_pass", "ssd_chunk_scan", "ssd_diag_scan",
                  "ssd_forward_host"):
         getattr(lib, name).restype = ctypes.c_int
@@ -261,3 +263,28 @@ def forward_noalloc(x, a, Bm, Cm, D=None, chunk=256, *, y=None, final_state=None
                                       _ptr(D), _ptr(y), _ptr(final_state), _stream(stream)),
            "ssd_forward_noalloc")
     return y, final_state
+
+
+def decode_step(x, a, Bm, Cm, D, state, *, y=None, stream=None):
+    """One recurrent step for a batch of single tokens, in place on ``state``.
+
+    x [B,H,P], Bm/Cm [B,G,N] (float32 or bfloat16), a [B,H] or [B,H,N] float32
+    log-decays, D [H] float32 or None, state [B,H,N,P] float32 (updated).
+    Returns y [B,H,P]."""
+    for name, t in (("x", x), ("a", a), ("Bm", Bm), ("Cm", Cm), ("state", state)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if a.dtype != torch.float32 or state.dtype != torch.float32:
+        raise ValueError("a and state must be float32")
+    if Bm.dtype != x.dtype or Cm.dtype != x.dtype:
+        raise ValueError("x, Bm, Cm must share dtype")
+    B, H, P = x.shape
+    G, N = Bm.shape[1], Bm.shape[2]
+    if tuple(state.shape) != (B, H, N, P):
+        raise ValueError("state must be [B,H,N,P]")
+    shape = make_shape(B, 1, H, P, G, N, 1, a.dim() == 3, x.dtype)
+    if y is None:
+        y = torch.empty_like(x)
+    _check(load().ssd_decode_step(ctypes.byref(shape), _ptr(x), _ptr(a), _ptr(Bm), _ptr(Cm), _ptr(D),
+                                  _ptr(state), _ptr(y), _stream(stream)), "ssd_decode_step")
+    return y

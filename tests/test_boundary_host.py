@@ -139,3 +139,18 @@ def test_auto_path_choice(lib):
     assert ssd.auto_path(ssd.make_shape(4, 8192, 80, 64, 1, 128, 256, dtype="f32")) == ssd.PATH_MODULAR
     assert ssd.auto_path(ssd.make_shape(4, 4096, 16, 64, 1, 64, 128, a_per_state=True)) == ssd.PATH_MODULAR
     assert ssd.auto_path(ssd.make_shape(1, 100, 2, 64, 1, 128, 64)) == -1  # T % chunk != 0
+
+
+def test_decode_step_validates(lib):
+    """The decode step takes T == 1 and chunk == 1 and rejects null or
+    misaligned pointers before any launch."""
+    good = ssd.make_shape(2, 1, 4, 64, 1, 128, 1)
+    p = ctypes.c_void_p(1 << 20)  # never dereferenced: every call below fails validation
+    f = ctypes.cast(p, ctypes.POINTER(ctypes.c_float))
+    def call(shape, x=p, a=f, bm=p, cm=p, st=f, y=p):
+        return lib.ssd_decode_step(ctypes.byref(shape), x, a, bm, cm, None, st, y, None)
+    assert call(ssd.make_shape(2, 4, 4, 64, 1, 128, 1)) == ssd.SSD_ERR_INVALID_ARG   # T != 1
+    assert call(ssd.make_shape(2, 1, 4, 64, 1, 128, 4)) == ssd.SSD_ERR_INVALID_ARG   # chunk != 1
+    assert call(good, x=None) == ssd.SSD_ERR_INVALID_ARG
+    assert call(good, st=None) == ssd.SSD_ERR_INVALID_ARG
+    assert call(good, y=ctypes.c_void_p((1 << 20) + 4)) == ssd.SSD_ERR_INVALID_ARG  # misaligned

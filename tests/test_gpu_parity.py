@@ -350,3 +350,52 @@ def test_split_sequence_resumes(path):
     y = torch.cat([y1, y2], dim=1).float()
     assert rel_err(y.cpu().numpy(), y_full.float().cpu().numpy()) <= TOL_BF16
     assert rel_err(f1.cpu().numpy(), f_full.cpu().numpy()) <= TOL_BF16
+
+
+DECODE_CASES = [
+    small_case(B=3, T=1, H=8, P=64, N=128, G=2, chunk=1, dtype="bf16", seed=71),
+    small_case(B=2, T=1, H=3, P=70, N=33, G=3, chunk=1, dtype="f32", seed=72),
+    small_case(B=2, T=1, H=4, P=64, N=64, G=1, chunk=1, dtype="bf16", a_per_state=True, seed=73),
+    small_case(B=1, T=1, H=2, P=250, N=20, G=1, chunk=1, dtype="f32", seed=74),
+]
+
+
+@pytest.mark.parametrize("w", DECODE_CASES, ids=_ids(DECODE_CASES))
+def test_decode_step_matches_oracle(w):
+    """One decode step from a given state equals one step of the oracle's
+    recurrence from that state (y and the updated state)."""
+    inp = generate(w)
+    dev = to_dev(inp)
+    g = torch.Generator().manual_seed(w.seed + 3)
+    h0 = torch.randn((w.B, w.H, w.N, w.P), generator=g).to(torch.float32)
+    state = h0.cuda()
+    y = ssd.decode_step(dev["x"][:, 0].contiguous(), dev["a"][:, 0].contiguous(),
+                        dev["Bm"][:, 0].contiguous(), dev["Cm"][:, 0].contiguous(), dev["D"], state)
+    torch.cuda.synchronize()
+    prob = O.Problem(*(inp[k].to(torch.float64).numpy() for k in ("x", "a", "Bm", "Cm", "D")))
+    ref = O.recurrence(prob, initial=h0.to(torch.float64).numpy())
+    yr = ref["y"].reshape(w.B, w.H, 1, w.P)[:, :, 0]
+    tol = tol_for(w)
+    assert rel_err(y.float().cpu().numpy().astype(np.float64), yr) <= tol
+    assert rel_err(state.cpu().numpy().astype(np.float64), ref["final"].reshape(w.B, w.H, w.N, w.P)) <= tol
+
+
+def test_prefill_then_decode_continues_the_sequence():
+    """ssd_forward over the first T0 tokens, then one decode step per token
+    from its final state, reproduces the forward over all tokens."""
+    w = small_case(B=2, T=512 + 16, H=4, P=64, N=128, G=1, chunk=16, dtype="bf16", seed=75)
+    inp = generate(w)
+    dev = to_dev(inp)
+    T0 = 512
+    y_all, f_all = ssd.forward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], dev["D"], 16)
+    _, state = ssd.forward(dev["x"][:, :T0].contiguous(), dev["a"][:, :T0].contiguous(),
+                           dev["Bm"][:, :T0].contiguous(), dev["Cm"][:, :T0].contiguous(), dev["D"], 256)
+    ys = []
+    for t in range(T0, w.T):
+        ys.append(ssd.decode_step(dev["x"][:, t].contiguous(), dev["a"][:, t].contiguous(),
+                                  dev["Bm"][:, t].contiguous(), dev["Cm"][:, t].contiguous(), dev["D"],
+                                  state))
+    torch.cuda.synchronize()
+    y_dec = torch.stack(ys, dim=1).float().cpu().numpy()
+    assert rel_err(y_dec, y_all[:, T0:].float().cpu().numpy()) <= TOL_BF16
+    assert rel_err(state.cpu().numpy(), f_all.cpu().numpy()) <= TOL_BF16
