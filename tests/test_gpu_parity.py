@@ -399,3 +399,39 @@ def test_prefill_then_decode_continues_the_sequence():
     y_dec = torch.stack(ys, dim=1).float().cpu().numpy()
     assert rel_err(y_dec, y_all[:, T0:].float().cpu().numpy()) <= TOL_BF16
     assert rel_err(state.cpu().numpy(), f_all.cpu().numpy()) <= TOL_BF16
+
+
+@pytest.mark.parametrize("path", [ssd.PATH_FUSED, ssd.PATH_MODULAR], ids=["fused", "modular"])
+def test_cuda_graph_capture_and_replay(path):
+    """The forward records into a CUDA graph (workspace reset, TMA descriptors
+    and launches all captured) and each replay computes on the inputs' current
+    contents, matching an eager call bit for bit."""
+    w = small_case(B=2, T=1024, H=8, P=64, N=128, G=1, chunk=256, dtype="bf16", seed=81)
+    inp = generate(w)
+    dev = to_dev(inp)
+    shape = ssd.shape_of(dev["x"], dev["a"], dev["Bm"], w.chunk)
+    ws = ssd.alloc_workspace(shape)
+    y = torch.empty_like(dev["x"])
+    fin = torch.empty((w.B, w.H, w.N, w.P), dtype=torch.float32, device="cuda")
+    run = lambda: ssd.forward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], dev["D"], w.chunk, y=y,
+                              final_state=fin, workspace=ws, path=path)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        run()  # warm-up outside the capture
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        run()
+    for seed in (82, 83):
+        new = generate(small_case(B=2, T=1024, H=8, P=64, N=128, G=1, chunk=256, dtype="bf16", seed=seed))
+        for k in dev:
+            dev[k].copy_(new[k].cuda())
+        graph.replay()
+        torch.cuda.synchronize()
+        assert ssd.device_status(ws) == ssd.SSD_OK
+        y_g, f_g = y.clone(), fin.clone()
+        y_e, f_e = ssd.forward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], dev["D"], w.chunk, path=path)
+        torch.cuda.synchronize()
+        assert torch.equal(y_g, y_e) and torch.equal(f_g, f_e)
