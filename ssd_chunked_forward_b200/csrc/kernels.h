@@ -24,6 +24,11 @@ cudaError_t launch_chunk_scan_simt(const Dims& d, const void* x, const void* Bm,
                                    const float* cum, const float* Hin, const float* D, void* y,
                                    cudaStream_t st);
 
+// output step for the per-state decay (called by launch_chunk_scan_simt)
+cudaError_t launch_diag_scan_simt(const Dims& d, const void* x, const void* Bm, const void* Cm,
+                                  const float* cum, const float* Hin, const float* D, void* y,
+                                  cudaStream_t st);
+
 // one recurrent step for single tokens (decode): state[B,H,N,P] updated in place
 cudaError_t launch_decode_step(const Dims& d, const void* x, const float* a, const void* Bm,
                                const void* Cm, const float* D, float* state, void* y,
