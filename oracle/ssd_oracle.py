@@ -218,3 +218,29 @@ def to_bthp(res_y: np.ndarray, chains: np.ndarray, B: int, H: int) -> np.ndarray
     for c, (b, h) in enumerate(chains):
         out[b, :, h, :] = res_y[c]
     return out
+
+
+def discretize(dt_raw, dt_bias, A_log, x):
+    """The selective discretisation in front of the operator, plain fp64 numpy
+    (llms.blog "The Selection Mechanism": Delta_t = softplus(Parameter +
+    W_Delta x_t), Abar_t = exp(Delta_t A), Bbar_t = Delta_t B_t; and
+    "Continuous-to-Discrete Discretization": Bbar ~ Delta B).  With the
+    operator's inputs as log-decays and the per-head step folded into the
+    input (Bbar_t x_t = B_t (Delta_t x_t)):
+        dt = softplus(dt_raw + dt_bias)                  [B,T,H]
+        a  = dt * A,  A = -exp(A_log)                    [B,T,H] (A_log [H])
+                                                         or [B,T,H,N] (A_log [H,N])
+        xd = dt * x                                      [B,T,H,P]
+    softplus(z) = log(1 + e^z), evaluated as max(z, 0) + log1p(e^{-|z|}).
+    Returns (a, xd, dt)."""
+    z = np.asarray(dt_raw, dtype=np.float64)
+    if dt_bias is not None:
+        z = z + np.asarray(dt_bias, dtype=np.float64)[None, None, :]
+    dt = np.maximum(z, 0.0) + np.log1p(np.exp(-np.abs(z)))
+    A = -np.exp(np.asarray(A_log, dtype=np.float64))
+    if A.ndim == 1:
+        a = dt * A[None, None, :]
+    else:
+        a = dt[..., None] * A[None, None, :, :]
+    xd = dt[..., None] * np.asarray(x, dtype=np.float64)
+    return a, xd, dt

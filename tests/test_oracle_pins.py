@@ -284,3 +284,48 @@ def test_zero_initial_state_is_the_default():
     a = O.recurrence(prob)
     b = O.recurrence(prob, initial=np.zeros((2, 2, 4, 3)))
     assert np.array_equal(a["y"], b["y"]) and np.array_equal(a["final"], b["final"])
+
+
+def test_discretize_softplus_identities():
+    """softplus fixed by its definition log(1 + e^z): softplus(z) - softplus(-z)
+    = z, softplus(0) = ln 2, softplus(z) -> z for large z and -> e^z for very
+    negative z; a = dt * (-exp(A_log)) and xd = dt * x."""
+    z = np.array([-40.0, -5.0, -0.3, 0.0, 0.7, 3.0, 25.0, 60.0])
+    raw = z.reshape(1, -1, 1)
+    _, _, dt_p = O.discretize(raw, None, np.zeros(1), np.ones((1, z.size, 1, 1)))
+    _, _, dt_m = O.discretize(-raw, None, np.zeros(1), np.ones((1, z.size, 1, 1)))
+    assert np.allclose(dt_p - dt_m, raw, rtol=0, atol=1e-13)
+    assert abs(dt_p[0, 3, 0] - math.log(2.0)) < 1e-15
+    assert abs(dt_p[0, 7, 0] - 60.0) < 1e-12
+    assert abs(dt_p[0, 0, 0] / math.exp(-40.0) - 1.0) < 1e-12
+    rng = np.random.default_rng(91)
+    raw = rng.standard_normal((2, 5, 3))
+    bias = rng.standard_normal(3)
+    A_log = rng.uniform(0.0, 2.0, size=3)
+    x = rng.standard_normal((2, 5, 3, 4))
+    a, xd, dt = O.discretize(raw, bias, A_log, x)
+    direct = np.log(1.0 + np.exp(raw + bias))
+    assert np.allclose(dt, direct, rtol=1e-14, atol=0)
+    assert np.allclose(a, -dt * np.exp(A_log), rtol=1e-15, atol=0)
+    assert np.allclose(xd, dt[..., None] * x, rtol=1e-15, atol=0)
+    a4, _, _ = O.discretize(raw, bias, np.tile(A_log[:, None], (1, 6)), x)
+    assert a4.shape == (2, 5, 3, 6) and np.allclose(a4[..., 2], a, rtol=1e-15, atol=0)
+
+
+def test_discretize_step_folds_into_the_input():
+    """Bbar_t x_t = (Delta_t B_t) x_t: running the operator with the input
+    scaled by dt equals running it with B scaled by dt (one group per head),
+    and the decays are log(Abar) = dt * A (Abar = exp(Delta A))."""
+    rng = np.random.default_rng(92)
+    B_, T, H, P, N = 1, 20, 2, 3, 4
+    raw = rng.standard_normal((B_, T, H))
+    A_log = rng.uniform(-1.0, 1.0, size=H)
+    x = rng.standard_normal((B_, T, H, P))
+    Bm = rng.standard_normal((B_, T, H, N)) / 2
+    Cm = rng.standard_normal((B_, T, H, N)) / 2
+    a, xd, dt = O.discretize(raw, None, A_log, x)
+    assert np.allclose(np.exp(a), np.exp(dt * -np.exp(A_log)[None, None, :]), rtol=1e-15, atol=0)
+    r1 = O.recurrence(Problem(xd, a, Bm, Cm, None))
+    Bbar = Bm * dt[..., None]          # G = H: each head's own B, scaled by its step
+    r2 = O.recurrence(Problem(x, a, Bbar, Cm, None))
+    assert rel_inf(r1["y"], r2["y"]) < 1e-12 and rel_inf(r1["final"], r2["final"]) < 1e-12
