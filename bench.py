@@ -369,6 +369,50 @@ def run_decode(args, device):
     return 0
 
 
+def run_discretize(args, device):
+    """ssd_discretize on the workload's shape: dt_raw and x in, a and x_out out,
+    each once (algorithmic bytes); L2 flushed before every step."""
+    w = WORKLOADS[args.workload]
+    g = torch.Generator().manual_seed(w.seed + 600)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    raw = torch.randn((w.B, w.T, w.H), generator=g).to(device)
+    bias = torch.randn((w.H,), generator=g).to(device)
+    A_log = torch.rand((w.H, w.N) if w.a_per_state else (w.H,), generator=g).to(device)
+    x = torch.randn((w.B, w.T, w.H, w.P), generator=g).to(dt).to(device)
+    a_out = torch.empty((w.B, w.T, w.H) + ((w.N,) if w.a_per_state else ()), dtype=torch.float32,
+                        device=device)
+    x_out = torch.empty_like(x)
+    scratch = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    st = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        scratch.fill_(1)
+        ssd.discretize(raw, bias, A_log, x, a_out=a_out, x_out=x_out)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for e0, e1 in ev:
+        scratch.fill_(1)
+        e0.record(st)
+        ssd.discretize(raw, bias, A_log, x, a_out=a_out, x_out=x_out)
+        e1.record(st)
+    torch.cuda.synchronize()
+    ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev)
+    byts = (raw.numel() * 4 + 2 * x.numel() * x.element_size() + a_out.numel() * 4
+            + bias.numel() * 4 + A_log.numel() * 4)
+    peaks, src = load_peaks()
+    achieved = byts / (ms / 1e3) / 1e9
+    print(json.dumps({
+        "metric": "SSD discretisation tokens/s (B*T per second)", "value": w.tokens / (ms / 1e3),
+        "unit": "tokens/s", "ms_per_step": ms, "steps": args.steps, "warmup": args.warmup,
+        "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name + "_discretize", "B": w.B, "T": w.T, "H": w.H, "P": w.P,
+                   "a_per_state": w.a_per_state, "l2": "flushed (256 MB write) before every step"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "algorithmic_bytes_per_launch": byts,
+                     "kernel": "ssd_discretize", "peak_source": f"{src} (hbm_gbs)"},
+        "gpu_launches": args.steps}))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -381,6 +425,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--B", type=int, default=None, help="override the batch (profiling small cases)")
     ap.add_argument("--T", type=int, default=None, help="override the sequence length")
+    ap.add_argument("--discretize", action="store_true",
+                    help="time the discretisation front end (ssd_discretize) on the workload's "
+                         "inputs instead of the forward; prints its own JSON line")
     ap.add_argument("--decode", action="store_true",
                     help="time the recurrent decode step (one token per chain) on the workload's "
                          "batch and heads instead of the forward; prints its own JSON line")
@@ -398,6 +445,8 @@ def main():
     device = torch.device("cuda", local)
     if args.decode:
         return run_decode(args, device)
+    if args.discretize:
+        return run_discretize(args, device)
     dist = None
     if world > 1:
         import torch.distributed as dist

@@ -237,6 +237,23 @@ ssd_status ssd_diag_scan(const ssd_shape* shape, const void* x, const void* Bm, 
                          const float* cum, const float* Hin, const float* D, void* y,
                          ssd_stream stream, unsigned impl);
 
+/* The selective discretisation that produces the operator's inputs
+ * ("State Space Models and Mamba ...", llms.blog, "The Selection Mechanism":
+ * Delta_t = softplus(Parameter + W_Delta x_t), Abar_t = exp(Delta_t A),
+ * Bbar_t = Delta_t B_t; "Continuous-to-Discrete Discretization": Bbar ~ Delta B):
+ *     dt = softplus(dt_raw + dt_bias)      per (b, t, h)
+ *     a  = -dt * exp(A_log)                log-decay, log Abar with A = -exp(A_log)
+ *     x_out = dt * x                       Bbar_t x_t = B_t (dt x_t)
+ * dt_raw[B][T][H] fp32 (the W_Delta x_t projection), dt_bias[H] fp32 or NULL,
+ * A_log[H] (or [H][N] when shape->a_per_state) fp32, x[B][T][H][P] (dtype);
+ * outputs a_out[B][T][H] (or [B][T][H][N]) fp32 and x_out[B][T][H][P]
+ * (dtype; may alias x).  Feed (x_out, a_out) to ssd_forward*.  Device
+ * pointers, 16-byte aligned, asynchronous on `stream`; SSD_ERR_INVALID_ARG for
+ * a bad shape or pointer, SSD_ERR_CUDA if the launch fails. */
+ssd_status ssd_discretize(const ssd_shape* shape, const float* dt_raw, const float* dt_bias,
+                          const float* A_log, const void* x, float* a_out, void* x_out,
+                          ssd_stream stream);
+
 /* One recurrent step for a batch of single tokens -- the inference (decode)
  * form of the same operator: per (batch b, head h),
  *     h <- exp(a) o h + B x^T,     y = C^T h + D[h] x

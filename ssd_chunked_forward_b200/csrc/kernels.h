@@ -29,6 +29,11 @@ cudaError_t launch_diag_scan_simt(const Dims& d, const void* x, const void* Bm, 
                                   const float* cum, const float* Hin, const float* D, void* y,
                                   cudaStream_t st);
 
+// the selective discretisation: a = -softplus(dt_raw + dt_bias) exp(A_log), x_out = dt x
+cudaError_t launch_discretize(const Dims& d, const float* dt_raw, const float* dt_bias,
+                              const float* A_log, const void* x, float* a_out, void* x_out,
+                              cudaStream_t st);
+
 // one recurrent step for single tokens (decode): state[B,H,N,P] updated in place
 cudaError_t launch_decode_step(const Dims& d, const void* x, const float* a, const void* Bm,
                                const void* Cm, const float* D, float* state, void* y,

@@ -393,6 +393,18 @@ ssd_status ssd_diag_scan(const ssd_shape* shape, const void* x, const void* Bm, 
     return scan_common(shape, x, Bm, Cm, cum, Hin, D, y, stream, impl, true);
 }
 
+ssd_status ssd_discretize(const ssd_shape* shape, const float* dt_raw, const float* dt_bias,
+                          const float* A_log, const void* x, float* a_out, void* x_out,
+                          ssd_stream stream) {
+    if (check_shape(shape) != SSD_OK) return SSD_ERR_INVALID_ARG;
+    if (!dt_raw || !A_log || !x || !a_out || !x_out) return SSD_ERR_INVALID_ARG;
+    if (!aligned16(dt_raw) || !aligned16(A_log) || !aligned16(x) || !aligned16(a_out) ||
+        !aligned16(x_out) || (dt_bias && !aligned16(dt_bias)))
+        return SSD_ERR_INVALID_ARG;
+    return cuda_status(ssd::launch_discretize(dims_of(shape), dt_raw, dt_bias, A_log, x, a_out,
+                                              x_out, (cudaStream_t)stream));
+}
+
 ssd_status ssd_decode_step(const ssd_shape* shape, const void* x, const float* a, const void* Bm,
                            const void* Cm, const float* D, float* state, void* y,
                            ssd_stream stream) {

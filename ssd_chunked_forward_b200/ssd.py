@@ -26,7 +26,7 @@ EXPORTS = [
     "ssd_forward_path", "ssd_device_status", "ssd_chunk_cumsum", "ssd_chunk_state",
     "ssd_state_pass", "ssd_chunk_scan", "ssd_diag_scan", "ssd_forward_host_bytes",
     "ssd_forward_host", "ssd_forward_noalloc", "ssd_auto_path", "ssd_forward_init",
-    "ssd_decode_step",
+    "ssd_decode_step", "ssd_discretize",
 ]
 
 
@@ -79,8 +79,9 @@ def load(path: str = LIB_PATH):
     lib.ssd_forward_host.argtypes = [sp, vp, fp, vp, vp, fp, vp, fp, vp, sz, vp]
     lib.ssd_forward_noalloc.argtypes = [sp, vp, fp, vp, vp, fp, vp, fp, vp]
     lib.ssd_decode_step.argtypes = [sp, vp, fp, vp, vp, fp, fp, vp, vp]
+    lib.ssd_discretize.argtypes = [sp, fp, fp, fp, vp, fp, vp, vp]
     for name in ("ssd_forward_noalloc", "ssd_forward", "ssd_forward_path", "ssd_forward_init",
-                 "ssd_device_status", "ssd_chunk_cumsum", "ssd_decode_step",
+                 "ssd_device_status", "ssd_chunk_cumsum", "ssd_decode_step", "ssd_discretize",
                  "ssd_chunk_state", "ssd_state_pass", "ssd_chunk_scan", "ssd_diag_scan",
                  "ssd_forward_host"):
         getattr(lib, name).restype = ctypes.c_int
@@ -288,3 +289,25 @@ def decode_step(x, a, Bm, Cm, D, state, *, y=None, stream=None):
     _check(load().ssd_decode_step(ctypes.byref(shape), _ptr(x), _ptr(a), _ptr(Bm), _ptr(Cm), _ptr(D),
                                   _ptr(state), _ptr(y), _stream(stream)), "ssd_decode_step")
     return y
+
+
+def discretize(dt_raw, dt_bias, A_log, x, *, a_out=None, x_out=None, stream=None):
+    """dt = softplus(dt_raw + dt_bias); returns (a, x_out): a = -dt exp(A_log)
+    ([B,T,H], or [B,T,H,N] when A_log is [H,N]) and x_out = dt x ([B,T,H,P],
+    x's dtype), the inputs of forward()."""
+    for name, t in (("dt_raw", dt_raw), ("A_log", A_log), ("x", x)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if dt_raw.dtype != torch.float32 or A_log.dtype != torch.float32:
+        raise ValueError("dt_raw and A_log must be float32")
+    B, T, H, P = x.shape
+    per_state = A_log.dim() == 2
+    N = A_log.shape[1] if per_state else 1
+    shape = make_shape(B, T, H, P, 1, N, 1, per_state, x.dtype)
+    if a_out is None:
+        a_out = torch.empty((B, T, H) + ((N,) if per_state else ()), dtype=torch.float32, device=x.device)
+    if x_out is None:
+        x_out = torch.empty_like(x)
+    _check(load().ssd_discretize(ctypes.byref(shape), _ptr(dt_raw), _ptr(dt_bias), _ptr(A_log), _ptr(x),
+                                 _ptr(a_out), _ptr(x_out), _stream(stream)), "ssd_discretize")
+    return a_out, x_out

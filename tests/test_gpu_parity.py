@@ -8,6 +8,8 @@ inputs with fp32 accumulation, as ||y - y_ref||_inf / ||y_ref||_inf.
 """
 from __future__ import annotations
 
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -435,3 +437,54 @@ def test_cuda_graph_capture_and_replay(path):
         y_e, f_e = ssd.forward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], dev["D"], w.chunk, path=path)
         torch.cuda.synchronize()
         assert torch.equal(y_g, y_e) and torch.equal(f_g, f_e)
+
+
+@pytest.mark.parametrize("per_state,dtype", [(False, "bf16"), (True, "bf16"), (False, "f32")],
+                         ids=["scalar_bf16", "per_state_bf16", "scalar_f32"])
+def test_discretize_matches_oracle(per_state, dtype):
+    """ssd_discretize against the oracle's fp64 discretisation, then the forward
+    on its outputs against the oracle recurrence on the oracle's outputs."""
+    B, T, H, P, N, G = 2, 512, 4, 64, 128 if not per_state else 64, 1
+    g = torch.Generator().manual_seed(93 + per_state)
+    dt_raw = (torch.randn((B, T, H), generator=g, dtype=torch.float64) * 1.5 - 2.0).to(torch.float32)
+    dt_bias = torch.randn((H,), generator=g, dtype=torch.float64).to(torch.float32)
+    A_log = (torch.rand((H, N) if per_state else (H,), generator=g, dtype=torch.float64) * math.log(16)).to(torch.float32)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    x = torch.randn((B, T, H, P), generator=g, dtype=torch.float64).to(tdt)
+    Bm = (torch.randn((B, T, G, N), generator=g, dtype=torch.float64) / math.sqrt(N)).to(tdt)
+    Cm = (torch.randn((B, T, G, N), generator=g, dtype=torch.float64) / math.sqrt(N)).to(tdt)
+    D = torch.randn((H,), generator=g, dtype=torch.float64).to(torch.float32)
+    a_g, x_g = ssd.discretize(dt_raw.cuda(), dt_bias.cuda(), A_log.cuda(), x.cuda())
+    torch.cuda.synchronize()
+    f64 = lambda t: t.to(torch.float64).numpy()
+    a_r, x_r, _ = O.discretize(f64(dt_raw), f64(dt_bias), f64(A_log), f64(x))
+    assert rel_err(a_g.cpu().numpy().astype(np.float64), a_r) <= 1e-6
+    assert rel_err(x_g.float().cpu().numpy().astype(np.float64), x_r) <= (4e-3 if dtype == "bf16" else 1e-6)
+    # in place on x gives the same
+    xc = x.cuda()
+    ssd.discretize(dt_raw.cuda(), dt_bias.cuda(), A_log.cuda(), xc, x_out=xc)
+    torch.cuda.synchronize()
+    assert torch.equal(xc, x_g)
+    # the forward on the discretised inputs
+    y, fin = ssd.forward(x_g, a_g, Bm.cuda(), Cm.cuda(), D.cuda(), 256 if not per_state else 128)
+    torch.cuda.synchronize()
+    ref = O.recurrence(O.Problem(x_r, a_r, f64(Bm), f64(Cm), f64(D)))
+    yr = ref["y"].reshape(B, H, T, P).transpose(0, 2, 1, 3)
+    tol = TOL_BF16 if dtype == "bf16" else 1e-4
+    assert rel_err(y.float().cpu().numpy().astype(np.float64), yr) <= tol
+    assert rel_err(fin.cpu().numpy().astype(np.float64), ref["final"].reshape(B, H, N, P)) <= tol
+
+
+def test_discretize_odd_rows():
+    """Rows whose length is not a multiple of 16 bytes (the per-row path)."""
+    B, T, H, P, N = 1, 33, 3, 70, 5
+    g = torch.Generator().manual_seed(95)
+    dt_raw = torch.randn((B, T, H), generator=g, dtype=torch.float64).to(torch.float32)
+    A_log = torch.rand((H, N), generator=g, dtype=torch.float64).to(torch.float32)
+    x = torch.randn((B, T, H, P), generator=g, dtype=torch.float64).to(torch.float32)
+    a_g, x_g = ssd.discretize(dt_raw.cuda(), None, A_log.cuda(), x.cuda())
+    torch.cuda.synchronize()
+    f64 = lambda t: t.to(torch.float64).numpy()
+    a_r, x_r, _ = O.discretize(f64(dt_raw), None, f64(A_log), f64(x))
+    assert rel_err(a_g.cpu().numpy().astype(np.float64), a_r) <= 1e-6
+    assert rel_err(x_g.cpu().numpy().astype(np.float64), x_r) <= 1e-6
