@@ -254,6 +254,28 @@ ssd_status ssd_discretize(const ssd_shape* shape, const float* dt_raw, const flo
                           const float* A_log, const void* x, float* a_out, void* x_out,
                           ssd_stream stream);
 
+/* Sequences split into S segments along T (one per rank, say): the exchange
+ * step that lets each segment resume from its true incoming state -- the
+ * passing of one summarised state between pieces, as between chunks ("State
+ * Space Duality", aiwiki, "Two algorithms for one operator"), one level up;
+ * the pages give no multi-device form, this is its plainest reading.
+ *
+ * ssd_decay_total: total[b][h] = sum_t a[b][t][h] (or [b][h][n] per state),
+ * the log-decay a segment applies to the state it receives.  shape: the
+ * segment's (B, T, H, N, a_per_state; other fields valid as for ssd_forward).
+ *
+ * ssd_state_combine: from each segment's final state started at zero,
+ * finals[S][B][H][N][P], and its total, totals[S][B][H] (or [S][B][H][N]),
+ *     h_in[0] = h0 (or zero),  h_in[s+1] = exp(totals[s]) o h_in[s] + finals[s],
+ * written to h_in[S+1][B][H][N][P]: h_in[s] enters segment s (pass it to
+ * ssd_forward_init), h_in[S] is the state after the whole sequence.  shape
+ * gives B, H, N, P, a_per_state.  All fp32 device pointers, 16-byte aligned,
+ * asynchronous on `stream`; SSD_ERR_INVALID_ARG for a bad shape, S < 1 or a
+ * bad pointer. */
+ssd_status ssd_decay_total(const ssd_shape* shape, const float* a, float* total, ssd_stream stream);
+ssd_status ssd_state_combine(const ssd_shape* shape, int segments, const float* finals,
+                             const float* totals, const float* h0, float* h_in, ssd_stream stream);
+
 /* One recurrent step for a batch of single tokens -- the inference (decode)
  * form of the same operator: per (batch b, head h),
  *     h <- exp(a) o h + B x^T,     y = C^T h + D[h] x

@@ -34,6 +34,12 @@ cudaError_t launch_discretize(const Dims& d, const float* dt_raw, const float* d
                               const float* A_log, const void* x, float* a_out, void* x_out,
                               cudaStream_t st);
 
+// segments of a sequence: total log-decay per chain, and the incoming state of
+// each segment from the others' final states (see segments.cu)
+cudaError_t launch_decay_total(const Dims& d, const float* a, float* tot, cudaStream_t st);
+cudaError_t launch_state_combine(const Dims& d, int S, const float* fin, const float* tot,
+                                 const float* h0, float* h_in, cudaStream_t st);
+
 // one recurrent step for single tokens (decode): state[B,H,N,P] updated in place
 cudaError_t launch_decode_step(const Dims& d, const void* x, const float* a, const void* Bm,
                                const void* Cm, const float* D, float* state, void* y,

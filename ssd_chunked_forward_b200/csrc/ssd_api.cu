@@ -405,6 +405,22 @@ ssd_status ssd_discretize(const ssd_shape* shape, const float* dt_raw, const flo
                                               x_out, (cudaStream_t)stream));
 }
 
+ssd_status ssd_decay_total(const ssd_shape* shape, const float* a, float* total, ssd_stream stream) {
+    if (check_shape(shape) != SSD_OK || !a || !total || !aligned16(a) || !aligned16(total))
+        return SSD_ERR_INVALID_ARG;
+    return cuda_status(ssd::launch_decay_total(dims_of(shape), a, total, (cudaStream_t)stream));
+}
+
+ssd_status ssd_state_combine(const ssd_shape* shape, int segments, const float* finals,
+                             const float* totals, const float* h0, float* h_in, ssd_stream stream) {
+    if (check_shape(shape) != SSD_OK || segments < 1 || !finals || !totals || !h_in)
+        return SSD_ERR_INVALID_ARG;
+    if (!aligned16(finals) || !aligned16(totals) || !aligned16(h_in) || (h0 && !aligned16(h0)))
+        return SSD_ERR_INVALID_ARG;
+    return cuda_status(ssd::launch_state_combine(dims_of(shape), segments, finals, totals, h0, h_in,
+                                                 (cudaStream_t)stream));
+}
+
 ssd_status ssd_decode_step(const ssd_shape* shape, const void* x, const float* a, const void* Bm,
                            const void* Cm, const float* D, float* state, void* y,
                            ssd_stream stream) {

@@ -26,7 +26,7 @@ EXPORTS = [
     "ssd_forward_path", "ssd_device_status", "ssd_chunk_cumsum", "ssd_chunk_state",
     "ssd_state_pass", "ssd_chunk_scan", "ssd_diag_scan", "ssd_forward_host_bytes",
     "ssd_forward_host", "ssd_forward_noalloc", "ssd_auto_path", "ssd_forward_init",
-    "ssd_decode_step", "ssd_discretize",
+    "ssd_decode_step", "ssd_discretize", "ssd_decay_total", "ssd_state_combine",
 ]
 
 
@@ -80,8 +80,11 @@ def load(path: str = LIB_PATH):
     lib.ssd_forward_noalloc.argtypes = [sp, vp, fp, vp, vp, fp, vp, fp, vp]
     lib.ssd_decode_step.argtypes = [sp, vp, fp, vp, vp, fp, fp, vp, vp]
     lib.ssd_discretize.argtypes = [sp, fp, fp, fp, vp, fp, vp, vp]
+    lib.ssd_decay_total.argtypes = [sp, fp, fp, vp]
+    lib.ssd_state_combine.argtypes = [sp, ctypes.c_int, fp, fp, fp, fp, vp]
     for name in ("ssd_forward_noalloc", "ssd_forward", "ssd_forward_path", "ssd_forward_init",
                  "ssd_device_status", "ssd_chunk_cumsum", "ssd_decode_step", "ssd_discretize",
+                 "ssd_decay_total", "ssd_state_combine",
                  "ssd_chunk_state", "ssd_state_pass", "ssd_chunk_scan", "ssd_diag_scan",
                  "ssd_forward_host"):
         getattr(lib, name).restype = ctypes.c_int
@@ -311,3 +314,36 @@ def discretize(dt_raw, dt_bias, A_log, x, *, a_out=None, x_out=None, stream=None
     _check(load().ssd_discretize(ctypes.byref(shape), _ptr(dt_raw), _ptr(dt_bias), _ptr(A_log), _ptr(x),
                                  _ptr(a_out), _ptr(x_out), _stream(stream)), "ssd_discretize")
     return a_out, x_out
+
+
+def decay_total(a, *, out=None, stream=None):
+    """Total log-decay of each chain over the sequence: a [B,T,H] -> [B,H]
+    (a [B,T,H,N] -> [B,H,N])."""
+    if not a.is_cuda or not a.is_contiguous() or a.dtype != torch.float32:
+        raise ValueError("a must be a contiguous float32 CUDA tensor")
+    B, T, H = a.shape[:3]
+    per_state = a.dim() == 4
+    N = a.shape[3] if per_state else 1
+    shape = make_shape(B, T, H, 1, 1, N, 1, per_state, torch.float32)
+    if out is None:
+        out = torch.empty((B, H) + ((N,) if per_state else ()), dtype=torch.float32, device=a.device)
+    _check(load().ssd_decay_total(ctypes.byref(shape), _ptr(a), _ptr(out), _stream(stream)),
+           "ssd_decay_total")
+    return out
+
+
+def state_combine(finals, totals, h0=None, *, out=None, stream=None):
+    """finals [S,B,H,N,P] (each segment's final state from zero), totals
+    [S,B,H] or [S,B,H,N] -> h_in [S+1,B,H,N,P]: h_in[s] enters segment s,
+    h_in[S] is the state after all of them (h0, or zero, enters segment 0)."""
+    for name, t in (("finals", finals), ("totals", totals)):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.float32:
+            raise ValueError(f"{name} must be a contiguous float32 CUDA tensor")
+    S, B, H, N, P = finals.shape
+    per_state = totals.dim() == 4
+    shape = make_shape(B, 1, H, P, 1, N, 1, per_state, torch.float32)
+    if out is None:
+        out = torch.empty((S + 1, B, H, N, P), dtype=torch.float32, device=finals.device)
+    _check(load().ssd_state_combine(ctypes.byref(shape), int(S), _ptr(finals), _ptr(totals), _ptr(h0),
+                                    _ptr(out), _stream(stream)), "ssd_state_combine")
+    return out

@@ -488,3 +488,38 @@ def test_discretize_odd_rows():
     a_r, x_r, _ = O.discretize(f64(dt_raw), None, f64(A_log), f64(x))
     assert rel_err(a_g.cpu().numpy().astype(np.float64), a_r) <= 1e-6
     assert rel_err(x_g.cpu().numpy().astype(np.float64), x_r) <= 1e-6
+
+
+@pytest.mark.parametrize("per_state", [False, True], ids=["scalar", "per_state"])
+def test_sequence_segments_with_library_kernels(per_state):
+    """A sequence cut into 4 segments, each run from zero, combined by
+    ssd_decay_total + ssd_state_combine and rerun from its incoming state
+    (what each rank does in the sharded forward), equals the forward over the
+    whole sequence; the combine's last state is the sequence's final state."""
+    if per_state:
+        w = small_case(B=2, T=1024, H=4, P=64, N=64, G=1, chunk=128, dtype="bf16", a_per_state=True, seed=103)
+    else:
+        w = small_case(B=2, T=4096, H=8, P=64, N=128, G=1, chunk=256, dtype="bf16", seed=104)
+    inp = generate(w)
+    dev = to_dev(inp)
+    y_full, f_full = ssd.forward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], dev["D"], w.chunk)
+    S = 4
+    Ts = w.T // S
+    seg = lambda t, s: t[:, s * Ts:(s + 1) * Ts].contiguous()
+    parts = [[seg(dev[k], s) for k in ("x", "a", "Bm", "Cm")] for s in range(S)]
+    fins, tots = [], []
+    for x, a, Bm, Cm in parts:
+        _, f = ssd.forward(x, a, Bm, Cm, dev["D"], w.chunk)
+        fins.append(f)
+        tots.append(ssd.decay_total(a))
+    totals = torch.stack(tots).contiguous()
+    h_in = ssd.state_combine(torch.stack(fins).contiguous(), totals)
+    ys = [ssd.forward(x, a, Bm, Cm, dev["D"], w.chunk, initial_state=h_in[s].contiguous())[0]
+          for s, (x, a, Bm, Cm) in enumerate(parts)]
+    torch.cuda.synchronize()
+    assert rel_err(torch.cat(ys, dim=1).float().cpu().numpy(), y_full.float().cpu().numpy()) <= TOL_BF16
+    assert rel_err(h_in[S].cpu().numpy(), f_full.cpu().numpy()) <= TOL_BF16
+    # the totals themselves: sums of the segment's log-decays
+    a64 = inp["a"].to(torch.float64)
+    ref_tot = torch.stack([a64[:, s * Ts:(s + 1) * Ts].sum(dim=1) for s in range(S)]).numpy()
+    assert rel_err(totals.cpu().numpy().astype(np.float64), ref_tot) <= 1e-5
