@@ -31,9 +31,13 @@
  *        final_state    [B, H, N, P]   f32, may be NULL
  *        cum            [B, H, nc, Q]  f32  ([B, H, nc, Q, N] when a_per_state)
  *        states         [B, H, nc, N, P] f32
- *  - Requirements: all sizes >= 1, T % chunk == 0, H % G == 0, chunk <= 1024,
- *    N <= 256, P <= 256.  Violations return SSD_ERR_INVALID_ARG before any
- *    work is queued.
+ *  - Requirements: all sizes >= 1, H % G == 0, chunk <= 1024, N <= 256,
+ *    P <= 256; the per-step entry points (ssd_chunk_cumsum ... ssd_diag_scan)
+ *    also need T % chunk == 0.  The whole-forward entry points accept any T:
+ *    the result does not depend on the chunk, so when T % chunk != 0 they run
+ *    with the largest chunk <= the requested one that divides T (a multiple
+ *    of 128 when T allows one; otherwise the CUDA-core path serves it).
+ *    Violations return SSD_ERR_INVALID_ARG before any work is queued.
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
  *    compute entry point is asynchronous on it; a return of SSD_OK means the
  *    work was queued.  Launch failures return SSD_ERR_CUDA.  Problems found

@@ -50,9 +50,16 @@ ssd_status scratch_address(void** out) {
 
 }  // namespace
 
-extern "C" ssd_status ssd_forward_noalloc(const ssd_shape* shape, const void* x, const float* a,
+namespace ssd {
+ssd_shape forward_shape(const ssd_shape* s);  // ssd_api.cu: the chunk used for T % chunk != 0
+}
+
+extern "C" ssd_status ssd_forward_noalloc(const ssd_shape* shape_in, const void* x, const float* a,
                                           const void* Bm, const void* Cm, const float* D, void* y,
                                           float* final_state, ssd_stream stream) {
+    if (!shape_in) return SSD_ERR_INVALID_ARG;
+    const ssd_shape fs = ssd::forward_shape(shape_in);
+    const ssd_shape* shape = &fs;
     if (ssd_workspace_size(shape) == 0) return SSD_ERR_INVALID_ARG;  // invalid shape
     if (!x || !a || !Bm || !Cm || !y) return SSD_ERR_INVALID_ARG;
     const uintptr_t m = (uintptr_t)x | (uintptr_t)a | (uintptr_t)Bm | (uintptr_t)Cm |

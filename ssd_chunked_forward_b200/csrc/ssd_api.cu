@@ -128,6 +128,26 @@ ssd_status run_modular(const Dims& d0, const void* x, const float* a, const void
 }  // namespace
 
 namespace ssd {
+// The forward-level entry points accept T % chunk != 0: the result does not
+// depend on the chunk (the chunked evaluation is exact for every chunk), so
+// they run with the largest chunk <= the requested one that divides T,
+// preferring a multiple of 128 (the tensor-core block) when T allows one.
+ssd_shape forward_shape(const ssd_shape* s) {
+    ssd_shape r = *s;
+    if (s->T < 1 || s->chunk < 1 || s->T % s->chunk == 0) return r;
+    int q = 0;
+    if (s->T % 128 == 0)
+        for (int c = (s->chunk / 128) * 128; c >= 128 && !q; c -= 128)
+            if (s->T % c == 0) q = c;
+    for (int c = s->chunk < s->T ? s->chunk : s->T; c >= 1 && !q; --c)
+        if (s->T % c == 0) q = c;
+    r.chunk = q;
+    return r;
+}
+
+}  // namespace ssd
+
+namespace ssd {
 cudaError_t launch_fused_ordered(const Dims& d, const void* x, const float* a, const void* Bm,
                                  const void* Cm, const float* D, void* y, float* fin, float* ring,
                                  unsigned* flags, int* status, bool test_stall, cudaStream_t st,
@@ -169,12 +189,18 @@ const char* ssd_status_string(ssd_status s) {
     return "SSD_ERR_UNKNOWN";
 }
 
-size_t ssd_workspace_size(const ssd_shape* shape) {
+size_t ssd_workspace_size(const ssd_shape* shape_in) {
+    if (!shape_in) return 0;
+    const ssd_shape fs = ssd::forward_shape(shape_in);
+    const ssd_shape* shape = &fs;
     if (check_shape(shape) != SSD_OK) return 0;
     return workspace_bytes(dims_of(shape));
 }
 
-int ssd_path_supported(const ssd_shape* shape, unsigned path) {
+int ssd_path_supported(const ssd_shape* shape_in, unsigned path) {
+    if (!shape_in) return 0;
+    const ssd_shape fs = ssd::forward_shape(shape_in);
+    const ssd_shape* shape = &fs;
     if (check_shape(shape) != SSD_OK) return 0;
     const Dims d = dims_of(shape);
     switch (path) {
@@ -186,7 +212,10 @@ int ssd_path_supported(const ssd_shape* shape, unsigned path) {
     }
 }
 
-int ssd_auto_path(const ssd_shape* shape) {
+int ssd_auto_path(const ssd_shape* shape_in) {
+    if (!shape_in) return -1;
+    const ssd_shape fs = ssd::forward_shape(shape_in);
+    const ssd_shape* shape = &fs;
     if (check_shape(shape) != SSD_OK) return -1;
     const Dims d = dims_of(shape);
     // fewer chains than this: the fused kernel's per-block hand-off (~4 us on
@@ -197,10 +226,13 @@ int ssd_auto_path(const ssd_shape* shape) {
     return SSD_PATH_MODULAR;
 }
 
-ssd_status ssd_forward_init(const ssd_shape* shape, const void* x, const float* a, const void* Bm,
+ssd_status ssd_forward_init(const ssd_shape* shape_in, const void* x, const float* a, const void* Bm,
                             const void* Cm, const float* D, const float* initial_state, void* y,
                             float* final_state, void* workspace, size_t ws_bytes,
                             ssd_stream stream, unsigned path, unsigned flags) {
+    if (!shape_in) return SSD_ERR_INVALID_ARG;
+    const ssd_shape fs = ssd::forward_shape(shape_in);
+    const ssd_shape* shape = &fs;
     ssd_status st = check_shape(shape);
     if (st != SSD_OK) return st;
     if (!x || !a || !Bm || !Cm || !y) return SSD_ERR_INVALID_ARG;
@@ -270,15 +302,21 @@ static size_t host_layout(const ssd_shape* s, size_t off[8]) {
     return total;
 }
 
-size_t ssd_forward_host_bytes(const ssd_shape* shape) {
+size_t ssd_forward_host_bytes(const ssd_shape* shape_in) {
+    if (!shape_in) return 0;
+    const ssd_shape fs = ssd::forward_shape(shape_in);
+    const ssd_shape* shape = &fs;
     if (check_shape(shape) != SSD_OK) return 0;
     size_t off[8];
     return host_layout(shape, off);
 }
 
-ssd_status ssd_forward_host(const ssd_shape* shape, const void* x_h, const float* a_h,
+ssd_status ssd_forward_host(const ssd_shape* shape_in, const void* x_h, const float* a_h,
                             const void* Bm_h, const void* Cm_h, const float* D_h, void* y_h,
                             float* final_h, void* dev_buf, size_t dev_bytes, ssd_stream stream) {
+    if (!shape_in) return SSD_ERR_INVALID_ARG;
+    const ssd_shape fs = ssd::forward_shape(shape_in);
+    const ssd_shape* shape = &fs;
     ssd_status st = check_shape(shape);
     if (st != SSD_OK) return st;
     if (!x_h || !a_h || !Bm_h || !Cm_h || !y_h) return SSD_ERR_INVALID_ARG;

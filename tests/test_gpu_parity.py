@@ -49,6 +49,18 @@ EDGE = [
     small_case(B=1, T=1024, H=1, P=8, N=8, G=1, chunk=1024, dtype="f32", seed=12),
 ]
 
+# T % chunk != 0: the whole forward runs with the largest chunk <= the
+# requested one that divides T (chunk invariance), so these reach the fused
+# kernel (T=384 -> 128, T=640 -> 128) and the CUDA-core paths (T=1000 -> 250,
+# T=997 -> 1, T=200 -> 100)
+RAGGED = [
+    small_case(B=1, T=384, H=4, P=64, N=128, G=1, chunk=256, dtype="bf16", seed=71),
+    small_case(B=2, T=640, H=3, P=64, N=128, G=1, chunk=512, dtype="bf16", seed=72),
+    small_case(B=1, T=1000, H=2, P=64, N=128, G=1, chunk=256, dtype="bf16", seed=73),
+    small_case(B=1, T=997, H=2, P=12, N=10, G=1, chunk=256, dtype="f32", seed=74),
+    small_case(B=2, T=200, H=2, P=16, N=24, G=2, chunk=128, dtype="f32", a_per_state=True, seed=75),
+]
+
 
 def _ids(cases):
     return [c.name + ("_diag" if c.a_per_state else "") + "_" + c.dtype for c in cases]
@@ -62,7 +74,7 @@ def _paths():
     return [ssd.PATH_SIMT, ssd.PATH_MODULAR, ssd.PATH_AUTO, ssd.PATH_FUSED]
 
 
-@pytest.mark.parametrize("w", CASES + EDGE, ids=_ids(CASES + EDGE))
+@pytest.mark.parametrize("w", CASES + EDGE + RAGGED, ids=_ids(CASES + EDGE + RAGGED))
 @pytest.mark.parametrize("path", _paths(), ids=["simt", "modular", "auto", "fused"])
 def test_forward_matches_oracle(w, path):
     inp = generate(w)
@@ -306,7 +318,7 @@ INIT_CASES = [
 ]
 
 
-@pytest.mark.parametrize("w", INIT_CASES, ids=_ids(INIT_CASES))
+@pytest.mark.parametrize("w", INIT_CASES + RAGGED[:3], ids=_ids(INIT_CASES + RAGGED[:3]))
 @pytest.mark.parametrize("path", _paths(), ids=["simt", "modular", "auto", "fused"])
 def test_initial_state_matches_oracle(w, path):
     """ssd_forward_init: every chain starts from a given state h_{-1}; y and the
