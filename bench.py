@@ -61,7 +61,7 @@ def kernel_bytes(w, name):
     """Algorithmic bytes of one launch of a step kernel: each tensor it must
     read or write, once."""
     B, T, H, P, N, G, Q = w.B, w.T, w.H, w.P, w.N, w.G, w.chunk
-    nc = T // Q
+    nc = -(-T // Q)
     el = 2 if w.dtype == "bf16" else 4
     na = N if w.a_per_state else 1
     x = B * T * H * P * el
@@ -294,7 +294,7 @@ def time_steps_split(w, dev, flush, reps, impl):
     w = step_workload(w, impl)
     shape = ssd.shape_of(dev["x"], dev["a"], dev["Bm"], w.chunk)
     st = torch.cuda.current_stream()
-    nc = w.T // w.chunk
+    nc = -(-w.T // w.chunk)
     cum_t = torch.empty(w.B * w.H * nc * w.chunk * (w.N if w.a_per_state else 1),
                         dtype=torch.float32, device=dev["x"].device)
     states = torch.empty((w.B, w.H, nc, w.N, w.P), dtype=torch.float32, device=dev["x"].device)

@@ -22,7 +22,7 @@
  *  - Every tensor argument is a DEVICE pointer to a contiguous row-major
  *    buffer that the caller owns; the library allocates nothing and keeps no
  *    state between calls.  Tensors are 16-byte aligned.
- *  - Shapes (nc = T / chunk, Q = chunk):
+ *  - Shapes (nc = ceil(T / chunk), Q = chunk):
  *        x, y           [B, T, H, P]   dtype (f32 or bf16)
  *        a              [B, T, H]      f32 log-decays (a <= 0 assumed, not checked)
  *                       [B, T, H, N]   when a_per_state != 0
@@ -32,12 +32,15 @@
  *        cum            [B, H, nc, Q]  f32  ([B, H, nc, Q, N] when a_per_state)
  *        states         [B, H, nc, N, P] f32
  *  - Requirements: all sizes >= 1, H % G == 0, chunk <= 1024, N <= 256,
- *    P <= 256; the per-step entry points (ssd_chunk_cumsum ... ssd_diag_scan)
- *    also need T % chunk == 0.  The whole-forward entry points accept any T:
- *    the result does not depend on the chunk, so when T % chunk != 0 they run
- *    with the largest chunk <= the requested one that divides T (a multiple
- *    of 128 when T allows one; otherwise the CUDA-core path serves it).
- *    Violations return SSD_ERR_INVALID_ARG before any work is queued.
+ *    P <= 256, T <= 2^31 - 1025.  Violations return SSD_ERR_INVALID_ARG
+ *    before any work is queued.
+ *  - T need not be a multiple of chunk: the last chunk then holds the
+ *    T - (nc-1) Q remaining tokens.  Its positions past T count as a = 0 and
+ *    x = B = C = 0 (no decay, no input, no output): cum stays flat there,
+ *    they add nothing to any state, and nothing is read or written past T in
+ *    x, a, Bm, Cm or y.  (The pages' chunked algorithm splits T into whole
+ *    chunks; the padding leaves y and the final state exactly as the
+ *    recurrence gives them.)
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
  *    compute entry point is asynchronous on it; a return of SSD_OK means the
  *    work was queued.  Launch failures return SSD_ERR_CUDA.  Problems found

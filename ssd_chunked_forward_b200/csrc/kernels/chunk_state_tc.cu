@@ -81,7 +81,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int k = bid % nc;
     const int b = bid / nc;
     const int h0 = g * HG + slice * hpb;
-    const int row0 = b * T + k * Q;  // token row in [B*T]
+    const int t0 = k * Q;  // first token of the chunk (the last chunk may run past T)
 
     if (threadIdx.x == 0) {
         tc::mbar_init(&bars->b_full, 1);
@@ -112,8 +112,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::prefetch_tmap(&tm_x);
             tc::prefetch_tmap(&tm_b);
             tc::mbar_arrive_expect_tx(&bars->b_full, 2 * kTileBytes);
-            tc::tma_load_3d(sB, &tm_b, &bars->b_full, 0, g, row0);
-            tc::tma_load_3d(sB + kTileBytes, &tm_b, &bars->b_full, 64, g, row0);
+            tc::tma_load_4d(sB, &tm_b, &bars->b_full, 0, g, t0, b);
+            tc::tma_load_4d(sB + kTileBytes, &tm_b, &bars->b_full, 64, g, t0, b);
             for (int i = 0; i < hpb; ++i) {
                 const int st = i & 1;
                 if (i >= 2 && !tc::mbar_wait(&bars->x_empty[st], ((i >> 1) - 1) & 1, abort_v)) {
@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 tc::mbar_arrive_expect_tx(&bars->x_full[st], kTileBytes);
-                tc::tma_load_3d(sX + st * kTileBytes, &tm_x, &bars->x_full[st], 0, h0 + i, row0);
+                tc::tma_load_4d(sX + st * kTileBytes, &tm_x, &bars->x_full[st], 0, h0 + i, t0, b);
             }
             // leave no copy in flight: the last loads must have landed
             for (int i = hpb - 2 < 0 ? 0 : hpb - 2; i < hpb; ++i)
@@ -255,9 +255,9 @@ cudaError_t launch_chunk_state_tc(const Dims& d, const void* x, const void* Bm, 
                                   float* states, cudaStream_t st) {
     if (!chunk_state_tc_supported(d)) return cudaErrorNotSupported;
     CUtensorMap tx, tb;
-    cudaError_t e = make_tmap_bf16_3d(&tx, x, d.P, d.H, (uint64_t)d.B * d.T, d.Q);
+    cudaError_t e = make_tmap_bf16_4d(&tx, x, d.P, d.H, d.T, d.B, d.Q);
     if (e != cudaSuccess) return e;
-    e = make_tmap_bf16_3d(&tb, Bm, d.N, d.G, (uint64_t)d.B * d.T, d.Q);
+    e = make_tmap_bf16_4d(&tb, Bm, d.N, d.G, d.T, d.B, d.Q);
     if (e != cudaSuccess) return e;
     const int hpb = heads_per_cta(d);
     const long long blocks = (long long)d.B * d.nc * d.G * ((d.H / d.G) / hpb);

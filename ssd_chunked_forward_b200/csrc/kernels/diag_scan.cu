@@ -50,12 +50,14 @@ __global__ void __launch_bounds__(256) diag_scan_simt_kernel(
     const int tid = threadIdx.x, ti = tid >> 3, tp = tid & 7;
     const float* cumk = cum + ((size_t)bh * nc + k) * (size_t)Q * N;
     const size_t tk = (size_t)k * Q;
+    const int qv = min(Q, Tlen - k * Q);  // rows of this chunk before T
+    if (i0 >= qv) return;                 // a tile wholly past T (the whole block leaves)
     auto ocol = [&](int m) { return m < 4 ? 4 * tp + m : 28 + 4 * tp + m; };  // output column of acc[m]
 
     for (int idx = tid; idx < 32 * N; idx += 256) {
         const int ii = idx / N, n = idx % N, i = i0 + ii;
-        Cs[ii * NS + n] = (i < Q) ? to_f32(Cm[(((size_t)b * Tlen + tk + i) * G + g) * N + n]) : 0.f;
-        cr[ii * NS + n] = (i < Q) ? cumk[(size_t)i * N + n] * kL2e : 0.f;
+        Cs[ii * NS + n] = (i < qv) ? to_f32(Cm[(((size_t)b * Tlen + tk + i) * G + g) * N + n]) : 0.f;
+        cr[ii * NS + n] = (i < qv) ? cumk[(size_t)i * N + n] * kL2e : 0.f;
     }
     for (int n = tid; n < N; n += 256) rf[n] = i0 > 0 ? cumk[(size_t)(i0 - 1) * N + n] * kL2e : 0.f;
     __syncthreads();
@@ -70,27 +72,27 @@ __global__ void __launch_bounds__(256) diag_scan_simt_kernel(
 #pragma unroll
     for (int m = 0; m < 8; ++m) acc[m] = 0.f;
     const int i = i0 + ti;
-    const int i_last = min(i0 + 31, Q - 1);
+    const int i_last = min(i0 + 31, qv - 1);
     for (int j0 = 0; j0 <= i_last; j0 += 32) {
         const bool on_diag = (j0 == i0);
         __syncthreads();
         for (int idx = tid; idx < 32 * N; idx += 256) {
             const int jj = idx / N, n = idx % N, j = j0 + jj;
-            const float bv = (j < Q) ? to_f32(Bm[(((size_t)b * Tlen + tk + j) * G + g) * N + n]) : 0.f;
-            const float cj = (j < Q) ? cumk[(size_t)j * N + n] * kL2e : 0.f;
+            const float bv = (j < qv) ? to_f32(Bm[(((size_t)b * Tlen + tk + j) * G + g) * N + n]) : 0.f;
+            const float cj = (j < qv) ? cumk[(size_t)j * N + n] * kL2e : 0.f;
             ct[n * kTS + jj] = cj;
             // off the diagonal: B~_j = B_j exp(cum_e - cum_j), exponent <= 0
             Bt[n * kTS + jj] = on_diag ? bv : bv * ex2_approx(rf[n] - cj);
         }
         for (int idx = tid; idx < 32 * 64; idx += 256) {
             const int jj = idx / 64, p = idx % 64, j = j0 + jj;
-            Xs[jj * kXS + p] = (j < Q && p0 + p < P)
+            Xs[jj * kXS + p] = (j < qv && p0 + p < P)
                                    ? to_f32(x[(((size_t)b * Tlen + tk + j) * H + h) * P + p0 + p])
                                    : 0.f;
         }
         __syncthreads();
         float sc[4] = {0.f, 0.f, 0.f, 0.f};
-        if (i < Q) {
+        if (i < qv) {
             if (on_diag) {
                 const float* ci = Cs + ti * NS;
                 const float* cri = cr + ti * NS;
@@ -150,7 +152,7 @@ __global__ void __launch_bounds__(256) diag_scan_simt_kernel(
             acc[6] = fmaf(cv, hb.z, acc[6]); acc[7] = fmaf(cv, hb.w, acc[7]);
         }
     }
-    if (i >= Q) return;
+    if (i >= qv) return;
     const float dv = D ? D[h] : 0.f;
     const size_t row = (((size_t)b * Tlen + tk + i) * H + h) * P;
 #pragma unroll

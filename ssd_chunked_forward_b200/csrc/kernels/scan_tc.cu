@@ -240,7 +240,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x) {
                 const Item w = decode_item(it, p, B);
-                const int row0 = w.b * p.T + w.j * kBlk;
                 for (int i = 0; i < p.hpb; ++i, ++xc) {
                     const uint32_t st = xc % kStages;
                     if (xc >= kStages &&
@@ -249,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc::mbar_arrive_expect_tx(&bars->x_full[st], kTile);
-                    tc::tma_load_3d(sX + st * kTile, &tm_x, &bars->x_full[st], 0, w.h0 + i, row0);
+                    tc::tma_load_4d(sX + st * kTile, &tm_x, &bars->x_full[st], 0, w.h0 + i, w.j * kBlk, w.b);
                 }
             }
             if (!ok) fail();
@@ -264,16 +263,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             for (int it = blockIdx.x; it < p.n_items; it += gridDim.x, ++itc) {
                 const Item w = decode_item(it, p, B);
-                const int row0 = w.b * p.T + w.j * kBlk;
+                const int t0 = w.j * kBlk;
                 if (itc > 0 && !tc::mbar_wait(&bars->bc_empty, (itc - 1) & 1, abort_v)) {
                     ok = false;
                     break;
                 }
                 tc::mbar_arrive_expect_tx(&bars->bc_full, 4 * kTile);
-                tc::tma_load_3d(sB, &tm_b, &bars->bc_full, 0, w.g, row0);
-                tc::tma_load_3d(sB + kTile, &tm_b, &bars->bc_full, 64, w.g, row0);
-                tc::tma_load_3d(sC, &tm_c, &bars->bc_full, 0, w.g, row0);
-                tc::tma_load_3d(sC + kTile, &tm_c, &bars->bc_full, 64, w.g, row0);
+                tc::tma_load_4d(sB, &tm_b, &bars->bc_full, 0, w.g, t0, w.b);
+                tc::tma_load_4d(sB + kTile, &tm_b, &bars->bc_full, 64, w.g, t0, w.b);
+                tc::tma_load_4d(sC, &tm_c, &bars->bc_full, 0, w.g, t0, w.b);
+                tc::tma_load_4d(sC + kTile, &tm_c, &bars->bc_full, 64, w.g, t0, w.b);
             }
             if (!ok) fail();
             if (itc > 0) tc::mbar_wait(&bars->bc_full, (itc - 1) & 1, nullptr, 200000000ull);
@@ -512,9 +511,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const Item w = decode_item(it, p, B);
                 dnext = (p.D && gt < p.hpb) ? __ldg(p.D + w.h0 + gt) : 0.f;
                 if (MODE == kFused) {
-                    const float* arow = p.a + (size_t)(w.b * p.T + w.j * kBlk + gt) * p.H + w.h0;
+                    // tokens past T (the partial last block) decay by 1: a = 0
+                    const int t = w.j * kBlk + gt;
+                    const float* arow = p.a + ((size_t)w.b * p.T + t) * p.H + w.h0;
 #pragma unroll
-                    for (int i = 0; i < kHpbMax; ++i) anext[i] = i < p.hpb ? __ldg(arow + i) : 0.f;
+                    for (int i = 0; i < kHpbMax; ++i) anext[i] = (i < p.hpb && t < p.T) ? __ldg(arow + i) : 0.f;
                 } else {
 #pragma unroll
                     for (int i = 0; i < kHpbMax; ++i)
@@ -669,7 +670,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool alive = true;
             for (int it = blockIdx.x; alive && it < p.n_items; it += gridDim.x, ++itc) {
                 const Item w = decode_item(it, p, B);
-                const int tok0 = w.b * p.T + w.j * kBlk;
+                const int t0 = w.j * kBlk;
                 const bool last_blk = (w.j == p.nblk - 1);
                 const float* cumbuf = sCum + (itc & 1) * (kHpbMax * kBlk);
                 if (!sync_ok(tc::mbar_wait(&bars->cum_full[itc & 1], (itc >> 1) & 1, abort_v))) break;
@@ -792,7 +793,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (lane == 0) tc::mbar_arrive(&bars->yv_empty[eb]);
                         group_sync();
                         if (gt == 0) {
-                            tc::tma_store_3d(&tm_y, sY, 0, w.h0 + hi, tok0);
+                            tc::tma_store_4d(&tm_y, sY, 0, w.h0 + hi, t0, w.b);  // rows past T are not written
                             tc::bulk_commit();
                         }
                     }
@@ -842,10 +843,11 @@ cudaError_t launch(const Dims& d, const void* x, const void* Bm, const void* Cm,
                    const float* states, uint64_t state_rows, ScanParams p, cudaStream_t st,
                    const float* init = nullptr) {
     CUtensorMap tx, tb, tcm, ty, ts, ti;
-    cudaError_t e = make_tmap_bf16_3d(&tx, x, d.P, d.H, (uint64_t)d.B * d.T, kBlk);
-    if (e == cudaSuccess) e = make_tmap_bf16_3d(&tb, Bm, d.N, d.G, (uint64_t)d.B * d.T, kBlk);
-    if (e == cudaSuccess) e = make_tmap_bf16_3d(&tcm, Cm, d.N, d.G, (uint64_t)d.B * d.T, kBlk);
-    if (e == cudaSuccess) e = make_tmap_bf16_3d(&ty, y, d.P, d.H, (uint64_t)d.B * d.T, kBlk);
+    // [B][T][heads or groups][64 or 128]: a block running past T reads zeros
+    cudaError_t e = make_tmap_bf16_4d(&tx, x, d.P, d.H, d.T, d.B, kBlk);
+    if (e == cudaSuccess) e = make_tmap_bf16_4d(&tb, Bm, d.N, d.G, d.T, d.B, kBlk);
+    if (e == cudaSuccess) e = make_tmap_bf16_4d(&tcm, Cm, d.N, d.G, d.T, d.B, kBlk);
+    if (e == cudaSuccess) e = make_tmap_bf16_4d(&ty, y, d.P, d.H, d.T, d.B, kBlk);
     if (e == cudaSuccess) e = make_tmap_f32_rows64(&ts, states, state_rows);
     // the initial states [B*H*N][P] (a stand-in map over `states` when there are none)
     if (e == cudaSuccess)
@@ -854,7 +856,7 @@ cudaError_t launch(const Dims& d, const void* x, const void* Bm, const void* Cm,
     p.has_init = init ? 1 : 0;
     if (e != cudaSuccess) return e;
     p.T = d.T; p.H = d.H; p.G = d.G;
-    p.nblk = d.T / kBlk;
+    p.nblk = (d.T + kBlk - 1) / kBlk;  // the last block may be partial
     p.hpb = heads_per_item(d);
     p.nslices = d.G * ((d.H / d.G) / p.hpb);
     const long long items = (long long)p.nblk * d.B * p.nslices;
@@ -881,7 +883,7 @@ cudaError_t launch_chunk_scan_tc(const Dims& d, const void* x, const void* Bm, c
     ScanParams p = {};
     p.cum = cum;
     p.D = D;
-    return launch<kScan>(d, x, Bm, Cm, y, Hin, (uint64_t)d.B * d.H * (d.T / kBlk) * kN, p, st);
+    return launch<kScan>(d, x, Bm, Cm, y, Hin, (uint64_t)d.B * d.H * d.nc * kN, p, st);
 }
 
 bool fused_supported(const Dims& d) {

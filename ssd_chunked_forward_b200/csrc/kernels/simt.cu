@@ -29,9 +29,10 @@ __global__ void __launch_bounds__(256) chunk_cumsum_scalar_kernel(const float* _
     const int k = blockIdx.x, b = blockIdx.y, h0 = blockIdx.z * kCumHeads;
     const int hn = min(kCumHeads, H - h0);
     const size_t base = ((size_t)b * T + (size_t)k * Q) * H + h0;
+    const int qv = min(Q, T - k * Q);  // tokens of this chunk before T; the rest count as a = 0
     for (int idx = threadIdx.x; idx < Q * kCumHeads; idx += blockDim.x) {
         const int j = idx / kCumHeads, hh = idx % kCumHeads;
-        sm[idx] = (hh < hn) ? a[base + (size_t)j * H + hh] : 0.f;
+        sm[idx] = (hh < hn && j < qv) ? a[base + (size_t)j * H + hh] : 0.f;
     }
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -64,6 +65,7 @@ __global__ void __launch_bounds__(256) chunk_cumsum_diag_kernel(const float* __r
                                                                 int H, int N, int Q, int nc) {
     const int k = blockIdx.x, bh = blockIdx.y;
     const int b = bh / H, h = bh % H;
+    const int qv = min(Q, T - k * Q);  // tokens past T count as a = 0
     for (int n = threadIdx.x; n < N; n += blockDim.x) {
         const float* src = a + (((size_t)b * T + (size_t)k * Q) * H + h) * N + n;
         float* dst = cum + ((size_t)bh * nc + k) * (size_t)Q * N + n;
@@ -71,7 +73,7 @@ __global__ void __launch_bounds__(256) chunk_cumsum_diag_kernel(const float* __r
         float run = 0.f;
 #pragma unroll 8
         for (int j = 0; j < Q; ++j) {
-            run += src[(size_t)j * step];
+            if (j < qv) run += src[(size_t)j * step];
             dst[(size_t)j * N] = run;
         }
     }
@@ -116,11 +118,12 @@ __global__ void __launch_bounds__(256) chunk_state_simt_kernel(
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
     const float* cumk = cum + ((size_t)bh * nc + k) * (size_t)Q * (DIAG ? N : 1);
-    for (int j0 = 0; j0 < Q; j0 += 32) {
+    const int qv = min(Q, Tlen - k * Q);  // tokens past T add nothing
+    for (int j0 = 0; j0 < qv; j0 += 32) {
         for (int idx = threadIdx.x; idx < 32 * 64; idx += 256) {
             const int jj = idx / 64, c = idx % 64, j = j0 + jj;
             float bv = 0.f, xv = 0.f;
-            if (j < Q) {
+            if (j < qv) {
                 const size_t t = (size_t)k * Q + j;
                 if (n0 + c < N) {
                     float w;
@@ -272,28 +275,30 @@ __global__ void __launch_bounds__(256) chunk_scan_simt_kernel(
     const int tid = threadIdx.x, ti = tid >> 3, tp = tid & 7;
     const float* cumk = cum + ((size_t)bh * nc + k) * (size_t)Q;
     const size_t tk = (size_t)k * Q;
+    const int qv = min(Q, Tlen - k * Q);  // rows of this chunk before T
+    if (i0 >= qv) return;                 // a tile wholly past T (the whole block leaves)
 
     for (int idx = tid; idx < 32 * N; idx += 256) {
         const int ii = idx / N, n = idx % N, i = i0 + ii;
-        Cs[ii * NS + n] = (i < Q) ? to_f32(Cm[(((size_t)b * Tlen + tk + i) * G + g) * N + n]) : 0.f;
+        Cs[ii * NS + n] = (i < qv) ? to_f32(Cm[(((size_t)b * Tlen + tk + i) * G + g) * N + n]) : 0.f;
     }
-    if (tid < 32) cr[tid] = (i0 + tid < Q) ? cumk[i0 + tid] : 0.f;
+    if (tid < 32) cr[tid] = (i0 + tid < qv) ? cumk[i0 + tid] : 0.f;
 
     float acc[8];
 #pragma unroll
     for (int m = 0; m < 8; ++m) acc[m] = 0.f;
-    const int i_last = min(i0 + 31, Q - 1);
+    const int i_last = min(i0 + 31, qv - 1);
     for (int j0 = 0; j0 <= i_last; j0 += 32) {
         __syncthreads();
         for (int idx = tid; idx < 32 * N; idx += 256) {
             const int jj = idx / N, n = idx % N, j = j0 + jj;
             Bs[jj * NS + n] =
-                (j < Q) ? to_f32(Bm[(((size_t)b * Tlen + tk + j) * G + g) * N + n]) : 0.f;
+                (j < qv) ? to_f32(Bm[(((size_t)b * Tlen + tk + j) * G + g) * N + n]) : 0.f;
         }
-        if (tid < 32) cc[tid] = (j0 + tid < Q) ? cumk[j0 + tid] : 0.f;
+        if (tid < 32) cc[tid] = (j0 + tid < qv) ? cumk[j0 + tid] : 0.f;
         for (int idx = tid; idx < 32 * 64; idx += 256) {
             const int jj = idx / 64, p = idx % 64, j = j0 + jj;
-            Xs[jj * 65 + p] = (j < Q && p0 + p < P)
+            Xs[jj * 65 + p] = (j < qv && p0 + p < P)
                                   ? to_f32(x[(((size_t)b * Tlen + tk + j) * H + h) * P + p0 + p])
                                   : 0.f;
         }
@@ -303,7 +308,7 @@ __global__ void __launch_bounds__(256) chunk_scan_simt_kernel(
             const int jj = tp * 4 + c;
             const int i = i0 + ti, j = j0 + jj;
             float s = 0.f;
-            if (j <= i && i < Q) {
+            if (j <= i && i < qv) {
                 const float* ci = Cs + ti * NS;
                 const float* bj = Bs + jj * NS;
                 for (int n = 0; n < N; ++n) s = fmaf(ci[n], bj[n], s);
@@ -339,7 +344,7 @@ __global__ void __launch_bounds__(256) chunk_scan_simt_kernel(
         }
     }
     const int i = i0 + ti;
-    if (i >= Q) return;
+    if (i >= qv) return;
     const float sc = expf(cr[ti]);
     const float dv = D ? D[h] : 0.f;
     const size_t row = (((size_t)b * Tlen + tk + i) * H + h) * P;

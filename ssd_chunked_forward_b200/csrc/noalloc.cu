@@ -50,16 +50,10 @@ ssd_status scratch_address(void** out) {
 
 }  // namespace
 
-namespace ssd {
-ssd_shape forward_shape(const ssd_shape* s);  // ssd_api.cu: the chunk used for T % chunk != 0
-}
-
-extern "C" ssd_status ssd_forward_noalloc(const ssd_shape* shape_in, const void* x, const float* a,
+extern "C" ssd_status ssd_forward_noalloc(const ssd_shape* shape, const void* x, const float* a,
                                           const void* Bm, const void* Cm, const float* D, void* y,
                                           float* final_state, ssd_stream stream) {
-    if (!shape_in) return SSD_ERR_INVALID_ARG;
-    const ssd_shape fs = ssd::forward_shape(shape_in);
-    const ssd_shape* shape = &fs;
+    if (!shape) return SSD_ERR_INVALID_ARG;
     if (ssd_workspace_size(shape) == 0) return SSD_ERR_INVALID_ARG;  // invalid shape
     if (!x || !a || !Bm || !Cm || !y) return SSD_ERR_INVALID_ARG;
     const uintptr_t m = (uintptr_t)x | (uintptr_t)a | (uintptr_t)Bm | (uintptr_t)Cm |
@@ -78,7 +72,7 @@ extern "C" ssd_status ssd_forward_noalloc(const ssd_shape* shape_in, const void*
 
     ssd::Dims d;
     d.B = shape->B; d.T = shape->T; d.H = shape->H; d.P = shape->P; d.G = shape->G;
-    d.N = shape->N; d.Q = shape->chunk; d.nc = shape->T / shape->chunk;
+    d.N = shape->N; d.Q = shape->chunk; d.nc = (shape->T + shape->chunk - 1) / shape->chunk;
     d.diag = shape->a_per_state != 0;
     d.bf16 = shape->dtype == SSD_DTYPE_BF16;
 

@@ -26,12 +26,13 @@ ssd_status check_shape(const ssd_shape* s) {
     if (!s) return SSD_ERR_INVALID_ARG;
     if (s->B < 1 || s->T < 1 || s->H < 1 || s->P < 1 || s->G < 1 || s->N < 1 || s->chunk < 1)
         return SSD_ERR_INVALID_ARG;
-    if (s->T % s->chunk != 0 || s->H % s->G != 0) return SSD_ERR_INVALID_ARG;
+    if (s->H % s->G != 0) return SSD_ERR_INVALID_ARG;
     if (s->chunk > 1024 || s->N > 256 || s->P > 256) return SSD_ERR_INVALID_ARG;
+    if (s->T > 0x7fffffff - 1024) return SSD_ERR_INVALID_ARG;  // k * chunk + j stays an int
     if (s->dtype != SSD_DTYPE_F32 && s->dtype != SSD_DTYPE_BF16) return SSD_ERR_INVALID_ARG;
     if (s->a_per_state != 0 && s->a_per_state != 1) return SSD_ERR_INVALID_ARG;
     // every flattened index fits comfortably in 63 bits; guard the int grid dims
-    const long long nc = s->T / s->chunk;
+    const long long nc = ((long long)s->T + s->chunk - 1) / s->chunk;
     if ((long long)s->B * s->H > 0x7fffffffLL || nc * ((s->chunk + 31) / 32) > 0x7fffffffLL)
         return SSD_ERR_INVALID_ARG;
     return SSD_OK;
@@ -40,7 +41,7 @@ ssd_status check_shape(const ssd_shape* s) {
 Dims dims_of(const ssd_shape* s) {
     Dims d;
     d.B = s->B; d.T = s->T; d.H = s->H; d.P = s->P; d.G = s->G; d.N = s->N; d.Q = s->chunk;
-    d.nc = s->T / s->chunk;
+    d.nc = (s->T + s->chunk - 1) / s->chunk;  // the last chunk may end past T
     d.diag = s->a_per_state != 0;
     d.bf16 = s->dtype == SSD_DTYPE_BF16;
     return d;
@@ -53,7 +54,7 @@ Dims modular_dims(const Dims& d) {
     Dims e = d;
     if (d.Q % 128 == 0 && d.Q > 128) {
         e.Q = 128;
-        e.nc = d.T / 128;
+        e.nc = (d.T + 127) / 128;
         if (!ssd::chunk_scan_tc_supported(e)) return d;
     }
     return e;
@@ -128,26 +129,6 @@ ssd_status run_modular(const Dims& d0, const void* x, const float* a, const void
 }  // namespace
 
 namespace ssd {
-// The forward-level entry points accept T % chunk != 0: the result does not
-// depend on the chunk (the chunked evaluation is exact for every chunk), so
-// they run with the largest chunk <= the requested one that divides T,
-// preferring a multiple of 128 (the tensor-core block) when T allows one.
-ssd_shape forward_shape(const ssd_shape* s) {
-    ssd_shape r = *s;
-    if (s->T < 1 || s->chunk < 1 || s->T % s->chunk == 0) return r;
-    int q = 0;
-    if (s->T % 128 == 0)
-        for (int c = (s->chunk / 128) * 128; c >= 128 && !q; c -= 128)
-            if (s->T % c == 0) q = c;
-    for (int c = s->chunk < s->T ? s->chunk : s->T; c >= 1 && !q; --c)
-        if (s->T % c == 0) q = c;
-    r.chunk = q;
-    return r;
-}
-
-}  // namespace ssd
-
-namespace ssd {
 cudaError_t launch_fused_ordered(const Dims& d, const void* x, const float* a, const void* Bm,
                                  const void* Cm, const float* D, void* y, float* fin, float* ring,
                                  unsigned* flags, int* status, bool test_stall, cudaStream_t st,
@@ -189,18 +170,14 @@ const char* ssd_status_string(ssd_status s) {
     return "SSD_ERR_UNKNOWN";
 }
 
-size_t ssd_workspace_size(const ssd_shape* shape_in) {
-    if (!shape_in) return 0;
-    const ssd_shape fs = ssd::forward_shape(shape_in);
-    const ssd_shape* shape = &fs;
+size_t ssd_workspace_size(const ssd_shape* shape) {
+    if (!shape) return 0;
     if (check_shape(shape) != SSD_OK) return 0;
     return workspace_bytes(dims_of(shape));
 }
 
-int ssd_path_supported(const ssd_shape* shape_in, unsigned path) {
-    if (!shape_in) return 0;
-    const ssd_shape fs = ssd::forward_shape(shape_in);
-    const ssd_shape* shape = &fs;
+int ssd_path_supported(const ssd_shape* shape, unsigned path) {
+    if (!shape) return 0;
     if (check_shape(shape) != SSD_OK) return 0;
     const Dims d = dims_of(shape);
     switch (path) {
@@ -212,10 +189,8 @@ int ssd_path_supported(const ssd_shape* shape_in, unsigned path) {
     }
 }
 
-int ssd_auto_path(const ssd_shape* shape_in) {
-    if (!shape_in) return -1;
-    const ssd_shape fs = ssd::forward_shape(shape_in);
-    const ssd_shape* shape = &fs;
+int ssd_auto_path(const ssd_shape* shape) {
+    if (!shape) return -1;
     if (check_shape(shape) != SSD_OK) return -1;
     const Dims d = dims_of(shape);
     // fewer chains than this: the fused kernel's per-block hand-off (~4 us on
@@ -226,13 +201,11 @@ int ssd_auto_path(const ssd_shape* shape_in) {
     return SSD_PATH_MODULAR;
 }
 
-ssd_status ssd_forward_init(const ssd_shape* shape_in, const void* x, const float* a, const void* Bm,
+ssd_status ssd_forward_init(const ssd_shape* shape, const void* x, const float* a, const void* Bm,
                             const void* Cm, const float* D, const float* initial_state, void* y,
                             float* final_state, void* workspace, size_t ws_bytes,
                             ssd_stream stream, unsigned path, unsigned flags) {
-    if (!shape_in) return SSD_ERR_INVALID_ARG;
-    const ssd_shape fs = ssd::forward_shape(shape_in);
-    const ssd_shape* shape = &fs;
+    if (!shape) return SSD_ERR_INVALID_ARG;
     ssd_status st = check_shape(shape);
     if (st != SSD_OK) return st;
     if (!x || !a || !Bm || !Cm || !y) return SSD_ERR_INVALID_ARG;
@@ -302,21 +275,17 @@ static size_t host_layout(const ssd_shape* s, size_t off[8]) {
     return total;
 }
 
-size_t ssd_forward_host_bytes(const ssd_shape* shape_in) {
-    if (!shape_in) return 0;
-    const ssd_shape fs = ssd::forward_shape(shape_in);
-    const ssd_shape* shape = &fs;
+size_t ssd_forward_host_bytes(const ssd_shape* shape) {
+    if (!shape) return 0;
     if (check_shape(shape) != SSD_OK) return 0;
     size_t off[8];
     return host_layout(shape, off);
 }
 
-ssd_status ssd_forward_host(const ssd_shape* shape_in, const void* x_h, const float* a_h,
+ssd_status ssd_forward_host(const ssd_shape* shape, const void* x_h, const float* a_h,
                             const void* Bm_h, const void* Cm_h, const float* D_h, void* y_h,
                             float* final_h, void* dev_buf, size_t dev_bytes, ssd_stream stream) {
-    if (!shape_in) return SSD_ERR_INVALID_ARG;
-    const ssd_shape fs = ssd::forward_shape(shape_in);
-    const ssd_shape* shape = &fs;
+    if (!shape) return SSD_ERR_INVALID_ARG;
     ssd_status st = check_shape(shape);
     if (st != SSD_OK) return st;
     if (!x_h || !a_h || !Bm_h || !Cm_h || !y_h) return SSD_ERR_INVALID_ARG;

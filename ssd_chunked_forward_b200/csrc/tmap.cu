@@ -27,16 +27,19 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
-cudaError_t make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
-                              uint64_t d2, uint32_t box_rows) {
+cudaError_t make_tmap_bf16_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
+                              uint64_t d2, uint64_t d3, uint32_t box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return cudaErrorNotSupported;
     if (((uintptr_t)base & 15u) != 0 || (d0 * 2) % 16 != 0) return cudaErrorInvalidValue;
-    const cuuint64_t dims[3] = {d0, d1, d2};
-    const cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};  // bytes, dims 1 and 2
-    const cuuint32_t box[3] = {64, 1, box_rows};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+    const cuuint64_t dims[4] = {d0, d1, d2, d3};
+    const cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};  // bytes, dims 1..3
+    const cuuint32_t box[4] = {64, 1, box_rows, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    // elements outside the tensor read as zero (OOB_FILL_NONE) and are not
+    // written by stores: a box that runs past a sequence's last token is the
+    // zero padding of the partial last chunk
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;

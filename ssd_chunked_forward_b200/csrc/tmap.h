@@ -8,12 +8,15 @@
 
 namespace ssd {
 
-// A 3-D bf16 tensor map over a row-major [d2][d1][d0] array (d0 innermost),
-// box (64, 1, rows) with 128-byte swizzle: one box is `rows` rows of 64
-// elements = 128 bytes, landing in shared memory as rows of 128 bytes.
-// Returns cudaSuccess or an error (bad alignment, missing driver entry point).
-cudaError_t make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
-                              uint64_t d2, uint32_t box_rows);
+// A 4-D bf16 tensor map over a row-major [d3][d2][d1][d0] array (d0
+// innermost; for the token tensors d3 = batch, d2 = tokens, d1 = heads or
+// groups), box (64, 1, rows, 1) with 128-byte swizzle: one box is `rows`
+// tokens of 64 elements = 128 bytes, landing in shared memory as rows of 128
+// bytes.  Rows past d2 read as zero and are not stored, so a box never
+// crosses into the next batch row.  Returns cudaSuccess or an error (bad
+// alignment, missing driver entry point).
+cudaError_t make_tmap_bf16_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
+                              uint64_t d2, uint64_t d3, uint32_t box_rows);
 
 // A 2-D fp32 tensor map over a row-major [rows][64] array, box (32, 128) with
 // 128-byte swizzle: one box is 128 rows of 32 floats = 128 bytes; a 128 x 64

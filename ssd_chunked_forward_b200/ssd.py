@@ -204,7 +204,7 @@ def device_status(workspace, stream=None) -> int:
 
 
 def chunk_cumsum(shape: Shape, a, cum=None, stream=None):
-    nc = shape.T // shape.chunk
+    nc = -(-shape.T // shape.chunk)  # the last chunk may end past T
     if cum is None:
         dims = (shape.B, shape.H, nc, shape.chunk) + ((shape.N,) if shape.a_per_state else ())
         cum = torch.empty(dims, dtype=torch.float32, device=a.device)
@@ -214,7 +214,7 @@ def chunk_cumsum(shape: Shape, a, cum=None, stream=None):
 
 
 def chunk_state(shape: Shape, x, Bm, cum, states=None, impl=IMPL_AUTO, stream=None):
-    nc = shape.T // shape.chunk
+    nc = -(-shape.T // shape.chunk)  # the last chunk may end past T
     if states is None:
         states = torch.empty((shape.B, shape.H, nc, shape.N, shape.P), dtype=torch.float32,
                              device=x.device)

@@ -43,7 +43,7 @@ class Workload:
 
     @property
     def nc(self) -> int:
-        return self.T // self.chunk
+        return -(-self.T // self.chunk)
 
     @property
     def tokens(self) -> int:

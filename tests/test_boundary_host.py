@@ -79,35 +79,20 @@ def test_invalid_shapes_rejected(lib, bad):
     assert code == ssd.SSD_ERR_INVALID_ARG
 
 
-def _forward_chunk(T, chunk):
-    """The chunk the whole forward runs with: the largest one <= chunk that
-    divides T, a multiple of 128 when T has one (chunk invariance)."""
-    if T % chunk == 0:
-        return chunk
-    if T % 128 == 0:
-        for c in range(chunk // 128 * 128, 127, -128):
-            if T % c == 0:
-                return c
-    return max(c for c in range(1, min(chunk, T) + 1) if T % c == 0)
-
-
 @pytest.mark.parametrize("T,chunk", [(500, 256), (1000, 256), (997, 256), (384, 256),
                                      (640, 512), (1024, 1000), (96, 256)])
-def test_ragged_T_accepted_by_whole_forward(lib, T, chunk):
-    """T % chunk != 0: the whole forward runs with a smaller chunk that
-    divides T, so its workspace is that shape's and the step entry points,
-    which keep the requested chunk, still refuse the shape."""
+def test_ragged_T_is_a_partial_last_chunk(lib, T, chunk):
+    """T % chunk != 0: the last chunk holds the remaining tokens; the buffers
+    are laid out for ceil(T / chunk) chunks (ceil(T / 128) blocks on the
+    tensor-core modular path), never more than the padded length needs, and
+    the paths served and AUTO's choice equal those of the padded length."""
     s = _shape(T=T, chunk=chunk)
-    q = _forward_chunk(T, chunk)
-    assert ssd.workspace_size(s) == ssd.workspace_size(_shape(T=T, chunk=q)) > 0
-    assert ssd.path_supported(s, ssd.PATH_AUTO)
-    assert ssd.path_supported(s, ssd.PATH_MODULAR)
-    # the tensor-core paths need a 128-multiple chunk
-    assert ssd.path_supported(s, ssd.PATH_FUSED) == (q % 128 == 0)
-    assert ssd.auto_path(s) == ssd.auto_path(_shape(T=T, chunk=q))
-    if T % chunk:
-        ok = 1 << 20
-        assert lib.ssd_chunk_cumsum(ctypes.byref(s), ok, ok, None) == ssd.SSD_ERR_INVALID_ARG
+    Tp = -(-T // chunk) * chunk
+    padded = _shape(T=Tp, chunk=chunk)
+    assert 0 < ssd.workspace_size(s) <= ssd.workspace_size(padded)
+    for path in (ssd.PATH_AUTO, ssd.PATH_SIMT, ssd.PATH_MODULAR, ssd.PATH_FUSED):
+        assert ssd.path_supported(s, path) == ssd.path_supported(padded, path)
+    assert ssd.auto_path(s) == ssd.auto_path(padded)
 
 
 def test_null_and_misaligned_pointers_rejected(lib):
@@ -168,7 +153,7 @@ def test_auto_path_choice(lib):
     assert ssd.auto_path(ssd.make_shape(1, 262144, 32, 64, 8, 128, 256)) == ssd.PATH_MODULAR  # 32
     assert ssd.auto_path(ssd.make_shape(4, 8192, 80, 64, 1, 128, 256, dtype="f32")) == ssd.PATH_MODULAR
     assert ssd.auto_path(ssd.make_shape(4, 4096, 16, 64, 1, 64, 128, a_per_state=True)) == ssd.PATH_MODULAR
-    # T % chunk != 0 runs with chunk 50 (divides 100), on the modular path
+    # T % chunk != 0: a partial last chunk; 2 chains is few, so modular
     assert ssd.auto_path(ssd.make_shape(1, 100, 2, 64, 1, 128, 64)) == ssd.PATH_MODULAR
     assert ssd.auto_path(ssd.make_shape(1, 100, 3, 64, 2, 128, 64)) == -1  # H % G != 0
 

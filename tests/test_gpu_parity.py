@@ -49,16 +49,21 @@ EDGE = [
     small_case(B=1, T=1024, H=1, P=8, N=8, G=1, chunk=1024, dtype="f32", seed=12),
 ]
 
-# T % chunk != 0: the whole forward runs with the largest chunk <= the
-# requested one that divides T (chunk invariance), so these reach the fused
-# kernel (T=384 -> 128, T=640 -> 128) and the CUDA-core paths (T=1000 -> 250,
-# T=997 -> 1, T=200 -> 100)
+# T % chunk != 0: the last chunk (and, on the tensor-core paths, the last
+# 128-token block) holds the remaining tokens; the kernels read zeros past T
+# and write nothing there
 RAGGED = [
     small_case(B=1, T=384, H=4, P=64, N=128, G=1, chunk=256, dtype="bf16", seed=71),
-    small_case(B=2, T=640, H=3, P=64, N=128, G=1, chunk=512, dtype="bf16", seed=72),
     small_case(B=1, T=1000, H=2, P=64, N=128, G=1, chunk=256, dtype="bf16", seed=73),
+    small_case(B=2, T=77, H=3, P=64, N=128, G=1, chunk=256, dtype="bf16", seed=72),
+    small_case(B=2, T=4000, H=8, P=64, N=128, G=2, chunk=256, dtype="bf16", seed=76),
     small_case(B=1, T=997, H=2, P=12, N=10, G=1, chunk=256, dtype="f32", seed=74),
     small_case(B=2, T=200, H=2, P=16, N=24, G=2, chunk=128, dtype="f32", a_per_state=True, seed=75),
+]
+# per-step cases with a partial last chunk (tensor-core steps take chunk 128)
+STEP_RAGGED = [
+    small_case(B=2, T=333, H=3, P=64, N=128, G=1, chunk=128, dtype="bf16", seed=77),
+    small_case(B=1, T=150, H=2, P=20, N=12, G=1, chunk=64, dtype="f32", a_per_state=True, seed=78),
 ]
 
 
@@ -90,21 +95,27 @@ def test_forward_matches_oracle(w, path):
 
 
 def _oracle_chunked(inp, w):
-    """O3 per chain, as [B,H,...] float64 arrays."""
-    prob = O.Problem(*(inp[k].to(torch.float64).numpy() for k in ("x", "a", "Bm", "Cm", "D")))
+    """O3 per chain, as [B,H,...] float64 arrays.  A partial last chunk is
+    the input padded with a = 0 and x = B = C = 0 (the padding is pinned on
+    the CPU to leave y[:T] and the final state unchanged)."""
+    arrs = [inp[k].to(torch.float64).numpy() for k in ("x", "a", "Bm", "Cm")]
+    nc = -(-w.T // w.chunk)
+    Tp = nc * w.chunk
+    if Tp != w.T:
+        arrs = [np.pad(v, [(0, 0), (0, Tp - w.T)] + [(0, 0)] * (v.ndim - 2)) for v in arrs]
+    prob = O.Problem(*arrs, inp["D"].to(torch.float64).numpy())
     r = O.chunked(prob, w.chunk)
-    nc = w.T // w.chunk
     cum = r["cum"].reshape(w.B, w.H, nc, w.chunk, -1)
     if not w.a_per_state:
         cum = cum[..., 0]
     S = r["S"].reshape(w.B, w.H, nc, w.N, w.P)
     Hin = r["Hin"].reshape(w.B, w.H, nc, w.N, w.P)
-    y = r["y"].reshape(w.B, w.H, w.T, w.P).transpose(0, 2, 1, 3)
+    y = r["y"].reshape(w.B, w.H, Tp, w.P).transpose(0, 2, 1, 3)[:, : w.T]
     fin = r["final"].reshape(w.B, w.H, w.N, w.P)
     return cum, S, Hin, y, fin
 
 
-@pytest.mark.parametrize("w", CASES, ids=_ids(CASES))
+@pytest.mark.parametrize("w", CASES + STEP_RAGGED, ids=_ids(CASES + STEP_RAGGED))
 def test_step_chunk_cumsum(w):
     inp = generate(w)
     dev = to_dev(inp)
@@ -115,7 +126,7 @@ def test_step_chunk_cumsum(w):
     assert rel_err(cum.cpu().numpy().astype(np.float64), ref) < 1e-5
 
 
-@pytest.mark.parametrize("w", CASES, ids=_ids(CASES))
+@pytest.mark.parametrize("w", CASES + STEP_RAGGED, ids=_ids(CASES + STEP_RAGGED))
 @pytest.mark.parametrize("impl", [ssd.IMPL_SIMT, ssd.IMPL_TC], ids=["simt", "tc"])
 def test_step_chunk_state(w, impl):
     inp = generate(w)
@@ -133,7 +144,7 @@ def test_step_chunk_state(w, impl):
     assert rel_err(got.cpu().numpy().astype(np.float64), S) <= tol_for(w)
 
 
-@pytest.mark.parametrize("w", CASES, ids=_ids(CASES))
+@pytest.mark.parametrize("w", CASES + STEP_RAGGED, ids=_ids(CASES + STEP_RAGGED))
 def test_step_state_pass(w):
     inp = generate(w)
     shape = ssd.make_shape(w.B, w.T, w.H, w.P, w.G, w.N, w.chunk, w.a_per_state, w.dtype)
@@ -147,7 +158,7 @@ def test_step_state_pass(w):
     assert rel_err(fin_d.cpu().numpy().astype(np.float64), fin) < 1e-5
 
 
-@pytest.mark.parametrize("w", CASES, ids=_ids(CASES))
+@pytest.mark.parametrize("w", CASES + STEP_RAGGED, ids=_ids(CASES + STEP_RAGGED))
 @pytest.mark.parametrize("impl", [ssd.IMPL_SIMT, ssd.IMPL_TC], ids=["simt", "tc"])
 def test_step_chunk_scan(w, impl):
     inp = generate(w)

@@ -278,6 +278,40 @@ def test_initial_state_free_response(per_state):
     assert rel_inf(res["final"].reshape(fin_ref.shape), fin_ref) < 1e-12
 
 
+def pad_problem(prob, Tp):
+    """The problem extended to Tp tokens with a = 0 and x = B = C = 0 past T:
+    the reading of a partial last chunk (tokens past T decay by 1 and carry no
+    input and no readout)."""
+    T = prob.x.shape[1]
+    def ext(arr):
+        w = [(0, 0)] * arr.ndim
+        w[1] = (0, Tp - T)
+        return np.pad(arr, w)
+    return O.Problem(ext(prob.x), ext(prob.a), ext(prob.Bm), ext(prob.Cm), prob.D)
+
+
+@pytest.mark.parametrize("per_state", [False, True])
+@pytest.mark.parametrize("T,q", [(13, 4), (30, 8), (7, 16)])
+def test_zero_padding_is_a_partial_last_chunk(per_state, T, q):
+    """Padding past T with a = 0 and x = B = C = 0 leaves y[:T] and the final
+    state of the recurrence exactly as they were (each padded step multiplies
+    the state by e^0 = 1 and adds B x^T = 0), and the chunked form over the
+    padded length agrees with the unpadded recurrence: the padded chunk count
+    ceil(T / q) with a partial last chunk is the same operator."""
+    rng = np.random.default_rng(61 + T + per_state)
+    prob = random_problem(rng, B=2, T=T, H=3, P=4, G=1, N=5, per_state=per_state)
+    B, _, H, _ = prob.x.shape
+    Tp = -(-T // q) * q
+    ref = O.recurrence(prob)
+    padded = pad_problem(prob, Tp)
+    rp = O.recurrence(padded)
+    assert np.array_equal(all_y(rp, B, H)[:, :, :T], all_y(ref, B, H))
+    assert np.array_equal(rp["final"], ref["final"])
+    rc = O.chunked(padded, q)
+    assert rel_inf(all_y(rc, B, H)[:, :, :T], all_y(ref, B, H)) < 1e-12
+    assert rel_inf(rc["final"], ref["final"]) < 1e-12
+
+
 def test_zero_initial_state_is_the_default():
     rng = np.random.default_rng(51)
     prob = random_problem(rng, B=2, T=9, H=2, P=3, G=2, N=4)
