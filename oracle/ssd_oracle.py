@@ -9,6 +9,8 @@ Routes (see the C file for the equations and their sources):
   recurrence(...)  O1, the step recurrence h_t = e^{a_t} h_{t-1} + B_t x_t^T
   brute(...)       O2, the materialised 1-semiseparable matrix (tiny T)
   chunked(...)     O3, the chunked algorithm with every intermediate
+  backward(...)    O4, gradients of the recurrence by its adjoint (numpy fp64)
+  discretize(...)  the selective discretisation in front of the operator (numpy)
 
 Parity is pinned for every route (tests/test_oracle_pins.py); nothing here is
 "parity unpinned".
@@ -244,3 +246,63 @@ def discretize(dt_raw, dt_bias, A_log, x):
         a = dt[..., None] * A[None, None, :, :]
     xd = dt[..., None] * np.asarray(x, dtype=np.float64)
     return a, xd, dt
+
+
+def backward(prob: Problem, dy, dfinal=None, initial=None):
+    """Gradients of the scalar l = sum_t dy_t . y_t + <dfinal, h_{T-1}> with
+    respect to every input, by reverse-mode differentiation of the step
+    recurrence (O1): the plain definition, in fp64 numpy, with every state
+    h_t kept (the pages' kernels recompute the states in the backward pass
+    instead of storing them -- llms.blog "State Space Models and Mamba ...",
+    "Hardware-Aware Parallel Associative Scan", item on the direct output
+    projection).
+
+    Forward   h_t = e^{a_t} o h_{t-1} + B_t x_t^T,  y_t = h_t^T C_t + D x_t
+    Adjoint   g_t = dl/dh_t = C_t dy_t^T + e^{a_{t+1}} o g_{t+1},
+              g_{T-1} = C_{T-1} dy_{T-1}^T + dfinal
+    then      dx_t = g_t^T B_t + D dy_t        dB_t = g_t x_t (summed over a group's heads)
+              dC_t = h_t dy_t                  da_t = <g_t, e^{a_t} o h_{t-1}>  (per n if per-state)
+              dD   = sum_t dy_t . x_t          d initial = e^{a_0} o g_0
+    dy [B,T,H,P], dfinal / initial [B,H,N,P] or None (zero).  Returns a dict
+    dx, da, dBm, dCm, dD, dinit with the inputs' shapes."""
+    p = _prep(prob)
+    B, T, H, P, G, N = p.dims
+    hg = H // G
+    dy = _f64(dy)
+    per_state = p.a_per_state
+    grp = np.arange(H) // hg
+    h = np.zeros((B, H, N, P)) if initial is None else _f64(initial).copy()
+    hs = np.zeros((T + 1, B, H, N, P))  # hs[t + 1] = h_t, hs[0] = h_{-1}
+    hs[0] = h
+    for t in range(T):
+        e = np.exp(p.a[:, t])                                  # [B,H] or [B,H,N]
+        e = e[..., None, None] if not per_state else e[..., None]
+        Bt = p.Bm[:, t][:, grp]                                # [B,H,N]
+        h = e * h + Bt[..., None] * p.x[:, t][:, :, None, :]
+        hs[t + 1] = h
+    g = np.zeros((B, H, N, P)) if dfinal is None else _f64(dfinal).copy()
+    dx = np.zeros_like(p.x)
+    da = np.zeros_like(p.a)
+    dBh = np.zeros((B, T, H, N))
+    dCh = np.zeros((B, T, H, N))
+    Dv = np.zeros(H) if p.D is None else p.D
+    for t in range(T - 1, -1, -1):
+        Ct = p.Cm[:, t][:, grp]                                # [B,H,N]
+        Bt = p.Bm[:, t][:, grp]
+        g = g + Ct[..., None] * dy[:, t][:, :, None, :]        # g_t
+        dx[:, t] = np.einsum("bhnp,bhn->bhp", g, Bt) + Dv[None, :, None] * dy[:, t]
+        dBh[:, t] = np.einsum("bhnp,bhp->bhn", g, p.x[:, t])
+        dCh[:, t] = np.einsum("bhnp,bhp->bhn", hs[t + 1], dy[:, t])
+        e = np.exp(p.a[:, t])
+        if per_state:
+            da[:, t] = np.einsum("bhnp,bhnp->bhn", g, e[..., None] * hs[t])
+            g = e[..., None] * g
+        else:
+            da[:, t] = np.einsum("bhnp,bhnp->bh", g, hs[t]) * e
+            g = e[..., None, None] * g
+    dBm = dBh.reshape(B, T, G, hg, N).sum(axis=3)
+    dCm = dCh.reshape(B, T, G, hg, N).sum(axis=3)
+    dD = np.einsum("bthp,bthp->h", dy, p.x)
+    return {"dx": dx, "da": da, "dBm": dBm, "dCm": dCm, "dD": dD, "dinit": g,
+            "y": np.einsum("tbhnp,bthn->bthp", hs[1:], p.Cm[:, :, grp]) + Dv[None, None, :, None] * p.x,
+            "final": hs[T]}
