@@ -369,6 +369,78 @@ def run_decode(args, device):
     return 0
 
 
+# fp32 FMA issue rate of the CUDA cores: 148 SMs x 128 fp32 lanes x 2 flops
+# x 1.965 GHz (the part's maximum SM clock)
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def backward_flops(w):
+    """Algorithmic flops of the chunked backward: per chain and chunk, four
+    quadratic forms (pair scores over K plus pair-weighted sums over Mc, with
+    K + Mc = N + P, on the Q (Q + 1) / 2 causal pairs, plus the Q x K x Mc
+    boundary term) and three chunk-state contractions (the recomputed states,
+    the adjoint readout states; Q x N x P each, the boundary terms counted
+    above)."""
+    Q, N, P = w.chunk, w.N, w.P
+    nc = -(-w.T // Q)
+    per_chunk = 4 * (Q * (Q + 1) * (N + P) + 2 * Q * N * P) + 2 * (2 * Q * N * P)
+    return w.B * w.H * nc * per_chunk
+
+
+def run_backward(args, device):
+    """ssd_backward on the workload: dy (and a loss on the final state) in, the
+    six gradients out; L2 flushed before every step.  The backward runs on
+    CUDA cores in fp32, so its roofline is the fp32 FMA rate."""
+    w = WORKLOADS[args.workload]
+    if args.B or args.T:
+        w = w.scaled(B=args.B or w.B, T=args.T or w.T, name=w.name + f"_B{args.B or w.B}_T{args.T or w.T}")
+    dev = {k: (v.to(device) if v is not None else None) for k, v in generate(w).items()}
+    g = torch.Generator().manual_seed(w.seed + 700)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    dy = torch.randn((w.B, w.T, w.H, w.P), generator=g).to(dt).to(device)
+    dfin = torch.randn((w.B, w.H, w.N, w.P), generator=g).to(device)
+    shape = ssd.shape_of(dev["x"], dev["a"], dev["Bm"], w.chunk)
+    ws = torch.empty(ssd.backward_workspace_size(shape), dtype=torch.uint8, device=device)
+    scratch = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    st = torch.cuda.current_stream()
+    call = lambda: ssd.backward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], dev["D"], dy, w.chunk,
+                                dfinal=dfin, workspace=ws)
+    for _ in range(args.warmup):
+        scratch.fill_(1)
+        call()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for e0, e1 in ev:
+        scratch.fill_(1)
+        e0.record(st)
+        call()
+        e1.record(st)
+    torch.cuda.synchronize()
+    ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev)
+    el = 2 if w.dtype == "bf16" else 4
+    tok = w.B * w.T
+    byts = (2 * 2 * tok * w.H * w.P * el + 2 * tok * w.H * 4 + 2 * 2 * tok * w.G * w.N * el
+            + 2 * w.B * w.H * w.N * w.P * 4 + 2 * w.H * 4)
+    flops = backward_flops(w)
+    achieved = flops / (ms / 1e3) / 1e12
+    peaks, src = load_peaks()
+    print(json.dumps({
+        "metric": "SSD backward tokens/s", "value": tok / (ms / 1e3), "unit": "tokens/s",
+        "ms_per_step": ms, "steps": args.steps, "warmup": args.warmup, "dtype": w.dtype,
+        "data": "synthetic",
+        "config": {"workload": w.name + "_backward", "B": w.B, "T": w.T, "H": w.H, "P": w.P,
+                   "N": w.N, "G": w.G, "chunk": w.chunk, "loss": "sum(dy * y) + <dfinal, final>",
+                   "l2": "flushed (256 MB write) before every step"},
+        "roofline": {"bound": "alu", "achieved": achieved, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
+                     "frac": achieved / FP32_ALU_TFLOPS, "algorithmic_flops_per_step": flops,
+                     "kernel": "ssd_backward (13 launches)",
+                     "peak_source": "fp32 FMA rate from unit counts and the maximum SM clock"},
+        "hbm_view": {"algorithmic_bytes_per_step": byts, "achieved_gbs": byts / (ms / 1e3) / 1e9,
+                     "frac_of_measured_hbm": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]},
+        "gpu_launches": 13 * args.steps}))
+    return 0
+
+
 def run_discretize(args, device):
     """ssd_discretize on the workload's shape: dt_raw and x in, a and x_out out,
     each once (algorithmic bytes); L2 flushed before every step."""
@@ -428,6 +500,9 @@ def main():
     ap.add_argument("--discretize", action="store_true",
                     help="time the discretisation front end (ssd_discretize) on the workload's "
                          "inputs instead of the forward; prints its own JSON line")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward (ssd_backward, scalar decay) on the workload instead "
+                         "of the forward; prints its own JSON line")
     ap.add_argument("--decode", action="store_true",
                     help="time the recurrent decode step (one token per chain) on the workload's "
                          "batch and heads instead of the forward; prints its own JSON line")
@@ -445,6 +520,8 @@ def main():
     device = torch.device("cuda", local)
     if args.decode:
         return run_decode(args, device)
+    if args.backward:
+        return run_backward(args, device)
     if args.discretize:
         return run_discretize(args, device)
     dist = None

@@ -301,6 +301,41 @@ ssd_status ssd_decode_step(const ssd_shape* shape, const void* x, const float* a
                            const void* Cm, const float* D, float* state, void* y,
                            ssd_stream stream);
 
+/* Backward of the forward (scalar decay): the gradients of
+ *     l = sum_{b,t,h} dy[b,t,h,:] . y[b,t,h,:] + <dfinal, final_state>
+ * with respect to x, a, Bm, Cm, D and initial_state, for the forward that
+ * ssd_forward_init computes from the same inputs.  The forward states are
+ * recomputed inside the call rather than kept by the forward (llms.blog
+ * "State Space Models and Mamba ...", "Hardware-Aware Parallel Associative
+ * Scan": intermediate states are recomputed in the backward pass), and the
+ * adjoint state runs backwards through the same chunks ("State Space
+ * Duality", "Two algorithms for one operator", applied to the transposed
+ * operator).
+ *   inputs   x, Bm, Cm, dy (dtype of the shape; dy [B][T][H][P]); a [B][T][H]
+ *            fp32; D [H] fp32 or NULL; initial_state [B][H][N][P] fp32 or NULL
+ *            (zero); dfinal [B][H][N][P] fp32 or NULL (no loss on the final state)
+ *   outputs  dx [B][T][H][P], dBm, dCm [B][T][G][N] (dtype; dB and dC summed
+ *            over the heads of each group), da [B][T][H] fp32, dD [H] fp32 or
+ *            NULL (not wanted), dinit [B][H][N][P] fp32 or NULL (not wanted);
+ *            every output is overwritten, none accumulated into
+ *   workspace  device memory of ssd_backward_workspace_size(shape) bytes,
+ *            256-byte aligned, owned by the caller (recomputed states, the
+ *            adjoint chunk states, fp32 per-head partials); reusable once the
+ *            call's work on `stream` has finished
+ * All device pointers, 16-byte aligned; asynchronous on `stream`.  A partial
+ * last chunk (T % chunk != 0) is handled as in the forward.  Arithmetic is
+ * fp32 on CUDA cores.  Returns SSD_ERR_INVALID_ARG for a bad shape or
+ * pointer, SSD_ERR_UNSUPPORTED for a_per_state, SSD_ERR_WORKSPACE for a
+ * missing, misaligned or small workspace, SSD_ERR_CUDA if a launch fails. */
+ssd_status ssd_backward(const ssd_shape* shape, const void* x, const float* a, const void* Bm,
+                        const void* Cm, const float* D, const float* initial_state, const void* dy,
+                        const float* dfinal, void* dx, float* da, void* dBm, void* dCm, float* dD,
+                        float* dinit, void* workspace, size_t ws_bytes, ssd_stream stream);
+
+/* Bytes of workspace ssd_backward needs for this shape; 0 if the shape is
+ * invalid or not served (a_per_state). */
+size_t ssd_backward_workspace_size(const ssd_shape* shape);
+
 #ifdef __cplusplus
 }
 #endif

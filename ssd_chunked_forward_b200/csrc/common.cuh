@@ -27,6 +27,13 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+// sum over the 32 lanes, returned in every lane
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
 __device__ __forceinline__ float warp_inclusive_scan(float v) {
     const int lane = threadIdx.x & 31;
 #pragma unroll

@@ -45,6 +45,36 @@ cudaError_t launch_decode_step(const Dims& d, const void* x, const float* a, con
                                const void* Cm, const float* D, float* state, void* y,
                                cudaStream_t st);
 
+// ---- backward (scalar decay, CUDA cores, fp32) ------------------------------
+// dstates[b,h,k] = sum_j exp(cum_j) C_j dy_j^T: each chunk's readout term of the
+// adjoint of the state entering it
+cudaError_t launch_chunk_dstate_simt(const Dims& d, const void* dy, const void* Cm,
+                                     const float* cum, float* dstates, cudaStream_t st);
+
+struct BackwardArgs {
+    const void* x; const float* a; const void* Bm; const void* Cm; const float* D;
+    const float* init;    // [B,H,N,P] or null (zero)
+    const void* dy;       // [B,T,H,P]
+    const float* dfinal;  // [B,H,N,P] or null (zero)
+    void* dx; float* da; void* dBm; void* dCm;
+    float* dD;            // [H] or null
+    float* dinit;         // [B,H,N,P] or null
+};
+struct BackwardScratch {
+    float* cum;      // [B,H,nc,Q]
+    float* states;   // [B,H,nc,N,P]  states entering each chunk
+    float* dstates;  // [B,H,nc,N,P]  adjoint at each chunk's last token
+    float* fin;      // [B,H,N,P]
+    float* cdot;     // [B,H,nc]
+    float* dDpart;   // [B,H,nc]
+    float* ytil;     // [B,T,H,P]  y - D x
+    float* dxt;      // [B,T,H,P]  dx - D dy
+    float* dBh;      // [B,T,H,N]  per head
+    float* dCh;      // [B,T,H,N]  per head
+};
+cudaError_t launch_backward(const Dims& d, const BackwardArgs& g, const BackwardScratch& w,
+                            cudaStream_t st);
+
 // ---- tensor-core kernels (tcgen05 + TMEM + TMA) ----------------------------
 bool chunk_state_tc_supported(const Dims& d);
 cudaError_t launch_chunk_state_tc(const Dims& d, const void* x, const void* Bm, const float* cum,

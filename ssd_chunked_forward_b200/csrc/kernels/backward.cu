@@ -1,0 +1,364 @@
+// backward.cu -- gradients of the chunked SSD forward (scalar decay), on CUDA
+// cores in fp32.
+//
+// The loss is l = sum_t dy_t . y_t + <dfinal, h_{T-1}>.  Its adjoint state
+// g_t = dl/dh_t runs backwards through the same chunk structure as the
+// forward runs h: inside a chunk as a quadratic (anti-causal) form, between
+// chunks as one summarised N x P state per chunk boundary -- the chunked
+// algorithm of "State Space Duality", "Two algorithms for one operator",
+// applied to the transposed operator.  The forward states are recomputed, not
+// stored by the forward (llms.blog "State Space Models and Mamba ...",
+// "Hardware-Aware Parallel Associative Scan": intermediate states are
+// recomputed in the backward pass).  With c the in-chunk cumulative decay,
+// Hin_k the state entering chunk k and G_k the adjoint at its last token:
+//
+//   Gin_k  = sum_t e^{c_t} C_t dy_t^T + e^{c_end} G_k,  G_{k-1} = Gin_k, G_last = dfinal
+//   y~_t   = sum_{s<=t} (C_t.B_s) e^{c_t-c_s} x_s  + e^{c_t} Hin_k^T C_t     (y - D x)
+//   dC_t   = sum_{s<=t} (dy_t.x_s) e^{c_t-c_s} B_s + e^{c_t} Hin_k dy_t
+//   dx~_t  = sum_{s>=t} (B_t.C_s) e^{c_s-c_t} dy_s + e^{c_end-c_t} G_k^T B_t  (dx - D dy)
+//   dB_t   = sum_{s>=t} (x_t.dy_s) e^{c_s-c_t} C_s + e^{c_end-c_t} G_k x_t
+//   da_t   = sum_{s>=t in the chunk} (dy_s.y~_s - x_s.dx~_s) + <G_k, Hin_{k+1}>
+//   dD     = sum_t dy_t.x_t,   d initial = Gin_0
+//
+// The last line follows from a_t entering every decay factor that spans t:
+// the output pairs (s' <= t <= s) within the chunk give the two inner
+// products, and the pairs reaching past the chunk end give the boundary term.
+// dB and dC are formed per head and summed over each group's heads.
+#include "../common.cuh"
+#include "../kernels.h"
+
+namespace ssd {
+namespace {
+
+// ------------------------------------------------ reverse state pass ----
+// One thread per (b, h, n, p): G_k into slot k of dstates (which held the
+// chunk's own readout term), Gin_0 into dinit.
+__global__ void __launch_bounds__(256) reverse_pass_kernel(const float* __restrict__ cum,
+                                                           float* __restrict__ dstates,
+                                                           const float* __restrict__ dfinal,
+                                                           float* __restrict__ dinit, int N, int P,
+                                                           int Q, int nc, long long total) {
+    const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= total) return;
+    const int NP = N * P;
+    const long long bh = e / NP;
+    const int r = (int)(e - bh * NP);
+    float* sp = dstates + bh * (long long)nc * NP + r;
+    const float* ce = cum + bh * (long long)nc * Q + (Q - 1);
+    float g = dfinal ? dfinal[bh * NP + r] : 0.f;
+    for (int k = nc - 1; k >= 0; --k) {
+        const float s = sp[(size_t)k * NP];
+        const float dec = expf(ce[(size_t)k * Q]);
+        sp[(size_t)k * NP] = g;
+        g = fmaf(dec, g, s);
+    }
+    if (dinit) dinit[bh * NP + r] = g;
+}
+
+// ------------------------------------------------ boundary inner product ----
+// out[bh, k] = <G_k, Hin_{k+1}> (Hin_nc = the final state).  Block per (k, bh).
+__global__ void __launch_bounds__(256) chunk_dot_kernel(const float* __restrict__ G,
+                                                        const float* __restrict__ Hin,
+                                                        const float* __restrict__ fin,
+                                                        float* __restrict__ out, int NP, int nc) {
+    const int k = blockIdx.x, bh = blockIdx.y;
+    const float* g = G + ((size_t)bh * nc + k) * NP;
+    const float* h = (k + 1 < nc) ? Hin + ((size_t)bh * nc + k + 1) * NP : fin + (size_t)bh * NP;
+    float s = 0.f;
+    for (int i = threadIdx.x; i < NP; i += blockDim.x) s = fmaf(g[i], h[i], s);
+    s = warp_sum(s);
+    __shared__ float red[8];
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float t = 0.f;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red[w];
+        out[(size_t)bh * nc + k] = t;
+    }
+}
+
+// ------------------------------------------------ chunk quadratic forms ----
+// A token operand of one chain: element (b, t, h, i) at
+// p[(b * T + t) * ld_t + (h / hdiv) * ld_h + i] -- x and dy are [B,T,H,P]
+// (ld_t = H P, ld_h = P, hdiv = 1), B and C are [B,T,G,N] (ld_t = G N,
+// ld_h = N, hdiv = H / G).
+struct Opd {
+    const void* p;
+    int ld_t, ld_h, hdiv;
+};
+
+template <typename T>
+__device__ __forceinline__ float opd_at(const Opd& o, int b, int Tlen, int t, int h, int i) {
+    return to_f32(static_cast<const T*>(o.p)[((size_t)b * Tlen + t) * o.ld_t + (size_t)(h / o.hdiv) * o.ld_h + i]);
+}
+
+// out[b, kQ+i, h, m] for one 32-row tile and 64 columns of one chunk:
+//   causal (ANTI = false):  sum_{j<=i} (U_i.V_j) e^{c_i-c_j} Z_j[m] + e^{c_i}       sum_kk U_i[kk] M[kk,m]
+//   anti   (ANTI = true):   sum_{j>=i} (U_i.V_j) e^{c_j-c_i} Z_j[m] + e^{c_end-c_i} sum_kk U_i[kk] M[kk,m]
+// U, V have K columns (the contracted dimension), Z and out have Mc columns;
+// M is the chunk's fp32 N x P state (Hin_k or G_k) read as K x Mc through the
+// strides (sk, sm).  Rows past T (the partial last chunk) are neither read
+// nor written.  Thread (ti = tid/8, tp = tid%8): row ti, columns tp + 8 m.
+template <typename T, bool ANTI>
+__global__ void __launch_bounds__(256) chunk_form_kernel(Opd U, Opd V, Opd Z,
+                                                         const float* __restrict__ cum,
+                                                         const float* __restrict__ Mst, int sk,
+                                                         int sm, float* __restrict__ out, int Tlen,
+                                                         int H, int K, int Mc, int Q, int nc,
+                                                         int NP) {
+    extern __shared__ float smem[];
+    const int KS = K + 1;
+    float* Us = smem;            // [32][KS]
+    float* Vs = Us + 32 * KS;    // [32][KS]
+    float* Zs = Vs + 32 * KS;    // [32][65]
+    float* Ps = Zs + 32 * 65;    // [32][33]
+    float* Ms = Ps + 32 * 33;    // [32][65]
+    float* cr = Ms + 32 * 65;    // [32]
+    float* cc = cr + 32;         // [32]
+    const int nrt = (Q + 31) / 32;
+    const int k = blockIdx.x / nrt, i0 = (blockIdx.x % nrt) * 32;
+    const int bh = blockIdx.y, b = bh / H, h = bh % H;
+    const int m0 = blockIdx.z * 64;
+    const int tid = threadIdx.x, ti = tid >> 3, tp = tid & 7;
+    const int tk = k * Q;
+    const int qv = min(Q, Tlen - tk);  // rows of this chunk before T
+    if (i0 >= qv) return;              // a tile wholly past T (the whole block leaves)
+    const float* cumk = cum + ((size_t)bh * nc + k) * (size_t)Q;
+
+    for (int idx = tid; idx < 32 * K; idx += 256) {
+        const int ii = idx / K, kk = idx % K, i = i0 + ii;
+        Us[ii * KS + kk] = (i < qv) ? opd_at<T>(U, b, Tlen, tk + i, h, kk) : 0.f;
+    }
+    if (tid < 32) cr[tid] = (i0 + tid < qv) ? cumk[i0 + tid] : 0.f;
+
+    float acc[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) acc[m] = 0.f;
+    const int i = i0 + ti;
+    const int j_first = ANTI ? i0 : 0;
+    const int j_end = ANTI ? qv : min(i0 + 32, qv);  // one past the last column token
+    for (int j0 = j_first; j0 < j_end; j0 += 32) {
+        __syncthreads();
+        for (int idx = tid; idx < 32 * K; idx += 256) {
+            const int jj = idx / K, kk = idx % K, j = j0 + jj;
+            Vs[jj * KS + kk] = (j < qv) ? opd_at<T>(V, b, Tlen, tk + j, h, kk) : 0.f;
+        }
+        if (tid < 32) cc[tid] = (j0 + tid < qv) ? cumk[j0 + tid] : 0.f;
+        for (int idx = tid; idx < 32 * 64; idx += 256) {
+            const int jj = idx / 64, m = idx % 64, j = j0 + jj;
+            Zs[jj * 65 + m] = (j < qv && m0 + m < Mc) ? opd_at<T>(Z, b, Tlen, tk + j, h, m0 + m) : 0.f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int jj = tp * 4 + c;
+            const int j = j0 + jj;
+            float s = 0.f;
+            const bool keep = ANTI ? (j >= i) : (j <= i);
+            if (keep && i < qv && j < qv) {
+                const float* ui = Us + ti * KS;
+                const float* vj = Vs + jj * KS;
+                for (int kk = 0; kk < K; ++kk) s = fmaf(ui[kk], vj[kk], s);
+                s *= ANTI ? expf(cc[jj] - cr[ti]) : expf(cr[ti] - cc[jj]);
+            }
+            Ps[ti * 33 + jj] = s;
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int jj = 0; jj < 32; ++jj) {
+            const float pv = Ps[ti * 33 + jj];
+#pragma unroll
+            for (int m = 0; m < 8; ++m) acc[m] = fmaf(pv, Zs[jj * 65 + tp + 8 * m], acc[m]);
+        }
+    }
+    // boundary-state term
+    float acc2[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) acc2[m] = 0.f;
+    const float* Mk = Mst + ((size_t)bh * nc + k) * (size_t)NP;
+    for (int k0 = 0; k0 < K; k0 += 32) {
+        __syncthreads();
+        for (int idx = tid; idx < 32 * 64; idx += 256) {
+            const int kk = idx / 64, m = idx % 64;
+            Ms[kk * 65 + m] = (k0 + kk < K && m0 + m < Mc)
+                                  ? Mk[(size_t)(k0 + kk) * sk + (size_t)(m0 + m) * sm]
+                                  : 0.f;
+        }
+        __syncthreads();
+        const int kmax = min(32, K - k0);
+        for (int kk = 0; kk < kmax; ++kk) {
+            const float uv = Us[ti * KS + k0 + kk];
+#pragma unroll
+            for (int m = 0; m < 8; ++m) acc2[m] = fmaf(uv, Ms[kk * 65 + tp + 8 * m], acc2[m]);
+        }
+    }
+    if (i >= qv) return;
+    const float sc = ANTI ? expf(cumk[Q - 1] - cr[ti]) : expf(cr[ti]);
+    float* o = out + (((size_t)b * Tlen + tk + i) * H + h) * Mc;
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+        const int mm = m0 + tp + 8 * m;
+        if (mm < Mc) o[mm] = fmaf(sc, acc2[m], acc[m]);
+    }
+}
+
+// ------------------------------------------------ per-token outputs ----
+// Block per (chunk k, bh); warp per token: dx = dx~ + D dy (input dtype),
+// r_t = dy.y~ - x.dx~, then da = the in-chunk suffix sum of r plus the
+// boundary term; the chunk's share of dD (sum dy.x) goes to dDpart.
+template <typename T>
+__global__ void __launch_bounds__(256) token_grad_kernel(
+    const T* __restrict__ x, const T* __restrict__ dy, const float* __restrict__ ytil,
+    const float* __restrict__ dxt, const float* __restrict__ D, const float* __restrict__ cdot,
+    T* __restrict__ dx, float* __restrict__ da, float* __restrict__ dDpart, int Tlen, int H, int P,
+    int Q, int nc) {
+    extern __shared__ float rs[];  // [Q]
+    __shared__ float red[8];
+    const int k = blockIdx.x, bh = blockIdx.y, b = bh / H, h = bh % H;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tk = k * Q;
+    const int qv = min(Q, Tlen - tk);
+    const float dv = D ? D[h] : 0.f;
+    float dsum = 0.f;
+    for (int j = warp; j < qv; j += 8) {
+        const size_t row = (((size_t)b * Tlen + tk + j) * H + h) * P;
+        float r = 0.f, xd = 0.f;
+        for (int p = lane; p < P; p += 32) {
+            const float xv = to_f32(x[row + p]), gv = to_f32(dy[row + p]);
+            const float dxs = dxt[row + p];
+            r = fmaf(gv, ytil[row + p], r);
+            r = fmaf(-xv, dxs, r);
+            xd = fmaf(gv, xv, xd);
+            dx[row + p] = from_f32<T>(fmaf(dv, gv, dxs));
+        }
+        r = warp_sum(r);
+        xd = warp_sum(xd);
+        if (lane == 0) rs[j] = r;
+        dsum += xd;  // the same value in every lane
+    }
+    if (lane == 0) red[warp] = dsum;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float run = cdot[(size_t)bh * nc + k];
+        for (int j = qv - 1; j >= 0; --j) {
+            run += rs[j];
+            da[((size_t)b * Tlen + tk + j) * H + h] = run;
+        }
+        float t = 0.f;
+        for (int w = 0; w < 8; ++w) t += red[w];
+        dDpart[(size_t)bh * nc + k] = t;
+    }
+}
+
+__global__ void dD_reduce_kernel(const float* __restrict__ dDpart, float* __restrict__ dD, int B,
+                                 int H, int nc) {
+    const int h = blockIdx.x * blockDim.x + threadIdx.x;
+    if (h >= H) return;
+    float s = 0.f;
+    for (int b = 0; b < B; ++b)
+        for (int k = 0; k < nc; ++k) s += dDpart[((size_t)b * H + h) * nc + k];
+    dD[h] = s;
+}
+
+// out[b,t,g,n] = sum of in[b,t,h,n] over the heads h of group g (fp32 in,
+// input dtype out), for dB and dC at once.
+template <typename T>
+__global__ void __launch_bounds__(256) group_sum_kernel(const float* __restrict__ dBh,
+                                                        const float* __restrict__ dCh,
+                                                        T* __restrict__ dB, T* __restrict__ dC,
+                                                        long long rows, int H, int G, int N) {
+    const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long total = rows * G * N;
+    if (e >= total) return;
+    const int n = (int)(e % N);
+    const long long rg = e / N;  // (b*T + t) * G + g
+    const int g = (int)(rg % G);
+    const long long bt = rg / G;
+    const int hg = H / G;
+    const float* pb = dBh + (bt * H + (long long)g * hg) * N + n;
+    const float* pc = dCh + (bt * H + (long long)g * hg) * N + n;
+    float sb = 0.f, sc = 0.f;
+    for (int i = 0; i < hg; ++i) {
+        sb += pb[(size_t)i * N];
+        sc += pc[(size_t)i * N];
+    }
+    dB[e] = from_f32<T>(sb);
+    dC[e] = from_f32<T>(sc);
+}
+
+template <typename T, bool ANTI>
+cudaError_t launch_form(const Dims& d, Opd U, Opd V, Opd Z, const float* cum, const float* Mst,
+                        int sk, int sm, float* out, int K, int Mc, cudaStream_t st) {
+    const size_t smem = (size_t)(2 * 32 * (K + 1) + 32 * 65 + 32 * 33 + 32 * 65 + 64) * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(chunk_form_kernel<T, ANTI>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(d.nc * ((d.Q + 31) / 32), d.B * d.H, (Mc + 63) / 64);
+    chunk_form_kernel<T, ANTI><<<grid, 256, smem, st>>>(U, V, Z, cum, Mst, sk, sm, out, d.T, d.H, K,
+                                                        Mc, d.Q, d.nc, d.N * d.P);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t run_backward_t(const Dims& d, const BackwardArgs& g, const BackwardScratch& w,
+                           cudaStream_t st) {
+    const Opd ox{g.x, d.H * d.P, d.P, 1};
+    const Opd ody{g.dy, d.H * d.P, d.P, 1};
+    const Opd oB{g.Bm, d.G * d.N, d.N, d.H / d.G};
+    const Opd oC{g.Cm, d.G * d.N, d.N, d.H / d.G};
+    cudaError_t e;
+    // y~ (causal; U = C, V = B, Z = x; Hin as N x P)
+    if ((e = launch_form<T, false>(d, oC, oB, ox, w.cum, w.states, d.P, 1, w.ytil, d.N, d.P, st))) return e;
+    // dC per head (causal; U = dy, V = x, Z = B; Hin read as P x N)
+    if ((e = launch_form<T, false>(d, ody, ox, oB, w.cum, w.states, 1, d.P, w.dCh, d.P, d.N, st))) return e;
+    // dx~ (anti-causal; U = B, V = C, Z = dy; G as N x P)
+    if ((e = launch_form<T, true>(d, oB, oC, ody, w.cum, w.dstates, d.P, 1, w.dxt, d.N, d.P, st))) return e;
+    // dB per head (anti-causal; U = x, V = dy, Z = C; G read as P x N)
+    if ((e = launch_form<T, true>(d, ox, ody, oC, w.cum, w.dstates, 1, d.P, w.dBh, d.P, d.N, st))) return e;
+    {
+        dim3 grid(d.nc, d.B * d.H);
+        const size_t smem = (size_t)d.Q * sizeof(float);
+        token_grad_kernel<T><<<grid, 256, smem, st>>>(
+            (const T*)g.x, (const T*)g.dy, w.ytil, w.dxt, g.D, w.cdot, (T*)g.dx, g.da, w.dDpart,
+            d.T, d.H, d.P, d.Q, d.nc);
+        if ((e = cudaGetLastError())) return e;
+    }
+    if (g.dD) {
+        dD_reduce_kernel<<<(d.H + 127) / 128, 128, 0, st>>>(w.dDpart, g.dD, d.B, d.H, d.nc);
+        if ((e = cudaGetLastError())) return e;
+    }
+    {
+        const long long rows = (long long)d.B * d.T;
+        const long long total = rows * d.G * d.N;
+        group_sum_kernel<T><<<(unsigned)((total + 255) / 256), 256, 0, st>>>(
+            w.dBh, w.dCh, (T*)g.dBm, (T*)g.dCm, rows, d.H, d.G, d.N);
+        if ((e = cudaGetLastError())) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t launch_backward(const Dims& d, const BackwardArgs& g, const BackwardScratch& w,
+                            cudaStream_t st) {
+    if (d.diag) return cudaErrorNotSupported;
+    cudaError_t e;
+    // forward states, recomputed: in-chunk cumsum, chunk states, states entering each chunk
+    if ((e = launch_chunk_cumsum(d, g.a, w.cum, st))) return e;
+    if ((e = launch_chunk_state_simt(d, g.x, g.Bm, w.cum, w.states, st))) return e;
+    if ((e = launch_state_pass(d, w.cum, w.states, w.fin, g.init, st))) return e;
+    // adjoint states: each chunk's readout term, then the reverse pass
+    if ((e = launch_chunk_dstate_simt(d, g.dy, g.Cm, w.cum, w.dstates, st))) return e;
+    {
+        const long long total = (long long)d.B * d.H * d.N * d.P;
+        reverse_pass_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(
+            w.cum, w.dstates, g.dfinal, g.dinit, d.N, d.P, d.Q, d.nc, total);
+        if ((e = cudaGetLastError())) return e;
+    }
+    chunk_dot_kernel<<<dim3(d.nc, d.B * d.H), 256, 0, st>>>(w.dstates, w.states, w.fin, w.cdot,
+                                                            d.N * d.P, d.nc);
+    if ((e = cudaGetLastError())) return e;
+    return d.bf16 ? run_backward_t<__nv_bfloat16>(d, g, w, st) : run_backward_t<float>(d, g, w, st);
+}
+
+}  // namespace ssd

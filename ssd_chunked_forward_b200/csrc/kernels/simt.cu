@@ -101,7 +101,9 @@ cudaError_t launch_chunk_cumsum(const Dims& d, const float* a, float* cum, cudaS
 // ============================================================ step 2 ======
 // states[b,h,k,n,p] = sum_j B[j,n] w[j,n] x[j,p], w = exp(cum_end - cum_j).
 // Block = (chunk, b*H+h, 64x64 output tile); 16x16 threads, 4x4 outputs each.
-template <typename T, bool DIAG>
+// FROM_START (scalar decay, backward): w = exp(cum_j), the decay from the
+// state entering the chunk to token j, with (C, dy) in place of (B, x).
+template <typename T, bool DIAG, bool FROM_START = false>
 __global__ void __launch_bounds__(256) chunk_state_simt_kernel(
     const T* __restrict__ x, const T* __restrict__ Bm, const float* __restrict__ cum,
     float* __restrict__ states, int Tlen, int H, int P, int G, int N, int Q, int nc) {
@@ -129,6 +131,8 @@ __global__ void __launch_bounds__(256) chunk_state_simt_kernel(
                     float w;
                     if (DIAG)
                         w = expf(cumk[(size_t)(Q - 1) * N + n0 + c] - cumk[(size_t)j * N + n0 + c]);
+                    else if (FROM_START)
+                        w = expf(cumk[j]);
                     else
                         w = expf(cumk[Q - 1] - cumk[j]);
                     bv = to_f32(Bm[(((size_t)b * Tlen + t) * G + g) * N + n0 + c]) * w;
@@ -180,6 +184,20 @@ cudaError_t launch_chunk_state_simt(const Dims& d, const void* x, const void* Bm
         if (d.diag) SSD_CS_LAUNCH(float, true); else SSD_CS_LAUNCH(float, false);
     }
 #undef SSD_CS_LAUNCH
+    return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_dstate_simt(const Dims& d, const void* dy, const void* Cm,
+                                     const float* cum, float* dstates, cudaStream_t st) {
+    if (d.diag) return cudaErrorNotSupported;
+    dim3 grid(d.nc, d.B * d.H, ((d.N + 63) / 64) * ((d.P + 63) / 64));
+    if (d.bf16)
+        chunk_state_simt_kernel<__nv_bfloat16, false, true><<<grid, 256, 0, st>>>(
+            (const __nv_bfloat16*)dy, (const __nv_bfloat16*)Cm, cum, dstates, d.T, d.H, d.P, d.G,
+            d.N, d.Q, d.nc);
+    else
+        chunk_state_simt_kernel<float, false, true><<<grid, 256, 0, st>>>(
+            (const float*)dy, (const float*)Cm, cum, dstates, d.T, d.H, d.P, d.G, d.N, d.Q, d.nc);
     return cudaGetLastError();
 }
 

@@ -102,6 +102,37 @@ Workspace carve(void* ws, const Dims& d) {
 
 ssd_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA; }
 
+// The backward's scratch, in order, each piece 256-byte aligned; returns the
+// total size.  With a base, fills the pointers.
+size_t backward_layout(const Dims& d, void* base, ssd::BackwardScratch* w) {
+    const size_t f = sizeof(float);
+    const size_t chains = (size_t)d.B * d.H;
+    const size_t sizes[10] = {
+        chains * d.nc * d.Q * f,                  // cum
+        chains * d.nc * d.N * d.P * f,            // states
+        chains * d.nc * d.N * d.P * f,            // dstates
+        chains * d.N * d.P * f,                   // fin
+        chains * d.nc * f,                        // cdot
+        chains * d.nc * f,                        // dDpart
+        (size_t)d.B * d.T * d.H * d.P * f,        // ytil
+        (size_t)d.B * d.T * d.H * d.P * f,        // dxt
+        (size_t)d.B * d.T * d.H * d.N * f,        // dBh
+        (size_t)d.B * d.T * d.H * d.N * f,        // dCh
+    };
+    float** slots[10] = {};
+    if (w) {
+        float** s[10] = {&w->cum, &w->states, &w->dstates, &w->fin, &w->cdot, &w->dDpart,
+                         &w->ytil, &w->dxt, &w->dBh, &w->dCh};
+        for (int i = 0; i < 10; ++i) slots[i] = s[i];
+    }
+    size_t off = 0;
+    for (int i = 0; i < 10; ++i) {
+        if (base && slots[i]) *slots[i] = (float*)((char*)base + off);
+        off += round_up(sizes[i], kAlign);
+    }
+    return off;
+}
+
 // one event per device: the end of the last fused launch
 constexpr int kMaxDevices = 64;
 std::mutex g_fused_mu;
@@ -438,6 +469,32 @@ ssd_status ssd_decode_step(const ssd_shape* shape, const void* x, const float* a
         return SSD_ERR_INVALID_ARG;
     return cuda_status(ssd::launch_decode_step(dims_of(shape), x, a, Bm, Cm, D, state, y,
                                                (cudaStream_t)stream));
+}
+
+ssd_status ssd_backward(const ssd_shape* shape, const void* x, const float* a, const void* Bm,
+                        const void* Cm, const float* D, const float* initial_state, const void* dy,
+                        const float* dfinal, void* dx, float* da, void* dBm, void* dCm, float* dD,
+                        float* dinit, void* workspace, size_t ws_bytes, ssd_stream stream) {
+    ssd_status st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    if (shape->a_per_state) return SSD_ERR_UNSUPPORTED;
+    if (!x || !a || !Bm || !Cm || !dy || !dx || !da || !dBm || !dCm) return SSD_ERR_INVALID_ARG;
+    const void* ptrs[] = {x, a, Bm, Cm, D, initial_state, dy, dfinal, dx, da, dBm, dCm, dD, dinit};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return SSD_ERR_INVALID_ARG;
+    const Dims d = dims_of(shape);
+    const size_t need = backward_layout(d, nullptr, nullptr);
+    if (!workspace || ((uintptr_t)workspace % kAlign) != 0 || ws_bytes < need)
+        return SSD_ERR_WORKSPACE;
+    ssd::BackwardScratch w;
+    backward_layout(d, workspace, &w);
+    ssd::BackwardArgs g{x, a, Bm, Cm, D, initial_state, dy, dfinal, dx, da, dBm, dCm, dD, dinit};
+    return cuda_status(ssd::launch_backward(d, g, w, (cudaStream_t)stream));
+}
+
+size_t ssd_backward_workspace_size(const ssd_shape* shape) {
+    if (check_shape(shape) != SSD_OK || shape->a_per_state) return 0;
+    return backward_layout(dims_of(shape), nullptr, nullptr);
 }
 
 }  // extern "C"

@@ -27,6 +27,7 @@ EXPORTS = [
     "ssd_state_pass", "ssd_chunk_scan", "ssd_diag_scan", "ssd_forward_host_bytes",
     "ssd_forward_host", "ssd_forward_noalloc", "ssd_auto_path", "ssd_forward_init",
     "ssd_decode_step", "ssd_discretize", "ssd_decay_total", "ssd_state_combine",
+    "ssd_backward", "ssd_backward_workspace_size",
 ]
 
 
@@ -82,9 +83,12 @@ def load(path: str = LIB_PATH):
     lib.ssd_discretize.argtypes = [sp, fp, fp, fp, vp, fp, vp, vp]
     lib.ssd_decay_total.argtypes = [sp, fp, fp, vp]
     lib.ssd_state_combine.argtypes = [sp, ctypes.c_int, fp, fp, fp, fp, vp]
+    lib.ssd_backward.argtypes = [sp, vp, fp, vp, vp, fp, fp, vp, fp, vp, fp, vp, vp, fp, fp, vp, sz, vp]
+    lib.ssd_backward_workspace_size.argtypes = [sp]
+    lib.ssd_backward_workspace_size.restype = sz
     for name in ("ssd_forward_noalloc", "ssd_forward", "ssd_forward_path", "ssd_forward_init",
                  "ssd_device_status", "ssd_chunk_cumsum", "ssd_decode_step", "ssd_discretize",
-                 "ssd_decay_total", "ssd_state_combine",
+                 "ssd_decay_total", "ssd_state_combine", "ssd_backward",
                  "ssd_chunk_state", "ssd_state_pass", "ssd_chunk_scan", "ssd_diag_scan",
                  "ssd_forward_host"):
         getattr(lib, name).restype = ctypes.c_int
@@ -347,3 +351,44 @@ def state_combine(finals, totals, h0=None, *, out=None, stream=None):
     _check(load().ssd_state_combine(ctypes.byref(shape), int(S), _ptr(finals), _ptr(totals), _ptr(h0),
                                     _ptr(out), _stream(stream)), "ssd_state_combine")
     return out
+
+
+def backward_workspace_size(shape: Shape) -> int:
+    return int(load().ssd_backward_workspace_size(ctypes.byref(shape)))
+
+
+def backward(x, a, Bm, Cm, D, dy, chunk=256, *, dfinal=None, initial_state=None, want_dD=True,
+             want_dinit=True, workspace=None, stream=None):
+    """Gradients of sum(dy * y) + <dfinal, final_state> for the forward of the
+    same inputs (scalar decay): returns dict dx, da, dBm, dCm, dD (or None),
+    dinit (or None).  Shapes and dtypes as for forward(); dy like x; dfinal
+    and initial_state [B,H,N,P] float32 or None.  Asynchronous on the current
+    torch stream (or ``stream``)."""
+    _check_inputs(x, a, Bm, Cm, D)
+    if dy.shape != x.shape or dy.dtype != x.dtype or not dy.is_contiguous():
+        raise ValueError("dy must be a contiguous tensor of x's shape and dtype")
+    B, T, H, P = x.shape
+    N = Bm.shape[3]
+    for name, t in (("dfinal", dfinal), ("initial_state", initial_state)):
+        if t is not None and (t.dtype != torch.float32 or not t.is_contiguous()
+                              or tuple(t.shape) != (B, H, N, P)):
+            raise ValueError(f"{name} must be a contiguous float32 [B,H,N,P] tensor")
+    shape = shape_of(x, a, Bm, chunk)
+    need = backward_workspace_size(shape)
+    if need == 0:
+        raise SSDError(SSD_ERR_UNSUPPORTED, "ssd_backward_workspace_size")
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    out = {
+        "dx": torch.empty_like(x), "da": torch.empty_like(a),
+        "dBm": torch.empty_like(Bm), "dCm": torch.empty_like(Cm),
+        "dD": torch.empty(H, dtype=torch.float32, device=x.device) if want_dD else None,
+        "dinit": torch.empty((B, H, N, P), dtype=torch.float32, device=x.device) if want_dinit else None,
+    }
+    _check(load().ssd_backward(ctypes.byref(shape), _ptr(x), _ptr(a), _ptr(Bm), _ptr(Cm), _ptr(D),
+                               _ptr(initial_state), _ptr(dy), _ptr(dfinal), _ptr(out["dx"]),
+                               _ptr(out["da"]), _ptr(out["dBm"]), _ptr(out["dCm"]), _ptr(out["dD"]),
+                               _ptr(out["dinit"]), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "ssd_backward")
+    return out
+

@@ -1,0 +1,104 @@
+"""GPU parity of the backward (ssd_backward, through the C ABI) against the
+oracle's adjoint of the recurrence, on the same seeded inputs.
+
+Every gradient (dx, da, dBm, dCm, dD, d initial) is compared with the parity
+metric ||g - g_ref||_inf / ||g_ref||_inf: 1e-4 for fp32 inputs, 2e-2 for bf16
+inputs (fp32 arithmetic; dx, dB, dC rounded to bf16 on output).  Cases span
+several chunks and row tiles, a partial last chunk, grouped B/C, a loss on
+the final state and a given initial state.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import ssd_oracle as O
+from ssd_chunked_forward_b200 import ssd
+from ssd_chunked_forward_b200.workloads import generate, small_case
+from tests.gpu_helpers import rel_err, to_dev, tol_for
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    ssd.load()
+
+
+CASES = [
+    small_case(B=2, T=96, H=3, P=24, N=20, G=1, chunk=32, dtype="f32", seed=81),
+    small_case(B=1, T=150, H=4, P=70, N=33, G=2, chunk=64, dtype="f32", seed=82),
+    small_case(B=1, T=512, H=4, P=64, N=128, G=1, chunk=256, dtype="bf16", seed=83),
+    small_case(B=2, T=300, H=4, P=64, N=128, G=2, chunk=128, dtype="bf16", seed=84),
+    small_case(B=1, T=7, H=2, P=5, N=3, G=1, chunk=7, dtype="f32", seed=85),
+    small_case(B=1, T=5, H=1, P=3, N=2, G=1, chunk=1, dtype="f32", seed=86),
+]
+
+
+def _ids(cases):
+    return [c.name + "_" + c.dtype for c in cases]
+
+
+def _extras(w, with_init, with_dfinal):
+    g = torch.Generator().manual_seed(w.seed + 101)
+    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    dy = torch.randn((w.B, w.T, w.H, w.P), generator=g).to(dt)
+    init = torch.randn((w.B, w.H, w.N, w.P), generator=g) if with_init else None
+    dfin = torch.randn((w.B, w.H, w.N, w.P), generator=g) if with_dfinal else None
+    return dy, init, dfin
+
+
+def _run(w, with_init, with_dfinal):
+    inp = generate(w)
+    dy, init, dfin = _extras(w, with_init, with_dfinal)
+    dev = to_dev(inp)
+    got = ssd.backward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], dev["D"], dy.cuda(), w.chunk,
+                       dfinal=None if dfin is None else dfin.cuda(),
+                       initial_state=None if init is None else init.cuda())
+    torch.cuda.synchronize()
+    f = lambda t: None if t is None else t.to(torch.float64).numpy()
+    prob = O.Problem(*(f(inp[k]) for k in ("x", "a", "Bm", "Cm", "D")))
+    ref = O.backward(prob, f(dy), dfinal=f(dfin), initial=f(init))
+    return got, ref
+
+
+@pytest.mark.parametrize("w", CASES, ids=_ids(CASES))
+@pytest.mark.parametrize("with_init,with_dfinal", [(False, False), (True, True)],
+                         ids=["plain", "init_dfinal"])
+def test_backward_matches_oracle(w, with_init, with_dfinal):
+    got, ref = _run(w, with_init, with_dfinal)
+    tol = tol_for(w)
+    errs = {}
+    for k in ("dx", "da", "dBm", "dCm", "dD", "dinit"):
+        g = got[k].float().cpu().numpy().astype(np.float64)
+        errs[k] = rel_err(g, ref[k])
+    assert all(e <= tol for e in errs.values()), errs
+
+
+def test_backward_rejects_per_state_and_bad_workspace():
+    """The per-state variant is not served (SSD_ERR_UNSUPPORTED) and a short
+    workspace is refused before any launch."""
+    w = small_case(B=1, T=64, H=2, P=16, N=16, G=1, chunk=32, dtype="f32", a_per_state=True, seed=87)
+    dev = to_dev(generate(w))
+    shape = ssd.shape_of(dev["x"], dev["a"], dev["Bm"], w.chunk)
+    assert ssd.backward_workspace_size(shape) == 0
+    with pytest.raises(ssd.SSDError) as e:
+        ssd.backward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], dev["D"], dev["x"].clone(), w.chunk)
+    assert e.value.code == ssd.SSD_ERR_UNSUPPORTED
+    w2 = small_case(B=1, T=64, H=2, P=16, N=16, G=1, chunk=32, dtype="f32", seed=88)
+    dev = to_dev(generate(w2))
+    shape = ssd.shape_of(dev["x"], dev["a"], dev["Bm"], w2.chunk)
+    need = ssd.backward_workspace_size(shape)
+    ws = torch.empty(need - 256, dtype=torch.uint8, device="cuda")
+    outs = [torch.empty_like(dev[k]) for k in ("x", "a", "Bm", "Cm")]
+    code = ssd.load().ssd_backward(
+        ctypes.byref(shape), dev["x"].data_ptr(), dev["a"].data_ptr(), dev["Bm"].data_ptr(),
+        dev["Cm"].data_ptr(), None, None, dev["x"].data_ptr(), None, outs[0].data_ptr(),
+        outs[1].data_ptr(), outs[2].data_ptr(), outs[3].data_ptr(), None, None, ws.data_ptr(),
+        ws.numel(), None)
+    assert code == ssd.SSD_ERR_WORKSPACE
