@@ -92,13 +92,19 @@ __device__ __forceinline__ float opd_at(const Opd& o, int b, int Tlen, int t, in
     return to_f32(static_cast<const T*>(o.p)[((size_t)b * Tlen + t) * o.ld_t + (size_t)(h / o.hdiv) * o.ld_h + i]);
 }
 
-// out[b, kQ+i, h, m] for one 32-row tile and 64 columns of one chunk:
+// out[b, kQ+i, h, m] for one 64-row tile and 64 columns of one chunk:
 //   causal (ANTI = false):  sum_{j<=i} (U_i.V_j) e^{c_i-c_j} Z_j[m] + e^{c_i}       sum_kk U_i[kk] M[kk,m]
 //   anti   (ANTI = true):   sum_{j>=i} (U_i.V_j) e^{c_j-c_i} Z_j[m] + e^{c_end-c_i} sum_kk U_i[kk] M[kk,m]
 // U, V have K columns (the contracted dimension), Z and out have Mc columns;
 // M is the chunk's fp32 N x P state (Hin_k or G_k) read as K x Mc through the
 // strides (sk, sm).  Rows past T (the partial last chunk) are neither read
-// nor written.  Thread (ti = tid/8, tp = tid%8): row ti, columns tp + 8 m.
+// nor written.  Thread (r = tid/16, c = tid%16) owns a 4 x 4 register block:
+// rows 4r..4r+3 and score / output columns 4c..4c+3.  The operands sit in
+// shared memory k-major (U^T, V^T, and the masked scores transposed), so each
+// step of every contraction is two 16-byte loads for 16 FMAs.
+constexpr int kFT = 64;  // tile rows / columns
+constexpr int kFS = 68;  // row stride of the shared tiles (16-byte aligned rows)
+
 template <typename T, bool ANTI>
 __global__ void __launch_bounds__(256) chunk_form_kernel(Opd U, Opd V, Opd Z,
                                                          const float* __restrict__ cum,
@@ -106,99 +112,128 @@ __global__ void __launch_bounds__(256) chunk_form_kernel(Opd U, Opd V, Opd Z,
                                                          int sm, float* __restrict__ out, int Tlen,
                                                          int H, int K, int Mc, int Q, int nc,
                                                          int NP) {
-    extern __shared__ float smem[];
-    const int KS = K + 1;
-    float* Us = smem;            // [32][KS]
-    float* Vs = Us + 32 * KS;    // [32][KS]
-    float* Zs = Vs + 32 * KS;    // [32][65]
-    float* Ps = Zs + 32 * 65;    // [32][33]
-    float* Ms = Ps + 32 * 33;    // [32][65]
-    float* cr = Ms + 32 * 65;    // [32]
-    float* cc = cr + 32;         // [32]
-    const int nrt = (Q + 31) / 32;
-    const int k = blockIdx.x / nrt, i0 = (blockIdx.x % nrt) * 32;
+    extern __shared__ __align__(16) float smem[];
+    float* UT = smem;              // [K][kFS]   U^T of the tile's rows
+    float* VT = UT + K * kFS;      // [K][kFS]   V^T of a column tile
+    float* PT = VT + K * kFS;      // [kFT][kFS] masked scores, transposed (column-major)
+    float* ZM = PT + kFT * kFS;    // [kFT][kFS] Z of a column tile; later M's rows
+    float* cr = ZM + kFT * kFS;    // [kFT]
+    float* cc = cr + kFT;          // [kFT]
+    const int nrt = (Q + kFT - 1) / kFT;
+    const int k = blockIdx.x / nrt, i0 = (blockIdx.x % nrt) * kFT;
     const int bh = blockIdx.y, b = bh / H, h = bh % H;
-    const int m0 = blockIdx.z * 64;
-    const int tid = threadIdx.x, ti = tid >> 3, tp = tid & 7;
+    const int m0 = blockIdx.z * kFT;
+    const int tid = threadIdx.x, r = tid >> 4, c = tid & 15;
     const int tk = k * Q;
     const int qv = min(Q, Tlen - tk);  // rows of this chunk before T
     if (i0 >= qv) return;              // a tile wholly past T (the whole block leaves)
     const float* cumk = cum + ((size_t)bh * nc + k) * (size_t)Q;
 
-    for (int idx = tid; idx < 32 * K; idx += 256) {
+    for (int idx = tid; idx < kFT * K; idx += 256) {
         const int ii = idx / K, kk = idx % K, i = i0 + ii;
-        Us[ii * KS + kk] = (i < qv) ? opd_at<T>(U, b, Tlen, tk + i, h, kk) : 0.f;
+        UT[kk * kFS + ii] = (i < qv) ? opd_at<T>(U, b, Tlen, tk + i, h, kk) : 0.f;
     }
-    if (tid < 32) cr[tid] = (i0 + tid < qv) ? cumk[i0 + tid] : 0.f;
+    if (tid < kFT) cr[tid] = (i0 + tid < qv) ? cumk[i0 + tid] : 0.f;
 
-    float acc[8];
+    float acc[4][4];
 #pragma unroll
-    for (int m = 0; m < 8; ++m) acc[m] = 0.f;
-    const int i = i0 + ti;
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[a][q] = 0.f;
     const int j_first = ANTI ? i0 : 0;
-    const int j_end = ANTI ? qv : min(i0 + 32, qv);  // one past the last column token
-    for (int j0 = j_first; j0 < j_end; j0 += 32) {
+    const int j_end = ANTI ? qv : min(i0 + kFT, qv);  // one past the last column token
+    for (int j0 = j_first; j0 < j_end; j0 += kFT) {
         __syncthreads();
-        for (int idx = tid; idx < 32 * K; idx += 256) {
+        for (int idx = tid; idx < kFT * K; idx += 256) {
             const int jj = idx / K, kk = idx % K, j = j0 + jj;
-            Vs[jj * KS + kk] = (j < qv) ? opd_at<T>(V, b, Tlen, tk + j, h, kk) : 0.f;
+            VT[kk * kFS + jj] = (j < qv) ? opd_at<T>(V, b, Tlen, tk + j, h, kk) : 0.f;
         }
-        if (tid < 32) cc[tid] = (j0 + tid < qv) ? cumk[j0 + tid] : 0.f;
-        for (int idx = tid; idx < 32 * 64; idx += 256) {
-            const int jj = idx / 64, m = idx % 64, j = j0 + jj;
-            Zs[jj * 65 + m] = (j < qv && m0 + m < Mc) ? opd_at<T>(Z, b, Tlen, tk + j, h, m0 + m) : 0.f;
+        if (tid < kFT) cc[tid] = (j0 + tid < qv) ? cumk[j0 + tid] : 0.f;
+        for (int idx = tid; idx < kFT * kFT; idx += 256) {
+            const int jj = idx / kFT, m = idx % kFT, j = j0 + jj;
+            ZM[jj * kFS + m] = (j < qv && m0 + m < Mc) ? opd_at<T>(Z, b, Tlen, tk + j, h, m0 + m) : 0.f;
         }
         __syncthreads();
+        // scores s[a][q] = U_{4r+a} . V_{4c+q}
+        float s[4][4];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const int jj = tp * 4 + c;
-            const int j = j0 + jj;
-            float s = 0.f;
-            const bool keep = ANTI ? (j >= i) : (j <= i);
-            if (keep && i < qv && j < qv) {
-                const float* ui = Us + ti * KS;
-                const float* vj = Vs + jj * KS;
-                for (int kk = 0; kk < K; ++kk) s = fmaf(ui[kk], vj[kk], s);
-                s *= ANTI ? expf(cc[jj] - cr[ti]) : expf(cr[ti] - cc[jj]);
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) s[a][q] = 0.f;
+#pragma unroll 4
+        for (int kk = 0; kk < K; ++kk) {
+            const float4 u = *reinterpret_cast<const float4*>(UT + kk * kFS + 4 * r);
+            const float4 v = *reinterpret_cast<const float4*>(VT + kk * kFS + 4 * c);
+            const float uu[4] = {u.x, u.y, u.z, u.w}, vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) s[a][q] = fmaf(uu[a], vv[q], s[a][q]);
+        }
+        // causal / anti-causal mask and decay; store transposed
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int jj = 4 * c + q, j = j0 + jj;
+            float pv[4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                const int ii = 4 * r + a, i = i0 + ii;
+                const bool keep = (ANTI ? (j >= i) : (j <= i)) && i < qv && j < qv;
+                pv[a] = keep ? s[a][q] * expf(ANTI ? cc[jj] - cr[ii] : cr[ii] - cc[jj]) : 0.f;
             }
-            Ps[ti * 33 + jj] = s;
+            *reinterpret_cast<float4*>(PT + jj * kFS + 4 * r) = make_float4(pv[0], pv[1], pv[2], pv[3]);
         }
         __syncthreads();
 #pragma unroll 4
-        for (int jj = 0; jj < 32; ++jj) {
-            const float pv = Ps[ti * 33 + jj];
+        for (int jj = 0; jj < kFT; ++jj) {
+            const float4 p = *reinterpret_cast<const float4*>(PT + jj * kFS + 4 * r);
+            const float4 z = *reinterpret_cast<const float4*>(ZM + jj * kFS + 4 * c);
+            const float pp[4] = {p.x, p.y, p.z, p.w}, zz[4] = {z.x, z.y, z.z, z.w};
 #pragma unroll
-            for (int m = 0; m < 8; ++m) acc[m] = fmaf(pv, Zs[jj * 65 + tp + 8 * m], acc[m]);
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) acc[a][q] = fmaf(pp[a], zz[q], acc[a][q]);
         }
     }
-    // boundary-state term
-    float acc2[8];
+    // boundary-state term, M's rows in tiles of kFT (reusing the Z tile)
+    float acc2[4][4];
 #pragma unroll
-    for (int m = 0; m < 8; ++m) acc2[m] = 0.f;
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc2[a][q] = 0.f;
     const float* Mk = Mst + ((size_t)bh * nc + k) * (size_t)NP;
-    for (int k0 = 0; k0 < K; k0 += 32) {
+    for (int k0 = 0; k0 < K; k0 += kFT) {
         __syncthreads();
-        for (int idx = tid; idx < 32 * 64; idx += 256) {
-            const int kk = idx / 64, m = idx % 64;
-            Ms[kk * 65 + m] = (k0 + kk < K && m0 + m < Mc)
-                                  ? Mk[(size_t)(k0 + kk) * sk + (size_t)(m0 + m) * sm]
-                                  : 0.f;
+        for (int idx = tid; idx < kFT * kFT; idx += 256) {
+            const int kk = idx / kFT, m = idx % kFT;
+            ZM[kk * kFS + m] = (k0 + kk < K && m0 + m < Mc)
+                                   ? Mk[(size_t)(k0 + kk) * sk + (size_t)(m0 + m) * sm]
+                                   : 0.f;
         }
         __syncthreads();
-        const int kmax = min(32, K - k0);
+        const int kmax = min(kFT, K - k0);
         for (int kk = 0; kk < kmax; ++kk) {
-            const float uv = Us[ti * KS + k0 + kk];
+            const float4 u = *reinterpret_cast<const float4*>(UT + (k0 + kk) * kFS + 4 * r);
+            const float4 mv = *reinterpret_cast<const float4*>(ZM + kk * kFS + 4 * c);
+            const float uu[4] = {u.x, u.y, u.z, u.w}, mm[4] = {mv.x, mv.y, mv.z, mv.w};
 #pragma unroll
-            for (int m = 0; m < 8; ++m) acc2[m] = fmaf(uv, Ms[kk * 65 + tp + 8 * m], acc2[m]);
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) acc2[a][q] = fmaf(uu[a], mm[q], acc2[a][q]);
         }
     }
-    if (i >= qv) return;
-    const float sc = ANTI ? expf(cumk[Q - 1] - cr[ti]) : expf(cr[ti]);
-    float* o = out + (((size_t)b * Tlen + tk + i) * H + h) * Mc;
+    const float cend = cumk[Q - 1];
 #pragma unroll
-    for (int m = 0; m < 8; ++m) {
-        const int mm = m0 + tp + 8 * m;
-        if (mm < Mc) o[mm] = fmaf(sc, acc2[m], acc[m]);
+    for (int a = 0; a < 4; ++a) {
+        const int ii = 4 * r + a, i = i0 + ii;
+        if (i >= qv) continue;
+        const float sc = ANTI ? expf(cend - cr[ii]) : expf(cr[ii]);
+        float* o = out + (((size_t)b * Tlen + tk + i) * H + h) * Mc;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int m = m0 + 4 * c + q;
+            if (m < Mc) o[m] = fmaf(sc, acc2[a][q], acc[a][q]);
+        }
     }
 }
 
@@ -289,11 +324,11 @@ __global__ void __launch_bounds__(256) group_sum_kernel(const float* __restrict_
 template <typename T, bool ANTI>
 cudaError_t launch_form(const Dims& d, Opd U, Opd V, Opd Z, const float* cum, const float* Mst,
                         int sk, int sm, float* out, int K, int Mc, cudaStream_t st) {
-    const size_t smem = (size_t)(2 * 32 * (K + 1) + 32 * 65 + 32 * 33 + 32 * 65 + 64) * sizeof(float);
+    const size_t smem = (size_t)(2 * K * kFS + 2 * kFT * kFS + 2 * kFT) * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(chunk_form_kernel<T, ANTI>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(d.nc * ((d.Q + 31) / 32), d.B * d.H, (Mc + 63) / 64);
+    dim3 grid(d.nc * ((d.Q + kFT - 1) / kFT), d.B * d.H, (Mc + kFT - 1) / kFT);
     chunk_form_kernel<T, ANTI><<<grid, 256, smem, st>>>(U, V, Z, cum, Mst, sk, sm, out, d.T, d.H, K,
                                                         Mc, d.Q, d.nc, d.N * d.P);
     return cudaGetLastError();
