@@ -105,7 +105,93 @@ __device__ __forceinline__ float opd_at(const Opd& o, int b, int Tlen, int t, in
 constexpr int kFT = 64;  // tile rows / columns
 constexpr int kFS = 68;  // row stride of the shared tiles (16-byte aligned rows)
 
-template <typename T, bool ANTI>
+// 16 bytes of a row (8 bf16 or 4 fp32 values) as floats
+template <typename T>
+__device__ __forceinline__ void load16(const T* p, float* out);
+template <>
+__device__ __forceinline__ void load16<__nv_bfloat16>(const __nv_bfloat16* p, float* out) {
+    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        __nv_bfloat162 v2;
+        memcpy(&v2, &w[e], 4);
+        const float2 f = __bfloat1622float2(v2);
+        out[2 * e] = f.x;
+        out[2 * e + 1] = f.y;
+    }
+}
+template <>
+__device__ __forceinline__ void load16<float>(const float* p, float* out) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(p));
+    out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
+}
+
+template <typename T>
+__device__ __forceinline__ const T* opd_row(const Opd& o, int b, int Tlen, int t, int h) {
+    return static_cast<const T*>(o.p) + ((size_t)b * Tlen + t) * o.ld_t + (size_t)(h / o.hdiv) * o.ld_h;
+}
+
+// dst[kk * kFS + rr] = operand(row tk + r0 + rr, kk) for the kFT rows of a
+// tile (zero for rows at or past qv): the tile transposed to k-major.  VEC
+// reads 16 bytes per thread (K a multiple of 16 / sizeof(T)).
+template <typename T, bool VEC>
+__device__ __forceinline__ void load_kmajor(float* dst, const Opd& o, int b, int Tlen, int tk, int r0,
+                                            int qv, int h, int K, int tid) {
+    if (VEC) {
+        constexpr int W = 16 / sizeof(T);
+        const int KV = K / W;
+        for (int v = tid; v < kFT * KV; v += 256) {
+            const int rr = v / KV, kv = v - rr * KV, row = r0 + rr;
+            float e[W];
+            if (row < qv) {
+                load16<T>(opd_row<T>(o, b, Tlen, tk + row, h) + kv * W, e);
+            } else {
+#pragma unroll
+                for (int w = 0; w < W; ++w) e[w] = 0.f;
+            }
+#pragma unroll
+            for (int w = 0; w < W; ++w) dst[(kv * W + w) * kFS + rr] = e[w];
+        }
+    } else {
+        for (int idx = tid; idx < kFT * K; idx += 256) {
+            const int rr = idx / K, kk = idx % K, row = r0 + rr;
+            dst[kk * kFS + rr] = (row < qv) ? opd_at<T>(o, b, Tlen, tk + row, h, kk) : 0.f;
+        }
+    }
+}
+
+// dst[rr * kFS + m] = operand(row tk + r0 + rr, m0 + m) for m < kFT (zero past
+// qv or Mc).  VEC: Mc a multiple of 16 / sizeof(T).
+template <typename T, bool VEC>
+__device__ __forceinline__ void load_mmajor(float* dst, const Opd& o, int b, int Tlen, int tk, int r0,
+                                            int qv, int h, int m0, int Mc, int tid) {
+    if (VEC) {
+        constexpr int W = 16 / sizeof(T);
+        constexpr int MV = kFT / W;
+        for (int v = tid; v < kFT * MV; v += 256) {
+            const int rr = v / MV, mv = v % MV, row = r0 + rr, m = m0 + mv * W;
+            float e[W];
+            if (row < qv && m < Mc) {
+                load16<T>(opd_row<T>(o, b, Tlen, tk + row, h) + m, e);
+            } else {
+#pragma unroll
+                for (int w = 0; w < W; ++w) e[w] = 0.f;
+            }
+#pragma unroll
+            for (int w = 0; w < W; w += 4)
+                *reinterpret_cast<float4*>(dst + rr * kFS + mv * W + w) =
+                    make_float4(e[w], e[w + 1], e[w + 2], e[w + 3]);
+        }
+    } else {
+        for (int idx = tid; idx < kFT * kFT; idx += 256) {
+            const int rr = idx / kFT, m = idx % kFT, row = r0 + rr;
+            dst[rr * kFS + m] = (row < qv && m0 + m < Mc) ? opd_at<T>(o, b, Tlen, tk + row, h, m0 + m) : 0.f;
+        }
+    }
+}
+
+template <typename T, bool ANTI, bool VEC>
 __global__ void __launch_bounds__(256) chunk_form_kernel(Opd U, Opd V, Opd Z,
                                                          const float* __restrict__ cum,
                                                          const float* __restrict__ Mst, int sk,
@@ -129,10 +215,7 @@ __global__ void __launch_bounds__(256) chunk_form_kernel(Opd U, Opd V, Opd Z,
     if (i0 >= qv) return;              // a tile wholly past T (the whole block leaves)
     const float* cumk = cum + ((size_t)bh * nc + k) * (size_t)Q;
 
-    for (int idx = tid; idx < kFT * K; idx += 256) {
-        const int ii = idx / K, kk = idx % K, i = i0 + ii;
-        UT[kk * kFS + ii] = (i < qv) ? opd_at<T>(U, b, Tlen, tk + i, h, kk) : 0.f;
-    }
+    load_kmajor<T, VEC>(UT, U, b, Tlen, tk, i0, qv, h, K, tid);
     if (tid < kFT) cr[tid] = (i0 + tid < qv) ? cumk[i0 + tid] : 0.f;
 
     float acc[4][4];
@@ -144,15 +227,9 @@ __global__ void __launch_bounds__(256) chunk_form_kernel(Opd U, Opd V, Opd Z,
     const int j_end = ANTI ? qv : min(i0 + kFT, qv);  // one past the last column token
     for (int j0 = j_first; j0 < j_end; j0 += kFT) {
         __syncthreads();
-        for (int idx = tid; idx < kFT * K; idx += 256) {
-            const int jj = idx / K, kk = idx % K, j = j0 + jj;
-            VT[kk * kFS + jj] = (j < qv) ? opd_at<T>(V, b, Tlen, tk + j, h, kk) : 0.f;
-        }
+        load_kmajor<T, VEC>(VT, V, b, Tlen, tk, j0, qv, h, K, tid);
         if (tid < kFT) cc[tid] = (j0 + tid < qv) ? cumk[j0 + tid] : 0.f;
-        for (int idx = tid; idx < kFT * kFT; idx += 256) {
-            const int jj = idx / kFT, m = idx % kFT, j = j0 + jj;
-            ZM[jj * kFS + m] = (j < qv && m0 + m < Mc) ? opd_at<T>(Z, b, Tlen, tk + j, h, m0 + m) : 0.f;
-        }
+        load_mmajor<T, VEC>(ZM, Z, b, Tlen, tk, j0, qv, h, m0, Mc, tid);
         __syncthreads();
         // scores s[a][q] = U_{4r+a} . V_{4c+q}
         float s[4][4];
@@ -321,17 +398,28 @@ __global__ void __launch_bounds__(256) group_sum_kernel(const float* __restrict_
     dC[e] = from_f32<T>(sc);
 }
 
-template <typename T, bool ANTI>
-cudaError_t launch_form(const Dims& d, Opd U, Opd V, Opd Z, const float* cum, const float* Mst,
-                        int sk, int sm, float* out, int K, int Mc, cudaStream_t st) {
+template <typename T, bool ANTI, bool VEC>
+cudaError_t launch_form_v(const Dims& d, Opd U, Opd V, Opd Z, const float* cum, const float* Mst,
+                          int sk, int sm, float* out, int K, int Mc, cudaStream_t st) {
     const size_t smem = (size_t)(2 * K * kFS + 2 * kFT * kFS + 2 * kFT) * sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(chunk_form_kernel<T, ANTI>,
+    cudaError_t e = cudaFuncSetAttribute(chunk_form_kernel<T, ANTI, VEC>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(d.nc * ((d.Q + kFT - 1) / kFT), d.B * d.H, (Mc + kFT - 1) / kFT);
-    chunk_form_kernel<T, ANTI><<<grid, 256, smem, st>>>(U, V, Z, cum, Mst, sk, sm, out, d.T, d.H, K,
-                                                        Mc, d.Q, d.nc, d.N * d.P);
+    chunk_form_kernel<T, ANTI, VEC><<<grid, 256, smem, st>>>(U, V, Z, cum, Mst, sk, sm, out, d.T, d.H,
+                                                             K, Mc, d.Q, d.nc, d.N * d.P);
     return cudaGetLastError();
+}
+
+// 16-byte row reads need every row length (N, P) a multiple of 16 bytes of
+// elements; the pointers are 16-byte aligned (checked at the boundary)
+template <typename T, bool ANTI>
+cudaError_t launch_form(const Dims& d, Opd U, Opd V, Opd Z, const float* cum, const float* Mst,
+                        int sk, int sm, float* out, int K, int Mc, cudaStream_t st) {
+    constexpr int W = 16 / sizeof(T);
+    if (d.N % W == 0 && d.P % W == 0)
+        return launch_form_v<T, ANTI, true>(d, U, V, Z, cum, Mst, sk, sm, out, K, Mc, st);
+    return launch_form_v<T, ANTI, false>(d, U, V, Z, cum, Mst, sk, sm, out, K, Mc, st);
 }
 
 template <typename T>
