@@ -468,7 +468,10 @@ cudaError_t launch_backward(const Dims& d, const BackwardArgs& g, const Backward
     cudaError_t e;
     // forward states, recomputed: in-chunk cumsum, chunk states, states entering each chunk
     if ((e = launch_chunk_cumsum(d, g.a, w.cum, st))) return e;
-    if ((e = launch_chunk_state_simt(d, g.x, g.Bm, w.cum, w.states, st))) return e;
+    // (the tensor-core chunk-state kernel serves the bf16 Mamba-2 heads)
+    e = chunk_state_tc_supported(d) ? launch_chunk_state_tc(d, g.x, g.Bm, w.cum, w.states, st)
+                                    : launch_chunk_state_simt(d, g.x, g.Bm, w.cum, w.states, st);
+    if (e) return e;
     if ((e = launch_state_pass(d, w.cum, w.states, w.fin, g.init, st))) return e;
     // adjoint states: each chunk's readout term, then the reverse pass
     if ((e = launch_chunk_dstate_simt(d, g.dy, g.Cm, w.cum, w.dstates, st))) return e;

@@ -80,6 +80,38 @@ def test_backward_matches_oracle(w, with_init, with_dfinal):
     assert all(e <= tol for e in errs.values()), errs
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_backward_maximum_sizes(dtype):
+    """N = P = 256 (the largest the boundary takes: the widest shared tiles)
+    with a partial last chunk."""
+    w = small_case(B=1, T=200, H=2, P=256, N=256, G=1, chunk=128, dtype=dtype, seed=91)
+    got, ref = _run(w, True, True)
+    errs = {k: rel_err(got[k].float().cpu().numpy().astype(np.float64), ref[k])
+            for k in ("dx", "da", "dBm", "dCm", "dD", "dinit")}
+    assert all(e <= tol_for(w) for e in errs.values()), errs
+
+
+def test_backward_without_D_and_deterministic():
+    """D = NULL is D = 0 (dx carries no skip term; dD is still sum dy.x), and
+    two calls on the same inputs give bit-identical gradients."""
+    w = small_case(B=2, T=256, H=4, P=64, N=128, G=2, chunk=128, dtype="bf16", seed=92)
+    inp = generate(w)
+    dev = to_dev(inp)
+    dy, _, dfin = _extras(w, False, True)
+    run = lambda: ssd.backward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], None, dy.cuda(), w.chunk,
+                               dfinal=dfin.cuda())
+    g1, g2 = run(), run()
+    torch.cuda.synchronize()
+    for k in ("dx", "da", "dBm", "dCm", "dD", "dinit"):
+        assert torch.equal(g1[k], g2[k]), k
+    f = lambda t: t.to(torch.float64).numpy()
+    prob = O.Problem(f(inp["x"]), f(inp["a"]), f(inp["Bm"]), f(inp["Cm"]), None)
+    ref = O.backward(prob, f(dy), dfinal=f(dfin))
+    errs = {k: rel_err(g1[k].float().cpu().numpy().astype(np.float64), ref[k])
+            for k in ("dx", "da", "dBm", "dCm", "dD", "dinit")}
+    assert all(e <= tol_for(w) for e in errs.values()), errs
+
+
 def test_backward_rejects_per_state_and_bad_workspace():
     """The per-state variant is not served (SSD_ERR_UNSUPPORTED) and a short
     workspace is refused before any launch."""
