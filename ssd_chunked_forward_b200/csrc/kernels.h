@@ -45,7 +45,7 @@ cudaError_t launch_decode_step(const Dims& d, const void* x, const float* a, con
                                const void* Cm, const float* D, float* state, void* y,
                                cudaStream_t st);
 
-// ---- backward (scalar decay, CUDA cores, fp32) ------------------------------
+// ---- backward (CUDA cores, fp32) --------------------------------------------
 // dstates[b,h,k] = sum_j exp(cum_j) C_j dy_j^T: each chunk's readout term of the
 // adjoint of the state entering it
 cudaError_t launch_chunk_dstate_simt(const Dims& d, const void* dy, const void* Cm,
@@ -61,19 +61,24 @@ struct BackwardArgs {
     float* dinit;         // [B,H,N,P] or null
 };
 struct BackwardScratch {
-    float* cum;      // [B,H,nc,Q]
+    float* cum;      // [B,H,nc,Q] ([B,H,nc,Q,N] per-state)
     float* states;   // [B,H,nc,N,P]  states entering each chunk
     float* dstates;  // [B,H,nc,N,P]  adjoint at each chunk's last token
     float* fin;      // [B,H,N,P]
-    float* cdot;     // [B,H,nc]
+    float* cdot;     // [B,H,nc] ([B,H,nc,N] per-state)
     float* dDpart;   // [B,H,nc]
-    float* ytil;     // [B,T,H,P]  y - D x
+    float* ytil;     // [B,T,H,P]  y - D x (scalar decay only)
     float* dxt;      // [B,T,H,P]  dx - D dy
     float* dBh;      // [B,T,H,N]  per head
     float* dCh;      // [B,T,H,N]  per head
 };
 cudaError_t launch_backward(const Dims& d, const BackwardArgs& g, const BackwardScratch& w,
                             cudaStream_t st);
+// per-state decay (backward_diag.cu): everything up to dD and the group sums
+constexpr int kBackwardDiagMaxN = 128;
+bool backward_diag_supported(const Dims& d);
+cudaError_t launch_backward_diag(const Dims& d, const BackwardArgs& g, const BackwardScratch& w,
+                                 cudaStream_t st);
 
 // ---- tensor-core kernels (tcgen05 + TMEM + TMA) ----------------------------
 bool chunk_state_tc_supported(const Dims& d);

@@ -26,9 +26,16 @@
 // dB and dC are formed per head and summed over each group's heads.
 #include "../common.cuh"
 #include "../kernels.h"
+#include "bwd_tiles.cuh"
 
 namespace ssd {
 namespace {
+
+using bwd::Opd;
+using bwd::kFS;
+using bwd::kFT;
+using bwd::load_kmajor;
+using bwd::load_mmajor;
 
 // ------------------------------------------------ reverse state pass ----
 // One thread per (b, h, n, p): G_k into slot k of dstates (which held the
@@ -77,21 +84,6 @@ __global__ void __launch_bounds__(256) chunk_dot_kernel(const float* __restrict_
     }
 }
 
-// ------------------------------------------------ chunk quadratic forms ----
-// A token operand of one chain: element (b, t, h, i) at
-// p[(b * T + t) * ld_t + (h / hdiv) * ld_h + i] -- x and dy are [B,T,H,P]
-// (ld_t = H P, ld_h = P, hdiv = 1), B and C are [B,T,G,N] (ld_t = G N,
-// ld_h = N, hdiv = H / G).
-struct Opd {
-    const void* p;
-    int ld_t, ld_h, hdiv;
-};
-
-template <typename T>
-__device__ __forceinline__ float opd_at(const Opd& o, int b, int Tlen, int t, int h, int i) {
-    return to_f32(static_cast<const T*>(o.p)[((size_t)b * Tlen + t) * o.ld_t + (size_t)(h / o.hdiv) * o.ld_h + i]);
-}
-
 // out[b, kQ+i, h, m] for one 64-row tile and 64 columns of one chunk:
 //   causal (ANTI = false):  sum_{j<=i} (U_i.V_j) e^{c_i-c_j} Z_j[m] + e^{c_i}       sum_kk U_i[kk] M[kk,m]
 //   anti   (ANTI = true):   sum_{j>=i} (U_i.V_j) e^{c_j-c_i} Z_j[m] + e^{c_end-c_i} sum_kk U_i[kk] M[kk,m]
@@ -102,95 +94,6 @@ __device__ __forceinline__ float opd_at(const Opd& o, int b, int Tlen, int t, in
 // rows 4r..4r+3 and score / output columns 4c..4c+3.  The operands sit in
 // shared memory k-major (U^T, V^T, and the masked scores transposed), so each
 // step of every contraction is two 16-byte loads for 16 FMAs.
-constexpr int kFT = 64;  // tile rows / columns
-constexpr int kFS = 68;  // row stride of the shared tiles (16-byte aligned rows)
-
-// 16 bytes of a row (8 bf16 or 4 fp32 values) as floats
-template <typename T>
-__device__ __forceinline__ void load16(const T* p, float* out);
-template <>
-__device__ __forceinline__ void load16<__nv_bfloat16>(const __nv_bfloat16* p, float* out) {
-    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(p));
-    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        __nv_bfloat162 v2;
-        memcpy(&v2, &w[e], 4);
-        const float2 f = __bfloat1622float2(v2);
-        out[2 * e] = f.x;
-        out[2 * e + 1] = f.y;
-    }
-}
-template <>
-__device__ __forceinline__ void load16<float>(const float* p, float* out) {
-    const float4 v = __ldg(reinterpret_cast<const float4*>(p));
-    out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
-}
-
-template <typename T>
-__device__ __forceinline__ const T* opd_row(const Opd& o, int b, int Tlen, int t, int h) {
-    return static_cast<const T*>(o.p) + ((size_t)b * Tlen + t) * o.ld_t + (size_t)(h / o.hdiv) * o.ld_h;
-}
-
-// dst[kk * kFS + rr] = operand(row tk + r0 + rr, kk) for the kFT rows of a
-// tile (zero for rows at or past qv): the tile transposed to k-major.  VEC
-// reads 16 bytes per thread (K a multiple of 16 / sizeof(T)).
-template <typename T, bool VEC>
-__device__ __forceinline__ void load_kmajor(float* dst, const Opd& o, int b, int Tlen, int tk, int r0,
-                                            int qv, int h, int K, int tid) {
-    if (VEC) {
-        constexpr int W = 16 / sizeof(T);
-        const int KV = K / W;
-        for (int v = tid; v < kFT * KV; v += 256) {
-            const int rr = v / KV, kv = v - rr * KV, row = r0 + rr;
-            float e[W];
-            if (row < qv) {
-                load16<T>(opd_row<T>(o, b, Tlen, tk + row, h) + kv * W, e);
-            } else {
-#pragma unroll
-                for (int w = 0; w < W; ++w) e[w] = 0.f;
-            }
-#pragma unroll
-            for (int w = 0; w < W; ++w) dst[(kv * W + w) * kFS + rr] = e[w];
-        }
-    } else {
-        for (int idx = tid; idx < kFT * K; idx += 256) {
-            const int rr = idx / K, kk = idx % K, row = r0 + rr;
-            dst[kk * kFS + rr] = (row < qv) ? opd_at<T>(o, b, Tlen, tk + row, h, kk) : 0.f;
-        }
-    }
-}
-
-// dst[rr * kFS + m] = operand(row tk + r0 + rr, m0 + m) for m < kFT (zero past
-// qv or Mc).  VEC: Mc a multiple of 16 / sizeof(T).
-template <typename T, bool VEC>
-__device__ __forceinline__ void load_mmajor(float* dst, const Opd& o, int b, int Tlen, int tk, int r0,
-                                            int qv, int h, int m0, int Mc, int tid) {
-    if (VEC) {
-        constexpr int W = 16 / sizeof(T);
-        constexpr int MV = kFT / W;
-        for (int v = tid; v < kFT * MV; v += 256) {
-            const int rr = v / MV, mv = v % MV, row = r0 + rr, m = m0 + mv * W;
-            float e[W];
-            if (row < qv && m < Mc) {
-                load16<T>(opd_row<T>(o, b, Tlen, tk + row, h) + m, e);
-            } else {
-#pragma unroll
-                for (int w = 0; w < W; ++w) e[w] = 0.f;
-            }
-#pragma unroll
-            for (int w = 0; w < W; w += 4)
-                *reinterpret_cast<float4*>(dst + rr * kFS + mv * W + w) =
-                    make_float4(e[w], e[w + 1], e[w + 2], e[w + 3]);
-        }
-    } else {
-        for (int idx = tid; idx < kFT * kFT; idx += 256) {
-            const int rr = idx / kFT, m = idx % kFT, row = r0 + rr;
-            dst[rr * kFS + m] = (row < qv && m0 + m < Mc) ? opd_at<T>(o, b, Tlen, tk + row, h, m0 + m) : 0.f;
-        }
-    }
-}
-
 template <typename T, bool ANTI, bool VEC>
 __global__ void __launch_bounds__(256) chunk_form_kernel(Opd U, Opd V, Opd Z,
                                                          const float* __restrict__ cum,
@@ -446,26 +349,34 @@ cudaError_t run_backward_t(const Dims& d, const BackwardArgs& g, const BackwardS
             d.T, d.H, d.P, d.Q, d.nc);
         if ((e = cudaGetLastError())) return e;
     }
+    return cudaSuccess;
+}
+
+// dD from the per-chunk partial sums; dB and dC summed over each group's heads
+template <typename T>
+cudaError_t finish_t(const Dims& d, const BackwardArgs& g, const BackwardScratch& w,
+                     cudaStream_t st) {
+    cudaError_t e;
     if (g.dD) {
         dD_reduce_kernel<<<(d.H + 127) / 128, 128, 0, st>>>(w.dDpart, g.dD, d.B, d.H, d.nc);
         if ((e = cudaGetLastError())) return e;
     }
-    {
-        const long long rows = (long long)d.B * d.T;
-        const long long total = rows * d.G * d.N;
-        group_sum_kernel<T><<<(unsigned)((total + 255) / 256), 256, 0, st>>>(
-            w.dBh, w.dCh, (T*)g.dBm, (T*)g.dCm, rows, d.H, d.G, d.N);
-        if ((e = cudaGetLastError())) return e;
-    }
-    return cudaSuccess;
+    const long long rows = (long long)d.B * d.T;
+    const long long total = rows * d.G * d.N;
+    group_sum_kernel<T><<<(unsigned)((total + 255) / 256), 256, 0, st>>>(
+        w.dBh, w.dCh, (T*)g.dBm, (T*)g.dCm, rows, d.H, d.G, d.N);
+    return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_backward(const Dims& d, const BackwardArgs& g, const BackwardScratch& w,
                             cudaStream_t st) {
-    if (d.diag) return cudaErrorNotSupported;
     cudaError_t e;
+    if (d.diag) {
+        if ((e = launch_backward_diag(d, g, w, st))) return e;
+        return d.bf16 ? finish_t<__nv_bfloat16>(d, g, w, st) : finish_t<float>(d, g, w, st);
+    }
     // forward states, recomputed: in-chunk cumsum, chunk states, states entering each chunk
     if ((e = launch_chunk_cumsum(d, g.a, w.cum, st))) return e;
     // (the tensor-core chunk-state kernel serves the bf16 Mamba-2 heads)
@@ -484,7 +395,12 @@ cudaError_t launch_backward(const Dims& d, const BackwardArgs& g, const Backward
     chunk_dot_kernel<<<dim3(d.nc, d.B * d.H), 256, 0, st>>>(w.dstates, w.states, w.fin, w.cdot,
                                                             d.N * d.P, d.nc);
     if ((e = cudaGetLastError())) return e;
-    return d.bf16 ? run_backward_t<__nv_bfloat16>(d, g, w, st) : run_backward_t<float>(d, g, w, st);
+    if (d.bf16) {
+        if ((e = run_backward_t<__nv_bfloat16>(d, g, w, st))) return e;
+        return finish_t<__nv_bfloat16>(d, g, w, st);
+    }
+    if ((e = run_backward_t<float>(d, g, w, st))) return e;
+    return finish_t<float>(d, g, w, st);
 }
 
 }  // namespace ssd

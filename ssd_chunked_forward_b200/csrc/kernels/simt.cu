@@ -101,8 +101,9 @@ cudaError_t launch_chunk_cumsum(const Dims& d, const float* a, float* cum, cudaS
 // ============================================================ step 2 ======
 // states[b,h,k,n,p] = sum_j B[j,n] w[j,n] x[j,p], w = exp(cum_end - cum_j).
 // Block = (chunk, b*H+h, 64x64 output tile); 16x16 threads, 4x4 outputs each.
-// FROM_START (scalar decay, backward): w = exp(cum_j), the decay from the
-// state entering the chunk to token j, with (C, dy) in place of (B, x).
+// FROM_START (backward): w = exp(cum_j), the decay from the state entering
+// the chunk to token j (per n for the per-state decay), with (C, dy) in place
+// of (B, x).
 template <typename T, bool DIAG, bool FROM_START = false>
 __global__ void __launch_bounds__(256) chunk_state_simt_kernel(
     const T* __restrict__ x, const T* __restrict__ Bm, const float* __restrict__ cum,
@@ -129,7 +130,9 @@ __global__ void __launch_bounds__(256) chunk_state_simt_kernel(
                 const size_t t = (size_t)k * Q + j;
                 if (n0 + c < N) {
                     float w;
-                    if (DIAG)
+                    if (DIAG && FROM_START)
+                        w = expf(cumk[(size_t)j * N + n0 + c]);
+                    else if (DIAG)
                         w = expf(cumk[(size_t)(Q - 1) * N + n0 + c] - cumk[(size_t)j * N + n0 + c]);
                     else if (FROM_START)
                         w = expf(cumk[j]);
@@ -189,15 +192,16 @@ cudaError_t launch_chunk_state_simt(const Dims& d, const void* x, const void* Bm
 
 cudaError_t launch_chunk_dstate_simt(const Dims& d, const void* dy, const void* Cm,
                                      const float* cum, float* dstates, cudaStream_t st) {
-    if (d.diag) return cudaErrorNotSupported;
     dim3 grid(d.nc, d.B * d.H, ((d.N + 63) / 64) * ((d.P + 63) / 64));
-    if (d.bf16)
-        chunk_state_simt_kernel<__nv_bfloat16, false, true><<<grid, 256, 0, st>>>(
-            (const __nv_bfloat16*)dy, (const __nv_bfloat16*)Cm, cum, dstates, d.T, d.H, d.P, d.G,
-            d.N, d.Q, d.nc);
-    else
-        chunk_state_simt_kernel<float, false, true><<<grid, 256, 0, st>>>(
-            (const float*)dy, (const float*)Cm, cum, dstates, d.T, d.H, d.P, d.G, d.N, d.Q, d.nc);
+#define SSD_DS_LAUNCH(TT, DG)                                                                    \
+    chunk_state_simt_kernel<TT, DG, true><<<grid, 256, 0, st>>>(                                \
+        (const TT*)dy, (const TT*)Cm, cum, dstates, d.T, d.H, d.P, d.G, d.N, d.Q, d.nc)
+    if (d.bf16) {
+        if (d.diag) SSD_DS_LAUNCH(__nv_bfloat16, true); else SSD_DS_LAUNCH(__nv_bfloat16, false);
+    } else {
+        if (d.diag) SSD_DS_LAUNCH(float, true); else SSD_DS_LAUNCH(float, false);
+    }
+#undef SSD_DS_LAUNCH
     return cudaGetLastError();
 }
 

@@ -108,13 +108,13 @@ size_t backward_layout(const Dims& d, void* base, ssd::BackwardScratch* w) {
     const size_t f = sizeof(float);
     const size_t chains = (size_t)d.B * d.H;
     const size_t sizes[10] = {
-        chains * d.nc * d.Q * f,                  // cum
+        chains * d.nc * d.Q * (d.diag ? d.N : 1) * f,  // cum
         chains * d.nc * d.N * d.P * f,            // states
         chains * d.nc * d.N * d.P * f,            // dstates
         chains * d.N * d.P * f,                   // fin
-        chains * d.nc * f,                        // cdot
+        chains * d.nc * (d.diag ? d.N : 1) * f,   // cdot
         chains * d.nc * f,                        // dDpart
-        (size_t)d.B * d.T * d.H * d.P * f,        // ytil
+        d.diag ? 0 : (size_t)d.B * d.T * d.H * d.P * f,  // ytil
         (size_t)d.B * d.T * d.H * d.P * f,        // dxt
         (size_t)d.B * d.T * d.H * d.N * f,        // dBh
         (size_t)d.B * d.T * d.H * d.N * f,        // dCh
@@ -477,7 +477,7 @@ ssd_status ssd_backward(const ssd_shape* shape, const void* x, const float* a, c
                         float* dinit, void* workspace, size_t ws_bytes, ssd_stream stream) {
     ssd_status st = check_shape(shape);
     if (st != SSD_OK) return st;
-    if (shape->a_per_state) return SSD_ERR_UNSUPPORTED;
+    if (shape->a_per_state && !ssd::backward_diag_supported(dims_of(shape))) return SSD_ERR_UNSUPPORTED;
     if (!x || !a || !Bm || !Cm || !dy || !dx || !da || !dBm || !dCm) return SSD_ERR_INVALID_ARG;
     const void* ptrs[] = {x, a, Bm, Cm, D, initial_state, dy, dfinal, dx, da, dBm, dCm, dD, dinit};
     for (const void* p : ptrs)
@@ -493,7 +493,8 @@ ssd_status ssd_backward(const ssd_shape* shape, const void* x, const float* a, c
 }
 
 size_t ssd_backward_workspace_size(const ssd_shape* shape) {
-    if (check_shape(shape) != SSD_OK || shape->a_per_state) return 0;
+    if (check_shape(shape) != SSD_OK) return 0;
+    if (shape->a_per_state && !ssd::backward_diag_supported(dims_of(shape))) return 0;
     return backward_layout(dims_of(shape), nullptr, nullptr);
 }
 

@@ -97,15 +97,17 @@ def test_ragged_T_is_a_partial_last_chunk(lib, T, chunk):
 
 def test_backward_workspace_and_validation(lib):
     """The backward's workspace holds the recomputed and adjoint chunk states
-    and the fp32 per-head partials; the per-state variant is not served; bad
-    pointers and a short workspace are refused before any launch."""
+    and the fp32 per-head partials; the per-state variant is served up to
+    N = 128; bad pointers and a short workspace are refused before any launch."""
     s = _shape()  # B=2, T=512, H=4, P=64, N=128, chunk 256
     need = ssd.backward_workspace_size(s)
     nc, f = 2, 4
     pieces = [2 * 4 * nc * 256 * f, 2 * 2 * 4 * nc * 128 * 64 * f, 2 * 4 * 128 * 64 * f,
               2 * 2 * 512 * 4 * 64 * f, 2 * 2 * 512 * 4 * 128 * f]
     assert need >= sum(pieces)
-    assert ssd.backward_workspace_size(_shape(a_per_state=True)) == 0
+    # the per-state variant is served up to N = 128
+    assert ssd.backward_workspace_size(_shape(a_per_state=True)) > need
+    assert ssd.backward_workspace_size(_shape(a_per_state=True, N=256)) == 0
     ok = 1 << 20
     f_ = lambda *a: lib.ssd_backward(ctypes.byref(s), *a)
     args = [ok, ok, ok, ok, None, None, ok, None, ok, ok, ok, ok, None, None, ok, need, None]
@@ -117,7 +119,7 @@ def test_backward_workspace_and_validation(lib):
     assert f_(*bad) == ssd.SSD_ERR_WORKSPACE
     bad = list(args); bad[14] = ok + 16        # workspace misaligned
     assert f_(*bad) == ssd.SSD_ERR_WORKSPACE
-    sp = _shape(a_per_state=True)
+    sp = _shape(a_per_state=True, N=256)
     assert lib.ssd_backward(ctypes.byref(sp), *args) == ssd.SSD_ERR_UNSUPPORTED
 
 

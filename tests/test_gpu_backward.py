@@ -40,8 +40,19 @@ CASES = [
 ]
 
 
+# per-state decay (a [B,T,H,N]); served up to N = 128
+DIAG_CASES = [
+    small_case(B=1, T=150, H=2, P=20, N=12, G=1, chunk=64, dtype="f32", a_per_state=True, seed=93),
+    small_case(B=2, T=256, H=2, P=64, N=64, G=1, chunk=128, dtype="bf16", a_per_state=True, seed=94),
+    small_case(B=2, T=200, H=4, P=16, N=24, G=2, chunk=128, dtype="f32", a_per_state=True, seed=95),
+    small_case(B=1, T=130, H=2, P=64, N=128, G=1, chunk=64, dtype="bf16", a_per_state=True, seed=96),
+    small_case(B=1, T=70, H=2, P=256, N=32, G=1, chunk=64, dtype="f32", a_per_state=True, seed=97),
+    small_case(B=1, T=5, H=1, P=3, N=2, G=1, chunk=1, dtype="f32", a_per_state=True, seed=98),
+]
+
+
 def _ids(cases):
-    return [c.name + "_" + c.dtype for c in cases]
+    return [c.name + ("_diag" if c.a_per_state else "") + "_" + c.dtype for c in cases]
 
 
 def _extras(w, with_init, with_dfinal):
@@ -67,7 +78,7 @@ def _run(w, with_init, with_dfinal):
     return got, ref
 
 
-@pytest.mark.parametrize("w", CASES, ids=_ids(CASES))
+@pytest.mark.parametrize("w", CASES + DIAG_CASES, ids=_ids(CASES + DIAG_CASES))
 @pytest.mark.parametrize("with_init,with_dfinal", [(False, False), (True, True)],
                          ids=["plain", "init_dfinal"])
 def test_backward_matches_oracle(w, with_init, with_dfinal):
@@ -113,9 +124,9 @@ def test_backward_without_D_and_deterministic():
 
 
 def test_backward_rejects_per_state_and_bad_workspace():
-    """The per-state variant is not served (SSD_ERR_UNSUPPORTED) and a short
-    workspace is refused before any launch."""
-    w = small_case(B=1, T=64, H=2, P=16, N=16, G=1, chunk=32, dtype="f32", a_per_state=True, seed=87)
+    """The per-state variant above N = 128 is not served (SSD_ERR_UNSUPPORTED)
+    and a short workspace is refused before any launch."""
+    w = small_case(B=1, T=64, H=2, P=16, N=256, G=1, chunk=32, dtype="f32", a_per_state=True, seed=87)
     dev = to_dev(generate(w))
     shape = ssd.shape_of(dev["x"], dev["a"], dev["Bm"], w.chunk)
     assert ssd.backward_workspace_size(shape) == 0
