@@ -301,7 +301,7 @@ ssd_status ssd_decode_step(const ssd_shape* shape, const void* x, const float* a
                            const void* Cm, const float* D, float* state, void* y,
                            ssd_stream stream);
 
-/* Backward of the forward (scalar decay): the gradients of
+/* Backward of the forward: the gradients of
  *     l = sum_{b,t,h} dy[b,t,h,:] . y[b,t,h,:] + <dfinal, final_state>
  * with respect to x, a, Bm, Cm, D and initial_state, for the forward that
  * ssd_forward_init computes from the same inputs.  The forward states are
@@ -312,10 +312,10 @@ ssd_status ssd_decode_step(const ssd_shape* shape, const void* x, const float* a
  * Duality", "Two algorithms for one operator", applied to the transposed
  * operator).
  *   inputs   x, Bm, Cm, dy (dtype of the shape; dy [B][T][H][P]); a [B][T][H]
- *            fp32; D [H] fp32 or NULL; initial_state [B][H][N][P] fp32 or NULL
+ *            (or [B][T][H][N] when a_per_state) fp32; D [H] fp32 or NULL; initial_state [B][H][N][P] fp32 or NULL
  *            (zero); dfinal [B][H][N][P] fp32 or NULL (no loss on the final state)
  *   outputs  dx [B][T][H][P], dBm, dCm [B][T][G][N] (dtype; dB and dC summed
- *            over the heads of each group), da [B][T][H] fp32, dD [H] fp32 or
+ *            over the heads of each group), da (a's shape) fp32, dD [H] fp32 or
  *            NULL (not wanted), dinit [B][H][N][P] fp32 or NULL (not wanted);
  *            every output is overwritten, none accumulated into
  *   workspace  device memory of ssd_backward_workspace_size(shape) bytes,
@@ -325,7 +325,9 @@ ssd_status ssd_decode_step(const ssd_shape* shape, const void* x, const float* a
  * All device pointers, 16-byte aligned; asynchronous on `stream`.  A partial
  * last chunk (T % chunk != 0) is handled as in the forward.  Arithmetic is
  * fp32 on CUDA cores.  Returns SSD_ERR_INVALID_ARG for a bad shape or
- * pointer, SSD_ERR_UNSUPPORTED for a_per_state, SSD_ERR_WORKSPACE for a
+ * pointer, SSD_ERR_UNSUPPORTED for a_per_state with N > 128 (the per-state
+ * decay is the diagonal SSM of "On Structured State-Space Duality", item (i);
+ * each state row is a scalar-decay system of its own), SSD_ERR_WORKSPACE for a
  * missing, misaligned or small workspace, SSD_ERR_CUDA if a launch fails. */
 ssd_status ssd_backward(const ssd_shape* shape, const void* x, const float* a, const void* Bm,
                         const void* Cm, const float* D, const float* initial_state, const void* dy,
@@ -333,7 +335,7 @@ ssd_status ssd_backward(const ssd_shape* shape, const void* x, const float* a, c
                         float* dinit, void* workspace, size_t ws_bytes, ssd_stream stream);
 
 /* Bytes of workspace ssd_backward needs for this shape; 0 if the shape is
- * invalid or not served (a_per_state). */
+ * invalid or not served (a_per_state with N > 128). */
 size_t ssd_backward_workspace_size(const ssd_shape* shape);
 
 #ifdef __cplusplus

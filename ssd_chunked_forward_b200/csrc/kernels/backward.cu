@@ -1,5 +1,5 @@
-// backward.cu -- gradients of the chunked SSD forward (scalar decay), on CUDA
-// cores in fp32.
+// backward.cu -- gradients of the chunked SSD forward (scalar decay; the
+// per-state decay is in backward_diag.cu), on CUDA cores in fp32.
 //
 // The loss is l = sum_t dy_t . y_t + <dfinal, h_{T-1}>.  Its adjoint state
 // g_t = dl/dh_t runs backwards through the same chunk structure as the

@@ -360,9 +360,9 @@ def backward_workspace_size(shape: Shape) -> int:
 def backward(x, a, Bm, Cm, D, dy, chunk=256, *, dfinal=None, initial_state=None, want_dD=True,
              want_dinit=True, workspace=None, stream=None):
     """Gradients of sum(dy * y) + <dfinal, final_state> for the forward of the
-    same inputs (scalar decay): returns dict dx, da, dBm, dCm, dD (or None),
-    dinit (or None).  Shapes and dtypes as for forward(); dy like x; dfinal
-    and initial_state [B,H,N,P] float32 or None.  Asynchronous on the current
+    same inputs (scalar decay, or per-state up to N = 128): returns dict dx,
+    da, dBm, dCm, dD (or None), dinit (or None).  Shapes and dtypes as for
+    forward(); dy like x; dfinal and initial_state [B,H,N,P] float32 or None.  Asynchronous on the current
     torch stream (or ``stream``)."""
     _check_inputs(x, a, Bm, Cm, D)
     if dy.shape != x.shape or dy.dtype != x.dtype or not dy.is_contiguous():
