@@ -1,5 +1,6 @@
-"""Sequence-sharded forward: one sequence split along T over the ranks of a
-process group (rank r holds tokens [r T/W, (r+1) T/W) of every batch row).
+"""Sequence-sharded forward and backward: one sequence split along T over the
+ranks of a process group (rank r holds tokens [r T/W, (r+1) T/W) of every
+batch row).
 
 Each rank runs its segment from a zero state, the ranks exchange each
 segment's final state and total log-decay in one all-gather, every rank
@@ -7,8 +8,11 @@ combines them into the state entering its own segment, and the ranks after
 the first rerun their segment from that state -- the passing of one
 summarised state between pieces, as the chunked algorithm does between chunks
 ("State Space Duality", "Two algorithms for one operator"), one level up.
-All arithmetic runs in the library's kernels (ssd.forward, ssd.decay_total,
-ssd.state_combine); this module only orders the calls and the collective.
+The backward runs the same exchange for the entering states, then the
+adjoint's exchange in the other direction (sequence_sharded_backward).  All
+arithmetic runs in the library's kernels (ssd.forward, ssd.decay_total,
+ssd.state_combine, ssd.backward); this module only orders the calls and the
+collectives.
 """
 from __future__ import annotations
 
@@ -23,11 +27,12 @@ from . import ssd
 
 @dataclass
 class SegmentOps:
-    """The three computations a rank performs; the defaults are the library's
-    (tests on machines without a GPU substitute the fp64 oracle)."""
+    """The computations a rank performs; the defaults are the library's (tests
+    on machines without a GPU substitute the fp64 oracle)."""
     forward: Callable = None        # (x, a, Bm, Cm, D, chunk, initial_state) -> (y, final)
     decay_total: Callable = None    # a -> total log-decay per chain
     state_combine: Callable = None  # (finals [W,...], totals [W,...], h0) -> h_in [W+1,...]
+    backward: Callable = None       # (x, a, Bm, Cm, D, dy, chunk, dfinal, init) -> dict of gradients
 
     def __post_init__(self):
         if self.forward is None:
@@ -37,6 +42,9 @@ class SegmentOps:
             self.decay_total = ssd.decay_total
         if self.state_combine is None:
             self.state_combine = ssd.state_combine
+        if self.backward is None:
+            self.backward = lambda x, a, Bm, Cm, D, dy, chunk, dfinal, init: ssd.backward(
+                x, a, Bm, Cm, D, dy, chunk, dfinal=dfinal, initial_state=init)
 
 
 def _all_gather(t: torch.Tensor, group) -> torch.Tensor:
@@ -50,6 +58,20 @@ def _all_gather(t: torch.Tensor, group) -> torch.Tensor:
     return out
 
 
+def _entering_states(x, a, Bm, Cm, D, chunk, group, initial_state, ops):
+    """y of the segment from zero, its total decay, and the state entering
+    every segment (h_in [W+1, ...]; h_in[W] is the sequence's final state),
+    through one all-gather of the final states and totals."""
+    y, fin = ops.forward(x, a, Bm, Cm, D, chunk, None)
+    tot = ops.decay_total(a)
+    packed = torch.cat([fin.reshape(-1), tot.reshape(-1).to(fin.dtype)])
+    gathered = _all_gather(packed, group)
+    nf = fin.numel()
+    finals = gathered[:, :nf].reshape((gathered.shape[0],) + tuple(fin.shape)).contiguous()
+    totals = gathered[:, nf:].reshape((gathered.shape[0],) + tuple(tot.shape)).contiguous()
+    return y, totals, ops.state_combine(finals, totals, initial_state)
+
+
 def sequence_sharded_forward(x, a, Bm, Cm, D, chunk, *, group=None, initial_state=None,
                              ops: SegmentOps | None = None):
     """This rank's segment of y, and the final state of the whole sequence.
@@ -60,15 +82,44 @@ def sequence_sharded_forward(x, a, Bm, Cm, D, chunk, *, group=None, initial_stat
     all-gather (of the final states and of the total decays, packed)."""
     ops = ops or SegmentOps()
     rank = dist.get_rank(group)
-    y, fin = ops.forward(x, a, Bm, Cm, D, chunk, None)
-    tot = ops.decay_total(a)
-    # one collective: final state and total decay of every segment, packed
-    packed = torch.cat([fin.reshape(-1), tot.reshape(-1).to(fin.dtype)])
-    gathered = _all_gather(packed, group)
-    nf = fin.numel()
-    finals = gathered[:, :nf].reshape((gathered.shape[0],) + tuple(fin.shape)).contiguous()
-    totals = gathered[:, nf:].reshape((gathered.shape[0],) + tuple(tot.shape)).contiguous()
-    h_in = ops.state_combine(finals, totals, initial_state)
+    y, _, h_in = _entering_states(x, a, Bm, Cm, D, chunk, group, initial_state, ops)
     if rank > 0 or initial_state is not None:
         y, _ = ops.forward(x, a, Bm, Cm, D, chunk, h_in[rank].contiguous())
     return y, h_in[-1]
+
+
+def sequence_sharded_backward(x, a, Bm, Cm, D, dy, chunk, *, group=None, initial_state=None,
+                              dfinal=None, ops: SegmentOps | None = None):
+    """Gradients of sum(dy * y) + <dfinal, final state> over the whole
+    sequence, for this rank's segment (dx, da, dBm, dCm) and for the shared
+    inputs (dD, d initial state; the same on every rank).
+
+    The state entering each segment comes from the forward's exchange.  The
+    adjoint runs the other way: the adjoint at the end of segment r is the
+    adjoint entering segment r+1, which is that segment's own contribution
+    (its backward with no loss on its end, started from its entering state)
+    plus its total decay times the adjoint at its end -- the forward's
+    combine run over the segments in reverse order, from dfinal.  So each
+    rank runs its backward once with no end loss, one all-gather exchanges
+    the entering-state adjoints (with each segment's share of dD), every rank
+    combines them, and the ranks before the last (or all, given dfinal) rerun
+    their backward with the adjoint at their end."""
+    ops = ops or SegmentOps()
+    rank = dist.get_rank(group)
+    _, totals, h_in = _entering_states(x, a, Bm, Cm, D, chunk, group, initial_state, ops)
+    init = h_in[rank].contiguous()
+    g = ops.backward(x, a, Bm, Cm, D, dy, chunk, None, init)
+    din, dD = g["dinit"], g["dD"]
+    packed = torch.cat([din.reshape(-1), dD.reshape(-1).to(din.dtype)])
+    gathered = _all_gather(packed, group)
+    world = gathered.shape[0]
+    nd = din.numel()
+    dinits = gathered[:, :nd].reshape((world,) + tuple(din.shape))
+    dD_all = gathered[:, nd:].sum(dim=0)
+    # reverse combine: adj[s] = adjoint at the end of segment W-1-s; adj[W] = d initial
+    adj = ops.state_combine(dinits.flip(0).contiguous(), totals.flip(0).contiguous(), dfinal)
+    g_end = adj[world - 1 - rank].contiguous()
+    if rank < world - 1 or dfinal is not None:
+        g = ops.backward(x, a, Bm, Cm, D, dy, chunk, g_end, init)
+    return {"dx": g["dx"], "da": g["da"], "dBm": g["dBm"], "dCm": g["dCm"],
+            "dD": dD_all.to(dD.dtype), "dinit": adj[world]}

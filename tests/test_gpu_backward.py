@@ -18,7 +18,7 @@ import torch
 from oracle import ssd_oracle as O
 from ssd_chunked_forward_b200 import ssd
 from ssd_chunked_forward_b200.workloads import generate, small_case
-from tests.gpu_helpers import rel_err, to_dev, tol_for
+from tests.gpu_helpers import TOL_BF16, rel_err, to_dev, tol_for
 
 pytestmark = pytest.mark.gpu
 
@@ -145,3 +145,42 @@ def test_backward_rejects_per_state_and_bad_workspace():
         outs[1].data_ptr(), outs[2].data_ptr(), outs[3].data_ptr(), None, None, ws.data_ptr(),
         ws.numel(), None)
     assert code == ssd.SSD_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("per_state", [False, True], ids=["scalar", "per_state"])
+def test_backward_over_segments_with_library_kernels(per_state):
+    """The sharded backward's steps on one GPU, the sequence cut into 4
+    segments: entering states by ssd_state_combine, each segment's backward
+    with no end loss, the entering-state adjoints combined in reverse order
+    from dfinal, and each segment's backward rerun with the adjoint at its
+    end -- equal to the backward of the whole sequence."""
+    if per_state:
+        w = small_case(B=2, T=1024, H=4, P=64, N=64, G=1, chunk=128, dtype="bf16", a_per_state=True, seed=105)
+    else:
+        w = small_case(B=2, T=2048, H=4, P=64, N=128, G=2, chunk=256, dtype="bf16", seed=106)
+    inp = generate(w)
+    dev = to_dev(inp)
+    dy, _, dfin = _extras(w, False, True)
+    dy, dfin = dy.cuda(), dfin.cuda()
+    full = ssd.backward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], dev["D"], dy, w.chunk, dfinal=dfin)
+    S = 4
+    Ts = w.T // S
+    seg = lambda t, s: t[:, s * Ts:(s + 1) * Ts].contiguous()
+    parts = [[seg(t, s) for t in (dev["x"], dev["a"], dev["Bm"], dev["Cm"], dy)] for s in range(S)]
+    fins = [ssd.forward(x, a, Bm, Cm, dev["D"], w.chunk)[1] for x, a, Bm, Cm, _ in parts]
+    tots = torch.stack([ssd.decay_total(p[1]) for p in parts]).contiguous()
+    h_in = ssd.state_combine(torch.stack(fins).contiguous(), tots)
+    g1 = [ssd.backward(x, a, Bm, Cm, dev["D"], g, w.chunk, initial_state=h_in[s].contiguous())
+          for s, (x, a, Bm, Cm, g) in enumerate(parts)]
+    dinits = torch.stack([g["dinit"] for g in g1])
+    adj = ssd.state_combine(dinits.flip(0).contiguous(), tots.flip(0).contiguous(), dfin)
+    g2 = [ssd.backward(x, a, Bm, Cm, dev["D"], g, w.chunk, dfinal=adj[S - 1 - s].contiguous(),
+                       initial_state=h_in[s].contiguous())
+          for s, (x, a, Bm, Cm, g) in enumerate(parts)]
+    torch.cuda.synchronize()
+    f = lambda t: t.float().cpu().numpy().astype(np.float64)
+    errs = {k: rel_err(f(torch.cat([g[k] for g in g2], dim=1)), f(full[k]))
+            for k in ("dx", "da", "dBm", "dCm")}
+    errs["dD"] = rel_err(f(sum(g["dD"] for g in g1)), f(full["dD"]))
+    errs["dinit"] = rel_err(f(adj[S]), f(full["dinit"]))
+    assert all(e <= TOL_BF16 for e in errs.values()), errs

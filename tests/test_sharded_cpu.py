@@ -61,7 +61,15 @@ def _oracle_ops():
             out.append(h)
         return torch.stack(out)
 
-    return SegmentOps(forward=forward, decay_total=decay_total, state_combine=state_combine)
+    def backward(x, a, Bm, Cm, D, dy, chunk, dfinal, init):
+        prob = O.Problem(x.numpy(), a.numpy(), Bm.numpy(), Cm.numpy(), D.numpy())
+        r = O.backward(prob, dy.numpy(), dfinal=None if dfinal is None else dfinal.numpy(),
+                       initial=None if init is None else init.numpy())
+        return {k: torch.from_numpy(np.ascontiguousarray(r[k]))
+                for k in ("dx", "da", "dBm", "dCm", "dD", "dinit")}
+
+    return SegmentOps(forward=forward, decay_total=decay_total, state_combine=state_combine,
+                      backward=backward)
 
 
 def _rank_main(rank, world, port, out_dir, per_state, with_init):
@@ -99,3 +107,55 @@ def test_two_rank_sequence_sharding(tmp_path, per_state, with_init):
     for r in range(world):  # every rank holds the whole sequence's final state
         f = np.load(tmp_path / f"f{r}.npy")
         assert np.max(np.abs(f - full["final"].reshape(B, H, N, P))) <= 1e-12 * np.max(np.abs(f))
+
+
+def _bwd_rank_main(rank, world, port, out_dir, per_state, with_init, with_dfinal):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    from ssd_chunked_forward_b200.sharded import sequence_sharded_backward
+
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    x, a, Bm, Cm, D, h0 = (torch.from_numpy(v) for v in _problem(per_state))
+    dy, dfin = (torch.from_numpy(v) for v in _bwd_extras(per_state))
+    T = x.shape[1]
+    sl = slice(rank * T // world, (rank + 1) * T // world)
+    seg = lambda t: t[:, sl].contiguous()
+    g = sequence_sharded_backward(seg(x), seg(a), seg(Bm), seg(Cm), D, seg(dy), 0, ops=_oracle_ops(),
+                                  initial_state=h0 if with_init else None,
+                                  dfinal=dfin if with_dfinal else None)
+    dist.barrier()
+    dist.destroy_process_group()
+    for k, v in g.items():
+        np.save(os.path.join(out_dir, f"{k}{rank}.npy"), v.numpy())
+
+
+def _bwd_extras(per_state):
+    rng = np.random.default_rng(211 + per_state)
+    B, T, H, P, N = 2, 24, 2, 3, 4
+    return rng.standard_normal((B, T, H, P)), rng.standard_normal((B, H, N, P))
+
+
+@pytest.mark.timeout(300)
+@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("per_state,with_init,with_dfinal",
+                         [(False, False, False), (False, True, True), (True, True, True)])
+def test_sequence_sharded_backward(tmp_path, world, per_state, with_init, with_dfinal):
+    """The sharded backward (two all-gathers: entering states forwards,
+    entering-state adjoints backwards) equals the backward of the whole
+    sequence: each rank's slice of dx, da, dB, dC, and dD and the initial
+    state's gradient on every rank."""
+    from oracle import ssd_oracle as O
+    mp.spawn(_bwd_rank_main, args=(world, _free_port(), str(tmp_path), per_state, with_init, with_dfinal),
+             nprocs=world, join=True)
+    x, a, Bm, Cm, D, h0 = _problem(per_state)
+    dy, dfin = _bwd_extras(per_state)
+    ref = O.backward(O.Problem(x, a, Bm, Cm, D), dy, dfinal=dfin if with_dfinal else None,
+                     initial=h0 if with_init else None)
+    for k in ("dx", "da", "dBm", "dCm"):
+        got = np.concatenate([np.load(tmp_path / f"{k}{r}.npy") for r in range(world)], axis=1)
+        assert np.max(np.abs(got - ref[k])) <= 1e-12 * np.max(np.abs(ref[k])), k
+    for r in range(world):
+        for k in ("dD", "dinit"):
+            got = np.load(tmp_path / f"{k}{r}.npy")
+            assert np.max(np.abs(got - ref[k])) <= 1e-12 * max(1.0, np.max(np.abs(ref[k]))), (k, r)
+
