@@ -88,3 +88,29 @@ def test_single_process_helpers():
     import bench
     assert bench.max_over_ranks(3.25) == 3.25
     assert bench.whole_job_rate(1000, 4, 2.0) == pytest.approx(2.0e6)
+
+
+def test_reference_arm_json_contract():
+    """`bench.py --impl reference` (the oracle on host cores) prints one JSON
+    line with the contract's keys, its own cpu_baseline and an e2e object
+    with no host-device traffic."""
+    import subprocess
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "tiny_f32", "--steps", "2", "--warmup", "3"],
+                         capture_output=True, text=True, timeout=240, cwd=ROOT,
+                         env={**os.environ, "WORLD_SIZE": "1", "RANK": "0"})
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for k in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+              "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+              "cpu_baseline", "e2e", "gpu_launches"):
+        assert k in d, k
+    assert d["impl"] == "reference" and d["steps"] == 2 and d["warmup"] == 3
+    assert d["value"] > 0 and d["higher_is_better"] is True
+    assert d["config"]["workload"] == "tiny_f32"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["cores"] >= 1 and d["cpu_baseline"]["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
