@@ -1,6 +1,8 @@
 /*
  * ssd.h -- C ABI of libssd: the chunked Structured State-Space Duality (SSD)
- * forward on NVIDIA B200 (sm_100a).
+ * forward on NVIDIA B200 (sm_100a), with the entry points around it (its
+ * backward, the recurrent decode step, the discretisation in front of it and
+ * the exchange step of a sequence split into segments).
  *
  * The operation (for each batch b and head h, with g = h / (H/G)):
  *
