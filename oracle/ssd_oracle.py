@@ -248,6 +248,15 @@ def discretize(dt_raw, dt_bias, A_log, x):
     return a, xd, dt
 
 
+_BACKWARD_MUTATION = 0
+
+
+def set_backward_mutation(m: int) -> None:
+    """Plant mistake number ``m`` in backward() (0 = none).  Tests only."""
+    global _BACKWARD_MUTATION
+    _BACKWARD_MUTATION = int(m)
+
+
 def backward(prob: Problem, dy, dfinal=None, initial=None):
     """Gradients of the scalar l = sum_t dy_t . y_t + <dfinal, h_{T-1}> with
     respect to every input, by reverse-mode differentiation of the step
@@ -280,7 +289,8 @@ def backward(prob: Problem, dy, dfinal=None, initial=None):
         Bt = p.Bm[:, t][:, grp]                                # [B,H,N]
         h = e * h + Bt[..., None] * p.x[:, t][:, :, None, :]
         hs[t + 1] = h
-    g = np.zeros((B, H, N, P)) if dfinal is None else _f64(dfinal).copy()
+    mut = _BACKWARD_MUTATION
+    g = np.zeros((B, H, N, P)) if (dfinal is None or mut == 1) else _f64(dfinal).copy()
     dx = np.zeros_like(p.x)
     da = np.zeros_like(p.a)
     dBh = np.zeros((B, T, H, N))
@@ -289,17 +299,17 @@ def backward(prob: Problem, dy, dfinal=None, initial=None):
     for t in range(T - 1, -1, -1):
         Ct = p.Cm[:, t][:, grp]                                # [B,H,N]
         Bt = p.Bm[:, t][:, grp]
-        g = g + Ct[..., None] * dy[:, t][:, :, None, :]        # g_t
-        dx[:, t] = np.einsum("bhnp,bhn->bhp", g, Bt) + Dv[None, :, None] * dy[:, t]
-        dBh[:, t] = np.einsum("bhnp,bhp->bhn", g, p.x[:, t])
-        dCh[:, t] = np.einsum("bhnp,bhp->bhn", hs[t + 1], dy[:, t])
+        g = g + (Bt if mut == 2 else Ct)[..., None] * dy[:, t][:, :, None, :]  # g_t
+        dx[:, t] = np.einsum("bhnp,bhn->bhp", g, Bt) + (0 if mut == 3 else Dv[None, :, None] * dy[:, t])
+        dBh[:, t] = np.einsum("bhnp,bhp->bhn", hs[t + 1] if mut == 4 else g, p.x[:, t])
+        dCh[:, t] = np.einsum("bhnp,bhp->bhn", hs[t] if mut == 5 else hs[t + 1], dy[:, t])
         e = np.exp(p.a[:, t])
         if per_state:
-            da[:, t] = np.einsum("bhnp,bhnp->bhn", g, e[..., None] * hs[t])
-            g = e[..., None] * g
+            da[:, t] = np.einsum("bhnp,bhnp->bhn", g, (1 if mut == 6 else e[..., None]) * hs[t])
+            g = (1 if mut == 7 else e[..., None]) * g
         else:
-            da[:, t] = np.einsum("bhnp,bhnp->bh", g, hs[t]) * e
-            g = e[..., None, None] * g
+            da[:, t] = np.einsum("bhnp,bhnp->bh", g, hs[t]) * (1 if mut == 6 else e)
+            g = (1 if mut == 7 else e[..., None, None]) * g
     dBm = dBh.reshape(B, T, G, hg, N).sum(axis=3)
     dCm = dCh.reshape(B, T, G, hg, N).sum(axis=3)
     dD = np.einsum("bthp,bthp->h", dy, p.x)

@@ -69,3 +69,33 @@ def test_planted_mistake_is_caught(clean_mutation, m):
     failed = _failing_pins()
     O.set_mutation(0)
     assert failed, f"mutation {m} ({MUTATIONS[m]}) passed every pin"
+
+
+BACKWARD_MUTATIONS = {
+    1: "loss on the final state dropped",
+    2: "adjoint picks up B instead of C",
+    3: "dx without the D term",
+    4: "dB from the state instead of the adjoint",
+    5: "dC from the state before the step",
+    6: "da without the decay factor",
+    7: "adjoint not decayed between steps",
+}
+
+
+@pytest.mark.parametrize("m", sorted(BACKWARD_MUTATIONS), ids=lambda m: BACKWARD_MUTATIONS[m])
+def test_backward_pins_catch_planted_mistake(m):
+    """Each planted mistake in the oracle's backward makes its finite-difference
+    pin fail (the pin differentiates the forward oracle, which the planted
+    mistake does not touch)."""
+    from tests import test_oracle_backward as bpins
+    O.set_backward_mutation(m)
+    try:
+        caught = False
+        for per_state in (False, True):
+            try:
+                bpins.test_backward_matches_finite_differences(per_state, 1, 2)
+            except AssertionError:
+                caught = True
+        assert caught, BACKWARD_MUTATIONS[m]
+    finally:
+        O.set_backward_mutation(0)
