@@ -108,7 +108,7 @@ const char* ssd_status_string(ssd_status s);
  * valid shape needs at least 256 bytes, so 0 is unambiguous. */
 size_t ssd_workspace_size(const ssd_shape* shape);
 
-/* 1 if `path` (SSD_PATH_*) serves this shape on this build, else 0. */
+/* 1 if `path` (SSD_PATH_*) serves this shape in this library, else 0. */
 int ssd_path_supported(const ssd_shape* shape, unsigned path);
 
 /* The path SSD_PATH_AUTO runs for this shape (SSD_PATH_FUSED or
