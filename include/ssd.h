@@ -327,8 +327,8 @@ ssd_status ssd_decode_step(const ssd_shape* shape, const void* x, const float* a
  * All device pointers, 16-byte aligned; asynchronous on `stream`.  A partial
  * last chunk (T % chunk != 0) is handled as in the forward.  Arithmetic is
  * fp32 on CUDA cores (the recomputed chunk states of bf16 heads with N = 128,
- * P = 64 on tensor cores, bf16 operands with fp32 accumulation).  Returns SSD_ERR_INVALID_ARG for a bad shape or
- * pointer, SSD_ERR_UNSUPPORTED for a_per_state with N > 128 (the per-state
+ * P = 64 on tensor cores, bf16 operands with fp32 accumulation).  Returns
+ * SSD_ERR_INVALID_ARG for a bad shape or pointer, SSD_ERR_UNSUPPORTED for a_per_state with N > 128 (the per-state
  * decay is the diagonal SSM of "On Structured State-Space Duality", item (i);
  * each state row is a scalar-decay system of its own), SSD_ERR_WORKSPACE for a
  * missing, misaligned or small workspace, SSD_ERR_CUDA if a launch fails. */
