@@ -113,7 +113,7 @@ def traffic_record(kernel, workload):
 # ---------------------------------------------------------------- clocks ----
 
 class ClockSampler:
-    """Samples SM clock and throttle reasons through NVML every ~10 ms."""
+    """Samples SM clock and throttle reasons through NVML every ~2 ms."""
 
     REASONS = {
         0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
@@ -138,14 +138,20 @@ class ClockSampler:
             self.err = repr(e)
         self._stop = threading.Event()
 
+    def _sample(self):
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            pass
+
     def _run(self):
+        # every ~2 ms, so that even a timed region of a few milliseconds gets
+        # several samples; one more when the region ends
         while not self._stop.is_set():
-            try:
-                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
-                self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-            except Exception:
-                pass
-            time.sleep(0.01)
+            self._sample()
+            time.sleep(0.002)
+        self._sample()
 
     def __enter__(self):
         if self.ok:
@@ -263,6 +269,21 @@ def max_over_ranks(value: float, dist=None, device="cpu") -> float:
     return float(t.item())
 
 
+def step_stats(step_ms):
+    """Median, 10th and 90th percentile and mean of the per-step device times
+    (ms); the median is the step time the metric uses."""
+    v = sorted(step_ms)
+    def pct(q):
+        if len(v) == 1:
+            return v[0]
+        pos = q * (len(v) - 1)
+        lo = int(pos)
+        hi = min(lo + 1, len(v) - 1)
+        return v[lo] + (v[hi] - v[lo]) * (pos - lo)
+    return {"median": statistics.median(v), "p10": pct(0.10), "p90": pct(0.90),
+            "mean": statistics.mean(v)}
+
+
 def whole_job_rate(tokens_per_rank: int, world: int, ms: float) -> float:
     """Tokens per second of the whole job: every rank's tokens over the
     slowest rank's time per step."""
@@ -320,7 +341,7 @@ def time_steps_split(w, dev, flush, reps, impl):
         for i, n in enumerate(names):
             times[n].append(ev[i].elapsed_time(ev[i + 1]))
     del cum_t, states, fin, y
-    return {n: statistics.mean(v) for n, v in times.items()}
+    return {n: statistics.median(v) for n, v in times.items()}
 
 
 def run_decode(args, device):
@@ -350,7 +371,7 @@ def run_decode(args, device):
         ssd.decode_step(x, a, Bm, Cm, D, state, y=y)
         e1.record(st)
     torch.cuda.synchronize()
-    ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev)
+    ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in ev)
     el = 2 if w.dtype == "bf16" else 4
     byts = (2 * w.B * w.H * w.N * w.P * 4 + 2 * w.B * w.H * w.P * el
             + w.B * w.H * (w.N if w.a_per_state else 1) * 4 + 2 * w.B * w.G * w.N * el + w.H * 4)
@@ -416,7 +437,7 @@ def run_backward(args, device):
         call()
         e1.record(st)
     torch.cuda.synchronize()
-    ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev)
+    ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in ev)
     el = 2 if w.dtype == "bf16" else 4
     tok = w.B * w.T
     byts = (2 * 2 * tok * w.H * w.P * el + 2 * tok * w.H * 4 + 2 * 2 * tok * w.G * w.N * el
@@ -467,7 +488,7 @@ def run_discretize(args, device):
         ssd.discretize(raw, bias, A_log, x, a_out=a_out, x_out=x_out)
         e1.record(st)
     torch.cuda.synchronize()
-    ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev)
+    ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in ev)
     byts = (raw.numel() * 4 + 2 * x.numel() * x.element_size() + a_out.numel() * 4
             + bias.numel() * 4 + A_log.numel() * 4)
     peaks, src = load_peaks()
@@ -581,7 +602,8 @@ def main():
     if code != ssd.SSD_OK:
         raise SystemExit(f"device status after timing: {ssd.status_string(code)}")
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    ms = max_over_ranks(sum(step_ms) / len(step_ms), dist, device)
+    stats = step_stats(step_ms)
+    ms = max_over_ranks(stats["median"], dist, device)
     value = whole_job_rate(w.tokens, world, ms)
 
     # ---- dominant kernel: per-kernel split with events --------------------
@@ -661,6 +683,9 @@ def main():
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
             "data": "synthetic",
+            "step_ms": {"median": ms, "p10": stats["p10"], "p90": stats["p90"], "mean": stats["mean"],
+                        "note": "this rank's per-step device times; ms_per_step is the median "
+                                "(the slowest rank's under torchrun)"},
             "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "P": w.P, "N": w.N,
                        "G": w.G, "chunk": w.chunk, "a_per_state": w.a_per_state,
                        "global_batch": w.B * world, "seq_len": w.T,

@@ -193,12 +193,18 @@ ssd_status ssd_forward_host(const ssd_shape* shape, const void* x_h, const float
  *  - The first call on a device looks up the array's device address (with that
  *    device current) and caches it; make that first call before any stream
  *    capture.
- *  - Every call shares the one array: calls that overlap on the GPU (other
- *    streams, other host threads) race and must be serialised by the caller.
- *    The array keeps the last call's contents; the status word and hand-off
- *    counters are cleared at the start of each call.
- *  - The device status word is not exposed; use ssd_forward with a workspace
- *    when ssd_device_status is needed. */
+ *  - Every call shares the one array.  The array keeps the last call's
+ *    contents; the status word and hand-off counters are cleared at the start
+ *    of each call.  Calls from one process on one device are ordered by the
+ *    library, whatever their streams (the clear waits for the previous call's
+ *    kernel), except while a stream is being captured into a graph: captured
+ *    calls, and calls from other processes, that overlap on the GPU race and
+ *    must be serialised by the caller.
+ *  - The device status word is not exposed.  If a bounded hand-off wait inside
+ *    the kernel runs out (2 s; it does not on a healthy GPU), the call has
+ *    already returned SSD_OK and y and the final state are left incomplete;
+ *    use ssd_forward with a workspace and ssd_device_status when that
+ *    condition must be observed. */
 ssd_status ssd_forward_noalloc(const ssd_shape* shape, const void* x, const float* a,
                                const void* Bm, const void* Cm, const float* D, void* y,
                                float* final_state, ssd_stream stream);

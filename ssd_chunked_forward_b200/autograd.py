@@ -2,11 +2,11 @@
 takes part in a torch graph, and its backward is the library's ssd_backward
 (the gradients of sum(dy * y) + <dfinal, final> that autograd asks for).
 
-The forward keeps only its inputs for the backward; the states are
-recomputed there (llms.blog "State Space Models and Mamba ...",
-"Hardware-Aware Parallel Associative Scan": intermediate states are
-recomputed during the backward pass rather than saved).  All arithmetic runs
-in the library's kernels; this module only passes tensors.
+The forward keeps only its inputs for the backward, which rebuilds the chunk
+states from them instead of storing them during the forward (the memory
+trade named on llms.blog "State Space Models and Mamba ...", section
+"Hardware-Aware Parallel Associative Scan").  All arithmetic runs in the
+library's kernels; this module only passes tensors.
 """
 from __future__ import annotations
 

@@ -101,10 +101,13 @@ cudaError_t launch_fused_tc(const Dims& d, const void* x, const float* a, const 
 // launch_fused_tc ordered after the previous fused launch on this device, on
 // whatever stream that was: the persistent kernel's blocks wait on one
 // another, which needs all of them resident, so two such kernels must not
-// share the GPU.  Skipped while `st` is being captured into a graph.
+// share the GPU.  Skipped while `st` is being captured into a graph.  When
+// `clear` is given, its first `clear_bytes` bytes are zeroed on `st` after
+// that wait and before the launch (scratch shared by successive launches).
 cudaError_t launch_fused_ordered(const Dims& d, const void* x, const float* a, const void* Bm,
                                  const void* Cm, const float* D, void* y, float* fin, float* ring,
                                  unsigned* flags, int* status, bool test_stall, cudaStream_t st,
-                                 const float* init = nullptr);
+                                 const float* init = nullptr, void* clear = nullptr,
+                                 size_t clear_bytes = 0);
 
 }  // namespace ssd

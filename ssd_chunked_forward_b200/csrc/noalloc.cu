@@ -77,9 +77,11 @@ extern "C" ssd_status ssd_forward_noalloc(const ssd_shape* shape, const void* x,
     d.bf16 = shape->dtype == SSD_DTYPE_BF16;
 
     cudaStream_t cs = (cudaStream_t)stream;
-    // the status word and the per-chain counters start at zero on every call
-    if (cudaMemsetAsync(p, 0, kCtrl + kFlags, cs) != cudaSuccess) return SSD_ERR_CUDA;
-    const cudaError_t e =
-        ssd::launch_fused_ordered(d, x, a, Bm, Cm, D, y, final_state, ring, flags, ctrl, false, cs);
+    // The status word and the per-chain counters start at zero on every call.
+    // The clear is queued inside the library's ordering of fused launches, so
+    // it cannot overtake a previous call's kernel that still reads them, even
+    // from another stream of this device.
+    const cudaError_t e = ssd::launch_fused_ordered(d, x, a, Bm, Cm, D, y, final_state, ring, flags,
+                                                    ctrl, false, cs, nullptr, p, kCtrl + kFlags);
     return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }

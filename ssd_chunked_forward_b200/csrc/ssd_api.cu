@@ -22,6 +22,12 @@ inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
+// The CUDA-core step kernels and the backward put the (batch, head) chain index
+// in gridDim.y, which holds at most 65535; larger batches are served by the
+// fused kernel alone (its grid is one-dimensional).
+constexpr long long kMaxGridY = 65535;
+bool chains_fit_grid_y(const ssd_shape* s) { return (long long)s->B * s->H <= kMaxGridY; }
+
 ssd_status check_shape(const ssd_shape* s) {
     if (!s) return SSD_ERR_INVALID_ARG;
     if (s->B < 1 || s->T < 1 || s->H < 1 || s->P < 1 || s->G < 1 || s->N < 1 || s->chunk < 1)
@@ -163,13 +169,18 @@ namespace ssd {
 cudaError_t launch_fused_ordered(const Dims& d, const void* x, const float* a, const void* Bm,
                                  const void* Cm, const float* D, void* y, float* fin, float* ring,
                                  unsigned* flags, int* status, bool test_stall, cudaStream_t st,
-                                 const float* init) {
+                                 const float* init, void* clear, size_t clear_bytes) {
     cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
     if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) return cudaErrorInvalidValue;
     int dev = 0;
     if (cap != cudaStreamCaptureStatusNone || cudaGetDevice(&dev) != cudaSuccess || dev < 0 ||
-        dev >= kMaxDevices)
+        dev >= kMaxDevices) {
+        if (clear) {
+            cudaError_t e = cudaMemsetAsync(clear, 0, clear_bytes, st);
+            if (e != cudaSuccess) return e;
+        }
         return launch_fused_tc(d, x, a, Bm, Cm, D, y, fin, ring, flags, status, test_stall, st, init);
+    }
     std::lock_guard<std::mutex> lock(g_fused_mu);
     if (!g_fused_done[dev]) {
         cudaError_t e = cudaEventCreateWithFlags(&g_fused_done[dev], cudaEventDisableTiming);
@@ -177,6 +188,10 @@ cudaError_t launch_fused_ordered(const Dims& d, const void* x, const float* a, c
     }
     if (g_fused_seen[dev]) {
         cudaError_t e = cudaStreamWaitEvent(st, g_fused_done[dev], 0);
+        if (e != cudaSuccess) return e;
+    }
+    if (clear) {  // after the wait: the previous launch may still read this memory
+        cudaError_t e = cudaMemsetAsync(clear, 0, clear_bytes, st);
         if (e != cudaSuccess) return e;
     }
     cudaError_t e = launch_fused_tc(d, x, a, Bm, Cm, D, y, fin, ring, flags, status, test_stall, st, init);
@@ -211,10 +226,11 @@ int ssd_path_supported(const ssd_shape* shape, unsigned path) {
     if (!shape) return 0;
     if (check_shape(shape) != SSD_OK) return 0;
     const Dims d = dims_of(shape);
+    const int fits = chains_fit_grid_y(shape) ? 1 : 0;
     switch (path) {
-        case SSD_PATH_AUTO: return 1;
-        case SSD_PATH_SIMT: return 1;
-        case SSD_PATH_MODULAR: return 1;
+        case SSD_PATH_AUTO: return (fits || ssd::fused_supported(d)) ? 1 : 0;
+        case SSD_PATH_SIMT: return fits;
+        case SSD_PATH_MODULAR: return fits;
         case SSD_PATH_FUSED: return ssd::fused_supported(d) ? 1 : 0;
         default: return 0;
     }
@@ -228,7 +244,8 @@ int ssd_auto_path(const ssd_shape* shape) {
     // B200) times the chain length exceeds the modular path's cost (~53 ns per
     // head-block, i.e. chains x 53 ns per block)
     constexpr long long kFusedMinChains = 76;
-    if (ssd::fused_supported(d) && (long long)d.B * d.H >= kFusedMinChains) return SSD_PATH_FUSED;
+    if (ssd::fused_supported(d) && ((long long)d.B * d.H >= kFusedMinChains || !chains_fit_grid_y(shape)))
+        return SSD_PATH_FUSED;
     return SSD_PATH_MODULAR;
 }
 
@@ -250,12 +267,13 @@ ssd_status ssd_forward_init(const ssd_shape* shape, const void* x, const float* 
     if (!workspace || ((uintptr_t)workspace % kAlign) != 0) return SSD_ERR_WORKSPACE;
     if (ws_bytes < ssd_workspace_size(shape)) return SSD_ERR_WORKSPACE;
     if (!ssd_path_supported(shape, path)) return SSD_ERR_UNSUPPORTED;
+    if (path == SSD_PATH_AUTO) path = (unsigned)ssd_auto_path(shape);
+    if (!ssd_path_supported(shape, path)) return SSD_ERR_UNSUPPORTED;
     cudaStream_t cs = (cudaStream_t)stream;
     const Workspace w = carve(workspace, d);
     // status word and per-chain counters start at zero on every call
     if (cudaMemsetAsync(w.ctrl, 0, kCtrlBytes + flags_bytes(d), cs) != cudaSuccess)
         return SSD_ERR_CUDA;
-    if (path == SSD_PATH_AUTO) path = (unsigned)ssd_auto_path(shape);
     switch (path) {
         case SSD_PATH_SIMT:
             return run_modular(d, x, a, Bm, Cm, D, y, final_state, w, cs, false, initial_state);
@@ -367,6 +385,7 @@ ssd_status ssd_device_status(const void* workspace, ssd_stream stream) {
 ssd_status ssd_chunk_cumsum(const ssd_shape* shape, const float* a, float* cum, ssd_stream stream) {
     ssd_status st = check_shape(shape);
     if (st != SSD_OK) return st;
+    if (!chains_fit_grid_y(shape)) return SSD_ERR_UNSUPPORTED;
     if (!a || !cum || !aligned16(a) || !aligned16(cum)) return SSD_ERR_INVALID_ARG;
     return cuda_status(ssd::launch_chunk_cumsum(dims_of(shape), a, cum, (cudaStream_t)stream));
 }
@@ -375,6 +394,7 @@ ssd_status ssd_chunk_state(const ssd_shape* shape, const void* x, const void* Bm
                            float* states, ssd_stream stream, unsigned impl) {
     ssd_status st = check_shape(shape);
     if (st != SSD_OK) return st;
+    if (!chains_fit_grid_y(shape)) return SSD_ERR_UNSUPPORTED;
     if (!x || !Bm || !cum || !states) return SSD_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(Bm) || !aligned16(cum) || !aligned16(states))
         return SSD_ERR_INVALID_ARG;
@@ -392,6 +412,7 @@ ssd_status ssd_state_pass(const ssd_shape* shape, const float* cum, float* state
                           float* final_state, ssd_stream stream) {
     ssd_status st = check_shape(shape);
     if (st != SSD_OK) return st;
+    if (!chains_fit_grid_y(shape)) return SSD_ERR_UNSUPPORTED;
     if (!cum || !states || !aligned16(cum) || !aligned16(states) ||
         (final_state && !aligned16(final_state)))
         return SSD_ERR_INVALID_ARG;
@@ -405,6 +426,7 @@ static ssd_status scan_common(const ssd_shape* shape, const void* x, const void*
     ssd_status st = check_shape(shape);
     if (st != SSD_OK) return st;
     if ((shape->a_per_state != 0) != want_diag) return SSD_ERR_INVALID_ARG;
+    if (!chains_fit_grid_y(shape)) return SSD_ERR_UNSUPPORTED;
     if (!x || !Bm || !Cm || !cum || !Hin || !y) return SSD_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(Bm) || !aligned16(Cm) || !aligned16(cum) || !aligned16(Hin) ||
         !aligned16(y) || (D && !aligned16(D)))
@@ -478,6 +500,7 @@ ssd_status ssd_backward(const ssd_shape* shape, const void* x, const float* a, c
     ssd_status st = check_shape(shape);
     if (st != SSD_OK) return st;
     if (shape->a_per_state && !ssd::backward_diag_supported(dims_of(shape))) return SSD_ERR_UNSUPPORTED;
+    if (!chains_fit_grid_y(shape)) return SSD_ERR_UNSUPPORTED;
     if (!x || !a || !Bm || !Cm || !dy || !dx || !da || !dBm || !dCm) return SSD_ERR_INVALID_ARG;
     const void* ptrs[] = {x, a, Bm, Cm, D, initial_state, dy, dfinal, dx, da, dBm, dCm, dD, dinit};
     for (const void* p : ptrs)
@@ -495,6 +518,7 @@ ssd_status ssd_backward(const ssd_shape* shape, const void* x, const float* a, c
 size_t ssd_backward_workspace_size(const ssd_shape* shape) {
     if (check_shape(shape) != SSD_OK) return 0;
     if (shape->a_per_state && !ssd::backward_diag_supported(dims_of(shape))) return 0;
+    if (!chains_fit_grid_y(shape)) return 0;
     return backward_layout(dims_of(shape), nullptr, nullptr);
 }
 

@@ -75,3 +75,49 @@ def parity_on_chains(inp, y, fin, chains, t_end=None):
         fr = np.concatenate([r[1][None] for r in refs])
         ef = rel_err(fs, fr)
     return ey, ef
+
+
+def whole_tensor_parity(inp, y, fin, nthreads=None, budget_bytes=3 << 30):
+    """||y - y_ref||_inf / ||y_ref||_inf over the WHOLE output tensor, and the
+    same metric over the whole final state, against O1 (fp64 recurrence).
+
+    The oracle runs on batches of consecutive B/C groups of one batch row (a
+    group's heads share Bm/Cm, so a sub-problem of whole groups keeps the
+    head-to-group map), and the comparison streams chain by chain, so neither
+    the fp64 y nor the fp64 inputs are ever held whole.  Returns
+    (y_err, final_err, max|y_ref|)."""
+    import os
+    x, a, Bm, Cm, D = inp["x"], inp["a"], inp["Bm"], inp["Cm"], inp["D"]
+    B, T, H, P = x.shape
+    G, N = Bm.shape[2], Bm.shape[3]
+    HG = H // G
+    nthreads = nthreads or (os.cpu_count() or 1)
+    # fp64 bytes one chain costs: x and y, its share of B/C and a
+    per_chain = 8 * T * (2 * P + 2 * N / HG + (N if a.dim() == 4 else 1))
+    groups_per_batch = max(1, min(G, max(1, nthreads // HG), int(budget_bytes // (per_chain * HG))))
+    f = lambda t: t.to(torch.float64).numpy()
+    dmax = rmax = fdmax = frmax = 0.0
+    yc = y.cpu() if y.is_cuda else y
+    fc = (fin.cpu() if fin.is_cuda else fin) if fin is not None else None
+    for b in range(B):
+        for g0 in range(0, G, groups_per_batch):
+            g1 = min(G, g0 + groups_per_batch)
+            h0, h1 = g0 * HG, g1 * HG
+            prob = O.Problem(f(x[b:b + 1, :, h0:h1].contiguous()), f(a[b:b + 1, :, h0:h1].contiguous()),
+                             f(Bm[b:b + 1, :, g0:g1].contiguous()), f(Cm[b:b + 1, :, g0:g1].contiguous()),
+                             f(D[h0:h1].contiguous()))
+            r = O.recurrence(prob, nthreads=nthreads)
+            del prob
+            for c in range(h1 - h0):
+                ref = r["y"][c]
+                got = yc[b, :, h0 + c, :].to(torch.float64).numpy()
+                dmax = max(dmax, float(np.max(np.abs(got - ref))))
+                rmax = max(rmax, float(np.max(np.abs(ref))))
+                if fc is not None:
+                    fr = r["final"][c]
+                    fdmax = max(fdmax, float(np.max(np.abs(fc[b, h0 + c].numpy().astype(np.float64) - fr))))
+                    frmax = max(frmax, float(np.max(np.abs(fr))))
+            del r
+    ey = dmax / (rmax if rmax > 0 else 1.0)
+    ef = None if fc is None else fdmax / (frmax if frmax > 0 else 1.0)
+    return ey, ef, rmax

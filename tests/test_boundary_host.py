@@ -199,3 +199,30 @@ def test_decode_step_validates(lib):
     assert call(good, x=None) == ssd.SSD_ERR_INVALID_ARG
     assert call(good, st=None) == ssd.SSD_ERR_INVALID_ARG
     assert call(good, y=ctypes.c_void_p((1 << 20) + 4)) == ssd.SSD_ERR_INVALID_ARG  # misaligned
+
+
+def test_chain_count_beyond_grid_y_refused_before_launch(lib):
+    """The CUDA-core steps and the backward index (batch, head) chains along
+    gridDim.y (at most 65535).  A batch with more chains is refused with
+    SSD_ERR_UNSUPPORTED before anything is queued; the fused kernel (a flat
+    grid) still serves it, so AUTO picks it."""
+    big = ssd.make_shape(1024, 256, 80, 64, 1, 128, 256)        # 81920 chains
+    assert ssd.path_supported(big, ssd.PATH_FUSED)
+    assert not ssd.path_supported(big, ssd.PATH_MODULAR)
+    assert not ssd.path_supported(big, ssd.PATH_SIMT)
+    assert ssd.auto_path(big) == ssd.PATH_FUSED
+    assert ssd.backward_workspace_size(big) == 0
+    ok = 1 << 20
+    ws = ssd.workspace_size(big)
+    g = lambda path: lib.ssd_forward_path(ctypes.byref(big), ok, ok, ok, ok, None, ok, None,
+                                          ok, ws, None, path, 0)
+    assert g(ssd.PATH_MODULAR) == ssd.SSD_ERR_UNSUPPORTED
+    assert g(ssd.PATH_SIMT) == ssd.SSD_ERR_UNSUPPORTED
+    args = [ok, ok, ok, ok, None, None, ok, None, ok, ok, ok, ok, None, None, ok, 1 << 40, None]
+    assert lib.ssd_backward(ctypes.byref(big), *args) == ssd.SSD_ERR_UNSUPPORTED
+    assert lib.ssd_chunk_cumsum(ctypes.byref(big), ok, ok, None) == ssd.SSD_ERR_UNSUPPORTED
+    assert lib.ssd_state_pass(ctypes.byref(big), ok, ok, None, None) == ssd.SSD_ERR_UNSUPPORTED
+    assert lib.ssd_chunk_scan(ctypes.byref(big), ok, ok, ok, ok, ok, None, ok, None, 0) == \
+        ssd.SSD_ERR_UNSUPPORTED
+    f32 = ssd.make_shape(1024, 256, 80, 64, 1, 128, 256, dtype="f32")  # no fused kernel for fp32
+    assert not ssd.path_supported(f32, ssd.PATH_AUTO)
