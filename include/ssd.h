@@ -84,12 +84,18 @@ enum {
     SSD_PATH_MODULAR = 1, /* chunk_cumsum -> chunk_state -> state_pass -> chunk_scan
                              (or diag_scan), each a separate kernel, states in HBM */
     SSD_PATH_SIMT = 2,    /* the same four steps on CUDA cores only (fp32 math)  */
-    SSD_PATH_FUSED = 3    /* one persistent kernel: chunk states, inter-chunk pass
+    SSD_PATH_FUSED = 3,   /* one persistent kernel: chunk states, inter-chunk pass
                              and outputs fused; states never leave L2.  Its blocks
                              wait on one another, so the library orders every fused
                              launch on a device after the previous one, whatever
                              the stream (copies and other kernels still overlap);
                              not while the stream is being captured into a graph */
+    SSD_PATH_SPLIT = 4    /* few long sequences: each is cut into S pieces; the
+                             state every piece builds from zero (tensor cores, no
+                             outputs), the combine of those states into the state
+                             entering every piece, then the fused kernel over all
+                             pieces at once, each from its entering state.  Same
+                             shapes as SSD_PATH_FUSED, T long enough to split */
 };
 
 /* Implementations for the per-step entry points. */
@@ -99,6 +105,16 @@ enum { SSD_IMPL_AUTO = 0, SSD_IMPL_SIMT = 1, SSD_IMPL_TC = 2 };
  * is never published, so the bounded wait behind it must run out and report
  * SSD_ERR_TIMEOUT through ssd_device_status().  Never set it otherwise. */
 #define SSD_FLAG_TEST_STALL 0x100u
+
+/* Test hook, not for production use: the next `count` calls of any entry
+ * point that queues GPU work (the forwards, the steps, the backward, the
+ * decode step, the segment calls) return SSD_ERR_CUDA after their argument
+ * checks, queueing nothing -- as a failed launch would -- so that callers'
+ * error handling can be tested without a real CUDA failure.  Process-wide;
+ * count <= 0 clears it.  ssd_test_pending_failures() returns how many are
+ * left.  No counterpart on the pages. */
+void ssd_test_fail_calls(int count);
+int ssd_test_pending_failures(void);
 
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* ssd_status_string(ssd_status s);
@@ -111,16 +127,16 @@ size_t ssd_workspace_size(const ssd_shape* shape);
 /* 1 if `path` (SSD_PATH_*) serves this shape in this library, else 0. */
 int ssd_path_supported(const ssd_shape* shape, unsigned path);
 
-/* The path SSD_PATH_AUTO runs for this shape (SSD_PATH_FUSED or
- * SSD_PATH_MODULAR), or -1 for an invalid shape.  The fused kernel hands each
- * (batch, head) chain's state from one 128-token block to the next, so its
- * time is bounded below by the chain length times that hand-off (about 4 us
- * per block measured on B200); the modular path pays about 2.6x the fused
- * path's memory traffic but runs all blocks of a chain at once.  With fewer
- * than 76 chains (batch x heads) the chain bound exceeds the modular path's
- * cost at any sequence length, so AUTO takes the modular path there.  This
- * choice has no counterpart on the pages; it only picks between two exact
- * evaluations of the same forward. */
+/* The path SSD_PATH_AUTO runs for this shape (SSD_PATH_FUSED, SSD_PATH_SPLIT
+ * or SSD_PATH_MODULAR), or -1 for an invalid shape.  The fused kernel hands
+ * each (batch, head) chain's state from one 128-token block to the next, so
+ * its time is bounded below by the chain length times that hand-off; with at
+ * least 76 chains (batch x heads) the chains are short enough for the work to
+ * hide it and AUTO runs the fused kernel.  With fewer, long chains AUTO cuts
+ * every sequence into pieces (SSD_PATH_SPLIT) when T allows it (pieces of at
+ * least 4096 tokens, T divisible by the piece count), else it runs the
+ * modular path, which has no chain.  This choice has no counterpart on the
+ * pages; it only picks between exact evaluations of the same forward. */
 int ssd_auto_path(const ssd_shape* shape);
 
 /* The whole forward: y (and final_state when non-NULL) from x, a, Bm, Cm, D.
@@ -290,6 +306,25 @@ ssd_status ssd_discretize(const ssd_shape* shape, const float* dt_raw, const flo
 ssd_status ssd_decay_total(const ssd_shape* shape, const float* a, float* total, ssd_stream stream);
 ssd_status ssd_state_combine(const ssd_shape* shape, int segments, const float* finals,
                              const float* totals, const float* h0, float* h_in, ssd_stream stream);
+
+/* ssd_segment_state: the state a segment builds from a zero start and its
+ * total log-decay, without its outputs -- what the exchange needs from each
+ * segment before any of them runs its forward:
+ *     final_state[b][h][n][p] = sum_t B_t[n] exp(sum_{u=t+1..T-1} a_u) x_t[p]
+ *     total[b][h]             = sum_t a_t          (per n when a_per_state)
+ * i.e. the final state of ssd_forward on the segment and ssd_decay_total's
+ * result, at the cost of reading x, a and Bm once (no Cm, no y).  The Mamba-2
+ * head shapes (bf16, N = 128, P = 64, scalar decay) run one tensor-core pass
+ * (the per-block products B^T (w o X), w_t = exp(sum_{u>t} a_u), accumulated
+ * in TMEM); other shapes run the first three steps of the modular path.
+ * workspace: as for ssd_forward (ssd_workspace_size bytes, 256-byte aligned;
+ * its status word reports a bounded wait that ran out).  final_state and
+ * total are fp32 device pointers, 16-byte aligned; asynchronous on `stream`;
+ * SSD_ERR_INVALID_ARG / SSD_ERR_WORKSPACE / SSD_ERR_UNSUPPORTED before any
+ * work is queued, SSD_ERR_CUDA if a launch fails. */
+ssd_status ssd_segment_state(const ssd_shape* shape, const void* x, const float* a, const void* Bm,
+                             float* final_state, float* total, void* workspace, size_t ws_bytes,
+                             ssd_stream stream);
 
 /* One recurrent step for a batch of single tokens -- the inference (decode)
  * form of the same operator: per (batch b, head h),

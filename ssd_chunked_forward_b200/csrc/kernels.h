@@ -6,6 +6,10 @@
 
 namespace ssd {
 
+// The test hook of ssd_test_fail_calls: true (once per pending count) when the
+// calling entry point must return SSD_ERR_CUDA without queueing work.
+bool take_injected_failure();
+
 struct Dims {
     int B, T, H, P, G, N, Q, nc;
     bool diag;  // per-state log-decay a[B,T,H,N]
@@ -93,10 +97,37 @@ cudaError_t launch_chunk_scan_tc(const Dims& d, const void* x, const void* Bm, c
 // L2-resident ring with bounded waits) and the outputs; 128-token blocks
 bool fused_supported(const Dims& d);
 size_t fused_ring_bytes(const Dims& d);
+// seg > 1: the B rows of d are pieces of B / seg longer sequences (row b is
+// piece b % seg of sequence b / seg); piece k of sequence b starts from
+// init[(k * (B / seg) + b)] and the last piece writes the final state fin[b].
 cudaError_t launch_fused_tc(const Dims& d, const void* x, const float* a, const void* Bm,
                             const void* Cm, const float* D, void* y, float* fin, float* ring,
                             unsigned* flags, int* status, bool test_stall, cudaStream_t st,
-                            const float* init = nullptr);
+                            const float* init = nullptr, int seg = 1);
+
+// The state each piece of a sequence builds from a zero start and the piece's
+// total log-decay: the [B][T] rows viewed as [B*S][T/S] pieces (T % S == 0);
+// fin is [S][B][H][N][P], tot [S][B][H] (bf16, N = 128, P = 64, scalar decay)
+bool segment_state_tc_supported(const Dims& d);
+cudaError_t launch_segment_state_tc(const Dims& d, int S, const void* x, const float* a, const void* Bm,
+                                    float* fin, float* tot, int* status, cudaStream_t st);
+
+// Block states of the per-state decay (bf16, N = 64, P = 64) on tensor cores:
+// states[b][h][j] = sum_s B_s o exp(c_127 - c_s) x_s^T over 128-token block j
+// ([B][H][nblk][N][P]) and the block totals tot[b][h][j][n] = c_127[n]
+bool diag_state_tc_supported(const Dims& d);
+cudaError_t launch_diag_state_tc(const Dims& d, const void* x, const float* a, const void* Bm,
+                                 float* states, float* tot, int* status, cudaStream_t st);
+
+// Output of the per-state decay (bf16, N = 64, P = 64) on tensor cores, one CTA
+// per (b, h, 128-token block): Hin [B][H][nblk][N][P] is the state entering
+// each block (32-token sub-blocks inside; see diag_scan_tc.cu)
+bool diag_scan_tc_supported(const Dims& d);
+// decay: the log-decays a [B][T][H][N], or (from_cum, 128-token chunks only)
+// the step-1 prefix sums cum [B][H][nc][128][N]
+cudaError_t launch_diag_scan_tc(const Dims& d, const void* x, const float* decay, bool from_cum, const void* Bm,
+                                const void* Cm, const float* Hin, const float* D, void* y, int* status,
+                                cudaStream_t st);
 
 // launch_fused_tc ordered after the previous fused launch on this device, on
 // whatever stream that was: the persistent kernel's blocks wait on one
@@ -108,6 +139,6 @@ cudaError_t launch_fused_ordered(const Dims& d, const void* x, const float* a, c
                                  const void* Cm, const float* D, void* y, float* fin, float* ring,
                                  unsigned* flags, int* status, bool test_stall, cudaStream_t st,
                                  const float* init = nullptr, void* clear = nullptr,
-                                 size_t clear_bytes = 0);
+                                 size_t clear_bytes = 0, int seg = 1);
 
 }  // namespace ssd

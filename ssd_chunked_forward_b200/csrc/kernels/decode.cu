@@ -35,26 +35,37 @@ __global__ void __launch_bounds__(kDecThreads) decode_step_kernel(
         sE[n] = expf(DIAG ? ab[n] : ab[0]);
     }
     for (int p = tid; p < P; p += kDecThreads) sX[p] = to_f32(x[(size_t)bh * P + p]);
-    __syncthreads();
     // column p = tid % pw (pw = min(P, threads) lanes per row), rows n = slice,
     // slice + ns, ...; each thread loads a batch of its rows before updating any,
     // so a block has its whole state in flight at once (one memory latency, not
-    // one per row)
+    // one per row).  The first batch is issued before the barrier on the
+    // per-token vectors, so both memory latencies overlap.
     constexpr int kRows = 16;
     const int pw = P < kDecThreads ? P : kDecThreads;
     const int ns = kDecThreads / pw;  // row slices
     float* hs = state + (size_t)bh * N * P;
+    float hv[kRows];
+    {
+        const int p = tid % pw, sl = tid / pw;
+#pragma unroll
+        for (int r = 0; r < kRows; ++r) {
+            const int n = sl + r * ns;
+            hv[r] = (sl < ns && p < P && n < N) ? hs[(size_t)n * P + p] : 0.f;
+        }
+    }
+    __syncthreads();
     for (int p0 = 0; p0 < P; p0 += pw) {
         const int p = p0 + tid % pw, sl = tid / pw;
         float acc = 0.f;
         if (sl < ns && p < P) {
             const float xp = sX[p];
             for (int n0 = sl; n0 < N; n0 += kRows * ns) {
-                float hv[kRows];
+                if (p0 > 0 || n0 > sl) {  // later batches load here
 #pragma unroll
-                for (int r = 0; r < kRows; ++r) {
-                    const int n = n0 + r * ns;
-                    hv[r] = n < N ? hs[(size_t)n * P + p] : 0.f;
+                    for (int r = 0; r < kRows; ++r) {
+                        const int n = n0 + r * ns;
+                        hv[r] = n < N ? hs[(size_t)n * P + p] : 0.f;
+                    }
                 }
 #pragma unroll
                 for (int r = 0; r < kRows; ++r) {

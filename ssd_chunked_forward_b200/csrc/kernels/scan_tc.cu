@@ -886,25 +886,4 @@ cudaError_t launch_chunk_scan_tc(const Dims& d, const void* x, const void* Bm, c
     return launch<kScan>(d, x, Bm, Cm, y, Hin, (uint64_t)d.B * d.H * d.nc * kN, p, st);
 }
 
-bool fused_supported(const Dims& d) {
-    return d.bf16 && !d.diag && d.N == kN && d.P == kP && d.Q % kBlk == 0;
-}
-
-size_t fused_ring_bytes(const Dims& d) { return (size_t)d.B * d.H * 2 * kN * kP * sizeof(float); }
-
-cudaError_t launch_fused_tc(const Dims& d, const void* x, const float* a, const void* Bm,
-                            const void* Cm, const float* D, void* y, float* fin, float* ring,
-                            unsigned* flags, int* status, bool test_stall, cudaStream_t st,
-                            const float* init) {
-    if (!fused_supported(d)) return cudaErrorNotSupported;
-    ScanParams p = {};
-    p.a = a;
-    p.D = D;
-    p.flags = flags;
-    p.fin = fin;
-    p.status = status;
-    p.test_stall = test_stall ? 1 : 0;
-    return launch<kFused>(d, x, Bm, Cm, y, ring, (uint64_t)d.B * d.H * 2 * kN, p, st, init);
-}
-
 }  // namespace ssd

@@ -62,6 +62,7 @@ extern "C" ssd_status ssd_forward_noalloc(const ssd_shape* shape, const void* x,
     if (!ssd_path_supported(shape, SSD_PATH_FUSED)) return SSD_ERR_UNSUPPORTED;
     if ((long long)shape->B * shape->H > kMaxChains) return SSD_ERR_WORKSPACE;
 
+    if (ssd::take_injected_failure()) return SSD_ERR_CUDA;
     void* base = nullptr;
     ssd_status st = scratch_address(&base);
     if (st != SSD_OK) return st;

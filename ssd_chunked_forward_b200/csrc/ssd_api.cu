@@ -3,6 +3,7 @@
 // stream.  No allocation happens here; every buffer belongs to the caller.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <mutex>
 #include <stdint.h>
 #include <string.h>
@@ -82,12 +83,88 @@ struct Workspace {
     float* states;    // modular path
 };
 
+// Pieces per sequence of the split path: the largest power of two S with
+// T % S == 0, pieces of at least 4096 tokens and at most 1024 chains over all
+// pieces (so that the fused kernel's two-slot ring stays in L2); 1 when the
+// shape is not split.
+constexpr int kSplitMinPiece = 4096;
+constexpr long long kSplitMaxChains = 1024;
+int split_pieces(const Dims& d) {
+    if (!ssd::fused_supported(d) || !ssd::segment_state_tc_supported(d)) return 1;
+    const long long chains = (long long)d.B * d.H;
+    int S = 1;
+    while (S < 1024 && d.T % (2 * S) == 0 && d.T / (2 * S) >= kSplitMinPiece &&
+           chains * 2 * S <= kSplitMaxChains)
+        S *= 2;
+    return S;
+}
+Dims pieces_dims(const Dims& d, int S) {
+    Dims v = d;
+    v.B = d.B * S;
+    v.T = d.T / S;
+    v.nc = (v.T + d.Q - 1) / d.Q;
+    return v;
+}
+
+// Split path scratch, after the status word: per-piece counters and ring for
+// the fused kernel over all pieces, the pieces' own states [S][B][H][N][P],
+// their total log-decays [S][B][H], and the entering states [S+1][B][H][N][P].
+struct SplitWorkspace {
+    unsigned* flags;
+    float* ring;
+    float* fin;
+    float* tot;
+    float* h_in;
+};
+size_t split_bytes(const Dims& d, int S, void* ws, SplitWorkspace* w) {
+    const Dims v = pieces_dims(d, S);
+    const size_t chain_state = (size_t)d.N * d.P * sizeof(float);
+    const size_t bh = (size_t)d.B * d.H;
+    const size_t sizes[5] = {flags_bytes(v), ssd::fused_ring_bytes(v), S * bh * chain_state,
+                             S * bh * sizeof(float), (S + 1) * bh * chain_state};
+    size_t off = kCtrlBytes;
+    void** slots[5] = {};
+    if (w) {
+        void** s_[5] = {(void**)&w->flags, (void**)&w->ring, (void**)&w->fin, (void**)&w->tot,
+                        (void**)&w->h_in};
+        for (int i = 0; i < 5; ++i) slots[i] = s_[i];
+    }
+    for (int i = 0; i < 5; ++i) {
+        if (ws && slots[i]) *slots[i] = (char*)ws + off;
+        off += round_up(sizes[i], kAlign);
+    }
+    return off;
+}
+
+// Per-state tensor-core steps (bf16, N = 64, P = 64): after the status word,
+// the 128-token block states [B][H][nblk][N][P] (the state entering each block
+// once the pass has run) and the block totals [B][H][nblk][N].
+struct DiagWorkspace {
+    float* states;
+    float* tot;
+};
+size_t diag_tc_bytes(const Dims& d, void* ws, DiagWorkspace* w) {
+    const size_t nblk = (d.T + 127) / 128;
+    const size_t st = round_up((size_t)d.B * d.H * nblk * d.N * d.P * sizeof(float), kAlign);
+    const size_t tot = round_up((size_t)d.B * d.H * nblk * d.N * sizeof(float), kAlign);
+    if (ws && w) {
+        w->states = (float*)((char*)ws + kCtrlBytes);
+        w->tot = (float*)((char*)ws + kCtrlBytes + st);
+    }
+    return kCtrlBytes + st + tot;
+}
+
 size_t workspace_bytes(const Dims& d) {
     const Dims m = modular_dims(d);
     const size_t cum = round_up(cum_bytes(m) > cum_bytes(d) ? cum_bytes(m) : cum_bytes(d), kAlign);
     const size_t st = round_up(states_bytes(m) > states_bytes(d) ? states_bytes(m) : states_bytes(d), kAlign);
     const size_t ring = ssd::fused_supported(d) ? round_up(ssd::fused_ring_bytes(d), kAlign) : 0;
-    return kCtrlBytes + flags_bytes(d) + ring + cum + st;
+    const size_t base = kCtrlBytes + flags_bytes(d) + ring + cum + st;
+    const int S = split_pieces(d);
+    const size_t split = S > 1 ? split_bytes(d, S, nullptr, nullptr) : 0;
+    const size_t diag = ssd::diag_scan_tc_supported(d) ? diag_tc_bytes(d, nullptr, nullptr) : 0;
+    const size_t most = base > split ? base : split;
+    return most > diag ? most : diag;
 }
 
 Workspace carve(void* ws, const Dims& d) {
@@ -107,6 +184,12 @@ Workspace carve(void* ws, const Dims& d) {
 }
 
 ssd_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA; }
+
+// Test hook: the next g_fail_calls calls that would queue GPU work return
+// SSD_ERR_CUDA instead, queueing nothing (callers' error paths can then be
+// tested without a real CUDA failure).
+std::atomic<int> g_fail_calls{0};
+bool injected_failure() { return ssd::take_injected_failure(); }
 
 // The backward's scratch, in order, each piece 256-byte aligned; returns the
 // total size.  With a base, fills the pointers.
@@ -147,7 +230,21 @@ bool g_fused_seen[kMaxDevices] = {};
 
 ssd_status run_modular(const Dims& d0, const void* x, const float* a, const void* Bm,
                        const void* Cm, const float* D, void* y, float* fin, const Workspace& w,
-                       cudaStream_t st, bool allow_tc, const float* init) {
+                       cudaStream_t st, bool allow_tc, const float* init, void* ws) {
+    if (allow_tc && ssd::diag_state_tc_supported(d0) && ssd::diag_scan_tc_supported(d0)) {
+        // per-state decay on tensor cores: the block states and totals (step 2,
+        // prefix sums done in the kernel), the pass over blocks (step 3, in
+        // place, on 128-token blocks), the outputs (step 5)
+        DiagWorkspace dw;
+        diag_tc_bytes(d0, ws, &dw);
+        Dims blk = d0;
+        blk.Q = 1;  // the pass reads one total per block: a "chunk" of one position
+        blk.nc = (d0.T + 127) / 128;
+        cudaError_t e = ssd::launch_diag_state_tc(d0, x, a, Bm, dw.states, dw.tot, w.ctrl, st);
+        if (e == cudaSuccess) e = ssd::launch_state_pass(blk, dw.tot, dw.states, fin, init, st);
+        if (e == cudaSuccess) e = ssd::launch_diag_scan_tc(d0, x, a, false, Bm, Cm, dw.states, D, y, w.ctrl, st);
+        return cuda_status(e);
+    }
     const Dims d = allow_tc ? modular_dims(d0) : d0;
     cudaError_t e = ssd::launch_chunk_cumsum(d, a, w.cum, st);
     if (e != cudaSuccess) return SSD_ERR_CUDA;
@@ -166,10 +263,18 @@ ssd_status run_modular(const Dims& d0, const void* x, const float* a, const void
 }  // namespace
 
 namespace ssd {
+bool take_injected_failure() {
+    int n = g_fail_calls.load();
+    while (n > 0) {
+        if (g_fail_calls.compare_exchange_weak(n, n - 1)) return true;
+    }
+    return false;
+}
+
 cudaError_t launch_fused_ordered(const Dims& d, const void* x, const float* a, const void* Bm,
                                  const void* Cm, const float* D, void* y, float* fin, float* ring,
                                  unsigned* flags, int* status, bool test_stall, cudaStream_t st,
-                                 const float* init, void* clear, size_t clear_bytes) {
+                                 const float* init, void* clear, size_t clear_bytes, int seg) {
     cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
     if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) return cudaErrorInvalidValue;
     int dev = 0;
@@ -179,7 +284,7 @@ cudaError_t launch_fused_ordered(const Dims& d, const void* x, const float* a, c
             cudaError_t e = cudaMemsetAsync(clear, 0, clear_bytes, st);
             if (e != cudaSuccess) return e;
         }
-        return launch_fused_tc(d, x, a, Bm, Cm, D, y, fin, ring, flags, status, test_stall, st, init);
+        return launch_fused_tc(d, x, a, Bm, Cm, D, y, fin, ring, flags, status, test_stall, st, init, seg);
     }
     std::lock_guard<std::mutex> lock(g_fused_mu);
     if (!g_fused_done[dev]) {
@@ -194,7 +299,7 @@ cudaError_t launch_fused_ordered(const Dims& d, const void* x, const float* a, c
         cudaError_t e = cudaMemsetAsync(clear, 0, clear_bytes, st);
         if (e != cudaSuccess) return e;
     }
-    cudaError_t e = launch_fused_tc(d, x, a, Bm, Cm, D, y, fin, ring, flags, status, test_stall, st, init);
+    cudaError_t e = launch_fused_tc(d, x, a, Bm, Cm, D, y, fin, ring, flags, status, test_stall, st, init, seg);
     if (e != cudaSuccess) return e;
     e = cudaEventRecord(g_fused_done[dev], st);
     if (e == cudaSuccess) g_fused_seen[dev] = true;
@@ -216,6 +321,10 @@ const char* ssd_status_string(ssd_status s) {
     return "SSD_ERR_UNKNOWN";
 }
 
+void ssd_test_fail_calls(int count) { g_fail_calls.store(count > 0 ? count : 0); }
+
+int ssd_test_pending_failures(void) { return g_fail_calls.load(); }
+
 size_t ssd_workspace_size(const ssd_shape* shape) {
     if (!shape) return 0;
     if (check_shape(shape) != SSD_OK) return 0;
@@ -232,6 +341,7 @@ int ssd_path_supported(const ssd_shape* shape, unsigned path) {
         case SSD_PATH_SIMT: return fits;
         case SSD_PATH_MODULAR: return fits;
         case SSD_PATH_FUSED: return ssd::fused_supported(d) ? 1 : 0;
+        case SSD_PATH_SPLIT: return split_pieces(d) > 1 ? 1 : 0;
         default: return 0;
     }
 }
@@ -246,6 +356,7 @@ int ssd_auto_path(const ssd_shape* shape) {
     constexpr long long kFusedMinChains = 76;
     if (ssd::fused_supported(d) && ((long long)d.B * d.H >= kFusedMinChains || !chains_fit_grid_y(shape)))
         return SSD_PATH_FUSED;
+    if (split_pieces(d) > 1) return SSD_PATH_SPLIT;
     return SSD_PATH_MODULAR;
 }
 
@@ -262,7 +373,7 @@ ssd_status ssd_forward_init(const ssd_shape* shape, const void* x, const float* 
         (initial_state && !aligned16(initial_state)))
         return SSD_ERR_INVALID_ARG;
     if ((flags & ~SSD_FLAG_TEST_STALL) != 0) return SSD_ERR_INVALID_ARG;
-    if (path > SSD_PATH_FUSED) return SSD_ERR_INVALID_ARG;
+    if (path > SSD_PATH_SPLIT) return SSD_ERR_INVALID_ARG;
     const Dims d = dims_of(shape);
     if (!workspace || ((uintptr_t)workspace % kAlign) != 0) return SSD_ERR_WORKSPACE;
     if (ws_bytes < ssd_workspace_size(shape)) return SSD_ERR_WORKSPACE;
@@ -271,12 +382,28 @@ ssd_status ssd_forward_init(const ssd_shape* shape, const void* x, const float* 
     if (!ssd_path_supported(shape, path)) return SSD_ERR_UNSUPPORTED;
     cudaStream_t cs = (cudaStream_t)stream;
     const Workspace w = carve(workspace, d);
+    if (injected_failure()) return SSD_ERR_CUDA;
+    if (path == SSD_PATH_SPLIT) {
+        const int S = split_pieces(d);
+        const Dims v = pieces_dims(d, S);
+        SplitWorkspace sw;
+        split_bytes(d, S, workspace, &sw);
+        // status word and the pieces' counters start at zero on every call
+        if (cudaMemsetAsync(w.ctrl, 0, (char*)sw.flags - (char*)w.ctrl + flags_bytes(v), cs) != cudaSuccess)
+            return SSD_ERR_CUDA;
+        cudaError_t e = ssd::launch_segment_state_tc(d, S, x, a, Bm, sw.fin, sw.tot, w.ctrl, cs);
+        if (e == cudaSuccess) e = ssd::launch_state_combine(d, S, sw.fin, sw.tot, initial_state, sw.h_in, cs);
+        if (e == cudaSuccess)
+            e = ssd::launch_fused_ordered(v, x, a, Bm, Cm, D, y, final_state, sw.ring, sw.flags, w.ctrl,
+                                          (flags & SSD_FLAG_TEST_STALL) != 0, cs, sw.h_in, nullptr, 0, S);
+        return cuda_status(e);
+    }
     // status word and per-chain counters start at zero on every call
     if (cudaMemsetAsync(w.ctrl, 0, kCtrlBytes + flags_bytes(d), cs) != cudaSuccess)
         return SSD_ERR_CUDA;
     switch (path) {
         case SSD_PATH_SIMT:
-            return run_modular(d, x, a, Bm, Cm, D, y, final_state, w, cs, false, initial_state);
+            return run_modular(d, x, a, Bm, Cm, D, y, final_state, w, cs, false, initial_state, workspace);
         case SSD_PATH_FUSED:
             return cuda_status(ssd::launch_fused_ordered(d, x, a, Bm, Cm, D, y, final_state, w.ring,
                                                          w.flags, w.ctrl,
@@ -284,7 +411,7 @@ ssd_status ssd_forward_init(const ssd_shape* shape, const void* x, const float* 
                                                          initial_state));
         case SSD_PATH_MODULAR:
         default:
-            return run_modular(d, x, a, Bm, Cm, D, y, final_state, w, cs, true, initial_state);
+            return run_modular(d, x, a, Bm, Cm, D, y, final_state, w, cs, true, initial_state, workspace);
     }
 }
 
@@ -349,6 +476,7 @@ ssd_status ssd_forward_host(const ssd_shape* shape, const void* x_h, const float
     const size_t nx = (size_t)d.B * d.T * d.H * d.P * el;
     const size_t na = (size_t)d.B * d.T * d.H * (d.diag ? d.N : 1) * sizeof(float);
     const size_t nbc = (size_t)d.B * d.T * d.G * d.N * el;
+    if (injected_failure()) return SSD_ERR_CUDA;
     if (cudaMemcpyAsync(base + off[0], x_h, nx, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
         cudaMemcpyAsync(base + off[1], a_h, na, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
         cudaMemcpyAsync(base + off[2], Bm_h, nbc, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
@@ -387,6 +515,7 @@ ssd_status ssd_chunk_cumsum(const ssd_shape* shape, const float* a, float* cum, 
     if (st != SSD_OK) return st;
     if (!chains_fit_grid_y(shape)) return SSD_ERR_UNSUPPORTED;
     if (!a || !cum || !aligned16(a) || !aligned16(cum)) return SSD_ERR_INVALID_ARG;
+    if (injected_failure()) return SSD_ERR_CUDA;
     return cuda_status(ssd::launch_chunk_cumsum(dims_of(shape), a, cum, (cudaStream_t)stream));
 }
 
@@ -402,6 +531,7 @@ ssd_status ssd_chunk_state(const ssd_shape* shape, const void* x, const void* Bm
     const Dims d = dims_of(shape);
     const bool tc_ok = ssd::chunk_state_tc_supported(d);
     if (impl == SSD_IMPL_TC && !tc_ok) return SSD_ERR_UNSUPPORTED;
+    if (injected_failure()) return SSD_ERR_CUDA;
     const bool use_tc = impl == SSD_IMPL_TC || (impl == SSD_IMPL_AUTO && tc_ok);
     cudaStream_t cs = (cudaStream_t)stream;
     return cuda_status(use_tc ? ssd::launch_chunk_state_tc(d, x, Bm, cum, states, cs)
@@ -416,6 +546,7 @@ ssd_status ssd_state_pass(const ssd_shape* shape, const float* cum, float* state
     if (!cum || !states || !aligned16(cum) || !aligned16(states) ||
         (final_state && !aligned16(final_state)))
         return SSD_ERR_INVALID_ARG;
+    if (injected_failure()) return SSD_ERR_CUDA;
     return cuda_status(
         ssd::launch_state_pass(dims_of(shape), cum, states, final_state, nullptr, (cudaStream_t)stream));
 }
@@ -433,10 +564,13 @@ static ssd_status scan_common(const ssd_shape* shape, const void* x, const void*
         return SSD_ERR_INVALID_ARG;
     if (impl > SSD_IMPL_TC) return SSD_ERR_INVALID_ARG;
     const Dims d = dims_of(shape);
-    const bool tc_ok = ssd::chunk_scan_tc_supported(d);
+    const bool tc_ok = want_diag ? (ssd::diag_scan_tc_supported(d) && d.Q == 128) : ssd::chunk_scan_tc_supported(d);
     if (impl == SSD_IMPL_TC && !tc_ok) return SSD_ERR_UNSUPPORTED;
     const bool use_tc = impl == SSD_IMPL_TC || (impl == SSD_IMPL_AUTO && tc_ok);
     cudaStream_t cs = (cudaStream_t)stream;
+    if (injected_failure()) return SSD_ERR_CUDA;
+    if (use_tc && want_diag)
+        return cuda_status(ssd::launch_diag_scan_tc(d, x, cum, true, Bm, Cm, Hin, D, y, nullptr, cs));
     return cuda_status(use_tc ? ssd::launch_chunk_scan_tc(d, x, Bm, Cm, cum, Hin, D, y, cs)
                               : ssd::launch_chunk_scan_simt(d, x, Bm, Cm, cum, Hin, D, y, cs));
 }
@@ -461,6 +595,7 @@ ssd_status ssd_discretize(const ssd_shape* shape, const float* dt_raw, const flo
     if (!aligned16(dt_raw) || !aligned16(A_log) || !aligned16(x) || !aligned16(a_out) ||
         !aligned16(x_out) || (dt_bias && !aligned16(dt_bias)))
         return SSD_ERR_INVALID_ARG;
+    if (injected_failure()) return SSD_ERR_CUDA;
     return cuda_status(ssd::launch_discretize(dims_of(shape), dt_raw, dt_bias, A_log, x, a_out,
                                               x_out, (cudaStream_t)stream));
 }
@@ -468,6 +603,7 @@ ssd_status ssd_discretize(const ssd_shape* shape, const float* dt_raw, const flo
 ssd_status ssd_decay_total(const ssd_shape* shape, const float* a, float* total, ssd_stream stream) {
     if (check_shape(shape) != SSD_OK || !a || !total || !aligned16(a) || !aligned16(total))
         return SSD_ERR_INVALID_ARG;
+    if (injected_failure()) return SSD_ERR_CUDA;
     return cuda_status(ssd::launch_decay_total(dims_of(shape), a, total, (cudaStream_t)stream));
 }
 
@@ -477,8 +613,35 @@ ssd_status ssd_state_combine(const ssd_shape* shape, int segments, const float* 
         return SSD_ERR_INVALID_ARG;
     if (!aligned16(finals) || !aligned16(totals) || !aligned16(h_in) || (h0 && !aligned16(h0)))
         return SSD_ERR_INVALID_ARG;
+    if (injected_failure()) return SSD_ERR_CUDA;
     return cuda_status(ssd::launch_state_combine(dims_of(shape), segments, finals, totals, h0, h_in,
                                                  (cudaStream_t)stream));
+}
+
+ssd_status ssd_segment_state(const ssd_shape* shape, const void* x, const float* a, const void* Bm,
+                             float* final_state, float* total, void* workspace, size_t ws_bytes,
+                             ssd_stream stream) {
+    ssd_status st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    if (!x || !a || !Bm || !final_state || !total) return SSD_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(a) || !aligned16(Bm) || !aligned16(final_state) || !aligned16(total))
+        return SSD_ERR_INVALID_ARG;
+    if (!workspace || ((uintptr_t)workspace % kAlign) != 0) return SSD_ERR_WORKSPACE;
+    if (ws_bytes < ssd_workspace_size(shape)) return SSD_ERR_WORKSPACE;
+    const Dims d = dims_of(shape);
+    if (injected_failure()) return SSD_ERR_CUDA;
+    const bool tc = ssd::segment_state_tc_supported(d);
+    if (!tc && !chains_fit_grid_y(shape)) return SSD_ERR_UNSUPPORTED;
+    cudaStream_t cs = (cudaStream_t)stream;
+    const Workspace w = carve(workspace, d);
+    if (cudaMemsetAsync(w.ctrl, 0, kCtrlBytes, cs) != cudaSuccess) return SSD_ERR_CUDA;
+    if (tc) return cuda_status(ssd::launch_segment_state_tc(d, 1, x, a, Bm, final_state, total, w.ctrl, cs));
+    // other shapes: the modular path's first three steps (CUDA cores), then the total
+    cudaError_t e = ssd::launch_chunk_cumsum(d, a, w.cum, cs);
+    if (e == cudaSuccess) e = ssd::launch_chunk_state_simt(d, x, Bm, w.cum, w.states, cs);
+    if (e == cudaSuccess) e = ssd::launch_state_pass(d, w.cum, w.states, final_state, nullptr, cs);
+    if (e == cudaSuccess) e = ssd::launch_decay_total(d, a, total, cs);
+    return cuda_status(e);
 }
 
 ssd_status ssd_decode_step(const ssd_shape* shape, const void* x, const float* a, const void* Bm,
@@ -489,6 +652,7 @@ ssd_status ssd_decode_step(const ssd_shape* shape, const void* x, const float* a
     if (!aligned16(x) || !aligned16(a) || !aligned16(Bm) || !aligned16(Cm) || !aligned16(state) ||
         !aligned16(y) || (D && !aligned16(D)))
         return SSD_ERR_INVALID_ARG;
+    if (injected_failure()) return SSD_ERR_CUDA;
     return cuda_status(ssd::launch_decode_step(dims_of(shape), x, a, Bm, Cm, D, state, y,
                                                (cudaStream_t)stream));
 }
@@ -509,6 +673,7 @@ ssd_status ssd_backward(const ssd_shape* shape, const void* x, const float* a, c
     const size_t need = backward_layout(d, nullptr, nullptr);
     if (!workspace || ((uintptr_t)workspace % kAlign) != 0 || ws_bytes < need)
         return SSD_ERR_WORKSPACE;
+    if (injected_failure()) return SSD_ERR_CUDA;
     ssd::BackwardScratch w;
     backward_layout(d, workspace, &w);
     ssd::BackwardArgs g{x, a, Bm, Cm, D, initial_state, dy, dfinal, dx, da, dBm, dCm, dD, dinit};

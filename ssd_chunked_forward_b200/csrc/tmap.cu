@@ -45,6 +45,22 @@ cudaError_t make_tmap_bf16_4d(CUtensorMap* map, const void* base, uint64_t d0, u
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+cudaError_t make_tmap_f32_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                             uint64_t d3, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    if (((uintptr_t)base & 15u) != 0 || (d0 * 4) % 16 != 0 || d0 > 256) return cudaErrorInvalidValue;
+    const cuuint64_t dims[4] = {d0, d1, d2, d3};
+    const cuuint64_t strides[3] = {d0 * 4, d0 * d1 * 4, d0 * d1 * d2 * 4};  // bytes, dims 1..3
+    const cuuint32_t box[4] = {(cuuint32_t)d0, 1, box_rows, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    // dense rows of d0 floats in shared memory; rows past the tensor read zero
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(base), dims, strides, box,
+                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 cudaError_t make_tmap_f32_rows64(CUtensorMap* map, const void* base, uint64_t rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return cudaErrorNotSupported;

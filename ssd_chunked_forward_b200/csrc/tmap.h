@@ -18,6 +18,13 @@ namespace ssd {
 cudaError_t make_tmap_bf16_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
                               uint64_t d2, uint64_t d3, uint32_t box_rows);
 
+// A 4-D fp32 tensor map over a row-major [d3][d2][d1][d0] array (d0 <= 256
+// innermost, e.g. the per-state log-decays [B][T][H][N]), box (d0, 1, rows,
+// 1) without swizzle: one box lands as `rows` dense rows of d0 floats.  Rows
+// past d2 read as zero.
+cudaError_t make_tmap_f32_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                             uint64_t d3, uint32_t box_rows);
+
 // A 2-D fp32 tensor map over a row-major [rows][64] array, box (32, 128) with
 // 128-byte swizzle: one box is 128 rows of 32 floats = 128 bytes; a 128 x 64
 // tile is two boxes (columns 0-31 and 32-63).

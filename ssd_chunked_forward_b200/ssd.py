@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(_HERE, "libssd.so")
 
 SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_WORKSPACE, SSD_ERR_CUDA, SSD_ERR_TIMEOUT = range(6)
 SSD_DTYPE_F32, SSD_DTYPE_BF16 = 0, 1
-PATH_AUTO, PATH_MODULAR, PATH_SIMT, PATH_FUSED = 0, 1, 2, 3
+PATH_AUTO, PATH_MODULAR, PATH_SIMT, PATH_FUSED, PATH_SPLIT = 0, 1, 2, 3, 4
 IMPL_AUTO, IMPL_SIMT, IMPL_TC = 0, 1, 2
 FLAG_TEST_STALL = 0x100
 
@@ -27,7 +27,8 @@ EXPORTS = [
     "ssd_state_pass", "ssd_chunk_scan", "ssd_diag_scan", "ssd_forward_host_bytes",
     "ssd_forward_host", "ssd_forward_noalloc", "ssd_auto_path", "ssd_forward_init",
     "ssd_decode_step", "ssd_discretize", "ssd_decay_total", "ssd_state_combine",
-    "ssd_backward", "ssd_backward_workspace_size",
+    "ssd_segment_state", "ssd_backward", "ssd_backward_workspace_size",
+    "ssd_test_fail_calls", "ssd_test_pending_failures",
 ]
 
 
@@ -83,12 +84,17 @@ def load(path: str = LIB_PATH):
     lib.ssd_discretize.argtypes = [sp, fp, fp, fp, vp, fp, vp, vp]
     lib.ssd_decay_total.argtypes = [sp, fp, fp, vp]
     lib.ssd_state_combine.argtypes = [sp, ctypes.c_int, fp, fp, fp, fp, vp]
+    lib.ssd_segment_state.argtypes = [sp, vp, fp, vp, fp, fp, vp, sz, vp]
+    lib.ssd_test_fail_calls.argtypes = [ctypes.c_int]
+    lib.ssd_test_fail_calls.restype = None
+    lib.ssd_test_pending_failures.argtypes = []
+    lib.ssd_test_pending_failures.restype = ctypes.c_int
     lib.ssd_backward.argtypes = [sp, vp, fp, vp, vp, fp, fp, vp, fp, vp, fp, vp, vp, fp, fp, vp, sz, vp]
     lib.ssd_backward_workspace_size.argtypes = [sp]
     lib.ssd_backward_workspace_size.restype = sz
     for name in ("ssd_forward_noalloc", "ssd_forward", "ssd_forward_path", "ssd_forward_init",
                  "ssd_device_status", "ssd_chunk_cumsum", "ssd_decode_step", "ssd_discretize",
-                 "ssd_decay_total", "ssd_state_combine", "ssd_backward",
+                 "ssd_decay_total", "ssd_state_combine", "ssd_segment_state", "ssd_backward",
                  "ssd_chunk_state", "ssd_state_pass", "ssd_chunk_scan", "ssd_diag_scan",
                  "ssd_forward_host"):
         getattr(lib, name).restype = ctypes.c_int
@@ -141,7 +147,8 @@ def path_supported(shape: Shape, path: int) -> bool:
 
 
 def auto_path(shape: Shape) -> int:
-    """The path SSD_PATH_AUTO takes for this shape (PATH_FUSED or PATH_MODULAR)."""
+    """The path SSD_PATH_AUTO takes for this shape (PATH_FUSED, PATH_SPLIT or
+    PATH_MODULAR)."""
     return int(load().ssd_auto_path(ctypes.byref(shape)))
 
 
@@ -351,6 +358,27 @@ def state_combine(finals, totals, h0=None, *, out=None, stream=None):
     _check(load().ssd_state_combine(ctypes.byref(shape), int(S), _ptr(finals), _ptr(totals), _ptr(h0),
                                     _ptr(out), _stream(stream)), "ssd_state_combine")
     return out
+
+
+def segment_state(x, a, Bm, chunk=256, *, final_state=None, total=None, workspace=None, stream=None):
+    """The state a segment builds from a zero start, [B,H,N,P] fp32, and its
+    total log-decay [B,H] (or [B,H,N]), without computing its outputs."""
+    for name, t in (("x", x), ("a", a), ("Bm", Bm)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    shape = shape_of(x, a, Bm, chunk)
+    B, T, H, P = x.shape
+    N = Bm.shape[3]
+    if final_state is None:
+        final_state = torch.empty((B, H, N, P), dtype=torch.float32, device=x.device)
+    if total is None:
+        total = torch.empty((B, H) + ((N,) if a.dim() == 4 else ()), dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = alloc_workspace(shape, x.device)
+    _check(load().ssd_segment_state(ctypes.byref(shape), _ptr(x), _ptr(a), _ptr(Bm), _ptr(final_state),
+                                    _ptr(total), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "ssd_segment_state")
+    return final_state, total
 
 
 def backward_workspace_size(shape: Shape) -> int:

@@ -172,13 +172,20 @@ def test_host_entry_point_validates(lib):
 
 def test_auto_path_choice(lib):
     """AUTO takes the fused kernel for the Mamba-2 shapes with enough (batch,
-    head) chains and the modular path for few long chains, fp32 and the
+    head) chains, the split path for few long chains whose length divides into
+    pieces of >= 4096 tokens, and the modular path for the rest, fp32 and the
     per-state variant; an invalid shape gives -1."""
     fused = ssd.make_shape(4, 8192, 80, 64, 1, 128, 256)            # 320 chains
     assert ssd.auto_path(fused) == ssd.PATH_FUSED
     assert ssd.auto_path(ssd.make_shape(8, 2048, 24, 64, 1, 128, 256)) == ssd.PATH_FUSED   # 192
     assert ssd.auto_path(ssd.make_shape(1, 8192, 80, 64, 1, 128, 256)) == ssd.PATH_FUSED   # 80
-    assert ssd.auto_path(ssd.make_shape(1, 262144, 32, 64, 8, 128, 256)) == ssd.PATH_MODULAR  # 32
+    assert ssd.auto_path(ssd.make_shape(1, 262144, 32, 64, 8, 128, 256)) == ssd.PATH_SPLIT  # 32
+    assert ssd.auto_path(ssd.make_shape(1, 4096, 32, 64, 8, 128, 256)) == ssd.PATH_MODULAR  # too short
+    assert ssd.auto_path(ssd.make_shape(1, 8193, 32, 64, 8, 128, 256)) == ssd.PATH_MODULAR  # T odd
+    long1 = ssd.make_shape(1, 262144, 32, 64, 8, 128, 256)
+    assert ssd.path_supported(long1, ssd.PATH_SPLIT)
+    assert not ssd.path_supported(ssd.make_shape(1, 262144, 32, 64, 8, 128, 256, dtype="f32"),
+                                  ssd.PATH_SPLIT)
     assert ssd.auto_path(ssd.make_shape(4, 8192, 80, 64, 1, 128, 256, dtype="f32")) == ssd.PATH_MODULAR
     assert ssd.auto_path(ssd.make_shape(4, 4096, 16, 64, 1, 64, 128, a_per_state=True)) == ssd.PATH_MODULAR
     # T % chunk != 0: a partial last chunk; 2 chains is few, so modular
@@ -226,3 +233,29 @@ def test_chain_count_beyond_grid_y_refused_before_launch(lib):
         ssd.SSD_ERR_UNSUPPORTED
     f32 = ssd.make_shape(1024, 256, 80, 64, 1, 128, 256, dtype="f32")  # no fused kernel for fp32
     assert not ssd.path_supported(f32, ssd.PATH_AUTO)
+
+
+def test_injected_cuda_failure_hook(lib):
+    """ssd_test_fail_calls(n): the next n calls that would queue GPU work
+    return SSD_ERR_CUDA after their argument checks (which still come first),
+    and the binding raises SSDError with that code."""
+    s = _shape()
+    ok = 1 << 20
+    ws = ssd.workspace_size(s)
+    lib.ssd_test_fail_calls(3)
+    try:
+        assert lib.ssd_test_pending_failures() == 3
+        # a bad argument is still reported as such, and does not consume the count
+        assert lib.ssd_forward(ctypes.byref(s), None, ok, ok, ok, None, ok, None, ok, ws, None) == \
+            ssd.SSD_ERR_INVALID_ARG
+        assert lib.ssd_test_pending_failures() == 3
+        assert lib.ssd_forward(ctypes.byref(s), ok, ok, ok, ok, None, ok, None, ok, ws, None) == \
+            ssd.SSD_ERR_CUDA
+        assert lib.ssd_chunk_cumsum(ctypes.byref(s), ok, ok, None) == ssd.SSD_ERR_CUDA
+        assert lib.ssd_test_pending_failures() == 1
+        with pytest.raises(ssd.SSDError) as e:
+            ssd._check(lib.ssd_decay_total(ctypes.byref(s), ok, ok, None), "ssd_decay_total")
+        assert e.value.code == ssd.SSD_ERR_CUDA
+        assert lib.ssd_test_pending_failures() == 0
+    finally:
+        lib.ssd_test_fail_calls(0)

@@ -40,6 +40,11 @@ CASES = [
     small_case(B=1, T=2048, H=16, P=64, N=128, G=1, chunk=128, dtype="bf16", seed=14),
     small_case(B=2, T=256, H=2, P=64, N=64, G=1, chunk=128, dtype="bf16", a_per_state=True, seed=6),
     small_case(B=1, T=60, H=2, P=10, N=12, G=1, chunk=20, dtype="f32", a_per_state=True, seed=7),
+    # per-state tensor-core steps: an odd number of 128-token blocks; groups, a
+    # partial last block and fast decay (a sub-block's decay far beyond fp32's range)
+    small_case(B=1, T=384, H=3, P=64, N=64, G=1, chunk=128, dtype="bf16", a_per_state=True, seed=31),
+    small_case(B=2, T=1000, H=4, P=64, N=64, G=2, chunk=128, dtype="bf16", a_per_state=True, seed=32,
+               u_mean=-1.0),
 ]
 EDGE = [
     small_case(B=1, T=1, H=1, P=1, N=1, G=1, chunk=1, dtype="f32", seed=8),
@@ -513,36 +518,113 @@ def test_discretize_odd_rows():
     assert rel_err(x_g.cpu().numpy().astype(np.float64), x_r) <= 1e-6
 
 
-@pytest.mark.parametrize("per_state", [False, True], ids=["scalar", "per_state"])
-def test_sequence_segments_with_library_kernels(per_state):
-    """A sequence cut into 4 segments, each run from zero, combined by
-    ssd_decay_total + ssd_state_combine and rerun from its incoming state
-    (what each rank does in the sharded forward), equals the forward over the
-    whole sequence; the combine's last state is the sequence's final state."""
-    if per_state:
-        w = small_case(B=2, T=1024, H=4, P=64, N=64, G=1, chunk=128, dtype="bf16", a_per_state=True, seed=103)
-    else:
-        w = small_case(B=2, T=4096, H=8, P=64, N=128, G=1, chunk=256, dtype="bf16", seed=104)
+SEGMENT_CASES = [
+    small_case(B=2, T=4096, H=8, P=64, N=128, G=1, chunk=256, dtype="bf16", seed=104),
+    small_case(B=1, T=4000, H=4, P=64, N=128, G=2, chunk=256, dtype="bf16", seed=105, u_mean=-4.0),
+    small_case(B=2, T=1024, H=4, P=64, N=64, G=1, chunk=128, dtype="bf16", a_per_state=True, seed=103),
+    small_case(B=1, T=600, H=3, P=20, N=12, G=1, chunk=64, dtype="f32", seed=106),
+]
+
+
+@pytest.mark.parametrize("w", SEGMENT_CASES, ids=_ids(SEGMENT_CASES))
+@pytest.mark.parametrize("with_init", [False, True], ids=["zero", "init"])
+def test_sequence_segments_with_library_kernels(w, with_init):
+    """What every rank of the sequence-sharded forward does, with the
+    library's kernels, for a sequence cut into 4 segments: each segment's
+    state from zero and total decay (ssd_segment_state), their combine into
+    the state entering every segment (ssd_state_combine), and one forward per
+    segment from that state (ssd_forward_init).  The segments' y, joined, and
+    the combine's last state equal the fp64 recurrence over the whole
+    sequence (the oracle, not the library's whole-sequence forward); the
+    segment states and totals equal the oracle's too."""
     inp = generate(w)
     dev = to_dev(inp)
-    y_full, f_full = ssd.forward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], dev["D"], w.chunk)
     S = 4
-    Ts = w.T // S
-    seg = lambda t, s: t[:, s * Ts:(s + 1) * Ts].contiguous()
+    bounds = [round(s * w.T / S) for s in range(S + 1)]
+    # a fresh (16-byte aligned) copy per segment, as each rank would hold
+    seg = lambda t, s: t[:, bounds[s]:bounds[s + 1]].clone()
     parts = [[seg(dev[k], s) for k in ("x", "a", "Bm", "Cm")] for s in range(S)]
+    h0 = None
+    if with_init:
+        g = torch.Generator().manual_seed(w.seed + 3)
+        h0 = torch.randn((w.B, w.H, w.N, w.P), generator=g, dtype=torch.float64).to(torch.float32)
     fins, tots = [], []
     for x, a, Bm, Cm in parts:
-        _, f = ssd.forward(x, a, Bm, Cm, dev["D"], w.chunk)
+        f, tot = ssd.segment_state(x, a, Bm, w.chunk)
         fins.append(f)
-        tots.append(ssd.decay_total(a))
+        tots.append(tot)
     totals = torch.stack(tots).contiguous()
-    h_in = ssd.state_combine(torch.stack(fins).contiguous(), totals)
+    h_in = ssd.state_combine(torch.stack(fins).contiguous(), totals, None if h0 is None else h0.cuda())
     ys = [ssd.forward(x, a, Bm, Cm, dev["D"], w.chunk, initial_state=h_in[s].contiguous())[0]
           for s, (x, a, Bm, Cm) in enumerate(parts)]
     torch.cuda.synchronize()
-    assert rel_err(torch.cat(ys, dim=1).float().cpu().numpy(), y_full.float().cpu().numpy()) <= TOL_BF16
-    assert rel_err(h_in[S].cpu().numpy(), f_full.cpu().numpy()) <= TOL_BF16
-    # the totals themselves: sums of the segment's log-decays
-    a64 = inp["a"].to(torch.float64)
-    ref_tot = torch.stack([a64[:, s * Ts:(s + 1) * Ts].sum(dim=1) for s in range(S)]).numpy()
-    assert rel_err(totals.cpu().numpy().astype(np.float64), ref_tot) <= 1e-5
+    tol = tol_for(w)
+    f64 = lambda t: t.to(torch.float64).numpy()
+    prob = O.Problem(*(f64(inp[k]) for k in ("x", "a", "Bm", "Cm", "D")))
+    ref = O.recurrence(prob, initial=None if h0 is None else f64(h0))
+    yr = ref["y"].reshape(w.B, w.H, w.T, w.P).transpose(0, 2, 1, 3)
+    y = torch.cat(ys, dim=1).float().cpu().numpy().astype(np.float64)
+    assert rel_err(y, yr) <= tol, f"y rel err {rel_err(y, yr):.3e}"
+    fr = ref["final"].reshape(w.B, w.H, w.N, w.P)
+    assert rel_err(h_in[S].cpu().numpy().astype(np.float64), fr) <= tol
+    # each segment's own state from zero and total log-decay against the oracle
+    for s in range(S):
+        sub = O.Problem(*(f64(seg(inp[k], s)) for k in ("x", "a", "Bm", "Cm")), f64(inp["D"]))
+        rs = O.recurrence(sub, want_y=False)
+        assert rel_err(fins[s].cpu().numpy().astype(np.float64),
+                       rs["final"].reshape(w.B, w.H, w.N, w.P)) <= tol, f"segment {s} state"
+        a64 = f64(seg(inp["a"], s))
+        assert rel_err(tots[s].cpu().numpy().astype(np.float64), a64.sum(axis=1)) <= 1e-5
+
+
+# few long sequences: SSD_PATH_SPLIT cuts each into pieces (the piece states
+# from zero, their combine, then the fused kernel over all pieces); pieces of
+# 4100 tokens end inside a 128-token block
+SPLIT_CASES = [
+    small_case(B=1, T=16384, H=4, P=64, N=128, G=1, chunk=256, dtype="bf16", seed=81, u_mean=-4.0),
+    small_case(B=2, T=12288, H=2, P=64, N=128, G=2, chunk=256, dtype="bf16", seed=82),
+    small_case(B=1, T=8200, H=3, P=64, N=128, G=1, chunk=128, dtype="bf16", seed=83, u_mean=-5.0),
+]
+
+
+@pytest.mark.parametrize("w", SPLIT_CASES, ids=_ids(SPLIT_CASES))
+@pytest.mark.parametrize("with_init", [False, True], ids=["zero", "init"])
+def test_split_path_matches_oracle(w, with_init):
+    """The split path equals the fp64 recurrence over the whole sequence, from
+    a zero or a given initial state; AUTO takes it for these shapes."""
+    inp = generate(w)
+    dev = to_dev(inp)
+    shape = ssd.shape_of(dev["x"], dev["a"], dev["Bm"], w.chunk)
+    assert ssd.path_supported(shape, ssd.PATH_SPLIT)
+    assert ssd.auto_path(shape) == ssd.PATH_SPLIT
+    h0 = None
+    if with_init:
+        g = torch.Generator().manual_seed(w.seed + 9)
+        h0 = torch.randn((w.B, w.H, w.N, w.P), generator=g, dtype=torch.float64).to(torch.float32)
+    y, fin = ssd.forward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], dev["D"], w.chunk, path=ssd.PATH_SPLIT,
+                         initial_state=None if h0 is None else h0.cuda())
+    torch.cuda.synchronize()
+    prob = O.Problem(*(inp[k].to(torch.float64).numpy() for k in ("x", "a", "Bm", "Cm", "D")))
+    ref = O.recurrence(prob, initial=None if h0 is None else h0.to(torch.float64).numpy())
+    yr = ref["y"].reshape(w.B, w.H, w.T, w.P).transpose(0, 2, 1, 3)
+    ey = rel_err(y.float().cpu().numpy().astype(np.float64), yr)
+    ef = rel_err(fin.cpu().numpy().astype(np.float64), ref["final"].reshape(w.B, w.H, w.N, w.P))
+    assert ey <= TOL_BF16, f"y rel err {ey:.3e}"
+    assert ef <= TOL_BF16, f"final rel err {ef:.3e}"
+
+
+def test_per_state_extreme_decay():
+    """Per-state decays down to -1e4 (the state forgets at once) mixed with
+    slow ones: the tensor-core steps stay finite and match the oracle (every
+    weight they form is a product of factors <= 1)."""
+    w = small_case(B=1, T=512, H=2, P=64, N=64, G=1, chunk=128, dtype="bf16", a_per_state=True, seed=33)
+    inp = generate(w)
+    g = torch.Generator().manual_seed(34)
+    mask = torch.rand(inp["a"].shape, generator=g) < 0.05
+    inp["a"] = torch.where(mask, torch.full_like(inp["a"], -1e4), inp["a"]).contiguous()
+    dev = to_dev(inp)
+    for path in (ssd.PATH_MODULAR, ssd.PATH_AUTO):
+        y, fin = run_forward(w, dev, path=path)
+        assert torch.isfinite(y.float()).all() and torch.isfinite(fin).all()
+        ey, ef = parity_on_chains(inp, y, fin, _all_chains(w))
+        assert ey <= TOL_BF16 and ef <= TOL_BF16, (path, ey, ef)

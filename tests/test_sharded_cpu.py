@@ -47,8 +47,13 @@ def _oracle_ops():
         y = r["y"].reshape(B, H, T, P).transpose(0, 2, 1, 3)
         return torch.from_numpy(np.ascontiguousarray(y)), torch.from_numpy(r["final"].reshape(B, H, N, P))
 
-    def decay_total(a):
-        return a.sum(dim=1)
+    def segment_state(x, a, Bm, chunk):
+        # the segment's final state from zero (y not needed) and its total decay
+        B, T, H, P = x.shape
+        N = Bm.shape[3]
+        Cz = np.zeros(Bm.shape)
+        r = O.recurrence(O.Problem(x.numpy(), a.numpy(), Bm.numpy(), Cz, None), want_y=False)
+        return torch.from_numpy(r["final"].reshape(B, H, N, P)), a.sum(dim=1)
 
     def state_combine(finals, totals, h0):
         S = finals.shape[0]
@@ -68,7 +73,7 @@ def _oracle_ops():
         return {k: torch.from_numpy(np.ascontiguousarray(r[k]))
                 for k in ("dx", "da", "dBm", "dCm", "dD", "dinit")}
 
-    return SegmentOps(forward=forward, decay_total=decay_total, state_combine=state_combine,
+    return SegmentOps(forward=forward, segment_state=segment_state, state_combine=state_combine,
                       backward=backward)
 
 
@@ -140,8 +145,9 @@ def _bwd_extras(per_state):
 @pytest.mark.parametrize("per_state,with_init,with_dfinal",
                          [(False, False, False), (False, True, True), (True, True, True)])
 def test_sequence_sharded_backward(tmp_path, world, per_state, with_init, with_dfinal):
-    """The sharded backward (two all-gathers: entering states forwards,
-    entering-state adjoints backwards) equals the backward of the whole
+    """The sharded backward (entering states forwards by one all-gather,
+    entering-state adjoints backwards by another, dD summed by an all-reduce)
+    equals the backward of the whole
     sequence: each rank's slice of dx, da, dB, dC, and dD and the initial
     state's gradient on every rank."""
     from oracle import ssd_oracle as O
