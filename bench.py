@@ -80,6 +80,10 @@ def kernel_bytes(w, name):
         return x + 2 * bc + cum + st + x + H * 4
     if name == "fused":
         return algorithmic(w)[1]
+    if name == "segment_state":
+        return x + bc // 2 + a + B * H * N * P * 4  # x, Bm, a once; a state per piece (small)
+    if name == "state_combine":
+        return 0
     raise KeyError(name)
 
 
@@ -292,10 +296,53 @@ def whole_job_rate(tokens_per_rank: int, world: int, ms: float) -> float:
 
 # ---------------------------------------------------------------- GPU leg ----
 
+def per_state_tc(w):
+    """The per-state shapes whose modular path runs on tensor cores (three
+    launches: block states with the decay sums inside, the pass, the outputs)."""
+    return w.a_per_state and w.dtype == "bf16" and w.N == 64 and w.P == 64
+
+
 def step_kernels(w, path_used):
     if path_used == "fused":
         return ["fused"]
+    if path_used == "split":
+        return ["segment_state", "state_combine", "fused"]
+    if path_used == "modular" and per_state_tc(w):
+        return ["chunk_state", "state_pass", "diag_scan"]
     return ["chunk_cumsum", "chunk_state", "state_pass", "diag_scan" if w.a_per_state else "chunk_scan"]
+
+
+def time_split_path(w, dev, flush, reps, S):
+    """Device times (ms) of the split path's three launches, called one by one
+    through the library on the [B*S][T/S] view of the inputs: the pieces'
+    states from zero (ssd_segment_state), their combine (ssd_state_combine),
+    and the forward over all pieces from their entering states
+    (ssd_forward_init; the fused kernel)."""
+    B, T = w.B, w.T
+    L = T // S
+    view = {k: dev[k].view((B * S, L) + tuple(dev[k].shape[2:])) for k in ("x", "a", "Bm", "Cm")}
+    st = torch.cuda.current_stream()
+    times = {"segment_state": [], "state_combine": [], "fused": []}
+    for r in range(reps):
+        flush()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev[0].record(st)
+        fin, tot = ssd.segment_state(view["x"], view["a"], view["Bm"], w.chunk)
+        ev[1].record(st)
+        finals = fin.view(B, S, w.H, w.N, w.P).transpose(0, 1).contiguous()
+        totals = tot.view(B, S, w.H).transpose(0, 1).contiguous()
+        h_in = ssd.state_combine(finals, totals)
+        ev[2].record(st)
+        init = h_in[:S].transpose(0, 1).reshape(B * S, w.H, w.N, w.P).contiguous()
+        ssd.forward(view["x"], view["a"], view["Bm"], view["Cm"], dev["D"], w.chunk, initial_state=init,
+                    path=ssd.PATH_FUSED)
+        ev[3].record(st)
+        torch.cuda.synchronize()
+        if r == 0:
+            continue
+        for i, n in enumerate(times):
+            times[n].append(ev[i].elapsed_time(ev[i + 1]))
+    return {n: statistics.median(v) for n, v in times.items()}
 
 
 def step_workload(w, impl):
@@ -321,7 +368,11 @@ def time_steps_split(w, dev, flush, reps, impl):
     states = torch.empty((w.B, w.H, nc, w.N, w.P), dtype=torch.float32, device=dev["x"].device)
     fin = torch.empty((w.B, w.H, w.N, w.P), dtype=torch.float32, device=dev["x"].device)
     y = torch.empty_like(dev["x"])
-    names = step_kernels(w, "modular")
+    # the four step entry points; for the per-state tensor-core shapes the
+    # forward itself folds the prefix sums into the other kernels, and its
+    # block-state and output kernels are these steps' kernels reading a instead
+    # of the prefix sums (the same bytes)
+    names = ["chunk_cumsum", "chunk_state", "state_pass", "diag_scan" if w.a_per_state else "chunk_scan"]
     times = {n: [] for n in names}
     for r in range(reps):
         flush()
@@ -341,7 +392,10 @@ def time_steps_split(w, dev, flush, reps, impl):
         for i, n in enumerate(names):
             times[n].append(ev[i].elapsed_time(ev[i + 1]))
     del cum_t, states, fin, y
-    return {n: statistics.median(v) for n, v in times.items()}
+    out = {n: statistics.median(v) for n, v in times.items()}
+    if impl != ssd.IMPL_SIMT and per_state_tc(w):
+        out.pop("chunk_cumsum")  # not launched by the forward
+    return out
 
 
 def run_decode(args, device):
@@ -561,7 +615,7 @@ def main():
         raise SystemExit(f"path {args.path} does not serve workload {w.name}")
     path_used = args.path
     if path == ssd.PATH_AUTO:
-        path_used = "fused" if ssd.auto_path(shape) == ssd.PATH_FUSED else "modular"
+        path_used = {ssd.PATH_FUSED: "fused", ssd.PATH_SPLIT: "split"}.get(ssd.auto_path(shape), "modular")
     ws = ssd.alloc_workspace(shape, device)
     y = torch.empty_like(dev["x"])
     fin = torch.empty((w.B, w.H, w.N, w.P), dtype=torch.float32, device=device)
@@ -612,12 +666,14 @@ def main():
     t_roof = max(flops / (peaks["bf16_tflops"] * 1e12), byts / (peaks["hbm_gbs"] * 1e9))
     if path_used == "fused":
         split = {"fused": ms}
+    elif path_used == "split":
+        split = time_split_path(w, dev, flush, 11, ssd.split_pieces(shape))
     else:
         impl = ssd.IMPL_SIMT if path_used == "simt" else ssd.IMPL_AUTO
         split = time_steps_split(w, dev, flush, 11, impl)
     dom = max(split, key=split.get)
     dom_ms = split[dom]
-    dom_bytes = kernel_bytes(w if path_used == "fused" else
+    dom_bytes = kernel_bytes(w if path_used in ("fused", "split") else
                              step_workload(w, ssd.IMPL_SIMT if path_used == "simt" else ssd.IMPL_AUTO), dom)
     achieved = dom_bytes / (dom_ms / 1e3) / 1e9
     kernel_name = {"fused": "ssd_fused_kernel"}.get(dom, "ssd_" + dom)

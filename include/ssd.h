@@ -139,6 +139,12 @@ int ssd_path_supported(const ssd_shape* shape, unsigned path);
  * pages; it only picks between exact evaluations of the same forward. */
 int ssd_auto_path(const ssd_shape* shape);
 
+/* The number of pieces S that SSD_PATH_SPLIT cuts each sequence into for this
+ * shape (each piece T / S tokens: the rows of the [B * S][T / S] view of the
+ * tensors), 1 when the split path does not serve the shape, 0 for an invalid
+ * shape. */
+int ssd_split_pieces(const ssd_shape* shape);
+
 /* The whole forward: y (and final_state when non-NULL) from x, a, Bm, Cm, D.
  * `workspace` (device, >= ssd_workspace_size bytes, 256-byte aligned) is
  * scratch owned by the caller and must not be shared by calls that overlap

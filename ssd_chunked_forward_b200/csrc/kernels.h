@@ -116,7 +116,9 @@ cudaError_t launch_segment_state_tc(const Dims& d, int S, const void* x, const f
 // states[b][h][j] = sum_s B_s o exp(c_127 - c_s) x_s^T over 128-token block j
 // ([B][H][nblk][N][P]) and the block totals tot[b][h][j][n] = c_127[n]
 bool diag_state_tc_supported(const Dims& d);
-cudaError_t launch_diag_state_tc(const Dims& d, const void* x, const float* a, const void* Bm,
+// decay: a [B][T][H][N], or (from_cum, 128-token chunks) the step-1 prefix sums;
+// tot may be null
+cudaError_t launch_diag_state_tc(const Dims& d, const void* x, const float* decay, bool from_cum, const void* Bm,
                                  float* states, float* tot, int* status, cudaStream_t st);
 
 // Output of the per-state decay (bf16, N = 64, P = 64) on tensor cores, one CTA

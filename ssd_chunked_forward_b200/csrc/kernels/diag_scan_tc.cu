@@ -246,18 +246,28 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int k = 0; k < 32; ++k) sA[g_off(32 * r + k, n)] = ex2_approx(av[k] * kLog2e);
             if (rq_or(false)) goto done;  // group Q holds its C rows
+            // E_t from the prefix sum since the sub-block's start; F_s from the
+            // suffix sum to its end, taken backwards, so that a large decay
+            // before s never enters the sum for s (no cancellation)
             c = 0.f;
 #pragma unroll
             for (int k = 0; k < 32; ++k) {
                 const int t = 32 * r + k;
                 c += av[k];
-                const float F = ex2_approx((cend - c) * kLog2e);
                 const float E = ex2_approx(c * kLog2e);
+                const uint32_t off = tc::sw128_offset(t, n >> 3) + (n & 7) * 2;
+                const float cv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sC + off));
+                *reinterpret_cast<__nv_bfloat16*>(sC + off) = __float2bfloat16_rn(cv * E);
+            }
+            float suf = 0.f;
+#pragma unroll
+            for (int k = 31; k >= 0; --k) {
+                const int t = 32 * r + k;
+                const float F = ex2_approx(suf * kLog2e);
+                suf += av[k];
                 const uint32_t off = tc::sw128_offset(t, n >> 3) + (n & 7) * 2;
                 const float bv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sB + off));
                 *reinterpret_cast<__nv_bfloat16*>(sAz + (r & 1) * kTile + off) = __float2bfloat16_rn(bv * F);
-                const float cv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sC + off));
-                *reinterpret_cast<__nv_bfloat16*>(sC + off) = __float2bfloat16_rn(cv * E);
             }
             tc::fence_proxy_async_smem();
             __syncwarp();

@@ -67,9 +67,10 @@ __device__ __forceinline__ bool group_or(bool pred) {
 
 struct DiagParams {
     float* states;  // [B][H][nblk][N][P]
-    float* tot;     // [B][H][nblk][N]
+    float* tot;     // [B][H][nblk][N] or null
     int* status;
     int T, H, G, nblk, npairs;
+    int from_cum;   // the decay tile holds in-chunk prefix sums (128-token chunks), not a
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -123,7 +124,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::mbar_arrive_expect_tx(&bars->full, 2 * kATile + 4 * kTile);
             for (int jb = 0; jb < 2; ++jb) {
                 const int t0 = (j0 + jb) * kBlk;
-                tc::tma_load_4d(sA + jb * (kBlk * kN), &tm_a, &bars->full, 0, h, t0, b);
+                if (p.from_cum)  // cum [B][H][nc][128][N] viewed as rows of N; a missing block reads zeros
+                    tc::tma_load_4d(sA + jb * (kBlk * kN), &tm_a, &bars->full, 0, 0,
+                                    (bh * p.nblk + (j0 + jb < p.nblk ? j0 + jb : p.nblk)) * kBlk, 0);
+                else
+                    tc::tma_load_4d(sA + jb * (kBlk * kN), &tm_a, &bars->full, 0, h, t0, b);
                 tc::tma_load_4d(sX + jb * kTile, &tm_x, &bars->full, 0, h, t0, b);
                 tc::tma_load_4d(sB + jb * kTile, &tm_b, &bars->full, 0, g, t0, b);
             }
@@ -166,25 +171,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!group_or(!ok || *abort_v != 0)) {
             for (int jb = 0; jb < 2; ++jb) {
                 const float* ab = sA + jb * (kBlk * kN);
-                // the sum of this thread's 64 tokens of column n; the two halves'
-                // sums give the prefix before the upper half and the block total
+                // the sum of this thread's 64 tokens of column n; the block total
+                // is the two halves' sums
                 float part = 0.f;
-                for (int k = 0; k < 64; ++k) part += ab[(64 * half + k) * kN + n];
+                if (!p.from_cum)
+                    for (int k = 0; k < 64; ++k) part += ab[(64 * half + k) * kN + n];
                 sTot[half * kN + n] = part;
                 asm volatile("bar.sync 1, 128;" ::: "memory");
-                const float lower = sTot[n], tot = lower + sTot[kN + n];
-                float c = half == 0 ? 0.f : lower;  // inclusive prefix before this thread's first token
+                const float tot = p.from_cum ? ab[(kBlk - 1) * kN + n] : sTot[n] + sTot[kN + n];
+                // w_s = exp(sum_{u > s} a_u): a suffix sum taken from the block's end
+                // (from the upper half's sum for the lower half), so that a large
+                // decay before s never enters the sum for s; from prefix sums, the
+                // difference to the last one
+                float suf = half == 0 ? sTot[kN + n] : 0.f;
                 const uint8_t* bsrc = sB + jb * kTile;
                 uint8_t* adst = sAz + jb * 2 * kTile + jb * kTile;  // m-half jb, rows of block jb
-                for (int k = 0; k < 64; ++k) {
+                for (int k = 63; k >= 0; --k) {
                     const int s = 64 * half + k;
-                    c += ab[s * kN + n];
-                    const float wgt = ex2_approx((tot - c) * kLog2e);  // exp(sum_{u>s} a_u) <= 1
+                    const float e = p.from_cum ? tot - ab[s * kN + n] : suf;
+                    const float wgt = ex2_approx(e * kLog2e);  // <= 1
+                    if (!p.from_cum) suf += ab[s * kN + n];
                     const uint32_t off = tc::sw128_offset(s, n >> 3) + (n & 7) * 2;
                     const float bv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(bsrc + off));
                     *reinterpret_cast<__nv_bfloat16*>(adst + off) = __float2bfloat16_rn(bv * wgt);
                 }
-                if (half == 0 && j0 + jb < p.nblk)
+                if (half == 0 && p.tot && j0 + jb < p.nblk)
                     p.tot[((size_t)bh * p.nblk + j0 + jb) * kN + n] = tot;
                 asm volatile("bar.sync 1, 128;" ::: "memory");  // sTot is reused by the next block
             }
@@ -229,19 +240,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 bool diag_state_tc_supported(const Dims& d) { return d.bf16 && d.diag && d.N == kN && d.P == kP; }
 
-cudaError_t launch_diag_state_tc(const Dims& d, const void* x, const float* a, const void* Bm,
+cudaError_t launch_diag_state_tc(const Dims& d, const void* x, const float* decay, bool from_cum, const void* Bm,
                                  float* states, float* tot, int* status, cudaStream_t st) {
-    if (!diag_state_tc_supported(d)) return cudaErrorNotSupported;
+    if (!diag_state_tc_supported(d) || (from_cum && d.Q != kBlk)) return cudaErrorNotSupported;
+    const int nblk = (d.T + kBlk - 1) / kBlk;
     CUtensorMap ta, tx, tb;
-    cudaError_t e = make_tmap_f32_4d(&ta, a, d.N, d.H, d.T, d.B, kBlk);
+    cudaError_t e = from_cum ? make_tmap_f32_4d(&ta, decay, d.N, 1, (uint64_t)d.B * d.H * nblk * kBlk, 1, kBlk)
+                             : make_tmap_f32_4d(&ta, decay, d.N, d.H, d.T, d.B, kBlk);
     if (e == cudaSuccess) e = make_tmap_bf16_4d(&tx, x, d.P, d.H, d.T, d.B, kBlk);
     if (e == cudaSuccess) e = make_tmap_bf16_4d(&tb, Bm, d.N, d.G, d.T, d.B, kBlk);
     if (e != cudaSuccess) return e;
     DiagParams p = {};
     p.states = states; p.tot = tot; p.status = status;
     p.T = d.T; p.H = d.H; p.G = d.G;
-    p.nblk = (d.T + kBlk - 1) / kBlk;
+    p.nblk = nblk;
     p.npairs = (p.nblk + 1) / 2;
+    p.from_cum = from_cum ? 1 : 0;
     const long long blocks = (long long)d.B * d.H * p.npairs;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
     e = cudaFuncSetAttribute(diag_state_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);

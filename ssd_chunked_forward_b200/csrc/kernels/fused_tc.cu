@@ -27,23 +27,24 @@
 //
 // The recurrence across blocks: each (b, h) chain hands its fp32 state from
 // block j-1 to block j through a two-slot ring in global memory (it stays in
-// L2) and a per-chain counter of published blocks.  The state never passes
-// through shared memory: the state-step threads load the incoming state from
-// the ring into registers, add the block's own state read from TMEM and store
-// the result to the ring (kept in their register order, so every access is
-// coalesced); a publisher thread then fences once and moves the
-// chain counter, and a poller thread acquires the predecessor's counter and
-// wakes the state-step threads.  Work items
+// L2) and a per-chain counter of published blocks.  A loader thread acquires
+// the predecessor's counter and copies the incoming state into shared memory
+// with one bulk copy (two buffers, so the next head's copy overlaps this
+// head's step); the state-step threads add the block's own state read from
+// TMEM and store the result to the ring straight from registers (kept in
+// their register order, so every access is coalesced); a publisher thread
+// then fences once and moves the chain counter.  Work items
 // are ordered block-major and dealt round-robin to persistent CTAs, so the
 // block a CTA waits for always belongs to a smaller item index and can finish;
 // every wait is bounded and reports a timeout instead of hanging.
 //
 // Warp roles (640 threads):
-//   warp 0  lane 0 streams x tiles (TMA, four stages); lane 1 loads the B
-//           (double-buffered) and C tiles; lane 2 issues the output products
-//   warp 1  owns TMEM; lane 0 issues S and Z; lane 1 publishes the outgoing
-//           states (one gpu-scope fence, then the chain counter)
-//   warp 2  lane 0 polls the chain counters
+//   warp 0  lane 0 streams x tiles (TMA, two stages); lane 1 loads the B and
+//           C tiles of an item; lane 2 issues the output products
+//   warp 1  owns TMEM; lane 0 issues S and Z
+//   warp 2  lane 0 polls the chain counters and copies each incoming state
+//           into one of two shared-memory buffers; lane 1 publishes the
+//           outgoing states (one gpu-scope fence, then the chain counter)
 //   warp 3  in-block prefix sums of the decays (one item ahead)
 //   4-11    group A: per-head decay vectors, w o X, P and C~ (thread = tile row,
 //           two warps per TMEM lane quadrant splitting the columns)
@@ -64,7 +65,7 @@ constexpr int kBlk = 128;
 constexpr int kN = 128;
 constexpr int kP = 64;
 constexpr int kHpbMax = 8;
-constexpr int kXStages = 3;
+constexpr int kXStages = 2;
 constexpr int kThreads = 640;
 constexpr uint32_t kTile = kBlk * 128;  // 128 rows x 128 bytes (bf16)
 
@@ -76,14 +77,14 @@ constexpr uint32_t COL_CB = 320;
 constexpr uint32_t COL_ZY = 384;  // + 64 * buffer
 
 struct __align__(8) Bars {
-    uint64_t b_full[2], b_empty[2], c_full, c_empty;
+    uint64_t b_full, b_empty, c_full, c_empty;
     uint64_t s_full, s_free;
     uint64_t x_full[kXStages], x_empty[kXStages];
-    uint64_t xw_full[2], xw_free[2];
+    uint64_t xw_full, xw_free;
     uint64_t a_full[2], p_free[2], ct_free;
     uint64_t z_full[2], sh_full, sh_free;
     uint64_t y_full[2], zy_free[2];
-    uint64_t hin_ready[2], hin_taken[2];
+    uint64_t hin_full[2], hin_free[2];
     uint64_t pub_ready[2], pub_done[2];
     uint64_t cum_full[2], cum_free[2];
     uint64_t done_sz, done_y;
@@ -106,11 +107,12 @@ struct FusedParams {
 };
 
 // shared memory (offsets from the 1024-aligned base)
-constexpr uint32_t OFF_B = 0;                               // 2 slots x two 64-column boxes
-constexpr uint32_t OFF_C = OFF_B + 4 * kTile;               // two boxes
+constexpr uint32_t OFF_B = 0;                               // two 64-column boxes
+constexpr uint32_t OFF_C = OFF_B + 2 * kTile;               // two boxes
 constexpr uint32_t OFF_X = OFF_C + 2 * kTile;               // kXStages tiles
-constexpr uint32_t OFF_XW = OFF_X + kXStages * kTile;       // two buffers
-constexpr uint32_t OFF_H = OFF_XW + 2 * kTile;              // bf16 Hin, [n][p]
+constexpr uint32_t OFF_XW = OFF_X + kXStages * kTile;       // w o X
+constexpr uint32_t OFF_HIN = OFF_XW + kTile;                // 2 x fp32 incoming state (ring order)
+constexpr uint32_t OFF_H = OFF_HIN + 4 * kTile;             // bf16 Hin, [n][p]
 constexpr uint32_t OFF_Y = OFF_H + kTile;                   // bf16 y staging for the TMA store
 constexpr uint32_t OFF_CUM = OFF_Y + kTile;                 // [2][kHpbMax][128] fp32
 constexpr uint32_t OFF_VEC = OFF_CUM + 2 * kHpbMax * kBlk * 4;  // 6 x [128] fp32
@@ -192,6 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* sXw = sm + OFF_XW;
     uint8_t* sH = sm + OFF_H;
     uint8_t* sY = sm + OFF_Y;
+    float* sHin = reinterpret_cast<float*>(sm + OFF_HIN);
     float* sCum = reinterpret_cast<float*>(sm + OFF_CUM);  // [2][kHpbMax][128]
     float* sC2 = reinterpret_cast<float*>(sm + OFF_VEC);   // cum * log2(e)
     float* sW = sC2 + kBlk;                                // exp(cum_127 - cum_s)
@@ -207,22 +210,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
-            tc::mbar_init(&bars->b_full[s], 1);
-            tc::mbar_init(&bars->b_empty[s], 1);   // the item's last Z product
-            tc::mbar_init(&bars->xw_full[s], 8);   // group A warps
-            tc::mbar_init(&bars->xw_free[s], 1);   // Z product
+            tc::mbar_init(&bars->hin_full[s], 1);  // loader (+ the bulk copy's bytes)
+            tc::mbar_init(&bars->hin_free[s], 8);  // group B read the incoming state
+
             tc::mbar_init(&bars->a_full[s], 8);    // group A: P and C~ written
             tc::mbar_init(&bars->p_free[s], 1);    // output product
             tc::mbar_init(&bars->z_full[s], 1);    // Z product
             tc::mbar_init(&bars->y_full[s], 1);    // output product
             tc::mbar_init(&bars->zy_free[s], 8);   // group B read the output
-            tc::mbar_init(&bars->hin_ready[s], 1); // poller
-            tc::mbar_init(&bars->hin_taken[s], 8); // group B passed hin_ready
+
             tc::mbar_init(&bars->pub_ready[s], 8); // group B stored an outgoing state
             tc::mbar_init(&bars->pub_done[s], 1);  // the publisher released it
             tc::mbar_init(&bars->cum_full[s], 1);  // decay warp
             tc::mbar_init(&bars->cum_free[s], 16); // groups A and B
         }
+        tc::mbar_init(&bars->xw_full, 8);     // group A warps
+        tc::mbar_init(&bars->xw_free, 1);     // Z product
+        tc::mbar_init(&bars->b_full, 1);
+        tc::mbar_init(&bars->b_empty, 1);     // the item's last Z product
         tc::mbar_init(&bars->c_full, 1);
         tc::mbar_init(&bars->c_empty, 9);  // S product + group A's copy into TMEM
         tc::mbar_init(&bars->s_full, 1);
@@ -283,11 +288,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int it = blockIdx.x; it < p.n_items; it += gridDim.x) {
                 const Item w = decode_item(it, p);
                 const int t0 = w.j * kBlk;
-                const uint32_t sl = nb & 1;
-                if (nb >= 2 && !wait(&bars->b_empty[sl], ((nb >> 1) - 1) & 1)) { ok = false; break; }
-                tc::mbar_arrive_expect_tx(&bars->b_full[sl], 2 * kTile);
-                tc::tma_load_4d(sB + sl * 2 * kTile, &tm_b, &bars->b_full[sl], 0, w.g, t0, w.b);
-                tc::tma_load_4d(sB + sl * 2 * kTile + kTile, &tm_b, &bars->b_full[sl], 64, w.g, t0, w.b);
+                if (nb >= 1 && !wait(&bars->b_empty, (nb - 1) & 1)) { ok = false; break; }
+                tc::mbar_arrive_expect_tx(&bars->b_full, 2 * kTile);
+                tc::tma_load_4d(sB, &tm_b, &bars->b_full, 0, w.g, t0, w.b);
+                tc::tma_load_4d(sB + kTile, &tm_b, &bars->b_full, 64, w.g, t0, w.b);
                 ++nb;
                 if (ncl >= 1 && !wait(&bars->c_empty, (ncl - 1) & 1)) { ok = false; break; }
                 tc::mbar_arrive_expect_tx(&bars->c_full, 2 * kTile);
@@ -297,8 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok) fail();
             // no copy may still be landing in shared memory when the CTA exits
-            for (uint32_t c = nb > 2 ? nb - 2 : 0; c < nb; ++c)
-                tc::mbar_wait(&bars->b_full[c & 1], (c >> 1) & 1, nullptr, 200000000ull);
+            if (nb > 0) tc::mbar_wait(&bars->b_full, (nb - 1) & 1, nullptr, 200000000ull);
             if (ncl > 0) tc::mbar_wait(&bars->c_full, (ncl - 1) & 1, nullptr, 200000000ull);
         } else if (lane == 2) {
             // =========================== output products y = [P | C~] [X ; Hin] ====
@@ -315,17 +318,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!ok) break;
                     tc::tc_fence_after();
                     const uint32_t acc = tmem + COL_ZY + 64 * s;
+                    // the incoming-state half first, so that its operands free early
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)  // K = n: C~ from TMEM, Hin MN-major
+                        tc::mma_ts(acc, tmem + COL_CT + kk * 8, tc::desc_adv(dH, kk * 2048), id_y, kk > 0);
+                    tc::mma_commit(&bars->sh_free);
+                    tc::mma_commit(&bars->ct_free);
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)  // K = s: P from TMEM, X MN-major
                         tc::mma_ts(acc, tmem + COL_P + 64 * s + kk * 8,
-                                   tc::desc_adv(dX, st * kTile + kk * 2048), id_y, kk > 0);
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)  // K = n: C~ from TMEM, Hin MN-major
-                        tc::mma_ts(acc, tmem + COL_CT + kk * 8, tc::desc_adv(dH, kk * 2048), id_y, 1);
+                                   tc::desc_adv(dX, st * kTile + kk * 2048), id_y, 1);
                     tc::mma_commit(&bars->y_full[s]);
                     tc::mma_commit(&bars->p_free[s]);
-                    tc::mma_commit(&bars->ct_free);
-                    tc::mma_commit(&bars->sh_free);
                     tc::mma_commit(&bars->x_empty[st]);
                 }
             }
@@ -345,8 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t hc = 0, itc = 0;
             bool ok = true;
             for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x, ++itc) {
-                const uint32_t sl = itc & 1;
-                ok = wait(&bars->b_full[sl], (itc >> 1) & 1) && wait(&bars->c_full, itc & 1) &&
+                ok = wait(&bars->b_full, itc & 1) && wait(&bars->c_full, itc & 1) &&
                      (itc == 0 || wait(&bars->s_free, (itc - 1) & 1));
                 if (!ok) break;
                 tc::tc_fence_after();
@@ -354,31 +357,80 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * kTile + (kk & 3) * 32;
-                    tc::mma_ss(tmem + COL_S, tc::desc_adv(dC, off), tc::desc_adv(dBk, sl * 2 * kTile + off), id_s,
-                               kk > 0);
+                    tc::mma_ss(tmem + COL_S, tc::desc_adv(dC, off), tc::desc_adv(dBk, off), id_s, kk > 0);
                 }
                 tc::mma_commit(&bars->s_full);
                 tc::mma_commit(&bars->c_empty);
                 for (int i = 0; i < p.hpb; ++i, ++hc) {
                     // Z = B^T (w o X): M = n (MN-major B tile), N = p, K = s
                     const uint32_t s = hc & 1, u = hc >> 1;
-                    ok = wait(&bars->xw_full[s], u & 1) && (u == 0 || wait(&bars->zy_free[s], (u - 1) & 1));
+                    ok = wait(&bars->xw_full, hc & 1) && (u == 0 || wait(&bars->zy_free[s], (u - 1) & 1));
                     if (!ok) break;
                     tc::tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        tc::mma_ss(tmem + COL_ZY + 64 * s, tc::desc_adv(dBm, sl * 2 * kTile + kk * 2048),
-                                   tc::desc_adv(dXw, s * kTile + kk * 2048), id_z, kk > 0);
+                        tc::mma_ss(tmem + COL_ZY + 64 * s, tc::desc_adv(dBm, kk * 2048),
+                                   tc::desc_adv(dXw, kk * 2048), id_z, kk > 0);
+                    tc::mma_commit(&bars->xw_free);
                     tc::mma_commit(&bars->z_full[s]);
-                    tc::mma_commit(&bars->xw_free[s]);
                 }
                 if (!ok) break;
-                tc::mma_commit(&bars->b_empty[sl]);
+                tc::mma_commit(&bars->b_empty);
             }
             if (!ok) fail();
             // every product issued must be complete before TMEM is released
             tc::mma_commit(&bars->done_sz);
             tc::mbar_wait(&bars->done_sz, 0, nullptr, 200000000ull);
+        }
+    } else if (warp == 2) {
+        if (lane == 0) {
+            // ================================ incoming-state loader ====
+            // waits for the predecessor block's counter, then copies its state
+            // (32 KB, in the ring's thread order) into shared memory in one bulk
+            // copy; block 0 copies the given initial state ([n][p]) or nothing
+            uint32_t hc = 0;
+            bool ok = true;
+            for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x) {
+                const Item w = decode_item(it, p);
+                for (int i = 0; i < p.hpb; ++i, ++hc) {
+                    const int chain = w.b * p.H + w.h0 + i;
+                    // group B has read the state two heads back from this buffer
+                    const uint32_t hs = hc & 1, hu = hc >> 1;
+                    float* dst = sHin + hs * (kN * kP);
+                    if (hu > 0 && !wait(&bars->hin_free[hs], (hu - 1) & 1)) { ok = false; break; }
+                    if (w.j > 0) {
+                        const unsigned* f = p.flags + (w.b * p.H + w.h0 + i);
+                        const uint64_t t0 = tc::globaltimer_ns();
+                        uint32_t nap = 16;
+                        for (uint32_t spin = 0; ld_acquire_u32(f) < (unsigned)w.j; ++spin) {
+                            if ((spin & 7) == 7) {
+                                if (*abort_v || (p.status && *(volatile int*)p.status) ||
+                                    tc::globaltimer_ns() - t0 > 2000000000ull) {
+                                    ok = false;
+                                    break;
+                                }
+                            }
+                            __nanosleep(nap);
+                            if (nap < 128) nap <<= 1;
+                        }
+                        if (!ok) break;
+                        tc::fence_proxy_async_global();  // the acquire orders the bulk read
+                        tc::mbar_arrive_expect_tx(&bars->hin_full[hs], kN * kP * 4);
+                        tc::bulk_load(dst, p.ring + (size_t)(chain * 2 + ((w.j - 1) & 1)) * (kN * kP), kN * kP * 4,
+                                      &bars->hin_full[hs]);
+                    } else if (p.init) {
+                        const size_t ic = ((size_t)(w.b % p.seg) * p.B0 + w.b / p.seg) * p.H + w.h0 + i;
+                        tc::mbar_arrive_expect_tx(&bars->hin_full[hs], kN * kP * 4);
+                        tc::bulk_load(dst, p.init + ic * (kN * kP), kN * kP * 4, &bars->hin_full[hs]);
+                    } else {
+                        tc::mbar_arrive(&bars->hin_full[hs]);  // a zero state: nothing to load
+                    }
+                }
+            }
+            if (!ok) fail();
+            // no copy may still be landing in shared memory when the CTA exits
+            for (uint32_t c = hc > 2 ? hc - 2 : 0; c < hc; ++c)
+                tc::mbar_wait(&bars->hin_full[c & 1], (c >> 1) & 1, nullptr, 200000000ull);
         } else if (lane == 1) {
             // ============================================ state publisher ====
             // Group B stores each outgoing state straight from registers and
@@ -397,39 +449,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int chain = w.b * p.H + w.h0 + i;
                     if (!(p.test_stall && chain == 0 && w.j == 0)) st_relaxed_u32(p.flags + chain, (unsigned)(w.j + 1));
                     tc::mbar_arrive(&bars->pub_done[s]);
-                }
-            }
-            if (!ok) fail();
-        }
-    } else if (warp == 2) {
-        if (lane == 0) {
-            // ============================================= chain poller ====
-            uint32_t hc = 0;
-            bool ok = true;
-            for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x) {
-                const Item w = decode_item(it, p);
-                for (int i = 0; i < p.hpb; ++i, ++hc) {
-                    const uint32_t s = hc & 1, u = hc >> 1;
-                    // the slot's previous head was taken by group B
-                    if (u > 0 && !wait(&bars->hin_taken[s], (u - 1) & 1)) { ok = false; break; }
-                    if (w.j > 0) {
-                        const unsigned* f = p.flags + (w.b * p.H + w.h0 + i);
-                        const uint64_t t0 = tc::globaltimer_ns();
-                        uint32_t nap = 16;
-                        for (uint32_t spin = 0; ld_acquire_u32(f) < (unsigned)w.j; ++spin) {
-                            if ((spin & 7) == 7) {
-                                if (*abort_v || (p.status && *(volatile int*)p.status) ||
-                                    tc::globaltimer_ns() - t0 > 2000000000ull) {
-                                    ok = false;
-                                    break;
-                                }
-                            }
-                            __nanosleep(nap);
-                            if (nap < 128) nap <<= 1;
-                        }
-                        if (!ok) break;
-                    }
-                    tc::mbar_arrive(&bars->hin_ready[s]);
                 }
             }
             if (!ok) fail();
@@ -554,11 +573,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     group_sync();
                     // ---- T2: w o X for the block state
                     bool ok = wait(&bars->x_full[st], (hc / kXStages) & 1) &&
-                              (u == 0 || wait(&bars->xw_free[s], (u - 1) & 1));
+                              (hc == 0 || wait(&bars->xw_free, (hc - 1) & 1));
                     if (!sync_ok(ok)) { alive = false; break; }
                     {
                         const uint8_t* xs = sX + st * kTile;
-                        uint8_t* xw = sXw + s * kTile;
+                        uint8_t* xw = sXw;
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             const int c = gt + 256 * q;
@@ -575,7 +594,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc::fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        tc::mbar_arrive(&bars->xw_full[s]);
+                        tc::mbar_arrive(&bars->xw_full);
                         tc::mbar_arrive(&bars->x_empty[st]);
                     }
                     // ---- T3: P = S o L + D I -> bf16 -> TMEM (A operand of the output)
@@ -591,36 +610,38 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float rowf = quad > 0 ? ex2_approx(r2 - sC2[32 * quad - 1]) : 0.f;
                         const float* colf = sColf + (quad > 0 ? (quad - 1) * kBlk : 0);
                         const uint32_t pcol = COL_P + 64 * s;
+                        // this warp's 64 columns as four 16-column pieces (two per
+                        // 32-column sub-block sb; rolled loops keep the code small)
 #pragma unroll 1
-                        for (int k = 0; k < 2; ++k) {
-                            const int sb = 2 * cg + k;
-                            const int s0 = 32 * sb;
-                            uint32_t pk[16];
+                        for (int k = 0; k < 4; ++k) {
+                            const int sb = 2 * cg + (k >> 1);
+                            const int s0 = 32 * sb + 16 * (k & 1);  // first column of the piece
+                            uint32_t pk[8];
                             if (sb > quad) {
                                 // above the diagonal P is zero for every head: written
                                 // once per buffer, never overwritten
                                 if (u != 0) continue;
 #pragma unroll
-                                for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                                for (int e = 0; e < 8; ++e) pk[e] = 0u;
                             } else {
-                                float v[32];
-                                tc::tmem_ld32(lane_base + COL_S + s0, v);
+                                float v[16];
+                                tc::tmem_ld16(lane_base + COL_S + s0, v);
                                 tc::tmem_ld_wait();
                                 if (sb < quad) {
                                     const float4* cf = reinterpret_cast<const float4*>(colf + s0);
                                     const float2 rr = make_float2(rowf, rowf);
                                     float2* v2 = reinterpret_cast<float2*>(v);
 #pragma unroll
-                                    for (int e4 = 0; e4 < 8; ++e4) {
+                                    for (int e4 = 0; e4 < 4; ++e4) {
                                         const float4 f = cf[e4];
                                         v2[2 * e4] = tc::mul2(v2[2 * e4], tc::mul2(rr, make_float2(f.x, f.y)));
                                         v2[2 * e4 + 1] = tc::mul2(v2[2 * e4 + 1], tc::mul2(rr, make_float2(f.z, f.w)));
                                     }
                                 } else {
                                     const float4* c2 = reinterpret_cast<const float4*>(sC2 + s0);
-                                    const int rl = row - s0;  // the diagonal's column in the sub-block
+                                    const int rl = row - s0;  // the diagonal's column in the piece
 #pragma unroll
-                                    for (int e4 = 0; e4 < 8; ++e4) {
+                                    for (int e4 = 0; e4 < 4; ++e4) {
                                         const float4 f = c2[e4];
                                         const float m[4] = {f.x, f.y, f.z, f.w};
 #pragma unroll
@@ -633,9 +654,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     }
                                 }
 #pragma unroll
-                                for (int e = 0; e < 16; ++e) pk[e] = tc::pack_bf16x2(v[2 * e], v[2 * e + 1]);
+                                for (int e = 0; e < 8; ++e) pk[e] = tc::pack_bf16x2(v[2 * e], v[2 * e + 1]);
                             }
-                            tc::tmem_st16(lane_base + pcol + (s0 >> 1), pk);
+                            tc::tmem_st8(lane_base + pcol + (s0 >> 1), pk);
                         }
                     }
                     // ---- T4: C~ = exp(cum_t) C -> bf16 -> TMEM (the output's second K block)
@@ -645,15 +666,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     {
                         const float ec = sEc[row];
                         const float2 e2 = make_float2(ec, ec);
-                        float v[32];
-                        tc::tmem_ld32(lane_base + COL_CB + 32 * cg, v);
-                        tc::tmem_ld_wait();
-#pragma unroll
+#pragma unroll 1
                         for (int h2 = 0; h2 < 2; ++h2) {
+                            float v[16];
+                            tc::tmem_ld16(lane_base + COL_CB + 32 * cg + 16 * h2, v);
+                            tc::tmem_ld_wait();
                             uint32_t pk[16];
 #pragma unroll
                             for (int e = 0; e < 16; ++e) {
-                                const uint32_t u2 = __float_as_uint(v[16 * h2 + e]);
+                                const uint32_t u2 = __float_as_uint(v[e]);
                                 const float2 r = tc::mul2(tc::unpack_bf16x2(u2), e2);
                                 pk[e] = tc::pack_bf16x2(r.x, r.y);
                             }
@@ -674,45 +695,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         } else {
             // ------------------------------------------------------ group B ----
-            // Per head: the state step (incoming state from the ring, the block's
-            // own state from TMEM, the outgoing state to the ring and the
-            // publish), then the output of the previous head.
-            float hin[32];
-            bool have_next = false;  // hin already holds this head's incoming state
+            // Per head: the state step (incoming state from shared memory, the
+            // block's own state from TMEM, the outgoing state to the ring and
+            // the hand-off to the publisher), then the output of the previous head.
             uint32_t hc = 0, itc = 0, npub = 0;
             bool alive = true;
-            bool prev = false;       // an output of the previous head is pending
+            bool prev = false;  // an output of the previous head is pending
             int prev_b = 0, prev_h = 0, prev_t0 = 0;
             uint32_t prev_s = 0, prev_u = 0;
-
-            // Both helpers decide warp-uniformly before any warp-wide instruction.
-            auto load_hin = [&](int b, int h, int j, uint32_t s, uint32_t u) -> bool {
-                if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->hin_ready[s], u & 1, abort_v))) return false;
-                if (lane == 0) tc::mbar_arrive(&bars->hin_taken[s]);
-                const int chain = b * p.H + h;
-                if (j > 0) {
-                    // the predecessor's state, in the ring's thread order (coalesced)
-                    const float* src = p.ring + (size_t)(chain * 2 + ((j - 1) & 1)) * (kN * kP);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float4 v = ld_cg_f4(src + ring_f4(quad, cg, q, lane));
-                        hin[4 * q] = v.x; hin[4 * q + 1] = v.y; hin[4 * q + 2] = v.z; hin[4 * q + 3] = v.w;
-                    }
-                } else if (p.init) {
-                    // the given initial state, [n][p] (read once per chain)
-                    const size_t ic = ((size_t)(b % p.seg) * p.B0 + b / p.seg) * p.H + h;
-                    const float* src = p.init + (ic * kN + row) * kP + 32 * cg;
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float4 v = ld_cg_f4(src + 4 * q);
-                        hin[4 * q] = v.x; hin[4 * q + 1] = v.y; hin[4 * q + 2] = v.z; hin[4 * q + 3] = v.w;
-                    }
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) hin[e] = 0.f;
-                }
-                return true;
-            };
             auto output = [&]() -> bool {
                 // y of the previous head: TMEM -> bf16 -> shared staging -> one TMA
                 // store (rows past T are not written)
@@ -752,70 +742,82 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t s = hc & 1, u = hc >> 1;
                     const int h = w.h0 + i;
                     const int chain = w.b * p.H + h;
-                    // ---- incoming state (unless prefetched), the block's own state
-                    bool ok = have_next || load_hin(w.b, h, w.j, s, u);
-                    have_next = false;
-                    ok = ok && wait(&bars->z_full[s], u & 1) && (hc == 0 || wait(&bars->sh_free, (hc - 1) & 1));
+                    // ---- the incoming state (shared memory), the block's own state
+                    // (TMEM), the bf16 operand buffer free, the publisher's slot free
+                    const uint32_t ps = npub & 1, pu = npub >> 1;
+                    bool ok = wait(&bars->hin_full[s], u & 1) && wait(&bars->z_full[s], u & 1) &&
+                              (hc == 0 || wait(&bars->sh_free, (hc - 1) & 1)) &&
+                              (last_blk || pu == 0 || wait(&bars->pub_done[ps], (pu - 1) & 1));
                     if (!sync_ok(ok)) { alive = false; break; }
                     tc::tc_fence_after();
-                    float z[32];
-                    tc::tmem_ld32(lane_base + COL_ZY + 64 * s + 32 * cg, z);
-                    // bf16 Hin, rows n, 64 p (MN-major B operand of the output)
+                    // h_j = exp(cum_127) Hin + Z, 16 of this thread's 32 columns at a
+                    // time: Hin also goes to the bf16 operand (rows n, 64 p, MN-major),
+                    // h_j to the ring in the threads' order (coalesced) or, after the
+                    // last block, to the final state ([n][p], once per chain)
+                    const float eL = ex2_approx(cumbuf[i * kBlk + kBlk - 1] * kLog2e);
+                    const float2 e2 = make_float2(eL, eL);
+                    const float* hsrc = sHin + s * (kN * kP);
+                    const bool to_fin = last_blk && p.fin && w.b % p.seg == p.seg - 1;
+                    float* ring_dst = p.ring + (size_t)(chain * 2 + (w.j & 1)) * (kN * kP);
+                    float* fin_dst = p.fin + (((size_t)(w.b / p.seg) * p.H + h) * kN + row) * kP + 32 * cg;
+#pragma unroll 1
+                    for (int hh = 0; hh < 2; ++hh) {
+                        float z[16];
+                        tc::tmem_ld16(lane_base + COL_ZY + 64 * s + 32 * cg + 16 * hh, z);
+                        float hin[16];
+                        if (w.j > 0) {
 #pragma unroll
-                    for (int c8 = 0; c8 < 4; ++c8) {
-                        uint4 v;
-                        v.x = tc::pack_bf16x2(hin[8 * c8 + 0], hin[8 * c8 + 1]);
-                        v.y = tc::pack_bf16x2(hin[8 * c8 + 2], hin[8 * c8 + 3]);
-                        v.z = tc::pack_bf16x2(hin[8 * c8 + 4], hin[8 * c8 + 5]);
-                        v.w = tc::pack_bf16x2(hin[8 * c8 + 6], hin[8 * c8 + 7]);
-                        *reinterpret_cast<uint4*>(sH + tc::sw128_offset(row, 4 * cg + c8)) = v;
+                            for (int q = 0; q < 4; ++q) {
+                                const float4 v = *reinterpret_cast<const float4*>(hsrc + ring_f4(quad, cg, 4 * hh + q, lane));
+                                hin[4 * q] = v.x; hin[4 * q + 1] = v.y; hin[4 * q + 2] = v.z; hin[4 * q + 3] = v.w;
+                            }
+                        } else if (p.init) {
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                const float4 v = *reinterpret_cast<const float4*>(hsrc + row * kP + 32 * cg + 16 * hh + 4 * q);
+                                hin[4 * q] = v.x; hin[4 * q + 1] = v.y; hin[4 * q + 2] = v.z; hin[4 * q + 3] = v.w;
+                            }
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) hin[e] = 0.f;
+                        }
+#pragma unroll
+                        for (int c8 = 0; c8 < 2; ++c8) {
+                            uint4 v;
+                            v.x = tc::pack_bf16x2(hin[8 * c8 + 0], hin[8 * c8 + 1]);
+                            v.y = tc::pack_bf16x2(hin[8 * c8 + 2], hin[8 * c8 + 3]);
+                            v.z = tc::pack_bf16x2(hin[8 * c8 + 4], hin[8 * c8 + 5]);
+                            v.w = tc::pack_bf16x2(hin[8 * c8 + 6], hin[8 * c8 + 7]);
+                            *reinterpret_cast<uint4*>(sH + tc::sw128_offset(row, 4 * cg + 2 * hh + c8)) = v;
+                        }
+                        tc::tmem_ld_wait();
+                        {
+                            float2* z2 = reinterpret_cast<float2*>(z);
+                            const float2* h2 = reinterpret_cast<const float2*>(hin);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) z2[e] = tc::fma2(e2, h2[e], z2[e]);
+                        }
+                        if (!last_blk) {
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                *reinterpret_cast<float4*>(ring_dst + ring_f4(quad, cg, 4 * hh + q, lane)) =
+                                    make_float4(z[4 * q], z[4 * q + 1], z[4 * q + 2], z[4 * q + 3]);
+                        } else if (to_fin) {
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                *reinterpret_cast<float4*>(fin_dst + 16 * hh + 4 * q) =
+                                    make_float4(z[4 * q], z[4 * q + 1], z[4 * q + 2], z[4 * q + 3]);
+                        }
                     }
-                    tc::tmem_ld_wait();
                     tc::fence_proxy_async_smem();
                     tc::tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) tc::mbar_arrive(&bars->sh_full);  // Hin written and Z read
-                    // ---- h_j = exp(cum_127) Hin + Z, to the ring (or the final state)
-                    const float eL = ex2_approx(cumbuf[i * kBlk + kBlk - 1] * kLog2e);
-                    {
-                        const float2 e2 = make_float2(eL, eL);
-                        float2* z2 = reinterpret_cast<float2*>(z);
-                        const float2* h2 = reinterpret_cast<const float2*>(hin);
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) z2[e] = tc::fma2(e2, h2[e], z2[e]);
+                    if (lane == 0) {
+                        tc::mbar_arrive(&bars->hin_free[s]);
+                        tc::mbar_arrive(&bars->sh_full);  // Hin written and Z read
+                        if (!last_blk) tc::mbar_arrive(&bars->pub_ready[ps]);  // the state is stored
                     }
-                    if (!last_blk) {
-                        // to the ring in the threads' order (coalesced)
-                        float* dst = p.ring + (size_t)(chain * 2 + (w.j & 1)) * (kN * kP);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            *reinterpret_cast<float4*>(dst + ring_f4(quad, cg, q, lane)) =
-                                make_float4(z[4 * q], z[4 * q + 1], z[4 * q + 2], z[4 * q + 3]);
-                    } else if (p.fin && w.b % p.seg == p.seg - 1) {
-                        // the final state, [n][p] (once per chain)
-                        float* dst = p.fin + (((size_t)(w.b / p.seg) * p.H + h) * kN + row) * kP + 32 * cg;
-#pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            *reinterpret_cast<float4*>(dst + 4 * q) = make_float4(z[4 * q], z[4 * q + 1], z[4 * q + 2], z[4 * q + 3]);
-                    }
-                    if (!last_blk) {
-                        // hand the stored state to the publisher (its slot's previous
-                        // publish is done, so the barrier phase cannot be overtaken)
-                        const uint32_t ps = npub & 1, pu = npub >> 1;
-                        if (!sync_ok(pu == 0 || wait(&bars->pub_done[ps], (pu - 1) & 1))) { alive = false; break; }
-                        __syncwarp();
-                        if (lane == 0) tc::mbar_arrive(&bars->pub_ready[ps]);
-                        ++npub;
-                    }
-                    // ---- prefetch the next head's incoming state when it is ready
-                    int it2, i2;
-                    if (next_head(it, i, p, it2, i2)) {
-                        const uint32_t s2 = (hc + 1) & 1, u2 = (hc + 1) >> 1;
-                        if (__all_sync(0xffffffffu, tc::mbar_try_wait(&bars->hin_ready[s2], u2 & 1))) {
-                            const Item w2 = decode_item(it2, p);
-                            have_next = load_hin(w2.b, w2.h0 + i2, w2.j, s2, u2);
-                        }
-                    }
+                    if (!last_blk) ++npub;
                     // ---- the previous head's output
                     if (prev && !output()) { alive = false; break; }
                     prev = true;

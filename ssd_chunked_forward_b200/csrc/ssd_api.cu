@@ -240,7 +240,7 @@ ssd_status run_modular(const Dims& d0, const void* x, const float* a, const void
         Dims blk = d0;
         blk.Q = 1;  // the pass reads one total per block: a "chunk" of one position
         blk.nc = (d0.T + 127) / 128;
-        cudaError_t e = ssd::launch_diag_state_tc(d0, x, a, Bm, dw.states, dw.tot, w.ctrl, st);
+        cudaError_t e = ssd::launch_diag_state_tc(d0, x, a, false, Bm, dw.states, dw.tot, w.ctrl, st);
         if (e == cudaSuccess) e = ssd::launch_state_pass(blk, dw.tot, dw.states, fin, init, st);
         if (e == cudaSuccess) e = ssd::launch_diag_scan_tc(d0, x, a, false, Bm, Cm, dw.states, D, y, w.ctrl, st);
         return cuda_status(e);
@@ -344,6 +344,11 @@ int ssd_path_supported(const ssd_shape* shape, unsigned path) {
         case SSD_PATH_SPLIT: return split_pieces(d) > 1 ? 1 : 0;
         default: return 0;
     }
+}
+
+int ssd_split_pieces(const ssd_shape* shape) {
+    if (!shape || check_shape(shape) != SSD_OK) return 0;
+    return split_pieces(dims_of(shape));
 }
 
 int ssd_auto_path(const ssd_shape* shape) {
@@ -529,11 +534,14 @@ ssd_status ssd_chunk_state(const ssd_shape* shape, const void* x, const void* Bm
         return SSD_ERR_INVALID_ARG;
     if (impl > SSD_IMPL_TC) return SSD_ERR_INVALID_ARG;
     const Dims d = dims_of(shape);
-    const bool tc_ok = ssd::chunk_state_tc_supported(d);
+    const bool diag_tc = ssd::diag_state_tc_supported(d) && d.Q == 128;
+    const bool tc_ok = ssd::chunk_state_tc_supported(d) || diag_tc;
     if (impl == SSD_IMPL_TC && !tc_ok) return SSD_ERR_UNSUPPORTED;
     if (injected_failure()) return SSD_ERR_CUDA;
     const bool use_tc = impl == SSD_IMPL_TC || (impl == SSD_IMPL_AUTO && tc_ok);
     cudaStream_t cs = (cudaStream_t)stream;
+    if (use_tc && diag_tc)  // per-state decay: from the step-1 prefix sums
+        return cuda_status(ssd::launch_diag_state_tc(d, x, cum, true, Bm, states, nullptr, nullptr, cs));
     return cuda_status(use_tc ? ssd::launch_chunk_state_tc(d, x, Bm, cum, states, cs)
                               : ssd::launch_chunk_state_simt(d, x, Bm, cum, states, cs));
 }

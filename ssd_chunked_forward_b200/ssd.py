@@ -28,7 +28,7 @@ EXPORTS = [
     "ssd_forward_host", "ssd_forward_noalloc", "ssd_auto_path", "ssd_forward_init",
     "ssd_decode_step", "ssd_discretize", "ssd_decay_total", "ssd_state_combine",
     "ssd_segment_state", "ssd_backward", "ssd_backward_workspace_size",
-    "ssd_test_fail_calls", "ssd_test_pending_failures",
+    "ssd_test_fail_calls", "ssd_test_pending_failures", "ssd_split_pieces",
 ]
 
 
@@ -66,6 +66,8 @@ def load(path: str = LIB_PATH):
     lib.ssd_path_supported.restype = ctypes.c_int
     lib.ssd_auto_path.argtypes = [sp]
     lib.ssd_auto_path.restype = ctypes.c_int
+    lib.ssd_split_pieces.argtypes = [sp]
+    lib.ssd_split_pieces.restype = ctypes.c_int
     lib.ssd_forward.argtypes = [sp, vp, fp, vp, vp, fp, vp, fp, vp, sz, vp]
     lib.ssd_forward_path.argtypes = [sp, vp, fp, vp, vp, fp, vp, fp, vp, sz, vp, ctypes.c_uint, ctypes.c_uint]
     lib.ssd_forward_init.argtypes = [sp, vp, fp, vp, vp, fp, fp, vp, fp, vp, sz, vp, ctypes.c_uint,
@@ -150,6 +152,11 @@ def auto_path(shape: Shape) -> int:
     """The path SSD_PATH_AUTO takes for this shape (PATH_FUSED, PATH_SPLIT or
     PATH_MODULAR)."""
     return int(load().ssd_auto_path(ctypes.byref(shape)))
+
+
+def split_pieces(shape: Shape) -> int:
+    """Pieces per sequence of the split path (1: not split, 0: invalid)."""
+    return int(load().ssd_split_pieces(ctypes.byref(shape)))
 
 
 def alloc_workspace(shape: Shape, device=None) -> torch.Tensor:

@@ -212,8 +212,10 @@ def test_diag_broadcast_equals_scalar():
     a4 = dev["a"].unsqueeze(-1).expand(*dev["a"].shape, w.N).contiguous()
     y2, f2 = ssd.forward(dev["x"], a4, dev["Bm"], dev["Cm"], dev["D"], w.chunk)
     torch.cuda.synchronize()
+    # the per-state path rounds its tensor-core operands (B o w) to bf16, the
+    # scalar path for N = 64 runs on CUDA cores in fp32: both within the bf16 bar
     assert rel_err(y2.float().cpu().numpy(), y1.float().cpu().numpy()) <= TOL_BF16
-    assert rel_err(f2.cpu().numpy(), f1.cpu().numpy()) <= 1e-3
+    assert rel_err(f2.cpu().numpy(), f1.cpu().numpy()) <= TOL_BF16
 
 
 def test_grouping_equals_replication():
