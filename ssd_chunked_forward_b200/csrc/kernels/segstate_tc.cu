@@ -48,8 +48,8 @@ struct __align__(8) SegBars {
 constexpr uint32_t OFF_B = 0;                          // 2 stages x two 64-column boxes
 constexpr uint32_t OFF_X = OFF_B + 4 * kTile;          // kXStages tiles
 constexpr uint32_t OFF_XW = OFF_X + kXStages * kTile;  // two buffers
-constexpr uint32_t OFF_RED = OFF_XW + 2 * kTile;       // [4] warp totals
-constexpr uint32_t OFF_BAR = OFF_RED + 64;
+constexpr uint32_t OFF_RED = OFF_XW + 2 * kTile;       // [4][kHpbMax] warp totals
+constexpr uint32_t OFF_BAR = OFF_RED + 4 * kHpbMax * 4;
 constexpr uint32_t OFF_MISC = OFF_BAR + ((sizeof(SegBars) + 15) / 16) * 16;
 constexpr size_t kSmemBytes = 1024 + OFF_MISC + 16;
 static_assert(kSmemBytes <= 232448, "shared memory above the 227 KB per-block limit");
@@ -190,53 +190,97 @@ __global__ void __launch_bounds__(kThreads, 1)
                 : "memory");
             return r != 0;
         };
+        // this thread's token of a block, all the slice's heads (contiguous in
+        // memory: one 16-byte load when they line up); tokens past the piece
+        // decay by 1: a = 0
+        const bool vec = (p.H & 3) == 0 && (h0 & 3) == 0 && (p.hpb & 3) == 0;
+        auto load_a = [&](int jb, float (&dst)[kHpbMax]) {
+            const int tt = (p.nblk - 1 - jb) * kBlk + t;
+            const float* row = p.a + ((size_t)bv * p.L + tt) * p.H + h0;
+#pragma unroll
+            for (int i4 = 0; i4 < kHpbMax / 4; ++i4) {
+                float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (tt < p.L && 4 * i4 < p.hpb) {
+                    if (vec) {
+                        f = __ldg(reinterpret_cast<const float4*>(row) + i4);
+                    } else {
+                        f.x = __ldg(row + 4 * i4);
+                        f.y = 4 * i4 + 1 < p.hpb ? __ldg(row + 4 * i4 + 1) : 0.f;
+                        f.z = 4 * i4 + 2 < p.hpb ? __ldg(row + 4 * i4 + 2) : 0.f;
+                        f.w = 4 * i4 + 3 < p.hpb ? __ldg(row + 4 * i4 + 3) : 0.f;
+                    }
+                }
+                dst[4 * i4] = f.x; dst[4 * i4 + 1] = f.y; dst[4 * i4 + 2] = f.z; dst[4 * i4 + 3] = f.w;
+            }
+        };
+        float anext[kHpbMax];
+        load_a(0, anext);
         bool ok = true;
-        for (int q = 0; q < nq; ++q) {
-            const int jb = q / p.hpb, i = q - jb * p.hpb;
-            const int tt = (p.nblk - 1 - jb) * kBlk + t;  // token within the piece
-            const float av = tt < p.L ? __ldg(p.a + ((size_t)bv * p.L + tt) * p.H + h0 + i) : 0.f;
-            // inclusive prefix sum over the block's 128 tokens
-            const float wsum = warp_inclusive_scan(av);
-            if (lane == 31) sRed[tw] = wsum;
+        for (int jb = 0; ok && jb < p.nblk; ++jb) {
+            float av[kHpbMax];
+#pragma unroll
+            for (int i = 0; i < kHpbMax; ++i) av[i] = anext[i];
+            if (jb + 1 < p.nblk) load_a(jb + 1, anext);  // one block ahead
+            // w_t = exp(sum of a over the tokens after t up to the piece's end):
+            // suffix sums taken directly (a difference of prefix sums would
+            // cancel in fp32 when one token decays by thousands)
+            float excl[kHpbMax];
+#pragma unroll
+            for (int i = 0; i < kHpbMax; ++i) {
+                float v = av[i];
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float u = __shfl_down_sync(0xffffffffu, v, o);
+                    if (lane + o < 32) v += u;
+                }
+                const float nx = __shfl_down_sync(0xffffffffu, v, 1);
+                excl[i] = lane < 31 ? nx : 0.f;
+                if (lane == 0) sRed[tw * kHpbMax + i] = v;  // the warp's total
+            }
             asm volatile("bar.sync 1, 128;" ::: "memory");
-            float off = 0.f, total = 0.f;
+            float wgt[kHpbMax];
 #pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                const float r = sRed[w];
-                off += w < tw ? r : 0.f;
-                total += r;
+            for (int i = 0; i < kHpbMax; ++i) {
+                float later = 0.f, total = 0.f;
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    const float r = sRed[w * kHpbMax + i];
+                    later += w > tw ? r : 0.f;
+                    total += r;
+                }
+                wgt[i] = ex2_approx(((excl[i] + later) + carry[i]) * kLog2e);
+                carry[i] += total;
             }
-            const float cum = wsum + off;
-            float ci = 0.f;  // carry of head i (registers stay indexed by constants)
+            for (int i = 0; i < p.hpb; ++i) {
+                const int q = jb * p.hpb + i;
+                float wi = 0.f;  // registers stay indexed by constants
 #pragma unroll
-            for (int k = 0; k < kHpbMax; ++k) ci = k == i ? carry[k] : ci;
-            const float wgt = ex2_approx(((total - cum) + ci) * kLog2e);
+                for (int k = 0; k < kHpbMax; ++k) wi = k == i ? wgt[k] : wi;
+                const uint32_t st = q % kXStages, s = q & 1;
+                ok = tc::mbar_wait(&bars->x_full[st], (q / kXStages) & 1, abort_v) &&
+                     (q < 2 || tc::mbar_wait(&bars->xw_free[s], ((q >> 1) - 1) & 1, abort_v));
+                if (!ok) fail();
+                // (also orders this block's sRed reads before the next block's writes)
+                if (group_or(!ok || *abort_v != 0)) { ok = false; break; }
+                // row t of x times w_t (the swizzle permutes chunks within the row)
+                const uint8_t* xs = sX + st * kTile + t * 128;
+                uint8_t* xw = sXw + s * kTile + t * 128;
+                const uint32_t w2 = tc::pack_bf16x2(wi, wi);
 #pragma unroll
-            for (int k = 0; k < kHpbMax; ++k) carry[k] = k == i ? ci + total : carry[k];
-            const uint32_t st = q % kXStages, s = q & 1;
-            ok = tc::mbar_wait(&bars->x_full[st], (q / kXStages) & 1, abort_v) &&
-                 (q < 2 || tc::mbar_wait(&bars->xw_free[s], ((q >> 1) - 1) & 1, abort_v));
-            if (!ok) fail();
-            // (also orders this step's sRed reads before the next step's writes)
-            if (group_or(!ok || *abort_v != 0)) { ok = false; break; }
-            // row t of x times w_t (the swizzle permutes chunks within the row)
-            const uint8_t* xs = sX + st * kTile + t * 128;
-            uint8_t* xw = sXw + s * kTile + t * 128;
-            const uint32_t w2 = tc::pack_bf16x2(wgt, wgt);
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint4 v = *reinterpret_cast<const uint4*>(xs + c * 16);
-                v.x = tc::mul_bf16x2(v.x, w2);
-                v.y = tc::mul_bf16x2(v.y, w2);
-                v.z = tc::mul_bf16x2(v.z, w2);
-                v.w = tc::mul_bf16x2(v.w, w2);
-                *reinterpret_cast<uint4*>(xw + c * 16) = v;
-            }
-            tc::fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                tc::mbar_arrive(&bars->xw_full[s]);
-                tc::mbar_arrive(&bars->x_empty[st]);
+                for (int c = 0; c < 8; ++c) {
+                    uint4 v = *reinterpret_cast<const uint4*>(xs + c * 16);
+                    v.x = tc::mul_bf16x2(v.x, w2);
+                    v.y = tc::mul_bf16x2(v.y, w2);
+                    v.z = tc::mul_bf16x2(v.z, w2);
+                    v.w = tc::mul_bf16x2(v.w, w2);
+                    *reinterpret_cast<uint4*>(xw + c * 16) = v;
+                }
+                tc::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tc::mbar_arrive(&bars->xw_full[s]);
+                    tc::mbar_arrive(&bars->x_empty[st]);
+                }
             }
         }
         // ---- drain: thread = state row n, one head at a time
