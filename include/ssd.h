@@ -182,6 +182,14 @@ ssd_status ssd_forward_init(const ssd_shape* shape, const void* x, const float* 
  * error. */
 ssd_status ssd_device_status(const void* workspace, ssd_stream stream);
 
+/* Diagnosis of a timeout: synchronises `stream` and writes where the first
+ * bounded wait that ran out in a fused-path kernel gave up -- the source line
+ * of the wait in the library's kernel file, the block and the thread index --
+ * or zeros when none did.  Any pointer may be null.  Returns as
+ * ssd_device_status(). */
+ssd_status ssd_device_status_where(const void* workspace, ssd_stream stream, int* line, int* block,
+                                   int* thread);
+
 /* ---- the forward from host memory --------------------------------------- */
 
 /* Device bytes ssd_forward_host() needs in `dev_buf` for this shape: staging

@@ -253,10 +253,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::tc_fence_after();
     const uint32_t tmem = *sTmem;
 
-    auto fail = [&]() {
+    // A wait that gives up marks the CTA aborted and sets the status word; the
+    // first one also leaves where it happened in the next three words (source
+    // line, block, thread), for diagnosis.
+    auto fail_at = [&](int line) {
         *reinterpret_cast<volatile int*>(sAbort) = 1;
-        if (p.status) atomicExch(p.status, kDevTimeout);
+        if (p.status) {
+            if (atomicCAS(p.status + 1, 0, line) == 0) {
+                p.status[2] = (int)blockIdx.x;
+                p.status[3] = (int)threadIdx.x;
+            }
+            atomicExch(p.status, kDevTimeout);
+        }
     };
+#define fail() fail_at(__LINE__)
     auto wait = [&](uint64_t* bar, uint32_t parity) -> bool { return tc::mbar_wait(bar, parity, abort_v); };
 
     if (warp == 0) {
@@ -838,6 +848,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem, 512);
     }
+#undef fail
 }
 
 int num_sms() {

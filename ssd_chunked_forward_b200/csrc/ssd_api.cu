@@ -515,6 +515,19 @@ ssd_status ssd_device_status(const void* workspace, ssd_stream stream) {
     return SSD_ERR_CUDA;
 }
 
+ssd_status ssd_device_status_where(const void* workspace, ssd_stream stream, int* line, int* block,
+                                   int* thread) {
+    const ssd_status st = ssd_device_status(workspace, stream);
+    if (st == SSD_ERR_WORKSPACE || st == SSD_ERR_CUDA) return st;
+    int words[4] = {0, 0, 0, 0};
+    if (cudaMemcpy(words, workspace, sizeof(words), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return SSD_ERR_CUDA;
+    if (line) *line = words[1];
+    if (block) *block = words[2];
+    if (thread) *thread = words[3];
+    return st;
+}
+
 ssd_status ssd_chunk_cumsum(const ssd_shape* shape, const float* a, float* cum, ssd_stream stream) {
     ssd_status st = check_shape(shape);
     if (st != SSD_OK) return st;

@@ -29,6 +29,7 @@ EXPORTS = [
     "ssd_decode_step", "ssd_discretize", "ssd_decay_total", "ssd_state_combine",
     "ssd_segment_state", "ssd_backward", "ssd_backward_workspace_size",
     "ssd_test_fail_calls", "ssd_test_pending_failures", "ssd_split_pieces",
+    "ssd_device_status_where",
 ]
 
 
@@ -73,6 +74,8 @@ def load(path: str = LIB_PATH):
     lib.ssd_forward_init.argtypes = [sp, vp, fp, vp, vp, fp, fp, vp, fp, vp, sz, vp, ctypes.c_uint,
                                      ctypes.c_uint]
     lib.ssd_device_status.argtypes = [vp, vp]
+    ip = ctypes.POINTER(ctypes.c_int)
+    lib.ssd_device_status_where.argtypes = [vp, vp, ip, ip, ip]
     lib.ssd_chunk_cumsum.argtypes = [sp, fp, fp, vp]
     lib.ssd_chunk_state.argtypes = [sp, vp, vp, fp, fp, vp, ctypes.c_uint]
     lib.ssd_state_pass.argtypes = [sp, fp, fp, fp, vp]
@@ -98,7 +101,7 @@ def load(path: str = LIB_PATH):
                  "ssd_device_status", "ssd_chunk_cumsum", "ssd_decode_step", "ssd_discretize",
                  "ssd_decay_total", "ssd_state_combine", "ssd_segment_state", "ssd_backward",
                  "ssd_chunk_state", "ssd_state_pass", "ssd_chunk_scan", "ssd_diag_scan",
-                 "ssd_forward_host"):
+                 "ssd_forward_host", "ssd_device_status_where"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -219,6 +222,15 @@ def forward(x, a, Bm, Cm, D=None, chunk=256, *, y=None, final_state=None, want_f
 def device_status(workspace, stream=None) -> int:
     """Synchronise and return the workspace status word (SSD_OK or an error)."""
     return int(load().ssd_device_status(_ptr(workspace), _stream(stream)))
+
+
+def device_status_where(workspace, stream=None):
+    """(status, source line, block, thread) of the first bounded wait that ran
+    out in a fused-path kernel; zeros when none did."""
+    line, block, thread = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    st = int(load().ssd_device_status_where(_ptr(workspace), _stream(stream), ctypes.byref(line),
+                                            ctypes.byref(block), ctypes.byref(thread)))
+    return st, line.value, block.value, thread.value
 
 
 def chunk_cumsum(shape: Shape, a, cum=None, stream=None):

@@ -293,9 +293,12 @@ def test_fused_bounded_wait_reports_timeout():
     ssd.forward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], dev["D"], w.chunk, workspace=ws,
                 path=ssd.PATH_FUSED, flags=ssd.FLAG_TEST_STALL)
     assert ssd.device_status(ws) == ssd.SSD_ERR_TIMEOUT
+    st, line, block, thread = ssd.device_status_where(ws)
+    assert st == ssd.SSD_ERR_TIMEOUT and line > 0 and 0 <= block and 0 <= thread < 1024
     y, fin = ssd.forward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], dev["D"], w.chunk, workspace=ws,
                          path=ssd.PATH_FUSED)
     assert ssd.device_status(ws) == ssd.SSD_OK
+    assert ssd.device_status_where(ws) == (ssd.SSD_OK, 0, 0, 0)
     ey, ef = parity_on_chains(inp, y, fin, _all_chains(w))
     assert ey <= TOL_BF16 and ef <= TOL_BF16
 
