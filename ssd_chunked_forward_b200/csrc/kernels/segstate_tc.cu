@@ -262,18 +262,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) fail();
                 // (also orders this block's sRed reads before the next block's writes)
                 if (group_or(!ok || *abort_v != 0)) { ok = false; break; }
-                // row t of x times w_t (the swizzle permutes chunks within the row)
+                // row t of x times w_t (the swizzle permutes chunks within the row;
+                // every chunk takes the same weight, so each thread starts at its
+                // own chunk and the eight rows of a quarter-warp meet no bank twice)
                 const uint8_t* xs = sX + st * kTile + t * 128;
                 uint8_t* xw = sXw + s * kTile + t * 128;
                 const uint32_t w2 = tc::pack_bf16x2(wi, wi);
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    uint4 v = *reinterpret_cast<const uint4*>(xs + c * 16);
+                    const int cc = (c + t) & 7;
+                    uint4 v = *reinterpret_cast<const uint4*>(xs + cc * 16);
                     v.x = tc::mul_bf16x2(v.x, w2);
                     v.y = tc::mul_bf16x2(v.y, w2);
                     v.z = tc::mul_bf16x2(v.z, w2);
                     v.w = tc::mul_bf16x2(v.w, w2);
-                    *reinterpret_cast<uint4*>(xw + c * 16) = v;
+                    *reinterpret_cast<uint4*>(xw + cc * 16) = v;
                 }
                 tc::fence_proxy_async_smem();
                 __syncwarp();
