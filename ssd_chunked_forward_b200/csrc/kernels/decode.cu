@@ -90,14 +90,98 @@ __global__ void __launch_bounds__(kDecThreads) decode_step_kernel(
     }
 }
 
+// The same step with 16-byte state accesses, for P a multiple of 4 with P/4
+// dividing the block: thread (column group p4 of 4 columns, row slice sl)
+// owns rows sl, sl + ns, ... of those 4 columns, all loaded before anything
+// else waits, few registers, so every block of a batch is resident at once.
+template <typename T, bool DIAG>
+__global__ void __launch_bounds__(kDecThreads, DIAG ? 2 : 3) decode_step_v4_kernel(
+    const T* __restrict__ x, const float* __restrict__ a, const T* __restrict__ Bm,
+    const T* __restrict__ Cm, const float* __restrict__ D, float* __restrict__ state,
+    T* __restrict__ y, int H, int P, int G, int N) {
+    extern __shared__ float sm[];
+    const int pw4 = P >> 2;                 // column groups
+    const int ns = kDecThreads / pw4;       // row slices
+    float* sB = sm;                         // [N]
+    float* sC = sB + N;                     // [N]
+    float* sE = sC + N;                     // [N]
+    float* sX = sE + N;                     // [P]
+    float* sY = sX + P;                     // [ns][P] partial sums of y
+    const int bh = blockIdx.x, b = bh / H, h = bh % H, g = h / (H / G);
+    const int tid = threadIdx.x;
+    const int p4 = tid % pw4, sl = tid / pw4;
+    float4* hs = reinterpret_cast<float4*>(state + (size_t)bh * N * P);
+    constexpr int kR = 4;  // rows per thread (N <= 4 ns)
+    float4 hv[kR];
+#pragma unroll
+    for (int r = 0; r < kR; ++r) {
+        const int n = sl + r * ns;
+        hv[r] = n < N ? hs[(size_t)n * pw4 + p4] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    const float* ab = a + (size_t)bh * (DIAG ? N : 1);
+    for (int n = tid; n < N; n += kDecThreads) {
+        sB[n] = to_f32(Bm[((size_t)b * G + g) * N + n]);
+        sC[n] = to_f32(Cm[((size_t)b * G + g) * N + n]);
+        sE[n] = ex2_approx((DIAG ? ab[n] : ab[0]) * 1.4426950408889634f);
+    }
+    for (int q = tid; q < P; q += kDecThreads) sX[q] = to_f32(x[(size_t)bh * P + q]);
+    __syncthreads();
+    const float4 xv = make_float4(sX[4 * p4], sX[4 * p4 + 1], sX[4 * p4 + 2], sX[4 * p4 + 3]);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int r = 0; r < kR; ++r) {
+        const int n = sl + r * ns;
+        if (n < N) {
+            const float e = sE[n], bn = sB[n], cn = sC[n];
+            float4 hn;
+            hn.x = fmaf(e, hv[r].x, bn * xv.x);
+            hn.y = fmaf(e, hv[r].y, bn * xv.y);
+            hn.z = fmaf(e, hv[r].z, bn * xv.z);
+            hn.w = fmaf(e, hv[r].w, bn * xv.w);
+            hs[(size_t)n * pw4 + p4] = hn;
+            acc.x = fmaf(cn, hn.x, acc.x);
+            acc.y = fmaf(cn, hn.y, acc.y);
+            acc.z = fmaf(cn, hn.z, acc.z);
+            acc.w = fmaf(cn, hn.w, acc.w);
+        }
+    }
+    reinterpret_cast<float4*>(sY)[sl * pw4 + p4] = acc;
+    __syncthreads();
+    for (int q = tid; q < P; q += kDecThreads) {
+        float s = 0.f;
+        for (int k = 0; k < ns; ++k) s += sY[k * P + q];
+        y[(size_t)bh * P + q] = from_f32<T>(s + (D ? D[h] : 0.f) * sX[q]);
+    }
+}
+
+bool decode_v4_ok(const Dims& d) {
+    if (d.P % 4 != 0) return false;
+    const int pw4 = d.P / 4;
+    if (pw4 > kDecThreads || kDecThreads % pw4 != 0) return false;
+    return d.N <= 4 * (kDecThreads / pw4);
+}
+
 }  // namespace
 
 cudaError_t launch_decode_step(const Dims& d, const void* x, const float* a, const void* Bm,
                                const void* Cm, const float* D, float* state, void* y,
                                cudaStream_t st) {
+    const unsigned grid = (unsigned)(d.B * d.H);
+    if (decode_v4_ok(d)) {
+        const size_t smem4 = (size_t)(3 * d.N + d.P + (kDecThreads / (d.P / 4)) * d.P) * sizeof(float);
+#define SSD_DEC4_LAUNCH(TT, DG)                                                                   \
+    decode_step_v4_kernel<TT, DG><<<grid, kDecThreads, smem4, st>>>(                              \
+        (const TT*)x, a, (const TT*)Bm, (const TT*)Cm, D, state, (TT*)y, d.H, d.P, d.G, d.N)
+        if (d.bf16) {
+            if (d.diag) SSD_DEC4_LAUNCH(__nv_bfloat16, true); else SSD_DEC4_LAUNCH(__nv_bfloat16, false);
+        } else {
+            if (d.diag) SSD_DEC4_LAUNCH(float, true); else SSD_DEC4_LAUNCH(float, false);
+        }
+#undef SSD_DEC4_LAUNCH
+        return cudaGetLastError();
+    }
     const int pw = d.P < kDecThreads ? d.P : kDecThreads;
     const size_t smem = (size_t)(3 * d.N + d.P + (kDecThreads / pw) * pw) * sizeof(float);
-    const unsigned grid = (unsigned)(d.B * d.H);
 #define SSD_DEC_LAUNCH(TT, DG)                                                                    \
     decode_step_kernel<TT, DG><<<grid, kDecThreads, smem, st>>>(                                  \
         (const TT*)x, a, (const TT*)Bm, (const TT*)Cm, D, state, (TT*)y, d.H, d.P, d.G, d.N)
