@@ -176,6 +176,22 @@ ssd_status ssd_forward_init(const ssd_shape* shape, const void* x, const float* 
                             void* workspace, size_t ws_bytes, ssd_stream stream, unsigned path,
                             unsigned flags);
 
+/* The selective discretisation and the forward in one pass: the result of
+ * ssd_discretize() (dt = softplus(dt_raw + dt_bias), a = -dt exp(A_log),
+ * x_out = dt x; "State Space Models and Mamba ...", llms.blog, "The Selection
+ * Mechanism") fed to ssd_forward(), without writing x_out or a: the fused
+ * kernel forms dt and a in its decay scan and scales each x tile by dt in
+ * shared memory, so y = SSD(dt x, a, Bm, Cm) + D (dt x).  dt scales x after
+ * rounding to bf16 (a relative change below 2^-8 of each token's input).
+ * x[B][T][H][P] bf16, dt_raw[B][T][H] fp32, dt_bias[H] fp32 or NULL,
+ * A_log[H] fp32; the rest as ssd_forward (same workspace size).  Served for
+ * the fused path's shapes (bf16, N = 128, P = 64, chunk % 128 == 0, scalar
+ * decay), else SSD_ERR_UNSUPPORTED (call ssd_discretize, then ssd_forward). */
+ssd_status ssd_forward_discretized(const ssd_shape* shape, const void* x, const float* dt_raw,
+                                   const float* dt_bias, const float* A_log, const void* Bm,
+                                   const void* Cm, const float* D, void* y, float* final_state,
+                                   void* workspace, size_t ws_bytes, ssd_stream stream);
+
 /* Synchronises `stream`, then returns the status word a previous
  * ssd_forward* call on this workspace left (SSD_OK, or SSD_ERR_TIMEOUT when
  * a bounded device wait ran out), or SSD_ERR_CUDA when the stream reports an

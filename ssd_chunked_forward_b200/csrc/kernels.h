@@ -100,10 +100,17 @@ size_t fused_ring_bytes(const Dims& d);
 // seg > 1: the B rows of d are pieces of B / seg longer sequences (row b is
 // piece b % seg of sequence b / seg); piece k of sequence b starts from
 // init[(k * (B / seg) + b)] and the last piece writes the final state fin[b].
+// The discretisation in front of the operator, done inside the fused kernel:
+// dt = softplus(dt_raw + dt_bias), a = -dt exp(A_log), input dt x.
+struct Discretisation {
+    const float* dt_raw;   // [B,T,H]
+    const float* dt_bias;  // [H] or null
+    const float* A_log;    // [H]
+};
 cudaError_t launch_fused_tc(const Dims& d, const void* x, const float* a, const void* Bm,
                             const void* Cm, const float* D, void* y, float* fin, float* ring,
                             unsigned* flags, int* status, bool test_stall, cudaStream_t st,
-                            const float* init = nullptr, int seg = 1);
+                            const float* init = nullptr, int seg = 1, const Discretisation* disc = nullptr);
 
 // The state each piece of a sequence builds from a zero start and the piece's
 // total log-decay: the [B][T] rows viewed as [B*S][T/S] pieces (T % S == 0);
@@ -141,6 +148,7 @@ cudaError_t launch_fused_ordered(const Dims& d, const void* x, const float* a, c
                                  const void* Cm, const float* D, void* y, float* fin, float* ring,
                                  unsigned* flags, int* status, bool test_stall, cudaStream_t st,
                                  const float* init = nullptr, void* clear = nullptr,
-                                 size_t clear_bytes = 0, int seg = 1);
+                                 size_t clear_bytes = 0, int seg = 1,
+                                 const Discretisation* disc = nullptr);
 
 }  // namespace ssd

@@ -92,6 +92,11 @@ struct __align__(8) Bars {
 
 struct FusedParams {
     const float* a;        // log-decays [B,T,H]
+    // discretisation in front (when dt_raw is set; a is then unused):
+    // dt = softplus(dt_raw + dt_bias), a = -dt exp(A_log), the input dt x
+    const float* dt_raw;   // [B,T,H]
+    const float* dt_bias;  // [H] or null
+    const float* A_log;    // [H]
     const float* D;        // [H] or null
     const float* init;     // [B*H][N][P] initial states or null (zero)
     float* ring;           // [B*H][2][N][P]
@@ -117,7 +122,8 @@ constexpr uint32_t OFF_Y = OFF_H + kTile;                   // bf16 y staging fo
 constexpr uint32_t OFF_CUM = OFF_Y + kTile;                 // [2][kHpbMax][128] fp32
 constexpr uint32_t OFF_VEC = OFF_CUM + 2 * kHpbMax * kBlk * 4;  // 6 x [128] fp32
 constexpr uint32_t OFF_DV = OFF_VEC + 6 * kBlk * 4;         // [2][kHpbMax]
-constexpr uint32_t OFF_BAR = OFF_DV + 2 * kHpbMax * 4;
+constexpr uint32_t OFF_DT = OFF_DV + 2 * kHpbMax * 4;     // [2][kHpbMax][128] bf16 steps dt
+constexpr uint32_t OFF_BAR = OFF_DT + 2 * kHpbMax * kBlk * 2;
 constexpr uint32_t OFF_MISC = OFF_BAR + ((sizeof(Bars) + 15) / 16) * 16;
 constexpr size_t kSmemBytes = 1024 + OFF_MISC + 16;
 static_assert(kSmemBytes <= 232448, "shared memory above the 227 KB per-block limit");
@@ -201,6 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* sColf = sW + kBlk;                              // [3][128]
     float* sEc = sColf + 3 * kBlk;                         // exp(cum_t)
     float* sDv = reinterpret_cast<float*>(sm + OFF_DV);    // [2][kHpbMax]
+    __nv_bfloat16* sDt = reinterpret_cast<__nv_bfloat16*>(sm + OFF_DT);  // [2][kHpbMax][128]
     Bars* bars = reinterpret_cast<Bars*>(sm + OFF_BAR);
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
     int* sAbort = reinterpret_cast<int*>(sm + OFF_MISC + 4);
@@ -479,10 +486,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             // decay by 1: a = 0
             float av[4][kHpbMax];
             const bool vec = (p.H & 3) == 0 && (w.h0 & 3) == 0 && (p.hpb & 3) == 0;
+            const float* src = p.dt_raw ? p.dt_raw : p.a;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int t = tb + q;
-                const float* row = p.a + ((size_t)w.b * p.T + t) * p.H + w.h0;
+                const float* row = src + ((size_t)w.b * p.T + t) * p.H + w.h0;
 #pragma unroll
                 for (int i4 = 0; i4 < kHpbMax / 4; ++i4) {
                     float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -497,6 +505,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                     av[q][4 * i4] = f.x; av[q][4 * i4 + 1] = f.y; av[q][4 * i4 + 2] = f.z; av[q][4 * i4 + 3] = f.w;
+                }
+            }
+            if (p.dt_raw) {
+                // the discretisation: dt = softplus(dt_raw + dt_bias) (kept as bf16
+                // for the input's scaling), a = -dt exp(A_log)
+#pragma unroll
+                for (int i = 0; i < kHpbMax; ++i) {
+                    if (i >= p.hpb) break;
+                    const float bias = p.dt_bias ? __ldg(p.dt_bias + w.h0 + i) : 0.f;
+                    const float A = -expf(__ldg(p.A_log + w.h0 + i));
+                    __nv_bfloat16* dtb = sDt + (buf * kHpbMax + i) * kBlk + lane * 4;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float z = av[q][i] + bias;
+                        const float dt = tb + q < p.T ? fmaxf(z, 0.f) + log1pf(expf(-fabsf(z))) : 0.f;
+                        dtb[q] = __float2bfloat16_rn(dt);
+                        av[q][i] = dt * A;
+                    }
                 }
             }
 #pragma unroll
@@ -586,7 +612,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                               (hc == 0 || wait(&bars->xw_free, (hc - 1) & 1));
                     if (!sync_ok(ok)) { alive = false; break; }
                     {
-                        const uint8_t* xs = sX + st * kTile;
+                        uint8_t* xs = sX + st * kTile;
                         uint8_t* xw = sXw;
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
@@ -594,6 +620,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const float wgt = sW[c >> 3];
                             const uint32_t w2 = tc::pack_bf16x2(wgt, wgt);
                             uint4 v = *reinterpret_cast<const uint4*>(xs + c * 16);
+                            if (p.dt_raw) {
+                                // the discretised input dt x, in place for the output product
+                                const __nv_bfloat16 dtb = sDt[(buf * kHpbMax + i) * kBlk + (c >> 3)];
+                                const uint32_t d2 = (uint32_t)__bfloat16_as_ushort(dtb) * 0x10001u;
+                                v.x = tc::mul_bf16x2(v.x, d2);
+                                v.y = tc::mul_bf16x2(v.y, d2);
+                                v.z = tc::mul_bf16x2(v.z, d2);
+                                v.w = tc::mul_bf16x2(v.w, d2);
+                                *reinterpret_cast<uint4*>(xs + c * 16) = v;
+                            }
                             v.x = tc::mul_bf16x2(v.x, w2);
                             v.y = tc::mul_bf16x2(v.y, w2);
                             v.z = tc::mul_bf16x2(v.z, w2);
@@ -879,7 +915,7 @@ size_t fused_ring_bytes(const Dims& d) { return (size_t)d.B * d.H * 2 * kN * kP 
 cudaError_t launch_fused_tc(const Dims& d, const void* x, const float* a, const void* Bm,
                             const void* Cm, const float* D, void* y, float* fin, float* ring,
                             unsigned* flags, int* status, bool test_stall, cudaStream_t st,
-                            const float* init, int seg) {
+                            const float* init, int seg, const Discretisation* disc) {
     if (!fused_supported(d) || seg < 1 || d.B % seg != 0) return cudaErrorNotSupported;
     CUtensorMap tx, tb, tcm, ty;
     // [B][T][heads or groups][64 or 128]: a block running past T reads zeros
@@ -893,6 +929,11 @@ cudaError_t launch_fused_tc(const Dims& d, const void* x, const float* a, const 
     p.a = a;
     p.D = D;
     p.init = init;
+    if (disc) {
+        p.dt_raw = disc->dt_raw;
+        p.dt_bias = disc->dt_bias;
+        p.A_log = disc->A_log;
+    }
     p.ring = ring;
     p.flags = flags;
     p.fin = fin;

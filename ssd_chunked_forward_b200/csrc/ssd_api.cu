@@ -274,7 +274,8 @@ bool take_injected_failure() {
 cudaError_t launch_fused_ordered(const Dims& d, const void* x, const float* a, const void* Bm,
                                  const void* Cm, const float* D, void* y, float* fin, float* ring,
                                  unsigned* flags, int* status, bool test_stall, cudaStream_t st,
-                                 const float* init, void* clear, size_t clear_bytes, int seg) {
+                                 const float* init, void* clear, size_t clear_bytes, int seg,
+                                 const Discretisation* disc) {
     cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
     if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) return cudaErrorInvalidValue;
     int dev = 0;
@@ -284,7 +285,7 @@ cudaError_t launch_fused_ordered(const Dims& d, const void* x, const float* a, c
             cudaError_t e = cudaMemsetAsync(clear, 0, clear_bytes, st);
             if (e != cudaSuccess) return e;
         }
-        return launch_fused_tc(d, x, a, Bm, Cm, D, y, fin, ring, flags, status, test_stall, st, init, seg);
+        return launch_fused_tc(d, x, a, Bm, Cm, D, y, fin, ring, flags, status, test_stall, st, init, seg, disc);
     }
     std::lock_guard<std::mutex> lock(g_fused_mu);
     if (!g_fused_done[dev]) {
@@ -299,7 +300,7 @@ cudaError_t launch_fused_ordered(const Dims& d, const void* x, const float* a, c
         cudaError_t e = cudaMemsetAsync(clear, 0, clear_bytes, st);
         if (e != cudaSuccess) return e;
     }
-    cudaError_t e = launch_fused_tc(d, x, a, Bm, Cm, D, y, fin, ring, flags, status, test_stall, st, init, seg);
+    cudaError_t e = launch_fused_tc(d, x, a, Bm, Cm, D, y, fin, ring, flags, status, test_stall, st, init, seg, disc);
     if (e != cudaSuccess) return e;
     e = cudaEventRecord(g_fused_done[dev], st);
     if (e == cudaSuccess) g_fused_seen[dev] = true;
@@ -418,6 +419,32 @@ ssd_status ssd_forward_init(const ssd_shape* shape, const void* x, const float* 
         default:
             return run_modular(d, x, a, Bm, Cm, D, y, final_state, w, cs, true, initial_state, workspace);
     }
+}
+
+ssd_status ssd_forward_discretized(const ssd_shape* shape, const void* x, const float* dt_raw,
+                                  const float* dt_bias, const float* A_log, const void* Bm,
+                                  const void* Cm, const float* D, void* y, float* final_state,
+                                  void* workspace, size_t ws_bytes, ssd_stream stream) {
+    if (!shape) return SSD_ERR_INVALID_ARG;
+    ssd_status st = check_shape(shape);
+    if (st != SSD_OK) return st;
+    if (!x || !dt_raw || !A_log || !Bm || !Cm || !y) return SSD_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(dt_raw) || !aligned16(A_log) || !aligned16(Bm) || !aligned16(Cm) ||
+        !aligned16(y) || (D && !aligned16(D)) || (dt_bias && !aligned16(dt_bias)) ||
+        (final_state && !aligned16(final_state)))
+        return SSD_ERR_INVALID_ARG;
+    const Dims d = dims_of(shape);
+    if (d.diag || !ssd::fused_supported(d)) return SSD_ERR_UNSUPPORTED;
+    if (!workspace || ((uintptr_t)workspace % kAlign) != 0) return SSD_ERR_WORKSPACE;
+    if (ws_bytes < ssd_workspace_size(shape)) return SSD_ERR_WORKSPACE;
+    cudaStream_t cs = (cudaStream_t)stream;
+    const Workspace w = carve(workspace, d);
+    if (injected_failure()) return SSD_ERR_CUDA;
+    // status word and per-chain counters start at zero on every call
+    if (cudaMemsetAsync(w.ctrl, 0, kCtrlBytes + flags_bytes(d), cs) != cudaSuccess) return SSD_ERR_CUDA;
+    const ssd::Discretisation disc = {dt_raw, dt_bias, A_log};
+    return cuda_status(ssd::launch_fused_ordered(d, x, nullptr, Bm, Cm, D, y, final_state, w.ring, w.flags,
+                                                 w.ctrl, false, cs, nullptr, nullptr, 0, 1, &disc));
 }
 
 ssd_status ssd_forward_path(const ssd_shape* shape, const void* x, const float* a, const void* Bm,

@@ -29,7 +29,7 @@ EXPORTS = [
     "ssd_decode_step", "ssd_discretize", "ssd_decay_total", "ssd_state_combine",
     "ssd_segment_state", "ssd_backward", "ssd_backward_workspace_size",
     "ssd_test_fail_calls", "ssd_test_pending_failures", "ssd_split_pieces",
-    "ssd_device_status_where",
+    "ssd_device_status_where", "ssd_forward_discretized",
 ]
 
 
@@ -87,6 +87,7 @@ def load(path: str = LIB_PATH):
     lib.ssd_forward_noalloc.argtypes = [sp, vp, fp, vp, vp, fp, vp, fp, vp]
     lib.ssd_decode_step.argtypes = [sp, vp, fp, vp, vp, fp, fp, vp, vp]
     lib.ssd_discretize.argtypes = [sp, fp, fp, fp, vp, fp, vp, vp]
+    lib.ssd_forward_discretized.argtypes = [sp, vp, fp, fp, fp, vp, vp, fp, vp, fp, vp, sz, vp]
     lib.ssd_decay_total.argtypes = [sp, fp, fp, vp]
     lib.ssd_state_combine.argtypes = [sp, ctypes.c_int, fp, fp, fp, fp, vp]
     lib.ssd_segment_state.argtypes = [sp, vp, fp, vp, fp, fp, vp, sz, vp]
@@ -101,7 +102,7 @@ def load(path: str = LIB_PATH):
                  "ssd_device_status", "ssd_chunk_cumsum", "ssd_decode_step", "ssd_discretize",
                  "ssd_decay_total", "ssd_state_combine", "ssd_segment_state", "ssd_backward",
                  "ssd_chunk_state", "ssd_state_pass", "ssd_chunk_scan", "ssd_diag_scan",
-                 "ssd_forward_host", "ssd_device_status_where"):
+                 "ssd_forward_host", "ssd_device_status_where", "ssd_forward_discretized"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -344,6 +345,34 @@ def discretize(dt_raw, dt_bias, A_log, x, *, a_out=None, x_out=None, stream=None
     _check(load().ssd_discretize(ctypes.byref(shape), _ptr(dt_raw), _ptr(dt_bias), _ptr(A_log), _ptr(x),
                                  _ptr(a_out), _ptr(x_out), _stream(stream)), "ssd_discretize")
     return a_out, x_out
+
+
+def forward_discretized(x, dt_raw, dt_bias, A_log, Bm, Cm, D=None, chunk=256, *, y=None, final_state=None,
+                        want_final=True, workspace=None, stream=None):
+    """discretize() followed by forward() in one fused pass (x_out and a are never
+    written): y = SSD(dt x, -dt exp(A_log), Bm, Cm) + D (dt x), dt = softplus(dt_raw
+    + dt_bias).  x [B,T,H,P] bf16, dt_raw [B,T,H] float32, dt_bias [H] or None,
+    A_log [H] float32 (scalar decay only)."""
+    for name, t in (("dt_raw", dt_raw), ("A_log", A_log)):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.float32:
+            raise ValueError(f"{name} must be a contiguous float32 CUDA tensor")
+    B, T, H, P = x.shape
+    if tuple(dt_raw.shape) != (B, T, H) or tuple(A_log.shape) != (H,):
+        raise ValueError("dt_raw must be [B,T,H] and A_log [H]")
+    _check_inputs(x, dt_raw, Bm, Cm, D)
+    shape = shape_of(x, dt_raw, Bm, chunk)
+    N = Bm.shape[3]
+    if y is None:
+        y = torch.empty_like(x)
+    if final_state is None and want_final:
+        final_state = torch.empty((B, H, N, P), dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = alloc_workspace(shape, x.device)
+    _check(load().ssd_forward_discretized(ctypes.byref(shape), _ptr(x), _ptr(dt_raw), _ptr(dt_bias),
+                                          _ptr(A_log), _ptr(Bm), _ptr(Cm), _ptr(D), _ptr(y),
+                                          _ptr(final_state), _ptr(workspace), workspace.numel(),
+                                          _stream(stream)), "ssd_forward_discretized")
+    return y, final_state
 
 
 def decay_total(a, *, out=None, stream=None):

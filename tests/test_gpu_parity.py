@@ -508,6 +508,58 @@ def test_discretize_matches_oracle(per_state, dtype):
     assert rel_err(fin.cpu().numpy().astype(np.float64), ref["final"].reshape(B, H, N, P)) <= tol
 
 
+FUSED_DISC_CASES = [
+    (2, 512, 4, 1, True),    # B, T, H, G, with dt_bias
+    (1, 1000, 8, 2, False),  # ragged last block, grouped, no bias
+    (2, 384, 3, 1, True),    # three heads per item (scalar decay loads)
+]
+
+
+@pytest.mark.parametrize("case", FUSED_DISC_CASES, ids=[f"B{c[0]}_T{c[1]}_H{c[2]}_G{c[3]}" for c in FUSED_DISC_CASES])
+def test_forward_discretized_matches_oracle(case):
+    """ssd_forward_discretized (the discretisation inside the fused forward)
+    against the oracle's fp64 discretisation followed by its recurrence, and
+    against the library's two launches (ssd_discretize, then ssd_forward)."""
+    B, T, H, G, with_bias = case
+    P, N = 64, 128
+    g = torch.Generator().manual_seed(97 + T)
+    dt_raw = (torch.randn((B, T, H), generator=g, dtype=torch.float64) * 1.5 - 2.0).to(torch.float32)
+    dt_bias = torch.randn((H,), generator=g, dtype=torch.float64).to(torch.float32) if with_bias else None
+    A_log = (torch.rand((H,), generator=g, dtype=torch.float64) * math.log(16)).to(torch.float32)
+    x = torch.randn((B, T, H, P), generator=g, dtype=torch.float64).to(torch.bfloat16)
+    Bm = (torch.randn((B, T, G, N), generator=g, dtype=torch.float64) / math.sqrt(N)).to(torch.bfloat16)
+    Cm = (torch.randn((B, T, G, N), generator=g, dtype=torch.float64) / math.sqrt(N)).to(torch.bfloat16)
+    D = torch.randn((H,), generator=g, dtype=torch.float64).to(torch.float32)
+    dev = lambda t: t.cuda() if t is not None else None
+    y, fin = ssd.forward_discretized(dev(x), dev(dt_raw), dev(dt_bias), dev(A_log), dev(Bm), dev(Cm), dev(D), 256)
+    torch.cuda.synchronize()
+    f64 = lambda t: t.to(torch.float64).numpy()
+    bias64 = f64(dt_bias) if dt_bias is not None else np.zeros((H,))
+    a_r, x_r, _ = O.discretize(f64(dt_raw), bias64, f64(A_log), f64(x))
+    ref = O.recurrence(O.Problem(x_r, a_r, f64(Bm), f64(Cm), f64(D)))
+    yr = ref["y"].reshape(B, H, T, P).transpose(0, 2, 1, 3)
+    assert rel_err(y.float().cpu().numpy().astype(np.float64), yr) <= TOL_BF16
+    assert rel_err(fin.cpu().numpy().astype(np.float64), ref["final"].reshape(B, H, N, P)) <= TOL_BF16
+    # the two-launch form of the same computation
+    a2, x2 = ssd.discretize(dev(dt_raw), dev(dt_bias), dev(A_log), dev(x))
+    y2, f2 = ssd.forward(x2, a2, dev(Bm), dev(Cm), dev(D), 256, path=ssd.PATH_FUSED)
+    torch.cuda.synchronize()
+    assert rel_err(y.float().cpu().numpy().astype(np.float64), y2.float().cpu().numpy().astype(np.float64)) <= TOL_BF16
+    assert rel_err(fin.cpu().numpy().astype(np.float64), f2.cpu().numpy().astype(np.float64)) <= TOL_BF16
+
+
+def test_forward_discretized_unsupported_shape():
+    """Shapes the fused path does not serve are refused before any launch."""
+    B, T, H, P, N = 1, 256, 2, 64, 128
+    x = torch.zeros((B, T, H, P), dtype=torch.float32, device="cuda")
+    dt_raw = torch.zeros((B, T, H), dtype=torch.float32, device="cuda")
+    A_log = torch.zeros((H,), dtype=torch.float32, device="cuda")
+    Bm = torch.zeros((B, T, 1, N), dtype=torch.float32, device="cuda")
+    with pytest.raises(ssd.SSDError) as e:
+        ssd.forward_discretized(x, dt_raw, None, A_log, Bm, Bm, None, 256)
+    assert e.value.code == ssd.SSD_ERR_UNSUPPORTED
+
+
 def test_discretize_odd_rows():
     """Rows whose length is not a multiple of 16 bytes (the per-row path)."""
     B, T, H, P, N = 1, 33, 3, 70, 5
