@@ -464,8 +464,9 @@ def backward_flops(w):
 
 def run_backward(args, device):
     """ssd_backward on the workload: dy (and a loss on the final state) in, the
-    six gradients out; L2 flushed before every step.  The backward runs on
-    CUDA cores in fp32, so its roofline is the fp32 FMA rate."""
+    six gradients out; L2 flushed before every step.  Its roofline is the bf16
+    tensor rate where the quadratic forms run on tensor cores, else the fp32
+    FMA rate of the CUDA cores."""
     w = WORKLOADS[args.workload]
     if args.B or args.T:
         w = w.scaled(B=args.B or w.B, T=args.T or w.T, name=w.name + f"_B{args.B or w.B}_T{args.T or w.T}")
@@ -499,6 +500,21 @@ def run_backward(args, device):
     flops = backward_flops(w)
     achieved = flops / (ms / 1e3) / 1e12
     peaks, src = load_peaks()
+    # bf16 heads with N = 128, P = 64 and 128/256-token chunks run the forms and
+    # the chunk states on tensor cores: the roofline is then the bf16 tensor rate
+    tc = (w.dtype == "bf16" and not w.a_per_state and w.N == 128 and w.P == 64
+          and w.chunk in (128, 256))
+    if tc:
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"], "algorithmic_flops_per_step": flops,
+                "kernel": "ssd_backward (13 launches; the four forms and both chunk-state "
+                          "contractions on tensor cores)",
+                "peak_source": f"{src} (bf16_tflops)"}
+    else:
+        roof = {"bound": "alu", "achieved": achieved, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
+                "frac": achieved / FP32_ALU_TFLOPS, "algorithmic_flops_per_step": flops,
+                "kernel": "ssd_backward (13 launches)",
+                "peak_source": "fp32 FMA rate from unit counts and the maximum SM clock"}
     print(json.dumps({
         "metric": "SSD backward tokens/s", "value": tok / (ms / 1e3), "unit": "tokens/s",
         "ms_per_step": ms, "steps": args.steps, "warmup": args.warmup, "dtype": w.dtype,
@@ -506,10 +522,7 @@ def run_backward(args, device):
         "config": {"workload": w.name + "_backward", "B": w.B, "T": w.T, "H": w.H, "P": w.P,
                    "N": w.N, "G": w.G, "chunk": w.chunk, "loss": "sum(dy * y) + <dfinal, final>",
                    "l2": "flushed (256 MB write) before every step"},
-        "roofline": {"bound": "alu", "achieved": achieved, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
-                     "frac": achieved / FP32_ALU_TFLOPS, "algorithmic_flops_per_step": flops,
-                     "kernel": "ssd_backward (13 launches)",
-                     "peak_source": "fp32 FMA rate from unit counts and the maximum SM clock"},
+        "roofline": roof,
         "hbm_view": {"algorithmic_bytes_per_step": byts, "achieved_gbs": byts / (ms / 1e3) / 1e9,
                      "frac_of_measured_hbm": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]},
         "gpu_launches": 13 * args.steps}))

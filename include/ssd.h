@@ -193,7 +193,7 @@ ssd_status ssd_forward_discretized(const ssd_shape* shape, const void* x, const 
                                    void* workspace, size_t ws_bytes, ssd_stream stream);
 
 /* Synchronises `stream`, then returns the status word a previous
- * ssd_forward* call on this workspace left (SSD_OK, or SSD_ERR_TIMEOUT when
+ * ssd_forward* or ssd_backward call on this workspace left (SSD_OK, or SSD_ERR_TIMEOUT when
  * a bounded device wait ran out), or SSD_ERR_CUDA when the stream reports an
  * error. */
 ssd_status ssd_device_status(const void* workspace, ssd_stream stream);
@@ -392,13 +392,18 @@ ssd_status ssd_decode_step(const ssd_shape* shape, const void* x, const float* a
  *            NULL (not wanted), dinit [B][H][N][P] fp32 or NULL (not wanted);
  *            every output is overwritten, none accumulated into
  *   workspace  device memory of ssd_backward_workspace_size(shape) bytes,
- *            256-byte aligned, owned by the caller (recomputed states, the
- *            adjoint chunk states, fp32 per-head partials); reusable once the
- *            call's work on `stream` has finished
+ *            256-byte aligned, owned by the caller (a status word, recomputed
+ *            states, the adjoint chunk states, fp32 per-head partials);
+ *            reusable once the call's work on `stream` has finished;
+ *            ssd_device_status(workspace) reads the call's status word
+ *            (SSD_ERR_TIMEOUT when a bounded device wait ran out)
  * All device pointers, 16-byte aligned; asynchronous on `stream`.  A partial
  * last chunk (T % chunk != 0) is handled as in the forward.  Arithmetic is
- * fp32 on CUDA cores (the recomputed chunk states of bf16 heads with N = 128,
- * P = 64 on tensor cores, bf16 operands with fp32 accumulation).  Returns
+ * fp32 on CUDA cores, except for bf16 heads with N = 128, P = 64: there the
+ * two chunk-state contractions and, for chunks of 128 or 256 tokens, the
+ * four quadratic forms run on tensor cores (bf16 operands -- the masked,
+ * decayed scores and the decay-scaled rows rounded to bf16 -- with fp32
+ * accumulation).  Returns
  * SSD_ERR_INVALID_ARG for a bad shape or pointer, SSD_ERR_UNSUPPORTED for a_per_state with N > 128 (the per-state
  * decay is the diagonal SSM of "On Structured State-Space Duality", item (i);
  * each state row is a scalar-decay system of its own), SSD_ERR_WORKSPACE for a

@@ -65,6 +65,7 @@ struct BackwardArgs {
     float* dinit;         // [B,H,N,P] or null
 };
 struct BackwardScratch {
+    int* status;     // device status word (kDevOk / kDevTimeout), zeroed per call
     float* cum;      // [B,H,nc,Q] ([B,H,nc,Q,N] per-state)
     float* states;   // [B,H,nc,N,P]  states entering each chunk
     float* dstates;  // [B,H,nc,N,P]  adjoint at each chunk's last token
@@ -86,8 +87,17 @@ cudaError_t launch_backward_diag(const Dims& d, const BackwardArgs& g, const Bac
 
 // ---- tensor-core kernels (tcgen05 + TMEM + TMA) ----------------------------
 bool chunk_state_tc_supported(const Dims& d);
+// from_start: weights exp(cum_s) (the adjoint readout state, given C and dy)
 cudaError_t launch_chunk_state_tc(const Dims& d, const void* x, const void* Bm, const float* cum,
-                                  float* states, cudaStream_t st);
+                                  float* states, cudaStream_t st, bool from_start = false,
+                                  int* status = nullptr);
+// the four chunk forms of the scalar-decay backward (y - Dx, dC, dx - D dy,
+// dB per head) as tcgen05 products; bf16, N = 128, P = 64, Q = 128 or 256
+bool backward_forms_tc_supported(const Dims& d);
+cudaError_t launch_backward_forms_tc(const Dims& d, const void* x, const void* dy, const void* Bm,
+                                     const void* Cm, const float* cum, const float* states,
+                                     const float* dstates, float* ytil, float* dCh, float* dxt,
+                                     float* dBh, int* status, cudaStream_t st);
 bool chunk_scan_tc_supported(const Dims& d);
 cudaError_t launch_chunk_scan_tc(const Dims& d, const void* x, const void* Bm, const void* Cm,
                                  const float* cum, const float* Hin, const float* D, void* y,

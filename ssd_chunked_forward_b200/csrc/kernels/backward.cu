@@ -28,6 +28,8 @@
 #include "../kernels.h"
 #include "bwd_tiles.cuh"
 
+#include <type_traits>
+
 namespace ssd {
 namespace {
 
@@ -333,14 +335,20 @@ cudaError_t run_backward_t(const Dims& d, const BackwardArgs& g, const BackwardS
     const Opd oB{g.Bm, d.G * d.N, d.N, d.H / d.G};
     const Opd oC{g.Cm, d.G * d.N, d.N, d.H / d.G};
     cudaError_t e;
-    // y~ (causal; U = C, V = B, Z = x; Hin as N x P)
-    if ((e = launch_form<T, false>(d, oC, oB, ox, w.cum, w.states, d.P, 1, w.ytil, d.N, d.P, st))) return e;
-    // dC per head (causal; U = dy, V = x, Z = B; Hin read as P x N)
-    if ((e = launch_form<T, false>(d, ody, ox, oB, w.cum, w.states, 1, d.P, w.dCh, d.P, d.N, st))) return e;
-    // dx~ (anti-causal; U = B, V = C, Z = dy; G as N x P)
-    if ((e = launch_form<T, true>(d, oB, oC, ody, w.cum, w.dstates, d.P, 1, w.dxt, d.N, d.P, st))) return e;
-    // dB per head (anti-causal; U = x, V = dy, Z = C; G read as P x N)
-    if ((e = launch_form<T, true>(d, ox, ody, oC, w.cum, w.dstates, 1, d.P, w.dBh, d.P, d.N, st))) return e;
+    if (std::is_same<T, __nv_bfloat16>::value && backward_forms_tc_supported(d)) {
+        if ((e = launch_backward_forms_tc(d, g.x, g.dy, g.Bm, g.Cm, w.cum, w.states, w.dstates, w.ytil,
+                                          w.dCh, w.dxt, w.dBh, w.status, st)))
+            return e;
+    } else {
+        // y~ (causal; U = C, V = B, Z = x; Hin as N x P)
+        if ((e = launch_form<T, false>(d, oC, oB, ox, w.cum, w.states, d.P, 1, w.ytil, d.N, d.P, st))) return e;
+        // dC per head (causal; U = dy, V = x, Z = B; Hin read as P x N)
+        if ((e = launch_form<T, false>(d, ody, ox, oB, w.cum, w.states, 1, d.P, w.dCh, d.P, d.N, st))) return e;
+        // dx~ (anti-causal; U = B, V = C, Z = dy; G as N x P)
+        if ((e = launch_form<T, true>(d, oB, oC, ody, w.cum, w.dstates, d.P, 1, w.dxt, d.N, d.P, st))) return e;
+        // dB per head (anti-causal; U = x, V = dy, Z = C; G read as P x N)
+        if ((e = launch_form<T, true>(d, ox, ody, oC, w.cum, w.dstates, 1, d.P, w.dBh, d.P, d.N, st))) return e;
+    }
     {
         dim3 grid(d.nc, d.B * d.H);
         const size_t smem = (size_t)d.Q * sizeof(float);
@@ -380,12 +388,14 @@ cudaError_t launch_backward(const Dims& d, const BackwardArgs& g, const Backward
     // forward states, recomputed: in-chunk cumsum, chunk states, states entering each chunk
     if ((e = launch_chunk_cumsum(d, g.a, w.cum, st))) return e;
     // (the tensor-core chunk-state kernel serves the bf16 Mamba-2 heads)
-    e = chunk_state_tc_supported(d) ? launch_chunk_state_tc(d, g.x, g.Bm, w.cum, w.states, st)
+    e = chunk_state_tc_supported(d) ? launch_chunk_state_tc(d, g.x, g.Bm, w.cum, w.states, st, false, w.status)
                                     : launch_chunk_state_simt(d, g.x, g.Bm, w.cum, w.states, st);
     if (e) return e;
     if ((e = launch_state_pass(d, w.cum, w.states, w.fin, g.init, st))) return e;
     // adjoint states: each chunk's readout term, then the reverse pass
-    if ((e = launch_chunk_dstate_simt(d, g.dy, g.Cm, w.cum, w.dstates, st))) return e;
+    e = chunk_state_tc_supported(d) ? launch_chunk_state_tc(d, g.dy, g.Cm, w.cum, w.dstates, st, true, w.status)
+                                    : launch_chunk_dstate_simt(d, g.dy, g.Cm, w.cum, w.dstates, st);
+    if (e) return e;
     {
         const long long total = (long long)d.B * d.H * d.N * d.P;
         reverse_pass_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(

@@ -4,7 +4,9 @@
 //   S[n, p] = sum_s B[s, n] * w_s * x[s, p],   w_s = exp(cum_{Q-1} - cum_s),
 // the state the chunk builds from a zero start (llms.blog "State Space Models
 // and Mamba ...", "The Chunk-Wise SSD Algorithm", item 3), written to
-// states[b, h, k] as an N x P fp32 tile.
+// states[b, h, k] as an N x P fp32 tile.  With from_start the weight is
+// w_s = exp(cum_s), the decay from the state entering the chunk to token s:
+// given (C, dy) for (B, x) this is the backward's adjoint readout state.
 //
 // As a GEMM: M = n (128), N = p (64), K = s (the chunk, 64/128/256).  Both
 // operands are read straight from the TMA-loaded tiles without transposition:
@@ -59,7 +61,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                           const __grid_constant__ CUtensorMap tm_b, const float* __restrict__ cum,
                           float* __restrict__ states, int T, int H, int G, int nc, int hpb,
-                          int* status) {
+                          int from_start, int* status) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     constexpr uint32_t kTileBytes = Q * 128;  // Q rows of 128 bytes
@@ -193,11 +195,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                  (i == 0 || tc::mbar_wait(&bars->xw_empty, (i - 1) & 1, abort_v));
             if (!ok) set_abort(sAbort, status);
             if (group_sync_or(!ok || *abort_v != 0)) { ok = false; break; }
-            const float cend = sCum[Q - 1];
+            const float cend = from_start ? 0.f : sCum[Q - 1];
+            const float sgn = from_start ? 1.f : -1.f;
             const uint8_t* xs = sX + st * kTileBytes;
             for (int c = ct; c < Q * 8; c += 128) {
                 const int s = c >> 3;  // token row; the 8 chunks of a row share w
-                const float w = __expf(cend - sCum[s]);
+                const float w = __expf(fmaf(sgn, sCum[s], cend));
                 uint4 v = *reinterpret_cast<const uint4*>(xs + c * 16);
                 uint32_t* u = reinterpret_cast<uint32_t*>(&v);
 #pragma unroll
@@ -252,7 +255,7 @@ bool chunk_state_tc_supported(const Dims& d) {
 }
 
 cudaError_t launch_chunk_state_tc(const Dims& d, const void* x, const void* Bm, const float* cum,
-                                  float* states, cudaStream_t st) {
+                                  float* states, cudaStream_t st, bool from_start, int* status) {
     if (!chunk_state_tc_supported(d)) return cudaErrorNotSupported;
     CUtensorMap tx, tb;
     cudaError_t e = make_tmap_bf16_4d(&tx, x, d.P, d.H, d.T, d.B, d.Q);
@@ -269,7 +272,7 @@ cudaError_t launch_chunk_state_tc(const Dims& d, const void* x, const void* Bm, 
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);       \
         if (e != cudaSuccess) return e;                                                       \
         chunk_state_tc_kernel<QQ><<<(unsigned)blocks, kThreads, sm, st>>>(                    \
-            tx, tb, cum, states, d.T, d.H, d.G, d.nc, hpb, nullptr);                          \
+            tx, tb, cum, states, d.T, d.H, d.G, d.nc, hpb, from_start ? 1 : 0, status);       \
     } while (0)
     if (d.Q == 64) SSD_CSTC(64);
     else if (d.Q == 128) SSD_CSTC(128);

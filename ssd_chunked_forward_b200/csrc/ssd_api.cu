@@ -214,7 +214,8 @@ size_t backward_layout(const Dims& d, void* base, ssd::BackwardScratch* w) {
                          &w->ytil, &w->dxt, &w->dBh, &w->dCh};
         for (int i = 0; i < 10; ++i) slots[i] = s[i];
     }
-    size_t off = 0;
+    if (base && w) w->status = (int*)base;  // the status word, as in the forward's workspace
+    size_t off = kCtrlBytes;
     for (int i = 0; i < 10; ++i) {
         if (base && slots[i]) *slots[i] = (float*)((char*)base + off);
         off += round_up(sizes[i], kAlign);
@@ -725,6 +726,7 @@ ssd_status ssd_backward(const ssd_shape* shape, const void* x, const float* a, c
     ssd::BackwardScratch w;
     backward_layout(d, workspace, &w);
     ssd::BackwardArgs g{x, a, Bm, Cm, D, initial_state, dy, dfinal, dx, da, dBm, dCm, dD, dinit};
+    if (cudaMemsetAsync(w.status, 0, kCtrlBytes, (cudaStream_t)stream) != cudaSuccess) return SSD_ERR_CUDA;
     return cuda_status(ssd::launch_backward(d, g, w, (cudaStream_t)stream));
 }
 

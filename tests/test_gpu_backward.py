@@ -35,6 +35,8 @@ CASES = [
     small_case(B=1, T=150, H=4, P=70, N=33, G=2, chunk=64, dtype="f32", seed=82),
     small_case(B=1, T=512, H=4, P=64, N=128, G=1, chunk=256, dtype="bf16", seed=83),
     small_case(B=2, T=300, H=4, P=64, N=128, G=2, chunk=128, dtype="bf16", seed=84),
+    # tensor-core forms: 256-token chunks, grouped B/C, a last chunk of 8 rows
+    small_case(B=2, T=520, H=4, P=64, N=128, G=2, chunk=256, dtype="bf16", seed=87),
     small_case(B=1, T=7, H=2, P=5, N=3, G=1, chunk=7, dtype="f32", seed=85),
     small_case(B=1, T=5, H=1, P=3, N=2, G=1, chunk=1, dtype="f32", seed=86),
 ]
@@ -103,15 +105,20 @@ def test_backward_maximum_sizes(dtype):
 
 
 def test_backward_without_D_and_deterministic():
-    """D = NULL is D = 0 (dx carries no skip term; dD is still sum dy.x), and
-    two calls on the same inputs give bit-identical gradients."""
+    """D = NULL is D = 0 (dx carries no skip term; dD is still sum dy.x), two
+    calls on the same inputs give bit-identical gradients, and the call leaves
+    SSD_OK in its workspace's status word."""
     w = small_case(B=2, T=256, H=4, P=64, N=128, G=2, chunk=128, dtype="bf16", seed=92)
     inp = generate(w)
     dev = to_dev(inp)
     dy, _, dfin = _extras(w, False, True)
+    shape = ssd.shape_of(dev["x"], dev["a"], dev["Bm"], w.chunk)
+    ws = torch.full((ssd.backward_workspace_size(shape),), 7, dtype=torch.uint8, device="cuda")
     run = lambda: ssd.backward(dev["x"], dev["a"], dev["Bm"], dev["Cm"], None, dy.cuda(), w.chunk,
-                               dfinal=dfin.cuda())
-    g1, g2 = run(), run()
+                               dfinal=dfin.cuda(), workspace=ws)
+    g1 = run()
+    assert ssd.device_status(ws) == ssd.SSD_OK
+    g2 = run()
     torch.cuda.synchronize()
     for k in ("dx", "da", "dBm", "dCm", "dD", "dinit"):
         assert torch.equal(g1[k], g2[k]), k
