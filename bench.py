@@ -36,7 +36,7 @@ from ssd_chunked_forward_b200.workloads import WORKLOADS, generate  # noqa: E402
 DEFAULT_WORKLOAD = "mamba2_2p7b"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PATHS = {"auto": ssd.PATH_AUTO, "modular": ssd.PATH_MODULAR, "simt": ssd.PATH_SIMT,
-         "fused": ssd.PATH_FUSED}
+         "fused": ssd.PATH_FUSED, "split": ssd.PATH_SPLIT}
 
 
 # ----------------------------------------------------------------- model ----

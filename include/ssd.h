@@ -417,6 +417,33 @@ ssd_status ssd_backward(const ssd_shape* shape, const void* x, const float* a, c
  * invalid or not served (a_per_state with N > 128). */
 size_t ssd_backward_workspace_size(const ssd_shape* shape);
 
+/* ---- the debug build's index checks ---------------------------------------
+ * The library also comes as a debug build (libssd_debug.so, compiled with
+ * SSD_DEBUG_CHECKS; the Python binding loads it when the environment variable
+ * SSD_DEBUG_CHECKS is 1).  There every global load and store that a kernel
+ * addresses itself (the tensor-memory-accelerator copies are bounded by their
+ * tensor maps) first checks its flat index against the extent of the buffer
+ * the shape gives.  A failed check does not trap and does not touch memory:
+ * it skips the access (a load reads 0), counts the failure and records the
+ * first one (source line in the library's kernel file, block, thread).  The
+ * results of a run without failures are those of the normal build. */
+
+/* 1 in the debug build, 0 in the normal one. */
+int ssd_debug_build(void);
+
+/* Synchronises the device, writes the count of failed checks since the last
+ * call and where the first one failed (line, linear block index, thread;
+ * zeros when none did), then clears the record.  Any pointer may be null.
+ * SSD_ERR_UNSUPPORTED in the normal build; SSD_ERR_CUDA if the device
+ * reports an error. */
+ssd_status ssd_debug_record(int* failed, int* line, int* block, int* thread);
+
+/* Test switch of the debug build: while on (non-zero), every check fails, so
+ * every checked access is skipped and recorded -- the recording path runs
+ * without any index being out of bounds.  SSD_ERR_UNSUPPORTED in the normal
+ * build. */
+ssd_status ssd_debug_fail_all(int on);
+
 #ifdef __cplusplus
 }
 #endif

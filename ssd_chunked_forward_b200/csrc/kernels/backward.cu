@@ -25,6 +25,7 @@
 // products, and the pairs reaching past the chunk end give the boundary term.
 // dB and dC are formed per head and summed over each group's heads.
 #include "../common.cuh"
+#include "../debug_checks.cuh"
 #include "../kernels.h"
 #include "bwd_tiles.cuh"
 
@@ -41,7 +42,11 @@ using bwd::load_mmajor;
 
 // ------------------------------------------------ reverse state pass ----
 // One thread per (b, h, n, p): G_k into slot k of dstates (which held the
-// chunk's own readout term), Gin_0 into dinit.
+// chunk's own readout term), Gin_0 into dinit.  Slots and chunk decays are
+// read in groups of kRevGroup chunks (last chunk first), the next group's
+// loads issued before the current group's updates, so a long chain keeps
+// 2 x kRevGroup loads in flight instead of waiting once per chunk.
+constexpr int kRevGroup = 8;
 __global__ void __launch_bounds__(256) reverse_pass_kernel(const float* __restrict__ cum,
                                                            float* __restrict__ dstates,
                                                            const float* __restrict__ dfinal,
@@ -54,12 +59,38 @@ __global__ void __launch_bounds__(256) reverse_pass_kernel(const float* __restri
     const int r = (int)(e - bh * NP);
     float* sp = dstates + bh * (long long)nc * NP + r;
     const float* ce = cum + bh * (long long)nc * Q + (Q - 1);
+    // the chain's last slot and last decay bound every access below
+    if (!SSD_INB(bh * (long long)nc * NP + (long long)(nc - 1) * NP + r, total * nc) ||
+        !SSD_INB(bh * (long long)nc * Q + (long long)nc * Q - 1, total / NP * nc * Q))
+        return;
+    float sb[kRevGroup], cb[kRevGroup];
+#pragma unroll
+    for (int u = 0; u < kRevGroup; ++u) {
+        const int k = nc - 1 - u;
+        sb[u] = k >= 0 ? sp[(size_t)k * NP] : 0.f;
+        cb[u] = k >= 0 ? ce[(size_t)k * Q] : 0.f;
+    }
     float g = dfinal ? dfinal[bh * NP + r] : 0.f;
-    for (int k = nc - 1; k >= 0; --k) {
-        const float s = sp[(size_t)k * NP];
-        const float dec = expf(ce[(size_t)k * Q]);
-        sp[(size_t)k * NP] = g;
-        g = fmaf(dec, g, s);
+    for (int k0 = nc - 1; k0 >= 0; k0 -= kRevGroup) {
+        float s[kRevGroup], c[kRevGroup];
+#pragma unroll
+        for (int u = 0; u < kRevGroup; ++u) {
+            s[u] = sb[u];
+            c[u] = cb[u];
+            const int kn = k0 - kRevGroup - u;
+            if (kn >= 0) {
+                sb[u] = sp[(size_t)kn * NP];
+                cb[u] = ce[(size_t)kn * Q];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kRevGroup; ++u) {
+            const int k = k0 - u;
+            if (k >= 0) {
+                sp[(size_t)k * NP] = g;
+                g = fmaf(expf(c[u]), g, s[u]);
+            }
+        }
     }
     if (dinit) dinit[bh * NP + r] = g;
 }
@@ -71,6 +102,7 @@ __global__ void __launch_bounds__(256) chunk_dot_kernel(const float* __restrict_
                                                         const float* __restrict__ fin,
                                                         float* __restrict__ out, int NP, int nc) {
     const int k = blockIdx.x, bh = blockIdx.y;
+    if (!SSD_INB(((long long)bh * nc + k + 1) * NP - 1, (long long)gridDim.y * nc * NP)) return;  // whole block
     const float* g = G + ((size_t)bh * nc + k) * NP;
     const float* h = (k + 1 < nc) ? Hin + ((size_t)bh * nc + k + 1) * NP : fin + (size_t)bh * NP;
     float s = 0.f;
@@ -118,6 +150,10 @@ __global__ void __launch_bounds__(256) chunk_form_kernel(Opd U, Opd V, Opd Z,
     const int tk = k * Q;
     const int qv = min(Q, Tlen - tk);  // rows of this chunk before T
     if (i0 >= qv) return;              // a tile wholly past T (the whole block leaves)
+    // the chunk's decays and state lie in their buffers (the whole block leaves if not)
+    if (!SSD_INB(((long long)bh * nc + k + 1) * Q - 1, (long long)gridDim.y * nc * Q) ||
+        !SSD_INB(((long long)bh * nc + k + 1) * NP - 1, (long long)gridDim.y * nc * NP))
+        return;
     const float* cumk = cum + ((size_t)bh * nc + k) * (size_t)Q;
 
     load_kmajor<T, VEC>(UT, U, b, Tlen, tk, i0, qv, h, K, tid);
@@ -214,7 +250,7 @@ __global__ void __launch_bounds__(256) chunk_form_kernel(Opd U, Opd V, Opd Z,
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             const int m = m0 + 4 * c + q;
-            if (m < Mc) o[m] = fmaf(sc, acc2[a][q], acc[a][q]);
+            if (m < Mc && SSD_INB(o - out + m, (long long)gridDim.y * Tlen * Mc)) o[m] = fmaf(sc, acc2[a][q], acc[a][q]);
         }
     }
 }
@@ -235,6 +271,10 @@ __global__ void __launch_bounds__(256) token_grad_kernel(
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tk = k * Q;
     const int qv = min(Q, Tlen - tk);
+    // every row of the chunk, and the chunk's partial sums, lie in their buffers
+    if (!SSD_INB((((long long)b * Tlen + tk + qv - 1) * H + h) * P + P - 1, (long long)gridDim.y * Tlen * P) ||
+        !SSD_INB((long long)bh * nc + k, (long long)gridDim.y * nc))
+        return;  // the whole block
     const float dv = D ? D[h] : 0.f;
     float dsum = 0.f;
     for (int j = warp; j < qv; j += 8) {
@@ -273,7 +313,8 @@ __global__ void dD_reduce_kernel(const float* __restrict__ dDpart, float* __rest
     if (h >= H) return;
     float s = 0.f;
     for (int b = 0; b < B; ++b)
-        for (int k = 0; k < nc; ++k) s += dDpart[((size_t)b * H + h) * nc + k];
+        for (int k = 0; k < nc; ++k)
+            if (SSD_INB(((long long)b * H + h) * nc + k, (long long)B * H * nc)) s += dDpart[((size_t)b * H + h) * nc + k];
     dD[h] = s;
 }
 
@@ -294,6 +335,7 @@ __global__ void __launch_bounds__(256) group_sum_kernel(const float* __restrict_
     const int hg = H / G;
     const float* pb = dBh + (bt * H + (long long)g * hg) * N + n;
     const float* pc = dCh + (bt * H + (long long)g * hg) * N + n;
+    if (!SSD_INB((bt * H + (long long)g * hg + hg - 1) * N + n, rows * H * N)) return;
     float sb = 0.f, sc = 0.f;
     for (int i = 0; i < hg; ++i) {
         sb += pb[(size_t)i * N];
@@ -330,10 +372,10 @@ cudaError_t launch_form(const Dims& d, Opd U, Opd V, Opd Z, const float* cum, co
 template <typename T>
 cudaError_t run_backward_t(const Dims& d, const BackwardArgs& g, const BackwardScratch& w,
                            cudaStream_t st) {
-    const Opd ox{g.x, d.H * d.P, d.P, 1};
-    const Opd ody{g.dy, d.H * d.P, d.P, 1};
-    const Opd oB{g.Bm, d.G * d.N, d.N, d.H / d.G};
-    const Opd oC{g.Cm, d.G * d.N, d.N, d.H / d.G};
+    const Opd ox{g.x, d.H * d.P, d.P, 1, (long long)d.B * d.T * d.H * d.P};
+    const Opd ody{g.dy, d.H * d.P, d.P, 1, (long long)d.B * d.T * d.H * d.P};
+    const Opd oB{g.Bm, d.G * d.N, d.N, d.H / d.G, (long long)d.B * d.T * d.G * d.N};
+    const Opd oC{g.Cm, d.G * d.N, d.N, d.H / d.G, (long long)d.B * d.T * d.G * d.N};
     cudaError_t e;
     if (std::is_same<T, __nv_bfloat16>::value && backward_forms_tc_supported(d)) {
         if ((e = launch_backward_forms_tc(d, g.x, g.dy, g.Bm, g.Cm, w.cum, w.states, w.dstates, w.ytil,

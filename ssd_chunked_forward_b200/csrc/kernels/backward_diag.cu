@@ -19,6 +19,7 @@
 // 2^x on the special-function unit from decays pre-scaled by log2(e), with
 // the exponent clamped at 0 where the term is masked out.  N <= 128.
 #include "../common.cuh"
+#include "../debug_checks.cuh"
 #include "../kernels.h"
 #include "bwd_tiles.cuh"
 
@@ -49,6 +50,10 @@ __global__ void __launch_bounds__(256) reverse_pass_diag_kernel(const float* __r
     const int n = r / P;
     float* sp = dstates + bh * (long long)nc * NP + r;
     const float* ce = cum + bh * (long long)nc * Q * N + (size_t)(Q - 1) * N + n;
+    // the chain's last slot and last decay bound every access below
+    if (!SSD_INB(bh * (long long)nc * NP + (long long)(nc - 1) * NP + r, total * nc) ||
+        !SSD_INB(bh * (long long)nc * Q * N + (long long)nc * Q * N - 1, total / NP * nc * Q * N))
+        return;
     float g = dfinal ? dfinal[bh * NP + r] : 0.f;
     for (int k = nc - 1; k >= 0; --k) {
         const float s = sp[(size_t)k * NP];
@@ -69,6 +74,7 @@ __global__ void __launch_bounds__(256) chunk_dot_diag_kernel(const float* __rest
     const int k = blockIdx.x, bh = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const size_t NP = (size_t)N * P;
+    if (!SSD_INB(((long long)bh * nc + k + 1) * NP - 1, (long long)gridDim.y * nc * NP)) return;  // whole block
     const float* g = G + ((size_t)bh * nc + k) * NP;
     const float* h = (k + 1 < nc) ? Hin + ((size_t)bh * nc + k + 1) * NP : fin + (size_t)bh * NP;
     for (int n = warp; n < N; n += 8) {
@@ -124,6 +130,10 @@ __global__ void __launch_bounds__(256) dx_diag_kernel(Opd Bo, Opd Co, Opd dYo,
     const int tk = k * Q;
     const int qv = min(Q, Tlen - tk);
     if (i0 >= qv) return;
+    // the chunk's decays and state lie in their buffers (the whole block leaves if not)
+    if (!SSD_INB(((long long)bh * nc + k + 1) * Q * N - 1, (long long)gridDim.y * nc * Q * N) ||
+        !SSD_INB(((long long)bh * nc + k + 1) * N * P - 1, (long long)gridDim.y * nc * N * P))
+        return;
     const float* cumk = cum + ((size_t)bh * nc + k) * (size_t)Q * N;
 
     load_kmajor<T, VEC>(UT, Bo, b, Tlen, tk, i0, qv, h, N, tid);
@@ -216,7 +226,7 @@ __global__ void __launch_bounds__(256) dx_diag_kernel(Opd Bo, Opd Co, Opd dYo,
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             const int m = m0 + 4 * c + q;
-            if (m < P) o[m] = acc[a][q];
+            if (m < P && SSD_INB(o - out + m, (long long)gridDim.y * Tlen * P)) o[m] = acc[a][q];
         }
     }
 }
@@ -248,6 +258,10 @@ __global__ void __launch_bounds__(256) dbc_diag_kernel(Opd U, Opd V, Opd Z,
     const int tk = k * Q;
     const int qv = min(Q, Tlen - tk);
     if (i0 >= qv) return;
+    // the chunk's decays and state lie in their buffers (the whole block leaves if not)
+    if (!SSD_INB(((long long)bh * nc + k + 1) * Q * N - 1, (long long)gridDim.y * nc * Q * N) ||
+        !SSD_INB(((long long)bh * nc + k + 1) * N * P - 1, (long long)gridDim.y * nc * N * P))
+        return;
     const float* cumk = cum + ((size_t)bh * nc + k) * (size_t)Q * N;
 
     load_kmajor<T, VEC>(UT, U, b, Tlen, tk, i0, qv, h, P, tid);
@@ -354,7 +368,7 @@ __global__ void __launch_bounds__(256) dbc_diag_kernel(Opd U, Opd V, Opd Z,
             const int n = m0 + 4 * c + q;
             if (n >= N) continue;
             const float sc = ex2_approx(fminf(ANTI ? ce[4 * c + q] - ci[a][q] : ci[a][q], 0.f));
-            o[n] = fmaf(sc, acc2[a][q], acc[a][q]);
+            if (SSD_INB(o - out + n, (long long)gridDim.y * Tlen * N)) o[n] = fmaf(sc, acc2[a][q], acc[a][q]);
         }
     }
 }
@@ -375,6 +389,11 @@ __global__ void __launch_bounds__(256) token_grad_diag_kernel(
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tk = k * Q;
     const int qv = min(Q, Tlen - tk);
+    // the chunk's last row bounds every token access below (the whole block leaves)
+    if (!SSD_INB((((long long)b * Tlen + tk + qv - 1) * H + h) * P + P - 1, (long long)gridDim.y * Tlen * P) ||
+        !SSD_INB((((long long)b * Tlen + tk + qv - 1) * H + h) * N + N - 1, (long long)gridDim.y * Tlen * N) ||
+        !SSD_INB((((long long)b * Tlen + tk + qv - 1) * G + g) * N + N - 1, (long long)(gridDim.y / H) * Tlen * G * N))
+        return;
     const float dv = D ? D[h] : 0.f;
     float dsum = 0.f;
     for (int j = warp; j < qv; j += 8) {
@@ -408,10 +427,10 @@ __global__ void __launch_bounds__(256) token_grad_diag_kernel(
 template <typename T, bool VEC>
 cudaError_t run_forms(const Dims& d, const BackwardArgs& g, const BackwardScratch& w,
                       cudaStream_t st) {
-    const Opd ox{g.x, d.H * d.P, d.P, 1};
-    const Opd ody{g.dy, d.H * d.P, d.P, 1};
-    const Opd oB{g.Bm, d.G * d.N, d.N, d.H / d.G};
-    const Opd oC{g.Cm, d.G * d.N, d.N, d.H / d.G};
+    const Opd ox{g.x, d.H * d.P, d.P, 1, (long long)d.B * d.T * d.H * d.P};
+    const Opd ody{g.dy, d.H * d.P, d.P, 1, (long long)d.B * d.T * d.H * d.P};
+    const Opd oB{g.Bm, d.G * d.N, d.N, d.H / d.G, (long long)d.B * d.T * d.G * d.N};
+    const Opd oC{g.Cm, d.G * d.N, d.N, d.H / d.G, (long long)d.B * d.T * d.G * d.N};
     const int nrt = (d.Q + kFT - 1) / kFT;
     cudaError_t e;
     {

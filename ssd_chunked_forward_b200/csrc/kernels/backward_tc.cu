@@ -3,7 +3,7 @@
 // 128 or 256 tokens).
 //
 // Each form gives, for the rows i of one chunk (c the in-chunk cumulative
-// decay, M the chunk's fp32 state, read as K x MC through two strides):
+// decay, M the chunk's fp32 state read as K x MC):
 //   causal:  out_i = sum_{j<=i} (U_i.V_j) e^{c_i - c_j} Z_j + e^{c_i} U_i M
 //   anti:    out_i = sum_{j>=i} (U_i.V_j) e^{c_j - c_i} Z_j + e^{c_end - c_i} U_i M
 // -- y - Dx, dC, dx - D dy and dB of the chunked backward (the adjoint of the
@@ -11,13 +11,20 @@
 // operator"; the roles of U, V, Z and M are in backward.cu).  Every factor is
 // <= 1 for a <= 0.
 //
-// One CTA per (chunk, 128-row tile, batch x head): TMA brings the U rows and
-// the V and Z rows of the tile's column range (one or two 128-token tiles);
-// S = U V^T (K-major operands) goes to TMEM; eight warps mask and decay S into
-// bf16 scores P~ in TMEM, scale the U rows by their factor in place and write
-// M as a bf16 operand; then out = P~ Z (A from TMEM) + U~ M accumulates in
-// TMEM and is stored as fp32.  Warp 0 issues the copies and the products.
+// One CTA per (chunk, 128-row tile, batch x head), two CTAs per SM (about
+// 100 KB of shared memory and 256 TMEM columns each), so one CTA's copies
+// overlap the other's arithmetic.  TMA brings the U rows and the V rows of
+// the tile's column range (one or two 128-token tiles); S = U V^T (K-major
+// operands) goes to TMEM, one 128-column tile per V tile.  Once S is done the
+// V space takes the Z rows (TMA) and M (bf16, written by the math warps from
+// fp32 read ahead into registers).  Eight warps mask and decay S into bf16
+// scores P~, packed in place into the first half of each S tile (64-column
+// pieces, every piece read before any is overwritten), and scale the U rows
+// by their factor; then out = P~ Z (A from TMEM) + U~ M accumulates in the
+// TMEM columns that S no longer needs, in 64-column halves, and is stored as
+// fp32.  Warp 0 issues the copies and the products.
 #include "../common.cuh"
+#include "../debug_checks.cuh"
 #include "../kernels.h"
 #include "../tc_common.cuh"
 #include "../tmap.h"
@@ -28,36 +35,42 @@ namespace {
 constexpr int kRowsT = 128;                  // rows of a tile (the MMA's M)
 constexpr uint32_t kBox = 128 * 128;         // 128 rows x 64 bf16 (one 128-byte swizzle box)
 constexpr int kFormThreads = 288;            // warp 0 + eight math warps
-constexpr uint32_t COL_S = 0, COL_PT = 256, COL_O = 384;
+constexpr uint32_t kTmemCols = 256;
+// TMEM: S of V tile v at columns 128 v (fp32), its packed P~ at 128 v (bf16
+// pairs, 64 columns); output half q (64 columns of MC) at 64 + 128 q
+__host__ __device__ constexpr uint32_t col_o(int q) { return 64u + 128u * (uint32_t)q; }
 
 struct FormParams {
     const float* cum;  // [B*H][nc][Q]
-    const float* Mst;  // [B*H][nc][N*P]
+    const float* Mst;  // [B*H][nc][K*MC]: M stored [K][MC] (MROW) or [MC][K]
     float* out;        // [B][T][H][MC]
-    int sk, sm;        // M[kk][m] = Mst[kk * sk + m * sm]
     int T, H, G, Q, nc, NP;
     int u_grp, v_grp, z_grp;  // operand indexed by B/C group (else by head)
     int* status;              // set to kDevTimeout when a bounded wait gives up
 };
 
 struct __align__(8) FormBars {
-    uint64_t full, s_full, p_full, o_full;
+    uint64_t full, s_full, z_full, p_full, o_full;
 };
 
 template <int K, int MC>
 struct FormSmem {
-    static constexpr uint32_t U = 0;                              // K/64 boxes
-    static constexpr uint32_t V = U + (K / 64) * kBox;            // 2 tiles x K/64 boxes
-    static constexpr uint32_t Z = V + 2 * (K / 64) * kBox;        // 2 tiles x MC/64 boxes
-    static constexpr uint32_t M = Z + 2 * (MC / 64) * kBox;       // MC/64 boxes of K rows
-    static constexpr uint32_t CUM = M + (MC / 64) * K * 128;      // [256] fp32
+    static constexpr uint32_t kV = 2 * (K / 64) * kBox;                    // two V tiles
+    static constexpr uint32_t kZM = 2 * (MC / 64) * kBox + (MC / 64) * K * 128;  // two Z tiles + M
+    static constexpr uint32_t U = 0;                                       // K/64 boxes
+    static constexpr uint32_t R = U + (K / 64) * kBox;                     // V, later Z and M
+    static constexpr uint32_t Z = R;
+    static constexpr uint32_t M = R + 2 * (MC / 64) * kBox;                // MC/64 boxes of K rows
+    static constexpr uint32_t CUM = R + (kV > kZM ? kV : kZM);             // [256] fp32
     static constexpr uint32_t BAR = CUM + 256 * 4;
     static constexpr uint32_t MISC = BAR + 64;
     static constexpr size_t bytes = 1024 + MISC + 16;
 };
+static_assert(FormSmem<128, 64>::bytes <= 113 * 1024 && FormSmem<64, 128>::bytes <= 113 * 1024,
+              "two CTAs per SM");
 
-template <int K, int MC, bool ANTI>
-__global__ void __launch_bounds__(kFormThreads, 1)
+template <int K, int MC, bool ANTI, bool MROW>
+__global__ void __launch_bounds__(kFormThreads, 2)
     chunk_form_tc_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_v,
                          const __grid_constant__ CUtensorMap tm_z, const FormParams p) {
     using L = FormSmem<K, MC>;
@@ -65,7 +78,7 @@ __global__ void __launch_bounds__(kFormThreads, 1)
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
     uint8_t* sU = sm + L::U;
-    uint8_t* sV = sm + L::V;
+    uint8_t* sV = sm + L::R;
     uint8_t* sZ = sm + L::Z;
     uint8_t* sM = sm + L::M;
     float* sCum = reinterpret_cast<float*>(sm + L::CUM);
@@ -82,16 +95,22 @@ __global__ void __launch_bounds__(kFormThreads, 1)
     const int jbase = ANTI ? i0 : 0;
     const int nt = ANTI ? (p.Q - i0) / kRowsT : i0 / kRowsT + 1;
     if (i0 >= qv) return;  // a tile wholly past T: nothing to write
+    // the chunk's decays and state lie in their buffers (the whole block
+    // leaves before any barrier if not)
+    if (!SSD_INB(((long long)bh * p.nc + k + 1) * p.Q - 1, (long long)gridDim.y * p.nc * p.Q) ||
+        !SSD_INB(((long long)bh * p.nc + k + 1) * p.NP - 1, (long long)gridDim.y * p.nc * p.NP))
+        return;
 
     if (threadIdx.x == 0) {
         tc::mbar_init(&bars->full, 1);
         tc::mbar_init(&bars->s_full, 1);
+        tc::mbar_init(&bars->z_full, 1);
         tc::mbar_init(&bars->p_full, 8);
         tc::mbar_init(&bars->o_full, 1);
         tc::fence_mbar_init();
     }
     if (warp == 0) {
-        tc::tmem_alloc(sTmem, 512);
+        tc::tmem_alloc(sTmem, kTmemCols);
         tc::tmem_relinquish();
     }
     for (int t = threadIdx.x; t < p.Q; t += kFormThreads)
@@ -109,16 +128,12 @@ __global__ void __launch_bounds__(kFormThreads, 1)
         if (lane == 0) {
             // ------------------------------------------ copies and products ----
             const int cu = p.u_grp ? g : h, cv = p.v_grp ? g : h, cz = p.z_grp ? g : h;
-            const uint32_t bytes = (uint32_t)((K / 64) * kBox * (1 + nt) + (MC / 64) * kBox * nt);
-            tc::mbar_arrive_expect_tx(&bars->full, bytes);
+            tc::mbar_arrive_expect_tx(&bars->full, (uint32_t)((K / 64) * kBox * (1 + nt)));
             for (int q = 0; q < K / 64; ++q) tc::tma_load_4d(sU + q * kBox, &tm_u, &bars->full, 64 * q, cu, tk + i0, b);
-            for (int v = 0; v < nt; ++v) {
-                const int tj = tk + jbase + v * kRowsT;
+            for (int v = 0; v < nt; ++v)
                 for (int q = 0; q < K / 64; ++q)
-                    tc::tma_load_4d(sV + (v * (K / 64) + q) * kBox, &tm_v, &bars->full, 64 * q, cv, tj, b);
-                for (int q = 0; q < MC / 64; ++q)
-                    tc::tma_load_4d(sZ + (v * (MC / 64) + q) * kBox, &tm_z, &bars->full, 64 * q, cz, tj, b);
-            }
+                    tc::tma_load_4d(sV + (v * (K / 64) + q) * kBox, &tm_v, &bars->full, 64 * q, cv,
+                                    tk + jbase + v * kRowsT, b);
             bool ok = tc::mbar_wait(&bars->full, 0, nullptr, kBudget);
             if (ok) {
                 tc::tc_fence_after();
@@ -130,29 +145,46 @@ __global__ void __launch_bounds__(kFormThreads, 1)
 #pragma unroll
                     for (int kk = 0; kk < K / 16; ++kk) {
                         const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
-                        tc::mma_ss(tmem + COL_S + 128 * v, tc::desc_adv(dU, off), tc::desc_adv(dV, off), id_s, kk > 0);
+                        tc::mma_ss(tmem + 128 * v, tc::desc_adv(dU, off), tc::desc_adv(dV, off), id_s, kk > 0);
                     }
                 }
             }
             tc::mma_commit(&bars->s_full);
+            // V is dead once S is done: the Z rows take its place
+            ok = tc::mbar_wait(&bars->s_full, 0, nullptr, kBudget) && ok;
+            if (ok) {
+                tc::mbar_arrive_expect_tx(&bars->z_full, (uint32_t)((MC / 64) * kBox * nt));
+                for (int v = 0; v < nt; ++v)
+                    for (int q = 0; q < MC / 64; ++q)
+                        tc::tma_load_4d(sZ + (v * (MC / 64) + q) * kBox, &tm_z, &bars->z_full, 64 * q, cz,
+                                        tk + jbase + v * kRowsT, b);
+            }
+            ok = ok && tc::mbar_wait(&bars->z_full, 0, nullptr, kBudget);
             ok = ok && tc::mbar_wait(&bars->p_full, 0, nullptr, kBudget);
             if (ok) {
                 tc::tc_fence_after();
-                // out = P~ Z (A from TMEM, K = the columns j; Z MN-major) + U~ M
-                constexpr uint32_t id_o = tc::idesc_bf16_f32(128, MC, 0, 1);
-                for (int v = 0; v < nt; ++v) {
-                    const uint64_t dZ = tc::smem_desc_sw128(tc::smem_u32(sZ + v * (MC / 64) * kBox), kBox, 1024);
+                // out = P~ Z (A from TMEM, K = the columns j; Z MN-major) + U~ M,
+                // in 64-column halves of MC
+                constexpr uint32_t id_o = tc::idesc_bf16_f32(128, 64, 0, 1);
+                for (int v = 0; v < nt; ++v)
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        tc::mma_ts(tmem + COL_O, tmem + COL_PT + 64 * v + kk * 8, tc::desc_adv(dZ, kk * 2048), id_o,
-                                   (v > 0 || kk > 0) ? 1u : 0u);
-                }
+                    for (int q = 0; q < MC / 64; ++q) {
+                        const uint64_t dZ =
+                            tc::smem_desc_sw128(tc::smem_u32(sZ + (v * (MC / 64) + q) * kBox), kBox, 1024);
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            tc::mma_ts(tmem + col_o(q), tmem + 128 * v + kk * 8, tc::desc_adv(dZ, kk * 2048),
+                                       id_o, (v > 0 || kk > 0) ? 1u : 0u);
+                    }
                 const uint64_t dU = tc::smem_desc_sw128(tc::smem_u32(sU), 16, 1024);
-                const uint64_t dM = tc::smem_desc_sw128(tc::smem_u32(sM), K * 128, 1024);
 #pragma unroll
-                for (int kk = 0; kk < K / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
-                    tc::mma_ss(tmem + COL_O, tc::desc_adv(dU, off), tc::desc_adv(dM, kk * 2048), id_o, 1u);
+                for (int q = 0; q < MC / 64; ++q) {
+                    const uint64_t dM = tc::smem_desc_sw128(tc::smem_u32(sM + q * (K * 128)), K * 128, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < K / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
+                        tc::mma_ss(tmem + col_o(q), tc::desc_adv(dU, off), tc::desc_adv(dM, kk * 2048), id_o, 1u);
+                    }
                 }
             }
             tc::mma_commit(&bars->o_full);
@@ -163,30 +195,70 @@ __global__ void __launch_bounds__(kFormThreads, 1)
         // ---------------------------------------------------- math warps ----
         const int mw = warp - 1;           // 0..7
         const int quad = warp & 3;         // TMEM lane quadrant
-        const int half = mw >> 2;          // 0/1: which half of the columns
+        const int half = mw >> 2;          // 0/1: which columns
         const int row = quad * 32 + lane;  // tile row = TMEM lane
         const int i = i0 + row;            // row within the chunk
         const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
         const float ci = sCum[i];
         const float cend = sCum[p.Q - 1];
-        // M (fp32, K x MC) as a bf16 MN-major operand: row kk, columns m in
-        // 64-wide boxes; one 16-byte piece (8 columns) per step
-        {
-            const int mt = threadIdx.x - 32;  // 0..255
-            const float* Mk = p.Mst + ((size_t)bh * p.nc + k) * (size_t)p.NP;
-            for (int c = mt; c < K * (MC / 8); c += 256) {
-                const int kk = c / (MC / 8), m8 = (c % (MC / 8)) * 8;
-                float f[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) f[e] = Mk[(size_t)kk * p.sk + (size_t)(m8 + e) * p.sm];
-                const uint4 w = make_uint4(tc::pack_bf16x2(f[0], f[1]), tc::pack_bf16x2(f[2], f[3]),
-                                           tc::pack_bf16x2(f[4], f[5]), tc::pack_bf16x2(f[6], f[7]));
-                *reinterpret_cast<uint4*>(sM + (m8 >> 6) * (K * 128) + tc::sw128_offset(kk, (m8 & 63) >> 3)) = w;
+        const int mt = threadIdx.x - 32;  // 0..255
+        const float* Mk = p.Mst + ((size_t)bh * p.nc + k) * (size_t)p.NP;
+        // the two warps of a lane quadrant (immediate barrier ids 1-4)
+        auto pair_sync = [&]() {
+            tc::tc_fence_before();
+            switch (quad) {
+                case 0: asm volatile("bar.sync 1, 64;" ::: "memory"); break;
+                case 1: asm volatile("bar.sync 2, 64;" ::: "memory"); break;
+                case 2: asm volatile("bar.sync 3, 64;" ::: "memory"); break;
+                default: asm volatile("bar.sync 4, 64;" ::: "memory"); break;
             }
+            tc::tc_fence_after();
+        };
+        // M (fp32, K x MC) read ahead with 16-byte loads: [K][MC] (MROW) a
+        // thread takes 8 consecutive columns of a row, four rows apart; [MC][K]
+        // a 4 x 8 block (4 rows kk, 8 columns m), one load per column
+        constexpr int kMTasks = MROW ? K * (MC / 8) / 256 : (K / 4) * (MC / 8) / 256;
+        static_assert(kMTasks >= 1 && (MROW ? K * (MC / 8) : (K / 4) * (MC / 8)) % 256 == 0, "M tasks");
+        float4 mv[8 * kMTasks / (MROW ? 4 : 1)];
+        if (MROW) {
+#pragma unroll
+            for (int u = 0; u < kMTasks; ++u) {
+                const int c = mt + 256 * u, kk = c / (MC / 8), m8 = (c % (MC / 8)) * 8;
+                mv[2 * u] = *reinterpret_cast<const float4*>(Mk + (size_t)kk * MC + m8);
+                mv[2 * u + 1] = *reinterpret_cast<const float4*>(Mk + (size_t)kk * MC + m8 + 4);
+            }
+        } else {
+            const int kk4 = (mt % (K / 4)) * 4, m8 = (mt / (K / 4)) * 8;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mv[e] = *reinterpret_cast<const float4*>(Mk + (size_t)(m8 + e) * K + kk4);
         }
         bool ok = tc::mbar_wait(&bars->s_full, 0, nullptr, kBudget);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok && lane == 0) timed_out();
+        {
+            // M into the V space (dead now that S is done) as a bf16 MN-major
+            // operand: row kk, columns m in 64-wide boxes of 16-byte pieces
+            auto put = [&](int kk, int m8, float f0, float f1, float f2, float f3, float f4, float f5, float f6,
+                           float f7) {
+                const uint4 w = make_uint4(tc::pack_bf16x2(f0, f1), tc::pack_bf16x2(f2, f3),
+                                           tc::pack_bf16x2(f4, f5), tc::pack_bf16x2(f6, f7));
+                *reinterpret_cast<uint4*>(sM + (m8 >> 6) * (K * 128) + tc::sw128_offset(kk, (m8 & 63) >> 3)) = w;
+            };
+            if (MROW) {
+#pragma unroll
+                for (int u = 0; u < kMTasks; ++u) {
+                    const int c = mt + 256 * u, kk = c / (MC / 8), m8 = (c % (MC / 8)) * 8;
+                    const float4 a0 = mv[2 * u], a1 = mv[2 * u + 1];
+                    put(kk, m8, a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w);
+                }
+            } else {
+                const int kk4 = (mt % (K / 4)) * 4, m8 = (mt / (K / 4)) * 8;
+                put(kk4, m8, mv[0].x, mv[1].x, mv[2].x, mv[3].x, mv[4].x, mv[5].x, mv[6].x, mv[7].x);
+                put(kk4 + 1, m8, mv[0].y, mv[1].y, mv[2].y, mv[3].y, mv[4].y, mv[5].y, mv[6].y, mv[7].y);
+                put(kk4 + 2, m8, mv[0].z, mv[1].z, mv[2].z, mv[3].z, mv[4].z, mv[5].z, mv[6].z, mv[7].z);
+                put(kk4 + 3, m8, mv[0].w, mv[1].w, mv[2].w, mv[3].w, mv[4].w, mv[5].w, mv[6].w, mv[7].w);
+            }
+        }
         if (ok) {
             tc::tc_fence_after();
             // U row i times its factor, in place (S has read U): half the row's chunks
@@ -203,30 +275,53 @@ __global__ void __launch_bounds__(kFormThreads, 1)
                 v.w = tc::mul_bf16x2(v.w, u2);
                 *ptr = v;
             }
-            // P~ = S masked and decayed, 16 columns at a time; warp half takes
-            // every other piece
-            for (int pc = half; pc < nt * 8; pc += 2) {
-                const int col0 = 16 * pc;  // column in the S tiles
-                float s[16];
-                tc::tmem_ld16(lane_base + COL_S + col0, s);
-                tc::tmem_ld_wait();
-                uint32_t pk[8];
+            // P~ = S masked and decayed, packed in place: with two V tiles
+            // warp half h takes tile h, with one the halves take a 64-column
+            // piece each; a piece is read and written 32 columns at a time,
+            // its packed scores landing in the first half of its tile.  The
+            // pair of warps of a lane quadrant meets once per piece: the owner
+            // of a tile's first piece after reading all of it, the other
+            // before its first write (which lands in the first piece).
+            const int npc = nt == 2 ? 2 : 1;
+            for (int u = 0; u < npc; ++u) {
+                const int tile = nt == 2 ? half : 0;
+                const int c0 = nt == 2 ? 64 * u : 64 * half;  // column of the piece in its tile
 #pragma unroll
-                for (int e2 = 0; e2 < 8; ++e2) {
-                    float pv[2];
+                for (int r = 0; r < 2; ++r) {
+                    const int cin = c0 + 32 * r;
+                    const uint32_t tbase = lane_base + 128 * tile;
+                    float s[32];
+                    tc::tmem_ld16(tbase + cin, *reinterpret_cast<float(*)[16]>(s));
+                    tc::tmem_ld16(tbase + cin + 16, *reinterpret_cast<float(*)[16]>(s + 16));
+                    tc::tmem_ld_wait();
+                    if (r == (c0 == 0 ? 1 : 0)) pair_sync();
+                    const int j0 = jbase + 128 * tile + cin;  // chunk column of s[0]
 #pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        const int e = 2 * e2 + q;
-                        const int j = jbase + col0 + e;
-                        const bool keep = (ANTI ? j >= i : j <= i) && j < qv && i < qv;
-                        const float ex = ex2_approx(keep ? (ANTI ? sCum[j] - ci : ci - sCum[j]) * 1.4426950408889634f : 0.f);
-                        pv[q] = keep ? s[e] * ex : 0.f;
+                    for (int g8 = 0; g8 < 2; ++g8) {
+                        uint32_t pk[8];
+#pragma unroll
+                        for (int e2 = 0; e2 < 8; ++e2) {
+                            float pv[2];
+#pragma unroll
+                            for (int q = 0; q < 2; ++q) {
+                                const int e = 16 * g8 + 2 * e2 + q;
+                                const int j = j0 + e;
+                                const bool keep = (ANTI ? j >= i : j <= i) && j < qv && i < qv;
+                                const float ex = ex2_approx(
+                                    keep ? (ANTI ? sCum[j] - ci : ci - sCum[j]) * 1.4426950408889634f : 0.f);
+                                pv[q] = keep ? s[e] * ex : 0.f;
+                            }
+                            pk[e2] = tc::pack_bf16x2(pv[0], pv[1]);
+                        }
+                        tc::tmem_st8(tbase + cin / 2 + 8 * g8, pk);
                     }
-                    pk[e2] = tc::pack_bf16x2(pv[0], pv[1]);
                 }
-                tc::tmem_st8(lane_base + COL_PT + (col0 >> 1), pk);
             }
             tc::tmem_st_wait();
+        } else {
+            // keep the pair barriers matched with a partner that did not fail
+            const int npc = nt == 2 ? 2 : 1;
+            for (int u = 0; u < npc; ++u) pair_sync();
         }
         tc::fence_proxy_async_smem();  // U~ and M for the products
         tc::tc_fence_before();
@@ -240,11 +335,11 @@ __global__ void __launch_bounds__(kFormThreads, 1)
             float* o = p.out + (((size_t)b * p.T + tk + i) * p.H + h) * MC;
 #pragma unroll
             for (int q16 = 0; q16 < MC / 32; ++q16) {
-                const int m0 = half * (MC / 2) + 16 * q16;
+                const int m0 = half * (MC / 2) + 16 * q16;  // output column
                 float v[16];
-                tc::tmem_ld16(lane_base + COL_O + m0, v);
+                tc::tmem_ld16(lane_base + col_o(m0 >> 6) + (m0 & 63), v);
                 tc::tmem_ld_wait();
-                if (i < qv) {
+                if (i < qv && SSD_INB((o - p.out) + m0 + 15, (long long)gridDim.y * p.T * MC)) {
 #pragma unroll
                     for (int e4 = 0; e4 < 4; ++e4)
                         *reinterpret_cast<float4*>(o + m0 + 4 * e4) =
@@ -257,13 +352,13 @@ __global__ void __launch_bounds__(kFormThreads, 1)
     __syncthreads();
     if (warp == 0) {
         tc::tc_fence_after();
-        tc::tmem_dealloc(tmem, 512);
+        tc::tmem_dealloc(tmem, kTmemCols);
     }
 }
 
-template <int K, int MC, bool ANTI>
+template <int K, int MC, bool ANTI, bool MROW>
 cudaError_t launch_form_tc_t(const Dims& d, const void* U, int ug, const void* V, int vg, const void* Z, int zg,
-                             const float* cum, const float* Mst, int sk, int smv, float* out,
+                             const float* cum, const float* Mst, float* out,
                              int* status, cudaStream_t st) {
     CUtensorMap tu, tv, tz;
     cudaError_t e = make_tmap_bf16_4d(&tu, U, K, ug ? d.G : d.H, d.T, d.B, kRowsT);
@@ -271,16 +366,16 @@ cudaError_t launch_form_tc_t(const Dims& d, const void* U, int ug, const void* V
     if (e == cudaSuccess) e = make_tmap_bf16_4d(&tz, Z, MC, zg ? d.G : d.H, d.T, d.B, kRowsT);
     if (e != cudaSuccess) return e;
     FormParams p = {};
-    p.cum = cum; p.Mst = Mst; p.out = out; p.sk = sk; p.sm = smv;
+    p.cum = cum; p.Mst = Mst; p.out = out;
     p.T = d.T; p.H = d.H; p.G = d.G; p.Q = d.Q; p.nc = d.nc; p.NP = d.N * d.P;
     p.u_grp = ug; p.v_grp = vg; p.z_grp = zg;
     p.status = status;
     using L = FormSmem<K, MC>;
-    e = cudaFuncSetAttribute(chunk_form_tc_kernel<K, MC, ANTI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(chunk_form_tc_kernel<K, MC, ANTI, MROW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)L::bytes);
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)(d.nc * (d.Q / kRowsT)), (unsigned)(d.B * d.H));
-    chunk_form_tc_kernel<K, MC, ANTI><<<grid, kFormThreads, L::bytes, st>>>(tu, tv, tz, p);
+    chunk_form_tc_kernel<K, MC, ANTI, MROW><<<grid, kFormThreads, L::bytes, st>>>(tu, tv, tz, p);
     return cudaGetLastError();
 }
 
@@ -298,16 +393,16 @@ cudaError_t launch_backward_forms_tc(const Dims& d, const void* x, const void* d
     if (!backward_forms_tc_supported(d)) return cudaErrorNotSupported;
     cudaError_t e;
     // y - D x: causal, U = C, V = B, Z = x, M = Hin (N x P)
-    e = launch_form_tc_t<128, 64, false>(d, Cm, 1, Bm, 1, x, 0, cum, states, d.P, 1, ytil, status, st);
+    e = launch_form_tc_t<128, 64, false, true>(d, Cm, 1, Bm, 1, x, 0, cum, states, ytil, status, st);
     if (e != cudaSuccess) return e;
     // dC per head: causal, U = dy, V = x, Z = B, M = Hin read as P x N
-    e = launch_form_tc_t<64, 128, false>(d, dy, 0, x, 0, Bm, 1, cum, states, 1, d.P, dCh, status, st);
+    e = launch_form_tc_t<64, 128, false, false>(d, dy, 0, x, 0, Bm, 1, cum, states, dCh, status, st);
     if (e != cudaSuccess) return e;
     // dx - D dy: anti-causal, U = B, V = C, Z = dy, M = G (N x P)
-    e = launch_form_tc_t<128, 64, true>(d, Bm, 1, Cm, 1, dy, 0, cum, dstates, d.P, 1, dxt, status, st);
+    e = launch_form_tc_t<128, 64, true, true>(d, Bm, 1, Cm, 1, dy, 0, cum, dstates, dxt, status, st);
     if (e != cudaSuccess) return e;
     // dB per head: anti-causal, U = x, V = dy, Z = C, M = G read as P x N
-    return launch_form_tc_t<64, 128, true>(d, x, 0, dy, 0, Cm, 1, cum, dstates, 1, d.P, dBh, status, st);
+    return launch_form_tc_t<64, 128, true, false>(d, x, 0, dy, 0, Cm, 1, cum, dstates, dBh, status, st);
 }
 
 }  // namespace ssd

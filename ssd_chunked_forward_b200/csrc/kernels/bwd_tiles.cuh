@@ -4,6 +4,7 @@
 #pragma once
 
 #include "../common.cuh"
+#include "../debug_checks.cuh"
 
 namespace ssd {
 namespace bwd {
@@ -16,11 +17,17 @@ namespace bwd {
 struct Opd {
     const void* p;
     int ld_t, ld_h, hdiv;
+    long long n;  // elements addressable from p (B * T * ld_t), for the debug build's checks
 };
+
+__device__ __forceinline__ long long opd_off(const Opd& o, int b, int Tlen, int t, int h) {
+    return ((long long)b * Tlen + t) * o.ld_t + (long long)(h / o.hdiv) * o.ld_h;
+}
 
 template <typename T>
 __device__ __forceinline__ float opd_at(const Opd& o, int b, int Tlen, int t, int h, int i) {
-    return to_f32(static_cast<const T*>(o.p)[((size_t)b * Tlen + t) * o.ld_t + (size_t)(h / o.hdiv) * o.ld_h + i]);
+    const long long off = opd_off(o, b, Tlen, t, h) + i;
+    return SSD_INB(off, o.n) ? to_f32(static_cast<const T*>(o.p)[off]) : 0.f;
 }
 
 constexpr int kFT = 64;  // tile rows / columns
@@ -65,7 +72,7 @@ __device__ __forceinline__ void load_kmajor(float* dst, const Opd& o, int b, int
         for (int v = tid; v < kFT * KV; v += 256) {
             const int rr = v / KV, kv = v - rr * KV, row = r0 + rr;
             float e[W];
-            if (row < qv) {
+            if (row < qv && SSD_INB(opd_off(o, b, Tlen, tk + row, h) + kv * W + W - 1, o.n)) {
                 load16<T>(opd_row<T>(o, b, Tlen, tk + row, h) + kv * W, e);
             } else {
 #pragma unroll
@@ -93,7 +100,7 @@ __device__ __forceinline__ void load_mmajor(float* dst, const Opd& o, int b, int
         for (int v = tid; v < kFT * MV; v += 256) {
             const int rr = v / MV, mv = v % MV, row = r0 + rr, m = m0 + mv * W;
             float e[W];
-            if (row < qv && m < Mc) {
+            if (row < qv && m < Mc && SSD_INB(opd_off(o, b, Tlen, tk + row, h) + m + W - 1, o.n)) {
                 load16<T>(opd_row<T>(o, b, Tlen, tk + row, h) + m, e);
             } else {
 #pragma unroll

@@ -20,6 +20,7 @@
 // B tile is loaded once per slice.  Warp roles: 0 TMA producer, 1 MMA issuer
 // (and TMEM owner), 2-5 weighting + drain (one TMEM lane quadrant each).
 #include "../common.cuh"
+#include "../debug_checks.cuh"
 #include "../kernels.h"
 #include "../tc_common.cuh"
 #include "../tmap.h"
@@ -84,6 +85,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int b = bid / nc;
     const int h0 = g * HG + slice * hpb;
     const int t0 = k * Q;  // first token of the chunk (the last chunk may run past T)
+    {
+        // the slice's last head bounds the decay reads and state stores (the
+        // whole block leaves before any barrier if not)
+        const long long nb = gridDim.x / ((long long)nc * G * slices);
+        const long long last = ((long long)b * H + h0 + hpb - 1) * nc + k;
+        if (!SSD_INB((last + 1) * Q - 1, nb * H * nc * Q) ||
+            !SSD_INB((last + 1) * kNState * kP - 1, nb * H * nc * kNState * kP))
+            return;
+    }
 
     if (threadIdx.x == 0) {
         tc::mbar_init(&bars->b_full, 1);

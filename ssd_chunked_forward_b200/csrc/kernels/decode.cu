@@ -8,6 +8,7 @@
 // every warp access is a contiguous row segment; y is reduced over the
 // n-slices in shared memory.
 #include "../common.cuh"
+#include "../debug_checks.cuh"
 #include "../kernels.h"
 
 namespace ssd {
@@ -29,6 +30,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_step_kernel(
     const int bh = blockIdx.x, b = bh / H, h = bh % H, g = h / (H / G);
     const int tid = threadIdx.x;
     const float* ab = a + (size_t)bh * (DIAG ? N : 1);
+    if (!SSD_INB((long long)bh * N * P + (long long)N * P - 1, (long long)gridDim.x * N * P)) return;
     for (int n = tid; n < N; n += kDecThreads) {
         sB[n] = to_f32(Bm[((size_t)b * G + g) * N + n]);
         sC[n] = to_f32(Cm[((size_t)b * G + g) * N + n]);
@@ -90,41 +92,51 @@ __global__ void __launch_bounds__(kDecThreads) decode_step_kernel(
     }
 }
 
-// The same step with 16-byte state accesses, for P a multiple of 4 with P/4
-// dividing the block: thread (column group p4 of 4 columns, row slice sl)
-// owns rows sl, sl + ns, ... of those 4 columns, all loaded before anything
-// else waits, few registers, so every block of a batch is resident at once.
+// The same step with 16-byte state accesses, the columns of each state split
+// over nsplit = P / cs blocks so that the grid spreads evenly over the SMs:
+// block (b, h, column slice q) of blockDim.x threads, thread (column group p4
+// of 4 columns, row slice sl) owning rows sl, sl + ns, ... (at most four) of
+// those 4 columns, all loaded before anything else waits.  y of the slice's
+// columns is reduced over the row slices in shared memory.
 template <typename T, bool DIAG>
 __global__ void __launch_bounds__(kDecThreads, DIAG ? 2 : 3) decode_step_v4_kernel(
     const T* __restrict__ x, const float* __restrict__ a, const T* __restrict__ Bm,
     const T* __restrict__ Cm, const float* __restrict__ D, float* __restrict__ state,
-    T* __restrict__ y, int H, int P, int G, int N) {
+    T* __restrict__ y, int H, int P, int G, int N, int cs) {
     extern __shared__ float sm[];
-    const int pw4 = P >> 2;                 // column groups
-    const int ns = kDecThreads / pw4;       // row slices
-    float* sB = sm;                         // [N]
-    float* sC = sB + N;                     // [N]
-    float* sE = sC + N;                     // [N]
-    float* sX = sE + N;                     // [P]
-    float* sY = sX + P;                     // [ns][P] partial sums of y
-    const int bh = blockIdx.x, b = bh / H, h = bh % H, g = h / (H / G);
+    const int nsplit = P / cs;
+    const int pw4 = cs >> 2;                 // column groups of this block
+    const int ns = (int)blockDim.x / pw4;    // row slices
+    float* sB = sm;                          // [N]
+    float* sC = sB + N;                      // [N]
+    float* sE = sC + N;                      // [N]
+    float* sX = sE + N;                      // [cs]
+    float* sY = sX + cs;                     // [ns][cs] partial sums of y
+    const int bh = blockIdx.x / nsplit, q = blockIdx.x % nsplit;
+    const int b = bh / H, h = bh % H, g = h / (H / G);
+    const int p0 = q * cs;
     const int tid = threadIdx.x;
     const int p4 = tid % pw4, sl = tid / pw4;
-    float4* hs = reinterpret_cast<float4*>(state + (size_t)bh * N * P);
+    // the chain's whole state and its y row lie inside the batch's buffers
+    if (!SSD_INB((long long)bh * N * P + (long long)N * P - 1, (long long)(gridDim.x / nsplit) * N * P) ||
+        !SSD_INB((long long)bh * P + p0 + cs - 1, (long long)(gridDim.x / nsplit) * P))
+        return;
+    float4* hs = reinterpret_cast<float4*>(state + (size_t)bh * N * P + p0);
+    const int P4 = P >> 2;
     constexpr int kR = 4;  // rows per thread (N <= 4 ns)
     float4 hv[kR];
 #pragma unroll
     for (int r = 0; r < kR; ++r) {
         const int n = sl + r * ns;
-        hv[r] = n < N ? hs[(size_t)n * pw4 + p4] : make_float4(0.f, 0.f, 0.f, 0.f);
+        hv[r] = n < N ? hs[(size_t)n * P4 + p4] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     const float* ab = a + (size_t)bh * (DIAG ? N : 1);
-    for (int n = tid; n < N; n += kDecThreads) {
+    for (int n = tid; n < N; n += blockDim.x) {
         sB[n] = to_f32(Bm[((size_t)b * G + g) * N + n]);
         sC[n] = to_f32(Cm[((size_t)b * G + g) * N + n]);
         sE[n] = ex2_approx((DIAG ? ab[n] : ab[0]) * 1.4426950408889634f);
     }
-    for (int q = tid; q < P; q += kDecThreads) sX[q] = to_f32(x[(size_t)bh * P + q]);
+    for (int c = tid; c < cs; c += blockDim.x) sX[c] = to_f32(x[(size_t)bh * P + p0 + c]);
     __syncthreads();
     const float4 xv = make_float4(sX[4 * p4], sX[4 * p4 + 1], sX[4 * p4 + 2], sX[4 * p4 + 3]);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -138,7 +150,7 @@ __global__ void __launch_bounds__(kDecThreads, DIAG ? 2 : 3) decode_step_v4_kern
             hn.y = fmaf(e, hv[r].y, bn * xv.y);
             hn.z = fmaf(e, hv[r].z, bn * xv.z);
             hn.w = fmaf(e, hv[r].w, bn * xv.w);
-            hs[(size_t)n * pw4 + p4] = hn;
+            hs[(size_t)n * P4 + p4] = hn;
             acc.x = fmaf(cn, hn.x, acc.x);
             acc.y = fmaf(cn, hn.y, acc.y);
             acc.z = fmaf(cn, hn.z, acc.z);
@@ -147,18 +159,34 @@ __global__ void __launch_bounds__(kDecThreads, DIAG ? 2 : 3) decode_step_v4_kern
     }
     reinterpret_cast<float4*>(sY)[sl * pw4 + p4] = acc;
     __syncthreads();
-    for (int q = tid; q < P; q += kDecThreads) {
+    for (int c = tid; c < cs; c += blockDim.x) {
         float s = 0.f;
-        for (int k = 0; k < ns; ++k) s += sY[k * P + q];
-        y[(size_t)bh * P + q] = from_f32<T>(s + (D ? D[h] : 0.f) * sX[q]);
+        for (int k = 0; k < ns; ++k) s += sY[k * cs + c];
+        y[(size_t)bh * P + p0 + c] = from_f32<T>(s + (D ? D[h] : 0.f) * sX[c]);
     }
 }
 
-bool decode_v4_ok(const Dims& d) {
+// The 16-byte variant's launch shape: 512-thread blocks and the widest
+// column slice cs (a multiple of 4 dividing P, cs / 4 dividing the block)
+// that leaves at most four rows per thread; false when none does (P % 4 != 0,
+// or N above 2048).  Narrower slices and smaller blocks spread the same batch
+// over more blocks but were not faster: a step this size is bound by one
+// memory round trip and the launch (measured 8-12 us over 64-5120 blocks).
+struct DecodeShape {
+    int threads, cs;
+};
+bool decode_v4_shape(const Dims& d, DecodeShape* out) {
     if (d.P % 4 != 0) return false;
-    const int pw4 = d.P / 4;
-    if (pw4 > kDecThreads || kDecThreads % pw4 != 0) return false;
-    return d.N <= 4 * (kDecThreads / pw4);
+    const int t = kDecThreads;
+    for (int cs = d.P; cs >= 4; cs -= 4) {
+        if (d.P % cs != 0 || t % (cs / 4) != 0) continue;
+        if (d.N <= 4 * (t / (cs / 4))) {
+            out->threads = t;
+            out->cs = cs;
+            return true;
+        }
+    }
+    return false;
 }
 
 }  // namespace
@@ -166,12 +194,14 @@ bool decode_v4_ok(const Dims& d) {
 cudaError_t launch_decode_step(const Dims& d, const void* x, const float* a, const void* Bm,
                                const void* Cm, const float* D, float* state, void* y,
                                cudaStream_t st) {
-    const unsigned grid = (unsigned)(d.B * d.H);
-    if (decode_v4_ok(d)) {
-        const size_t smem4 = (size_t)(3 * d.N + d.P + (kDecThreads / (d.P / 4)) * d.P) * sizeof(float);
+    DecodeShape ds;
+    if (decode_v4_shape(d, &ds)) {
+        const unsigned grid4 = (unsigned)(d.B * d.H * (d.P / ds.cs));
+        const int ns = ds.threads / (ds.cs / 4);
+        const size_t smem4 = (size_t)(3 * d.N + ds.cs + ns * ds.cs) * sizeof(float);
 #define SSD_DEC4_LAUNCH(TT, DG)                                                                   \
-    decode_step_v4_kernel<TT, DG><<<grid, kDecThreads, smem4, st>>>(                              \
-        (const TT*)x, a, (const TT*)Bm, (const TT*)Cm, D, state, (TT*)y, d.H, d.P, d.G, d.N)
+    decode_step_v4_kernel<TT, DG><<<grid4, ds.threads, smem4, st>>>(                              \
+        (const TT*)x, a, (const TT*)Bm, (const TT*)Cm, D, state, (TT*)y, d.H, d.P, d.G, d.N, ds.cs)
         if (d.bf16) {
             if (d.diag) SSD_DEC4_LAUNCH(__nv_bfloat16, true); else SSD_DEC4_LAUNCH(__nv_bfloat16, false);
         } else {
@@ -180,6 +210,7 @@ cudaError_t launch_decode_step(const Dims& d, const void* x, const float* a, con
 #undef SSD_DEC4_LAUNCH
         return cudaGetLastError();
     }
+    const unsigned grid = (unsigned)(d.B * d.H);
     const int pw = d.P < kDecThreads ? d.P : kDecThreads;
     const size_t smem = (size_t)(3 * d.N + d.P + (kDecThreads / pw) * pw) * sizeof(float);
 #define SSD_DEC_LAUNCH(TT, DG)                                                                    \

@@ -1,6 +1,7 @@
 // diag_scan.cu -- step 5 on CUDA cores: the chunk output for the per-state
 // (diagonal) decay, with the mask factorised per 32-token sub-block.
 #include "../common.cuh"
+#include "../debug_checks.cuh"
 #include "../kernels.h"
 
 namespace ssd {
@@ -52,6 +53,13 @@ __global__ void __launch_bounds__(256) diag_scan_simt_kernel(
     const size_t tk = (size_t)k * Q;
     const int qv = min(Q, Tlen - k * Q);  // rows of this chunk before T
     if (i0 >= qv) return;                 // a tile wholly past T (the whole block leaves)
+    // the chunk's last row of every operand, its decays and its state bound
+    // all the accesses below (the whole block leaves if not)
+    if (!SSD_INB((((long long)b * Tlen + tk + qv - 1) * H + h) * P + P - 1, (long long)gridDim.y * Tlen * P) ||
+        !SSD_INB((((long long)b * Tlen + tk + qv - 1) * G + g) * N + N - 1, (long long)(gridDim.y / H) * Tlen * G * N) ||
+        !SSD_INB(((long long)bh * nc + k + 1) * Q * N - 1, (long long)gridDim.y * nc * Q * N) ||
+        !SSD_INB(((long long)bh * nc + k + 1) * N * P - 1, (long long)gridDim.y * nc * N * P))
+        return;
     auto ocol = [&](int m) { return m < 4 ? 4 * tp + m : 28 + 4 * tp + m; };  // output column of acc[m]
 
     for (int idx = tid; idx < 32 * N; idx += 256) {

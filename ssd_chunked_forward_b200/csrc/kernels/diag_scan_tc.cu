@@ -33,6 +33,7 @@
 // group Q (the in-sub-block scores; warp w serves sub-block w & 3).  The
 // decays are scanned by groups R and Q together, thread = (n, sub-block).
 #include "../common.cuh"
+#include "../debug_checks.cuh"
 #include "../kernels.h"
 #include "../tc_common.cuh"
 #include "../tmap.h"
@@ -120,6 +121,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
     const int g = h / (p.H / p.G);
     const int t0 = j * kBlk;
+    // the block's entering state lies in its buffer (the whole block leaves
+    // before any barrier if not)
+    if (!SSD_INB(((long long)bh * p.nblk + j + 1) * kN * kP - 1, (long long)gridDim.x * kN * kP) ||
+        !SSD_INB(h, p.H))
+        return;
 
     if (threadIdx.x == 0) {
         tc::mbar_init(&bars->full, 1);

@@ -23,6 +23,7 @@
 // issuer and TMEM owner, 2-5 decays, weights and the A operand (thread =
 // (state index n, token half)), then the drain (thread = TMEM lane).
 #include "../common.cuh"
+#include "../debug_checks.cuh"
 #include "../kernels.h"
 #include "../tc_common.cuh"
 #include "../tmap.h"
@@ -96,6 +97,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int g = h / (p.H / p.G);
     const int j0 = 2 * pair;
     const bool two = j0 + 1 < p.nblk;  // the second block exists
+    // the chain's states and block totals lie in their buffers (the whole
+    // block leaves before any barrier if not)
+    if (!SSD_INB(((long long)bh + 1) * p.nblk * kN * kP - 1, (long long)(gridDim.x / p.npairs) * p.nblk * kN * kP) ||
+        !SSD_INB(((long long)bh + 1) * p.nblk * kN - 1, (long long)(gridDim.x / p.npairs) * p.nblk * kN))
+        return;
 
     if (threadIdx.x == 0) {
         tc::mbar_init(&bars->full, 1);

@@ -6,6 +6,7 @@
 // group share B).  Every element is read and written once, 16 bytes per
 // thread where the row length allows it (else one warp per row).
 #include "../common.cuh"
+#include "../debug_checks.cuh"
 #include "../kernels.h"
 
 namespace ssd {
@@ -32,6 +33,10 @@ __global__ void __launch_bounds__(kDiscThreads) discretize_kernel(
     const long long r = piece / per;
     const int q = (int)(piece - r * per);
     const int h = (int)(r % H);
+    // every index below is (row r < rows, element < P or N): one check of
+    // the row's last piece covers them
+    if (!SSD_INB(r * P + (long long)(q + 1) * kEl - 1, rows * P) || !SSD_INB(r * (DIAG ? N : 1), rows * (DIAG ? N : 1)))
+        return;
     const float dt = softplus_f(dt_raw[r] + (dt_bias ? dt_bias[h] : 0.f));
     if (DIAG) {
         for (int n = q; n < N; n += per) a_out[r * N + n] = -dt * expf(A_log[(size_t)h * N + n]);
@@ -69,6 +74,7 @@ __global__ void __launch_bounds__(kDiscThreads) discretize_rows_kernel(
     const int lane = threadIdx.x & 31;
     if (r >= rows) return;
     const int h = (int)(r % H);
+    if (!SSD_INB(r, rows)) return;
     const float dt = softplus_f(dt_raw[r] + (dt_bias ? dt_bias[h] : 0.f));
     if (DIAG) {
         for (int n = lane; n < N; n += 32) a_out[r * N + n] = -dt * expf(A_log[(size_t)h * N + n]);
@@ -77,7 +83,8 @@ __global__ void __launch_bounds__(kDiscThreads) discretize_rows_kernel(
     }
     const T* xr = x + r * P;
     T* yr = x_out + r * P;
-    for (int p = lane; p < P; p += 32) yr[p] = from_f32<T>(dt * to_f32(xr[p]));
+    for (int p = lane; p < P; p += 32)
+        if (SSD_INB(r * P + p, rows * P)) yr[p] = from_f32<T>(dt * to_f32(xr[p]));
 }
 
 }  // namespace

@@ -54,6 +54,7 @@
 // 256-319, the item's C tile 320-383 (bf16), and two accumulators 384-511
 // that hold Z of a head and then its output.
 #include "../common.cuh"
+#include "../debug_checks.cuh"
 #include "../kernels.h"
 #include "../tc_common.cuh"
 #include "../tmap.h"
@@ -280,6 +281,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             // =========================================== x tiles (TMA) ====
             tc::prefetch_tmap(&tm_x);
+            // each x tile is read once: let it leave L2 first
+            const uint64_t pol_stream = tc::policy_evict_first();
             uint32_t hc = 0;
             bool ok = true;
             for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x) {
@@ -288,7 +291,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t st = hc % kXStages, u = hc / kXStages;
                     if (u > 0 && !wait(&bars->x_empty[st], (u - 1) & 1)) { ok = false; break; }
                     tc::mbar_arrive_expect_tx(&bars->x_full[st], kTile);
-                    tc::tma_load_4d(sX + st * kTile, &tm_x, &bars->x_full[st], 0, w.h0 + i, w.j * kBlk, w.b);
+                    tc::tma_load_4d_hint(sX + st * kTile, &tm_x, &bars->x_full[st], 0, w.h0 + i, w.j * kBlk, w.b,
+                                         pol_stream);
                 }
             }
             if (!ok) fail();
@@ -432,11 +436,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         if (!ok) break;
                         tc::fence_proxy_async_global();  // the acquire orders the bulk read
+                        if (!SSD_INB((long long)(chain * 2 + 2) * kN * kP - 1, (long long)p.B * p.H * 2 * kN * kP)) {
+                            tc::mbar_arrive(&bars->hin_full[hs]);  // a failed check: no copy
+                            continue;
+                        }
                         tc::mbar_arrive_expect_tx(&bars->hin_full[hs], kN * kP * 4);
-                        tc::bulk_load(dst, p.ring + (size_t)(chain * 2 + ((w.j - 1) & 1)) * (kN * kP), kN * kP * 4,
-                                      &bars->hin_full[hs]);
+                        tc::bulk_load_hint(dst, p.ring + (size_t)(chain * 2 + ((w.j - 1) & 1)) * (kN * kP),
+                                           kN * kP * 4, &bars->hin_full[hs], tc::policy_evict_last());
                     } else if (p.init) {
                         const size_t ic = ((size_t)(w.b % p.seg) * p.B0 + w.b / p.seg) * p.H + w.h0 + i;
+                        if (!SSD_INB((long long)(ic + 1) * kN * kP - 1, (long long)p.B * p.H * kN * kP)) {
+                            tc::mbar_arrive(&bars->hin_full[hs]);  // a failed check: no copy
+                            continue;
+                        }
                         tc::mbar_arrive_expect_tx(&bars->hin_full[hs], kN * kP * 4);
                         tc::bulk_load(dst, p.init + ic * (kN * kP), kN * kP * 4, &bars->hin_full[hs]);
                     } else {
@@ -494,7 +506,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int i4 = 0; i4 < kHpbMax / 4; ++i4) {
                     float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (t < p.T && 4 * i4 < p.hpb) {
+                    if (t < p.T && 4 * i4 < p.hpb &&
+                        SSD_INB(((long long)w.b * p.T + t) * p.H + w.h0 + p.hpb - 1, (long long)p.B * p.T * p.H)) {
                         if (vec) {
                             f = __ldg(reinterpret_cast<const float4*>(row) + i4);
                         } else {
@@ -747,6 +760,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t hc = 0, itc = 0, npub = 0;
             bool alive = true;
             bool prev = false;  // an output of the previous head is pending
+            // the ring is read back by the next block: keep it in L2 under the
+            // streamed x and y
+            const uint64_t pol_ring = tc::policy_evict_last();
             int prev_b = 0, prev_h = 0, prev_t0 = 0;
             uint32_t prev_s = 0, prev_u = 0;
             auto output = [&]() -> bool {
@@ -772,7 +788,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc::fence_proxy_async_smem();
                 group_sync();
                 if (gt == 0) {
-                    tc::tma_store_4d(&tm_y, sY, 0, prev_h, prev_t0, prev_b);
+                    tc::tma_store_4d_hint(&tm_y, sY, 0, prev_h, prev_t0, prev_b, tc::policy_evict_first());
                     tc::bulk_commit();
                 }
                 return true;
@@ -843,12 +859,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                             for (int e = 0; e < 8; ++e) z2[e] = tc::fma2(e2, h2[e], z2[e]);
                         }
-                        if (!last_blk) {
+                        if (!last_blk && SSD_INB((long long)(chain * 2 + (w.j & 1) + 1) * kN * kP - 1,
+                                                 (long long)p.B * p.H * 2 * kN * kP)) {
 #pragma unroll
                             for (int q = 0; q < 4; ++q)
-                                *reinterpret_cast<float4*>(ring_dst + ring_f4(quad, cg, 4 * hh + q, lane)) =
-                                    make_float4(z[4 * q], z[4 * q + 1], z[4 * q + 2], z[4 * q + 3]);
-                        } else if (to_fin) {
+                                tc::st_global_hint(ring_dst + ring_f4(quad, cg, 4 * hh + q, lane),
+                                                   make_float4(z[4 * q], z[4 * q + 1], z[4 * q + 2], z[4 * q + 3]),
+                                                   pol_ring);
+                        } else if (to_fin && SSD_INB(fin_dst - p.fin + 16 * hh + 15, (long long)p.B / p.seg * p.H * kN * kP)) {
 #pragma unroll
                             for (int q = 0; q < 4; ++q)
                                 *reinterpret_cast<float4*>(fin_dst + 16 * hh + 4 * q) =

@@ -50,6 +50,7 @@
 #include <stdlib.h>
 
 #include "../common.cuh"
+#include "../debug_checks.cuh"
 #include "../kernels.h"
 #include "../tc_common.cuh"
 #include "../tmap.h"
@@ -515,11 +516,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int t = w.j * kBlk + gt;
                     const float* arow = p.a + ((size_t)w.b * p.T + t) * p.H + w.h0;
 #pragma unroll
-                    for (int i = 0; i < kHpbMax; ++i) anext[i] = (i < p.hpb && t < p.T) ? __ldg(arow + i) : 0.f;
+                    for (int i = 0; i < kHpbMax; ++i)
+                        anext[i] = (i < p.hpb && t < p.T &&
+                                    SSD_INB(((long long)w.b * p.T + t) * p.H + w.h0 + i, (long long)B * p.T * p.H))
+                                       ? __ldg(arow + i)
+                                       : 0.f;
                 } else {
 #pragma unroll
-                    for (int i = 0; i < kHpbMax; ++i)
-                        anext[i] = i < p.hpb ? __ldg(p.cum + (((size_t)w.b * p.H + w.h0 + i) * p.nblk + w.j) * kBlk + gt) : 0.f;
+                    for (int i = 0; i < kHpbMax; ++i) {
+                        const long long ci = (((long long)w.b * p.H + w.h0 + i) * p.nblk + w.j) * kBlk + gt;
+                        anext[i] = (i < p.hpb && SSD_INB(ci, (long long)B * p.H * p.nblk * kBlk)) ? __ldg(p.cum + ci) : 0.f;
+                    }
                 }
             };
             load_decays(blockIdx.x);
@@ -722,7 +729,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 for (int q = 0; q < 4; ++q)
                                     *reinterpret_cast<float4*>(sHout + state_off(row, cg, 4 * c + q)) =
                                         make_float4(zv[4 * q], zv[4 * q + 1], zv[4 * q + 2], zv[4 * q + 3]);
-                                if (last_blk && p.fin) {
+                                if (last_blk && p.fin &&
+                                    SSD_INB(((long long)chain * kN + row) * kP + 32 * cg + 16 * c + 15,
+                                            (long long)B * p.H * kN * kP)) {
                                     float4* fd = reinterpret_cast<float4*>(
                                         p.fin + ((size_t)chain * kN + row) * kP + 32 * cg + 16 * c);
 #pragma unroll

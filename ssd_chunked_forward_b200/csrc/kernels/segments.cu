@@ -7,6 +7,7 @@
 // passing of one summarised state between pieces as between chunks ("State
 // Space Duality", "Two algorithms for one operator"), one level up.
 #include "../common.cuh"
+#include "../debug_checks.cuh"
 #include "../kernels.h"
 
 namespace ssd {
@@ -21,6 +22,8 @@ __global__ void __launch_bounds__(256) decay_total_kernel(const float* __restric
     if (c >= total) return;
     const long long b = c / cols_per_b, j = c - b * cols_per_b;
     const float* p = a + (size_t)b * T * cols_per_b + j;
+    // the column's last token bounds every load below
+    if (!SSD_INB((p - a) + (long long)(T - 1) * cols_per_b, total * T)) return;
     float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;  // four partial sums: loads in flight
     int t = 0;
     for (; t + 3 < T; t += 4) {
@@ -44,6 +47,9 @@ __global__ void __launch_bounds__(256) state_combine_kernel(
     const int n = (int)((e - bh * NP) / P);
     const long long n_tot = per_state ? chain_elems / P : chain_elems / NP;  // totals per segment
     const long long ti = per_state ? bh * N + n : bh;
+    if (!SSD_INB((long long)S * chain_elems + e, (long long)(S + 1) * chain_elems) ||
+        !SSD_INB((long long)(S - 1) * n_tot + ti, (long long)S * n_tot))
+        return;
     float h = h0 ? h0[e] : 0.f;
     for (int s = 0; s < S; ++s) {
         h_in[(size_t)s * chain_elems + e] = h;

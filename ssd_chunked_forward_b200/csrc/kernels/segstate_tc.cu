@@ -23,6 +23,7 @@
 // 0 TMA producer, 1 MMA issuer (and TMEM owner), 2-5 decays and w o X
 // (thread = token row), then the drain (thread = state row).
 #include "../common.cuh"
+#include "../debug_checks.cuh"
 #include "../kernels.h"
 #include "../tc_common.cuh"
 #include "../tmap.h"
@@ -34,7 +35,7 @@ constexpr int kBlk = 128;
 constexpr int kN = 128;
 constexpr int kP = 64;
 constexpr int kHpbMax = 8;
-constexpr int kXStages = 3;
+constexpr int kXStages = 6;  // x tiles in flight per CTA (one CTA per SM streams the inputs)
 constexpr int kThreads = 192;
 constexpr uint32_t kTile = kBlk * 128;
 
@@ -87,6 +88,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int g = sl / (HG / p.hpb);
     const int h0 = g * HG + (sl - g * (HG / p.hpb)) * p.hpb;
     const int nq = p.nblk * p.hpb;  // (block, head) steps, blocks from the last
+    {
+        // the slice's last piece state and total, and its last decay row, lie
+        // in their buffers (the whole block leaves before any barrier if not)
+        const long long chain = ((long long)(bv % p.S) * p.B0 + bv / p.S) * p.H + h0 + p.hpb - 1;
+        if (!SSD_INB((chain + 1) * kN * kP - 1, (long long)p.S * p.B0 * p.H * kN * kP) ||
+            !SSD_INB(chain, (long long)p.S * p.B0 * p.H) ||
+            !SSD_INB(((long long)bv * p.L + p.L - 1) * p.H + h0 + p.hpb - 1, (long long)p.S * p.B0 * p.L * p.H))
+            return;
+    }
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {

@@ -11,6 +11,7 @@
 //   4 chunk_scan   : quadratic masked form in the chunk + incoming state
 //                    (+ the per-state decay version of the same output)
 #include "../common.cuh"
+#include "../debug_checks.cuh"
 #include "../kernels.h"
 
 namespace ssd {
@@ -32,7 +33,9 @@ __global__ void __launch_bounds__(256) chunk_cumsum_scalar_kernel(const float* _
     const int qv = min(Q, T - k * Q);  // tokens of this chunk before T; the rest count as a = 0
     for (int idx = threadIdx.x; idx < Q * kCumHeads; idx += blockDim.x) {
         const int j = idx / kCumHeads, hh = idx % kCumHeads;
-        sm[idx] = (hh < hn && j < qv) ? a[base + (size_t)j * H + hh] : 0.f;
+        sm[idx] = (hh < hn && j < qv && SSD_INB(base + (size_t)j * H + hh, (long long)gridDim.y * T * H))
+                      ? a[base + (size_t)j * H + hh]
+                      : 0.f;
     }
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -54,7 +57,8 @@ __global__ void __launch_bounds__(256) chunk_cumsum_scalar_kernel(const float* _
         }
         __syncwarp();
         float* out = cum + (((size_t)b * H + h0 + warp) * nc + k) * Q;
-        for (int j = lane; j < Q; j += 32) out[j] = sm[j * kCumHeads + warp];
+        for (int j = lane; j < Q; j += 32)
+            if (SSD_INB(out + j - cum, (long long)gridDim.y * H * nc * Q)) out[j] = sm[j * kCumHeads + warp];
     }
 }
 
@@ -73,8 +77,8 @@ __global__ void __launch_bounds__(256) chunk_cumsum_diag_kernel(const float* __r
         float run = 0.f;
 #pragma unroll 8
         for (int j = 0; j < Q; ++j) {
-            if (j < qv) run += src[(size_t)j * step];
-            dst[(size_t)j * N] = run;
+            if (j < qv && SSD_INB(src + (size_t)j * step - a, (long long)gridDim.y * T * N)) run += src[(size_t)j * step];
+            if (SSD_INB(dst + (size_t)j * N - cum, (long long)gridDim.y * nc * Q * N)) dst[(size_t)j * N] = run;
         }
     }
 }
@@ -128,7 +132,9 @@ __global__ void __launch_bounds__(256) chunk_state_simt_kernel(
             float bv = 0.f, xv = 0.f;
             if (j < qv) {
                 const size_t t = (size_t)k * Q + j;
-                if (n0 + c < N) {
+                if (n0 + c < N && SSD_INB(cumk - cum + (size_t)(Q - 1) * (DIAG ? N : 1) + (DIAG ? n0 + c : 0),
+                                          (long long)gridDim.y * nc * Q * (DIAG ? N : 1)) &&
+                    SSD_INB((((size_t)b * Tlen + t) * G + g) * N + n0 + c, (long long)(gridDim.y / H) * Tlen * G * N)) {
                     float w;
                     if (DIAG && FROM_START)
                         w = expf(cumk[(size_t)j * N + n0 + c]);
@@ -140,7 +146,8 @@ __global__ void __launch_bounds__(256) chunk_state_simt_kernel(
                         w = expf(cumk[Q - 1] - cumk[j]);
                     bv = to_f32(Bm[(((size_t)b * Tlen + t) * G + g) * N + n0 + c]) * w;
                 }
-                if (p0 + c < P) xv = to_f32(x[(((size_t)b * Tlen + t) * H + h) * P + p0 + c]);
+                if (p0 + c < P && SSD_INB((((size_t)b * Tlen + t) * H + h) * P + p0 + c, (long long)gridDim.y * Tlen * P))
+                    xv = to_f32(x[(((size_t)b * Tlen + t) * H + h) * P + p0 + c]);
             }
             Bs[jj][c] = bv;
             Xs[jj][c] = xv;
@@ -169,7 +176,8 @@ __global__ void __launch_bounds__(256) chunk_state_simt_kernel(
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int p = p0 + tp * 4 + j;
-            if (p < P) out[(size_t)n * P + p] = acc[i][j];
+            if (p < P && SSD_INB(out - states + (size_t)n * P + p, (long long)gridDim.y * nc * N * P))
+                out[(size_t)n * P + p] = acc[i][j];
         }
     }
 }
@@ -224,6 +232,12 @@ __global__ void __launch_bounds__(256) state_pass_kernel(const float* __restrict
     const long long bh = e / NP;
     const int r = (int)(e - bh * NP);
     const int n = r / P;
+    // every address below is (chain bh, its element r) at chunk k < nc: one
+    // check of the chain's last slot and decay covers them
+    if (!SSD_INB(bh * (long long)nc * NP + (long long)(nc - 1) * NP + r, total * nc) ||
+        !SSD_INB(bh * (long long)nc * Q * (DIAG ? N : 1) + (long long)nc * Q * (DIAG ? N : 1) - 1,
+                 total / NP * nc * Q * (DIAG ? N : 1)))
+        return;
     float* sp = states + bh * (long long)nc * NP + r;
     const float* ce = cum + bh * (long long)nc * Q * (DIAG ? N : 1) +
                       (DIAG ? (size_t)(Q - 1) * N + n : (size_t)(Q - 1));
@@ -302,7 +316,10 @@ __global__ void __launch_bounds__(256) chunk_scan_simt_kernel(
 
     for (int idx = tid; idx < 32 * N; idx += 256) {
         const int ii = idx / N, n = idx % N, i = i0 + ii;
-        Cs[ii * NS + n] = (i < qv) ? to_f32(Cm[(((size_t)b * Tlen + tk + i) * G + g) * N + n]) : 0.f;
+        Cs[ii * NS + n] = (i < qv && SSD_INB((((size_t)b * Tlen + tk + i) * G + g) * N + n,
+                                             (long long)(gridDim.y / H) * Tlen * G * N))
+                              ? to_f32(Cm[(((size_t)b * Tlen + tk + i) * G + g) * N + n])
+                              : 0.f;
     }
     if (tid < 32) cr[tid] = (i0 + tid < qv) ? cumk[i0 + tid] : 0.f;
 
@@ -314,13 +331,16 @@ __global__ void __launch_bounds__(256) chunk_scan_simt_kernel(
         __syncthreads();
         for (int idx = tid; idx < 32 * N; idx += 256) {
             const int jj = idx / N, n = idx % N, j = j0 + jj;
-            Bs[jj * NS + n] =
-                (j < qv) ? to_f32(Bm[(((size_t)b * Tlen + tk + j) * G + g) * N + n]) : 0.f;
+            Bs[jj * NS + n] = (j < qv && SSD_INB((((size_t)b * Tlen + tk + j) * G + g) * N + n,
+                                                 (long long)(gridDim.y / H) * Tlen * G * N))
+                                  ? to_f32(Bm[(((size_t)b * Tlen + tk + j) * G + g) * N + n])
+                                  : 0.f;
         }
         if (tid < 32) cc[tid] = (j0 + tid < qv) ? cumk[j0 + tid] : 0.f;
         for (int idx = tid; idx < 32 * 64; idx += 256) {
             const int jj = idx / 64, p = idx % 64, j = j0 + jj;
-            Xs[jj * 65 + p] = (j < qv && p0 + p < P)
+            Xs[jj * 65 + p] = (j < qv && p0 + p < P &&
+                               SSD_INB((((size_t)b * Tlen + tk + j) * H + h) * P + p0 + p, (long long)gridDim.y * Tlen * P))
                                   ? to_f32(x[(((size_t)b * Tlen + tk + j) * H + h) * P + p0 + p])
                                   : 0.f;
         }
@@ -355,7 +375,10 @@ __global__ void __launch_bounds__(256) chunk_scan_simt_kernel(
         __syncthreads();
         for (int idx = tid; idx < 32 * 64; idx += 256) {
             const int nn = idx / 64, p = idx % 64;
-            Hs[nn * 65 + p] = (n0 + nn < N && p0 + p < P) ? Hk[(size_t)(n0 + nn) * P + p0 + p] : 0.f;
+            Hs[nn * 65 + p] = (n0 + nn < N && p0 + p < P &&
+                               SSD_INB(Hk - Hin + (size_t)(n0 + nn) * P + p0 + p, (long long)gridDim.y * nc * N * P))
+                                  ? Hk[(size_t)(n0 + nn) * P + p0 + p]
+                                  : 0.f;
         }
         __syncthreads();
         const int nmax = min(32, N - n0);
@@ -373,7 +396,7 @@ __global__ void __launch_bounds__(256) chunk_scan_simt_kernel(
 #pragma unroll
     for (int m = 0; m < 8; ++m) {
         const int p = p0 + tp + 8 * m;
-        if (p < P) {
+        if (p < P && SSD_INB(row + p, (long long)gridDim.y * Tlen * P)) {
             const float xv = to_f32(x[row + p]);
             y[row + p] = from_f32<T>(fmaf(sc, acc2[m], acc[m]) + dv * xv);
         }

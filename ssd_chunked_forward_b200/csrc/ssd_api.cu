@@ -84,11 +84,13 @@ struct Workspace {
 };
 
 // Pieces per sequence of the split path: the largest power of two S with
-// T % S == 0, pieces of at least 4096 tokens and at most 1024 chains over all
-// pieces (so that the fused kernel's two-slot ring stays in L2); 1 when the
-// shape is not split.
+// T % S == 0, pieces of at least 4096 tokens and at most 512 chains over all
+// pieces (so that the fused kernel's two-slot ring, 64 KB per chain, stays in
+// L2: measured on the long-sequence workload, 1024 chains let most of the
+// hand-offs spill to DRAM, 256 make the chains too long); 1 when the shape is
+// not split.
 constexpr int kSplitMinPiece = 4096;
-constexpr long long kSplitMaxChains = 1024;
+constexpr long long kSplitMaxChains = 512;
 int split_pieces(const Dims& d) {
     if (!ssd::fused_supported(d) || !ssd::segment_state_tc_supported(d)) return 1;
     const long long chains = (long long)d.B * d.H;

@@ -14,6 +14,8 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libssd.so")
+# the index-checked build, loaded instead when SSD_DEBUG_CHECKS=1
+DEBUG_LIB_PATH = os.path.join(_HERE, "libssd_debug.so")
 
 SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_WORKSPACE, SSD_ERR_CUDA, SSD_ERR_TIMEOUT = range(6)
 SSD_DTYPE_F32, SSD_DTYPE_BF16 = 0, 1
@@ -29,7 +31,8 @@ EXPORTS = [
     "ssd_decode_step", "ssd_discretize", "ssd_decay_total", "ssd_state_combine",
     "ssd_segment_state", "ssd_backward", "ssd_backward_workspace_size",
     "ssd_test_fail_calls", "ssd_test_pending_failures", "ssd_split_pieces",
-    "ssd_device_status_where", "ssd_forward_discretized",
+    "ssd_device_status_where", "ssd_forward_discretized", "ssd_debug_build", "ssd_debug_record",
+    "ssd_debug_fail_all",
 ]
 
 
@@ -49,11 +52,14 @@ class Shape(ctypes.Structure):
 _lib = None
 
 
-def load(path: str = LIB_PATH):
-    """Open libssd.so (built by ``ssd_chunked_forward_b200.build``)."""
+def load(path: str = None):
+    """Open libssd.so (built by ``ssd_chunked_forward_b200.build``), or the
+    index-checked libssd_debug.so when the environment sets SSD_DEBUG_CHECKS=1."""
     global _lib
     if _lib is not None:
         return _lib
+    if path is None:
+        path = DEBUG_LIB_PATH if os.environ.get("SSD_DEBUG_CHECKS") == "1" else LIB_PATH
     if not os.path.exists(path):
         raise RuntimeError(f"libssd.so not built ({path}); run python -m ssd_chunked_forward_b200.build")
     lib = ctypes.CDLL(path)
@@ -76,6 +82,10 @@ def load(path: str = LIB_PATH):
     lib.ssd_device_status.argtypes = [vp, vp]
     ip = ctypes.POINTER(ctypes.c_int)
     lib.ssd_device_status_where.argtypes = [vp, vp, ip, ip, ip]
+    lib.ssd_debug_build.argtypes = []
+    lib.ssd_debug_build.restype = ctypes.c_int
+    lib.ssd_debug_record.argtypes = [ip, ip, ip, ip]
+    lib.ssd_debug_fail_all.argtypes = [ctypes.c_int]
     lib.ssd_chunk_cumsum.argtypes = [sp, fp, fp, vp]
     lib.ssd_chunk_state.argtypes = [sp, vp, vp, fp, fp, vp, ctypes.c_uint]
     lib.ssd_state_pass.argtypes = [sp, fp, fp, fp, vp]
@@ -223,6 +233,24 @@ def forward(x, a, Bm, Cm, D=None, chunk=256, *, y=None, final_state=None, want_f
 def device_status(workspace, stream=None) -> int:
     """Synchronise and return the workspace status word (SSD_OK or an error)."""
     return int(load().ssd_device_status(_ptr(workspace), _stream(stream)))
+
+
+def debug_build() -> bool:
+    """True when the loaded library is the index-checked debug build."""
+    return bool(load().ssd_debug_build())
+
+
+def debug_record():
+    """(failed checks, line, block, thread) since the last call, then cleared;
+    debug build only (raises SSDError otherwise)."""
+    vals = [ctypes.c_int(0) for _ in range(4)]
+    _check(load().ssd_debug_record(*(ctypes.byref(v) for v in vals)), "ssd_debug_record")
+    return tuple(v.value for v in vals)
+
+
+def debug_fail_all(on: bool) -> None:
+    """Debug build only: make every index check fail (and skip its access)."""
+    _check(load().ssd_debug_fail_all(1 if on else 0), "ssd_debug_fail_all")
 
 
 def device_status_where(workspace, stream=None):

@@ -36,6 +36,21 @@ def test_exports_every_declared_symbol(lib):
     assert sorted(ssd.EXPORTS) == names
 
 
+def test_debug_build_exports_and_reports(lib):
+    """The index-checked variant exports the same symbols and says it is the
+    debug build; the normal build says it is not and refuses the debug calls
+    (neither call touches the device)."""
+    import ctypes as C
+    from ssd_chunked_forward_b200.build import build
+    dbg = C.CDLL(build(debug=True))
+    for n in declared_functions():
+        assert hasattr(dbg, n), n
+    assert dbg.ssd_debug_build() == 1
+    assert lib.ssd_debug_build() == 0
+    assert lib.ssd_debug_record(None, None, None, None) == ssd.SSD_ERR_UNSUPPORTED
+    assert lib.ssd_debug_fail_all(1) == ssd.SSD_ERR_UNSUPPORTED
+
+
 def test_status_strings(lib):
     for code in range(6):
         s = ssd.status_string(code)

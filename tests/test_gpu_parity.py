@@ -392,6 +392,10 @@ DECODE_CASES = [
     small_case(B=2, T=1, H=3, P=70, N=33, G=3, chunk=1, dtype="f32", seed=72),
     small_case(B=2, T=1, H=4, P=64, N=64, G=1, chunk=1, dtype="bf16", a_per_state=True, seed=73),
     small_case(B=1, T=1, H=2, P=250, N=20, G=1, chunk=1, dtype="f32", seed=74),
+    # 16-byte kernel with the columns split over 4, 2 and 3 blocks (N = 256, P = 12)
+    small_case(B=2, T=1, H=3, P=128, N=256, G=1, chunk=1, dtype="f32", seed=76),
+    small_case(B=2, T=1, H=2, P=64, N=256, G=2, chunk=1, dtype="bf16", seed=77),
+    small_case(B=1, T=1, H=2, P=12, N=16, G=1, chunk=1, dtype="f32", a_per_state=True, seed=78),
 ]
 
 
