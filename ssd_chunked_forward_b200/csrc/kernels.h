@@ -93,11 +93,23 @@ cudaError_t launch_chunk_state_tc(const Dims& d, const void* x, const void* Bm, 
                                   int* status = nullptr);
 // the four chunk forms of the scalar-decay backward (y - Dx, dC, dx - D dy,
 // dB per head) as tcgen05 products; bf16, N = 128, P = 64, Q = 128 or 256
+// The y - Dx and dx - D dy forms do not store their rows: y - Dx leaves
+// r1 = dy . (y - Dx) per token and head, dx - D dy writes dx = (dx - D dy) + D dy
+// and leaves r2 = x . (dx - D dy) and xd = x . dy ([B][T][H] fp32 each).
+struct FormEpilogue {
+    const void* x;
+    const void* dy;
+    const float* D;
+    void* dx;
+    float* r1;
+    float* r2;
+    float* xd;
+};
 bool backward_forms_tc_supported(const Dims& d);
 cudaError_t launch_backward_forms_tc(const Dims& d, const void* x, const void* dy, const void* Bm,
                                      const void* Cm, const float* cum, const float* states,
-                                     const float* dstates, float* ytil, float* dCh, float* dxt,
-                                     float* dBh, int* status, cudaStream_t st);
+                                     const float* dstates, float* dCh, float* dBh, const FormEpilogue& ep,
+                                     int* status, cudaStream_t st);
 bool chunk_scan_tc_supported(const Dims& d);
 cudaError_t launch_chunk_scan_tc(const Dims& d, const void* x, const void* Bm, const void* Cm,
                                  const float* cum, const float* Hin, const float* D, void* y,

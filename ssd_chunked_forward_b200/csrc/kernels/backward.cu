@@ -307,6 +307,52 @@ __global__ void __launch_bounds__(256) token_grad_kernel(
     }
 }
 
+// da and the per-chunk dD share from the tensor-core forms' row sums: per
+// (chunk, b*H+h) one warp; lane l takes rows [Q/32 l, Q/32 (l+1)), suffix sums
+// within the lane, then across lanes, from the chunk's end (plus the boundary
+// term), as token_grad_kernel does from the stored rows.
+__global__ void __launch_bounds__(32) token_da_kernel(const float* __restrict__ r1, const float* __restrict__ r2,
+                                                      const float* __restrict__ xd, const float* __restrict__ cdot,
+                                                      float* __restrict__ da, float* __restrict__ dDpart, int Tlen,
+                                                      int H, int Q, int nc) {
+    const int k = blockIdx.x, bh = blockIdx.y, b = bh / H, h = bh % H;
+    const int lane = threadIdx.x;
+    const int tk = k * Q;
+    const int qv = min(Q, Tlen - tk);
+    const int per = (Q + 31) / 32;
+    const int j0 = lane * per;
+    if (!SSD_INB((((long long)b * Tlen + tk + qv - 1) * H + h), (long long)gridDim.y * Tlen) ||
+        !SSD_INB((long long)bh * nc + k, (long long)gridDim.y * nc))
+        return;  // the whole warp
+    float own = 0.f, dsum = 0.f;
+    for (int u = 0; u < per; ++u) {
+        const int j = j0 + u;
+        if (j < qv) {
+            const size_t t = ((size_t)b * Tlen + tk + j) * H + h;
+            own += r1[t] - r2[t];
+            dsum += xd[t];
+        }
+    }
+    // rows after this lane's: the lanes above, inclusive scan from the top
+    float above = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float v = __shfl_down_sync(0xffffffffu, above, o);
+        if (lane + o < 32) above += v;
+    }
+    float run = cdot[(size_t)bh * nc + k] + (above - own);
+    for (int u = per - 1; u >= 0; --u) {
+        const int j = j0 + u;
+        if (j < qv) {
+            const size_t t = ((size_t)b * Tlen + tk + j) * H + h;
+            run += r1[t] - r2[t];
+            da[t] = run;
+        }
+    }
+    dsum = warp_sum(dsum);
+    if (lane == 0) dDpart[(size_t)bh * nc + k] = dsum;
+}
+
 __global__ void dD_reduce_kernel(const float* __restrict__ dDpart, float* __restrict__ dD, int B,
                                  int H, int nc) {
     const int h = blockIdx.x * blockDim.x + threadIdx.x;
@@ -378,9 +424,15 @@ cudaError_t run_backward_t(const Dims& d, const BackwardArgs& g, const BackwardS
     const Opd oC{g.Cm, d.G * d.N, d.N, d.H / d.G, (long long)d.B * d.T * d.G * d.N};
     cudaError_t e;
     if (std::is_same<T, __nv_bfloat16>::value && backward_forms_tc_supported(d)) {
-        if ((e = launch_backward_forms_tc(d, g.x, g.dy, g.Bm, g.Cm, w.cum, w.states, w.dstates, w.ytil,
-                                          w.dCh, w.dxt, w.dBh, w.status, st)))
+        // the row sums for da and dD in the y - Dx buffer (3 x [B][T][H] of its [B][T][H][P])
+        const size_t bth = (size_t)d.B * d.T * d.H;
+        const FormEpilogue ep{g.x, g.dy, g.D, g.dx, w.ytil, w.ytil + bth, w.ytil + 2 * bth};
+        if ((e = launch_backward_forms_tc(d, g.x, g.dy, g.Bm, g.Cm, w.cum, w.states, w.dstates, w.dCh, w.dBh, ep,
+                                          w.status, st)))
             return e;
+        dim3 grid(d.nc, d.B * d.H);
+        token_da_kernel<<<grid, 32, 0, st>>>(ep.r1, ep.r2, ep.xd, w.cdot, g.da, w.dDpart, d.T, d.H, d.Q, d.nc);
+        return cudaGetLastError();
     } else {
         // y~ (causal; U = C, V = B, Z = x; Hin as N x P)
         if ((e = launch_form<T, false>(d, oC, oB, ox, w.cum, w.states, d.P, 1, w.ytil, d.N, d.P, st))) return e;

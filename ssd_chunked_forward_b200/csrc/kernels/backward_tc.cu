@@ -47,6 +47,14 @@ struct FormParams {
     int T, H, G, Q, nc, NP;
     int u_grp, v_grp, z_grp;  // operand indexed by B/C group (else by head)
     int* status;              // set to kDevTimeout when a bounded wait gives up
+    // epilogues that consume the row in place of storing it (EPI 1, 2):
+    const __nv_bfloat16* xg;   // x [B][T][H][P]
+    const __nv_bfloat16* dyg;  // dy [B][T][H][P]
+    const float* Dv;           // D [H] or null
+    __nv_bfloat16* dxo;        // EPI 2: dx = row + D dy [B][T][H][P]
+    float* r1;                 // EPI 1: dy . row per token and head [B][T][H]
+    float* r2;                 // EPI 2: x . row per token and head
+    float* xd;                 // EPI 2: x . dy per token and head
 };
 
 struct __align__(8) FormBars {
@@ -62,14 +70,17 @@ struct FormSmem {
     static constexpr uint32_t Z = R;
     static constexpr uint32_t M = R + 2 * (MC / 64) * kBox;                // MC/64 boxes of K rows
     static constexpr uint32_t CUM = R + (kV > kZM ? kV : kZM);             // [256] fp32
-    static constexpr uint32_t BAR = CUM + 256 * 4;
+    static constexpr uint32_t RED = CUM + 256 * 4;                         // [2][128] fp32 row partials
+    static constexpr uint32_t BAR = RED + 2 * 128 * 4;
     static constexpr uint32_t MISC = BAR + 64;
     static constexpr size_t bytes = 1024 + MISC + 16;
 };
 static_assert(FormSmem<128, 64>::bytes <= 113 * 1024 && FormSmem<64, 128>::bytes <= 113 * 1024,
               "two CTAs per SM");
 
-template <int K, int MC, bool ANTI, bool MROW>
+// EPI 0 stores the rows (fp32); EPI 1 (y - Dx) keeps only dy . row per row;
+// EPI 2 (dx - D dy) writes dx = row + D dy (bf16) and keeps x . row and x . dy
+template <int K, int MC, bool ANTI, bool MROW, int EPI>
 __global__ void __launch_bounds__(kFormThreads, 2)
     chunk_form_tc_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_v,
                          const __grid_constant__ CUtensorMap tm_z, const FormParams p) {
@@ -82,6 +93,7 @@ __global__ void __launch_bounds__(kFormThreads, 2)
     uint8_t* sZ = sm + L::Z;
     uint8_t* sM = sm + L::M;
     float* sCum = reinterpret_cast<float*>(sm + L::CUM);
+    float* sRed = reinterpret_cast<float*>(sm + L::RED);
     FormBars* bars = reinterpret_cast<FormBars*>(sm + L::BAR);
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + L::MISC);
 
@@ -330,20 +342,99 @@ __global__ void __launch_bounds__(kFormThreads, 2)
         const bool ok2 = tc::mbar_wait(&bars->o_full, 0, nullptr, kBudget);
         if (!__all_sync(0xffffffffu, ok2) && lane == 0) timed_out();
         ok = ok && __all_sync(0xffffffffu, ok2);
-        if (ok) {
-            tc::tc_fence_after();
-            float* o = p.out + (((size_t)b * p.T + tk + i) * p.H + h) * MC;
+        if (EPI == 0) {
+            if (ok) {
+                tc::tc_fence_after();
+                float* o = p.out + (((size_t)b * p.T + tk + i) * p.H + h) * MC;
 #pragma unroll
-            for (int q16 = 0; q16 < MC / 32; ++q16) {
-                const int m0 = half * (MC / 2) + 16 * q16;  // output column
+                for (int q16 = 0; q16 < MC / 32; ++q16) {
+                    const int m0 = half * (MC / 2) + 16 * q16;  // output column
+                    float v[16];
+                    tc::tmem_ld16(lane_base + col_o(m0 >> 6) + (m0 & 63), v);
+                    tc::tmem_ld_wait();
+                    if (i < qv && SSD_INB((o - p.out) + m0 + 15, (long long)gridDim.y * p.T * MC)) {
+#pragma unroll
+                        for (int e4 = 0; e4 < 4; ++e4)
+                            *reinterpret_cast<float4*>(o + m0 + 4 * e4) =
+                                make_float4(v[4 * e4], v[4 * e4 + 1], v[4 * e4 + 2], v[4 * e4 + 3]);
+                    }
+                }
+            }
+        } else {
+            // the row's half of the MC = P columns against the token's dy (and x)
+            // row: per-row dot products, summed over the two halves of a lane
+            // quadrant through shared memory, and (EPI 2) dx
+            static_assert(EPI == 0 || MC == 64, "row epilogues serve the P = 64 forms");
+            float pa = 0.f, pb = 0.f;  // EPI 1: dy . row; EPI 2: x . row, x . dy
+            const size_t ro = (((size_t)b * p.T + tk + i) * p.H + h) * MC + half * 32;
+            const bool live = ok && i < qv && SSD_INB((long long)ro + 31, (long long)gridDim.y * p.T * MC);
+            if (ok) tc::tc_fence_after();
+#pragma unroll
+            for (int q16 = 0; q16 < 2; ++q16) {
                 float v[16];
-                tc::tmem_ld16(lane_base + col_o(m0 >> 6) + (m0 & 63), v);
-                tc::tmem_ld_wait();
-                if (i < qv && SSD_INB((o - p.out) + m0 + 15, (long long)gridDim.y * p.T * MC)) {
+                if (ok) {
+                    tc::tmem_ld16(lane_base + col_o(0) + half * 32 + 16 * q16, v);
+                    tc::tmem_ld_wait();
+                }
+                if (live) {
+                    float dyv[16], xv[16];
+                    const uint4* dyp = reinterpret_cast<const uint4*>(p.dyg + ro + 16 * q16);
 #pragma unroll
-                    for (int e4 = 0; e4 < 4; ++e4)
-                        *reinterpret_cast<float4*>(o + m0 + 4 * e4) =
-                            make_float4(v[4 * e4], v[4 * e4 + 1], v[4 * e4 + 2], v[4 * e4 + 3]);
+                    for (int u = 0; u < 2; ++u) {
+                        const uint4 w = __ldg(dyp + u);
+                        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = tc::unpack_bf16x2(ws[e]);
+                            dyv[8 * u + 2 * e] = f.x;
+                            dyv[8 * u + 2 * e + 1] = f.y;
+                        }
+                    }
+                    if (EPI == 1) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) pa = fmaf(dyv[e], v[e], pa);
+                    } else {
+                        const uint4* xp = reinterpret_cast<const uint4*>(p.xg + ro + 16 * q16);
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const uint4 w = __ldg(xp + u);
+                            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 f = tc::unpack_bf16x2(ws[e]);
+                                xv[8 * u + 2 * e] = f.x;
+                                xv[8 * u + 2 * e + 1] = f.y;
+                            }
+                        }
+                        const float dv = p.Dv ? __ldg(p.Dv + h) : 0.f;
+                        uint32_t pk[8];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            pa = fmaf(xv[e], v[e], pa);
+                            pb = fmaf(xv[e], dyv[e], pb);
+                        }
+#pragma unroll
+                        for (int e2 = 0; e2 < 8; ++e2)
+                            pk[e2] = tc::pack_bf16x2(fmaf(dv, dyv[2 * e2], v[2 * e2]),
+                                                     fmaf(dv, dyv[2 * e2 + 1], v[2 * e2 + 1]));
+                        uint4* dxp = reinterpret_cast<uint4*>(p.dxo + ro + 16 * q16);
+                        dxp[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        dxp[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                    }
+                }
+            }
+            if (half == 1) {
+                sRed[row] = pa;
+                sRed[128 + row] = pb;
+            }
+            pair_sync();  // both halves of every quadrant, whatever ok says
+            if (live && half == 0) {
+                const size_t tr = ((size_t)b * p.T + tk + i) * p.H + h;
+                if (EPI == 1) {
+                    p.r1[tr] = pa + sRed[row];
+                } else {
+                    p.r2[tr] = pa + sRed[row];
+                    p.xd[tr] = pb + sRed[128 + row];
                 }
             }
         }
@@ -356,9 +447,9 @@ __global__ void __launch_bounds__(kFormThreads, 2)
     }
 }
 
-template <int K, int MC, bool ANTI, bool MROW>
+template <int K, int MC, bool ANTI, bool MROW, int EPI>
 cudaError_t launch_form_tc_t(const Dims& d, const void* U, int ug, const void* V, int vg, const void* Z, int zg,
-                             const float* cum, const float* Mst, float* out,
+                             const float* cum, const float* Mst, float* out, const FormEpilogue& ep,
                              int* status, cudaStream_t st) {
     CUtensorMap tu, tv, tz;
     cudaError_t e = make_tmap_bf16_4d(&tu, U, K, ug ? d.G : d.H, d.T, d.B, kRowsT);
@@ -370,12 +461,14 @@ cudaError_t launch_form_tc_t(const Dims& d, const void* U, int ug, const void* V
     p.T = d.T; p.H = d.H; p.G = d.G; p.Q = d.Q; p.nc = d.nc; p.NP = d.N * d.P;
     p.u_grp = ug; p.v_grp = vg; p.z_grp = zg;
     p.status = status;
+    p.xg = (const __nv_bfloat16*)ep.x; p.dyg = (const __nv_bfloat16*)ep.dy; p.Dv = ep.D;
+    p.dxo = (__nv_bfloat16*)ep.dx; p.r1 = ep.r1; p.r2 = ep.r2; p.xd = ep.xd;
     using L = FormSmem<K, MC>;
-    e = cudaFuncSetAttribute(chunk_form_tc_kernel<K, MC, ANTI, MROW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(chunk_form_tc_kernel<K, MC, ANTI, MROW, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)L::bytes);
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)(d.nc * (d.Q / kRowsT)), (unsigned)(d.B * d.H));
-    chunk_form_tc_kernel<K, MC, ANTI, MROW><<<grid, kFormThreads, L::bytes, st>>>(tu, tv, tz, p);
+    chunk_form_tc_kernel<K, MC, ANTI, MROW, EPI><<<grid, kFormThreads, L::bytes, st>>>(tu, tv, tz, p);
     return cudaGetLastError();
 }
 
@@ -388,21 +481,22 @@ bool backward_forms_tc_supported(const Dims& d) {
 
 cudaError_t launch_backward_forms_tc(const Dims& d, const void* x, const void* dy, const void* Bm,
                                      const void* Cm, const float* cum, const float* states,
-                                     const float* dstates, float* ytil, float* dCh, float* dxt, float* dBh,
+                                     const float* dstates, float* dCh, float* dBh, const FormEpilogue& ep,
                                      int* status, cudaStream_t st) {
     if (!backward_forms_tc_supported(d)) return cudaErrorNotSupported;
+    const FormEpilogue none{};
     cudaError_t e;
-    // y - D x: causal, U = C, V = B, Z = x, M = Hin (N x P)
-    e = launch_form_tc_t<128, 64, false, true>(d, Cm, 1, Bm, 1, x, 0, cum, states, ytil, status, st);
+    // y - D x: causal, U = C, V = B, Z = x, M = Hin (N x P); only dy . (y - Dx) is kept
+    e = launch_form_tc_t<128, 64, false, true, 1>(d, Cm, 1, Bm, 1, x, 0, cum, states, nullptr, ep, status, st);
     if (e != cudaSuccess) return e;
     // dC per head: causal, U = dy, V = x, Z = B, M = Hin read as P x N
-    e = launch_form_tc_t<64, 128, false, false>(d, dy, 0, x, 0, Bm, 1, cum, states, dCh, status, st);
+    e = launch_form_tc_t<64, 128, false, false, 0>(d, dy, 0, x, 0, Bm, 1, cum, states, dCh, none, status, st);
     if (e != cudaSuccess) return e;
-    // dx - D dy: anti-causal, U = B, V = C, Z = dy, M = G (N x P)
-    e = launch_form_tc_t<128, 64, true, true>(d, Bm, 1, Cm, 1, dy, 0, cum, dstates, dxt, status, st);
+    // dx - D dy: anti-causal, U = B, V = C, Z = dy, M = G (N x P); dx, x . (dx - D dy) and x . dy kept
+    e = launch_form_tc_t<128, 64, true, true, 2>(d, Bm, 1, Cm, 1, dy, 0, cum, dstates, nullptr, ep, status, st);
     if (e != cudaSuccess) return e;
     // dB per head: anti-causal, U = x, V = dy, Z = C, M = G read as P x N
-    return launch_form_tc_t<64, 128, true, false>(d, x, 0, dy, 0, Cm, 1, cum, dstates, dBh, status, st);
+    return launch_form_tc_t<64, 128, true, false, 0>(d, x, 0, dy, 0, Cm, 1, cum, dstates, dBh, none, status, st);
 }
 
 }  // namespace ssd
