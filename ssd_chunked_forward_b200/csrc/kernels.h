@@ -93,7 +93,8 @@ cudaError_t launch_chunk_state_tc(const Dims& d, const void* x, const void* Bm, 
                                   int* status = nullptr);
 // the four chunk forms of the scalar-decay backward (y - Dx, dC, dx - D dy,
 // dB per head) as tcgen05 products; bf16, N = 128, P = 64, Q = 128 or 256
-// The y - Dx and dx - D dy forms do not store their rows: y - Dx leaves
+// dC and dB come out summed over each group's heads (bf16 [B][T][G][N], the
+// final gradients).  The y - Dx and dx - D dy forms do not store their rows: y - Dx leaves
 // r1 = dy . (y - Dx) per token and head, dx - D dy writes dx = (dx - D dy) + D dy
 // and leaves r2 = x . (dx - D dy) and xd = x . dy ([B][T][H] fp32 each).
 struct FormEpilogue {
@@ -108,7 +109,7 @@ struct FormEpilogue {
 bool backward_forms_tc_supported(const Dims& d);
 cudaError_t launch_backward_forms_tc(const Dims& d, const void* x, const void* dy, const void* Bm,
                                      const void* Cm, const float* cum, const float* states,
-                                     const float* dstates, float* dCh, float* dBh, const FormEpilogue& ep,
+                                     const float* dstates, void* dCm, void* dBm, const FormEpilogue& ep,
                                      int* status, cudaStream_t st);
 bool chunk_scan_tc_supported(const Dims& d);
 cudaError_t launch_chunk_scan_tc(const Dims& d, const void* x, const void* Bm, const void* Cm,

@@ -427,7 +427,7 @@ cudaError_t run_backward_t(const Dims& d, const BackwardArgs& g, const BackwardS
         // the row sums for da and dD in the y - Dx buffer (3 x [B][T][H] of its [B][T][H][P])
         const size_t bth = (size_t)d.B * d.T * d.H;
         const FormEpilogue ep{g.x, g.dy, g.D, g.dx, w.ytil, w.ytil + bth, w.ytil + 2 * bth};
-        if ((e = launch_backward_forms_tc(d, g.x, g.dy, g.Bm, g.Cm, w.cum, w.states, w.dstates, w.dCh, w.dBh, ep,
+        if ((e = launch_backward_forms_tc(d, g.x, g.dy, g.Bm, g.Cm, w.cum, w.states, w.dstates, g.dCm, g.dBm, ep,
                                           w.status, st)))
             return e;
         dim3 grid(d.nc, d.B * d.H);
@@ -463,6 +463,8 @@ cudaError_t finish_t(const Dims& d, const BackwardArgs& g, const BackwardScratch
         dD_reduce_kernel<<<(d.H + 127) / 128, 128, 0, st>>>(w.dDpart, g.dD, d.B, d.H, d.nc);
         if ((e = cudaGetLastError())) return e;
     }
+    // (the tensor-core forms write dB and dC summed over the group already)
+    if (std::is_same<T, __nv_bfloat16>::value && backward_forms_tc_supported(d)) return cudaSuccess;
     const long long rows = (long long)d.B * d.T;
     const long long total = rows * d.G * d.N;
     group_sum_kernel<T><<<(unsigned)((total + 255) / 256), 256, 0, st>>>(

@@ -447,6 +447,336 @@ __global__ void __launch_bounds__(kFormThreads, 2)
     }
 }
 
+// ---------------------------------------------------------------------------
+// dC and dB summed over the heads of a B/C group in one CTA (K = P = 64,
+// MC = N = 128): per (chunk, 128-row tile, batch x group) the CTA walks the
+// group's heads, each head's S = U_h V_h^T, scores and U~_h M_h as above,
+// accumulating out = sum_h (P~_h Z + U~_h M_h) in TMEM (Z = B or C is the
+// group's own, loaded once), and stores the group sum as bf16 -- the per-head
+// fp32 rows and the separate sum over heads are never written.  The next
+// head's U and V rows load (TMA, two stages) under the current head's
+// products.  TMEM: S at columns 0-255 (scores packed in place), out at
+// 256-383.
+struct GroupFormParams {
+    const float* cum;  // [B*H][nc][Q]
+    const float* Mst;  // [B*H][nc][N*P], read as P x N
+    __nv_bfloat16* out;  // [B][T][G][N]
+    int T, H, G, Q, nc, NP;
+    int* status;
+};
+
+struct __align__(8) GroupFormBars {
+    uint64_t full[2], z_full, s_full, p_full, o_done;
+};
+
+struct GroupFormSmem {
+    static constexpr uint32_t U = 0;                   // 2 stages x 1 box (K = 64)
+    static constexpr uint32_t V = U + 2 * kBox;        // 2 stages x 2 tiles
+    static constexpr uint32_t Z = V + 4 * kBox;        // 2 tiles x 2 boxes (MC = 128)
+    static constexpr uint32_t M = Z + 4 * kBox;        // 2 boxes of 64 rows
+    static constexpr uint32_t CUM = M + 2 * 64 * 128;  // 2 stages x [256] fp32
+    static constexpr uint32_t BAR = CUM + 2 * 256 * 4;
+    static constexpr uint32_t MISC = BAR + 64;
+    static constexpr size_t bytes = 1024 + MISC + 16;
+};
+static_assert(GroupFormSmem::bytes <= 227 * 1024, "shared memory");
+
+template <bool ANTI>
+__global__ void __launch_bounds__(kFormThreads, 1)
+    chunk_form_group_tc_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_v,
+                               const __grid_constant__ CUtensorMap tm_z, const GroupFormParams p) {
+    using L = GroupFormSmem;
+    constexpr int K = 64, MC = 128;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+    uint8_t* sU = sm + L::U;
+    uint8_t* sV = sm + L::V;
+    uint8_t* sZ = sm + L::Z;
+    uint8_t* sM = sm + L::M;
+    float* sCum = reinterpret_cast<float*>(sm + L::CUM);
+    GroupFormBars* bars = reinterpret_cast<GroupFormBars*>(sm + L::BAR);
+    uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + L::MISC);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ntile = p.Q / kRowsT;
+    const int k = blockIdx.x / ntile, i0 = (blockIdx.x % ntile) * kRowsT;
+    const int bg = blockIdx.y, b = bg / p.G, g = bg % p.G;
+    const int HG = p.H / p.G, hfirst = g * HG;
+    const int tk = k * p.Q;
+    const int qv = min(p.Q, p.T - tk);
+    const int jbase = ANTI ? i0 : 0;
+    const int nt = ANTI ? (p.Q - i0) / kRowsT : i0 / kRowsT + 1;
+    if (i0 >= qv) return;  // a tile wholly past T: nothing to write
+    {
+        // the group's last head bounds the decay and state reads (the whole
+        // block leaves before any barrier if not)
+        const long long last = ((long long)b * p.H + hfirst + HG - 1) * p.nc + k;
+        if (!SSD_INB((last + 1) * p.Q - 1, (long long)(gridDim.y / p.G) * p.H * p.nc * p.Q) ||
+            !SSD_INB((last + 1) * p.NP - 1, (long long)(gridDim.y / p.G) * p.H * p.nc * p.NP))
+            return;
+    }
+
+    if (threadIdx.x == 0) {
+        tc::mbar_init(&bars->full[0], 1);
+        tc::mbar_init(&bars->full[1], 1);
+        tc::mbar_init(&bars->z_full, 1);
+        tc::mbar_init(&bars->s_full, 1);
+        tc::mbar_init(&bars->p_full, 8);
+        tc::mbar_init(&bars->o_done, 1);
+        tc::fence_mbar_init();
+    }
+    if (warp == 0) {
+        tc::tmem_alloc(sTmem, 512);
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = *sTmem;
+    constexpr uint32_t COL_OUT = 256;
+    constexpr uint64_t kBudget = 2000000000ull;  // 2 s per wait
+    auto timed_out = [&]() {
+        if (p.status) atomicExch(p.status, kDevTimeout);
+    };
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------ copies and products ----
+            auto load_head = [&](int hh) {
+                const int st = hh & 1, h = hfirst + hh;
+                tc::mbar_arrive_expect_tx(&bars->full[st], (uint32_t)(kBox * (1 + nt)));
+                tc::tma_load_4d(sU + st * kBox, &tm_u, &bars->full[st], 0, h, tk + i0, b);
+                for (int v = 0; v < nt; ++v)
+                    tc::tma_load_4d(sV + (2 * st + v) * kBox, &tm_v, &bars->full[st], 0, h, tk + jbase + v * kRowsT, b);
+            };
+            tc::mbar_arrive_expect_tx(&bars->z_full, (uint32_t)(2 * kBox * nt));
+            for (int v = 0; v < nt; ++v)
+                for (int q = 0; q < 2; ++q)
+                    tc::tma_load_4d(sZ + (2 * v + q) * kBox, &tm_z, &bars->z_full, 64 * q, g, tk + jbase + v * kRowsT, b);
+            load_head(0);
+            bool ok = tc::mbar_wait(&bars->z_full, 0, nullptr, kBudget);
+            constexpr uint32_t id_s = tc::idesc_bf16_f32(128, 128, 0, 0);
+            constexpr uint32_t id_o = tc::idesc_bf16_f32(128, 64, 0, 1);
+            for (int hh = 0; hh < HG; ++hh) {
+                const int st = hh & 1;
+                // the previous head's products are done: its S columns, its
+                // U stage and sM may be reused
+                if (hh > 0) ok = ok && tc::mbar_wait(&bars->o_done, (hh - 1) & 1, nullptr, kBudget);
+                if (!ok) break;
+                if (hh + 1 < HG) load_head(hh + 1);
+                ok = tc::mbar_wait(&bars->full[st], (hh >> 1) & 1, nullptr, kBudget);
+                if (!ok) break;
+                tc::tc_fence_after();
+                const uint64_t dU = tc::smem_desc_sw128(tc::smem_u32(sU + st * kBox), 16, 1024);
+                for (int v = 0; v < nt; ++v) {
+                    const uint64_t dV = tc::smem_desc_sw128(tc::smem_u32(sV + (2 * st + v) * kBox), 16, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < K / 16; ++kk)
+                        tc::mma_ss(tmem + 128 * v, tc::desc_adv(dU, kk * 32), tc::desc_adv(dV, kk * 32), id_s, kk > 0);
+                }
+                tc::mma_commit(&bars->s_full);
+                ok = tc::mbar_wait(&bars->p_full, hh & 1, nullptr, kBudget);
+                if (!ok) break;
+                tc::tc_fence_after();
+                for (int v = 0; v < nt; ++v)
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const uint64_t dZ = tc::smem_desc_sw128(tc::smem_u32(sZ + (2 * v + q) * kBox), kBox, 1024);
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            tc::mma_ts(tmem + COL_OUT + 64 * q, tmem + 128 * v + kk * 8, tc::desc_adv(dZ, kk * 2048),
+                                       id_o, (hh > 0 || v > 0 || kk > 0) ? 1u : 0u);
+                    }
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const uint64_t dM = tc::smem_desc_sw128(tc::smem_u32(sM + q * (K * 128)), K * 128, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < K / 16; ++kk)
+                        tc::mma_ss(tmem + COL_OUT + 64 * q, tc::desc_adv(dU, kk * 32), tc::desc_adv(dM, kk * 2048), id_o,
+                                   1u);
+                }
+                tc::mma_commit(&bars->o_done);
+            }
+            // every product done before the epilogue and the exit
+            if (!tc::mbar_wait(&bars->o_done, (HG - 1) & 1, nullptr, kBudget) || !ok) timed_out();
+        }
+    } else {
+        // ---------------------------------------------------- math warps ----
+        const int mw = warp - 1;
+        const int quad = warp & 3;
+        const int half = mw >> 2;
+        const int row = quad * 32 + lane;
+        const int i = i0 + row;
+        const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+        const int mt = threadIdx.x - 32;  // 0..255
+        auto pair_sync = [&]() {
+            tc::tc_fence_before();
+            switch (quad) {
+                case 0: asm volatile("bar.sync 1, 64;" ::: "memory"); break;
+                case 1: asm volatile("bar.sync 2, 64;" ::: "memory"); break;
+                case 2: asm volatile("bar.sync 3, 64;" ::: "memory"); break;
+                default: asm volatile("bar.sync 4, 64;" ::: "memory"); break;
+            }
+            tc::tc_fence_after();
+        };
+        auto math_sync = [&]() { asm volatile("bar.sync 5, 256;" ::: "memory"); };
+        // OR of a predicate over the 256 math threads (so that they all take
+        // the same branch: the pair barriers below must stay matched)
+        auto math_or = [&](bool pred) -> bool {
+            uint32_t r;
+            asm volatile(
+                "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\t"
+                "bar.red.or.pred po, 6, 256, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}"
+                : "=r"(r)
+                : "r"((uint32_t)pred)
+                : "memory");
+            return r != 0;
+        };
+        const int kk4 = (mt % (K / 4)) * 4, m8 = (mt / (K / 4)) * 8;  // this thread's 4 x 8 block of M
+        bool ok = true;
+        for (int hh = 0; hh < HG; ++hh) {
+            const int st = hh & 1, h = hfirst + hh;
+            const size_t chain = (size_t)b * p.H + h;
+            float* cumh = sCum + st * 256;
+            // the head's in-chunk decays, and its state read ahead ([N][P]: M[p][n])
+            for (int t = mt; t < p.Q; t += 256) cumh[t] = p.cum[(chain * p.nc + k) * p.Q + t];
+            const float* Mk = p.Mst + (chain * p.nc + k) * (size_t)p.NP;
+            float4 mv[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mv[e] = *reinterpret_cast<const float4*>(Mk + (size_t)(m8 + e) * K + kk4);
+            math_sync();  // cumh complete
+            const float ci = cumh[i];
+            const float cend = cumh[p.Q - 1];
+            bool okh = ok && tc::mbar_wait(&bars->s_full, hh & 1, nullptr, kBudget);
+            if (!okh) timed_out();
+            okh = !math_or(!okh);
+            // M into sM (the previous head's products are done: S of this head was
+            // issued after them)
+            {
+                auto put = [&](int kk, float f0, float f1, float f2, float f3, float f4, float f5, float f6, float f7) {
+                    const uint4 w = make_uint4(tc::pack_bf16x2(f0, f1), tc::pack_bf16x2(f2, f3),
+                                               tc::pack_bf16x2(f4, f5), tc::pack_bf16x2(f6, f7));
+                    *reinterpret_cast<uint4*>(sM + (m8 >> 6) * (K * 128) + tc::sw128_offset(kk, (m8 & 63) >> 3)) = w;
+                };
+                put(kk4, mv[0].x, mv[1].x, mv[2].x, mv[3].x, mv[4].x, mv[5].x, mv[6].x, mv[7].x);
+                put(kk4 + 1, mv[0].y, mv[1].y, mv[2].y, mv[3].y, mv[4].y, mv[5].y, mv[6].y, mv[7].y);
+                put(kk4 + 2, mv[0].z, mv[1].z, mv[2].z, mv[3].z, mv[4].z, mv[5].z, mv[6].z, mv[7].z);
+                put(kk4 + 3, mv[0].w, mv[1].w, mv[2].w, mv[3].w, mv[4].w, mv[5].w, mv[6].w, mv[7].w);
+            }
+            const int npc = nt == 2 ? 2 : 1;
+            if (okh) {
+                tc::tc_fence_after();
+                const float uf = ANTI ? ex2_approx((cend - ci) * 1.4426950408889634f)
+                                      : ex2_approx(ci * 1.4426950408889634f);
+                const uint32_t u2 = tc::pack_bf16x2(uf, uf);
+                uint8_t* sUs = sU + st * kBox;
+#pragma unroll
+                for (int cc = 0; cc < K / 16; ++cc) {
+                    const int c = half * (K / 16) + cc;
+                    uint4* ptr = reinterpret_cast<uint4*>(sUs + tc::sw128_offset(row, c));
+                    uint4 v = *ptr;
+                    v.x = tc::mul_bf16x2(v.x, u2);
+                    v.y = tc::mul_bf16x2(v.y, u2);
+                    v.z = tc::mul_bf16x2(v.z, u2);
+                    v.w = tc::mul_bf16x2(v.w, u2);
+                    *ptr = v;
+                }
+                for (int u = 0; u < npc; ++u) {
+                    const int tile = nt == 2 ? half : 0;
+                    const int c0 = nt == 2 ? 64 * u : 64 * half;
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) {
+                        const int cin = c0 + 32 * r;
+                        const uint32_t tbase = lane_base + 128 * tile;
+                        float sv[32];
+                        tc::tmem_ld16(tbase + cin, *reinterpret_cast<float(*)[16]>(sv));
+                        tc::tmem_ld16(tbase + cin + 16, *reinterpret_cast<float(*)[16]>(sv + 16));
+                        tc::tmem_ld_wait();
+                        if (r == (c0 == 0 ? 1 : 0)) pair_sync();
+                        const int j0 = jbase + 128 * tile + cin;
+#pragma unroll
+                        for (int g8 = 0; g8 < 2; ++g8) {
+                            uint32_t pk[8];
+#pragma unroll
+                            for (int e2 = 0; e2 < 8; ++e2) {
+                                float pv[2];
+#pragma unroll
+                                for (int q = 0; q < 2; ++q) {
+                                    const int e = 16 * g8 + 2 * e2 + q;
+                                    const int j = j0 + e;
+                                    const bool keep = (ANTI ? j >= i : j <= i) && j < qv && i < qv;
+                                    const float ex = ex2_approx(
+                                        keep ? (ANTI ? cumh[j] - ci : ci - cumh[j]) * 1.4426950408889634f : 0.f);
+                                    pv[q] = keep ? sv[e] * ex : 0.f;
+                                }
+                                pk[e2] = tc::pack_bf16x2(pv[0], pv[1]);
+                            }
+                            tc::tmem_st8(tbase + cin / 2 + 8 * g8, pk);
+                        }
+                    }
+                }
+                tc::tmem_st_wait();
+            } else {
+                for (int u = 0; u < npc; ++u) pair_sync();
+            }
+            tc::fence_proxy_async_smem();  // U~ and M for the products
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&bars->p_full);
+            ok = okh;
+            if (!ok) break;
+        }
+        // the group sum, as bf16, straight from TMEM
+        const bool okf = __all_sync(0xffffffffu, ok && tc::mbar_wait(&bars->o_done, (HG - 1) & 1, nullptr, kBudget));
+        if (okf) {
+            tc::tc_fence_after();
+            const size_t ro = (((size_t)b * p.T + tk + i) * p.G + g) * MC + half * 64;
+            const bool live = i < qv && SSD_INB((long long)ro + 63, (long long)(gridDim.y / p.G) * p.T * p.G * MC);
+#pragma unroll
+            for (int q16 = 0; q16 < 4; ++q16) {
+                float v[16];
+                tc::tmem_ld16(lane_base + COL_OUT + half * 64 + 16 * q16, v);
+                tc::tmem_ld_wait();
+                if (live) {
+                    uint32_t pk[8];
+#pragma unroll
+                    for (int e2 = 0; e2 < 8; ++e2) pk[e2] = tc::pack_bf16x2(v[2 * e2], v[2 * e2 + 1]);
+                    uint4* dst = reinterpret_cast<uint4*>(p.out + ro + 16 * q16);
+                    dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                }
+            }
+        }
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, 512);
+    }
+}
+
+template <bool ANTI>
+cudaError_t launch_form_group_tc_t(const Dims& d, const void* U, const void* V, const void* Z, const float* cum,
+                                   const float* Mst, void* out, int* status, cudaStream_t st) {
+    CUtensorMap tu, tv, tz;
+    cudaError_t e = make_tmap_bf16_4d(&tu, U, d.P, d.H, d.T, d.B, kRowsT);
+    if (e == cudaSuccess) e = make_tmap_bf16_4d(&tv, V, d.P, d.H, d.T, d.B, kRowsT);
+    if (e == cudaSuccess) e = make_tmap_bf16_4d(&tz, Z, d.N, d.G, d.T, d.B, kRowsT);
+    if (e != cudaSuccess) return e;
+    GroupFormParams p = {};
+    p.cum = cum; p.Mst = Mst; p.out = (__nv_bfloat16*)out;
+    p.T = d.T; p.H = d.H; p.G = d.G; p.Q = d.Q; p.nc = d.nc; p.NP = d.N * d.P;
+    p.status = status;
+    e = cudaFuncSetAttribute(chunk_form_group_tc_kernel<ANTI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)GroupFormSmem::bytes);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((unsigned)(d.nc * (d.Q / kRowsT)), (unsigned)(d.B * d.G));
+    chunk_form_group_tc_kernel<ANTI><<<grid, kFormThreads, GroupFormSmem::bytes, st>>>(tu, tv, tz, p);
+    return cudaGetLastError();
+}
+
 template <int K, int MC, bool ANTI, bool MROW, int EPI>
 cudaError_t launch_form_tc_t(const Dims& d, const void* U, int ug, const void* V, int vg, const void* Z, int zg,
                              const float* cum, const float* Mst, float* out, const FormEpilogue& ep,
@@ -481,22 +811,21 @@ bool backward_forms_tc_supported(const Dims& d) {
 
 cudaError_t launch_backward_forms_tc(const Dims& d, const void* x, const void* dy, const void* Bm,
                                      const void* Cm, const float* cum, const float* states,
-                                     const float* dstates, float* dCh, float* dBh, const FormEpilogue& ep,
+                                     const float* dstates, void* dCm, void* dBm, const FormEpilogue& ep,
                                      int* status, cudaStream_t st) {
     if (!backward_forms_tc_supported(d)) return cudaErrorNotSupported;
-    const FormEpilogue none{};
     cudaError_t e;
     // y - D x: causal, U = C, V = B, Z = x, M = Hin (N x P); only dy . (y - Dx) is kept
     e = launch_form_tc_t<128, 64, false, true, 1>(d, Cm, 1, Bm, 1, x, 0, cum, states, nullptr, ep, status, st);
     if (e != cudaSuccess) return e;
-    // dC per head: causal, U = dy, V = x, Z = B, M = Hin read as P x N
-    e = launch_form_tc_t<64, 128, false, false, 0>(d, dy, 0, x, 0, Bm, 1, cum, states, dCh, none, status, st);
+    // dC summed over each group's heads: causal, U = dy, V = x, Z = B, M = Hin read as P x N
+    e = launch_form_group_tc_t<false>(d, dy, x, Bm, cum, states, dCm, status, st);
     if (e != cudaSuccess) return e;
     // dx - D dy: anti-causal, U = B, V = C, Z = dy, M = G (N x P); dx, x . (dx - D dy) and x . dy kept
     e = launch_form_tc_t<128, 64, true, true, 2>(d, Bm, 1, Cm, 1, dy, 0, cum, dstates, nullptr, ep, status, st);
     if (e != cudaSuccess) return e;
-    // dB per head: anti-causal, U = x, V = dy, Z = C, M = G read as P x N
-    return launch_form_tc_t<64, 128, true, false, 0>(d, x, 0, dy, 0, Cm, 1, cum, dstates, dBh, none, status, st);
+    // dB summed over each group's heads: anti-causal, U = x, V = dy, Z = C, M = G read as P x N
+    return launch_form_group_tc_t<true>(d, x, dy, Cm, cum, dstates, dBm, status, st);
 }
 
 }  // namespace ssd
