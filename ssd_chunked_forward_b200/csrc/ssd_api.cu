@@ -198,6 +198,10 @@ bool injected_failure() { return ssd::take_injected_failure(); }
 size_t backward_layout(const Dims& d, void* base, ssd::BackwardScratch* w) {
     const size_t f = sizeof(float);
     const size_t chains = (size_t)d.B * d.H;
+    // the tensor-core forms keep three row sums per token and head in the
+    // y - Dx slot and write dx, dB and dC themselves: no per-head rows
+    const bool tc = ssd::backward_forms_tc_supported(d);
+    const size_t bth = (size_t)d.B * d.T * d.H;
     const size_t sizes[10] = {
         chains * d.nc * d.Q * (d.diag ? d.N : 1) * f,  // cum
         chains * d.nc * d.N * d.P * f,            // states
@@ -205,10 +209,10 @@ size_t backward_layout(const Dims& d, void* base, ssd::BackwardScratch* w) {
         chains * d.N * d.P * f,                   // fin
         chains * d.nc * (d.diag ? d.N : 1) * f,   // cdot
         chains * d.nc * f,                        // dDpart
-        d.diag ? 0 : (size_t)d.B * d.T * d.H * d.P * f,  // ytil
-        (size_t)d.B * d.T * d.H * d.P * f,        // dxt
-        (size_t)d.B * d.T * d.H * d.N * f,        // dBh
-        (size_t)d.B * d.T * d.H * d.N * f,        // dCh
+        tc ? 3 * bth * f : (d.diag ? 0 : bth * d.P * f),  // ytil (tensor cores: r1, r2, x . dy)
+        tc ? 0 : bth * d.P * f,                   // dxt
+        tc ? 0 : bth * d.N * f,                   // dBh
+        tc ? 0 : bth * d.N * f,                   // dCh
     };
     float** slots[10] = {};
     if (w) {

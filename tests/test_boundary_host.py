@@ -112,14 +112,18 @@ def test_ragged_T_is_a_partial_last_chunk(lib, T, chunk):
 
 def test_backward_workspace_and_validation(lib):
     """The backward's workspace holds the recomputed and adjoint chunk states
-    and the fp32 per-head partials; the per-state variant is served up to
-    N = 128; bad pointers and a short workspace are refused before any launch."""
-    s = _shape()  # B=2, T=512, H=4, P=64, N=128, chunk 256
+    and, on CUDA cores, the fp32 per-head partials (the tensor-core path keeps
+    three row sums per token and head instead); the per-state variant is
+    served up to N = 128; bad pointers and a short workspace are refused
+    before any launch."""
+    s = _shape()  # B=2, T=512, H=4, P=64, N=128, chunk 256, bf16: tensor cores
     need = ssd.backward_workspace_size(s)
     nc, f = 2, 4
-    pieces = [2 * 4 * nc * 256 * f, 2 * 2 * 4 * nc * 128 * 64 * f, 2 * 4 * 128 * 64 * f,
-              2 * 2 * 512 * 4 * 64 * f, 2 * 2 * 512 * 4 * 128 * f]
-    assert need >= sum(pieces)
+    states = [2 * 4 * nc * 256 * f, 2 * 2 * 4 * nc * 128 * 64 * f, 2 * 4 * 128 * 64 * f]
+    partials = [2 * 2 * 512 * 4 * 64 * f, 2 * 2 * 512 * 4 * 128 * f]
+    assert sum(states) + 3 * 2 * 512 * 4 * f <= need < sum(states) + sum(partials)
+    s32 = _shape(dtype="f32")  # CUDA cores: the per-head partials too
+    assert ssd.backward_workspace_size(s32) >= sum(states) + sum(partials)
     # the per-state variant is served up to N = 128
     assert ssd.backward_workspace_size(_shape(a_per_state=True)) > need
     assert ssd.backward_workspace_size(_shape(a_per_state=True, N=256)) == 0
