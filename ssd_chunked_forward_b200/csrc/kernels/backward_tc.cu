@@ -11,6 +11,11 @@
 // operator"; the roles of U, V, Z and M are in backward.cu).  Every factor is
 // <= 1 for a <= 0.
 //
+// y - Dx and dx - D dy run here (per head; their rows reduced in the
+// epilogue, see below); dC and dB run in chunk_form_group_tc_kernel further
+// down, summed over each group's heads.  The template also serves the other
+// operand shapes (K = 64, MC = 128, state read transposed, rows stored).
+//
 // One CTA per (chunk, 128-row tile, batch x head), two CTAs per SM (about
 // 100 KB of shared memory and 256 TMEM columns each), so one CTA's copies
 // overlap the other's arithmetic.  TMA brings the U rows and the V rows of
@@ -75,8 +80,7 @@ struct FormSmem {
     static constexpr uint32_t MISC = BAR + 64;
     static constexpr size_t bytes = 1024 + MISC + 16;
 };
-static_assert(FormSmem<128, 64>::bytes <= 113 * 1024 && FormSmem<64, 128>::bytes <= 113 * 1024,
-              "two CTAs per SM");
+static_assert(FormSmem<128, 64>::bytes <= 113 * 1024, "two CTAs per SM");
 
 // EPI 0 stores the rows (fp32); EPI 1 (y - Dx) keeps only dy . row per row;
 // EPI 2 (dx - D dy) writes dx = row + D dy (bf16) and keeps x . row and x . dy
@@ -339,6 +343,17 @@ __global__ void __launch_bounds__(kFormThreads, 2)
         tc::tc_fence_before();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&bars->p_full);
+        // the row epilogues' dy (and x) rows, read while the products run
+        const size_t ro = (((size_t)b * p.T + tk + i) * p.H + h) * MC + half * (MC / 2);
+        uint4 dyr[EPI ? 4 : 1], xr[EPI == 2 ? 4 : 1];
+        if (EPI != 0 && i < qv && SSD_INB((long long)ro + MC / 2 - 1, (long long)gridDim.y * p.T * MC)) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) dyr[u] = __ldg(reinterpret_cast<const uint4*>(p.dyg + ro) + u);
+            if (EPI == 2) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) xr[u] = __ldg(reinterpret_cast<const uint4*>(p.xg + ro) + u);
+            }
+        }
         const bool ok2 = tc::mbar_wait(&bars->o_full, 0, nullptr, kBudget);
         if (!__all_sync(0xffffffffu, ok2) && lane == 0) timed_out();
         ok = ok && __all_sync(0xffffffffu, ok2);
@@ -366,7 +381,6 @@ __global__ void __launch_bounds__(kFormThreads, 2)
             // quadrant through shared memory, and (EPI 2) dx
             static_assert(EPI == 0 || MC == 64, "row epilogues serve the P = 64 forms");
             float pa = 0.f, pb = 0.f;  // EPI 1: dy . row; EPI 2: x . row, x . dy
-            const size_t ro = (((size_t)b * p.T + tk + i) * p.H + h) * MC + half * 32;
             const bool live = ok && i < qv && SSD_INB((long long)ro + 31, (long long)gridDim.y * p.T * MC);
             if (ok) tc::tc_fence_after();
 #pragma unroll
@@ -378,10 +392,9 @@ __global__ void __launch_bounds__(kFormThreads, 2)
                 }
                 if (live) {
                     float dyv[16], xv[16];
-                    const uint4* dyp = reinterpret_cast<const uint4*>(p.dyg + ro + 16 * q16);
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
-                        const uint4 w = __ldg(dyp + u);
+                        const uint4 w = dyr[2 * q16 + u];
                         const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
@@ -394,10 +407,9 @@ __global__ void __launch_bounds__(kFormThreads, 2)
 #pragma unroll
                         for (int e = 0; e < 16; ++e) pa = fmaf(dyv[e], v[e], pa);
                     } else {
-                        const uint4* xp = reinterpret_cast<const uint4*>(p.xg + ro + 16 * q16);
 #pragma unroll
                         for (int u = 0; u < 2; ++u) {
-                            const uint4 w = __ldg(xp + u);
+                            const uint4 w = xr[2 * q16 + u];
                             const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
@@ -450,13 +462,17 @@ __global__ void __launch_bounds__(kFormThreads, 2)
 // ---------------------------------------------------------------------------
 // dC and dB summed over the heads of a B/C group in one CTA (K = P = 64,
 // MC = N = 128): per (chunk, 128-row tile, batch x group) the CTA walks the
-// group's heads, each head's S = U_h V_h^T, scores and U~_h M_h as above,
-// accumulating out = sum_h (P~_h Z + U~_h M_h) in TMEM (Z = B or C is the
-// group's own, loaded once), and stores the group sum as bf16 -- the per-head
-// fp32 rows and the separate sum over heads are never written.  The next
-// head's U and V rows load (TMA, two stages) under the current head's
-// products.  TMEM: S at columns 0-255 (scores packed in place), out at
-// 256-383.
+// group's heads, accumulating out = sum_h (P~_h Z + U~_h M_h) in TMEM (Z = B
+// or C is the group's own, loaded once), and stores the group sum as bf16 --
+// the per-head fp32 rows and the separate sum over heads are never written.
+// The work runs in steps, one per (head, V tile): S = U_h V_tile^T into one
+// of two 128-column TMEM buffers, the scores packed in place by the math
+// warps, then out += P~ Z_tile (and, at a head's last tile, + U~_h M_h).  The
+// issuing thread runs one step ahead -- S of step s goes out before the
+// output product of step s - 1 -- so the tensor core works on the next
+// scores while the math warps convert the current ones, and the next head's
+// U and V rows load (TMA, two stages) under the current head's steps.
+// TMEM: S buffers at columns 0 and 128, out at 256-383.
 struct GroupFormParams {
     const float* cum;  // [B*H][nc][Q]
     const float* Mst;  // [B*H][nc][N*P], read as P x N
@@ -466,17 +482,17 @@ struct GroupFormParams {
 };
 
 struct __align__(8) GroupFormBars {
-    uint64_t full[2], z_full, s_full, p_full, o_done;
+    uint64_t full[2], z_full, s_full[2], p_full[2], o_done[2];
 };
 
 struct GroupFormSmem {
     static constexpr uint32_t U = 0;                   // 2 stages x 1 box (K = 64)
     static constexpr uint32_t V = U + 2 * kBox;        // 2 stages x 2 tiles
     static constexpr uint32_t Z = V + 4 * kBox;        // 2 tiles x 2 boxes (MC = 128)
-    static constexpr uint32_t M = Z + 4 * kBox;        // 2 boxes of 64 rows
-    static constexpr uint32_t CUM = M + 2 * 64 * 128;  // 2 stages x [256] fp32
+    static constexpr uint32_t M = Z + 4 * kBox;        // 2 stages x 2 boxes of 64 rows
+    static constexpr uint32_t CUM = M + 2 * 2 * 64 * 128;  // 2 stages x [256] fp32
     static constexpr uint32_t BAR = CUM + 2 * 256 * 4;
-    static constexpr uint32_t MISC = BAR + 64;
+    static constexpr uint32_t MISC = BAR + 128;
     static constexpr size_t bytes = 1024 + MISC + 16;
 };
 static_assert(GroupFormSmem::bytes <= 227 * 1024, "shared memory");
@@ -507,23 +523,26 @@ __global__ void __launch_bounds__(kFormThreads, 1)
     const int qv = min(p.Q, p.T - tk);
     const int jbase = ANTI ? i0 : 0;
     const int nt = ANTI ? (p.Q - i0) / kRowsT : i0 / kRowsT + 1;
+    const int nsteps = HG * nt;
     if (i0 >= qv) return;  // a tile wholly past T: nothing to write
     {
         // the group's last head bounds the decay and state reads (the whole
         // block leaves before any barrier if not)
         const long long last = ((long long)b * p.H + hfirst + HG - 1) * p.nc + k;
+        (void)last;  // read by the checks of the debug build only
         if (!SSD_INB((last + 1) * p.Q - 1, (long long)(gridDim.y / p.G) * p.H * p.nc * p.Q) ||
             !SSD_INB((last + 1) * p.NP - 1, (long long)(gridDim.y / p.G) * p.H * p.nc * p.NP))
             return;
     }
 
     if (threadIdx.x == 0) {
-        tc::mbar_init(&bars->full[0], 1);
-        tc::mbar_init(&bars->full[1], 1);
+        for (int q = 0; q < 2; ++q) {
+            tc::mbar_init(&bars->full[q], 1);
+            tc::mbar_init(&bars->s_full[q], 1);
+            tc::mbar_init(&bars->p_full[q], 8);
+            tc::mbar_init(&bars->o_done[q], 1);
+        }
         tc::mbar_init(&bars->z_full, 1);
-        tc::mbar_init(&bars->s_full, 1);
-        tc::mbar_init(&bars->p_full, 8);
-        tc::mbar_init(&bars->o_done, 1);
         tc::fence_mbar_init();
     }
     if (warp == 0) {
@@ -550,56 +569,70 @@ __global__ void __launch_bounds__(kFormThreads, 1)
                 for (int v = 0; v < nt; ++v)
                     tc::tma_load_4d(sV + (2 * st + v) * kBox, &tm_v, &bars->full[st], 0, h, tk + jbase + v * kRowsT, b);
             };
+            constexpr uint32_t id_s = tc::idesc_bf16_f32(128, 128, 0, 0);
+            constexpr uint32_t id_o = tc::idesc_bf16_f32(128, 64, 0, 1);
+            // out += P~ Z_tile (+ U~ M at a head's last tile) for step s
+            auto output = [&](int s) -> bool {
+                const int hh = s / nt, v = s - hh * nt, bf = s & 1;
+                if (!tc::mbar_wait(&bars->p_full[bf], (s >> 1) & 1, nullptr, kBudget)) return false;
+                tc::tc_fence_after();
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const uint64_t dZ = tc::smem_desc_sw128(tc::smem_u32(sZ + (2 * v + q) * kBox), kBox, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        tc::mma_ts(tmem + COL_OUT + 64 * q, tmem + 128 * bf + kk * 8, tc::desc_adv(dZ, kk * 2048), id_o,
+                                   (s > 0 || kk > 0) ? 1u : 0u);
+                }
+                if (v == nt - 1) {
+                    const int st = hh & 1;
+                    const uint64_t dU = tc::smem_desc_sw128(tc::smem_u32(sU + st * kBox), 16, 1024);
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const uint64_t dM =
+                            tc::smem_desc_sw128(tc::smem_u32(sM + st * (2 * K * 128) + q * (K * 128)), K * 128, 1024);
+#pragma unroll
+                        for (int kk = 0; kk < K / 16; ++kk)
+                            tc::mma_ss(tmem + COL_OUT + 64 * q, tc::desc_adv(dU, kk * 32), tc::desc_adv(dM, kk * 2048),
+                                       id_o, 1u);
+                    }
+                }
+                tc::mma_commit(&bars->o_done[bf]);
+                return true;
+            };
             tc::mbar_arrive_expect_tx(&bars->z_full, (uint32_t)(2 * kBox * nt));
             for (int v = 0; v < nt; ++v)
                 for (int q = 0; q < 2; ++q)
                     tc::tma_load_4d(sZ + (2 * v + q) * kBox, &tm_z, &bars->z_full, 64 * q, g, tk + jbase + v * kRowsT, b);
             load_head(0);
             bool ok = tc::mbar_wait(&bars->z_full, 0, nullptr, kBudget);
-            constexpr uint32_t id_s = tc::idesc_bf16_f32(128, 128, 0, 0);
-            constexpr uint32_t id_o = tc::idesc_bf16_f32(128, 64, 0, 1);
-            for (int hh = 0; hh < HG; ++hh) {
-                const int st = hh & 1;
-                // the previous head's products are done: its S columns, its
-                // U stage and sM may be reused
-                if (hh > 0) ok = ok && tc::mbar_wait(&bars->o_done, (hh - 1) & 1, nullptr, kBudget);
-                if (!ok) break;
-                if (hh + 1 < HG) load_head(hh + 1);
-                ok = tc::mbar_wait(&bars->full[st], (hh >> 1) & 1, nullptr, kBudget);
+            for (int s = 0; ok && s < nsteps; ++s) {
+                const int hh = s / nt, v = s - hh * nt, bf = s & 1, st = hh & 1;
+                // this S buffer was read by the output product of step s - 2
+                if (s >= 2) ok = tc::mbar_wait(&bars->o_done[bf], ((s >> 1) - 1) & 1, nullptr, kBudget);
+                if (v == 0 && ok) ok = tc::mbar_wait(&bars->full[st], (hh >> 1) & 1, nullptr, kBudget);
                 if (!ok) break;
                 tc::tc_fence_after();
                 const uint64_t dU = tc::smem_desc_sw128(tc::smem_u32(sU + st * kBox), 16, 1024);
-                for (int v = 0; v < nt; ++v) {
-                    const uint64_t dV = tc::smem_desc_sw128(tc::smem_u32(sV + (2 * st + v) * kBox), 16, 1024);
+                const uint64_t dV = tc::smem_desc_sw128(tc::smem_u32(sV + (2 * st + v) * kBox), 16, 1024);
 #pragma unroll
-                    for (int kk = 0; kk < K / 16; ++kk)
-                        tc::mma_ss(tmem + 128 * v, tc::desc_adv(dU, kk * 32), tc::desc_adv(dV, kk * 32), id_s, kk > 0);
+                for (int kk = 0; kk < K / 16; ++kk)
+                    tc::mma_ss(tmem + 128 * bf, tc::desc_adv(dU, kk * 32), tc::desc_adv(dV, kk * 32), id_s, kk > 0);
+                tc::mma_commit(&bars->s_full[bf]);
+                if (s > 0 && !(ok = output(s - 1))) break;
+                // a head's first step: the previous head's products are all
+                // issued (its last output just went out); once they are done
+                // its U and V stage takes the next head's rows
+                if (v == 0 && hh + 1 < HG) {
+                    if (s > 0) ok = tc::mbar_wait(&bars->o_done[(s - 1) & 1], ((s - 1) >> 1) & 1, nullptr, kBudget);
+                    if (!ok) break;
+                    load_head(hh + 1);
                 }
-                tc::mma_commit(&bars->s_full);
-                ok = tc::mbar_wait(&bars->p_full, hh & 1, nullptr, kBudget);
-                if (!ok) break;
-                tc::tc_fence_after();
-                for (int v = 0; v < nt; ++v)
-#pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        const uint64_t dZ = tc::smem_desc_sw128(tc::smem_u32(sZ + (2 * v + q) * kBox), kBox, 1024);
-#pragma unroll
-                        for (int kk = 0; kk < 8; ++kk)
-                            tc::mma_ts(tmem + COL_OUT + 64 * q, tmem + 128 * v + kk * 8, tc::desc_adv(dZ, kk * 2048),
-                                       id_o, (hh > 0 || v > 0 || kk > 0) ? 1u : 0u);
-                    }
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const uint64_t dM = tc::smem_desc_sw128(tc::smem_u32(sM + q * (K * 128)), K * 128, 1024);
-#pragma unroll
-                    for (int kk = 0; kk < K / 16; ++kk)
-                        tc::mma_ss(tmem + COL_OUT + 64 * q, tc::desc_adv(dU, kk * 32), tc::desc_adv(dM, kk * 2048), id_o,
-                                   1u);
-                }
-                tc::mma_commit(&bars->o_done);
             }
+            if (ok) ok = output(nsteps - 1);
             // every product done before the epilogue and the exit
-            if (!tc::mbar_wait(&bars->o_done, (HG - 1) & 1, nullptr, kBudget) || !ok) timed_out();
+            if (!ok || !tc::mbar_wait(&bars->o_done[(nsteps - 1) & 1], ((nsteps - 1) >> 1) & 1, nullptr, kBudget))
+                timed_out();
         }
     } else {
         // ---------------------------------------------------- math warps ----
@@ -635,100 +668,109 @@ __global__ void __launch_bounds__(kFormThreads, 1)
         };
         const int kk4 = (mt % (K / 4)) * 4, m8 = (mt / (K / 4)) * 8;  // this thread's 4 x 8 block of M
         bool ok = true;
-        for (int hh = 0; hh < HG; ++hh) {
-            const int st = hh & 1, h = hfirst + hh;
-            const size_t chain = (size_t)b * p.H + h;
+        float ci = 0.f, cend = 0.f;
+        for (int s = 0; s < nsteps; ++s) {
+            const int hh = s / nt, v = s - hh * nt, bf = s & 1, st = hh & 1;
+            const size_t chain = (size_t)b * p.H + hfirst + hh;
             float* cumh = sCum + st * 256;
-            // the head's in-chunk decays, and its state read ahead ([N][P]: M[p][n])
-            for (int t = mt; t < p.Q; t += 256) cumh[t] = p.cum[(chain * p.nc + k) * p.Q + t];
-            const float* Mk = p.Mst + (chain * p.nc + k) * (size_t)p.NP;
             float4 mv[8];
+            if (v == 0) {
+                // the head's in-chunk decays, and its state read ahead ([N][P]: M[p][n])
+                for (int t = mt; t < p.Q; t += 256) cumh[t] = p.cum[(chain * p.nc + k) * p.Q + t];
+                const float* Mk = p.Mst + (chain * p.nc + k) * (size_t)p.NP;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) mv[e] = *reinterpret_cast<const float4*>(Mk + (size_t)(m8 + e) * K + kk4);
-            math_sync();  // cumh complete
-            const float ci = cumh[i];
-            const float cend = cumh[p.Q - 1];
-            bool okh = ok && tc::mbar_wait(&bars->s_full, hh & 1, nullptr, kBudget);
+                for (int e = 0; e < 8; ++e) mv[e] = *reinterpret_cast<const float4*>(Mk + (size_t)(m8 + e) * K + kk4);
+                math_sync();  // cumh complete
+                ci = cumh[i];
+                cend = cumh[p.Q - 1];
+            }
+            bool okh = ok && tc::mbar_wait(&bars->s_full[bf], (s >> 1) & 1, nullptr, kBudget);
             if (!okh) timed_out();
             okh = !math_or(!okh);
-            // M into sM (the previous head's products are done: S of this head was
-            // issued after them)
-            {
+            if (v == 0) {
+                // M into its stage (the products of two heads back are done:
+                // this step's S went out after them)
+                uint8_t* sMs = sM + st * (2 * K * 128);
                 auto put = [&](int kk, float f0, float f1, float f2, float f3, float f4, float f5, float f6, float f7) {
                     const uint4 w = make_uint4(tc::pack_bf16x2(f0, f1), tc::pack_bf16x2(f2, f3),
                                                tc::pack_bf16x2(f4, f5), tc::pack_bf16x2(f6, f7));
-                    *reinterpret_cast<uint4*>(sM + (m8 >> 6) * (K * 128) + tc::sw128_offset(kk, (m8 & 63) >> 3)) = w;
+                    *reinterpret_cast<uint4*>(sMs + (m8 >> 6) * (K * 128) + tc::sw128_offset(kk, (m8 & 63) >> 3)) = w;
                 };
                 put(kk4, mv[0].x, mv[1].x, mv[2].x, mv[3].x, mv[4].x, mv[5].x, mv[6].x, mv[7].x);
                 put(kk4 + 1, mv[0].y, mv[1].y, mv[2].y, mv[3].y, mv[4].y, mv[5].y, mv[6].y, mv[7].y);
                 put(kk4 + 2, mv[0].z, mv[1].z, mv[2].z, mv[3].z, mv[4].z, mv[5].z, mv[6].z, mv[7].z);
                 put(kk4 + 3, mv[0].w, mv[1].w, mv[2].w, mv[3].w, mv[4].w, mv[5].w, mv[6].w, mv[7].w);
             }
-            const int npc = nt == 2 ? 2 : 1;
             if (okh) {
                 tc::tc_fence_after();
-                const float uf = ANTI ? ex2_approx((cend - ci) * 1.4426950408889634f)
-                                      : ex2_approx(ci * 1.4426950408889634f);
-                const uint32_t u2 = tc::pack_bf16x2(uf, uf);
-                uint8_t* sUs = sU + st * kBox;
+                if (v == nt - 1) {
+                    // U row i times its factor, in place: every S of this head is done
+                    const float uf = ANTI ? ex2_approx((cend - ci) * 1.4426950408889634f)
+                                          : ex2_approx(ci * 1.4426950408889634f);
+                    const uint32_t u2 = tc::pack_bf16x2(uf, uf);
+                    uint8_t* sUs = sU + st * kBox;
 #pragma unroll
-                for (int cc = 0; cc < K / 16; ++cc) {
-                    const int c = half * (K / 16) + cc;
-                    uint4* ptr = reinterpret_cast<uint4*>(sUs + tc::sw128_offset(row, c));
-                    uint4 v = *ptr;
-                    v.x = tc::mul_bf16x2(v.x, u2);
-                    v.y = tc::mul_bf16x2(v.y, u2);
-                    v.z = tc::mul_bf16x2(v.z, u2);
-                    v.w = tc::mul_bf16x2(v.w, u2);
-                    *ptr = v;
+                    for (int cc = 0; cc < K / 16; ++cc) {
+                        const int c = half * (K / 16) + cc;
+                        uint4* ptr = reinterpret_cast<uint4*>(sUs + tc::sw128_offset(row, c));
+                        uint4 w = *ptr;
+                        w.x = tc::mul_bf16x2(w.x, u2);
+                        w.y = tc::mul_bf16x2(w.y, u2);
+                        w.z = tc::mul_bf16x2(w.z, u2);
+                        w.w = tc::mul_bf16x2(w.w, u2);
+                        *ptr = w;
+                    }
                 }
-                for (int u = 0; u < npc; ++u) {
-                    const int tile = nt == 2 ? half : 0;
-                    const int c0 = nt == 2 ? 64 * u : 64 * half;
+                // the tile's scores, packed in place: warp half h takes columns
+                // [64 h, 64 h + 64), read and written 32 at a time; the pair of
+                // warps of a lane quadrant meets once (half 0 after reading all
+                // of its columns, half 1 before its first write, which lands in
+                // half 0's columns)
+                const int c0 = 64 * half;
+                const uint32_t tbase = lane_base + 128 * bf;
 #pragma unroll
-                    for (int r = 0; r < 2; ++r) {
-                        const int cin = c0 + 32 * r;
-                        const uint32_t tbase = lane_base + 128 * tile;
-                        float sv[32];
-                        tc::tmem_ld16(tbase + cin, *reinterpret_cast<float(*)[16]>(sv));
-                        tc::tmem_ld16(tbase + cin + 16, *reinterpret_cast<float(*)[16]>(sv + 16));
-                        tc::tmem_ld_wait();
-                        if (r == (c0 == 0 ? 1 : 0)) pair_sync();
-                        const int j0 = jbase + 128 * tile + cin;
+                for (int r = 0; r < 2; ++r) {
+                    const int cin = c0 + 32 * r;
+                    float sv[32];
+                    tc::tmem_ld16(tbase + cin, *reinterpret_cast<float(*)[16]>(sv));
+                    tc::tmem_ld16(tbase + cin + 16, *reinterpret_cast<float(*)[16]>(sv + 16));
+                    tc::tmem_ld_wait();
+                    if (r == (half == 0 ? 1 : 0)) pair_sync();
+                    const int j0 = jbase + 128 * v + cin;
 #pragma unroll
-                        for (int g8 = 0; g8 < 2; ++g8) {
-                            uint32_t pk[8];
+                    for (int g8 = 0; g8 < 2; ++g8) {
+                        uint32_t pk[8];
 #pragma unroll
-                            for (int e2 = 0; e2 < 8; ++e2) {
-                                float pv[2];
+                        for (int e2 = 0; e2 < 8; ++e2) {
+                            float pv[2];
 #pragma unroll
-                                for (int q = 0; q < 2; ++q) {
-                                    const int e = 16 * g8 + 2 * e2 + q;
-                                    const int j = j0 + e;
-                                    const bool keep = (ANTI ? j >= i : j <= i) && j < qv && i < qv;
-                                    const float ex = ex2_approx(
-                                        keep ? (ANTI ? cumh[j] - ci : ci - cumh[j]) * 1.4426950408889634f : 0.f);
-                                    pv[q] = keep ? sv[e] * ex : 0.f;
-                                }
-                                pk[e2] = tc::pack_bf16x2(pv[0], pv[1]);
+                            for (int q = 0; q < 2; ++q) {
+                                const int e = 16 * g8 + 2 * e2 + q;
+                                const int j = j0 + e;
+                                const bool keep = (ANTI ? j >= i : j <= i) && j < qv && i < qv;
+                                const float ex = ex2_approx(
+                                    keep ? (ANTI ? cumh[j] - ci : ci - cumh[j]) * 1.4426950408889634f : 0.f);
+                                pv[q] = keep ? sv[e] * ex : 0.f;
                             }
-                            tc::tmem_st8(tbase + cin / 2 + 8 * g8, pk);
+                            pk[e2] = tc::pack_bf16x2(pv[0], pv[1]);
                         }
+                        tc::tmem_st8(tbase + cin / 2 + 8 * g8, pk);
                     }
                 }
                 tc::tmem_st_wait();
             } else {
-                for (int u = 0; u < npc; ++u) pair_sync();
+                pair_sync();
             }
             tc::fence_proxy_async_smem();  // U~ and M for the products
             tc::tc_fence_before();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&bars->p_full);
+            if (lane == 0) tc::mbar_arrive(&bars->p_full[bf]);
             ok = okh;
             if (!ok) break;
         }
         // the group sum, as bf16, straight from TMEM
-        const bool okf = __all_sync(0xffffffffu, ok && tc::mbar_wait(&bars->o_done, (HG - 1) & 1, nullptr, kBudget));
+        const bool okf = __all_sync(
+            0xffffffffu, ok && tc::mbar_wait(&bars->o_done[(nsteps - 1) & 1], ((nsteps - 1) >> 1) & 1, nullptr, kBudget));
         if (okf) {
             tc::tc_fence_after();
             const size_t ro = (((size_t)b * p.T + tk + i) * p.G + g) * MC + half * 64;
