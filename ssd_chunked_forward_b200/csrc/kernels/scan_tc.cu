@@ -1,6 +1,7 @@
-// scan_tc.cu -- the chunk output step on the fifth-generation tensor cores,
-// standalone (scan mode) and fused with the chunk-state and inter-chunk steps
-// (fused mode).
+// scan_tc.cu -- the chunk output step (S4) on the fifth-generation tensor
+// cores, for the modular path and the ssd_chunk_scan entry point: the states
+// entering each 128-token block come from the chunk-state and state-pass
+// steps.
 //
 // Unit of work: a block of 128 tokens (the MMA's M) of one batch row b, for a
 // slice of `hpb` heads that share one B/C group.  For the block's tokens
@@ -18,35 +19,17 @@
 // reaches shared memory or HBM.  The in-block mask uses 32-token sub-blocks:
 // below the diagonal sub-block L factorises as exp(cum_t - cum_e) exp(cum_e -
 // cum_s) with e the last token before row t's sub-block (both factors <= 1);
-// on it, exp2 runs per element.
+// on it, exp2 runs per element.  Work items are dealt round-robin over
+// persistent CTAs.
 //
-// Fused mode also forms the block's own state Z = B^T (w o X),
-// w_s = exp(cum_127 - cum_s) (item 3), and the recurrence
-//   h_j = exp(cum_127) h_{j-1} + Z_j                         (item 4)
-// across blocks: each (b, h) chain hands its fp32 state from block j-1 to
-// block j through a two-slot ring in global memory (it stays in L2) and a
-// per-chain counter.  Two dedicated threads move the states with TMA and do
-// the acquire (bounded wait on the counter) and the release, so the compute
-// warps never wait on a fence.  Work items are ordered block-major and
-// scheduled round-robin over persistent CTAs, so the block a CTA waits for
-// belongs to a smaller item index and can always finish.
-//
-// A chunk of 256 tokens is two such blocks: the strictly-lower 128x128 block
-// of its quadratic form goes through the exact factorisation
-// L[t,s] = exp(cum_t - cum_127) exp(cum_127 - cum_s), i.e. through the state
-// at the block boundary ("State Space Duality", "Two algorithms for one
-// operator": off-diagonal blocks are low-rank).
-//
-// Warp roles (640 threads): warp 0 lane 0 streams x, lane 1 loads B and C,
-// lane 2 issues V and Y; warp 1 issues S and Z and owns TMEM; 2-9 group A
-// (decay vectors, weighted x, masked scores P); 10-17 group B (state step,
-// output); 18 state loader; 19 state publisher (fused).  Each group has two
-// warps per TMEM lane quadrant (thread = tile row, the two warps splitting
-// the columns), and the two groups work on different heads at the same time.
-// TMEM (512 columns): scores S 0-127, P 128-191 (bf16 pairs), Z 192-255, then
-// Y and V for two heads (256 + 128 * (head & 1), + 64 for V).  Shared memory
-// holds the incoming and the outgoing fp32 state separately, so the loader
-// fetches the next head's state while the publisher still stores this one.
+// Warp roles (608 threads): warp 0 lane 0 streams x, lane 1 loads B and C,
+// lane 2 issues V and Y; warp 1 issues S and owns TMEM; 2-9 group A (decay
+// vectors, masked scores P); 10-17 group B (incoming state, output); 18 state
+// loader.  Each group has two warps per TMEM lane quadrant (thread = tile row,
+// the two warps splitting the columns), and the two groups work on different
+// heads at the same time.  TMEM (512 columns): scores S 0-127, P 128-191
+// (bf16 pairs), then Y and V for two heads (256 + 128 * (head & 1), + 64 for
+// V).
 #include <stdlib.h>
 
 #include "../common.cuh"
@@ -63,44 +46,36 @@ constexpr int kN = 128;
 constexpr int kP = 64;
 constexpr int kStages = 2;
 constexpr int kHpbMax = 8;
-constexpr int kThreads = 640;
+constexpr int kThreads = 608;
 constexpr uint32_t kTile = kBlk * 128;  // 128 rows x 128 bytes
 constexpr uint32_t kStateBytes = kN * kP * 4;
 
-enum { kScan = 0, kFused = 1 };
 
 struct __align__(8) Bars {
     uint64_t bc_full, bc_empty, s_full, s_empty;
     uint64_t x_full[kStages], x_empty[kStages];
-    uint64_t xw_full, xw_empty, p_full, p_empty, h_full, h_empty;
-    uint64_t hin_full, hin_free, hout_full, hout_free;
+    uint64_t p_full, p_empty, h_full, h_empty;
+    uint64_t hin_full, hin_free;
     uint64_t cum_full[2], cum_free[2];
-    uint64_t y_full[2], v_full[2], yv_empty[2], z_full, z_empty;
+    uint64_t y_full[2], v_full[2], yv_empty[2];
     uint64_t done_y;
     uint64_t done;
 };
 
 struct ScanParams {
-    const float* a;    // fused: log-decays [B,T,H]
-    const float* cum;  // scan: in-block cumsum [B,H,nblk,128]
+    const float* cum;  // in-block cumsum [B,H,nblk,128]
     const float* D;    // [H] or null
-    unsigned* flags;   // fused: [B*H] blocks published per chain
-    float* fin;        // fused: final state [B,H,N,P] or null
     int* status;       // device status word or null
     int T, H, G, nblk, hpb, nslices, n_items;
-    int test_stall;
-    int has_init;      // fused: chains start from tm_init's states, not zero
 };
 
 // smem layout (offsets from the 1024-aligned base)
 constexpr uint32_t OFF_B = 0;
 constexpr uint32_t OFF_C = OFF_B + 2 * kTile;
 constexpr uint32_t OFF_X = OFF_C + 2 * kTile;
-constexpr uint32_t OFF_XW = OFF_X + kStages * kTile;
-constexpr uint32_t OFF_H = OFF_XW + kTile;         // bf16 Hin, MN-major operand
+constexpr uint32_t OFF_H = OFF_X + kStages * kTile;  // bf16 Hin, MN-major operand
 constexpr uint32_t OFF_HIN = OFF_H + kTile;        // fp32 incoming state, two swizzled 128x32 boxes
-constexpr uint32_t OFF_HOUT = OFF_HIN + 2 * kTile; // fp32 outgoing state, same layout
-constexpr uint32_t OFF_Y = OFF_HOUT + 2 * kTile;   // bf16 y staging for the TMA store
+constexpr uint32_t OFF_Y = OFF_HIN + 2 * kTile;    // bf16 y staging for the TMA store
 constexpr uint32_t OFF_CUM = OFF_Y + kTile;
 constexpr uint32_t OFF_VEC = OFF_CUM + 2 * kHpbMax * kBlk * 4;
 constexpr uint32_t OFF_DV = OFF_VEC + 5 * kBlk * 4;  // [2][kHpbMax] D of the item's heads
@@ -112,18 +87,8 @@ static_assert(kSmemBytes <= 232448, "shared memory above the 227 KB per-block li
 // TMEM columns
 constexpr uint32_t COL_S = 0;    // scores, 128 fp32 columns
 constexpr uint32_t COL_P = 128;  // masked scores as the bf16 A operand, 64 columns
-constexpr uint32_t COL_Z = 192;  // block state, 64 columns
 __device__ __forceinline__ uint32_t col_y(int buf) { return 256 + 128 * buf; }
 __device__ __forceinline__ uint32_t col_v(int buf) { return 320 + 128 * buf; }
-
-__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
-    unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_release_u32(unsigned* p, unsigned v) {
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
 
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -150,26 +115,21 @@ __device__ __forceinline__ uint32_t state_off(int row, int half, int q) {
     return half * kTile + row * 128 + ((q ^ (row & 7)) << 4);
 }
 
-template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
                    const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y,
-                   const __grid_constant__ CUtensorMap tm_st, const __grid_constant__ CUtensorMap tm_init,
-                   const ScanParams p, int B) {
+                   const __grid_constant__ CUtensorMap tm_st, const ScanParams p, int B) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
     uint8_t* sB = sm + OFF_B;
     uint8_t* sC = sm + OFF_C;
     uint8_t* sX = sm + OFF_X;
-    uint8_t* sXw = sm + OFF_XW;
     uint8_t* sH = sm + OFF_H;
     uint8_t* sHin = sm + OFF_HIN;
-    uint8_t* sHout = sm + OFF_HOUT;
     uint8_t* sY = sm + OFF_Y;
     float* sCum = reinterpret_cast<float*>(sm + OFF_CUM);  // [2][kHpbMax][128]
-    float* sW = reinterpret_cast<float*>(sm + OFF_VEC);    // [128]
-    float* sColf = sW + kBlk;                              // [3][128]
+    float* sColf = reinterpret_cast<float*>(sm + OFF_VEC) + kBlk;  // [3][128]
     float* sC2 = sColf + 3 * kBlk;                         // [128] cum * log2(e)
     float* sDv = reinterpret_cast<float*>(sm + OFF_DV);    // [2][kHpbMax]
     Bars* bars = reinterpret_cast<Bars*>(sm + OFF_BAR);
@@ -186,21 +146,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mbar_init(&bars->s_empty, 8);
         for (int s = 0; s < kStages; ++s) {
             tc::mbar_init(&bars->x_full[s], 1);
-            // Y MMA commit (+ the 8 group-A warps that weight x, fused)
-            tc::mbar_init(&bars->x_empty[s], MODE == kFused ? 9 : 1);
+            // the Y MMA that read the stage
+            tc::mbar_init(&bars->x_empty[s], 1);
         }
-        tc::mbar_init(&bars->xw_full, 8);
-        tc::mbar_init(&bars->xw_empty, 1);
         tc::mbar_init(&bars->p_full, 8);
         tc::mbar_init(&bars->p_empty, 1);
         tc::mbar_init(&bars->h_full, 8);
         tc::mbar_init(&bars->h_empty, 1);
         tc::mbar_init(&bars->hin_full, 1);
         tc::mbar_init(&bars->hin_free, 8);   // group B read the incoming state
-        tc::mbar_init(&bars->hout_full, 8);  // group B wrote the outgoing state
-        tc::mbar_init(&bars->hout_free, 1);  // the publisher's store read it
-        tc::mbar_init(&bars->z_full, 1);
-        tc::mbar_init(&bars->z_empty, 8);
         for (int s = 0; s < 2; ++s) {
             tc::mbar_init(&bars->cum_full[s], 8);
             tc::mbar_init(&bars->cum_free[s], 8);
@@ -335,19 +289,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::mbar_wait(&bars->done_y, 0, nullptr, 200000000ull);
         }
     } else if (warp == 1) {
-        // ========================================= MMA issuer: S and Z ====
+        // ============================================= MMA issuer: S ====
         // (V and Y are issued by warp 0, lane 2)
         if (lane == 0) {
             constexpr uint32_t id_s = tc::idesc_bf16_f32(128, 128, 0, 0);
-            constexpr uint32_t id_z = tc::idesc_bf16_f32(128, kP, 1, 1);
             // operand descriptors at their tile bases (K-major: 16-element K
-            // steps inside a 64-element block, blocks kTile apart; MN-major:
-            // 16-row K steps of 2048 bytes)
+            // steps inside a 64-element block, blocks kTile apart)
             const uint64_t dC = tc::smem_desc_sw128(tc::smem_u32(sC), 16, 1024);
             const uint64_t dBk = tc::smem_desc_sw128(tc::smem_u32(sB), 16, 1024);
-            const uint64_t dBm = tc::smem_desc_sw128(tc::smem_u32(sB), kTile, 1024);
-            const uint64_t dXw = tc::smem_desc_sw128(tc::smem_u32(sXw), kTile, 1024);
-            uint32_t hc = 0, itc = 0;
+            uint32_t itc = 0;
             bool ok = true;
             for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x, ++itc) {
                 ok = tc::mbar_wait(&bars->bc_full, itc & 1, abort_v) &&
@@ -361,25 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc::mma_ss(tmem + COL_S, tc::desc_adv(dC, off), tc::desc_adv(dBk, off), id_s, kk > 0);
                 }
                 tc::mma_commit(&bars->s_full);
-                for (int i = 0; i < p.hpb; ++i, ++hc) {
-                    if (MODE == kFused) {
-                        // block state Z = B^T (w o X): M = n (MN-major B tile), N = p, K = s.
-                        // Its columns are free once group B's state step of the previous
-                        // head read them.
-                        ok = (hc < 1 || tc::mbar_wait(&bars->z_empty, (hc - 1) & 1, abort_v)) &&
-                             tc::mbar_wait(&bars->xw_full, hc & 1, abort_v);
-                        if (!ok) break;
-                        tc::tc_fence_after();
-#pragma unroll
-                        for (int kk = 0; kk < 8; ++kk)
-                            tc::mma_ss(tmem + COL_Z, tc::desc_adv(dBm, kk * 2048), tc::desc_adv(dXw, kk * 2048),
-                                       id_z, kk > 0);
-                        tc::mma_commit(&bars->z_full);
-                        tc::mma_commit(&bars->xw_empty);
-                    }
-                }
-                if (!ok) break;
-                tc::mma_commit(&bars->bc_empty);  // this item's S and Z products read B and C
+                tc::mma_commit(&bars->bc_empty);  // this item's S product read B and C
             }
             if (!ok) fail();
             // every MMA issued must be complete before TMEM is released
@@ -397,79 +329,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int i = 0; i < p.hpb; ++i, ++hc) {
                     const int chain = w.b * p.H + w.h0 + i;
                     if (hc > 0 && !tc::mbar_wait(&bars->hin_free, (hc - 1) & 1, abort_v)) { ok = false; break; }
-                    if (MODE == kFused) {
-                        if (w.j == 0) {
-                            if (p.has_init) {  // the given initial state of the chain
-                                tc::mbar_arrive_expect_tx(&bars->hin_full, kStateBytes);
-                                tc::tma_load_2d(sHin, &tm_init, &bars->hin_full, 0, chain * kN);
-                                tc::tma_load_2d(sHin + kTile, &tm_init, &bars->hin_full, 32, chain * kN);
-                            } else {
-                                tc::mbar_arrive(&bars->hin_full);  // zero state: nothing to load
-                            }
-                            continue;
-                        }
-                        // bounded wait for the previous block of this chain
-                        // (exponential back-off keeps this thread off the issue slots
-                        // of the compute warps that share its scheduler)
-                        const unsigned* f = p.flags + chain;
-                        const uint64_t t0 = tc::globaltimer_ns();
-                        uint32_t nap = 32;
-                        for (uint32_t spin = 0; ld_acquire_u32(f) < (unsigned)w.j; ++spin) {
-                            if ((spin & 7) == 7) {
-                                if (*abort_v || (p.status && *(volatile int*)p.status) ||
-                                    tc::globaltimer_ns() - t0 > 2000000000ull) {
-                                    ok = false;
-                                    break;
-                                }
-                            }
-                            __nanosleep(nap);
-                            if (nap < 256) nap <<= 1;
-                        }
-                        if (!ok) break;
-                        tc::fence_proxy_async_global();  // the acquire orders the TMA read
-                        const int r0 = (chain * 2 + ((w.j - 1) & 1)) * kN;
-                        tc::mbar_arrive_expect_tx(&bars->hin_full, kStateBytes);
-                        tc::tma_load_2d(sHin, &tm_st, &bars->hin_full, 0, r0);
-                        tc::tma_load_2d(sHin + kTile, &tm_st, &bars->hin_full, 32, r0);
-                    } else {
-                        const int r0 = (chain * p.nblk + w.j) * kN;
-                        tc::mbar_arrive_expect_tx(&bars->hin_full, kStateBytes);
-                        tc::tma_load_2d(sHin, &tm_st, &bars->hin_full, 0, r0);
-                        tc::tma_load_2d(sHin + kTile, &tm_st, &bars->hin_full, 32, r0);
-                    }
+                    const int r0 = (chain * p.nblk + w.j) * kN;
+                    tc::mbar_arrive_expect_tx(&bars->hin_full, kStateBytes);
+                    tc::tma_load_2d(sHin, &tm_st, &bars->hin_full, 0, r0);
+                    tc::tma_load_2d(sHin + kTile, &tm_st, &bars->hin_full, 32, r0);
                 }
             }
             if (!ok) fail();
             if (hc > 0) tc::mbar_wait(&bars->hin_full, (hc - 1) & 1, nullptr, 200000000ull);
-        }
-    } else if (warp == 19) {
-        // ============================================== state publisher ====
-        if (MODE == kFused && lane == 0) {
-            uint32_t hc = 0;
-            bool ok = true;
-            for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x) {
-                const Item w = decode_item(it, p, B);
-                for (int i = 0; i < p.hpb; ++i, ++hc) {
-                    const int chain = w.b * p.H + w.h0 + i;
-                    if (!tc::mbar_wait(&bars->hout_full, hc & 1, abort_v)) { ok = false; break; }
-                    const bool publish = !(p.test_stall && chain == 0 && w.j == 0);
-                    if (publish) {
-                        const int r0 = (chain * 2 + (w.j & 1)) * kN;
-                        tc::tma_store_2d(&tm_st, sHout, 0, r0);
-                        tc::tma_store_2d(&tm_st, sHout + kTile, 32, r0);
-                        tc::bulk_commit();
-                        tc::bulk_wait_read<0>();
-                    }
-                    tc::mbar_arrive(&bars->hout_free);
-                    if (publish) {
-                        tc::bulk_wait<0>();
-                        tc::fence_proxy_async_global();
-                        st_release_u32(p.flags + chain, (unsigned)(w.j + 1));
-                    }
-                }
-            }
-            if (!ok) fail();
-            tc::bulk_wait<0>();
         }
     } else {
         // ===================================== compute: two groups of 8 warps ====
@@ -504,29 +371,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         if (groupA) {
             // ---------------------------------------------------- group A ----
-            uint32_t hc = 0, xc = 0, itc = 0;
+            uint32_t hc = 0, itc = 0;
             float anext[kHpbMax];
             float dnext = 0.f;
             auto load_decays = [&](int it) {
                 if (cg != 0 || it >= p.n_items) return;
                 const Item w = decode_item(it, p, B);
                 dnext = (p.D && gt < p.hpb) ? __ldg(p.D + w.h0 + gt) : 0.f;
-                if (MODE == kFused) {
-                    // tokens past T (the partial last block) decay by 1: a = 0
-                    const int t = w.j * kBlk + gt;
-                    const float* arow = p.a + ((size_t)w.b * p.T + t) * p.H + w.h0;
 #pragma unroll
-                    for (int i = 0; i < kHpbMax; ++i)
-                        anext[i] = (i < p.hpb && t < p.T &&
-                                    SSD_INB(((long long)w.b * p.T + t) * p.H + w.h0 + i, (long long)B * p.T * p.H))
-                                       ? __ldg(arow + i)
-                                       : 0.f;
-                } else {
-#pragma unroll
-                    for (int i = 0; i < kHpbMax; ++i) {
-                        const long long ci = (((long long)w.b * p.H + w.h0 + i) * p.nblk + w.j) * kBlk + gt;
-                        anext[i] = (i < p.hpb && SSD_INB(ci, (long long)B * p.H * p.nblk * kBlk)) ? __ldg(p.cum + ci) : 0.f;
-                    }
+                for (int i = 0; i < kHpbMax; ++i) {
+                    const long long ci = (((long long)w.b * p.H + w.h0 + i) * p.nblk + w.j) * kBlk + gt;
+                    anext[i] = (i < p.hpb && SSD_INB(ci, (long long)B * p.H * p.nblk * kBlk)) ? __ldg(p.cum + ci) : 0.f;
                 }
             };
             load_decays(blockIdx.x);
@@ -545,22 +400,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 load_decays(it + gridDim.x);
                 group_sync();
-                if (MODE == kFused) {
-                    // group warp gw scans head gw (128 values, 4 per lane)
-                    for (int hh = gt >> 5; hh < p.hpb; hh += 8) {
-                        float* c = cumbuf + hh * kBlk + lane * 4;
-                        float v0 = c[0], v1 = v0 + c[1], v2 = v1 + c[2], v3 = v2 + c[3];
-                        const float excl = warp_inclusive_scan(v3) - v3;
-                        c[0] = v0 + excl; c[1] = v1 + excl; c[2] = v2 + excl; c[3] = v3 + excl;
-                    }
-                    group_sync();
-                }
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&bars->cum_full[itc & 1]);
 
                 bool ok = true;
-                for (int i = 0; i < p.hpb; ++i, ++hc, ++xc) {
-                    const uint32_t st = xc % kStages;
+                for (int i = 0; i < p.hpb; ++i, ++hc) {
                     const float* cum = cumbuf + i * kBlk;
                     // ---- T1: decay vectors of this head (thread = token row).  The
                     // previous head's mask build reads them, so wait for the group.
@@ -568,35 +412,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (cg == 0) {
                         const float c = cum[gt] * kLog2e;
                         sC2[gt] = c;
-                        sW[gt] = ex2_approx(cum[kBlk - 1] * kLog2e - c);
                         sColf[gt] = gt < 32 ? ex2_approx(cum[31] * kLog2e - c) : 0.f;
                         sColf[kBlk + gt] = gt < 64 ? ex2_approx(cum[63] * kLog2e - c) : 0.f;
                         sColf[2 * kBlk + gt] = gt < 96 ? ex2_approx(cum[95] * kLog2e - c) : 0.f;
-                    }
-                    // ---- T2: weighted copy of x for the block state (fused)
-                    if (MODE == kFused) {
-                        ok = tc::mbar_wait(&bars->x_full[st], (xc / kStages) & 1, abort_v) &&
-                             (hc == 0 || tc::mbar_wait(&bars->xw_empty, (hc - 1) & 1, abort_v));
-                        if (!sync_ok(ok)) { alive = false; break; }
-                        const uint8_t* xs = sX + st * kTile;
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const int c = gt + 256 * q;
-                            const float wgt = sW[c >> 3];
-                            const uint32_t w2 = tc::pack_bf16x2(wgt, wgt);
-                            uint4 v = *reinterpret_cast<const uint4*>(xs + c * 16);
-                            v.x = tc::mul_bf16x2(v.x, w2);
-                            v.y = tc::mul_bf16x2(v.y, w2);
-                            v.z = tc::mul_bf16x2(v.z, w2);
-                            v.w = tc::mul_bf16x2(v.w, w2);
-                            *reinterpret_cast<uint4*>(sXw + c * 16) = v;
-                        }
-                        tc::fence_proxy_async_smem();
-                        __syncwarp();
-                        if (lane == 0) {
-                            tc::mbar_arrive(&bars->xw_full);
-                            tc::mbar_arrive(&bars->x_empty[st]);
-                        }
                     }
                     // ---- T3: P = S o L + D I -> bf16, into TMEM as the A operand of Y = P X
                     ok = (i > 0 || tc::mbar_wait(&bars->s_full, itc & 1, abort_v)) &&
@@ -678,7 +496,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int it = blockIdx.x; alive && it < p.n_items; it += gridDim.x, ++itc) {
                 const Item w = decode_item(it, p, B);
                 const int t0 = w.j * kBlk;
-                const bool last_blk = (w.j == p.nblk - 1);
                 const float* cumbuf = sCum + (itc & 1) * (kHpbMax * kBlk);
                 if (!sync_ok(tc::mbar_wait(&bars->cum_full[itc & 1], (itc >> 1) & 1, abort_v))) break;
 
@@ -688,56 +505,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 bool ok = true;
                 for (int i = 0; i <= p.hpb; ++i) {
                     if (i < p.hpb) {
-                        // ---- T4: incoming state (and, fused, the block's own state out)
-                        const int h = w.h0 + i;
-                        const int chain = w.b * p.H + h;
+                        // ---- T4: incoming state
                         const float* cum = cumbuf + i * kBlk;
-                        ok = (MODE == kScan || tc::mbar_wait(&bars->z_full, hc & 1, abort_v)) &&
-                             (MODE == kScan || hc == 0 || tc::mbar_wait(&bars->hout_free, (hc - 1) & 1, abort_v)) &&
-                             (hc == 0 || tc::mbar_wait(&bars->h_empty, (hc - 1) & 1, abort_v)) &&
+                        ok = (hc == 0 || tc::mbar_wait(&bars->h_empty, (hc - 1) & 1, abort_v)) &&
                              tc::mbar_wait(&bars->hin_full, hc & 1, abort_v);
                         if (!sync_ok(ok)) { alive = false; break; }
                         tc::tc_fence_after();
-                        const bool zero_in = MODE == kFused && w.j == 0 && !p.has_init;
                         const float eL = ex2_approx(cum[kBlk - 1] * kLog2e);
                         // this warp's 32 columns of the state, 16 at a time
 #pragma unroll 1
                         for (int c = 0; c < 2; ++c) {
                             float hin[16];
-                            if (zero_in) {
 #pragma unroll
-                                for (int e = 0; e < 16; ++e) hin[e] = 0.f;
-                            } else {
-#pragma unroll
-                                for (int q = 0; q < 4; ++q) {
-                                    const float4 v = *reinterpret_cast<const float4*>(sHin + state_off(row, cg, 4 * c + q));
-                                    hin[4 * q] = v.x; hin[4 * q + 1] = v.y; hin[4 * q + 2] = v.z; hin[4 * q + 3] = v.w;
-                                }
-                            }
-                            if (MODE == kFused) {
-                                float zv[16];
-                                tc::tmem_ld16(lane_base + COL_Z + 32 * cg + 16 * c, zv);
-                                tc::tmem_ld_wait();
-                                {
-                                    const float2 e2 = make_float2(eL, eL);
-                                    float2* z2 = reinterpret_cast<float2*>(zv);
-                                    const float2* h2 = reinterpret_cast<const float2*>(hin);
-#pragma unroll
-                                    for (int e = 0; e < 8; ++e) z2[e] = tc::fma2(e2, h2[e], z2[e]);  // h_j
-                                }
-#pragma unroll
-                                for (int q = 0; q < 4; ++q)
-                                    *reinterpret_cast<float4*>(sHout + state_off(row, cg, 4 * c + q)) =
-                                        make_float4(zv[4 * q], zv[4 * q + 1], zv[4 * q + 2], zv[4 * q + 3]);
-                                if (last_blk && p.fin &&
-                                    SSD_INB(((long long)chain * kN + row) * kP + 32 * cg + 16 * c + 15,
-                                            (long long)B * p.H * kN * kP)) {
-                                    float4* fd = reinterpret_cast<float4*>(
-                                        p.fin + ((size_t)chain * kN + row) * kP + 32 * cg + 16 * c);
-#pragma unroll
-                                    for (int q = 0; q < 4; ++q)
-                                        fd[q] = make_float4(zv[4 * q], zv[4 * q + 1], zv[4 * q + 2], zv[4 * q + 3]);
-                                }
+                            for (int q = 0; q < 4; ++q) {
+                                const float4 v = *reinterpret_cast<const float4*>(sHin + state_off(row, cg, 4 * c + q));
+                                hin[4 * q] = v.x; hin[4 * q + 1] = v.y; hin[4 * q + 2] = v.z; hin[4 * q + 3] = v.w;
                             }
                             // Hin as the bf16 B operand of V = C Hin: rows n, 64 p (MN-major)
 #pragma unroll
@@ -750,18 +532,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 *reinterpret_cast<uint4*>(sH + tc::sw128_offset(row, 4 * cg + 2 * c + c8)) = v;
                             }
                         }
-                        // one proxy fence covers the outgoing state in sHout (read by the
-                        // publisher's TMA store) and the bf16 operand in sH (read by the MMA)
+                        // the bf16 operand in sH, for the V = C Hin product
                         tc::fence_proxy_async_smem();
                         tc::tc_fence_before();
                         __syncwarp();
                         if (lane == 0) {
                             tc::mbar_arrive(&bars->hin_free);
                             tc::mbar_arrive(&bars->h_full);
-                            if (MODE == kFused) {
-                                tc::mbar_arrive(&bars->hout_full);
-                                tc::mbar_arrive(&bars->z_empty);
-                            }
                         }
                         ++hc;
                     }
@@ -847,22 +624,15 @@ int heads_per_item(const Dims& d) {
     return largest;
 }
 
-template <int MODE>
 cudaError_t launch(const Dims& d, const void* x, const void* Bm, const void* Cm, void* y,
-                   const float* states, uint64_t state_rows, ScanParams p, cudaStream_t st,
-                   const float* init = nullptr) {
-    CUtensorMap tx, tb, tcm, ty, ts, ti;
+                   const float* states, uint64_t state_rows, ScanParams p, cudaStream_t st) {
+    CUtensorMap tx, tb, tcm, ty, ts;
     // [B][T][heads or groups][64 or 128]: a block running past T reads zeros
     cudaError_t e = make_tmap_bf16_4d(&tx, x, d.P, d.H, d.T, d.B, kBlk);
     if (e == cudaSuccess) e = make_tmap_bf16_4d(&tb, Bm, d.N, d.G, d.T, d.B, kBlk);
     if (e == cudaSuccess) e = make_tmap_bf16_4d(&tcm, Cm, d.N, d.G, d.T, d.B, kBlk);
     if (e == cudaSuccess) e = make_tmap_bf16_4d(&ty, y, d.P, d.H, d.T, d.B, kBlk);
     if (e == cudaSuccess) e = make_tmap_f32_rows64(&ts, states, state_rows);
-    // the initial states [B*H*N][P] (a stand-in map over `states` when there are none)
-    if (e == cudaSuccess)
-        e = init ? make_tmap_f32_rows64(&ti, init, (uint64_t)d.B * d.H * kN)
-                 : make_tmap_f32_rows64(&ti, states, state_rows);
-    p.has_init = init ? 1 : 0;
     if (e != cudaSuccess) return e;
     p.T = d.T; p.H = d.H; p.G = d.G;
     p.nblk = (d.T + kBlk - 1) / kBlk;  // the last block may be partial
@@ -872,10 +642,10 @@ cudaError_t launch(const Dims& d, const void* x, const void* Bm, const void* Cm,
     if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
     p.n_items = (int)items;
     const int grid = (int)(items < num_sms() ? items : num_sms());
-    e = cudaFuncSetAttribute(scan_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemBytes);
     if (e != cudaSuccess) return e;
-    scan_tc_kernel<MODE><<<grid, kThreads, kSmemBytes, st>>>(tx, tb, tcm, ty, ts, ti, p, d.B);
+    scan_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(tx, tb, tcm, ty, ts, p, d.B);
     return cudaGetLastError();
 }
 
@@ -892,7 +662,7 @@ cudaError_t launch_chunk_scan_tc(const Dims& d, const void* x, const void* Bm, c
     ScanParams p = {};
     p.cum = cum;
     p.D = D;
-    return launch<kScan>(d, x, Bm, Cm, y, Hin, (uint64_t)d.B * d.H * d.nc * kN, p, st);
+    return launch(d, x, Bm, Cm, y, Hin, (uint64_t)d.B * d.H * d.nc * kN, p, st);
 }
 
 }  // namespace ssd
