@@ -18,7 +18,9 @@
 //
 // One CTA serves (b, k) and a slice of heads that share one B/C group, so the
 // B tile is loaded once per slice.  Warp roles: 0 TMA producer, 1 MMA issuer
-// (and TMEM owner), 2-5 weighting + drain (one TMEM lane quadrant each).
+// (and TMEM owner), 2-5 weighting (into one of two weighted-x buffers, so the
+// next head's weighting does not wait for this head's product), 6-9 drain
+// (one TMEM lane quadrant each, two accumulators).
 #include "../common.cuh"
 #include "../debug_checks.cuh"
 #include "../kernels.h"
@@ -30,13 +32,13 @@ namespace {
 
 constexpr int kNState = 128;  // N (MMA M)
 constexpr int kP = 64;        // P (MMA N)
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr int kHeadsMax = 8;
 
 struct __align__(8) StateBarriers {
     uint64_t b_full;
     uint64_t x_full[2], x_empty[2];
-    uint64_t xw_full, xw_empty;
+    uint64_t xw_full[2], xw_empty[2];
     uint64_t acc_full[2], acc_empty[2];
 };
 
@@ -45,7 +47,7 @@ __device__ __forceinline__ void set_abort(int* abort_flag, int* status) {
     if (status) atomicExch(status, kDevTimeout);
 }
 
-// barrier over the 128 weighting/drain threads that ORs a predicate across them
+// barrier over the 128 weighting threads that ORs a predicate across them
 __device__ __forceinline__ bool group_sync_or(bool pred) {
     uint32_t r;
     asm volatile(
@@ -68,9 +70,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t kTileBytes = Q * 128;  // Q rows of 128 bytes
     uint8_t* sB = smem;                        // two n-halves
     uint8_t* sX = smem + 2 * kTileBytes;       // two stages
-    uint8_t* sXw = smem + 4 * kTileBytes;
-    float* sCum = reinterpret_cast<float*>(smem + 5 * kTileBytes);
-    StateBarriers* bars = reinterpret_cast<StateBarriers*>(sCum + Q);
+    uint8_t* sXw = smem + 4 * kTileBytes;      // two buffers
+    StateBarriers* bars = reinterpret_cast<StateBarriers*>(smem + 6 * kTileBytes);
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(bars + 1);
     int* sAbort = reinterpret_cast<int*>(sTmem + 1);
 
@@ -90,6 +91,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // whole block leaves before any barrier if not)
         const long long nb = gridDim.x / ((long long)nc * G * slices);
         const long long last = ((long long)b * H + h0 + hpb - 1) * nc + k;
+        (void)nb;
+        (void)last;  // read by the checks of the debug build only
         if (!SSD_INB((last + 1) * Q - 1, nb * H * nc * Q) ||
             !SSD_INB((last + 1) * kNState * kP - 1, nb * H * nc * kNState * kP))
             return;
@@ -103,8 +106,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::mbar_init(&bars->acc_full[s], 1);
             tc::mbar_init(&bars->acc_empty[s], 4);
         }
-        tc::mbar_init(&bars->xw_full, 4);
-        tc::mbar_init(&bars->xw_empty, 1);
+        for (int s = 0; s < 2; ++s) {
+            tc::mbar_init(&bars->xw_full[s], 4);
+            tc::mbar_init(&bars->xw_empty[s], 1);
+        }
         *sAbort = 0;
         tc::fence_mbar_init();
     }
@@ -145,13 +150,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t idesc = tc::idesc_bf16_f32(128, kP, 1, 1);
             bool ok = tc::mbar_wait(&bars->b_full, 0, abort_v);
             for (int i = 0; ok && i < hpb; ++i) {
-                const int buf = i & 1;
-                ok = tc::mbar_wait(&bars->xw_full, i & 1, abort_v) &&
+                const int buf = i & 1;  // accumulator and weighted-x buffer
+                ok = tc::mbar_wait(&bars->xw_full[buf], (i >> 1) & 1, abort_v) &&
                      (i < 2 || tc::mbar_wait(&bars->acc_empty[buf], ((i >> 1) - 1) & 1, abort_v));
                 if (!ok) break;
                 tc::tc_fence_after();
                 const uint32_t d = tmem + buf * kP;
-                const uint32_t a0 = tc::smem_u32(sB), b0 = tc::smem_u32(sXw);
+                const uint32_t a0 = tc::smem_u32(sB), b0 = tc::smem_u32(sXw + buf * kTileBytes);
 #pragma unroll
                 for (int kk = 0; kk < Q / 16; ++kk) {
                     // 16 K-rows (tokens) per MMA: 2 swizzle atoms of 8 rows
@@ -159,20 +164,73 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t bd = tc::smem_desc_sw128(b0 + kk * 2048, kTileBytes, 1024);
                     tc::mma_ss(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
                 }
-                tc::mma_commit(&bars->xw_empty);
+                tc::mma_commit(&bars->xw_empty[buf]);
                 tc::mma_commit(&bars->acc_full[buf]);
             }
             if (!ok) set_abort(sAbort, status);
         }
-    } else {
-        // ------------------------------------ weighting + drain (4 warps) ----
+    } else if (warp < 6) {
+        // ------------------------------------------- weighting (4 warps) ----
+        // thread ct takes the 16-byte chunks ct, ct + 128, ... of the x tile
+        // (rows ct / 8 + 16 m); its rows' decays, and the chunk's last, are
+        // read from global memory one head ahead
         const int ct = threadIdx.x - 64;  // 0..127
-        const int quad = warp & 3;        // TMEM lane quadrant of this warp
-        const int n = quad * 32 + lane;   // accumulator row = state index
+        constexpr int kRowsPer = Q / 16;  // rows per thread
+        float cw[kRowsPer], cl = 0.f;
+        auto load_cum = [&](int i) {
+            const float* cumk = cum + (((size_t)b * H + h0 + i) * nc + k) * Q;
+#pragma unroll
+            for (int m = 0; m < kRowsPer; ++m) cw[m] = __ldg(cumk + (ct >> 3) + 16 * m);
+            cl = __ldg(cumk + Q - 1);
+        };
         bool ok = true;
-        auto drain = [&](int i) -> bool {
+        if (hpb > 0) load_cum(0);
+        for (int i = 0; i < hpb; ++i) {
+            const int st = i & 1;
+            // the weight of row s: exp(cum_end - cum_s), or exp(cum_s) from the chunk start
+            float w[kRowsPer];
+            const float cend = from_start ? 0.f : cl;
+            const float sgn = from_start ? 1.f : -1.f;
+#pragma unroll
+            for (int m = 0; m < kRowsPer; ++m) w[m] = __expf(fmaf(sgn, cw[m], cend));
+            if (i + 1 < hpb) load_cum(i + 1);
+            ok = tc::mbar_wait(&bars->x_full[st], (i >> 1) & 1, abort_v) &&
+                 (i < 2 || tc::mbar_wait(&bars->xw_empty[st], ((i >> 1) - 1) & 1, abort_v));
+            if (!ok) set_abort(sAbort, status);
+            if (group_sync_or(!ok || *abort_v != 0)) { ok = false; break; }
+            const uint8_t* xs = sX + st * kTileBytes;
+            uint8_t* xw = sXw + st * kTileBytes;
+#pragma unroll
+            for (int m = 0; m < kRowsPer; ++m) {
+                const int c = ct + 128 * m;
+                uint4 v = *reinterpret_cast<const uint4*>(xs + c * 16);
+                uint32_t* u = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float2 f = tc::unpack_bf16x2(u[e]);
+                    u[e] = tc::pack_bf16x2(f.x * w[m], f.y * w[m]);
+                }
+                *reinterpret_cast<uint4*>(xw + c * 16) = v;
+            }
+            tc::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tc::mbar_arrive(&bars->xw_full[st]);
+                tc::mbar_arrive(&bars->x_empty[st]);
+            }
+        }
+        if (!ok) set_abort(sAbort, status);
+    } else {
+        // ----------------------------------------------- drain (4 warps) ----
+        const int quad = warp & 3;       // TMEM lane quadrant of this warp
+        const int n = quad * 32 + lane;  // accumulator row = state index
+        for (int i = 0; i < hpb; ++i) {
             const int buf = i & 1;
-            if (!tc::mbar_wait(&bars->acc_full[buf], (i >> 1) & 1, abort_v)) return false;
+            const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->acc_full[buf], (i >> 1) & 1, abort_v));
+            if (!ok) {
+                if (lane == 0) set_abort(sAbort, status);
+                break;
+            }
             tc::tc_fence_after();
             float v0[32], v1[32];
             const uint32_t t = tmem + ((uint32_t)(quad * 32) << 16) + buf * kP;
@@ -183,8 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&bars->acc_empty[buf]);
             // each thread owns one state row n: 64 contiguous floats (256 B)
-            const int h = h0 + i;
-            float* dst = states + ((((size_t)b * H + h) * nc + k) * kNState + n) * kP;
+            float* dst = states + ((((size_t)b * H + h0 + i) * nc + k) * kNState + n) * kP;
 #pragma unroll
             for (int j = 0; j < 8; ++j)
                 *reinterpret_cast<float4*>(dst + 4 * j) =
@@ -193,48 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < 8; ++j)
                 *reinterpret_cast<float4*>(dst + 32 + 4 * j) =
                     make_float4(v1[4 * j], v1[4 * j + 1], v1[4 * j + 2], v1[4 * j + 3]);
-            return true;
-        };
-        for (int i = 0; i < hpb; ++i) {
-            const int h = h0 + i;
-            const int st = i & 1;
-            // decay weights of this head's chunk
-            const float* cumk = cum + (((size_t)b * H + h) * nc + k) * Q;
-            for (int s = ct; s < Q; s += 128) sCum[s] = cumk[s];
-            ok = tc::mbar_wait(&bars->x_full[st], (i >> 1) & 1, abort_v) &&
-                 (i == 0 || tc::mbar_wait(&bars->xw_empty, (i - 1) & 1, abort_v));
-            if (!ok) set_abort(sAbort, status);
-            if (group_sync_or(!ok || *abort_v != 0)) { ok = false; break; }
-            const float cend = from_start ? 0.f : sCum[Q - 1];
-            const float sgn = from_start ? 1.f : -1.f;
-            const uint8_t* xs = sX + st * kTileBytes;
-            for (int c = ct; c < Q * 8; c += 128) {
-                const int s = c >> 3;  // token row; the 8 chunks of a row share w
-                const float w = __expf(fmaf(sgn, sCum[s], cend));
-                uint4 v = *reinterpret_cast<const uint4*>(xs + c * 16);
-                uint32_t* u = reinterpret_cast<uint32_t*>(&v);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    float2 f = tc::unpack_bf16x2(u[e]);
-                    u[e] = tc::pack_bf16x2(f.x * w, f.y * w);
-                }
-                *reinterpret_cast<uint4*>(sXw + c * 16) = v;
-            }
-            tc::fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                tc::mbar_arrive(&bars->xw_full);
-                tc::mbar_arrive(&bars->x_empty[st]);
-            }
-            if (i > 0) {
-                ok = drain(i - 1);
-                if (!ok) set_abort(sAbort, status);
-            }
-            // sCum is rewritten next head; the drain result decides for everyone
-            if (group_sync_or(!ok || *abort_v != 0)) { ok = false; break; }
         }
-        if (ok && hpb > 0) ok = drain(hpb - 1);
-        if (!ok) set_abort(sAbort, status);
     }
     tc::tc_fence_before();
     __syncthreads();
@@ -254,7 +270,7 @@ int heads_per_cta(const Dims& d) {
 
 template <int Q>
 size_t smem_bytes() {
-    return 1024 + 5 * Q * 128 + Q * 4 + sizeof(StateBarriers) + 16;
+    return 1024 + 6 * Q * 128 + sizeof(StateBarriers) + 16;
 }
 
 }  // namespace
