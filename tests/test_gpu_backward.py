@@ -37,6 +37,9 @@ CASES = [
     small_case(B=2, T=300, H=4, P=64, N=128, G=2, chunk=128, dtype="bf16", seed=84),
     # tensor-core forms: 256-token chunks, grouped B/C, a last chunk of 8 rows
     small_case(B=2, T=520, H=4, P=64, N=128, G=2, chunk=256, dtype="bf16", seed=87),
+    # the group-summing forms over longer head loops (8 and 4 heads per group)
+    small_case(B=1, T=1000, H=8, P=64, N=128, G=1, chunk=256, dtype="bf16", seed=88),
+    small_case(B=2, T=384, H=12, P=64, N=128, G=3, chunk=128, dtype="bf16", seed=89),
     small_case(B=1, T=7, H=2, P=5, N=3, G=1, chunk=7, dtype="f32", seed=85),
     small_case(B=1, T=5, H=1, P=3, N=2, G=1, chunk=1, dtype="f32", seed=86),
 ]
