@@ -491,7 +491,8 @@ struct GroupFormSmem {
     static constexpr uint32_t Z = V + 4 * kBox;        // 2 tiles x 2 boxes (MC = 128)
     static constexpr uint32_t M = Z + 4 * kBox;        // 2 stages x 2 boxes of 64 rows
     static constexpr uint32_t CUM = M + 2 * 2 * 64 * 128;  // 2 stages x [256] fp32
-    static constexpr uint32_t BAR = CUM + 2 * 256 * 4;
+    static constexpr uint32_t COLF = CUM + 2 * 256 * 4;    // 2 stages x [128] column factors
+    static constexpr uint32_t BAR = COLF + 2 * 128 * 4;
     static constexpr uint32_t MISC = BAR + 128;
     static constexpr size_t bytes = 1024 + MISC + 16;
 };
@@ -511,6 +512,7 @@ __global__ void __launch_bounds__(kFormThreads, 1)
     uint8_t* sZ = sm + L::Z;
     uint8_t* sM = sm + L::M;
     float* sCum = reinterpret_cast<float*>(sm + L::CUM);
+    float* sColf = reinterpret_cast<float*>(sm + L::COLF);
     GroupFormBars* bars = reinterpret_cast<GroupFormBars*>(sm + L::BAR);
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + L::MISC);
 
@@ -667,23 +669,51 @@ __global__ void __launch_bounds__(kFormThreads, 1)
             return r != 0;
         };
         const int kk4 = (mt % (K / 4)) * 4, m8 = (mt / (K / 4)) * 8;  // this thread's 4 x 8 block of M
+        // With two V tiles one of them lies wholly off the diagonal tile (causal:
+        // the first, every j < i; anti-causal: the second, every j > i).  There
+        // the decay factorises through the last token of the first tile,
+        // e^{+-(c_i - c_j)} = a_i b_j with a_i = e^{+-(c_i - c_127)} and
+        // b_j = e^{+-(c_127 - c_j)}, both <= 1: a row factor and a column factor
+        // instead of an exp per score (the rows and columns past T are zero
+        // scores already).
+        const int voff = nt == 2 ? (ANTI ? 1 : 0) : -1;  // the off-diagonal tile, if any
+        // a head's decay (one per thread: Q <= 256) and its state ([N][P]: M[p][n]),
+        // read one head ahead
+        float cpre = 0.f;
+        float4 mv[8];
+        auto prefetch = [&](int hh) {
+            const size_t chain = (size_t)b * p.H + hfirst + hh;
+            if (mt < p.Q) cpre = p.cum[(chain * p.nc + k) * p.Q + mt];
+            const float* Mk = p.Mst + (chain * p.nc + k) * (size_t)p.NP;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mv[e] = *reinterpret_cast<const float4*>(Mk + (size_t)(m8 + e) * K + kk4);
+        };
+        prefetch(0);
         bool ok = true;
-        float ci = 0.f, cend = 0.f;
+        float ci = 0.f, cend = 0.f, arow = 0.f;
         for (int s = 0; s < nsteps; ++s) {
             const int hh = s / nt, v = s - hh * nt, bf = s & 1, st = hh & 1;
-            const size_t chain = (size_t)b * p.H + hfirst + hh;
             float* cumh = sCum + st * 256;
-            float4 mv[8];
+            float* colf = sColf + st * 128;
+            float4 mcur[8];
             if (v == 0) {
-                // the head's in-chunk decays, and its state read ahead ([N][P]: M[p][n])
-                for (int t = mt; t < p.Q; t += 256) cumh[t] = p.cum[(chain * p.nc + k) * p.Q + t];
-                const float* Mk = p.Mst + (chain * p.nc + k) * (size_t)p.NP;
+                if (mt < p.Q) cumh[mt] = cpre;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) mv[e] = *reinterpret_cast<const float4*>(Mk + (size_t)(m8 + e) * K + kk4);
+                for (int e = 0; e < 8; ++e) mcur[e] = mv[e];
                 math_sync();  // cumh complete
                 ci = cumh[i];
                 cend = cumh[p.Q - 1];
+                if (voff >= 0) {
+                    const float cref = cumh[kRowsT - 1];
+                    arow = ex2_approx((ANTI ? cref - ci : ci - cref) * 1.4426950408889634f);
+                    if (mt < kRowsT) {
+                        const float cj = cumh[kRowsT * voff + mt];
+                        colf[mt] = ex2_approx((ANTI ? cj - cref : cref - cj) * 1.4426950408889634f);
+                    }
+                    math_sync();  // colf complete
+                }
             }
+            if (v == nt - 1 && hh + 1 < HG) prefetch(hh + 1);  // lands during this step
             bool okh = ok && tc::mbar_wait(&bars->s_full[bf], (s >> 1) & 1, nullptr, kBudget);
             if (!okh) timed_out();
             okh = !math_or(!okh);
@@ -696,10 +726,10 @@ __global__ void __launch_bounds__(kFormThreads, 1)
                                                tc::pack_bf16x2(f4, f5), tc::pack_bf16x2(f6, f7));
                     *reinterpret_cast<uint4*>(sMs + (m8 >> 6) * (K * 128) + tc::sw128_offset(kk, (m8 & 63) >> 3)) = w;
                 };
-                put(kk4, mv[0].x, mv[1].x, mv[2].x, mv[3].x, mv[4].x, mv[5].x, mv[6].x, mv[7].x);
-                put(kk4 + 1, mv[0].y, mv[1].y, mv[2].y, mv[3].y, mv[4].y, mv[5].y, mv[6].y, mv[7].y);
-                put(kk4 + 2, mv[0].z, mv[1].z, mv[2].z, mv[3].z, mv[4].z, mv[5].z, mv[6].z, mv[7].z);
-                put(kk4 + 3, mv[0].w, mv[1].w, mv[2].w, mv[3].w, mv[4].w, mv[5].w, mv[6].w, mv[7].w);
+                put(kk4, mcur[0].x, mcur[1].x, mcur[2].x, mcur[3].x, mcur[4].x, mcur[5].x, mcur[6].x, mcur[7].x);
+                put(kk4 + 1, mcur[0].y, mcur[1].y, mcur[2].y, mcur[3].y, mcur[4].y, mcur[5].y, mcur[6].y, mcur[7].y);
+                put(kk4 + 2, mcur[0].z, mcur[1].z, mcur[2].z, mcur[3].z, mcur[4].z, mcur[5].z, mcur[6].z, mcur[7].z);
+                put(kk4 + 3, mcur[0].w, mcur[1].w, mcur[2].w, mcur[3].w, mcur[4].w, mcur[5].w, mcur[6].w, mcur[7].w);
             }
             if (okh) {
                 tc::tc_fence_after();
@@ -737,24 +767,38 @@ __global__ void __launch_bounds__(kFormThreads, 1)
                     tc::tmem_ld_wait();
                     if (r == (half == 0 ? 1 : 0)) pair_sync();
                     const int j0 = jbase + 128 * v + cin;
+                    if (v == voff) {
 #pragma unroll
-                    for (int g8 = 0; g8 < 2; ++g8) {
-                        uint32_t pk[8];
+                        for (int g8 = 0; g8 < 2; ++g8) {
+                            uint32_t pk[8];
 #pragma unroll
-                        for (int e2 = 0; e2 < 8; ++e2) {
-                            float pv[2];
-#pragma unroll
-                            for (int q = 0; q < 2; ++q) {
-                                const int e = 16 * g8 + 2 * e2 + q;
-                                const int j = j0 + e;
-                                const bool keep = (ANTI ? j >= i : j <= i) && j < qv && i < qv;
-                                const float ex = ex2_approx(
-                                    keep ? (ANTI ? cumh[j] - ci : ci - cumh[j]) * 1.4426950408889634f : 0.f);
-                                pv[q] = keep ? sv[e] * ex : 0.f;
+                            for (int e2 = 0; e2 < 8; ++e2) {
+                                const int e = 16 * g8 + 2 * e2;
+                                pk[e2] = tc::pack_bf16x2(sv[e] * arow * colf[cin + e],
+                                                         sv[e + 1] * arow * colf[cin + e + 1]);
                             }
-                            pk[e2] = tc::pack_bf16x2(pv[0], pv[1]);
+                            tc::tmem_st8(tbase + cin / 2 + 8 * g8, pk);
                         }
-                        tc::tmem_st8(tbase + cin / 2 + 8 * g8, pk);
+                    } else {
+#pragma unroll
+                        for (int g8 = 0; g8 < 2; ++g8) {
+                            uint32_t pk[8];
+#pragma unroll
+                            for (int e2 = 0; e2 < 8; ++e2) {
+                                float pv[2];
+#pragma unroll
+                                for (int q = 0; q < 2; ++q) {
+                                    const int e = 16 * g8 + 2 * e2 + q;
+                                    const int j = j0 + e;
+                                    const bool keep = (ANTI ? j >= i : j <= i) && j < qv && i < qv;
+                                    const float ex = ex2_approx(
+                                        keep ? (ANTI ? cumh[j] - ci : ci - cumh[j]) * 1.4426950408889634f : 0.f);
+                                    pv[q] = keep ? sv[e] * ex : 0.f;
+                                }
+                                pk[e2] = tc::pack_bf16x2(pv[0], pv[1]);
+                            }
+                            tc::tmem_st8(tbase + cin / 2 + 8 * g8, pk);
+                        }
                     }
                 }
                 tc::tmem_st_wait();
