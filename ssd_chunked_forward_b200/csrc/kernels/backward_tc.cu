@@ -76,7 +76,8 @@ struct FormSmem {
     static constexpr uint32_t M = R + 2 * (MC / 64) * kBox;                // MC/64 boxes of K rows
     static constexpr uint32_t CUM = R + (kV > kZM ? kV : kZM);             // [256] fp32
     static constexpr uint32_t RED = CUM + 256 * 4;                         // [2][128] fp32 row partials
-    static constexpr uint32_t BAR = RED + 2 * 128 * 4;
+    static constexpr uint32_t COLF = RED + 2 * 128 * 4;                    // [128] column factors
+    static constexpr uint32_t BAR = COLF + 128 * 4;
     static constexpr uint32_t MISC = BAR + 64;
     static constexpr size_t bytes = 1024 + MISC + 16;
 };
@@ -98,6 +99,7 @@ __global__ void __launch_bounds__(kFormThreads, 2)
     uint8_t* sM = sm + L::M;
     float* sCum = reinterpret_cast<float*>(sm + L::CUM);
     float* sRed = reinterpret_cast<float*>(sm + L::RED);
+    float* sColf = reinterpret_cast<float*>(sm + L::COLF);
     FormBars* bars = reinterpret_cast<FormBars*>(sm + L::BAR);
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + L::MISC);
 
@@ -134,6 +136,19 @@ __global__ void __launch_bounds__(kFormThreads, 2)
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
+    // With two V tiles one lies wholly off the diagonal tile (causal: the
+    // first, every j < i; anti-causal: the second, every j > i); there the
+    // decay factorises through the first tile's last token into a row factor
+    // and a column factor, both <= 1 (the rows and columns past T are zero
+    // scores already)
+    const int voff = nt == 2 ? (ANTI ? 1 : 0) : -1;
+    if (voff >= 0) {
+        if (threadIdx.x < kRowsT) {
+            const float cref = sCum[kRowsT - 1], cj = sCum[kRowsT * voff + threadIdx.x];
+            sColf[threadIdx.x] = ex2_approx((ANTI ? cj - cref : cref - cj) * 1.4426950408889634f);
+        }
+        __syncthreads();
+    }
     const uint32_t tmem = *sTmem;
     constexpr uint64_t kBudget = 2000000000ull;  // 2 s per wait
     auto timed_out = [&]() {
@@ -291,17 +306,17 @@ __global__ void __launch_bounds__(kFormThreads, 2)
                 v.w = tc::mul_bf16x2(v.w, u2);
                 *ptr = v;
             }
-            // P~ = S masked and decayed, packed in place: with two V tiles
-            // warp half h takes tile h, with one the halves take a 64-column
-            // piece each; a piece is read and written 32 columns at a time,
-            // its packed scores landing in the first half of its tile.  The
-            // pair of warps of a lane quadrant meets once per piece: the owner
-            // of a tile's first piece after reading all of it, the other
-            // before its first write (which lands in the first piece).
-            const int npc = nt == 2 ? 2 : 1;
-            for (int u = 0; u < npc; ++u) {
-                const int tile = nt == 2 ? half : 0;
-                const int c0 = nt == 2 ? 64 * u : 64 * half;  // column of the piece in its tile
+            // P~ = S masked and decayed, packed in place, one V tile at a time:
+            // warp half h takes the tile's columns [64 h, 64 h + 64), read and
+            // written 32 at a time, the packed scores landing in the first half
+            // of the tile.  The pair of warps of a lane quadrant meets once per
+            // tile (half 0 after reading all of its columns, half 1 before its
+            // first write, which lands in half 0's columns).
+            const float arow = voff >= 0 ? ex2_approx((ANTI ? sCum[kRowsT - 1] - ci : ci - sCum[kRowsT - 1]) *
+                                                      1.4426950408889634f)
+                                         : 0.f;
+            for (int tile = 0; tile < nt; ++tile) {
+                const int c0 = 64 * half;
 #pragma unroll
                 for (int r = 0; r < 2; ++r) {
                     const int cin = c0 + 32 * r;
@@ -310,34 +325,47 @@ __global__ void __launch_bounds__(kFormThreads, 2)
                     tc::tmem_ld16(tbase + cin, *reinterpret_cast<float(*)[16]>(s));
                     tc::tmem_ld16(tbase + cin + 16, *reinterpret_cast<float(*)[16]>(s + 16));
                     tc::tmem_ld_wait();
-                    if (r == (c0 == 0 ? 1 : 0)) pair_sync();
+                    if (r == (half == 0 ? 1 : 0)) pair_sync();
                     const int j0 = jbase + 128 * tile + cin;  // chunk column of s[0]
+                    if (tile == voff) {
 #pragma unroll
-                    for (int g8 = 0; g8 < 2; ++g8) {
-                        uint32_t pk[8];
+                        for (int g8 = 0; g8 < 2; ++g8) {
+                            uint32_t pk[8];
 #pragma unroll
-                        for (int e2 = 0; e2 < 8; ++e2) {
-                            float pv[2];
-#pragma unroll
-                            for (int q = 0; q < 2; ++q) {
-                                const int e = 16 * g8 + 2 * e2 + q;
-                                const int j = j0 + e;
-                                const bool keep = (ANTI ? j >= i : j <= i) && j < qv && i < qv;
-                                const float ex = ex2_approx(
-                                    keep ? (ANTI ? sCum[j] - ci : ci - sCum[j]) * 1.4426950408889634f : 0.f);
-                                pv[q] = keep ? s[e] * ex : 0.f;
+                            for (int e2 = 0; e2 < 8; ++e2) {
+                                const int e = 16 * g8 + 2 * e2;
+                                pk[e2] = tc::pack_bf16x2(s[e] * arow * sColf[cin + e],
+                                                         s[e + 1] * arow * sColf[cin + e + 1]);
                             }
-                            pk[e2] = tc::pack_bf16x2(pv[0], pv[1]);
+                            tc::tmem_st8(tbase + cin / 2 + 8 * g8, pk);
                         }
-                        tc::tmem_st8(tbase + cin / 2 + 8 * g8, pk);
+                    } else {
+#pragma unroll
+                        for (int g8 = 0; g8 < 2; ++g8) {
+                            uint32_t pk[8];
+#pragma unroll
+                            for (int e2 = 0; e2 < 8; ++e2) {
+                                float pv[2];
+#pragma unroll
+                                for (int q = 0; q < 2; ++q) {
+                                    const int e = 16 * g8 + 2 * e2 + q;
+                                    const int j = j0 + e;
+                                    const bool keep = (ANTI ? j >= i : j <= i) && j < qv && i < qv;
+                                    const float ex = ex2_approx(
+                                        keep ? (ANTI ? sCum[j] - ci : ci - sCum[j]) * 1.4426950408889634f : 0.f);
+                                    pv[q] = keep ? s[e] * ex : 0.f;
+                                }
+                                pk[e2] = tc::pack_bf16x2(pv[0], pv[1]);
+                            }
+                            tc::tmem_st8(tbase + cin / 2 + 8 * g8, pk);
+                        }
                     }
                 }
             }
             tc::tmem_st_wait();
         } else {
             // keep the pair barriers matched with a partner that did not fail
-            const int npc = nt == 2 ? 2 : 1;
-            for (int u = 0; u < npc; ++u) pair_sync();
+            for (int tile = 0; tile < nt; ++tile) pair_sync();
         }
         tc::fence_proxy_async_smem();  // U~ and M for the products
         tc::tc_fence_before();
