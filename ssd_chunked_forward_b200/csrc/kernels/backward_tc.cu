@@ -77,7 +77,8 @@ struct FormSmem {
     static constexpr uint32_t CUM = R + (kV > kZM ? kV : kZM);             // [256] fp32
     static constexpr uint32_t RED = CUM + 256 * 4;                         // [2][128] fp32 row partials
     static constexpr uint32_t COLF = RED + 2 * 128 * 4;                    // [128] column factors
-    static constexpr uint32_t BAR = COLF + 128 * 4;
+    static constexpr uint32_t COLFD = COLF + 128 * 4;                      // [4][128] diagonal-tile factors
+    static constexpr uint32_t BAR = COLFD + 4 * 128 * 4;
     static constexpr uint32_t MISC = BAR + 64;
     static constexpr size_t bytes = 1024 + MISC + 16;
 };
@@ -100,6 +101,7 @@ __global__ void __launch_bounds__(kFormThreads, 2)
     float* sCum = reinterpret_cast<float*>(sm + L::CUM);
     float* sRed = reinterpret_cast<float*>(sm + L::RED);
     float* sColf = reinterpret_cast<float*>(sm + L::COLF);
+    float* sColfd = reinterpret_cast<float*>(sm + L::COLFD);
     FormBars* bars = reinterpret_cast<FormBars*>(sm + L::BAR);
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + L::MISC);
 
@@ -142,13 +144,24 @@ __global__ void __launch_bounds__(kFormThreads, 2)
     // and a column factor, both <= 1 (the rows and columns past T are zero
     // scores already)
     const int voff = nt == 2 ? (ANTI ? 1 : 0) : -1;
-    if (voff >= 0) {
-        if (threadIdx.x < kRowsT) {
-            const float cref = sCum[kRowsT - 1], cj = sCum[kRowsT * voff + threadIdx.x];
-            sColf[threadIdx.x] = ex2_approx((ANTI ? cj - cref : cref - cj) * 1.4426950408889634f);
+    // The diagonal tile's 32-token sub-blocks factorise the same way: row
+    // sub-block ri against column sub-blocks below it (causal) or above it
+    // (anti-causal) through the token at ri's start (causal: i0 + 32 ri - 1)
+    // or end (anti: i0 + 32 ri + 31); sColfd[ri][col] holds the column factors
+    for (int e = threadIdx.x; e < 4 * kRowsT; e += kFormThreads) {
+        const int ri = e >> 7, col = e & (kRowsT - 1);
+        float f = 0.f;
+        if (ANTI ? col >= 32 * ri + 32 : col < 32 * ri) {
+            const float cr = sCum[i0 + (ANTI ? 32 * ri + 31 : 32 * ri - 1)], cj = sCum[i0 + col];
+            f = ex2_approx((ANTI ? cj - cr : cr - cj) * 1.4426950408889634f);
         }
-        __syncthreads();
+        sColfd[e] = f;
     }
+    if (voff >= 0 && threadIdx.x < kRowsT) {
+        const float cref = sCum[kRowsT - 1], cj = sCum[kRowsT * voff + threadIdx.x];
+        sColf[threadIdx.x] = ex2_approx((ANTI ? cj - cref : cref - cj) * 1.4426950408889634f);
+    }
+    __syncthreads();
     const uint32_t tmem = *sTmem;
     constexpr uint64_t kBudget = 2000000000ull;  // 2 s per wait
     auto timed_out = [&]() {
@@ -315,6 +328,13 @@ __global__ void __launch_bounds__(kFormThreads, 2)
             const float arow = voff >= 0 ? ex2_approx((ANTI ? sCum[kRowsT - 1] - ci : ci - sCum[kRowsT - 1]) *
                                                       1.4426950408889634f)
                                          : 0.f;
+            // the row factor of the diagonal tile's sub-block factorisation (row sub-block = quad)
+            const bool has_d = ANTI ? quad < 3 : quad > 0;
+            const float adiag =
+                has_d ? ex2_approx((ANTI ? sCum[i0 + 32 * quad + 31] - ci : ci - sCum[i0 + 32 * quad - 1]) *
+                                   1.4426950408889634f)
+                      : 0.f;
+            const int tdiag = ANTI ? 0 : nt - 1;
             for (int tile = 0; tile < nt; ++tile) {
                 const int c0 = 64 * half;
 #pragma unroll
@@ -327,18 +347,27 @@ __global__ void __launch_bounds__(kFormThreads, 2)
                     tc::tmem_ld_wait();
                     if (r == (half == 0 ? 1 : 0)) pair_sync();
                     const int j0 = jbase + 128 * tile + cin;  // chunk column of s[0]
-                    if (tile == voff) {
+                    // the diagonal tile: this round's 32 columns are one sub-block rj
+                    const int rj = cin >> 5;
+                    const bool dfast = tile == tdiag && (ANTI ? rj > quad : rj < quad);
+                    const bool dzero = tile == tdiag && (ANTI ? rj < quad : rj > quad);
+                    if (tile == voff || dfast) {
+                        const float a = tile == voff ? arow : adiag;
+                        const float* cf = tile == voff ? sColf : sColfd + quad * kRowsT;
 #pragma unroll
                         for (int g8 = 0; g8 < 2; ++g8) {
                             uint32_t pk[8];
 #pragma unroll
                             for (int e2 = 0; e2 < 8; ++e2) {
                                 const int e = 16 * g8 + 2 * e2;
-                                pk[e2] = tc::pack_bf16x2(s[e] * arow * sColf[cin + e],
-                                                         s[e + 1] * arow * sColf[cin + e + 1]);
+                                pk[e2] = tc::pack_bf16x2(s[e] * a * cf[cin + e], s[e + 1] * a * cf[cin + e + 1]);
                             }
                             tc::tmem_st8(tbase + cin / 2 + 8 * g8, pk);
                         }
+                    } else if (dzero) {
+                        const uint32_t pk[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+                        tc::tmem_st8(tbase + cin / 2, pk);
+                        tc::tmem_st8(tbase + cin / 2 + 8, pk);
                     } else {
 #pragma unroll
                         for (int g8 = 0; g8 < 2; ++g8) {
@@ -520,7 +549,8 @@ struct GroupFormSmem {
     static constexpr uint32_t M = Z + 4 * kBox;        // 2 stages x 2 boxes of 64 rows
     static constexpr uint32_t CUM = M + 2 * 2 * 64 * 128;  // 2 stages x [256] fp32
     static constexpr uint32_t COLF = CUM + 2 * 256 * 4;    // 2 stages x [128] column factors
-    static constexpr uint32_t BAR = COLF + 2 * 128 * 4;
+    static constexpr uint32_t COLFD = COLF + 2 * 128 * 4;  // 2 stages x [4][128] diagonal-tile factors
+    static constexpr uint32_t BAR = COLFD + 2 * 4 * 128 * 4;
     static constexpr uint32_t MISC = BAR + 128;
     static constexpr size_t bytes = 1024 + MISC + 16;
 };
@@ -541,6 +571,7 @@ __global__ void __launch_bounds__(kFormThreads, 1)
     uint8_t* sM = sm + L::M;
     float* sCum = reinterpret_cast<float*>(sm + L::CUM);
     float* sColf = reinterpret_cast<float*>(sm + L::COLF);
+    float* sColfd = reinterpret_cast<float*>(sm + L::COLFD);
     GroupFormBars* bars = reinterpret_cast<GroupFormBars*>(sm + L::BAR);
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + L::MISC);
 
@@ -717,12 +748,18 @@ __global__ void __launch_bounds__(kFormThreads, 1)
             for (int e = 0; e < 8; ++e) mv[e] = *reinterpret_cast<const float4*>(Mk + (size_t)(m8 + e) * K + kk4);
         };
         prefetch(0);
+        // the diagonal tile: row sub-block quad against the column sub-blocks
+        // below it (causal) or above it (anti-causal), through the token at the
+        // row sub-block's start or end (per head: sColfd[ri][col])
+        const int tdiag = ANTI ? 0 : nt - 1;
+        const bool has_d = ANTI ? quad < 3 : quad > 0;
         bool ok = true;
-        float ci = 0.f, cend = 0.f, arow = 0.f;
+        float ci = 0.f, cend = 0.f, arow = 0.f, adiag = 0.f;
         for (int s = 0; s < nsteps; ++s) {
             const int hh = s / nt, v = s - hh * nt, bf = s & 1, st = hh & 1;
             float* cumh = sCum + st * 256;
             float* colf = sColf + st * 128;
+            float* colfd = sColfd + st * 4 * 128;
             float4 mcur[8];
             if (v == 0) {
                 if (mt < p.Q) cumh[mt] = cpre;
@@ -738,8 +775,20 @@ __global__ void __launch_bounds__(kFormThreads, 1)
                         const float cj = cumh[kRowsT * voff + mt];
                         colf[mt] = ex2_approx((ANTI ? cj - cref : cref - cj) * 1.4426950408889634f);
                     }
-                    math_sync();  // colf complete
                 }
+                if (has_d)
+                    adiag = ex2_approx((ANTI ? cumh[i0 + 32 * quad + 31] - ci : ci - cumh[i0 + 32 * quad - 1]) *
+                                       1.4426950408889634f);
+                for (int e = mt; e < 4 * kRowsT; e += 256) {
+                    const int ri = e >> 7, col = e & (kRowsT - 1);
+                    float f = 0.f;
+                    if (ANTI ? col >= 32 * ri + 32 : col < 32 * ri) {
+                        const float cr = cumh[i0 + (ANTI ? 32 * ri + 31 : 32 * ri - 1)], cj = cumh[i0 + col];
+                        f = ex2_approx((ANTI ? cj - cr : cr - cj) * 1.4426950408889634f);
+                    }
+                    colfd[e] = f;
+                }
+                math_sync();  // colf, colfd complete
             }
             if (v == nt - 1 && hh + 1 < HG) prefetch(hh + 1);  // lands during this step
             bool okh = ok && tc::mbar_wait(&bars->s_full[bf], (s >> 1) & 1, nullptr, kBudget);
@@ -795,18 +844,27 @@ __global__ void __launch_bounds__(kFormThreads, 1)
                     tc::tmem_ld_wait();
                     if (r == (half == 0 ? 1 : 0)) pair_sync();
                     const int j0 = jbase + 128 * v + cin;
-                    if (v == voff) {
+                    // the diagonal tile: this round's 32 columns are one sub-block rj
+                    const int rj = cin >> 5;
+                    const bool dfast = v == tdiag && (ANTI ? rj > quad : rj < quad);
+                    const bool dzero = v == tdiag && (ANTI ? rj < quad : rj > quad);
+                    if (v == voff || dfast) {
+                        const float a = v == voff ? arow : adiag;
+                        const float* cf = v == voff ? colf : colfd + quad * kRowsT;
 #pragma unroll
                         for (int g8 = 0; g8 < 2; ++g8) {
                             uint32_t pk[8];
 #pragma unroll
                             for (int e2 = 0; e2 < 8; ++e2) {
                                 const int e = 16 * g8 + 2 * e2;
-                                pk[e2] = tc::pack_bf16x2(sv[e] * arow * colf[cin + e],
-                                                         sv[e + 1] * arow * colf[cin + e + 1]);
+                                pk[e2] = tc::pack_bf16x2(sv[e] * a * cf[cin + e], sv[e + 1] * a * cf[cin + e + 1]);
                             }
                             tc::tmem_st8(tbase + cin / 2 + 8 * g8, pk);
                         }
+                    } else if (dzero) {
+                        const uint32_t pk[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+                        tc::tmem_st8(tbase + cin / 2, pk);
+                        tc::tmem_st8(tbase + cin / 2 + 8, pk);
                     } else {
 #pragma unroll
                         for (int g8 = 0; g8 < 2; ++g8) {
