@@ -13,8 +13,7 @@
 //
 // y - Dx and dx - D dy run here (per head; their rows reduced in the
 // epilogue, see below); dC and dB run in chunk_form_group_tc_kernel further
-// down, summed over each group's heads.  The template also serves the other
-// operand shapes (K = 64, MC = 128, state read transposed, rows stored).
+// down, summed over each group's heads.
 //
 // One CTA per (chunk, 128-row tile, batch x head), two CTAs per SM (about
 // 100 KB of shared memory and 256 TMEM columns each), so one CTA's copies
@@ -47,8 +46,7 @@ __host__ __device__ constexpr uint32_t col_o(int q) { return 64u + 128u * (uint3
 
 struct FormParams {
     const float* cum;  // [B*H][nc][Q]
-    const float* Mst;  // [B*H][nc][K*MC]: M stored [K][MC] (MROW) or [MC][K]
-    float* out;        // [B][T][H][MC]
+    const float* Mst;  // [B*H][nc][N*P]: M = the state, [K = N][MC = P]
     int T, H, G, Q, nc, NP;
     int u_grp, v_grp, z_grp;  // operand indexed by B/C group (else by head)
     int* status;              // set to kDevTimeout when a bounded wait gives up
@@ -84,12 +82,14 @@ struct FormSmem {
 };
 static_assert(FormSmem<128, 64>::bytes <= 113 * 1024, "two CTAs per SM");
 
-// EPI 0 stores the rows (fp32); EPI 1 (y - Dx) keeps only dy . row per row;
-// EPI 2 (dx - D dy) writes dx = row + D dy (bf16) and keeps x . row and x . dy
-template <int K, int MC, bool ANTI, bool MROW, int EPI>
+// EPI 1 (y - Dx) keeps only dy . row per row; EPI 2 (dx - D dy) writes
+// dx = row + D dy (bf16) and keeps x . row and x . dy
+template <bool ANTI, int EPI>
 __global__ void __launch_bounds__(kFormThreads, 2)
     chunk_form_tc_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_v,
                          const __grid_constant__ CUtensorMap tm_z, const FormParams p) {
+    constexpr int K = 128, MC = 64;  // U, V rows of N; Z, M, the output rows of P
+    static_assert(EPI == 1 || EPI == 2, "row epilogues");
     using L = FormSmem<K, MC>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -258,23 +258,16 @@ __global__ void __launch_bounds__(kFormThreads, 2)
             }
             tc::tc_fence_after();
         };
-        // M (fp32, K x MC) read ahead with 16-byte loads: [K][MC] (MROW) a
-        // thread takes 8 consecutive columns of a row, four rows apart; [MC][K]
-        // a 4 x 8 block (4 rows kk, 8 columns m), one load per column
-        constexpr int kMTasks = MROW ? K * (MC / 8) / 256 : (K / 4) * (MC / 8) / 256;
-        static_assert(kMTasks >= 1 && (MROW ? K * (MC / 8) : (K / 4) * (MC / 8)) % 256 == 0, "M tasks");
-        float4 mv[8 * kMTasks / (MROW ? 4 : 1)];
-        if (MROW) {
+        // M (fp32 [K][MC]) read ahead with 16-byte loads: a thread takes 8
+        // consecutive columns of a row, four rows apart
+        constexpr int kMTasks = K * (MC / 8) / 256;
+        static_assert(kMTasks >= 1 && K * (MC / 8) % 256 == 0, "M tasks");
+        float4 mv[2 * kMTasks];
 #pragma unroll
-            for (int u = 0; u < kMTasks; ++u) {
-                const int c = mt + 256 * u, kk = c / (MC / 8), m8 = (c % (MC / 8)) * 8;
-                mv[2 * u] = *reinterpret_cast<const float4*>(Mk + (size_t)kk * MC + m8);
-                mv[2 * u + 1] = *reinterpret_cast<const float4*>(Mk + (size_t)kk * MC + m8 + 4);
-            }
-        } else {
-            const int kk4 = (mt % (K / 4)) * 4, m8 = (mt / (K / 4)) * 8;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) mv[e] = *reinterpret_cast<const float4*>(Mk + (size_t)(m8 + e) * K + kk4);
+        for (int u = 0; u < kMTasks; ++u) {
+            const int c = mt + 256 * u, kk = c / (MC / 8), m8 = (c % (MC / 8)) * 8;
+            mv[2 * u] = *reinterpret_cast<const float4*>(Mk + (size_t)kk * MC + m8);
+            mv[2 * u + 1] = *reinterpret_cast<const float4*>(Mk + (size_t)kk * MC + m8 + 4);
         }
         bool ok = tc::mbar_wait(&bars->s_full, 0, nullptr, kBudget);
         ok = __all_sync(0xffffffffu, ok);
@@ -288,19 +281,11 @@ __global__ void __launch_bounds__(kFormThreads, 2)
                                            tc::pack_bf16x2(f4, f5), tc::pack_bf16x2(f6, f7));
                 *reinterpret_cast<uint4*>(sM + (m8 >> 6) * (K * 128) + tc::sw128_offset(kk, (m8 & 63) >> 3)) = w;
             };
-            if (MROW) {
 #pragma unroll
-                for (int u = 0; u < kMTasks; ++u) {
-                    const int c = mt + 256 * u, kk = c / (MC / 8), m8 = (c % (MC / 8)) * 8;
-                    const float4 a0 = mv[2 * u], a1 = mv[2 * u + 1];
-                    put(kk, m8, a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w);
-                }
-            } else {
-                const int kk4 = (mt % (K / 4)) * 4, m8 = (mt / (K / 4)) * 8;
-                put(kk4, m8, mv[0].x, mv[1].x, mv[2].x, mv[3].x, mv[4].x, mv[5].x, mv[6].x, mv[7].x);
-                put(kk4 + 1, m8, mv[0].y, mv[1].y, mv[2].y, mv[3].y, mv[4].y, mv[5].y, mv[6].y, mv[7].y);
-                put(kk4 + 2, m8, mv[0].z, mv[1].z, mv[2].z, mv[3].z, mv[4].z, mv[5].z, mv[6].z, mv[7].z);
-                put(kk4 + 3, m8, mv[0].w, mv[1].w, mv[2].w, mv[3].w, mv[4].w, mv[5].w, mv[6].w, mv[7].w);
+            for (int u = 0; u < kMTasks; ++u) {
+                const int c = mt + 256 * u, kk = c / (MC / 8), m8 = (c % (MC / 8)) * 8;
+                const float4 a0 = mv[2 * u], a1 = mv[2 * u + 1];
+                put(kk, m8, a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w);
             }
         }
         if (ok) {
@@ -402,8 +387,8 @@ __global__ void __launch_bounds__(kFormThreads, 2)
         if (lane == 0) tc::mbar_arrive(&bars->p_full);
         // the row epilogues' dy (and x) rows, read while the products run
         const size_t ro = (((size_t)b * p.T + tk + i) * p.H + h) * MC + half * (MC / 2);
-        uint4 dyr[EPI ? 4 : 1], xr[EPI == 2 ? 4 : 1];
-        if (EPI != 0 && i < qv && SSD_INB((long long)ro + MC / 2 - 1, (long long)gridDim.y * p.T * MC)) {
+        uint4 dyr[4], xr[EPI == 2 ? 4 : 1];
+        if (i < qv && SSD_INB((long long)ro + MC / 2 - 1, (long long)gridDim.y * p.T * MC)) {
 #pragma unroll
             for (int u = 0; u < 4; ++u) dyr[u] = __ldg(reinterpret_cast<const uint4*>(p.dyg + ro) + u);
             if (EPI == 2) {
@@ -414,29 +399,10 @@ __global__ void __launch_bounds__(kFormThreads, 2)
         const bool ok2 = tc::mbar_wait(&bars->o_full, 0, nullptr, kBudget);
         if (!__all_sync(0xffffffffu, ok2) && lane == 0) timed_out();
         ok = ok && __all_sync(0xffffffffu, ok2);
-        if (EPI == 0) {
-            if (ok) {
-                tc::tc_fence_after();
-                float* o = p.out + (((size_t)b * p.T + tk + i) * p.H + h) * MC;
-#pragma unroll
-                for (int q16 = 0; q16 < MC / 32; ++q16) {
-                    const int m0 = half * (MC / 2) + 16 * q16;  // output column
-                    float v[16];
-                    tc::tmem_ld16(lane_base + col_o(m0 >> 6) + (m0 & 63), v);
-                    tc::tmem_ld_wait();
-                    if (i < qv && SSD_INB((o - p.out) + m0 + 15, (long long)gridDim.y * p.T * MC)) {
-#pragma unroll
-                        for (int e4 = 0; e4 < 4; ++e4)
-                            *reinterpret_cast<float4*>(o + m0 + 4 * e4) =
-                                make_float4(v[4 * e4], v[4 * e4 + 1], v[4 * e4 + 2], v[4 * e4 + 3]);
-                    }
-                }
-            }
-        } else {
+        {
             // the row's half of the MC = P columns against the token's dy (and x)
             // row: per-row dot products, summed over the two halves of a lane
             // quadrant through shared memory, and (EPI 2) dx
-            static_assert(EPI == 0 || MC == 64, "row epilogues serve the P = 64 forms");
             float pa = 0.f, pb = 0.f;  // EPI 1: dy . row; EPI 2: x . row, x . dy
             const bool live = ok && i < qv && SSD_INB((long long)ro + 31, (long long)gridDim.y * p.T * MC);
             if (ok) tc::tc_fence_after();
@@ -949,28 +915,29 @@ cudaError_t launch_form_group_tc_t(const Dims& d, const void* U, const void* V, 
     return cudaGetLastError();
 }
 
-template <int K, int MC, bool ANTI, bool MROW, int EPI>
+template <bool ANTI, int EPI>
 cudaError_t launch_form_tc_t(const Dims& d, const void* U, int ug, const void* V, int vg, const void* Z, int zg,
-                             const float* cum, const float* Mst, float* out, const FormEpilogue& ep,
-                             int* status, cudaStream_t st) {
+                             const float* cum, const float* Mst, const FormEpilogue& ep, int* status,
+                             cudaStream_t st) {
+    constexpr int K = 128, MC = 64;
     CUtensorMap tu, tv, tz;
     cudaError_t e = make_tmap_bf16_4d(&tu, U, K, ug ? d.G : d.H, d.T, d.B, kRowsT);
     if (e == cudaSuccess) e = make_tmap_bf16_4d(&tv, V, K, vg ? d.G : d.H, d.T, d.B, kRowsT);
     if (e == cudaSuccess) e = make_tmap_bf16_4d(&tz, Z, MC, zg ? d.G : d.H, d.T, d.B, kRowsT);
     if (e != cudaSuccess) return e;
     FormParams p = {};
-    p.cum = cum; p.Mst = Mst; p.out = out;
+    p.cum = cum; p.Mst = Mst;
     p.T = d.T; p.H = d.H; p.G = d.G; p.Q = d.Q; p.nc = d.nc; p.NP = d.N * d.P;
     p.u_grp = ug; p.v_grp = vg; p.z_grp = zg;
     p.status = status;
     p.xg = (const __nv_bfloat16*)ep.x; p.dyg = (const __nv_bfloat16*)ep.dy; p.Dv = ep.D;
     p.dxo = (__nv_bfloat16*)ep.dx; p.r1 = ep.r1; p.r2 = ep.r2; p.xd = ep.xd;
     using L = FormSmem<K, MC>;
-    e = cudaFuncSetAttribute(chunk_form_tc_kernel<K, MC, ANTI, MROW, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(chunk_form_tc_kernel<ANTI, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)L::bytes);
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)(d.nc * (d.Q / kRowsT)), (unsigned)(d.B * d.H));
-    chunk_form_tc_kernel<K, MC, ANTI, MROW, EPI><<<grid, kFormThreads, L::bytes, st>>>(tu, tv, tz, p);
+    chunk_form_tc_kernel<ANTI, EPI><<<grid, kFormThreads, L::bytes, st>>>(tu, tv, tz, p);
     return cudaGetLastError();
 }
 
@@ -988,13 +955,13 @@ cudaError_t launch_backward_forms_tc(const Dims& d, const void* x, const void* d
     if (!backward_forms_tc_supported(d)) return cudaErrorNotSupported;
     cudaError_t e;
     // y - D x: causal, U = C, V = B, Z = x, M = Hin (N x P); only dy . (y - Dx) is kept
-    e = launch_form_tc_t<128, 64, false, true, 1>(d, Cm, 1, Bm, 1, x, 0, cum, states, nullptr, ep, status, st);
+    e = launch_form_tc_t<false, 1>(d, Cm, 1, Bm, 1, x, 0, cum, states, ep, status, st);
     if (e != cudaSuccess) return e;
     // dC summed over each group's heads: causal, U = dy, V = x, Z = B, M = Hin read as P x N
     e = launch_form_group_tc_t<false>(d, dy, x, Bm, cum, states, dCm, status, st);
     if (e != cudaSuccess) return e;
     // dx - D dy: anti-causal, U = B, V = C, Z = dy, M = G (N x P); dx, x . (dx - D dy) and x . dy kept
-    e = launch_form_tc_t<128, 64, true, true, 2>(d, Bm, 1, Cm, 1, dy, 0, cum, dstates, nullptr, ep, status, st);
+    e = launch_form_tc_t<true, 2>(d, Bm, 1, Cm, 1, dy, 0, cum, dstates, ep, status, st);
     if (e != cudaSuccess) return e;
     // dB summed over each group's heads: anti-causal, U = x, V = dy, Z = C, M = G read as P x N
     return launch_form_group_tc_t<true>(d, x, dy, Cm, cum, dstates, dBm, status, st);
