@@ -82,16 +82,13 @@ struct DsParams {
 };
 
 // g[t][n] in shared memory, fp32, 16 float4 chunks per row, chunk c of row t
-// at c ^ ((c >> 3) << 1) ^ ((t >> 2) & 1): the in-sub-block loop reads rows
-// t0 - k and t0 + 4 - k in one instruction, and these land in distinct banks
+// at (c >> 1) | ((c & 1) << 3): the eight lanes that read one row in the
+// in-sub-block loop take chunks 2 o + e (o = 0..7, e fixed), which land in
+// eight distinct bank groups
 __device__ __forceinline__ uint32_t g_off(int t, int n) {
     const int c = n >> 2;
-    const int cs = c ^ ((c >> 3) << 1) ^ ((t >> 2) & 1);
+    const int cs = (c >> 1) | ((c & 1) << 3);
     return (uint32_t)(t * 64 + cs * 4 + (n & 3));
-}
-
-__device__ __forceinline__ float bf16_at(const uint8_t* tile, int row, int col) {
-    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(tile + tc::sw128_offset(row, col >> 3) + (col & 7) * 2));
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -237,16 +234,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float cend = c;
             sG[r * kN + n] = ex2_approx(cend * kLog2e);
             // the raw C rows of group Q's in-sub-block loop are read below, before
-            // C o E overwrites them; every thread is done reading a
-            float craw[4][16];
-            const int qr = quad, qrg = lane >> 2, qq = lane & 3;  // group Q: sub-block, row group, n-quarter
-            const int tq = 32 * qr + 4 * qrg;                     // first row of the row group
+            // C o E overwrites them; every thread is done reading a.  Group Q:
+            // warp = sub-block qr, lane = (pair pi, n-eighth o); the pair takes
+            // the row groups 7 - pi and pi of the sub-block (four rows each)
+            float crA[4][8], crB[4][8];
+            const int qr = quad, pi = lane >> 3, o = lane & 7;
+            const int tqA = 32 * qr + 4 * (7 - pi), tqB = 32 * qr + 4 * pi;  // first rows
+            // eight bf16 of a row, columns [8 o, 8 o + 8), from a swizzled tile
+            auto row8 = [&](const uint8_t* tile, int t, float (&v)[8]) {
+                const uint4 u = *reinterpret_cast<const uint4*>(tile + tc::sw128_offset(t, o));
+                const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = tc::unpack_bf16x2(w4[e]);
+                    v[2 * e] = f.x; v[2 * e + 1] = f.y;
+                }
+            };
             if (rq_or(false)) goto done;
             if (!groupR) {
 #pragma unroll
-                for (int rr = 0; rr < 4; ++rr)
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) craw[rr][e] = bf16_at(sC, tq + rr, 16 * qq + e);
+                for (int rr = 0; rr < 4; ++rr) {
+                    row8(sC, tqA + rr, crA[rr]);
+                    row8(sC, tqB + rr, crB[rr]);
+                }
             }
             // g_t = exp(a_t) over a, in the swizzled layout
 #pragma unroll
@@ -282,96 +292,104 @@ __global__ void __launch_bounds__(kThreads, 1)
 
             if (!groupR) {
                 // ----------------------- in-sub-block scores (group Q) ----
-                // rows tq .. tq+3 (row group qrg of sub-block qr), n in
-                // [16 qq, 16 qq + 16); columns s from tq down to the sub-block's
-                // start: S[tq+rr][s] = sum_n C[tq+rr][n] B[s][n] prod_{k=s+1..tq+rr} g_k[n]
+                // S[t][s] = sum_n C[t][n] B[s][n] prod_{k=s+1..t} g_k[n] for s <= t in
+                // t's sub-block: a lane holds rows tq .. tq+3 of a row group and
+                // the n in [8 o, 8 o + 8); the row group's eight lanes sum over n
                 const int s_lo = 32 * qr;
-                const unsigned gmask = 0xFu << (4 * qrg);
-                auto grow = [&](int t, float (&v)[16]) {
+                auto grow = [&](int t, float (&v)[8]) {
 #pragma unroll
-                    for (int e4 = 0; e4 < 4; ++e4) {
-                        const float4 f = *reinterpret_cast<const float4*>(sA + g_off(t, 16 * qq + 4 * e4));
+                    for (int e4 = 0; e4 < 2; ++e4) {
+                        const float4 f = *reinterpret_cast<const float4*>(sA + g_off(t, 8 * o + 4 * e4));
                         v[4 * e4] = f.x; v[4 * e4 + 1] = f.y; v[4 * e4 + 2] = f.z; v[4 * e4 + 3] = f.w;
                     }
                 };
-                auto brow = [&](int s, float (&v)[16]) {
-#pragma unroll
-                    for (int h8 = 0; h8 < 2; ++h8) {
-                        const uint4 u = *reinterpret_cast<const uint4*>(sB + tc::sw128_offset(s, 2 * qq + h8));
-                        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 f = tc::unpack_bf16x2(w4[e]);
-                            v[8 * h8 + 2 * e] = f.x; v[8 * h8 + 2 * e + 1] = f.y;
-                        }
-                    }
-                };
-                // four partial dot products (one per row) -> lane qq holds row qq's sum
-                auto reduce4 = [&](const float (&d)[4]) -> float {
+                // four partial dot products (one per row) -> lanes o and o ^ 4 hold
+                // row (o & 3)'s sum over the row group's eight lanes
+                auto reduce8 = [&](const float (&d)[4]) -> float {
                     float e0, e1;
                     {
-                        const bool hi = qq & 2;
+                        const bool hi = o & 2;
                         const float k0 = hi ? d[2] : d[0], s0 = hi ? d[0] : d[2];
                         const float k1 = hi ? d[3] : d[1], s1 = hi ? d[1] : d[3];
-                        e0 = k0 + __shfl_xor_sync(gmask, s0, 2);
-                        e1 = k1 + __shfl_xor_sync(gmask, s1, 2);
+                        e0 = k0 + __shfl_xor_sync(0xffffffffu, s0, 2);
+                        e1 = k1 + __shfl_xor_sync(0xffffffffu, s1, 2);
                     }
-                    const bool lo = qq & 1;
+                    const bool lo = o & 1;
                     const float keep = lo ? e1 : e0, send = lo ? e0 : e1;
-                    return keep + __shfl_xor_sync(gmask, send, 1);
+                    const float q = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+                    return q + __shfl_xor_sync(0xffffffffu, q, 4);
                 };
-                // the pairs inside the row group: (tq+rr, tq+jj), 1 <= jj <= rr
-                {
-                    float gv[4][16], bv[16];
+                // the pairs inside a row group, (tq+rr, tq+jj) with 1 <= jj <= rr;
+                // then the rows' coefficients C o prod_{k = tq+1 .. tq+rr} g_k for
+                // the columns s <= tq
+                auto triangle = [&](int tq, float (&cr)[4][8]) {
+                    float gv[4][8], bv[8];
 #pragma unroll
                     for (int rr = 1; rr < 4; ++rr) grow(tq + rr, gv[rr]);
 #pragma unroll
                     for (int jj = 1; jj < 4; ++jj) {
-                        brow(tq + jj, bv);
+                        row8(sB, tq + jj, bv);
                         float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                         for (int rr = 0; rr < 4; ++rr) {
                             if (rr < jj) continue;
 #pragma unroll
-                            for (int e = 0; e < 16; ++e) {
+                            for (int e = 0; e < 8; ++e) {
                                 float w = 1.f;  // prod_{k = tq+jj+1 .. tq+rr} g_k
 #pragma unroll
                                 for (int kk = jj + 1; kk <= 3; ++kk)
                                     if (kk <= rr) w *= gv[kk][e];
-                                d[rr] += craw[rr][e] * bv[e] * w;
+                                d[rr] += cr[rr][e] * bv[e] * w;
                             }
                         }
-                        const float sv = reduce4(d);
-                        if (qq >= jj) sS[(tq + qq) * kSS + (tq + jj - s_lo)] = sv;
+                        const float sv = reduce8(d);
+                        if (o < 4 && o >= jj) sS[(tq + o) * kSS + (tq + jj - s_lo)] = sv;
                     }
-                    // coefficients C o prod_{k = tq+1 .. tq+rr} g_k for the columns s <= tq
-                    float pre[16];
+                    float pre[8];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) pre[e] = 1.f;
+                    for (int e = 0; e < 8; ++e) pre[e] = 1.f;
 #pragma unroll
                     for (int rr = 1; rr < 4; ++rr)
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) {
+                        for (int e = 0; e < 8; ++e) {
                             pre[e] *= gv[rr][e];
-                            craw[rr][e] *= pre[e];
+                            cr[rr][e] *= pre[e];
                         }
-                }
-                float u[16];  // prod_{k = s+1 .. tq} g_k
+                };
+                triangle(tqA, crA);
+                triangle(tqB, crB);
+                // the columns s from a row group's first row down to the sub-block's
+                // start: row group 7 - pi (29 - 4 pi columns), then row group pi
+                // (4 pi + 1), 30 steps for every lane; u = prod_{k = s+1 .. tq} g_k
+                const int lenA = 4 * (7 - pi) + 1;
+                float u[8];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) u[e] = 1.f;
-                for (int s = tq; s >= s_lo; --s) {
-                    float bv[16], gv[16];
-                    brow(s, bv);
+                for (int e = 0; e < 8; ++e) u[e] = 1.f;
+                int tq = tqA, s = tqA;
+                for (int it = 0; it < 30; ++it, --s) {
+                    if (it == lenA) {
+                        tq = tqB;
+                        s = tqB;
+#pragma unroll
+                        for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) crA[rr][e] = crB[rr][e];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) u[e] = 1.f;
+                    }
+                    float bv[8], gv[8];
+                    row8(sB, s, bv);
                     grow(s, gv);
                     float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
+                    for (int e = 0; e < 8; ++e) {
                         const float ub = u[e] * bv[e];
 #pragma unroll
-                        for (int rr = 0; rr < 4; ++rr) d[rr] += craw[rr][e] * ub;
+                        for (int rr = 0; rr < 4; ++rr) d[rr] += crA[rr][e] * ub;
                         u[e] *= gv[e];
                     }
-                    sS[(tq + qq) * kSS + (s - s_lo)] = reduce4(d);
+                    const float sv = reduce8(d);
+                    if (o < 4) sS[(tq + o) * kSS + (s - s_lo)] = sv;
                 }
                 asm volatile("bar.sync 2, 128;" ::: "memory");  // group Q's scores are complete
                 // ---- P rows of this sub-block into TMEM (thread = TMEM lane)
