@@ -30,8 +30,10 @@
 //
 // Warp roles (288 threads): 0 TMA and MMA issue (and TMEM); 1-4 group R
 // (thread = row of the block: C~ rows, the state chain, the output); 5-8
-// group Q (the in-sub-block scores; warp w serves sub-block w & 3).  The
-// decays are scanned by groups R and Q together, thread = (n, sub-block).
+// group Q (the in-sub-block scores: warp w takes row groups 7 - (w & 3) and
+// w & 3 of every sub-block, then moves the scores of sub-block w & 3, its
+// lane quadrant, into TMEM).  The decays are scanned by groups R and Q
+// together, thread = (n, sub-block).
 #include "../common.cuh"
 #include "../debug_checks.cuh"
 #include "../kernels.h"
@@ -60,8 +62,8 @@ constexpr uint32_t OFF_AZ = OFF_C + kTile;        // [2 m-halves][128 rows][64] 
 constexpr uint32_t OFF_H = OFF_AZ + 2 * kTile;    // h^(0..3) [4][64 rows][64] bf16
 constexpr int kSS = 33;                           // row stride of the scores (bank spread)
 constexpr int kZS = 68;                           // row stride of Z_1 (16-byte rows, bank spread)
-constexpr uint32_t OFF_S = OFF_H + 4 * kH;        // in-sub-block scores [128][kSS] fp32
-constexpr uint32_t OFF_Z1 = OFF_S + ((kBlk * kSS * 4 + 15) / 16) * 16;  // Z_1 [64][kZS] fp32
+constexpr uint32_t OFF_S = OFF_H + 4 * kH;        // in-sub-block scores, row t at s_row(t), fp32
+constexpr uint32_t OFF_Z1 = OFF_S + (((kBlk * kSS + 32) * 4 + 15) / 16) * 16;  // Z_1 [64][kZS] fp32
 constexpr uint32_t OFF_G = OFF_Z1 + 64 * kZS * 4;  // G_r [4][64] fp32
 constexpr uint32_t OFF_BAR = OFF_G + 4 * kN * 4;
 constexpr uint32_t OFF_MISC = OFF_BAR + ((sizeof(DsBars) + 15) / 16) * 16;
@@ -80,6 +82,10 @@ struct DsParams {
     int T, H, G, nblk;
     int from_cum;      // the decay tile holds in-chunk prefix sums (128-token chunks), not a
 };
+
+// row t of the in-sub-block scores: stride kSS, and each sub-block shifted by
+// eight more words, so that rows 32 apart fall in different banks
+__device__ __forceinline__ int s_row(int t) { return t * kSS + (t >> 5) * 8; }
 
 // g[t][n] in shared memory, fp32, 16 float4 chunks per row, chunk c of row t
 // at (c >> 1) | ((c & 1) << 3): the eight lanes that read one row in the
@@ -235,10 +241,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             sG[r * kN + n] = ex2_approx(cend * kLog2e);
             // the raw C rows of group Q's in-sub-block loop are read below, before
             // C o E overwrites them; every thread is done reading a.  Group Q:
-            // warp = sub-block qr, lane = (pair pi, n-eighth o); the pair takes
-            // the row groups 7 - pi and pi of the sub-block (four rows each)
+            // warp pi (its lane quadrant), lane = (sub-block qr, n-eighth o); the
+            // lane takes the row groups 7 - pi and pi of its sub-block (four rows
+            // each), so the column loops below run alike on every lane of a warp
             float crA[4][8], crB[4][8];
-            const int qr = quad, pi = lane >> 3, o = lane & 7;
+            const int pi = quad, qr = lane >> 3, o = lane & 7;
             const int tqA = 32 * qr + 4 * (7 - pi), tqB = 32 * qr + 4 * pi;  // first rows
             // eight bf16 of a row, columns [8 o, 8 o + 8), from a swizzled tile
             auto row8 = [&](const uint8_t* tile, int t, float (&v)[8]) {
@@ -343,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                         }
                         const float sv = reduce8(d);
-                        if (o < 4 && o >= jj) sS[(tq + o) * kSS + (tq + jj - s_lo)] = sv;
+                        if (o < 4 && o >= jj) sS[s_row(tq + o) + (tq + jj - s_lo)] = sv;
                     }
                     float pre[8];
 #pragma unroll
@@ -359,53 +366,47 @@ __global__ void __launch_bounds__(kThreads, 1)
                 triangle(tqA, crA);
                 triangle(tqB, crB);
                 // the columns s from a row group's first row down to the sub-block's
-                // start: row group 7 - pi (29 - 4 pi columns), then row group pi
-                // (4 pi + 1), 30 steps for every lane; u = prod_{k = s+1 .. tq} g_k
-                const int lenA = 4 * (7 - pi) + 1;
-                float u[8];
+                // start, u = prod_{k = s+1 .. tq} g_k: row group 7 - pi (29 - 4 pi
+                // columns), then row group pi (4 pi + 1), 30 steps for every warp
+                auto columns = [&](int tq, int steps, const float (&cr)[4][8]) {
+                    float u[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) u[e] = 1.f;
-                int tq = tqA, s = tqA;
-                for (int it = 0; it < 30; ++it, --s) {
-                    if (it == lenA) {
-                        tq = tqB;
-                        s = tqB;
+                    for (int e = 0; e < 8; ++e) u[e] = 1.f;
+                    int s = tq;
+#pragma unroll 2
+                    for (int it = 0; it < steps; ++it, --s) {
+                        float bv[8], gv[8];
+                        row8(sB, s, bv);
+                        grow(s, gv);
+                        float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                        for (int rr = 0; rr < 4; ++rr)
+                        for (int e = 0; e < 8; ++e) {
+                            const float ub = u[e] * bv[e];
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) crA[rr][e] = crB[rr][e];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) u[e] = 1.f;
+                            for (int rr = 0; rr < 4; ++rr) d[rr] += cr[rr][e] * ub;
+                            u[e] *= gv[e];
+                        }
+                        const float sv = reduce8(d);
+                        if (o < 4) sS[s_row(tq + o) + (s - s_lo)] = sv;
                     }
-                    float bv[8], gv[8];
-                    row8(sB, s, bv);
-                    grow(s, gv);
-                    float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float ub = u[e] * bv[e];
-#pragma unroll
-                        for (int rr = 0; rr < 4; ++rr) d[rr] += crA[rr][e] * ub;
-                        u[e] *= gv[e];
-                    }
-                    const float sv = reduce8(d);
-                    if (o < 4) sS[(tq + o) * kSS + (s - s_lo)] = sv;
-                }
+                };
+                columns(tqA, 4 * (7 - pi) + 1, crA);
+                columns(tqB, 4 * pi + 1, crB);
                 asm volatile("bar.sync 2, 128;" ::: "memory");  // group Q's scores are complete
                 // ---- P rows of this sub-block into TMEM (thread = TMEM lane)
                 {
-                    const int t = 32 * qr + lane;  // this warp's quadrant = sub-block qr
+                    const int t = 32 * quad + lane;  // this warp's quadrant = sub-block quad
                     const float dv = p.D ? __ldg(p.D + h) : 0.f;
                     uint32_t pk[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        float v0 = 2 * e <= lane ? sS[t * kSS + 2 * e] : 0.f;
-                        float v1 = 2 * e + 1 <= lane ? sS[t * kSS + 2 * e + 1] : 0.f;
+                        float v0 = 2 * e <= lane ? sS[s_row(t) + 2 * e] : 0.f;
+                        float v1 = 2 * e + 1 <= lane ? sS[s_row(t) + 2 * e + 1] : 0.f;
                         if (2 * e == lane) v0 += dv;
                         if (2 * e + 1 == lane) v1 += dv;
                         pk[e] = tc::pack_bf16x2(v0, v1);
                     }
-                    tc::tmem_st16(tmem + ((uint32_t)(quad * 32) << 16) + COL_P + 16 * qr, pk);
+                    tc::tmem_st16(tmem + ((uint32_t)(quad * 32) << 16) + COL_P + 16 * quad, pk);
                     tc::tmem_st_wait();
                     tc::tc_fence_before();
                     __syncwarp();
