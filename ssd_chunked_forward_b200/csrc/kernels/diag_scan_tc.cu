@@ -368,23 +368,62 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // the columns s from a row group's first row down to the sub-block's
                 // start, u = prod_{k = s+1 .. tq} g_k: row group 7 - pi (29 - 4 pi
                 // columns), then row group pi (4 pi + 1), 30 steps for every warp
+                // eight partial sums (rows 0-3 of column s, then of column s - 1)
+                // -> lane o holds value o summed over the row group's eight lanes
+                auto reduce8x8 = [&](const float (&d0)[4], const float (&d1)[4]) -> float {
+                    const bool h4 = o & 4, h2 = o & 2, h1 = o & 1;
+                    float b[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float keep = h4 ? d1[i] : d0[i], send = h4 ? d0[i] : d1[i];
+                        b[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+                    }
+                    float c[2];
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        const float keep = h2 ? b[2 + i] : b[i], send = h2 ? b[i] : b[2 + i];
+                        c[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+                    }
+                    const float keep = h1 ? c[1] : c[0], send = h1 ? c[0] : c[1];
+                    return keep + __shfl_xor_sync(0xffffffffu, send, 1);
+                };
                 auto columns = [&](int tq, int steps, const float (&cr)[4][8]) {
                     float u[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) u[e] = 1.f;
                     int s = tq;
-#pragma unroll 2
-                    for (int it = 0; it < steps; ++it, --s) {
-                        float bv[8], gv[8];
+                    // two columns a step, their sums reduced together
+                    for (int it = 0; it + 1 < steps; it += 2, s -= 2) {
+                        float b0[8], g0[8], b1[8], g1[8];
+                        row8(sB, s, b0);
+                        grow(s, g0);
+                        row8(sB, s - 1, b1);
+                        grow(s - 1, g1);
+                        float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const float ub0 = u[e] * b0[e];
+                            u[e] *= g0[e];
+                            const float ub1 = u[e] * b1[e];
+                            u[e] *= g1[e];
+#pragma unroll
+                            for (int rr = 0; rr < 4; ++rr) {
+                                d0[rr] += cr[rr][e] * ub0;
+                                d1[rr] += cr[rr][e] * ub1;
+                            }
+                        }
+                        const float sv = reduce8x8(d0, d1);
+                        sS[s_row(tq + (o & 3)) + (s - (o >> 2) - s_lo)] = sv;
+                    }
+                    if (steps & 1) {  // the sub-block's first column, s = s_lo
+                        float bv[8];
                         row8(sB, s, bv);
-                        grow(s, gv);
                         float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
                             const float ub = u[e] * bv[e];
 #pragma unroll
                             for (int rr = 0; rr < 4; ++rr) d[rr] += cr[rr][e] * ub;
-                            u[e] *= gv[e];
                         }
                         const float sv = reduce8(d);
                         if (o < 4) sS[s_row(tq + o) + (s - s_lo)] = sv;
