@@ -139,6 +139,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mbar_init(&bars->y_full, 1);
         *sAbort = 0;
         tc::fence_mbar_init();
+        // the block's tiles, in flight while TMEM is allocated
+        tc::mbar_arrive_expect_tx(&bars->full, 2 * kTile + 3 * kTile);
+        if (p.from_cum)  // cum [B][H][nc][128][N] viewed as rows of N
+            tc::tma_load_4d(sA, &tm_a, &bars->full, 0, 0, (bh * p.nblk + j) * kBlk, 0);
+        else
+            tc::tma_load_4d(sA, &tm_a, &bars->full, 0, h, t0, b);
+        tc::tma_load_4d(sX, &tm_x, &bars->full, 0, h, t0, b);
+        tc::tma_load_4d(sB, &tm_b, &bars->full, 0, g, t0, b);
+        tc::tma_load_4d(sC, &tm_c, &bars->full, 0, g, t0, b);
     }
     if (warp == 0) {
         tc::tmem_alloc(sTmem, 512);
@@ -166,15 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            // ------------------------------------------ TMA and MMA issue ----
-            tc::mbar_arrive_expect_tx(&bars->full, 2 * kTile + 3 * kTile);
-            if (p.from_cum)  // cum [B][H][nc][128][N] viewed as rows of N
-                tc::tma_load_4d(sA, &tm_a, &bars->full, 0, 0, (bh * p.nblk + j) * kBlk, 0);
-            else
-                tc::tma_load_4d(sA, &tm_a, &bars->full, 0, h, t0, b);
-            tc::tma_load_4d(sX, &tm_x, &bars->full, 0, h, t0, b);
-            tc::tma_load_4d(sB, &tm_b, &bars->full, 0, g, t0, b);
-            tc::tma_load_4d(sC, &tm_c, &bars->full, 0, g, t0, b);
+            // ------------------------------------------------- MMA issue ----
             bool ok = tc::mbar_wait(&bars->full, 0, abort_v) && tc::mbar_wait(&bars->az_full, 0, abort_v);
             constexpr uint32_t id_z = tc::idesc_bf16_f32(128, kP, 1, 1);
             constexpr uint32_t id_y = tc::idesc_bf16_f32(128, kP, 0, 1);
