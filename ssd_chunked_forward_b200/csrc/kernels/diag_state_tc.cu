@@ -109,6 +109,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mbar_init(&bars->acc_full, 1);
         *sAbort = 0;
         tc::fence_mbar_init();
+        // the two blocks' tiles, in flight while TMEM is allocated; a block
+        // past the sequence (odd block count) reads zeros
+        tc::mbar_arrive_expect_tx(&bars->full, 2 * kATile + 4 * kTile);
+        for (int jb = 0; jb < 2; ++jb) {
+            const int t0 = (j0 + jb) * kBlk;
+            if (p.from_cum)  // cum [B][H][nc][128][N] viewed as rows of N; a missing block reads zeros
+                tc::tma_load_4d(sA + jb * (kBlk * kN), &tm_a, &bars->full, 0, 0,
+                                (bh * p.nblk + (j0 + jb < p.nblk ? j0 + jb : p.nblk)) * kBlk, 0);
+            else
+                tc::tma_load_4d(sA + jb * (kBlk * kN), &tm_a, &bars->full, 0, h, t0, b);
+            tc::tma_load_4d(sX + jb * kTile, &tm_x, &bars->full, 0, h, t0, b);
+            tc::tma_load_4d(sB + jb * kTile, &tm_b, &bars->full, 0, g, t0, b);
+        }
     }
     if (warp == 1) {
         tc::tmem_alloc(sTmem, 64);
@@ -125,20 +138,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            // ---------------------------------------------- TMA producer ----
-            // a block past the sequence (odd block count) reads zeros
-            tc::mbar_arrive_expect_tx(&bars->full, 2 * kATile + 4 * kTile);
-            for (int jb = 0; jb < 2; ++jb) {
-                const int t0 = (j0 + jb) * kBlk;
-                if (p.from_cum)  // cum [B][H][nc][128][N] viewed as rows of N; a missing block reads zeros
-                    tc::tma_load_4d(sA + jb * (kBlk * kN), &tm_a, &bars->full, 0, 0,
-                                    (bh * p.nblk + (j0 + jb < p.nblk ? j0 + jb : p.nblk)) * kBlk, 0);
-                else
-                    tc::tma_load_4d(sA + jb * (kBlk * kN), &tm_a, &bars->full, 0, h, t0, b);
-                tc::tma_load_4d(sX + jb * kTile, &tm_x, &bars->full, 0, h, t0, b);
-                tc::tma_load_4d(sB + jb * kTile, &tm_b, &bars->full, 0, g, t0, b);
-            }
-            // no copy may still be landing in shared memory when the CTA exits
+            // ---------------------------------------- the tiles' arrival ----
+            // (issued at barrier init) no copy may still be landing in shared
+            // memory when the CTA exits
             tc::mbar_wait(&bars->full, 0, nullptr, 200000000ull);
         }
     } else if (warp == 1) {
